@@ -1,0 +1,256 @@
+"""Python face of the CPU oracle (sp24_oracle.c).
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and
+the CPU-baseline leg of ``bench.py`` may import this module.  It never
+imports the CUDA package and the CUDA package never imports it.
+
+Every function here is a thin numpy/ctypes wrapper around the C oracle, plus
+the few definitions that are plain arithmetic on numbers (dequantization,
+the tactic rule and the coverage ratio), each citing the page it restates.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional, Sequence
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "sp24_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the C oracle with plain gcc (no fast-math, no FP contraction)."""
+    if force or not os.path.exists(_LIB_PATH) or \
+            os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + ".tmp%d" % os.getpid()
+        subprocess.check_call([
+            "gcc", "-std=c11", "-O2", "-fPIC", "-shared", "-ffp-contract=off",
+            "-fno-fast-math", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        path = build()
+        L = ctypes.CDLL(path)
+        P = ctypes.c_void_p
+        I64 = ctypes.c_int64
+        sig = {
+            "orc_prune_group": (ctypes.c_int, [P, P, P]),
+            "orc_prune_compress_bf16": (None, [P, I64, I64, I64, P, P, P]),
+            "orc_prune_compress_bf16_hybrid": (None, [P, I64, I64, I64, P, P, P, P]),
+            "orc_prune_compress_e4m3": (None, [P, I64, I64, I64, P, P, P, P, P]),
+            "orc_decompress": (None, [P, P, I64, I64, ctypes.c_int, P]),
+            "orc_e4m3_decode": (ctypes.c_double, [ctypes.c_uint8]),
+            "orc_e4m3_encode": (ctypes.c_uint8, [ctypes.c_double]),
+            "orc_e4m3_encode_array": (None, [P, I64, P]),
+            "orc_e4m3_row_scale": (None, [ctypes.c_float, P, P]),
+            "orc_quantize_rows_e4m3": (None, [P, I64, I64, I64, P, P]),
+            "orc_meta_image": (None, [P, I64, I64, ctypes.c_int, P, P]),
+            "orc_gemm_f64": (None, [P, P, I64, I64, I64, P, P]),
+            "orc_gemm_f64_sampled": (None, [P, P, I64, P, P, I64, P, P]),
+            "orc_gemm_sparse_f64": (None, [P, I64, I64, P, P, I64, P]),
+            "orc_bf16_to_double": (ctypes.c_double, [ctypes.c_uint16]),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _p(a: Optional[np.ndarray]):
+    if a is None:
+        return None
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+# ---------------------------------------------------------------------------
+# exact number conversions
+# ---------------------------------------------------------------------------
+
+def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    """Exact value of bf16 bit patterns (bf16 = top 16 bits of an fp32)."""
+    u = bits.astype(np.uint32) << 16
+    return u.view(np.float32).astype(np.float64)
+
+
+_E4M3_TABLE = None
+
+
+def e4m3_table() -> np.ndarray:
+    """Value of each of the 256 E4M3 codes, from the oracle's own decoder."""
+    global _E4M3_TABLE
+    if _E4M3_TABLE is None:
+        L = lib()
+        _E4M3_TABLE = np.array([L.orc_e4m3_decode(i) for i in range(256)], dtype=np.float64)
+    return _E4M3_TABLE
+
+
+def e4m3_decode(codes: np.ndarray) -> np.ndarray:
+    return e4m3_table()[codes.astype(np.int64)]
+
+
+def e4m3_encode(x: np.ndarray) -> np.ndarray:
+    """Round-to-nearest-even, saturating E4M3 encoding of fp32 values."""
+    x = np.ascontiguousarray(np.asarray(x, dtype=np.float32).astype(np.float64))
+    q = np.empty(x.shape, dtype=np.uint8)
+    lib().orc_e4m3_encode_array(_p(x), x.size, _p(q))
+    return q
+
+
+def e4m3_row_scale(amax: float):
+    s = ctypes.c_float()
+    i = ctypes.c_float()
+    lib().orc_e4m3_row_scale(ctypes.c_float(amax), ctypes.byref(s), ctypes.byref(i))
+    return s.value, i.value
+
+
+# ---------------------------------------------------------------------------
+# prune / compress / decompress
+# ---------------------------------------------------------------------------
+
+def prune_group(v_bits: Sequence[int]):
+    """(nibble, i0, i1) for one group of four bf16 bit patterns."""
+    a = np.ascontiguousarray(np.asarray(v_bits, dtype=np.uint16))
+    i0 = ctypes.c_int()
+    i1 = ctypes.c_int()
+    nib = lib().orc_prune_group(_p(a), ctypes.byref(i0), ctypes.byref(i1))
+    return nib, i0.value, i1.value
+
+
+def prune_compress_bf16(W_bits: np.ndarray):
+    """Return (pruned [rows,K], values [rows,K/2], meta_canon [rows,K/8])."""
+    W = np.ascontiguousarray(W_bits, dtype=np.uint16)
+    rows, K = W.shape
+    assert K % 4 == 0
+    pruned = np.empty((rows, K), np.uint16)
+    values = np.empty((rows, K // 2), np.uint16)
+    meta = np.empty((rows, K // 8), np.uint8)
+    lib().orc_prune_compress_bf16(_p(W), rows, K, K, _p(pruned), _p(values), _p(meta))
+    return pruned, values, meta
+
+
+def prune_compress_bf16_hybrid(W_bits: np.ndarray, mask: np.ndarray):
+    """Hybrid bf16: (values, meta_canon, dense_out) with dense tiles copied."""
+    W = np.ascontiguousarray(W_bits, dtype=np.uint16)
+    rows, K = W.shape
+    values = np.empty((rows, K // 2), np.uint16)
+    meta = np.empty((rows, K // 8), np.uint8)
+    dense = np.zeros((rows, K), np.uint16)
+    m = np.ascontiguousarray(mask, dtype=np.uint8)
+    lib().orc_prune_compress_bf16_hybrid(_p(W), rows, K, K, _p(m), _p(values), _p(meta), _p(dense))
+    return values, meta, dense
+
+
+def prune_compress_e4m3(W_bits: np.ndarray, mask: Optional[np.ndarray] = None):
+    """Return (values_q [rows,K/2], meta_canon, scales [rows] f32, dense_q [rows,K])."""
+    W = np.ascontiguousarray(W_bits, dtype=np.uint16)
+    rows, K = W.shape
+    values = np.empty((rows, K // 2), np.uint8)
+    meta = np.empty((rows, K // 8), np.uint8)
+    scales = np.empty((rows,), np.float32)
+    dense = np.zeros((rows, K), np.uint8)
+    m = None if mask is None else np.ascontiguousarray(mask, dtype=np.uint8)
+    lib().orc_prune_compress_e4m3(_p(W), rows, K, K, _p(m), _p(values), _p(meta),
+                                  _p(scales), _p(dense))
+    return values, meta, scales, dense
+
+
+def decompress(values: np.ndarray, meta_canon: np.ndarray, rows: int, K: int) -> np.ndarray:
+    values = np.ascontiguousarray(values)
+    eb = values.dtype.itemsize
+    out = np.empty((rows, K), values.dtype)
+    lib().orc_decompress(_p(values), _p(np.ascontiguousarray(meta_canon)), rows, K, eb, _p(out))
+    return out
+
+
+def meta_image(meta_canon: np.ndarray, rows: int, K: int, is_8bit: bool,
+               mask: Optional[np.ndarray] = None) -> np.ndarray:
+    RB = (rows + 127) // 128
+    img = np.empty((RB * (K // 128) * 2048,), np.uint8)
+    m = None if mask is None else np.ascontiguousarray(mask, dtype=np.uint8)
+    lib().orc_meta_image(_p(np.ascontiguousarray(meta_canon)), rows, K, int(is_8bit), _p(m), _p(img))
+    return img
+
+
+def quantize_rows_e4m3(X_bits: np.ndarray):
+    """Per-row (per-token) E4M3: (q [rows,K], scales [rows])."""
+    X = np.ascontiguousarray(X_bits, dtype=np.uint16)
+    rows, K = X.shape
+    q = np.empty((rows, K), np.uint8)
+    s = np.empty((rows,), np.float32)
+    lib().orc_quantize_rows_e4m3(_p(X), rows, K, K, _p(q), _p(s))
+    return q, s
+
+
+# ---------------------------------------------------------------------------
+# GEMM (fp64)
+# ---------------------------------------------------------------------------
+
+def gemm_f64(X: np.ndarray, W: np.ndarray):
+    """Y = X W^T and A = |X| |W|^T elementwise-product sums, both fp64."""
+    X = np.ascontiguousarray(X, dtype=np.float64)
+    W = np.ascontiguousarray(W, dtype=np.float64)
+    M, K = X.shape
+    N = W.shape[0]
+    Y = np.empty((M, N), np.float64)
+    A = np.empty((M, N), np.float64)
+    lib().orc_gemm_f64(_p(X), _p(W), M, N, K, _p(Y), _p(A))
+    return Y, A
+
+
+def gemm_f64_sampled(X: np.ndarray, W: np.ndarray, ms: np.ndarray, ns: np.ndarray):
+    X = np.ascontiguousarray(X, dtype=np.float64)
+    W = np.ascontiguousarray(W, dtype=np.float64)
+    ms = np.ascontiguousarray(ms, dtype=np.int64)
+    ns = np.ascontiguousarray(ns, dtype=np.int64)
+    Y = np.empty(ms.shape, np.float64)
+    A = np.empty(ms.shape, np.float64)
+    lib().orc_gemm_f64_sampled(_p(X), _p(W), X.shape[1], _p(ms), _p(ns), ms.size, _p(Y), _p(A))
+    return Y, A
+
+
+def gemm_sparse_f64(X: np.ndarray, wvals: np.ndarray, meta_canon: np.ndarray):
+    X = np.ascontiguousarray(X, dtype=np.float64)
+    wv = np.ascontiguousarray(wvals, dtype=np.float64)
+    M, K = X.shape
+    N = wv.shape[0]
+    Y = np.empty((M, N), np.float64)
+    lib().orc_gemm_sparse_f64(_p(X), M, K, _p(wv), _p(np.ascontiguousarray(meta_canon)), N, _p(Y))
+    return Y
+
+
+def within_tolerance(y_gpu: np.ndarray, y_ref: np.ndarray, a_ref: np.ndarray,
+                     rel: float = 2e-3, abs_: float = 1e-6) -> np.ndarray:
+    """Per-element pass mask of |y_gpu - y| <= rel * sum_k |x_k w_k| + abs."""
+    return np.abs(y_gpu.astype(np.float64) - y_ref) <= rel * a_ref + abs_
+
+
+# ---------------------------------------------------------------------------
+# tactic rule and coverage  [P1 "Sparse Tactic Audit": latency is the sole
+# criterion; Sparse GPU-Time Coverage = time of selected sparse kernels over
+# total GPU time]
+# ---------------------------------------------------------------------------
+
+def select_tactic(t_sparse_samples, t_dense_samples):
+    """'sparse' iff median sparse time < median dense time (a tie -> dense)."""
+    ts = float(np.median(np.asarray(t_sparse_samples, dtype=np.float64)))
+    td = float(np.median(np.asarray(t_dense_samples, dtype=np.float64)))
+    return ("sparse" if ts < td else "dense"), ts, td
+
+
+def sparse_gpu_time_coverage(selected_times):
+    """selected_times: iterable of (tactic, time) for the kernels that ran."""
+    tot = sum(t for _, t in selected_times)
+    sp = sum(t for tac, t in selected_times if tac == "sparse")
+    return sp / tot if tot > 0 else 0.0

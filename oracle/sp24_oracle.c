@@ -1,0 +1,473 @@
+/*
+ * sp24_oracle.c -- CPU oracle for 2:4 semi-structured sparsity.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the
+ * benchmark's CPU-baseline leg may load this file's library.  The CUDA
+ * library never links, includes or calls it, and it never calls the CUDA
+ * library: the two share no code, header, table or constant generator.
+ *
+ * Everything here is written to be checked by eye against the pages it
+ * restates, so it is slow on purpose: plain loops, fp64 accumulation, no
+ * blocking and no reordering beyond the definitions.
+ *
+ * Sources (page title, then section):
+ *  [P1] "Production 2:4 Structured Sparsity for LLMs" (oh-bug.com),
+ *       "Core Mechanisms and Production States of 2:4 Structured Sparsity",
+ *       "Sparse Tactic Audit", "Dense Fallback and Hybrid Sparsity Design".
+ *  [P3] "2:4 Structured Sparsity Explained" (tensorcore.si),
+ *       "How 2:4 sparsity works" (format and storage table),
+ *       "How to make a model 2:4 sparse" (keep the two largest magnitudes).
+ *  [P4] the 2:4-versus-quantization paper (paperpeel.com/paper/2610.28947),
+ *       section 2 "Sparse tensor cores" (compressed operand A, 2-bit index per
+ *       kept value, groups along the reduction axis) and "Quantization"
+ *       (FP8 E4M3 with one scale per row or channel), section 5.1 (magnitude
+ *       pruning and round-to-nearest are the basic methods).
+ *  [EXT] OCP 8-bit floating point specification, E4M3 encoding (bias 7,
+ *       three mantissa bits, no infinities, largest finite 448).
+ *
+ * Readings where the pages are silent (each one is listed in the design notes):
+ *  R1 ties between equal magnitudes go to the lower index;
+ *  R2 a group always keeps exactly two positions, even when it holds fewer
+ *     than two non-zeros (a kept zero is stored as zero);
+ *  R3 metadata nibble of a group = i0 | (i1 << 2) with i0 < i1; the canonical
+ *     byte order is row-major, two groups per byte, even group in the low
+ *     nibble;
+ *  R4 E4M3 scale = amax / 448 and inverse = 448 / amax, each a correctly
+ *     rounded fp32 division; q = E4M3(round-to-nearest-even, saturating)
+ *     of the fp32 product v * inverse; amax == 0 gives scale 1 and q = 0;
+ *  R5 prune on bf16 magnitudes first, then quantize the kept values.
+ *
+ * Parity pins live in tests/test_oracle_pins.py.  The metadata image
+ * permutation (orc_meta_image) is pinned only by its bijectivity and by
+ * hand-derived positions from its written layout, and finally by the GPU
+ * GEMM, which reads it through the tensor cores: it says "parity pinned by
+ * layout spec" rather than by a page.
+ */
+#include <stdint.h>
+#include <stddef.h>
+#include <string.h>
+#include <math.h>
+
+/* ------------------------------------------------------------------ */
+/* bf16 helpers                                                         */
+/* ------------------------------------------------------------------ */
+
+/* Exact value of a bf16 bit pattern (bf16 is the top half of an fp32). */
+double orc_bf16_to_double(uint16_t b)
+{
+    uint32_t u = ((uint32_t)b) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+static float bf16_to_float(uint16_t b)
+{
+    uint32_t u = ((uint32_t)b) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/* Magnitude key: the bf16 bits without the sign.  For finite values the
+ * integer order of these keys is the order of |v| (IEEE sign-magnitude),
+ * and +0 / -0 compare equal. */
+static int mag_key(uint16_t b) { return (int)(b & 0x7FFFu); }
+
+/* ------------------------------------------------------------------ */
+/* 1. Magnitude 2:4 prune of one group of four  [P3 "How to make a     */
+/*    model 2:4 sparse"; P1 worked example]                             */
+/* ------------------------------------------------------------------ */
+
+/* Position i survives iff fewer than two other positions beat it, where j
+ * beats i when |v_j| > |v_i|, or |v_j| == |v_i| and j < i (reading R1).
+ * Exactly two positions survive for any input (reading R2).
+ * Returns the metadata nibble i0 | (i1 << 2) and the two kept indices. */
+int orc_prune_group(const uint16_t v[4], int *i0, int *i1)
+{
+    int kept[2];
+    int nk = 0;
+    for (int i = 0; i < 4; ++i) {
+        int beaten_by = 0;
+        for (int j = 0; j < 4; ++j) {
+            if (j == i) continue;
+            if (mag_key(v[j]) > mag_key(v[i])) beaten_by++;
+            else if (mag_key(v[j]) == mag_key(v[i]) && j < i) beaten_by++;
+        }
+        if (beaten_by < 2) kept[nk++] = i;   /* i ascends, so kept[0] < kept[1] */
+    }
+    /* nk == 2 always: the "beats" relation is a strict total order. */
+    *i0 = kept[0];
+    *i1 = kept[1];
+    return kept[0] | (kept[1] << 2);
+}
+
+/* ------------------------------------------------------------------ */
+/* 2. Prune + compress whole rows (bf16 values)  [P3 "How 2:4 sparsity */
+/*    works": half-size value array + 2-bit index per kept value]       */
+/* ------------------------------------------------------------------ */
+
+/* src: [rows x K] bf16 bits, row stride ld elements.  K % 4 == 0.
+ * pruned:     [rows x K]   bf16 bits, the zeroed dense matrix (may be NULL)
+ * values:     [rows x K/2] bf16 bits, kept values in ascending index order
+ * meta_canon: [rows x K/8] bytes, canonical nibbles (reading R3)          */
+void orc_prune_compress_bf16(const uint16_t *src, int64_t rows, int64_t K, int64_t ld,
+                             uint16_t *pruned, uint16_t *values, uint8_t *meta_canon)
+{
+    if (rows <= 0 || K <= 0) return;
+    for (int64_t r = 0; r < rows; ++r) {
+        if (meta_canon) memset(meta_canon + r * (K / 8), 0, (size_t)(K / 8));
+        for (int64_t g = 0; g < K / 4; ++g) {
+            const uint16_t *v = src + r * ld + 4 * g;
+            int i0, i1;
+            int nib = orc_prune_group(v, &i0, &i1);
+            if (values) {
+                values[r * (K / 2) + 2 * g + 0] = v[i0];
+                values[r * (K / 2) + 2 * g + 1] = v[i1];
+            }
+            if (pruned) {
+                for (int i = 0; i < 4; ++i)
+                    pruned[r * K + 4 * g + i] = (i == i0 || i == i1) ? v[i] : (uint16_t)0;
+            }
+            if (meta_canon) {
+                uint8_t *byte = meta_canon + r * (K / 8) + g / 2;
+                *byte |= (uint8_t)(nib << ((g % 2) * 4));
+            }
+        }
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* 3. Decompress: scatter kept values back into zeros  [P3 "How 2:4    */
+/*    sparsity works"]                                                  */
+/* ------------------------------------------------------------------ */
+
+/* Element-size agnostic: elem_bytes is 2 (bf16) or 1 (e4m3 codes). */
+void orc_decompress(const void *values, const uint8_t *meta_canon, int64_t rows, int64_t K,
+                    int elem_bytes, void *dst)
+{
+    const uint8_t *vb = (const uint8_t *)values;
+    uint8_t *db = (uint8_t *)dst;
+    memset(dst, 0, (size_t)(rows * K * elem_bytes));
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t g = 0; g < K / 4; ++g) {
+            int nib = (meta_canon[r * (K / 8) + g / 2] >> ((g % 2) * 4)) & 0xF;
+            int i0 = nib & 3, i1 = (nib >> 2) & 3;
+            memcpy(db + (r * K + 4 * g + i0) * elem_bytes,
+                   vb + (r * (K / 2) + 2 * g + 0) * elem_bytes, (size_t)elem_bytes);
+            memcpy(db + (r * K + 4 * g + i1) * elem_bytes,
+                   vb + (r * (K / 2) + 2 * g + 1) * elem_bytes, (size_t)elem_bytes);
+        }
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* 4. FP8 E4M3  [P4 "Quantization"; EXT: OCP FP8 spec]                  */
+/* ------------------------------------------------------------------ */
+
+/* Value of an E4M3 code: sign, 4-bit exponent (bias 7), 3-bit mantissa;
+ * exponent field 0 is subnormal (m * 2^-9); S.1111.111 is NaN; there are no
+ * infinities. */
+double orc_e4m3_decode(uint8_t q)
+{
+    int s = (q >> 7) & 1;
+    int e = (q >> 3) & 0xF;
+    int m = q & 7;
+    double mag;
+    if (e == 0xF && m == 7) return NAN;
+    if (e == 0) mag = ldexp((double)m, -9);
+    else        mag = ldexp(1.0 + m / 8.0, e - 7);
+    return s ? -mag : mag;
+}
+
+/* Round-to-nearest-even to E4M3 with saturation to +-448 (reading R4).
+ * x is an fp32 value carried exactly in a double. */
+uint8_t orc_e4m3_encode(double x)
+{
+    uint8_t sign = (x < 0.0 || (x == 0.0 && signbit(x))) ? 0x80 : 0x00;
+    double a = fabs(x);
+    if (a >= 448.0) return (uint8_t)(sign | 0x7E);        /* largest finite */
+    /* quantum (spacing of representable values) of the binade holding a;
+     * below the smallest normal 2^-6 the spacing is the subnormal step 2^-9 */
+    int e;
+    if (a < ldexp(1.0, -6)) {
+        e = -6;
+    } else {
+        e = (int)floor(log2(a));
+        /* guard log2 rounding at exact powers of two */
+        if (ldexp(1.0, e) > a) e -= 1;
+        if (ldexp(1.0, e + 1) <= a) e += 1;
+    }
+    double quantum = ldexp(1.0, e - 3);
+    double t = a / quantum;              /* exact: quantum is a power of two */
+    double fl = floor(t);
+    double frac = t - fl;
+    double n;
+    if (frac > 0.5) n = fl + 1.0;
+    else if (frac < 0.5) n = fl;
+    else n = (fmod(fl, 2.0) == 0.0) ? fl : fl + 1.0;      /* tie: to even */
+    double r = n * quantum;               /* the rounded magnitude */
+    if (r > 448.0) r = 448.0;             /* cannot happen below 448, kept for clarity */
+    if (r == 0.0) return sign;
+    /* encode r */
+    if (r < ldexp(1.0, -6)) {             /* subnormal: r = m * 2^-9 */
+        int m = (int)(r / ldexp(1.0, -9));
+        return (uint8_t)(sign | m);
+    }
+    int re = (int)floor(log2(r));
+    if (ldexp(1.0, re) > r) re -= 1;
+    if (ldexp(1.0, re + 1) <= r) re += 1;
+    int m = (int)((r / ldexp(1.0, re) - 1.0) * 8.0);
+    return (uint8_t)(sign | ((re + 7) << 3) | m);
+}
+
+/* fp32 correctly rounded quotient (the C compiler evaluates float / float in
+ * fp32 round-to-nearest under the default environment). */
+static float div_f32(float a, float b) { volatile float q = a / b; return q; }
+static float mul_f32(float a, float b) { volatile float p = a * b; return p; }
+
+/* Row scale and inverse from the row's amax (reading R4). */
+void orc_e4m3_row_scale(float amax, float *scale, float *inv)
+{
+    if (amax == 0.0f) { *scale = 1.0f; *inv = 0.0f; return; }
+    *scale = div_f32(amax, 448.0f);
+    *inv = div_f32(448.0f, amax);
+}
+
+/* Per-row E4M3 quantization of a dense bf16 matrix (X per token).
+ * q: [rows x K] codes; scales: [rows]. */
+void orc_quantize_rows_e4m3(const uint16_t *src, int64_t rows, int64_t K, int64_t ld,
+                            uint8_t *q, float *scales)
+{
+    for (int64_t r = 0; r < rows; ++r) {
+        float amax = 0.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            float a = fabsf(bf16_to_float(src[r * ld + k]));
+            if (a > amax) amax = a;
+        }
+        float scale, inv;
+        orc_e4m3_row_scale(amax, &scale, &inv);
+        scales[r] = scale;
+        for (int64_t k = 0; k < K; ++k)
+            q[r * K + k] = orc_e4m3_encode((double)mul_f32(bf16_to_float(src[r * ld + k]), inv));
+    }
+}
+
+/* Prune + compress with E4M3 output (reading R5: prune on bf16 magnitudes,
+ * then quantize kept values with the row scale).  The row amax is taken over
+ * the whole input row; for a sparse row it equals the pruned row's amax
+ * because every group keeps its largest magnitude.
+ *
+ * Hybrid tiles [P1 "Dense Fallback and Hybrid Sparsity Design"; P2 Spense and
+ * PATCH abstracts]: when tile_dense_mask is not NULL it holds one byte per
+ * 128 x 128 tile (row-block major, ceil(rows/128) x K/128); a non-zero byte
+ * keeps that tile dense.  A dense tile's values are quantized unpruned into
+ * dense_q ([rows x K], other tiles untouched); its slots in values are 0 and
+ * its canonical nibbles are 0x4 (indices 0 and 1).
+ * values_q: [rows x K/2]; meta_canon: [rows x K/8]; scales: [rows]. */
+void orc_prune_compress_e4m3(const uint16_t *src, int64_t rows, int64_t K, int64_t ld,
+                             const uint8_t *tile_dense_mask,
+                             uint8_t *values_q, uint8_t *meta_canon, float *scales,
+                             uint8_t *dense_q)
+{
+    int64_t KT = K / 128;
+    if (rows <= 0 || K <= 0) return;
+    for (int64_t r = 0; r < rows; ++r) {
+        float amax = 0.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            float a = fabsf(bf16_to_float(src[r * ld + k]));
+            if (a > amax) amax = a;
+        }
+        float scale, inv;
+        orc_e4m3_row_scale(amax, &scale, &inv);
+        scales[r] = scale;
+        memset(meta_canon + r * (K / 8), 0, (size_t)(K / 8));
+        for (int64_t g = 0; g < K / 4; ++g) {
+            const uint16_t *v = src + r * ld + 4 * g;
+            int dense_tile = tile_dense_mask &&
+                             tile_dense_mask[(r / 128) * KT + (4 * g) / 128] != 0;
+            int nib;
+            if (dense_tile) {
+                nib = 0x4;
+                values_q[r * (K / 2) + 2 * g + 0] = 0;
+                values_q[r * (K / 2) + 2 * g + 1] = 0;
+                for (int i = 0; i < 4; ++i)
+                    dense_q[r * K + 4 * g + i] =
+                        orc_e4m3_encode((double)mul_f32(bf16_to_float(v[i]), inv));
+            } else {
+                int i0, i1;
+                nib = orc_prune_group(v, &i0, &i1);
+                values_q[r * (K / 2) + 2 * g + 0] =
+                    orc_e4m3_encode((double)mul_f32(bf16_to_float(v[i0]), inv));
+                values_q[r * (K / 2) + 2 * g + 1] =
+                    orc_e4m3_encode((double)mul_f32(bf16_to_float(v[i1]), inv));
+            }
+            meta_canon[r * (K / 8) + g / 2] |= (uint8_t)(nib << ((g % 2) * 4));
+        }
+    }
+}
+
+/* Same hybrid treatment for bf16 output: dense tiles are copied unpruned
+ * into dense_out ([rows x K]); their value slots are 0 and nibbles 0x4. */
+void orc_prune_compress_bf16_hybrid(const uint16_t *src, int64_t rows, int64_t K, int64_t ld,
+                                    const uint8_t *tile_dense_mask,
+                                    uint16_t *values, uint8_t *meta_canon, uint16_t *dense_out)
+{
+    int64_t KT = K / 128;
+    if (rows <= 0 || K <= 0) return;
+    for (int64_t r = 0; r < rows; ++r) {
+        memset(meta_canon + r * (K / 8), 0, (size_t)(K / 8));
+        for (int64_t g = 0; g < K / 4; ++g) {
+            const uint16_t *v = src + r * ld + 4 * g;
+            int dense_tile = tile_dense_mask &&
+                             tile_dense_mask[(r / 128) * KT + (4 * g) / 128] != 0;
+            int nib;
+            if (dense_tile) {
+                nib = 0x4;
+                values[r * (K / 2) + 2 * g + 0] = 0;
+                values[r * (K / 2) + 2 * g + 1] = 0;
+                for (int i = 0; i < 4; ++i) dense_out[r * K + 4 * g + i] = v[i];
+            } else {
+                int i0, i1;
+                nib = orc_prune_group(v, &i0, &i1);
+                values[r * (K / 2) + 2 * g + 0] = v[i0];
+                values[r * (K / 2) + 2 * g + 1] = v[i1];
+            }
+            meta_canon[r * (K / 8) + g / 2] |= (uint8_t)(nib << ((g % 2) * 4));
+        }
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* 5. Metadata image: the canonical nibbles rearranged into the order   */
+/*    the sparse tensor-core instruction reads them from tensor memory. */
+/*    Written from the layout specification in include/sp24.h, not from */
+/*    the CUDA code.  Parity pinned by layout spec (see header).        */
+/* ------------------------------------------------------------------ */
+
+/* Image = sequence of 2048-byte chunks, chunk (rb, kc) at index
+ * rb * (K/128) + kc, for row block rb (128 rows, rows past the end count as
+ * all-zero rows whose groups keep indices 0 and 1, nibble 0x4) and K-chunk kc
+ * (128 consecutive K positions = 32 groups).  A chunk is 128 image rows of 16
+ * bytes; image row L is 4 little-endian 32-bit words w = 0..3.
+ *
+ * 16-bit operands (bf16): word w of image row L covers the 32 K positions
+ * [32w, 32w+32) of the chunk, split in two 16-position halves h:
+ *     h = (L / 8) % 2,  r = 16 * (L / 16) + (L % 8)
+ *     bits  0..15 = nibbles of groups 8w + 4h + 0..3 of row r     (nibble j at bits 4j)
+ *     bits 16..31 = nibbles of groups 8w + 4h + 0..3 of row r + 8
+ * 8-bit operands (e4m3): image row L is row L; its 16 bytes are the row's 32
+ * canonical nibbles of the chunk in order (group 2b in the low nibble of
+ * byte b). */
+static int canon_nib(const uint8_t *canon, int64_t rows, int64_t K, int64_t r, int64_t g)
+{
+    if (r >= rows) return 0x4;
+    return (canon[r * (K / 8) + g / 2] >> ((g % 2) * 4)) & 0xF;
+}
+
+void orc_meta_image(const uint8_t *canon, int64_t rows, int64_t K, int is_8bit,
+                    const uint8_t *tile_dense_mask, uint8_t *image)
+{
+    int64_t RB = (rows + 127) / 128, KC = K / 128;
+    for (int64_t rb = 0; rb < RB; ++rb) {
+        for (int64_t kc = 0; kc < KC; ++kc) {
+            uint8_t *chunk = image + (rb * KC + kc) * 2048;
+            int dense = tile_dense_mask && tile_dense_mask[rb * KC + kc] != 0;
+            for (int L = 0; L < 128; ++L) {
+                for (int w = 0; w < 4; ++w) {
+                    uint32_t word = 0;
+                    if (!is_8bit) {
+                        int h = (L / 8) % 2;
+                        int64_t r = rb * 128 + 16 * (L / 16) + (L % 8);
+                        for (int j = 0; j < 4; ++j) {
+                            int64_t g = kc * 32 + 8 * w + 4 * h + j;
+                            uint32_t lo = dense ? 0x4u : (uint32_t)canon_nib(canon, rows, K, r, g);
+                            uint32_t hi = dense ? 0x4u : (uint32_t)canon_nib(canon, rows, K, r + 8, g);
+                            word |= lo << (4 * j);
+                            word |= hi << (16 + 4 * j);
+                        }
+                    } else {
+                        int64_t r = rb * 128 + L;
+                        for (int j = 0; j < 8; ++j) {
+                            int64_t g = kc * 32 + 8 * w + j;
+                            uint32_t nib = dense ? 0x4u : (uint32_t)canon_nib(canon, rows, K, r, g);
+                            word |= nib << (4 * j);
+                        }
+                    }
+                    for (int b = 0; b < 4; ++b)
+                        chunk[L * 16 + w * 4 + b] = (uint8_t)((word >> (8 * b)) & 0xFF);
+                }
+            }
+        }
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* 6. GEMM in fp64 on dequantized operands  [P4 "Sparse tensor cores": */
+/*    the sparse product equals the dense product of the pruned matrix] */
+/* ------------------------------------------------------------------ */
+
+/* Y[m][n] = sum_k X[m][k] * W[n][k];  A[m][n] = sum_k |X[m][k] * W[n][k]|.
+ * X: [M x K], W: [N x K], both row-major fp64.  A may be NULL. */
+void orc_gemm_f64(const double *X, const double *W, int64_t M, int64_t N, int64_t K,
+                  double *Y, double *A)
+{
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t n = 0; n < N; ++n) {
+            double y = 0.0, a = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                double p = X[m * K + k] * W[n * K + k];
+                y += p;
+                a += fabs(p);
+            }
+            Y[m * N + n] = y;
+            if (A) A[m * N + n] = a;
+        }
+    }
+}
+
+/* The same contraction evaluated only at listed (m, n) pairs, for sampled
+ * checks at full problem sizes. */
+void orc_gemm_f64_sampled(const double *X, const double *W, int64_t K,
+                          const int64_t *ms, const int64_t *ns, int64_t count,
+                          double *Y, double *A)
+{
+    for (int64_t i = 0; i < count; ++i) {
+        double y = 0.0, a = 0.0;
+        for (int64_t k = 0; k < K; ++k) {
+            double p = X[ms[i] * K + k] * W[ns[i] * K + k];
+            y += p;
+            a += fabs(p);
+        }
+        Y[i] = y;
+        if (A) A[i] = a;
+    }
+}
+
+/* Sparse-sum form: for each kept value of W's row, the index selects the
+ * matching element of X's row [P4 "Sparse tensor cores"].
+ * wvals: [N x K/2] dequantized kept values; meta_canon: [N x K/8]. */
+void orc_gemm_sparse_f64(const double *X, int64_t M, int64_t K,
+                         const double *wvals, const uint8_t *meta_canon, int64_t N,
+                         double *Y)
+{
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t n = 0; n < N; ++n) {
+            double y = 0.0;
+            for (int64_t g = 0; g < K / 4; ++g) {
+                int nib = (meta_canon[n * (K / 8) + g / 2] >> ((g % 2) * 4)) & 0xF;
+                int i0 = nib & 3, i1 = (nib >> 2) & 3;
+                y += wvals[n * (K / 2) + 2 * g + 0] * X[m * K + 4 * g + i0];
+                y += wvals[n * (K / 2) + 2 * g + 1] * X[m * K + 4 * g + i1];
+            }
+            Y[m * N + n] = y;
+        }
+    }
+}
+
+/* Array form of orc_e4m3_encode for the Python wrapper (x holds fp32 values
+ * carried exactly in doubles). */
+void orc_e4m3_encode_array(const double *x, int64_t n, uint8_t *q)
+{
+    for (int64_t i = 0; i < n; ++i) q[i] = orc_e4m3_encode(x[i]);
+}

@@ -1,0 +1,342 @@
+"""Pins for the CPU oracle: each test ties the oracle to something other than
+itself -- a value the pages print, a closed form, an invariant, brute force,
+or an independent library routine.  CPU only.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as orc
+from semi_structured_sparse_02_b200 import inputs
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def bf16(values):
+    return inputs.to_bf16_bits(np.asarray(values, dtype=np.float32))
+
+
+# ---------------------------------------------------------------------------
+# prune: worked example, brute force over ties, torch top-k recipe
+# ---------------------------------------------------------------------------
+
+def test_worked_example_from_the_page():
+    g = json.load(open(os.path.join(GOLDEN, "worked_example.json")))
+    v = bf16(g["dense"])
+    nib, i0, i1 = orc.prune_group(v)
+    assert [i0, i1] == g["kept_indices"]
+    assert nib == (i0 | (i1 << 2)) == 0xC
+    # the canonical byte holds two groups: pad the row with an all-zero group
+    row = np.concatenate([v, bf16([0.0] * 4)]).reshape(1, 8)
+    pruned, values, meta = orc.prune_compress_bf16(row)
+    assert pruned[0, :4].tolist() == bf16(g["pruned"]).tolist()
+    assert values[0, :2].tolist() == bf16([g["dense"][0], g["dense"][3]]).tolist()
+    assert meta.tolist() == [[0x4C]]  # group 0 -> low nibble 0xC; zero group keeps 0,1
+
+
+def _stable_sort_rule(mags):
+    # The rule written a second way: sort positions by descending magnitude,
+    # equal magnitudes keeping ascending position order; keep the first two.
+    order = sorted(range(4), key=lambda i: (-mags[i], i))
+    return sorted(order[:2])
+
+
+def test_prune_brute_force_all_tie_patterns_and_signs():
+    levels = [0.0, 1.0, 2.0, 3.0]
+    for mags in itertools.product(range(4), repeat=4):
+        for signs in itertools.product([1.0, -1.0], repeat=4):
+            vals = [s * levels[m] for s, m in zip(signs, mags)]
+            _, i0, i1 = orc.prune_group(bf16(vals))
+            assert [i0, i1] == _stable_sort_rule([levels[m] for m in mags]), (vals, i0, i1)
+
+
+def test_prune_agrees_with_torch_topk_recipe_on_tie_free_data():
+    # "2:4 Structured Sparsity Explained", section "Running a 2:4 model in
+    # PyTorch": keep the top-2 |w| of each group of four via topk.
+    W = inputs.normal_bf16((64, 512), 1.0, seed=11)
+    w = torch.from_numpy(W.view(np.int16)).view(torch.bfloat16).float()
+    groups = w.abs().reshape(-1, 4)
+    tie_free = torch.tensor([len(set(g.tolist())) == 4 for g in groups])
+    mask = torch.zeros_like(groups, dtype=torch.bool)
+    mask.scatter_(1, groups.topk(2, dim=1).indices, True)
+    pruned, _, _ = orc.prune_compress_bf16(W)
+    ours = (torch.from_numpy(pruned.view(np.int16)).view(torch.bfloat16).float()
+            .reshape(-1, 4) != 0)
+    assert tie_free.float().mean() > 0.95
+    assert torch.equal(ours[tie_free], mask[tie_free])
+
+
+def test_pattern_exactly_two_indices_and_half_zeros():
+    W = inputs.normal_bf16((128, 1024), 0.02, seed=3)
+    pruned, values, meta = orc.prune_compress_bf16(W)
+    nibs = np.stack([meta & 0xF, meta >> 4], axis=-1).reshape(128, -1)
+    i0, i1 = nibs & 3, nibs >> 2
+    assert np.all(i0 < i1)  # two distinct positions per group, ascending
+    nz = (pruned.reshape(128, -1, 4) & 0x7FFF) != 0
+    assert np.all(nz.sum(-1) <= 2)
+    if np.all((W & 0x7FFF) != 0):  # continuous draws: no exact zeros
+        assert (pruned & 0x7FFF == 0).mean() == 0.5
+
+
+def test_kept_zeros_when_group_has_fewer_than_two_nonzeros():
+    v = bf16([0.0, 0.0, -0.0, 0.0])
+    assert orc.prune_group(v)[1:] == (0, 1)
+    v = bf16([0.0, 0.0, 5.0, 0.0])
+    assert orc.prune_group(v)[1:] == (0, 2)
+
+
+# ---------------------------------------------------------------------------
+# storage counts
+# ---------------------------------------------------------------------------
+
+def test_storage_36_bits_per_4_and_bit_identities():
+    s = json.load(open(os.path.join(GOLDEN, "storage.json")))
+    X, W = inputs.tiny(0)
+    _, values, meta = orc.prune_compress_bf16(W)
+    dense_bytes = W.nbytes
+    assert values.nbytes + meta.nbytes == 73728
+    assert dense_bytes == 131072
+    assert (values.nbytes + meta.nbytes) * 64 == dense_bytes * s["fp16_sparse_bits_per_4"]
+    assert abs((values.nbytes + meta.nbytes) / dense_bytes - s["fp16_sparse_relative_size_approx"]) < 0.01
+    # bits per element of 2:4 on b-bit values = b/2 + 1 (index bits counted)
+    bits_per_elem = (values.nbytes + meta.nbytes) * 8 / W.size
+    assert bits_per_elem == s["budget_fp16_bits_per_elem"]
+    vq, mq, sq, _ = orc.prune_compress_e4m3(W)
+    assert (vq.nbytes + mq.nbytes) * 8 / W.size == 5.0  # 0.625 of dense 8-bit
+    for m in range(1, 9):  # 2:4 on 2m-bit values costs as much as dense (m+1)-bit
+        assert (2 * m) / 2 + 1 == m + 1
+    for k in (4, 8, 16):
+        assert abs(k / (k / 2 + 1) - 2 * k / (k + 2)) < 1e-12
+    assert abs(math.log2(6) / 4 - s["ideal_index_bits_per_elem_approx"]) < 0.005
+    # the metadata costs exactly 1 bit per dense element (4 bits per group of 4)
+    assert mq.nbytes * 8 / W.size == s["hardware_index_bits_per_elem"]
+
+
+# ---------------------------------------------------------------------------
+# round trip
+# ---------------------------------------------------------------------------
+
+def test_decompress_of_compress_is_prune_bit_exact():
+    W = inputs.weights_with_outliers(256, 512, seed=5)
+    pruned, values, meta = orc.prune_compress_bf16(W)
+    assert np.array_equal(orc.decompress(values, meta, 256, 512), pruned)
+    vq, mq, sq, _ = orc.prune_compress_e4m3(W)
+    assert np.array_equal(mq, meta)  # quantizing does not change which values are kept
+    dq = orc.decompress(vq, mq, 256, 512)
+    inv = np.array([orc.e4m3_row_scale(float(a))[1] for a in
+                    np.abs(orc.bf16_bits_to_f64(W)).max(1).astype(np.float32)], np.float32)
+    expect = orc.e4m3_encode(orc.bf16_bits_to_f64(pruned).astype(np.float32) * inv[:, None])
+    assert np.array_equal(dq, expect)
+
+
+# ---------------------------------------------------------------------------
+# e4m3
+# ---------------------------------------------------------------------------
+
+def _all_finite_bf16():
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    vals = orc.bf16_bits_to_f64(bits)
+    return vals[np.isfinite(vals)]
+
+
+def test_e4m3_matches_torch_cast_in_range_exhaustive():
+    x = _all_finite_bf16()
+    for inv in (1.0, 0.37109375, 3.0, 1.0 / 3.0, 1000.0, 1e-3):
+        y = (x.astype(np.float32) * np.float32(inv)).astype(np.float32)
+        y = y[np.abs(y) < 448.0]
+        ours = orc.e4m3_encode(y)
+        ref = torch.from_numpy(y).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+        # torch gives +0 for tiny negatives that round to zero; compare values
+        assert np.array_equal(orc.e4m3_decode(ours), orc.e4m3_decode(ref))
+
+
+def test_e4m3_representables_fixed_points_midpoints_even_saturation():
+    codes = [c for c in range(256) if not math.isnan(orc.e4m3_decode(np.array([c]))[0])]
+    assert len(codes) == 254
+    vals = orc.e4m3_decode(np.array(codes))
+    assert np.array_equal(orc.e4m3_encode(vals), np.array(codes, np.uint8)) or \
+        np.array_equal(orc.e4m3_decode(orc.e4m3_encode(vals)), vals)
+    pos = np.unique(vals[vals >= 0])
+    assert pos.max() == 448.0 and pos[1] == 2.0 ** -9
+    mids = (pos[:-1] + pos[1:]) / 2
+    q = orc.e4m3_decode(orc.e4m3_encode(mids))
+    lo_code = orc.e4m3_encode(pos[:-1])
+    hi_code = orc.e4m3_encode(pos[1:])
+    expect = np.where(lo_code % 2 == 0, pos[:-1], pos[1:])
+    assert np.array_equal(q, expect)
+    assert np.all(lo_code % 2 != hi_code % 2)
+    assert orc.e4m3_encode(np.array([448.0, 460.0, 464.0, 1e4]))[:].tolist() == [0x7E] * 4
+    assert orc.e4m3_encode(np.array([-448.0, -1e6])).tolist() == [0xFE, 0xFE]
+    grid = np.linspace(-500, 500, 200001).astype(np.float32)
+    dec = orc.e4m3_decode(orc.e4m3_encode(grid))
+    assert np.all(np.diff(dec) >= 0)
+
+
+def test_row_scale_closed_form_and_amax_invariant():
+    W = inputs.weights_with_outliers(128, 1024, seed=9)
+    vq, mq, scales, _ = orc.prune_compress_e4m3(W)
+    w = orc.bf16_bits_to_f64(W)
+    pruned, _, _ = orc.prune_compress_bf16(W)
+    pw = orc.bf16_bits_to_f64(pruned)
+    amax = np.abs(w).max(1)
+    assert np.array_equal(np.abs(pw).max(1), amax)  # each group keeps its max
+    assert np.array_equal(scales, (amax.astype(np.float32) / np.float32(448.0)).astype(np.float32))
+    # the largest magnitude of each row lands on +-448
+    deq = orc.e4m3_decode(vq)
+    assert np.all(np.abs(deq).max(1) == 448.0)
+    s, inv = orc.e4m3_row_scale(0.0)
+    assert (s, inv) == (1.0, 0.0)
+    q, sc = orc.quantize_rows_e4m3(np.zeros((2, 64), np.uint16))
+    assert np.all(q == 0) and np.all(sc == 1.0)
+
+
+def test_quantized_error_within_half_ulp_of_scaled_value():
+    X = inputs.normal_bf16((8, 512), 1.0, seed=21)
+    q, s = orc.quantize_rows_e4m3(X)
+    x = orc.bf16_bits_to_f64(X)
+    deq = orc.e4m3_decode(q) * s[:, None].astype(np.float64)
+    # relative spacing of e4m3 normals is 2^-3: error <= half a spacing of |x|
+    # plus the subnormal step (2^-9 * s) for tiny values
+    bound = np.abs(x) * 2.0 ** -4 * (1 + 1e-6) + 2.0 ** -10 * s[:, None]
+    assert np.all(np.abs(deq - x) <= bound)
+
+
+# ---------------------------------------------------------------------------
+# metadata image layout
+# ---------------------------------------------------------------------------
+
+def _image_positions(is_8bit):
+    rows, K = 128, 128
+    pos = {}
+    base = np.full((rows, K // 8), 0x44, np.uint8)
+    for r in range(rows):
+        for g in range(32):
+            c = base.copy()
+            b = c[r, g // 2]
+            c[r, g // 2] = (b & 0xF0) | 0x9 if g % 2 == 0 else (b & 0x0F) | 0x90
+            img = orc.meta_image(c, rows, K, is_8bit)
+            nibs = np.stack([img & 0xF, img >> 4], -1).reshape(-1)
+            hit = np.nonzero(nibs == 0x9)[0]
+            assert hit.size == 1
+            pos[(r, g)] = int(hit[0])
+    return pos
+
+
+@pytest.mark.parametrize("is_8bit", [False, True])
+def test_meta_image_is_a_bijection_with_spec_positions(is_8bit):
+    pos = _image_positions(is_8bit)
+    assert sorted(pos.values()) == list(range(128 * 32))
+
+    def at(L, w, bit):  # nibble index of image row L, word w, bit offset
+        return (L * 16 + w * 4) * 2 + bit // 4
+
+    if not is_8bit:
+        assert pos[(0, 0)] == at(0, 0, 0)
+        assert pos[(8, 0)] == at(0, 0, 16)
+        assert pos[(0, 4)] == at(8, 0, 0)
+        assert pos[(16, 8)] == at(16, 1, 0)
+        assert pos[(9, 31)] == at(9, 3, 28)
+        assert pos[(127, 5)] == at(127, 0, 20)
+        assert pos[(119, 5)] == at(127, 0, 4)
+    else:
+        for (r, g), p in pos.items():
+            assert p == r * 32 + g
+
+
+def test_meta_image_pads_rows_with_valid_nibbles():
+    W = inputs.normal_bf16((40, 256), 1.0, seed=2)
+    _, _, meta = orc.prune_compress_bf16(W)
+    img = orc.meta_image(meta, 40, 256, False)
+    assert img.size == 2 * 2048
+    img8 = orc.meta_image(meta, 40, 256, True).reshape(2, 128, 16)
+    assert np.all(img8[:, 40:, :] == 0x44)
+
+
+# ---------------------------------------------------------------------------
+# GEMM
+# ---------------------------------------------------------------------------
+
+def test_gemm_f64_matches_numpy_matmul():
+    g = np.random.default_rng(1)
+    X = g.normal(size=(7, 96))
+    W = g.normal(size=(13, 96))
+    Y, A = orc.gemm_f64(X, W)
+    assert np.allclose(Y, X @ W.T, rtol=1e-12, atol=1e-12)
+    assert np.allclose(A, np.abs(X) @ np.abs(W).T, rtol=1e-12, atol=1e-12)
+    ms = np.array([0, 6, 3]); ns = np.array([12, 0, 5])
+    ys, as_ = orc.gemm_f64_sampled(X, W, ms, ns)
+    assert np.array_equal(ys, Y[ms, ns]) and np.array_equal(as_, A[ms, ns])
+
+
+def test_sparse_sum_equals_dense_product_of_pruned_matrix_exactly():
+    g = np.random.default_rng(2)
+    Xi = g.integers(-8, 9, size=(9, 64)).astype(np.float32)
+    Wi = g.integers(-8, 9, size=(17, 64)).astype(np.float32)
+    Wb = bf16(Wi)
+    pruned, values, meta = orc.prune_compress_bf16(Wb)
+    Xd = Xi.astype(np.float64)
+    Yd, _ = orc.gemm_f64(Xd, orc.bf16_bits_to_f64(pruned))
+    Ys = orc.gemm_sparse_f64(Xd, orc.bf16_bits_to_f64(values), meta)
+    assert np.array_equal(Yd, Ys)
+
+
+def test_already_two_four_weights_reduce_to_dense_gemm():
+    g = np.random.default_rng(3)
+    N, K = 16, 64
+    W = np.zeros((N, K), np.float32)
+    for n in range(N):
+        for q in range(K // 4):
+            idx = g.choice(4, size=2, replace=False)
+            W[n, 4 * q + idx] = g.integers(1, 9, size=2) * g.choice([-1, 1], size=2)
+    Wb = bf16(W)
+    pruned, values, meta = orc.prune_compress_bf16(Wb)
+    assert np.array_equal(pruned, Wb)  # prune is the identity on 2:4 input
+    X = g.integers(-5, 6, size=(5, K)).astype(np.float64)
+    Ys = orc.gemm_sparse_f64(X, orc.bf16_bits_to_f64(values), meta)
+    assert np.array_equal(Ys, X @ W.astype(np.float64).T)
+
+
+# ---------------------------------------------------------------------------
+# hybrid tiles
+# ---------------------------------------------------------------------------
+
+def test_hybrid_dense_tiles_and_sparse_tiles():
+    rows, K = 256, 512
+    W = inputs.normal_bf16((rows, K), 0.02, seed=4)
+    mask = inputs.hybrid_mask(rows, K, seed=4)
+    assert mask.sum() == round(0.25 * mask.size)
+    vq, mq, sq, dq = orc.prune_compress_e4m3(W, mask)
+    vq0, mq0, sq0, _ = orc.prune_compress_e4m3(W)
+    q_dense, s_dense = orc.quantize_rows_e4m3(W)
+    assert np.array_equal(sq, sq0) and np.array_equal(sq, s_dense)
+    for rb in range(2):
+        for kt in range(4):
+            rs, ks = slice(128 * rb, 128 * rb + 128), slice(128 * kt, 128 * kt + 128)
+            vs = slice(64 * kt, 64 * kt + 64)
+            ms_ = slice(16 * kt, 16 * kt + 16)
+            if mask[rb, kt]:
+                assert np.all(vq[rs, vs] == 0) and np.all(mq[rs, ms_] == 0x44)
+                assert np.array_equal(dq[rs, ks], q_dense[rs, ks])
+            else:
+                assert np.array_equal(vq[rs, vs], vq0[rs, vs])
+                assert np.array_equal(mq[rs, ms_], mq0[rs, ms_])
+                assert np.all(dq[rs, ks] == 0)
+
+
+# ---------------------------------------------------------------------------
+# tactic rule and manifest arithmetic
+# ---------------------------------------------------------------------------
+
+def test_manifest_example_arithmetic_and_tactic_rule():
+    m = json.load(open(os.path.join(GOLDEN, "manifest_example.json")))
+    assert m["sparse_selected_layers"] + m["dense_fallback_layers"] == m["candidate_layers"]
+    assert round(m["sparse_selected_layers"] / m["eligible_layers"], 4) == m["sparse_selection_ratio"]
+    assert orc.select_tactic([1.0, 2.0, 3.0], [2.0, 2.0, 2.0])[0] == "dense"   # tie -> dense
+    assert orc.select_tactic([1.0, 1.5, 9.0], [2.0, 2.0, 2.0])[0] == "sparse"
+    cov = orc.sparse_gpu_time_coverage([("sparse", 0.684), ("dense", 0.316)])
+    assert abs(cov - m["sparse_gpu_time_coverage"]) < 1e-12
