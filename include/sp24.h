@@ -1,0 +1,264 @@
+/*
+ * sp24.h -- C ABI of the B200 (sm_100a) 2:4 semi-structured sparse GEMM library.
+ *
+ * Y = X * W^T with X [M x K] and W [N x K], both row-major with K contiguous.
+ * 2:4 sparsity: in every group of four consecutive elements along the
+ * reduction axis K at most two are non-zero; the sparse operand is stored as
+ * a half-size value array plus a 2-bit position index for each kept value.
+ *   - "2:4 Structured Sparsity Explained" (tensorcore.si), section
+ *     "How 2:4 sparsity works": the format, 36 bits per group of four FP16.
+ *   - "Production 2:4 Structured Sparsity for LLMs" (oh-bug.com), section
+ *     "Core Mechanisms and Production States of 2:4 Structured Sparsity":
+ *     the worked example [0.42,-0.18,0.07,0.31] -> [0.42,0,0,0.31] and the
+ *     pruned / eligible / selected states.
+ *   - the 2:4-versus-quantization paper (paperpeel.com/paper/2610.28947),
+ *     section 2, "Sparse tensor cores": the sparse MMA takes its first operand
+ *     A compressed and uses the indices to select the matching elements of the
+ *     dense operand B; only one operand is sparse; groups lie along K.
+ *
+ * Conventions for every call:
+ *  - Pointers named *_dev are DEVICE pointers; the caller allocates and frees
+ *    every buffer.  The library allocates nothing on the device.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Every call is asynchronous on that stream unless stated.
+ *  - Argument errors are returned synchronously, before any launch.  A failed
+ *    launch returns SP24_ERR_CUDA.  A device-side bounded wait that expires
+ *    records a code in a device error word, read by sp24_last_device_error().
+ *  - bf16 data are passed as 16-bit patterns, e4m3 data as bytes (OCP FP8
+ *    E4M3: bias 7, 3 mantissa bits, no infinities, largest finite 448).
+ *  - Leading dimensions (ld*) are in elements; every row pitch must be a
+ *    multiple of 16 bytes and every base pointer 16-byte aligned
+ *    (SP24_ERR_ALIGNMENT otherwise).
+ *
+ * Magnitude prune (reading where the pages are silent): in each group the
+ * two positions with the largest |v| survive, comparing bf16 magnitude bits
+ * as integers; equal magnitudes go to the lower index; a group always keeps
+ * exactly two positions, so a group with fewer than two non-zeros keeps
+ * zeros ("How to make a model 2:4 sparse": keep the two with the largest
+ * magnitude).
+ *
+ * Metadata nibble of one group: i0 | (i1 << 2), i0 < i1 the kept positions.
+ *
+ * METADATA IMAGE LAYOUT (what sp24_prune_compress writes and sp24_gemm reads).
+ * The nibbles are stored in the order the sparse tensor-core instruction reads
+ * them from tensor memory, so the GEMM copies them to tensor memory with no
+ * rearrangement.  The image is a sequence of 2048-byte chunks; chunk (rb, kc),
+ * for row block rb (128 rows; rows past the end behave as all-zero rows whose
+ * groups keep positions 0 and 1, nibble 0x4) and K-chunk kc (128 consecutive
+ * K positions = 32 groups), sits at byte offset (rb * (K/128) + kc) * 2048.
+ * A chunk is 128 image rows L of 16 bytes = four little-endian 32-bit words w.
+ *  - 16-bit values (bf16): word w of image row L covers chunk positions
+ *    [32w, 32w+32) in two halves h = (L/8) % 2 of 16 positions; with
+ *    r = 16*(L/16) + L%8 (row within the block):
+ *        bits  0..15: nibbles of groups 8w+4h+0..3 of row r   (nibble j at bit 4j)
+ *        bits 16..31: nibbles of groups 8w+4h+0..3 of row r+8
+ *  - 8-bit values (e4m3): image row L is row L; its 16 bytes hold the row's 32
+ *    nibbles of the chunk in order, even group in the low nibble of a byte.
+ * sp24_meta_bytes() returns the image size.
+ */
+#ifndef SP24_H
+#define SP24_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum sp24_status {
+    SP24_OK = 0,
+    SP24_ERR_INVALID_ARG = 1,       /* a size or enum out of range              */
+    SP24_ERR_NULL = 2,              /* a required pointer is NULL               */
+    SP24_ERR_DTYPE = 3,             /* dtype combination not supported          */
+    SP24_ERR_ALIGNMENT = 4,         /* pointer, pitch or shape misaligned       */
+    SP24_ERR_NOT_2_4 = 5,           /* operand is not eligible for the sparse path */
+    SP24_ERR_UNSUPPORTED_DEVICE = 6,/* current device is not sm_100             */
+    SP24_ERR_CUDA = 7,              /* a CUDA runtime call failed               */
+    SP24_ERR_DEVICE_TIMEOUT = 8,    /* a device-side bounded wait expired       */
+    SP24_ERR_WORKSPACE = 9          /* workspace missing or too small           */
+} sp24_status;
+
+typedef enum sp24_dtype { SP24_BF16 = 0, SP24_E4M3 = 1, SP24_F32 = 2 } sp24_dtype;
+
+typedef enum sp24_tactic { SP24_TACTIC_SPARSE = 0, SP24_TACTIC_DENSE = 1 } sp24_tactic;
+
+/* ---------------------------------------------------------------------- */
+/* Sizes                                                                   */
+/* ---------------------------------------------------------------------- */
+
+/* Bytes of the compressed value array [rows x K/2] of `dtype` (BF16 or E4M3). */
+size_t sp24_values_bytes(int64_t rows, int64_t K, sp24_dtype dtype);
+
+/* Bytes of the metadata image: ceil(rows/128) * (K/128) * 2048. */
+size_t sp24_meta_bytes(int64_t rows, int64_t K);
+
+/* ---------------------------------------------------------------------- */
+/* Prune + compress (kernel 1)                                             */
+/* ---------------------------------------------------------------------- */
+
+/* Magnitude 2:4 prune of src along K and compression, in one pass over src
+ * for BF16 output (three stream-ordered launches for E4M3: row amax, prune,
+ * scale finalize).
+ *   src_dev     bf16 [rows x K], row pitch ld elements.
+ *   out_dtype   SP24_BF16: values are the kept bf16 values.
+ *               SP24_E4M3: kept values quantized per row: scale = amax/448,
+ *               inv = 448/amax (both correctly rounded fp32 divisions, amax
+ *               over the whole input row), q = E4M3 round-to-nearest-even
+ *               saturating of the fp32 product v*inv; amax == 0 gives scale 1
+ *               and q = 0 ("Quantization": FP8 E4M3 needs one scale per row;
+ *               section 5.1: round-to-nearest is the basic quantizer; prune
+ *               before quantize).
+ *   values_dev  [rows x K/2] of out_dtype, contiguous (row pitch K/2).
+ *   meta_dev    metadata image, sp24_meta_bytes(rows, K) bytes.
+ *   row_scales_dev  fp32 [rows], required for E4M3, ignored for BF16.
+ *   tile_dense_mask_dev  NULL, or one byte per 128 x 128 tile of src,
+ *               [ceil(rows/128) x K/128] row-block major; non-zero keeps that
+ *               tile dense (hybrid sparse-dense weights: "Dense Fallback and
+ *               Hybrid Sparsity Design"; the Spense and PATCH abstracts on the
+ *               SlideSparse page).  A dense tile is written unpruned (quantized
+ *               with the row scale for E4M3) into dense_tiles_dev; its value
+ *               slots are written as 0 and its metadata nibbles as 0x4.
+ *   dense_tiles_dev  [rows x K] of out_dtype, contiguous; only dense tiles are
+ *               written.  Required when the mask is given.
+ * Requirements: rows >= 1, K % 128 == 0, ld >= K, ld % 8 == 0.
+ */
+int sp24_prune_compress(const void *src_dev, int64_t rows, int64_t K, int64_t ld,
+                        sp24_dtype out_dtype, void *values_dev, void *meta_dev,
+                        float *row_scales_dev, const uint8_t *tile_dense_mask_dev,
+                        void *dense_tiles_dev, void *stream);
+
+/* Scatter compressed values back to a dense [rows x K] matrix of the same
+ * element type (bf16 bits or e4m3 codes); zeros elsewhere.  Exact inverse of
+ * the compression: decompress(compress(W)) == prune(W) bit for bit.
+ *   values_dev [rows x K/2], meta_dev metadata image, dst_dev [rows x K]. */
+int sp24_decompress(const void *values_dev, const void *meta_dev, int64_t rows, int64_t K,
+                    sp24_dtype dtype, void *dst_dev, void *stream);
+
+/* Per-row (per-token) E4M3 quantization of a dense bf16 matrix, same rule as
+ * the E4M3 prune path: q [rows x K] (row pitch K), scales fp32 [rows]. */
+int sp24_quantize_e4m3_rows(const void *src_dev, int64_t rows, int64_t K, int64_t ld,
+                            void *q_dev, float *scales_dev, void *stream);
+
+/* ---------------------------------------------------------------------- */
+/* GEMM (kernels 2 and 3)                                                  */
+/* ---------------------------------------------------------------------- */
+
+typedef struct sp24_gemm_args {
+    int64_t M, N, K;          /* Y [M x N] = X [M x K] * W [N x K]^T            */
+    sp24_dtype in_dtype;      /* SP24_BF16 or SP24_E4M3 (both operands)          */
+    sp24_dtype out_dtype;     /* SP24_BF16 or SP24_F32                           */
+    sp24_tactic tactic;       /* SPARSE: W given compressed; DENSE: W dense      */
+    const void *X;            /* device, [M x K] row pitch ldx                   */
+    int64_t ldx;
+    const void *W;            /* device; DENSE: [N x K] pitch ldw; SPARSE: values
+                                 [N x K/2] pitch ldw (elements of a values row)  */
+    int64_t ldw;
+    const void *W_meta;       /* device; SPARSE: metadata image of W             */
+    const float *x_scales;    /* device fp32 [M]; E4M3 only (per token)          */
+    const float *w_scales;    /* device fp32 [N]; E4M3 only (per output channel) */
+    const uint8_t *tile_dense_mask; /* device; SPARSE E4M3 only: NULL or the
+                                 [N/128 x K/128] hybrid tile mask                */
+    const void *W_dense_tiles;/* device [N x K] pitch K; read only at dense tiles */
+    void *Y;                  /* device, [M x N] row pitch ldy                   */
+    int64_t ldy;
+    void *workspace;          /* device split-K workspace (see below) or NULL    */
+    size_t workspace_bytes;
+} sp24_gemm_args;
+
+/* Bytes of split-K workspace the call will use (0 if it needs none).  The
+ * workspace must be zero-filled once before its first use; every call that
+ * returns SP24_OK leaves its counter words at zero again.  Calls that share a
+ * workspace must not overlap on the GPU. */
+size_t sp24_gemm_workspace_bytes(const sp24_gemm_args *args);
+
+/* Y = s_x[m] * s_w[n] * sum_k x[m,k] * w[n,k] (scales only for E4M3), fp32
+ * accumulation in tensor memory, one persistent tcgen05 kernel launch.
+ * SPARSE (sparse operand = W, "Sparse tensor cores"): requires N % 128 == 0,
+ * K % 128 == 0; SP24_ERR_NOT_2_4 otherwise.  DENSE: requires K % 16 == 0
+ * (bf16) / K % 16 == 0 (e4m3); any M, N >= 1. */
+int sp24_gemm(const sp24_gemm_args *args, void *stream);
+
+/* ---------------------------------------------------------------------- */
+/* Online activation prune + compress fused ahead of the GEMM (kernel 4)   */
+/* ---------------------------------------------------------------------- */
+
+/* Bytes of workspace sp24_prune_compress_activations_fused needs when the
+ * caller does not keep the compressed activations (values + image). */
+size_t sp24_activations_workspace_bytes(int64_t M, int64_t K);
+
+/* Every call: prune + compress X (bf16 [M x K], pitch ldx) along K, then
+ * Y [M x N] = X_pruned * W^T with W dense bf16 [N x K] (pitch ldw), X as the
+ * sparse operand ("Measuring speed": a dynamic operand pays for its own
+ * prune and compress; section 4.2: a fused kernel reads the operand once and
+ * writes the kept values and indices once).  The GEMM launch is chained to
+ * the prune launch by programmatic dependent launch on `stream`.
+ *   x_values_dev / x_meta_dev: where the compressed X goes ([M x K/2] bf16
+ *   and the image of M rows); both NULL -> placed in workspace_dev, which must
+ *   then hold sp24_activations_workspace_bytes(M, K) bytes.
+ * Requirements: K % 128 == 0, ldx % 8 == 0, ldw % 8 == 0, N >= 1. */
+int sp24_prune_compress_activations_fused(const void *X_dev, int64_t M, int64_t K, int64_t ldx,
+                                          const void *W_dev, int64_t N, int64_t ldw,
+                                          void *Y_dev, int64_t ldy, sp24_dtype out_dtype,
+                                          void *x_values_dev, void *x_meta_dev,
+                                          void *workspace_dev, size_t workspace_bytes,
+                                          void *stream);
+
+/* ---------------------------------------------------------------------- */
+/* Tactic selection (kernel 5)                                             */
+/* ---------------------------------------------------------------------- */
+
+typedef struct sp24_tactic_record {
+    double t_sparse_us;       /* median over iters (device time, CUDA events)   */
+    double t_dense_us;
+    double t_sparse_min_us;
+    double t_dense_min_us;
+    int32_t iters;
+    int32_t eligible;         /* 1 if the sparse call passed eligibility         */
+    int32_t selected;         /* sp24_tactic that the rule picked                */
+    int32_t reserved;
+    char reason[64];          /* why dense was chosen, "" if sparse was          */
+} sp24_tactic_record;
+
+/* Times the sparse call and the dense call of the same product on `stream`
+ * with CUDA events (warmup untimed runs each, then iters timed runs each,
+ * alternating), and selects SPARSE iff the sparse median is strictly below
+ * the dense median; a tie or an ineligible sparse call selects DENSE
+ * ("Sparse Tactic Audit": latency is the sole criterion; every fallback is
+ * logged with its reason).  Synchronizes `stream`.  Both argument sets must
+ * describe the same M, N, K and output buffer semantics. */
+int sp24_select_tactic(const sp24_gemm_args *sparse_args, const sp24_gemm_args *dense_args,
+                       int warmup, int iters, sp24_tactic_record *out, void *stream);
+
+/* ---------------------------------------------------------------------- */
+/* Status                                                                  */
+/* ---------------------------------------------------------------------- */
+
+const char *sp24_status_string(int status);
+
+/* Reads (synchronously, on the current device) the device error word that a
+ * bounded wait writes when it expires; SP24_OK if none.  Clears nothing. */
+int sp24_last_device_error(void);
+
+/* Clears the device error word of the current device (synchronous). */
+int sp24_clear_device_error(void);
+
+/* Upper bound, in nanoseconds of %globaltimer, of every device-side wait
+ * (mbarrier waits in the GEMM).  Default 2 s.  Takes effect for launches
+ * issued after the call. */
+void sp24_set_wait_timeout_ns(uint64_t ns);
+
+/* Launches a one-block kernel that waits (bounded by timeout_ns) on a
+ * barrier that nothing completes, so that the bounded-wait path can be tested
+ * without a fault.  Returns SP24_ERR_DEVICE_TIMEOUT when the wait expired as
+ * designed (synchronizes the stream). */
+int sp24_selftest_bounded_wait(uint64_t timeout_ns, void *stream);
+
+/* Number of kernels this library has launched in this process. */
+uint64_t sp24_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SP24_H */

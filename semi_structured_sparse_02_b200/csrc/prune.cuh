@@ -1,0 +1,310 @@
+// prune.cuh -- kernel 1 (magnitude 2:4 prune + compress, emitting values and
+// the metadata image the sparse MMA reads), the per-row E4M3 quantizer and
+// the decompress (scatter) kernel.  All are HBM-bound: 128-bit loads, each
+// input byte read once per pass, outputs written with coalesced stores.
+//
+// Method: "2:4 Structured Sparsity Explained" (tensorcore.si), sections
+// "How 2:4 sparsity works" and "How to make a model 2:4 sparse"; E4M3 with one
+// scale per row: the 2:4-versus-quantization paper, section 2 "Quantization".
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+
+#include "sp24_device.cuh"
+
+namespace sp24 {
+
+constexpr int kChunkRows = 128;   // rows per metadata chunk (MMA M)
+constexpr int kChunkK = 128;      // K positions per metadata chunk (32 groups)
+constexpr int kChunkBytes = 2048; // 128 image rows x 16 bytes
+constexpr int kPruneThreads = 256;
+
+// ---------------------------------------------------------------------------
+// One group of four: keep the two largest |v| (bf16 magnitude bits compared as
+// integers), ties to the lower index.  Position i loses to j < i when
+// |v_j| >= |v_i| and to j > i when |v_j| > |v_i|; it survives if it loses to
+// fewer than two positions.  Returns the nibble i0 | i1 << 2.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t prune_group4(uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                                 int& i0, int& i1) {
+  // a* are magnitude keys (bits & 0x7fff)
+  const int l0 = (a1 > a0) + (a2 > a0) + (a3 > a0);
+  const int l1 = (a0 >= a1) + (a2 > a1) + (a3 > a1);
+  const int l2 = (a0 >= a2) + (a1 >= a2) + (a3 > a2);
+  const int l3 = (a0 >= a3) + (a1 >= a3) + (a2 >= a3);
+  const bool k0 = l0 < 2, k1 = l1 < 2, k2 = l2 < 2, k3 = l3 < 2;
+  // exactly two of k0..k3 are set; pick them in ascending order
+  i0 = k0 ? 0 : (k1 ? 1 : 2);
+  i1 = k3 ? 3 : (k2 ? 2 : 1);
+  (void)k1;
+  return (uint32_t)i0 | ((uint32_t)i1 << 2);
+}
+
+__device__ __forceinline__ uint8_t e4m3_of(float v) {
+  return (uint8_t)__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3);
+}
+
+__device__ __forceinline__ float bf16_bits_to_float(uint32_t b) {
+  return __uint_as_float(b << 16);
+}
+
+// Inverse scale from the row amax: 448 / amax, correctly rounded; 0 for amax 0.
+__device__ __forceinline__ float e4m3_inv_scale(float amax) {
+  return amax == 0.0f ? 0.0f : __fdiv_rn(448.0f, amax);
+}
+
+// ---------------------------------------------------------------------------
+// Metadata image row from the canonical bytes of one chunk (see sp24.h).
+// canon: [128 rows][16 bytes], byte b of a row = groups 2b (low) and 2b+1.
+// ---------------------------------------------------------------------------
+template <bool kIs8Bit>
+__device__ __forceinline__ uint4 image_row(const uint8_t (*canon)[16], int L) {
+  uint32_t w[4];
+  if (kIs8Bit) {
+    const uint32_t* src = reinterpret_cast<const uint32_t*>(canon[L]);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) w[i] = src[i];
+  } else {
+    const int h = (L >> 3) & 1;
+    const int r = ((L >> 4) << 4) + (L & 7);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int b = 4 * i + 2 * h;
+      const uint32_t lo = (uint32_t)canon[r][b] | ((uint32_t)canon[r][b + 1] << 8);
+      const uint32_t hi = (uint32_t)canon[r + 8][b] | ((uint32_t)canon[r + 8][b + 1] << 8);
+      w[i] = lo | (hi << 16);
+    }
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// ---------------------------------------------------------------------------
+// Kernel 1: prune + compress.  Grid-stride over chunks (row block rb, K-chunk
+// kc) of 128 x 128.  A chunk is also one hybrid tile.
+// kOutE4M3: values are E4M3 codes quantized with inv = 448/amax, where the
+// row amax is read from amax_in (written by k_row_amax).
+// ---------------------------------------------------------------------------
+template <bool kOutE4M3>
+__global__ void __launch_bounds__(kPruneThreads)
+k_prune_compress(const uint16_t* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
+                 void* __restrict__ values, uint8_t* __restrict__ meta,
+                 const float* __restrict__ amax_in, const uint8_t* __restrict__ tile_mask,
+                 void* __restrict__ dense_out) {
+  __shared__ __align__(16) uint8_t canon[kChunkRows][16];
+  const int64_t KC = K / kChunkK;
+  const int64_t RB = (rows + kChunkRows - 1) / kChunkRows;
+  const int64_t n_chunks = RB * KC;
+  const int64_t half_k = K / 2;
+
+  for (int64_t c = blockIdx.x; c < n_chunks; c += gridDim.x) {
+    const int64_t rb = c / KC, kc = c % KC;
+    const bool dense_tile = tile_mask != nullptr && tile_mask[c] != 0;
+    for (int i = threadIdx.x; i < kChunkRows * 16; i += kPruneThreads) {
+      const int rl = i >> 4, seg = i & 15;
+      const int64_t row = rb * kChunkRows + rl;
+      const int64_t k0 = kc * kChunkK + seg * 8;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      const bool live = row < rows;
+      if (live) v = __ldg(reinterpret_cast<const uint4*>(src + row * ld + k0));
+      const uint32_t e[8] = {v.x & 0xFFFFu, v.x >> 16, v.y & 0xFFFFu, v.y >> 16,
+                             v.z & 0xFFFFu, v.z >> 16, v.w & 0xFFFFu, v.w >> 16};
+      float inv = 0.0f;
+      if (kOutE4M3 && live) inv = e4m3_inv_scale(amax_in[row]);
+      uint32_t nib[2];
+      uint32_t kept[4];
+      if (dense_tile) {
+        nib[0] = nib[1] = 0x4u;
+        kept[0] = kept[1] = kept[2] = kept[3] = 0u;
+        if (live) {
+          if (kOutE4M3) {
+            uint32_t q0 = 0, q1 = 0;
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              q0 |= (uint32_t)e4m3_of(__fmul_rn(bf16_bits_to_float(e[j]), inv)) << (8 * j);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              q1 |= (uint32_t)e4m3_of(__fmul_rn(bf16_bits_to_float(e[4 + j]), inv)) << (8 * j);
+            *reinterpret_cast<uint2*>(static_cast<uint8_t*>(dense_out) + row * K + k0) =
+                make_uint2(q0, q1);
+          } else {
+            *reinterpret_cast<uint4*>(static_cast<uint16_t*>(dense_out) + row * K + k0) = v;
+          }
+        }
+      } else {
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+          const uint32_t* x = e + 4 * g;
+          int i0, i1;
+          nib[g] = prune_group4(x[0] & 0x7FFFu, x[1] & 0x7FFFu, x[2] & 0x7FFFu, x[3] & 0x7FFFu,
+                                i0, i1);
+          kept[2 * g + 0] = x[i0];
+          kept[2 * g + 1] = x[i1];
+        }
+      }
+      if (live) {
+        if (kOutE4M3) {
+          uint32_t q = 0;
+          if (!dense_tile) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              q |= (uint32_t)e4m3_of(__fmul_rn(bf16_bits_to_float(kept[j]), inv)) << (8 * j);
+          }
+          *reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(values) + row * half_k + kc * 64 +
+                                       seg * 4) = q;
+        } else {
+          *reinterpret_cast<uint2*>(static_cast<uint16_t*>(values) + row * half_k + kc * 64 +
+                                    seg * 4) =
+              make_uint2(kept[0] | (kept[1] << 16), kept[2] | (kept[3] << 16));
+        }
+      }
+      canon[rl][seg] = (uint8_t)(nib[0] | (nib[1] << 4));
+    }
+    __syncthreads();
+    if (threadIdx.x < kChunkRows) {
+      const uint4 w = image_row<kOutE4M3>(canon, threadIdx.x);
+      *reinterpret_cast<uint4*>(meta + c * kChunkBytes + threadIdx.x * 16) = w;
+    }
+    __syncthreads();
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Row amax of a bf16 matrix: one warp per row, 16-byte loads.  The integer
+// max of the magnitude bits is the bf16 of the largest |v| (finite inputs).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+k_row_amax(const uint16_t* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
+           float* __restrict__ amax_out) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int64_t n_warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t row = warp; row < rows; row += n_warps) {
+    uint32_t m = 0;
+    const uint4* p = reinterpret_cast<const uint4*>(src + row * ld);
+    for (int64_t i = lane; i < K / 8; i += 32) {
+      const uint4 v = __ldg(p + i);
+      m = max(m, max(max(v.x & 0x7FFFu, v.x >> 16 & 0x7FFFu), max(v.y & 0x7FFFu, v.y >> 16 & 0x7FFFu)));
+      m = max(m, max(max(v.z & 0x7FFFu, v.z >> 16 & 0x7FFFu), max(v.w & 0x7FFFu, v.w >> 16 & 0x7FFFu)));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    if (lane == 0) amax_out[row] = bf16_bits_to_float(m);
+  }
+}
+
+// scale = amax / 448 (correctly rounded), 1 when amax == 0; in place.
+__global__ void k_finalize_scales(float* __restrict__ s, int64_t rows) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < rows) {
+    const float a = s[i];
+    s[i] = a == 0.0f ? 1.0f : __fdiv_rn(a, 448.0f);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Per-row (per-token) E4M3 quantization: one CTA per row.  Pass 1 reduces
+// the amax, pass 2 re-reads the row (L1/L2 resident) and writes codes.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+k_quantize_rows_e4m3(const uint16_t* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
+                     uint8_t* __restrict__ q, float* __restrict__ scales) {
+  __shared__ uint32_t red[8];
+  for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
+    const uint4* p = reinterpret_cast<const uint4*>(src + row * ld);
+    uint32_t m = 0;
+    for (int64_t i = threadIdx.x; i < K / 8; i += blockDim.x) {
+      const uint4 v = __ldg(p + i);
+      m = max(m, max(max(v.x & 0x7FFFu, v.x >> 16 & 0x7FFFu), max(v.y & 0x7FFFu, v.y >> 16 & 0x7FFFu)));
+      m = max(m, max(max(v.z & 0x7FFFu, v.z >> 16 & 0x7FFFu), max(v.w & 0x7FFFu, v.w >> 16 & 0x7FFFu)));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+      uint32_t t = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0u;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) t = max(t, __shfl_xor_sync(0xFFFFFFFFu, t, o));
+      if (threadIdx.x == 0) red[0] = t;
+    }
+    __syncthreads();
+    const float amax = bf16_bits_to_float(red[0]);
+    const float inv = e4m3_inv_scale(amax);
+    if (threadIdx.x == 0) scales[row] = amax == 0.0f ? 1.0f : __fdiv_rn(amax, 448.0f);
+    for (int64_t i = threadIdx.x; i < K / 8; i += blockDim.x) {
+      const uint4 v = __ldg(p + i);
+      const uint32_t e[8] = {v.x & 0xFFFFu, v.x >> 16, v.y & 0xFFFFu, v.y >> 16,
+                             v.z & 0xFFFFu, v.z >> 16, v.w & 0xFFFFu, v.w >> 16};
+      uint32_t lo = 0, hi = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) lo |= (uint32_t)e4m3_of(__fmul_rn(bf16_bits_to_float(e[j]), inv)) << (8 * j);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) hi |= (uint32_t)e4m3_of(__fmul_rn(bf16_bits_to_float(e[4 + j]), inv)) << (8 * j);
+      *reinterpret_cast<uint2*>(q + row * K + i * 8) = make_uint2(lo, hi);
+    }
+    __syncthreads();
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Decompress: scatter values back using the metadata image.
+// ---------------------------------------------------------------------------
+// Nibble of (row-in-block r, group g in chunk) inside one image chunk.
+template <bool kIs8Bit>
+__device__ __forceinline__ uint32_t image_nibble(const uint8_t* chunk, int r, int g) {
+  if (kIs8Bit) return (chunk[r * 16 + (g >> 1)] >> ((g & 1) * 4)) & 0xFu;
+  const int w = g >> 3, h = (g >> 2) & 1, j = g & 3;
+  const int L = ((r >> 4) << 4) + (h << 3) + (r & 7);
+  const int bit = ((r & 8) ? 16 : 0) + 4 * j;
+  const uint32_t word = *reinterpret_cast<const uint32_t*>(chunk + L * 16 + w * 4);
+  return (word >> bit) & 0xFu;
+}
+
+template <bool kIs8Bit>
+__global__ void __launch_bounds__(kPruneThreads)
+k_decompress(const void* __restrict__ values, const uint8_t* __restrict__ meta, int64_t rows,
+             int64_t K, void* __restrict__ dst) {
+  __shared__ __align__(16) uint8_t chunk[kChunkBytes];
+  const int64_t KC = K / kChunkK;
+  const int64_t RB = (rows + kChunkRows - 1) / kChunkRows;
+  const int64_t half_k = K / 2;
+  for (int64_t c = blockIdx.x; c < RB * KC; c += gridDim.x) {
+    const int64_t rb = c / KC, kc = c % KC;
+    for (int i = threadIdx.x; i < kChunkBytes / 16; i += kPruneThreads)
+      reinterpret_cast<uint4*>(chunk)[i] = reinterpret_cast<const uint4*>(meta + c * kChunkBytes)[i];
+    __syncthreads();
+    for (int i = threadIdx.x; i < kChunkRows * 16; i += kPruneThreads) {
+      const int rl = i >> 4, seg = i & 15;
+      const int64_t row = rb * kChunkRows + rl;
+      if (row >= rows) continue;
+      const int64_t k0 = kc * kChunkK + seg * 8;
+      const uint32_t n0 = image_nibble<kIs8Bit>(chunk, rl, 2 * seg);
+      const uint32_t n1 = image_nibble<kIs8Bit>(chunk, rl, 2 * seg + 1);
+      if (kIs8Bit) {
+        const uint32_t v = *reinterpret_cast<const uint32_t*>(
+            static_cast<const uint8_t*>(values) + row * half_k + kc * 64 + seg * 4);
+        uint8_t out[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        out[n0 & 3] = v & 0xFF;
+        out[(n0 >> 2) & 3] = (v >> 8) & 0xFF;
+        out[4 + (n1 & 3)] = (v >> 16) & 0xFF;
+        out[4 + ((n1 >> 2) & 3)] = (v >> 24) & 0xFF;
+        *reinterpret_cast<uint2*>(static_cast<uint8_t*>(dst) + row * K + k0) =
+            *reinterpret_cast<uint2*>(out);
+      } else {
+        const uint2 v = *reinterpret_cast<const uint2*>(
+            static_cast<const uint16_t*>(values) + row * half_k + kc * 64 + seg * 4);
+        uint16_t out[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        out[n0 & 3] = v.x & 0xFFFF;
+        out[(n0 >> 2) & 3] = v.x >> 16;
+        out[4 + (n1 & 3)] = v.y & 0xFFFF;
+        out[4 + ((n1 >> 2) & 3)] = v.y >> 16;
+        *reinterpret_cast<uint4*>(static_cast<uint16_t*>(dst) + row * K + k0) =
+            *reinterpret_cast<uint4*>(out);
+      }
+    }
+    __syncthreads();
+  }
+}
+
+}  // namespace sp24

@@ -1,0 +1,675 @@
+// sp24.cu -- the C ABI of libsp24.so (declared in include/sp24.h): argument
+// validation, TMA descriptor encoding, tile and split-K selection, kernel
+// launches and the timing-based tactic selector.  Single translation unit:
+// the kernels live in the headers included below.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "sp24.h"
+#include "sp24_device.cuh"
+#include "prune.cuh"
+#include "gemm.cuh"
+
+namespace sp24 {
+namespace {
+
+std::atomic<uint64_t> g_launches{0};
+std::atomic<uint64_t> g_timeout_ns{2000000000ull};
+
+constexpr int kMaxDevices = 64;
+
+// ---------------------------------------------------------------------------
+// device checks
+// ---------------------------------------------------------------------------
+struct DeviceInfo {
+  int checked = 0;
+  int ok = 0;
+  int sms = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+int current_device_info(DeviceInfo* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return SP24_ERR_UNSUPPORTED_DEVICE;
+  }
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.checked) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return SP24_ERR_UNSUPPORTED_DEVICE;
+    }
+    d.checked = 1;
+    d.ok = (major == 10 && minor == 0);
+    d.sms = sms;
+  }
+  if (!d.ok) return SP24_ERR_UNSUPPORTED_DEVICE;
+  *out = d;
+  return SP24_OK;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int dtype_bytes(int dt) { return dt == SP24_BF16 ? 2 : dt == SP24_E4M3 ? 1 : dt == SP24_F32 ? 4 : 0; }
+
+int launch_result(cudaError_t e) {
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return SP24_ERR_CUDA;
+  }
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return SP24_OK;
+}
+
+// ---------------------------------------------------------------------------
+// TMA descriptors (driver entry point fetched once through the runtime)
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+std::once_flag g_encode_once;
+
+EncodeTiledFn encode_fn() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    cudaGetLastError();
+  });
+  return g_encode;
+}
+
+// 2-D map over a row-major matrix [rows x inner] of 1- or 2-byte elements
+// with row pitch `pitch_bytes`; box = box_inner elements x box_rows rows.
+bool make_map(CUtensorMap* map, const void* base, int elem_bytes, uint64_t inner, uint64_t rows,
+              uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle sw) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {pitch_bytes};
+  const cuuint32_t box[2] = {box_inner, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapDataType dt =
+      elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  return enc(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------------------
+// GEMM planning
+// ---------------------------------------------------------------------------
+struct Plan {
+  int mode;        // kModeDense / kModeSparse / kModeHybrid
+  bool bf16;
+  bool a_is_w;
+  int bn;
+  int kt;          // logical K per stage
+  int stage_a_bytes;
+  int num_kt, tiles_a, tiles_b, splits, num_units;
+  size_t ws_bytes;
+};
+
+int pick_bn(int64_t rows_b) {
+  if (rows_b <= 16) return 16;
+  if (rows_b <= 32) return 32;
+  if (rows_b <= 64) return 64;
+  return 128;
+}
+
+int stage_k(int mode, bool bf16) {
+  if (mode == kModeHybrid) return 128;
+  if (mode == kModeSparse) return bf16 ? 128 : 256;
+  return bf16 ? 64 : 128;
+}
+
+size_t split_ws_bytes(const Plan& pl) {
+  if (pl.splits <= 1) return 0;
+  const size_t part = (size_t)pl.num_units * pl.bn * 128 * sizeof(float);
+  const size_t cnt = ((size_t)pl.tiles_a * pl.tiles_b * sizeof(unsigned int) + 255) & ~(size_t)255;
+  return part + cnt;
+}
+
+// Splits the K range of each output tile so that the persistent grid's
+// waves are balanced (decode shapes have fewer tiles than SMs).
+void choose_splits(Plan& pl, int sms, size_t ws_cap) {
+  const int64_t tiles = (int64_t)pl.tiles_a * pl.tiles_b;
+  pl.splits = 1;
+  if (tiles < 2 * sms) {
+    double best = 1e300;
+    const int max_s = std::min(pl.num_kt, 64);
+    for (int s = 1; s <= max_s; ++s) {
+      const int64_t units = tiles * s;
+      const int64_t waves = (units + sms - 1) / sms;
+      const int64_t kt_per = (pl.num_kt + s - 1) / s;
+      const double per_unit = (double)kt_per * pl.stage_a_bytes +
+                              (s > 1 ? 2.0 * pl.bn * 128 * 4 : 0.0);
+      const double cost = (double)waves * per_unit;
+      Plan t = pl;
+      t.splits = s;
+      t.num_units = (int)units;
+      if (split_ws_bytes(t) > ws_cap) break;
+      if (cost < best * 0.999) {
+        best = cost;
+        pl.splits = s;
+      }
+    }
+  }
+  pl.num_units = (int)(tiles * pl.splits);
+  pl.ws_bytes = split_ws_bytes(pl);
+}
+
+// ---------------------------------------------------------------------------
+// kernel launch for one instantiation
+// ---------------------------------------------------------------------------
+template <int kMode, bool kBf16, int kBN, bool kAIsW>
+int launch_gemm_inst(const CUtensorMap& ta, const CUtensorMap& ta2, const CUtensorMap& tb,
+                     const GemmParams& p, int grid, cudaStream_t stream) {
+  using C = GemmCfg<kMode, kBf16, kBN>;
+  static std::atomic<uint64_t> attr_set{0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const uint64_t bit = 1ull << (dev & 63);
+  if (!(attr_set.load() & bit)) {
+    if (cudaFuncSetAttribute(k_gemm<kMode, kBf16, kBN, kAIsW>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess) {
+      cudaGetLastError();
+      return SP24_ERR_CUDA;
+    }
+    attr_set.fetch_or(bit);
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = p.use_pdl ? 1 : 0;
+  return launch_result(cudaLaunchKernelEx(&cfg, k_gemm<kMode, kBf16, kBN, kAIsW>, ta, ta2, tb, p));
+}
+
+template <int kMode, bool kBf16, bool kAIsW>
+int launch_gemm_bn(int bn, const CUtensorMap& ta, const CUtensorMap& ta2, const CUtensorMap& tb,
+                   const GemmParams& p, int grid, cudaStream_t s) {
+  switch (bn) {
+    case 16: return launch_gemm_inst<kMode, kBf16, 16, kAIsW>(ta, ta2, tb, p, grid, s);
+    case 32: return launch_gemm_inst<kMode, kBf16, 32, kAIsW>(ta, ta2, tb, p, grid, s);
+    case 64: return launch_gemm_inst<kMode, kBf16, 64, kAIsW>(ta, ta2, tb, p, grid, s);
+    case 128: return launch_gemm_inst<kMode, kBf16, 128, kAIsW>(ta, ta2, tb, p, grid, s);
+    default: return SP24_ERR_INVALID_ARG;
+  }
+}
+
+int dispatch_gemm(const Plan& pl, const CUtensorMap& ta, const CUtensorMap& ta2, const CUtensorMap& tb,
+                  const GemmParams& p, int grid, cudaStream_t s) {
+  if (!pl.a_is_w) {
+    if (pl.mode == kModeSparse && pl.bf16 && pl.bn == 128)
+      return launch_gemm_inst<kModeSparse, true, 128, false>(ta, ta2, tb, p, grid, s);
+    return SP24_ERR_DTYPE;
+  }
+  if (pl.mode == kModeSparse)
+    return pl.bf16 ? launch_gemm_bn<kModeSparse, true, true>(pl.bn, ta, ta2, tb, p, grid, s)
+                   : launch_gemm_bn<kModeSparse, false, true>(pl.bn, ta, ta2, tb, p, grid, s);
+  if (pl.mode == kModeDense)
+    return pl.bf16 ? launch_gemm_bn<kModeDense, true, true>(pl.bn, ta, ta2, tb, p, grid, s)
+                   : launch_gemm_bn<kModeDense, false, true>(pl.bn, ta, ta2, tb, p, grid, s);
+  if (pl.mode == kModeHybrid && !pl.bf16)
+    return launch_gemm_bn<kModeHybrid, false, true>(pl.bn, ta, ta2, tb, p, grid, s);
+  return SP24_ERR_DTYPE;
+}
+
+// Validation of a GEMM argument set; no CUDA call.
+int validate_gemm(const sp24_gemm_args* a) {
+  if (a == nullptr) return SP24_ERR_NULL;
+  if (a->M < 1 || a->N < 1 || a->K < 1) return SP24_ERR_INVALID_ARG;
+  if (a->M > INT32_MAX / 2 || a->N > INT32_MAX / 2 || a->K > INT32_MAX / 2) return SP24_ERR_INVALID_ARG;
+  if (a->in_dtype != SP24_BF16 && a->in_dtype != SP24_E4M3) return SP24_ERR_DTYPE;
+  if (a->out_dtype != SP24_BF16 && a->out_dtype != SP24_F32) return SP24_ERR_DTYPE;
+  if (a->tactic != SP24_TACTIC_SPARSE && a->tactic != SP24_TACTIC_DENSE) return SP24_ERR_INVALID_ARG;
+  if (a->X == nullptr || a->W == nullptr || a->Y == nullptr) return SP24_ERR_NULL;
+  const bool e4 = a->in_dtype == SP24_E4M3;
+  if (e4 && (a->x_scales == nullptr || a->w_scales == nullptr)) return SP24_ERR_NULL;
+  const int eb = dtype_bytes(a->in_dtype);
+  const int ob = dtype_bytes(a->out_dtype);
+  const bool sparse = a->tactic == SP24_TACTIC_SPARSE;
+  if (sparse) {
+    if (a->W_meta == nullptr) return SP24_ERR_NULL;
+    if (a->N % 128 != 0 || a->K % 128 != 0) return SP24_ERR_NOT_2_4;
+    if (a->tile_dense_mask != nullptr) {
+      if (!e4) return SP24_ERR_DTYPE;
+      if (a->W_dense_tiles == nullptr) return SP24_ERR_NULL;
+      if (!aligned16(a->W_dense_tiles)) return SP24_ERR_ALIGNMENT;
+    }
+    if (a->ldw < a->K / 2) return SP24_ERR_INVALID_ARG;
+    if (!aligned16(a->W_meta)) return SP24_ERR_ALIGNMENT;
+  } else {
+    if (a->tile_dense_mask != nullptr) return SP24_ERR_INVALID_ARG;
+    if (a->ldw < a->K) return SP24_ERR_INVALID_ARG;
+    if (a->K % 16 != 0) return SP24_ERR_ALIGNMENT;
+  }
+  if (a->ldx < a->K || a->ldy < a->N) return SP24_ERR_INVALID_ARG;
+  if (!aligned16(a->X) || !aligned16(a->W)) return SP24_ERR_ALIGNMENT;
+  if ((a->ldx * eb) % 16 != 0 || (a->ldw * eb) % 16 != 0) return SP24_ERR_ALIGNMENT;
+  if ((reinterpret_cast<uintptr_t>(a->Y) % ob) != 0) return SP24_ERR_ALIGNMENT;
+  return SP24_OK;
+}
+
+Plan plan_gemm(const sp24_gemm_args* a, int sms, size_t ws_cap) {
+  Plan pl;
+  pl.bf16 = a->in_dtype == SP24_BF16;
+  pl.a_is_w = true;
+  pl.mode = a->tactic == SP24_TACTIC_DENSE ? kModeDense
+                                           : (a->tile_dense_mask ? kModeHybrid : kModeSparse);
+  pl.bn = pick_bn(a->M);
+  pl.kt = stage_k(pl.mode, pl.bf16);
+  pl.num_kt = (int)((a->K + pl.kt - 1) / pl.kt);
+  pl.tiles_a = (int)((a->N + kBlockA - 1) / kBlockA);
+  pl.tiles_b = (int)((a->M + pl.bn - 1) / pl.bn);
+  // bytes of the streamed operand per stage (A tile + metadata)
+  pl.stage_a_bytes = kBlockA * 128 + (pl.mode == kModeDense ? 0 : 2048 * (pl.bf16 ? 1 : 2));
+  choose_splits(pl, sms, ws_cap);
+  return pl;
+}
+
+int run_gemm(const sp24_gemm_args* a, cudaStream_t stream) {
+  DeviceInfo di;
+  int st = current_device_info(&di);
+  if (st != SP24_OK) return st;
+  size_t ws_cap = a->workspace != nullptr ? a->workspace_bytes : 0;
+  if (a->workspace != nullptr && !aligned16(a->workspace)) return SP24_ERR_ALIGNMENT;
+  Plan pl = plan_gemm(a, di.sms, ws_cap);
+  const int eb = dtype_bytes(a->in_dtype);
+  const int box_elems = 128 / eb;  // 128 bytes
+  CUtensorMap ta, ta2, tb;
+  bool ok = true;
+  if (pl.mode == kModeDense) {
+    ok &= make_map(&ta, a->W, eb, a->K, a->N, a->ldw * eb, box_elems, kBlockA,
+                   CU_TENSOR_MAP_SWIZZLE_128B);
+    ta2 = ta;
+  } else if (pl.mode == kModeSparse) {
+    ok &= make_map(&ta, a->W, eb, a->K / 2, a->N, a->ldw * eb, box_elems, kBlockA,
+                   CU_TENSOR_MAP_SWIZZLE_128B);
+    ta2 = ta;
+  } else {
+    ok &= make_map(&ta, a->W_dense_tiles, 1, a->K, a->N, a->K, 128, kBlockA, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok &= make_map(&ta2, a->W, 1, a->K / 2, a->N, a->ldw, 64, kBlockA, CU_TENSOR_MAP_SWIZZLE_64B);
+  }
+  ok &= make_map(&tb, a->X, eb, a->K, a->M, a->ldx * eb, box_elems, pl.bn, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!ok) return SP24_ERR_CUDA;
+
+  GemmParams p;
+  memset(&p, 0, sizeof p);
+  p.rows_a = (int32_t)a->N;
+  p.rows_b = (int32_t)a->M;
+  p.K = (int32_t)a->K;
+  p.num_kt = pl.num_kt;
+  p.tiles_a = pl.tiles_a;
+  p.tiles_b = pl.tiles_b;
+  p.splits = pl.splits;
+  p.num_units = pl.num_units;
+  p.out_f32 = a->out_dtype == SP24_F32;
+  p.use_pdl = 1;
+  p.meta = static_cast<const uint8_t*>(a->W_meta);
+  p.tile_mask = a->tile_dense_mask;
+  p.scale_a = a->in_dtype == SP24_E4M3 ? a->w_scales : nullptr;
+  p.scale_b = a->in_dtype == SP24_E4M3 ? a->x_scales : nullptr;
+  p.Y = a->Y;
+  p.ldy = a->ldy;
+  if (pl.splits > 1) {
+    p.ws_partials = static_cast<float*>(a->workspace);
+    p.ws_counters = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(a->workspace) +
+                                                    (size_t)pl.num_units * pl.bn * 128 * sizeof(float));
+  }
+  p.timeout_ns = g_timeout_ns.load();
+  const int grid = std::min(pl.num_units, di.sms);
+  return dispatch_gemm(pl, ta, ta2, tb, p, grid, stream);
+}
+
+}  // namespace
+}  // namespace sp24
+
+using namespace sp24;
+
+// ===========================================================================
+// C ABI
+// ===========================================================================
+extern "C" {
+
+size_t sp24_values_bytes(int64_t rows, int64_t K, sp24_dtype dtype) {
+  if (rows < 0 || K < 0) return 0;
+  const int eb = dtype_bytes(dtype);
+  return (size_t)rows * (size_t)(K / 2) * (size_t)eb;
+}
+
+size_t sp24_meta_bytes(int64_t rows, int64_t K) {
+  if (rows < 0 || K < 0) return 0;
+  return (size_t)((rows + 127) / 128) * (size_t)(K / 128) * 2048;
+}
+
+int sp24_prune_compress(const void* src, int64_t rows, int64_t K, int64_t ld, sp24_dtype out_dtype,
+                        void* values, void* meta, float* row_scales, const uint8_t* tile_mask,
+                        void* dense_tiles, void* stream) {
+  if (src == nullptr || values == nullptr || meta == nullptr) return SP24_ERR_NULL;
+  if (out_dtype != SP24_BF16 && out_dtype != SP24_E4M3) return SP24_ERR_DTYPE;
+  if (out_dtype == SP24_E4M3 && row_scales == nullptr) return SP24_ERR_NULL;
+  if (tile_mask != nullptr && dense_tiles == nullptr) return SP24_ERR_NULL;
+  if (rows < 1 || K < 128 || ld < K) return SP24_ERR_INVALID_ARG;
+  if (K % 128 != 0) return SP24_ERR_NOT_2_4;
+  if (ld % 8 != 0 || !aligned16(src) || !aligned16(values) || !aligned16(meta)) return SP24_ERR_ALIGNMENT;
+  if (dense_tiles != nullptr && !aligned16(dense_tiles)) return SP24_ERR_ALIGNMENT;
+  DeviceInfo di;
+  int st = current_device_info(&di);
+  if (st != SP24_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const uint16_t* src16 = static_cast<const uint16_t*>(src);
+  const int64_t chunks = ((rows + 127) / 128) * (K / 128);
+  const int grid = (int)std::min<int64_t>(chunks, (int64_t)di.sms * 4);
+  uint8_t* meta8 = static_cast<uint8_t*>(meta);
+  if (out_dtype == SP24_BF16) {
+    k_prune_compress<false><<<grid, kPruneThreads, 0, s>>>(src16, rows, K, ld, values, meta8, nullptr,
+                                                           tile_mask, dense_tiles);
+    return launch_result(cudaGetLastError());
+  }
+  const int agrid = (int)std::min<int64_t>((rows + 7) / 8, (int64_t)di.sms * 8);
+  k_row_amax<<<agrid, 256, 0, s>>>(src16, rows, K, ld, row_scales);
+  if ((st = launch_result(cudaGetLastError())) != SP24_OK) return st;
+  k_prune_compress<true><<<grid, kPruneThreads, 0, s>>>(src16, rows, K, ld, values, meta8, row_scales,
+                                                        tile_mask, dense_tiles);
+  if ((st = launch_result(cudaGetLastError())) != SP24_OK) return st;
+  k_finalize_scales<<<(int)((rows + 255) / 256), 256, 0, s>>>(row_scales, rows);
+  return launch_result(cudaGetLastError());
+}
+
+int sp24_decompress(const void* values, const void* meta, int64_t rows, int64_t K, sp24_dtype dtype,
+                    void* dst, void* stream) {
+  if (values == nullptr || meta == nullptr || dst == nullptr) return SP24_ERR_NULL;
+  if (dtype != SP24_BF16 && dtype != SP24_E4M3) return SP24_ERR_DTYPE;
+  if (rows < 1 || K < 128) return SP24_ERR_INVALID_ARG;
+  if (K % 128 != 0) return SP24_ERR_NOT_2_4;
+  if (!aligned16(values) || !aligned16(meta) || !aligned16(dst)) return SP24_ERR_ALIGNMENT;
+  DeviceInfo di;
+  int st = current_device_info(&di);
+  if (st != SP24_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t chunks = ((rows + 127) / 128) * (K / 128);
+  const int grid = (int)std::min<int64_t>(chunks, (int64_t)di.sms * 4);
+  const uint8_t* m8 = static_cast<const uint8_t*>(meta);
+  if (dtype == SP24_BF16) k_decompress<false><<<grid, kPruneThreads, 0, s>>>(values, m8, rows, K, dst);
+  else k_decompress<true><<<grid, kPruneThreads, 0, s>>>(values, m8, rows, K, dst);
+  return launch_result(cudaGetLastError());
+}
+
+int sp24_quantize_e4m3_rows(const void* src, int64_t rows, int64_t K, int64_t ld, void* q,
+                            float* scales, void* stream) {
+  if (src == nullptr || q == nullptr || scales == nullptr) return SP24_ERR_NULL;
+  if (rows < 1 || K < 1 || ld < K) return SP24_ERR_INVALID_ARG;
+  if (K % 16 != 0 || ld % 8 != 0 || !aligned16(src) || !aligned16(q)) return SP24_ERR_ALIGNMENT;
+  DeviceInfo di;
+  int st = current_device_info(&di);
+  if (st != SP24_OK) return st;
+  const int grid = (int)std::min<int64_t>(rows, (int64_t)di.sms * 8);
+  k_quantize_rows_e4m3<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint16_t*>(src), rows, K, ld, static_cast<uint8_t*>(q), scales);
+  return launch_result(cudaGetLastError());
+}
+
+size_t sp24_gemm_workspace_bytes(const sp24_gemm_args* a) {
+  if (validate_gemm(a) != SP24_OK) return 0;
+  DeviceInfo di;
+  if (current_device_info(&di) != SP24_OK) return 0;
+  Plan pl = plan_gemm(a, di.sms, (size_t)-1);
+  return pl.ws_bytes;
+}
+
+int sp24_gemm(const sp24_gemm_args* a, void* stream) {
+  int st = validate_gemm(a);
+  if (st != SP24_OK) return st;
+  return run_gemm(a, static_cast<cudaStream_t>(stream));
+}
+
+size_t sp24_activations_workspace_bytes(int64_t M, int64_t K) {
+  if (M < 1 || K < 128) return 0;
+  const size_t vals = ((size_t)M * (size_t)(K / 2) * 2 + 255) & ~(size_t)255;
+  return vals + sp24_meta_bytes(M, K);
+}
+
+int sp24_prune_compress_activations_fused(const void* X, int64_t M, int64_t K, int64_t ldx,
+                                          const void* W, int64_t N, int64_t ldw, void* Y, int64_t ldy,
+                                          sp24_dtype out_dtype, void* x_values, void* x_meta,
+                                          void* workspace, size_t workspace_bytes, void* stream) {
+  if (X == nullptr || W == nullptr || Y == nullptr) return SP24_ERR_NULL;
+  if (out_dtype != SP24_BF16 && out_dtype != SP24_F32) return SP24_ERR_DTYPE;
+  if (M < 1 || N < 1 || K < 128 || ldx < K || ldw < K || ldy < N) return SP24_ERR_INVALID_ARG;
+  if (K % 128 != 0) return SP24_ERR_NOT_2_4;
+  if ((x_values == nullptr) != (x_meta == nullptr)) return SP24_ERR_NULL;
+  if (ldx % 8 != 0 || ldw % 8 != 0 || !aligned16(X) || !aligned16(W)) return SP24_ERR_ALIGNMENT;
+  if (x_values == nullptr) {
+    if (workspace == nullptr) return SP24_ERR_WORKSPACE;
+    if (workspace_bytes < sp24_activations_workspace_bytes(M, K)) return SP24_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return SP24_ERR_ALIGNMENT;
+    x_values = workspace;
+    x_meta = static_cast<uint8_t*>(workspace) + (((size_t)M * (size_t)(K / 2) * 2 + 255) & ~(size_t)255);
+  }
+  if (!aligned16(x_values) || !aligned16(x_meta)) return SP24_ERR_ALIGNMENT;
+  DeviceInfo di;
+  int st = current_device_info(&di);
+  if (st != SP24_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t chunks = ((M + 127) / 128) * (K / 128);
+  const int grid = (int)std::min<int64_t>(chunks, (int64_t)di.sms * 4);
+  k_prune_compress<false><<<grid, kPruneThreads, 0, s>>>(static_cast<const uint16_t*>(X), M, K, ldx,
+                                                         x_values, static_cast<uint8_t*>(x_meta), nullptr,
+                                                         nullptr, nullptr);
+  if ((st = launch_result(cudaGetLastError())) != SP24_OK) return st;
+
+  // GEMM with X (compressed) as the sparse operand A and W dense as B.
+  Plan pl;
+  pl.mode = kModeSparse;
+  pl.bf16 = true;
+  pl.a_is_w = false;
+  pl.bn = 128;
+  pl.kt = 128;
+  pl.num_kt = (int)(K / 128);
+  pl.tiles_a = (int)((M + 127) / 128);
+  pl.tiles_b = (int)((N + 127) / 128);
+  pl.splits = 1;
+  pl.num_units = pl.tiles_a * pl.tiles_b;
+  CUtensorMap ta, tb;
+  bool ok = make_map(&ta, x_values, 2, K / 2, M, (K / 2) * 2, 64, kBlockA, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= make_map(&tb, W, 2, K, N, ldw * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!ok) return SP24_ERR_CUDA;
+  GemmParams p;
+  memset(&p, 0, sizeof p);
+  p.rows_a = (int32_t)M;
+  p.rows_b = (int32_t)N;
+  p.K = (int32_t)K;
+  p.num_kt = pl.num_kt;
+  p.tiles_a = pl.tiles_a;
+  p.tiles_b = pl.tiles_b;
+  p.splits = 1;
+  p.num_units = pl.num_units;
+  p.out_f32 = out_dtype == SP24_F32;
+  p.use_pdl = 1;
+  p.meta = static_cast<const uint8_t*>(x_meta);
+  p.Y = Y;
+  p.ldy = ldy;
+  p.timeout_ns = g_timeout_ns.load();
+  const int ggrid = std::min(pl.num_units, di.sms);
+  return dispatch_gemm(pl, ta, ta, tb, p, ggrid, s);
+}
+
+int sp24_select_tactic(const sp24_gemm_args* sparse_args, const sp24_gemm_args* dense_args, int warmup,
+                       int iters, sp24_tactic_record* out, void* stream) {
+  if (out == nullptr || dense_args == nullptr) return SP24_ERR_NULL;
+  if (warmup < 0 || iters < 1) return SP24_ERR_INVALID_ARG;
+  memset(out, 0, sizeof *out);
+  int st = validate_gemm(dense_args);
+  if (st != SP24_OK) return st;
+  if (dense_args->tactic != SP24_TACTIC_DENSE) return SP24_ERR_INVALID_ARG;
+  const int sp_st = validate_gemm(sparse_args);
+  const bool eligible = sp_st == SP24_OK && sparse_args->tactic == SP24_TACTIC_SPARSE &&
+                        sparse_args->M == dense_args->M && sparse_args->N == dense_args->N &&
+                        sparse_args->K == dense_args->K;
+  out->eligible = eligible ? 1 : 0;
+  out->iters = iters;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  std::vector<cudaEvent_t> ev;
+  const int n_ev = 2 * iters * (eligible ? 2 : 1);
+  ev.resize(n_ev);
+  for (int i = 0; i < n_ev; ++i) {
+    if (cudaEventCreate(&ev[i]) != cudaSuccess) {
+      for (int j = 0; j < i; ++j) cudaEventDestroy(ev[j]);
+      cudaGetLastError();
+      return SP24_ERR_CUDA;
+    }
+  }
+  auto cleanup = [&] {
+    for (auto e : ev) cudaEventDestroy(e);
+  };
+  for (int i = 0; i < warmup; ++i) {
+    if (eligible && (st = run_gemm(sparse_args, s)) != SP24_OK) { cleanup(); return st; }
+    if ((st = run_gemm(dense_args, s)) != SP24_OK) { cleanup(); return st; }
+  }
+  int e = 0;
+  for (int i = 0; i < iters; ++i) {
+    if (eligible) {
+      cudaEventRecord(ev[e++], s);
+      if ((st = run_gemm(sparse_args, s)) != SP24_OK) { cleanup(); return st; }
+      cudaEventRecord(ev[e++], s);
+    }
+    cudaEventRecord(ev[e++], s);
+    if ((st = run_gemm(dense_args, s)) != SP24_OK) { cleanup(); return st; }
+    cudaEventRecord(ev[e++], s);
+  }
+  if (cudaStreamSynchronize(s) != cudaSuccess) {
+    cleanup();
+    cudaGetLastError();
+    return SP24_ERR_CUDA;
+  }
+  std::vector<double> ts, td;
+  e = 0;
+  for (int i = 0; i < iters; ++i) {
+    float ms = 0.f;
+    if (eligible) {
+      cudaEventElapsedTime(&ms, ev[e], ev[e + 1]);
+      ts.push_back(ms * 1000.0);
+      e += 2;
+    }
+    cudaEventElapsedTime(&ms, ev[e], ev[e + 1]);
+    td.push_back(ms * 1000.0);
+    e += 2;
+  }
+  cleanup();
+  auto median = [](std::vector<double> v) {
+    std::sort(v.begin(), v.end());
+    const size_t n = v.size();
+    return n % 2 ? v[n / 2] : 0.5 * (v[n / 2 - 1] + v[n / 2]);
+  };
+  out->t_dense_us = median(td);
+  out->t_dense_min_us = *std::min_element(td.begin(), td.end());
+  if (eligible) {
+    out->t_sparse_us = median(ts);
+    out->t_sparse_min_us = *std::min_element(ts.begin(), ts.end());
+    if (out->t_sparse_us < out->t_dense_us) {
+      out->selected = SP24_TACTIC_SPARSE;
+      out->reason[0] = 0;
+    } else {
+      out->selected = SP24_TACTIC_DENSE;
+      snprintf(out->reason, sizeof out->reason, "Dense kernel %.2fx faster",
+               out->t_sparse_us / out->t_dense_us);
+    }
+  } else {
+    out->selected = SP24_TACTIC_DENSE;
+    snprintf(out->reason, sizeof out->reason, "%s",
+             (sp_st == SP24_ERR_ALIGNMENT || sp_st == SP24_ERR_NOT_2_4) ? "Alignment failure"
+                                                                          : "Not eligible");
+  }
+  return SP24_OK;
+}
+
+const char* sp24_status_string(int s) {
+  switch (s) {
+    case SP24_OK: return "ok";
+    case SP24_ERR_INVALID_ARG: return "invalid argument";
+    case SP24_ERR_NULL: return "required pointer is null";
+    case SP24_ERR_DTYPE: return "unsupported dtype combination";
+    case SP24_ERR_ALIGNMENT: return "pointer, pitch or shape misaligned";
+    case SP24_ERR_NOT_2_4: return "operand not eligible for the 2:4 sparse path";
+    case SP24_ERR_UNSUPPORTED_DEVICE: return "current device is not sm_100";
+    case SP24_ERR_CUDA: return "CUDA runtime call failed";
+    case SP24_ERR_DEVICE_TIMEOUT: return "device-side bounded wait expired";
+    case SP24_ERR_WORKSPACE: return "workspace missing or too small";
+    default: return "unknown status";
+  }
+}
+
+int sp24_last_device_error(void) {
+  DeviceInfo di;
+  int st = current_device_info(&di);
+  if (st != SP24_OK) return st;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_dev_error, sizeof v) != cudaSuccess) {
+    cudaGetLastError();
+    return SP24_ERR_CUDA;
+  }
+  return v == 0 ? SP24_OK : SP24_ERR_DEVICE_TIMEOUT;
+}
+
+int sp24_clear_device_error(void) {
+  DeviceInfo di;
+  int st = current_device_info(&di);
+  if (st != SP24_OK) return st;
+  const unsigned int z = 0;
+  if (cudaMemcpyToSymbol(g_dev_error, &z, sizeof z) != cudaSuccess) {
+    cudaGetLastError();
+    return SP24_ERR_CUDA;
+  }
+  return SP24_OK;
+}
+
+void sp24_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns.store(ns == 0 ? 1 : ns); }
+
+int sp24_selftest_bounded_wait(uint64_t timeout_ns, void* stream) {
+  DeviceInfo di;
+  int st = current_device_info(&di);
+  if (st != SP24_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  k_selftest_bounded_wait<<<1, 32, 0, s>>>(timeout_ns);
+  st = launch_result(cudaGetLastError());
+  if (st == SP24_OK && cudaStreamSynchronize(s) != cudaSuccess) {
+    cudaGetLastError();
+    st = SP24_ERR_CUDA;
+  }
+  if (st != SP24_OK) return st;
+  int v = -1;
+  if (cudaMemcpyFromSymbol(&v, g_selftest_result, sizeof v) != cudaSuccess) {
+    cudaGetLastError();
+    return SP24_ERR_CUDA;
+  }
+  return v == 0 ? SP24_ERR_DEVICE_TIMEOUT : SP24_OK;
+}
+
+uint64_t sp24_launch_count(void) { return g_launches.load(); }
+
+}  // extern "C"

@@ -1,0 +1,120 @@
+"""The C ABI on a machine without a GPU: the library loads, exports every
+function include/sp24.h declares, computes sizes, and rejects bad arguments
+with the documented status codes before any CUDA launch."""
+import ctypes
+
+import pytest
+import torch
+
+from semi_structured_sparse_02_b200 import build as sp24_build
+from semi_structured_sparse_02_b200 import sp24
+
+sp24_build.build()
+L = sp24.lib()
+
+FAKE = 0x7F0000000000  # 16-byte aligned, never dereferenced: validation fails first
+NO_GPU = not torch.cuda.is_available()
+
+
+def test_exports_every_declared_function():
+    names = sp24.header_functions()
+    assert len(names) >= 16
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_sizes():
+    assert sp24.values_bytes(256, 256, sp24.BF16) == 65536
+    assert sp24.values_bytes(256, 256, sp24.E4M3) == 32768
+    assert sp24.meta_bytes(256, 256) == 8192          # 256*256/8: one bit per element
+    assert sp24.meta_bytes(40, 256) == 4096           # rows padded to a 128-row block
+    assert sp24.values_bytes(256, 256, sp24.BF16) + sp24.meta_bytes(256, 256) == 73728
+
+
+def test_status_strings():
+    for s in range(10):
+        assert isinstance(sp24.status_string(s), str) and sp24.status_string(s)
+    assert sp24.status_string(sp24.SP24_ERR_NOT_2_4).startswith("operand not eligible")
+
+
+def prune(src=FAKE, rows=256, K=256, ld=256, dt=sp24.BF16, vals=FAKE, meta=FAKE, sc=None, mask=None,
+          dense=None):
+    return L.sp24_prune_compress(src, rows, K, ld, dt, vals, meta, sc, mask, dense, None)
+
+
+def test_prune_compress_validation():
+    assert prune(src=None) == sp24.SP24_ERR_NULL
+    assert prune(meta=None) == sp24.SP24_ERR_NULL
+    assert prune(dt=sp24.E4M3) == sp24.SP24_ERR_NULL          # scales required
+    assert prune(dt=sp24.F32) == sp24.SP24_ERR_DTYPE
+    assert prune(mask=FAKE) == sp24.SP24_ERR_NULL             # dense tiles required
+    assert prune(rows=0) == sp24.SP24_ERR_INVALID_ARG
+    assert prune(K=192, ld=192) == sp24.SP24_ERR_NOT_2_4
+    assert prune(ld=100) == sp24.SP24_ERR_INVALID_ARG
+    assert prune(ld=260) == sp24.SP24_ERR_ALIGNMENT
+    assert prune(src=FAKE + 8) == sp24.SP24_ERR_ALIGNMENT
+
+
+@pytest.mark.skipif(not NO_GPU, reason="only meaningful without a device")
+def test_valid_arguments_without_device_report_unsupported_device():
+    assert prune() == sp24.SP24_ERR_UNSUPPORTED_DEVICE
+    assert L.sp24_last_device_error() == sp24.SP24_ERR_UNSUPPORTED_DEVICE
+
+
+def gemm_args(**kw):
+    a = sp24.GemmArgs()
+    a.M, a.N, a.K = kw.get("M", 16), kw.get("N", 256), kw.get("K", 256)
+    a.in_dtype = kw.get("in_dtype", sp24.BF16)
+    a.out_dtype = kw.get("out_dtype", sp24.BF16)
+    a.tactic = kw.get("tactic", sp24.SPARSE)
+    a.X, a.ldx = kw.get("X", FAKE), kw.get("ldx", a.K)
+    a.W, a.ldw = kw.get("W", FAKE), kw.get("ldw", a.K // 2 if a.tactic == sp24.SPARSE else a.K)
+    a.W_meta = kw.get("W_meta", FAKE)
+    a.x_scales = kw.get("x_scales", None)
+    a.w_scales = kw.get("w_scales", None)
+    a.tile_dense_mask = kw.get("mask", None)
+    a.W_dense_tiles = kw.get("dense", None)
+    a.Y, a.ldy = kw.get("Y", FAKE), kw.get("ldy", a.N)
+    return a
+
+
+def g(**kw):
+    return L.sp24_gemm(ctypes.byref(gemm_args(**kw)), None)
+
+
+def test_gemm_validation():
+    assert L.sp24_gemm(None, None) == sp24.SP24_ERR_NULL
+    assert g(M=0) == sp24.SP24_ERR_INVALID_ARG
+    assert g(in_dtype=sp24.F32) == sp24.SP24_ERR_DTYPE
+    assert g(out_dtype=sp24.E4M3) == sp24.SP24_ERR_DTYPE
+    assert g(X=None) == sp24.SP24_ERR_NULL
+    assert g(W_meta=None) == sp24.SP24_ERR_NULL
+    assert g(N=200, ldy=200) == sp24.SP24_ERR_NOT_2_4           # sparse needs N % 128
+    assert g(K=320, ldx=320, ldw=160) == sp24.SP24_ERR_NOT_2_4  # sparse needs K % 128
+    assert g(in_dtype=sp24.E4M3) == sp24.SP24_ERR_NULL          # scales required
+    assert g(mask=FAKE, dense=FAKE) == sp24.SP24_ERR_DTYPE      # hybrid is e4m3 only
+    assert g(ldx=100) == sp24.SP24_ERR_INVALID_ARG
+    assert g(ldx=260) == sp24.SP24_ERR_ALIGNMENT
+    assert g(X=FAKE + 4) == sp24.SP24_ERR_ALIGNMENT
+    assert g(tactic=sp24.DENSE, K=200, ldx=200, ldw=200) == sp24.SP24_ERR_ALIGNMENT
+    assert g(tactic=7) == sp24.SP24_ERR_INVALID_ARG
+    assert L.sp24_gemm_workspace_bytes(ctypes.byref(gemm_args(M=0))) == 0
+
+
+def test_activation_and_selector_validation():
+    f = L.sp24_prune_compress_activations_fused
+    assert f(None, 16, 256, 256, FAKE, 256, 256, FAKE, 256, sp24.BF16, None, None, None, 0, None) \
+        == sp24.SP24_ERR_NULL
+    assert f(FAKE, 16, 192, 192, FAKE, 256, 192, FAKE, 256, sp24.BF16, None, None, None, 0, None) \
+        == sp24.SP24_ERR_NOT_2_4
+    assert f(FAKE, 16, 256, 256, FAKE, 256, 256, FAKE, 256, sp24.BF16, None, None, None, 0, None) \
+        == sp24.SP24_ERR_WORKSPACE
+    assert f(FAKE, 16, 256, 256, FAKE, 256, 256, FAKE, 256, sp24.BF16, FAKE, None, None, 0, None) \
+        == sp24.SP24_ERR_NULL
+    rec = sp24.TacticRecord()
+    assert L.sp24_select_tactic(None, None, 1, 1, ctypes.byref(rec), None) == sp24.SP24_ERR_NULL
+    d = gemm_args(tactic=sp24.DENSE)
+    assert L.sp24_select_tactic(None, ctypes.byref(d), 1, 0, ctypes.byref(rec), None) \
+        == sp24.SP24_ERR_INVALID_ARG
+    # values [16 x 128] bf16 (4096 B, 256-aligned) + one row block x 2 chunks of image
+    assert sp24.activations_workspace_bytes(16, 256) == 4096 + 2 * 2048

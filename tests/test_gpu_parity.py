@@ -1,0 +1,350 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Bit-exact: pruned/compressed values, the metadata image, E4M3 codes and
+scales, decompression.  Within |y - y_ref| <= 2e-3 * sum_k |x_k w_k| + 1e-6:
+GEMM outputs.  Shapes span several tiles plus ragged tails; the full-size
+cases check sampled outputs."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as orc
+from semi_structured_sparse_02_b200 import inputs, sp24
+from tests.gpu_helpers import (OracleSparseW, bits16, check_tolerance, dev, dev_bf16, oracle_x,
+                               u8, workspace_for)
+
+pytestmark = pytest.mark.gpu
+
+
+# ---------------------------------------------------------------------------
+# prune + compress (kernel 1), decompress, quantize
+# ---------------------------------------------------------------------------
+
+PRUNE_SHAPES = [(256, 256), (200, 384), (1, 128), (384, 1024), (130, 640)]
+
+
+@pytest.mark.parametrize("rows,K", PRUNE_SHAPES)
+def test_prune_compress_bf16_bit_exact(rows, K):
+    W = inputs.weights_with_outliers(rows, K, seed=rows + K)
+    ref = OracleSparseW(W, e4m3=False)
+    Wd = dev_bf16(W)
+    vals = torch.empty(rows, K // 2, dtype=torch.bfloat16, device="cuda")
+    meta = torch.empty(sp24.meta_bytes(rows, K), dtype=torch.uint8, device="cuda")
+    sp24.prune_compress(Wd, sp24.BF16, vals, meta)
+    torch.cuda.synchronize()
+    assert np.array_equal(bits16(vals), ref.values)
+    assert np.array_equal(u8(meta), ref.image)
+    dst = torch.empty(rows, K, dtype=torch.bfloat16, device="cuda")
+    sp24.decompress(vals, meta, rows, K, sp24.BF16, dst)
+    torch.cuda.synchronize()
+    assert np.array_equal(bits16(dst), orc.decompress(ref.values, ref.canon, rows, K))
+
+
+@pytest.mark.parametrize("rows,K", PRUNE_SHAPES)
+def test_prune_compress_e4m3_bit_exact(rows, K):
+    W = inputs.weights_with_outliers(rows, K, seed=7 * rows + K)
+    ref = OracleSparseW(W, e4m3=True)
+    Wd = dev_bf16(W)
+    vals = torch.empty(rows, K // 2, dtype=torch.uint8, device="cuda")
+    meta = torch.empty(sp24.meta_bytes(rows, K), dtype=torch.uint8, device="cuda")
+    sc = torch.empty(rows, dtype=torch.float32, device="cuda")
+    sp24.prune_compress(Wd, sp24.E4M3, vals, meta, row_scales=sc)
+    torch.cuda.synchronize()
+    assert np.array_equal(u8(vals), ref.values)
+    assert np.array_equal(u8(meta), ref.image)
+    assert np.array_equal(sc.cpu().numpy().view(np.uint32), ref.scales.view(np.uint32))
+    dst = torch.empty(rows, K, dtype=torch.uint8, device="cuda")
+    sp24.decompress(vals, meta, rows, K, sp24.E4M3, dst)
+    torch.cuda.synchronize()
+    assert np.array_equal(u8(dst), orc.decompress(ref.values, ref.canon, rows, K))
+
+
+def test_prune_handles_zero_rows_and_ties():
+    W = np.zeros((128, 256), np.uint16)
+    W[1, :8] = inputs.to_bf16_bits(np.array([1, 1, 1, 1, -2, 2, -2, 2], np.float32))
+    W[2, :4] = inputs.to_bf16_bits(np.array([0, 0, 3, 0], np.float32))
+    for e4 in (False, True):
+        ref = OracleSparseW(W, e4m3=e4)
+        vals = torch.empty(128, 128, dtype=torch.uint8 if e4 else torch.bfloat16, device="cuda")
+        meta = torch.empty(sp24.meta_bytes(128, 256), dtype=torch.uint8, device="cuda")
+        sc = torch.empty(128, dtype=torch.float32, device="cuda")
+        sp24.prune_compress(dev_bf16(W), sp24.E4M3 if e4 else sp24.BF16, vals, meta,
+                            row_scales=sc if e4 else None)
+        torch.cuda.synchronize()
+        assert np.array_equal(u8(meta), ref.image)
+        got = u8(vals) if e4 else bits16(vals)
+        assert np.array_equal(got, ref.values)
+        if e4:
+            assert np.array_equal(sc.cpu().numpy(), ref.scales)
+
+
+@pytest.mark.parametrize("e4", [False, True])
+def test_prune_hybrid_tiles_bit_exact(e4):
+    rows, K = 384, 1024
+    W = inputs.normal_bf16((rows, K), 0.02, seed=31)
+    mask = inputs.hybrid_mask(rows, K, seed=31)
+    ref = OracleSparseW(W, e4m3=e4, mask=mask)
+    vals = torch.empty(rows, K // 2, dtype=torch.uint8 if e4 else torch.bfloat16, device="cuda")
+    meta = torch.empty(sp24.meta_bytes(rows, K), dtype=torch.uint8, device="cuda")
+    dense = torch.zeros(rows, K, dtype=torch.uint8 if e4 else torch.bfloat16, device="cuda")
+    sc = torch.empty(rows, dtype=torch.float32, device="cuda")
+    sp24.prune_compress(dev_bf16(W), sp24.E4M3 if e4 else sp24.BF16, vals, meta,
+                        row_scales=sc if e4 else None, tile_mask=dev(mask), dense_tiles=dense)
+    torch.cuda.synchronize()
+    assert np.array_equal(u8(meta), ref.image)
+    if e4:
+        assert np.array_equal(u8(vals), ref.values)
+        assert np.array_equal(u8(dense), ref.dense)
+        assert np.array_equal(sc.cpu().numpy(), ref.scales)
+    else:
+        assert np.array_equal(bits16(vals), ref.values)
+        assert np.array_equal(bits16(dense), ref.dense)
+
+
+@pytest.mark.parametrize("rows,K", [(1, 5120), (16, 256), (128, 4096), (7, 25600)])
+def test_quantize_rows_e4m3_bit_exact(rows, K):
+    X = inputs.normal_bf16((rows, K), 1.0, seed=rows * 3 + K)
+    X[0, :] = 0  # an all-zero token: scale 1, codes 0
+    q_ref, s_ref = orc.quantize_rows_e4m3(X)
+    q = torch.empty(rows, K, dtype=torch.uint8, device="cuda")
+    s = torch.empty(rows, dtype=torch.float32, device="cuda")
+    sp24.quantize_e4m3_rows(dev_bf16(X), q, s)
+    torch.cuda.synchronize()
+    assert np.array_equal(u8(q), q_ref)
+    assert np.array_equal(s.cpu().numpy(), s_ref)
+
+
+# ---------------------------------------------------------------------------
+# GEMM (kernels 2 and 3)
+# ---------------------------------------------------------------------------
+
+GEMM_SHAPES = [
+    (16, 256, 256),     # the tiny configuration
+    (1, 384, 512),
+    (40, 256, 1280),
+    (130, 512, 768),    # two token tiles, ragged
+    (8, 1024, 4096),    # decode-like: split-K
+    (256, 384, 384),
+]
+
+
+def run_gemm(X_bits, W_bits, e4, tactic, out_f32, mask=None):
+    M, K = X_bits.shape
+    N = W_bits.shape[0]
+    xq, xs, X_hat = oracle_x(X_bits, e4)
+    Xd = dev(xq) if e4 else dev_bf16(xq)
+    Y = torch.empty(M, N, dtype=torch.float32 if out_f32 else torch.bfloat16, device="cuda")
+    if tactic == sp24.SPARSE:
+        ref = OracleSparseW(W_bits, e4m3=e4, mask=mask)
+        Wd = dev(ref.values) if e4 else dev_bf16(ref.values)
+        W_hat = ref.W_hat
+        a = sp24.gemm_args(Xd, Wd, Y, K, sp24.SPARSE, W_meta=dev(ref.image),
+                           x_scales=dev(xs) if e4 else None,
+                           w_scales=dev(ref.scales) if e4 else None,
+                           tile_mask=dev(mask) if mask is not None else None,
+                           W_dense_tiles=dev(ref.dense) if mask is not None else None)
+    else:
+        if e4:
+            wq, ws_ = orc.quantize_rows_e4m3(W_bits)
+            Wd = dev(wq)
+            W_hat = orc.e4m3_decode(wq) * ws_.astype(np.float64)[:, None]
+        else:
+            ws_ = None
+            Wd = dev_bf16(W_bits)
+            W_hat = orc.bf16_bits_to_f64(W_bits)
+        a = sp24.gemm_args(Xd, Wd, Y, K, sp24.DENSE, x_scales=dev(xs) if e4 else None,
+                           w_scales=dev(ws_) if e4 else None)
+    ws = workspace_for(a)
+    sp24.set_workspace(a, ws)
+    sp24.gemm(a)
+    torch.cuda.synchronize()
+    assert sp24.last_device_error() == sp24.SP24_OK
+    y_ref, a_ref = orc.gemm_f64(X_hat, W_hat)
+    return Y.float().cpu().numpy().astype(np.float64), y_ref, a_ref, a, ws
+
+
+@pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
+@pytest.mark.parametrize("e4", [False, True])
+@pytest.mark.parametrize("tactic", [sp24.SPARSE, sp24.DENSE])
+def test_gemm_parity(M, N, K, e4, tactic):
+    X, W = inputs.linear_pair(M, N, K, seed=M + N + K, outliers=True)
+    for out_f32 in (True, False):
+        y, y_ref, a_ref, _, _ = run_gemm(X, W, e4, tactic, out_f32)
+        check_tolerance(y, y_ref, a_ref, "M%d N%d K%d e4=%s tactic=%d f32=%s" % (M, N, K, e4, tactic, out_f32))
+
+
+@pytest.mark.parametrize("M,N,K", [(16, 200, 256), (3, 72, 128), (33, 136, 96)])
+def test_dense_gemm_ragged_n(M, N, K):
+    X, W = inputs.linear_pair(M, N, K, seed=5)
+    for e4 in (False, True):
+        y, y_ref, a_ref, _, _ = run_gemm(X, W, e4, sp24.DENSE, True)
+        check_tolerance(y, y_ref, a_ref, "dense ragged")
+
+
+def test_split_k_is_deterministic_and_leaves_counters_zero():
+    X, W = inputs.linear_pair(8, 1024, 4096, seed=77)
+    y1, y_ref, a_ref, args, ws = run_gemm(X, W, True, sp24.SPARSE, True)
+    assert ws is not None  # this decode shape runs split-K
+    sp24.gemm(args)
+    torch.cuda.synchronize()
+    check_tolerance(y1, y_ref, a_ref, "split-K")
+
+
+@pytest.mark.parametrize("M", [1, 16, 200])
+def test_hybrid_gemm_parity(M):
+    N, K = 512, 1024
+    X, W = inputs.linear_pair(M, N, K, seed=M + 3)
+    mask = inputs.hybrid_mask(N, K, seed=M)
+    y, y_ref, a_ref, _, _ = run_gemm(X, W, True, sp24.SPARSE, True, mask=mask)
+    check_tolerance(y, y_ref, a_ref, "hybrid")
+
+
+def test_gemm_with_gpu_pruned_weights_end_to_end():
+    M, N, K = 32, 640, 2048
+    X, W = inputs.linear_pair(M, N, K, seed=9, outliers=True)
+    Wd = dev_bf16(W)
+    vals = torch.empty(N, K // 2, dtype=torch.uint8, device="cuda")
+    meta = torch.empty(sp24.meta_bytes(N, K), dtype=torch.uint8, device="cuda")
+    ws_ = torch.empty(N, dtype=torch.float32, device="cuda")
+    sp24.prune_compress(Wd, sp24.E4M3, vals, meta, row_scales=ws_)
+    xq = torch.empty(M, K, dtype=torch.uint8, device="cuda")
+    xs = torch.empty(M, dtype=torch.float32, device="cuda")
+    sp24.quantize_e4m3_rows(dev_bf16(X), xq, xs)
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    a = sp24.gemm_args(xq, vals, Y, K, sp24.SPARSE, W_meta=meta, x_scales=xs, w_scales=ws_)
+    ws = workspace_for(a)
+    sp24.set_workspace(a, ws)
+    sp24.gemm(a)
+    torch.cuda.synchronize()
+    ref = OracleSparseW(W, e4m3=True)
+    _, _, X_hat = oracle_x(X, True)
+    y_ref, a_ref = orc.gemm_f64(X_hat, ref.W_hat)
+    check_tolerance(Y.float().cpu().numpy().astype(np.float64), y_ref, a_ref, "end to end")
+
+
+# ---------------------------------------------------------------------------
+# online activation prune + compress fused ahead of the GEMM (kernel 4)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("M,N,K", [(128, 384, 512), (200, 256, 1024), (1, 128, 128)])
+def test_activation_fused_parity(M, N, K):
+    X = inputs.student_t_bf16((M, K), 3.0, seed=M + K)
+    W = inputs.normal_bf16((N, K), 0.02, seed=N)
+    Y = torch.empty(M, N, dtype=torch.float32, device="cuda")
+    xv = torch.empty(M, K // 2, dtype=torch.bfloat16, device="cuda")
+    xm = torch.empty(sp24.meta_bytes(M, K), dtype=torch.uint8, device="cuda")
+    sp24.prune_compress_activations_fused(dev_bf16(X), dev_bf16(W), Y, x_values=xv, x_meta=xm)
+    torch.cuda.synchronize()
+    pruned, vals, canon = orc.prune_compress_bf16(X)
+    assert np.array_equal(bits16(xv), vals)
+    assert np.array_equal(u8(xm), orc.meta_image(canon, M, K, False))
+    y_ref, a_ref = orc.gemm_f64(orc.bf16_bits_to_f64(pruned), orc.bf16_bits_to_f64(W))
+    check_tolerance(Y.cpu().numpy().astype(np.float64), y_ref, a_ref, "activations")
+    # workspace variant, bf16 output
+    ws = torch.empty(sp24.activations_workspace_bytes(M, K), dtype=torch.uint8, device="cuda")
+    Y2 = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    sp24.prune_compress_activations_fused(dev_bf16(X), dev_bf16(W), Y2, workspace=ws)
+    torch.cuda.synchronize()
+    check_tolerance(Y2.float().cpu().numpy().astype(np.float64), y_ref, a_ref, "activations ws")
+
+
+# ---------------------------------------------------------------------------
+# full-size configurations, sampled outputs
+# ---------------------------------------------------------------------------
+
+def _sampled_check(X_hat_rows, W_hat_rows, y_gpu, ms, ns, what):
+    y_ref, a_ref = orc.gemm_f64_sampled(X_hat_rows, W_hat_rows, ms, ns)
+    check_tolerance(y_gpu[ms, ns], y_ref, a_ref, what)
+
+
+@pytest.mark.parametrize("N,K", inputs.DECODE_NK)
+def test_decode_full_size_sampled(N, K):
+    M = 8
+    X, W = inputs.linear_pair(M, N, K, seed=N + K)
+    Wd = dev_bf16(W)
+    vals = torch.empty(N, K // 2, dtype=torch.uint8, device="cuda")
+    meta = torch.empty(sp24.meta_bytes(N, K), dtype=torch.uint8, device="cuda")
+    ws_ = torch.empty(N, dtype=torch.float32, device="cuda")
+    sp24.prune_compress(Wd, sp24.E4M3, vals, meta, row_scales=ws_)
+    xq = torch.empty(M, K, dtype=torch.uint8, device="cuda")
+    xs = torch.empty(M, dtype=torch.float32, device="cuda")
+    sp24.quantize_e4m3_rows(dev_bf16(X), xq, xs)
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    a = sp24.gemm_args(xq, vals, Y, K, sp24.SPARSE, W_meta=meta, x_scales=xs, w_scales=ws_)
+    ws = workspace_for(a)
+    sp24.set_workspace(a, ws)
+    sp24.gemm(a)
+    torch.cuda.synchronize()
+    g = np.random.default_rng(1)
+    ns = g.choice(N, size=64, replace=False)
+    ms = g.integers(0, M, size=64)
+    # oracle on the sampled rows only
+    ref = OracleSparseW(W[ns], e4m3=True)
+    _, _, X_hat = oracle_x(X, True)
+    y_ref, a_ref = orc.gemm_f64_sampled(X_hat, ref.W_hat, ms, np.arange(ns.size))
+    y_gpu = Y.float().cpu().numpy().astype(np.float64)[ms, ns]
+    check_tolerance(y_gpu, y_ref, a_ref, "decode %dx%d" % (N, K))
+
+
+@pytest.mark.parametrize("e4", [False, True])
+def test_prefill_full_size_sampled(e4):
+    M, N, K = 2048, 4096, 4096
+    X, W = inputs.linear_pair(M, N, K, seed=123, outliers=True)
+    Wd = dev_bf16(W)
+    vals = torch.empty(N, K // 2, dtype=torch.uint8 if e4 else torch.bfloat16, device="cuda")
+    meta = torch.empty(sp24.meta_bytes(N, K), dtype=torch.uint8, device="cuda")
+    ws_ = torch.empty(N, dtype=torch.float32, device="cuda")
+    sp24.prune_compress(Wd, sp24.E4M3 if e4 else sp24.BF16, vals, meta, row_scales=ws_ if e4 else None)
+    if e4:
+        Xd = torch.empty(M, K, dtype=torch.uint8, device="cuda")
+        xs = torch.empty(M, dtype=torch.float32, device="cuda")
+        sp24.quantize_e4m3_rows(dev_bf16(X), Xd, xs)
+    else:
+        Xd, xs = dev_bf16(X), None
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    a = sp24.gemm_args(Xd, vals, Y, K, sp24.SPARSE, W_meta=meta, x_scales=xs,
+                       w_scales=ws_ if e4 else None)
+    sp24.gemm(a)
+    torch.cuda.synchronize()
+    g = np.random.default_rng(2)
+    ns = g.choice(N, size=48, replace=False)
+    ms = g.integers(0, M, size=48)
+    ref = OracleSparseW(W[ns], e4m3=e4)
+    xq, xsc, X_hat = oracle_x(X[ms], e4)
+    y_ref, a_ref = orc.gemm_f64_sampled(X_hat, ref.W_hat, np.arange(48), np.arange(48))
+    y_gpu = Y.float().cpu().numpy().astype(np.float64)[ms, ns]
+    check_tolerance(y_gpu, y_ref, a_ref, "prefill e4=%s" % e4)
+
+
+# ---------------------------------------------------------------------------
+# tactic selector (kernel 5) and the bounded wait
+# ---------------------------------------------------------------------------
+
+def test_select_tactic_record():
+    M, N, K = 8, 1024, 4096
+    X, W = inputs.linear_pair(M, N, K, seed=4)
+    _, _, _, sa, ws = run_gemm(X, W, True, sp24.SPARSE, False)
+    _, _, _, da, _ = run_gemm(X, W, True, sp24.DENSE, False)
+    rec = sp24.select_tactic(sa, da, warmup=2, iters=9)
+    assert rec["eligible"] and rec["iters"] == 9
+    assert rec["t_sparse_us"] > 0 and rec["t_dense_us"] > 0
+    assert rec["t_sparse_min_us"] <= rec["t_sparse_us"]
+    expect = orc.select_tactic([rec["t_sparse_us"]], [rec["t_dense_us"]])[0]
+    assert rec["selected"] == expect
+    assert (rec["reason"] == "") == (expect == "sparse")
+    # an ineligible sparse call (N not a multiple of 128) falls back to dense
+    sa.N = 1000
+    rec2 = sp24.select_tactic(sa, da, warmup=1, iters=3)
+    assert not rec2["eligible"] and rec2["selected"] == "dense" and rec2["reason"] == "Alignment failure"
+
+
+def test_bounded_wait_expires_without_fault_and_context_survives():
+    sp24.clear_device_error()
+    assert sp24.selftest_bounded_wait(2_000_000) == sp24.SP24_ERR_DEVICE_TIMEOUT
+    assert sp24.last_device_error() == sp24.SP24_ERR_DEVICE_TIMEOUT
+    assert sp24.clear_device_error() == sp24.SP24_OK
+    assert sp24.last_device_error() == sp24.SP24_OK
+    # the context is still usable
+    X, W = inputs.linear_pair(16, 256, 256, seed=0)
+    y, y_ref, a_ref, _, _ = run_gemm(X, W, False, sp24.SPARSE, True)
+    check_tolerance(y, y_ref, a_ref, "after self test")
