@@ -1,0 +1,487 @@
+#!/usr/bin/env python
+"""Benchmark of the 2:4 sparse GEMM hot path in the decode regime.
+
+Workload (one step): for M in {1, 8, 32, 128} and (N, K) in {(5120,5120),
+(25600,5120), (5120,25600), (10240,5120)}: cast the bf16 activations X [M x K]
+to E4M3 per token, then Y [M x N] = X * W^T with W pruned 2:4 along K and
+stored as E4M3 values + metadata with one fp32 scale per output channel
+(16 GEMMs, 32 kernel launches).  W ~ N(0, 0.02^2), X ~ N(0, 1), seeded.
+Each of the 16 GEMMs reads its own copy of W (852 MB of distinct weights per
+step, far above the 126 MB L2), so no weight is served from L2.
+
+The step is captured once in a CUDA graph and replayed; timing is CUDA
+events on the replay stream, max over ranks.  Under torchrun every rank runs
+an independent replica (the path has no exchange step).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "2:4 sparse GEMM TFLOPS & GB/s, % of roofline, speedup vs in-build dense"
+WORKLOAD = "decode-regime linear layers, e4m3 2:4 weights (per-channel scale), per-token e4m3 activations"
+L2_NOTE = ("inputs larger than L2: every GEMM of a step reads its own weight copy "
+           "(852 MB of distinct compressed weights per step vs 126 MB L2); no flush")
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", default="sp24", choices=["sp24", "reference"])
+    p.add_argument("--manifest", default="", help="write the tactic audit manifest here")
+    p.add_argument("--cpu-rows", type=int, default=256,
+                   help="weight rows per GEMM in the CPU-baseline sample")
+    return p.parse_args()
+
+
+def gemm_list():
+    from semi_structured_sparse_02_b200 import inputs
+    return [(M, N, K) for M in inputs.DECODE_M for (N, K) in inputs.DECODE_NK]
+
+
+def gemm_bytes(M, N, K):
+    """Algorithmic HBM bytes of one sparse e4m3 GEMM: W values (K/2 bytes per
+    row) + metadata (K/8) + W scales, X codes + scales, Y (bf16)."""
+    return N * K // 2 + N * K // 8 + 4 * N + M * K + 4 * M + 2 * M * N
+
+
+def quant_bytes(M, K):
+    return 2 * M * K + M * K + 4 * M
+
+
+def dense_gemm_bytes(M, N, K):
+    return N * K + 4 * N + M * K + 4 * M + 2 * M * N
+
+
+# ---------------------------------------------------------------------------
+# clocks
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        import torch
+        props = torch.cuda.get_device_properties(device_index)
+        self.bus = "%08X:%02X:%02X.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.bus, "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 7:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx.append(float(f[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[3:7]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# the CUDA path
+# ---------------------------------------------------------------------------
+def run_product(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from semi_structured_sparse_02_b200 import inputs, manifest, sp24
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    sp24.lib()  # raises if the CUDA library is missing
+    gemms = gemm_list()
+    shapes = sorted(set((N, K) for _, N, K in gemms))
+
+    # weights: prune + compress once per shape on the GPU, then one copy per GEMM
+    base = {}
+    for (N, K) in shapes:
+        Wb = inputs.normal_bf16((N, K), 0.02, seed=N + K)
+        W = torch.from_numpy(Wb.view(np.int16)).view(torch.bfloat16).to(dev)
+        vals = torch.empty(N, K // 2, dtype=torch.uint8, device=dev)
+        meta = torch.empty(sp24.meta_bytes(N, K), dtype=torch.uint8, device=dev)
+        wsc = torch.empty(N, dtype=torch.float32, device=dev)
+        sp24.prune_compress(W, sp24.E4M3, vals, meta, row_scales=wsc)
+        dq = torch.empty(N, K, dtype=torch.uint8, device=dev)
+        dsc = torch.empty(N, dtype=torch.float32, device=dev)
+        sp24.quantize_e4m3_rows(W, dq, dsc)
+        base[(N, K)] = (vals, meta, wsc, dq, dsc)
+        del W
+    torch.cuda.synchronize()
+
+    # activations and outputs live in single staging buffers (one copy each way for e2e)
+    x_elems = sum(M * K for M, _, K in gemms)
+    y_elems = sum(M * N for M, N, _ in gemms)
+    X_all = torch.empty(x_elems, dtype=torch.bfloat16, device=dev)
+    Y_all = torch.empty(y_elems, dtype=torch.bfloat16, device=dev)
+    Yd_all = torch.empty(y_elems, dtype=torch.bfloat16, device=dev)
+    inst = []
+    xo = yo = 0
+    for i, (M, N, K) in enumerate(gemms):
+        X = X_all[xo:xo + M * K].view(M, K)
+        X.copy_(torch.from_numpy(inputs.normal_bf16((M, K), 1.0, seed=1000 + i).view(np.int16))
+                .view(torch.bfloat16))
+        Y = Y_all[yo:yo + M * N].view(M, N)
+        Yd = Yd_all[yo:yo + M * N].view(M, N)
+        xo += M * K
+        yo += M * N
+        vals, meta, wsc, dq, dsc = (t.clone() for t in base[(N, K)])  # distinct copy per GEMM
+        xq = torch.empty(M, K, dtype=torch.uint8, device=dev)
+        xs = torch.empty(M, dtype=torch.float32, device=dev)
+        a_sp = sp24.gemm_args(xq, vals, Y, K, sp24.SPARSE, W_meta=meta, x_scales=xs, w_scales=wsc)
+        n = sp24.gemm_workspace_bytes(a_sp)
+        if n:
+            sp24.set_workspace(a_sp, torch.zeros(n, dtype=torch.uint8, device=dev))
+        a_dn = sp24.gemm_args(xq, dq, Yd, K, sp24.DENSE, x_scales=xs, w_scales=dsc)
+        n = sp24.gemm_workspace_bytes(a_dn)
+        if n:
+            sp24.set_workspace(a_dn, torch.zeros(n, dtype=torch.uint8, device=dev))
+        inst.append(dict(M=M, N=N, K=K, X=X, xq=xq, xs=xs, a_sp=a_sp, a_dn=a_dn))
+    del base
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.Stream(device=dev)
+
+    def step(kind):
+        for it in inst:
+            sp24.quantize_e4m3_rows(it["X"], it["xq"], it["xs"])
+            if kind == "sparse":
+                sp24.gemm(it["a_sp"])
+            elif kind == "dense":
+                sp24.gemm(it["a_dn"])
+            elif kind == "selected":
+                sp24.gemm(it["a_sp"] if it["tactic"] == "sparse" else it["a_dn"])
+
+    def gemm_only():
+        for it in inst:
+            sp24.gemm(it["a_sp"])
+
+    # tactic selection per GEMM (untimed), on the benchmark stream
+    with torch.cuda.stream(stream):
+        step("sparse")  # quantized X in place for the selector
+        records = {}
+        for it in inst:
+            r = sp24.select_tactic(it["a_sp"], it["a_dn"], warmup=3, iters=15, stream=stream)
+            it["tactic"] = r["selected"]
+            records["M%d_N%d_K%d" % (it["M"], it["N"], it["K"])] = r
+    man = manifest.build_manifest(records, revision="synthetic-seeded")
+    if args.manifest and rank == 0:
+        with open(args.manifest, "w") as f:
+            f.write(manifest.dumps(man))
+
+    # eager warm-up (sets kernel attributes), then capture the graphs
+    with torch.cuda.stream(stream):
+        for kind in ("sparse", "dense", "selected"):
+            step(kind)
+        gemm_only()
+    torch.cuda.synchronize()
+    graphs = {}
+    launches = {}
+    for kind in ("sparse", "dense", "selected", "gemm_only"):
+        g = torch.cuda.CUDAGraph()
+        c0 = sp24.launch_count()
+        with torch.cuda.graph(g, stream=stream):
+            if kind == "gemm_only":
+                gemm_only()
+            else:
+                step(kind)
+        launches[kind] = sp24.launch_count() - c0
+        graphs[kind] = g
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def time_graph(g, steps, warmup, sampler=None):
+        for _ in range(warmup):
+            g.replay()
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(steps):
+                g.replay()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([ms], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms = float(t.item())
+        return ms
+
+    K_steps, W_warm = args.steps, args.warmup
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.3)
+    t_wall0 = time.perf_counter()
+    ms_sparse = time_graph(graphs["sparse"], K_steps, W_warm)
+    t_wall = time.perf_counter() - t_wall0
+    # keep the GPU under the same load long enough for the clock record
+    extra = 0
+    if t_wall < 1.5:
+        n_more = int(max(1, (1.5 - t_wall) / max(ms_sparse / K_steps / 1e3, 1e-6)))
+        for _ in range(n_more):
+            graphs["sparse"].replay()
+        torch.cuda.synchronize()
+        extra = n_more
+    sampler.stop()
+    clocks = sampler.summary()
+    clocks["note"] = ("sampled over the timed replays" if extra == 0 else
+                      "sampled over the timed replays plus %d more replays of the same step" % extra)
+
+    ms_dense = time_graph(graphs["dense"], K_steps, W_warm)
+    ms_sel = time_graph(graphs["selected"], K_steps, W_warm)
+    ms_gemm = time_graph(graphs["gemm_only"], K_steps, W_warm)
+
+    # end to end through the public API: pinned host X in, host Y out, eager calls
+    X_host = torch.empty(x_elems, dtype=torch.bfloat16, pin_memory=True)
+    X_host.copy_(X_all.cpu())
+    Y_host = torch.empty(y_elems, dtype=torch.bfloat16, pin_memory=True)
+    e2e_steps = max(3, min(K_steps, 50))
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            X_all.copy_(X_host, non_blocking=True)
+            step("sparse")
+            Y_host.copy_(Y_all, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            X_all.copy_(X_host, non_blocking=True)
+            step("sparse")
+            Y_host.copy_(Y_all, non_blocking=True)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    ms_e2e = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms_e2e], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_e2e = float(t.item())
+
+    # accounting
+    step_bytes = sum(gemm_bytes(M, N, K) + quant_bytes(M, K) for M, N, K in gemms)
+    gemm_bytes_total = sum(gemm_bytes(M, N, K) for M, N, K in gemms)
+    step_flops = sum(2.0 * M * N * K for M, N, K in gemms)
+    t_step = ms_sparse / K_steps / 1e3
+    value = world * step_bytes / t_step / 1e9
+    t_gemm_launch = ms_gemm / K_steps / 1e3 / len(gemms)
+    bytes_per_launch = gemm_bytes_total / len(gemms)
+    peaks_path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(peaks_path):
+        peaks = json.load(open(peaks_path))
+        hbm_peak, peak_src = float(peaks["hbm_gbs"]), "measured"
+    else:
+        hbm_peak, peak_src = 6650.0, "fallback"
+    achieved = bytes_per_launch / t_gemm_launch / 1e9
+    e2e_value = world * step_bytes / (ms_e2e / e2e_steps / 1e3) / 1e9
+    out = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": K_steps,
+        "warmup": W_warm,
+        "ms_per_step": round(ms_sparse / K_steps, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "e4m3",
+        "data": "synthetic (seeded numpy normal draws rounded to bf16)",
+        "config": {
+            "workload": WORKLOAD,
+            "gemms_per_step": len(gemms),
+            "M": sorted(set(M for M, _, _ in gemms)),
+            "NK": [list(s) for s in shapes],
+            "parallelism": "replicas" if world > 1 else "single-gpu",
+            "l2": L2_NOTE,
+            "timing": "CUDA graph of one step replayed K times; CUDA events on the replay stream",
+        },
+        "tflops": round(world * step_flops / t_step / 1e12, 3),
+        "speedup_vs_dense": round(ms_dense / ms_sparse, 4),
+        "ms_per_step_dense": round(ms_dense / K_steps, 5),
+        "ms_per_step_selected": round(ms_sel / K_steps, 5),
+        "tactics": man["metrics"],
+        "roofline": {
+            "kernel": "k_gemm sparse e4m3 (tcgen05.mma.sp)",
+            "bound": "hbm",
+            "achieved": round(achieved, 1),
+            "peak": hbm_peak,
+            "peak_source": peak_src,
+            "unit": "GB/s",
+            "frac": round(achieved / hbm_peak, 4),
+            "traffic": None,
+            "bytes_per_launch": int(bytes_per_launch),
+            "us_per_launch": round(t_gemm_launch * 1e6, 3),
+        },
+        "clocks": clocks,
+        "e2e": {
+            "value": round(e2e_value, 2),
+            "unit": "GB/s",
+            "h2d_bytes_per_step": x_elems * 2,
+            "d2h_bytes_per_step": y_elems * 2,
+            "ms_per_step": round(ms_e2e / e2e_steps, 5),
+            "how": "eager public-API calls (sp24.quantize_e4m3_rows + sp24.gemm) with one pinned "
+                   "H2D copy of X and one D2H copy of Y per step",
+        },
+        "gpu_launches": launches["sparse"] * K_steps,
+    }
+    if rank == 0:
+        out["cpu_baseline"] = cpu_baseline(args.cpu_rows)
+    return out
+
+
+# ---------------------------------------------------------------------------
+# the CPU oracle (baseline leg and reference arm)
+# ---------------------------------------------------------------------------
+def oracle_gemm_sample(M, N, K, rows, seed):
+    """Time the oracle's per-call path for one decode GEMM on `rows` weight
+    rows: per-token E4M3 quantization of X, dequantization, fp64 sparse GEMM.
+    Weight preparation (prune + quantize, offline) is untimed.  Returns the
+    time scaled to the full N rows."""
+    from oracle import oracle as orc
+    from semi_structured_sparse_02_b200 import inputs
+    R = min(rows, N)
+    Wb = inputs.normal_bf16((R, K), 0.02, seed=seed)
+    vq, canon, wsc, _ = orc.prune_compress_e4m3(Wb)
+    wv = orc.e4m3_decode(vq) * wsc.astype(np.float64)[:, None]
+    Xb = inputs.normal_bf16((M, K), 1.0, seed=seed + 1)
+    t0 = time.perf_counter()
+    q, s = orc.quantize_rows_e4m3(Xb)
+    Xh = orc.e4m3_decode(q) * s.astype(np.float64)[:, None]
+    orc.gemm_sparse_f64(Xh, wv, canon)
+    dt = time.perf_counter() - t0
+    return dt * N / R
+
+
+def cpu_baseline(rows):
+    gemms = gemm_list()
+    t = 0.0
+    b = 0
+    for i, (M, N, K) in enumerate(gemms):
+        t += oracle_gemm_sample(M, N, K, rows, seed=7000 + i)
+        b += gemm_bytes(M, N, K) + quant_bytes(M, K)
+    return {"value": round(b / t / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": "all 16 decode GEMMs, %d weight rows each (time scaled by N/%d), "
+                      "single-threaded C oracle, fp64" % (rows, rows)}
+
+
+def run_reference(args, world):
+    gemms = gemm_list()
+    rows = 64
+    for i in range(args.warmup):
+        M, N, K = gemms[i % len(gemms)]
+        oracle_gemm_sample(M, N, K, rows, seed=9000 + i)
+    t = 0.0
+    b = 0
+    for i in range(args.steps):
+        M, N, K = gemms[i % len(gemms)]
+        t += oracle_gemm_sample(M, N, K, rows, seed=9100 + i)
+        b += gemm_bytes(M, N, K) + quant_bytes(M, K)
+    value = b / t / 1e9
+    line = {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": round(value, 4),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(t / args.steps * 1e3, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (seeded numpy normal draws rounded to bf16)",
+        "config": {"workload": WORKLOAD, "gemms_per_step": 1,
+                   "note": "the reference arm is the CPU oracle; one step = one of the 16 decode "
+                           "GEMMs in turn, on %d weight rows, time scaled to N rows" % rows},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": "one decode GEMM per step on %d weight rows" % rows},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args, world)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    out = run_product(args, rank, world, local_rank)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
