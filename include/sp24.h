@@ -140,6 +140,20 @@ int sp24_decompress(const void *values_dev, const void *meta_dev, int64_t rows, 
 int sp24_quantize_e4m3_rows(const void *src_dev, int64_t rows, int64_t K, int64_t ld,
                             void *q_dev, float *scales_dev, void *stream);
 
+/* One matrix of a grouped per-token quantization (host struct; pointers are
+ * device pointers, same meaning as in sp24_quantize_e4m3_rows). */
+typedef struct sp24_quant_item {
+    const void *src_dev;      /* bf16 [rows x K], row pitch ld elements          */
+    int64_t rows, K, ld;
+    void *q_dev;              /* e4m3 [rows x K], row pitch K                    */
+    float *scales_dev;        /* fp32 [rows]                                     */
+} sp24_quant_item;
+
+/* The per-token quantization of up to 32 independent matrices in one launch
+ * (same rule and results as sp24_quantize_e4m3_rows on each).  The item array
+ * is read on the host during the call. */
+int sp24_quantize_e4m3_rows_grouped(const sp24_quant_item *items, int n_items, void *stream);
+
 /* ---------------------------------------------------------------------- */
 /* GEMM (kernels 2 and 3)                                                  */
 /* ---------------------------------------------------------------------- */
@@ -162,14 +176,25 @@ typedef struct sp24_gemm_args {
     const void *W_dense_tiles;/* device [N x K] pitch K; read only at dense tiles */
     void *Y;                  /* device, [M x N] row pitch ldy                   */
     int64_t ldy;
-    void *workspace;          /* device split-K workspace (see below) or NULL    */
+    void *workspace;          /* device stream-K workspace (see below) or NULL   */
     size_t workspace_bytes;
+    uint32_t flags;           /* SP24_GEMM_* bits below, 0 for none              */
 } sp24_gemm_args;
 
-/* Bytes of split-K workspace the call will use (0 if it needs none).  The
- * workspace must be zero-filled once before its first use; every call that
- * returns SP24_OK leaves its counter words at zero again.  Calls that share a
- * workspace must not overlap on the GPU. */
+/* W, W_meta, w_scales, tile_dense_mask and W_dense_tiles are not written by
+ * the kernel that precedes the call in the stream (static weights): the GEMM
+ * starts streaming them before that kernel finishes (programmatic dependent
+ * launch).  X, x_scales and Y are always ordered after it. */
+#define SP24_GEMM_W_STATIC 1u
+
+/* Bytes of workspace the call would use for its stream-K schedule (0 if the
+ * shape needs none).  Shapes with fewer than two output tiles per SM split
+ * the tiles' K range evenly over all SMs and sum the partials in a fixed
+ * order; with a smaller or missing workspace the call falls back to whole
+ * tiles per CTA (same results up to fp32 summation order, fewer SMs busy).
+ * The workspace must be zero-filled once before its first use; every call
+ * that returns SP24_OK leaves its counter words at zero again.  Calls that
+ * share a workspace must not overlap on the GPU. */
 size_t sp24_gemm_workspace_bytes(const sp24_gemm_args *args);
 
 /* Y = s_x[m] * s_w[n] * sum_k x[m,k] * w[n,k] (scales only for E4M3), fp32

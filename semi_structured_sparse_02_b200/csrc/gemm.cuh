@@ -8,7 +8,19 @@
 //                shared -> tensor memory) and tcgen05.mma into one of two fp32
 //                accumulators in tensor memory, then tcgen05.commit.
 //   warps 2..5   epilogue: tcgen05.ld of the accumulator, scales, output
-//                store, or split-K partial store + last-arriver reduction.
+//                store; or a stream-K partial store + last-arriver reduction.
+//
+// Work schedule.  "Data-parallel": each CTA takes whole output tiles
+// round-robin.  "Stream-K" (few tiles, e.g. decode): the tiles' K-iterations
+// are laid end to end and every CTA streams one equal contiguous range of
+// them, so every SM moves the same number of bytes; a tile split between CTAs
+// is summed by whichever contributor finishes last, in contributor order.
+//
+// Kernel chaining.  Every CTA triggers the dependent grid at once
+// (programmatic dependent launch).  With p.w_static the producer starts
+// streaming the A operand (weights + metadata) before waiting on the
+// upstream grid; everything the upstream grid may write (B, scales of B,
+// the output) is touched only after griddepcontrol.wait.
 //
 // The sparse operand is always MMA operand A ("Sparse tensor cores", section
 // 2 of the 2:4-versus-quantization paper: the compressed first operand's
@@ -24,6 +36,7 @@
 namespace sp24 {
 
 enum GemmMode : int { kModeDense = 0, kModeSparse = 1, kModeHybrid = 2 };
+enum GemmSched : int { kSchedDataParallel = 0, kSchedStreamK = 1 };
 
 constexpr int kGemmThreads = 192;
 constexpr int kBlockA = 128;  // MMA M: rows of A per tile
@@ -33,18 +46,20 @@ struct GemmParams {
   int32_t K;                  // logical reduction length
   int32_t num_kt;             // K-stages per tile
   int32_t tiles_a, tiles_b;
-  int32_t splits;             // split-K factor
-  int32_t num_units;          // tiles_a * tiles_b * splits
+  int32_t sched;              // kSchedDataParallel / kSchedStreamK
+  int32_t maxseg;             // stream-K: partial slots per CTA
+  int64_t total_iters;        // stream-K: tiles * num_kt
   int32_t out_f32;            // 1: fp32 output, 0: bf16
-  int32_t use_pdl;            // wait on the upstream grid before loading
+  int32_t use_pdl;            // wait on the upstream grid before dependent loads
+  int32_t w_static;           // A operand is not written by the upstream grid
   const uint8_t* meta;        // metadata image of A (sparse / hybrid)
   const uint8_t* tile_mask;   // hybrid: [tiles_a x K/128]
   const float* scale_a;       // per-A-row scale (E4M3) or null
   const float* scale_b;       // per-B-row scale (E4M3) or null
   void* Y;
   int64_t ldy;
-  float* ws_partials;         // split-K partials [num_units][BN][128]
-  unsigned int* ws_counters;  // split-K arrival counters [tiles]
+  float* ws_partials;         // stream-K partials [grid][maxseg][128 rows][BN]
+  unsigned int* ws_counters;  // stream-K arrival counters [tiles]
   uint64_t timeout_ns;
 };
 
@@ -61,7 +76,7 @@ struct GemmCfg {
   static constexpr int kMetaChunks = kSparse ? (kBf16 ? 1 : 2) : (kHybrid ? 1 : 0);
   static constexpr int kMetaBytes = kMetaChunks * 2048;
   static constexpr int kStageBytes = kABytes + kBBytes + kMetaBytes;
-  static constexpr int kSmemBudget = 225 * 1024;
+  static constexpr int kSmemBudget = 212 * 1024;
   static constexpr int kStagesRaw = kSmemBudget / kStageBytes;
   static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
   static_assert(kStages >= 2, "stage too large");
@@ -71,19 +86,14 @@ struct GemmCfg {
   static constexpr int kTmemCols = kColsNeeded <= 32 ? 32 : kColsNeeded <= 64 ? 64 :
                                    kColsNeeded <= 128 ? 128 : kColsNeeded <= 256 ? 256 : 512;
   static_assert(kColsNeeded <= 512, "tensor memory overflow");
-  static constexpr int kMmasPerStage = 4;
-  // bookkeeping after the stages
+  // bookkeeping after the stages: barriers, slots, the B-scale slice, and a
+  // 2 KB output-staging tile per epilogue warp
   static constexpr int kBarOffset = kStages * kStageBytes;
-  static constexpr int kSmemBytes = kBarOffset + 256 + 1024;  // + barriers + alignment slack
+  static constexpr int kScaleOffset = kBarOffset + 256;
+  static constexpr int kEpiOffset = kScaleOffset + ((kBN * 4 + 127) / 128) * 128;
+  static constexpr int kSmemBytes = kEpiOffset + 4 * 2048 + 1024;  // + alignment slack
+  static_assert(kSmemBytes <= 232448, "shared memory overflow");
 };
-
-// Byte counts the producer expects for one stage.
-template <int kMode, bool kBf16, int kBN>
-__device__ __forceinline__ uint32_t stage_tx_bytes(bool hybrid_dense, int meta_chunks) {
-  using C = GemmCfg<kMode, kBf16, kBN>;
-  if (C::kHybrid) return hybrid_dense ? (C::kABytes + kBN * 128) : (kBlockA * 64 + kBN * 128 + 2048);
-  return C::kABytes + C::kBBytes + meta_chunks * 2048;
-}
 
 __device__ __forceinline__ void named_bar_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
@@ -101,6 +111,56 @@ __device__ __forceinline__ bool named_bar_red_and(int id, int count, bool pred) 
   return out != 0;
 }
 
+// GPU-scope acquire-release fetch-add: publishes (with the preceding CTA
+// barrier) the CTA's partial stores and acquires the other contributors'.
+__device__ __forceinline__ unsigned int atom_add_acq_rel_gpu(unsigned int* p, unsigned int v) {
+  unsigned int old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
+// ---------------------------------------------------------------------------
+// Work segments: a (tile, k-begin, k-end) range; j numbers the segments of
+// one CTA.  Every role of a CTA walks the same sequence.
+// ---------------------------------------------------------------------------
+struct SegIter {
+  int64_t it, it1;    // stream-K iteration cursor and end
+  int tile_dp;        // data-parallel tile cursor
+  int j;
+  __device__ __forceinline__ void init(const GemmParams& p, int cta, int grid) {
+    j = 0;
+    if (p.sched == kSchedStreamK) {
+      it = (int64_t)cta * p.total_iters / grid;
+      it1 = (int64_t)(cta + 1) * p.total_iters / grid;
+    } else {
+      tile_dp = cta;
+    }
+  }
+  __device__ __forceinline__ bool next(const GemmParams& p, int grid, int& tile, int& kb, int& ke,
+                                       int& seg) {
+    if (p.sched == kSchedStreamK) {
+      if (it >= it1) return false;
+      tile = (int)(it / p.num_kt);
+      kb = (int)(it - (int64_t)tile * p.num_kt);
+      ke = (int)min((int64_t)p.num_kt, (int64_t)kb + (it1 - it));
+      it += ke - kb;
+    } else {
+      if (tile_dp >= p.tiles_a * p.tiles_b) return false;
+      tile = tile_dp;
+      kb = 0;
+      ke = p.num_kt;
+      tile_dp += grid;
+    }
+    seg = j++;
+    return true;
+  }
+};
+
+// The CTA whose stream-K range holds iteration i.
+__device__ __forceinline__ int sk_owner(const GemmParams& p, int grid, int64_t i) {
+  return (int)(((i + 1) * grid - 1) / p.total_iters);
+}
+
 template <int kMode, bool kBf16, int kBN, bool kAIsW>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 k_gemm(const __grid_constant__ CUtensorMap tm_a,      // A: dense [rows_a x K] or values [rows_a x K/2]
@@ -109,6 +169,10 @@ k_gemm(const __grid_constant__ CUtensorMap tm_a,      // A: dense [rows_a x K] o
        const GemmParams p) {
   using C = GemmCfg<kMode, kBf16, kBN>;
   constexpr int S = C::kStages;
+
+  // the next kernel in the stream may launch now; it waits for our completion
+  // (griddepcontrol.wait) before it reads anything we write
+  pdl_launch_dependents();
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte alignment for the swizzled tiles
@@ -120,9 +184,12 @@ k_gemm(const __grid_constant__ CUtensorMap tm_a,      // A: dense [rows_a x K] o
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* last_flag = reinterpret_cast<int*>(tmem_slot + 2);
+  float* s_scale_b = reinterpret_cast<float*>(smem + C::kScaleOffset);
+  uint8_t* s_epi = smem + C::kEpiOffset;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const int grid = gridDim.x;
 
   auto full_bar = [&](int s) { return smem_u32(&bars[s]); };
   auto empty_bar = [&](int s) { return smem_u32(&bars[S + s]); };
@@ -155,16 +222,6 @@ k_gemm(const __grid_constant__ CUtensorMap tm_a,      // A: dense [rows_a x K] o
   tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (p.use_pdl) pdl_wait();
-
-  auto unit_coords = [&](int u, int& ta, int& tb, int& kb, int& ke) {
-    const int tile = u / p.splits;
-    const int s = u - tile * p.splits;
-    ta = tile % p.tiles_a;
-    tb = tile / p.tiles_a;
-    kb = (int)(((int64_t)s * p.num_kt) / p.splits);
-    ke = (int)(((int64_t)(s + 1) * p.num_kt) / p.splits);
-  };
   auto is_dense_tile = [&](int ta, int kt) -> bool {
     return p.tile_mask[(int64_t)ta * p.num_kt + kt] != 0;
   };
@@ -174,60 +231,101 @@ k_gemm(const __grid_constant__ CUtensorMap tm_a,      // A: dense [rows_a x K] o
     if (lane == 0) {
       const uint64_t pol_stream = policy_evict_first();  // A: read once
       const uint64_t pol_keep = policy_evict_last();     // B: re-read by many CTAs
-      int stage = 0;
-      uint32_t phase = 0;
       int armed[S];
       for (int s = 0; s < S; ++s) armed[s] = -1;
-      bool ok = true;
-      for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
-        int ta, tb, kb, ke;
-        unit_coords(u, ta, tb, kb, ke);
-        for (int kt = kb; kt < ke; ++kt) {
-          if (!mbar_wait(empty_bar(stage), phase ^ 1, p.timeout_ns, kDevErrWaitEmpty)) {
-            ok = false;
-            *abort_flag = 1;
-            break;
-          }
-          uint8_t* st = smem + stage * C::kStageBytes;
-          const uint32_t sa = smem_u32(st);
-          const uint32_t sb = sa + C::kABytes;
-          const uint32_t sm = sb + C::kBBytes;
-          const int32_t ya = ta * kBlockA, yb = tb * kBN;
-          if (C::kHybrid) {
-            const bool dense = is_dense_tile(ta, kt);
-            mbar_arrive_expect_tx(full_bar(stage), stage_tx_bytes<kMode, kBf16, kBN>(dense, 1));
-            if (dense) {
-              tma_load_2d(sa, &tm_a, full_bar(stage), kt * 128, ya, pol_stream);
-            } else {
-              tma_load_2d(sa, &tm_a2, full_bar(stage), kt * 64, ya, pol_stream);
-              bulk_load(sm, p.meta + ((int64_t)ta * p.num_kt + kt) * 2048, 2048, full_bar(stage),
-                        pol_stream);
-            }
-            tma_load_2d(sb, &tm_b, full_bar(stage), kt * 128, yb, pol_keep);
+
+      // the A-operand (and metadata) part of one stage; returns its bytes
+      auto load_a = [&](int stage, int ta, int kt, bool arm_only_a) -> void {
+        (void)arm_only_a;
+        const uint32_t sa = smem_u32(smem + stage * C::kStageBytes);
+        const uint32_t sm = sa + C::kABytes + C::kBBytes;
+        const int32_t ya = ta * kBlockA;
+        if (C::kHybrid) {
+          if (is_dense_tile(ta, kt)) {
+            tma_load_2d(sa, &tm_a, full_bar(stage), kt * 128, ya, pol_stream);
           } else {
-            int chunks = 0;
-            if (C::kSparse) {
-              const int kc_total = p.K / 128;
-              const int kc0 = kt * C::kMetaChunks;
-              chunks = min(C::kMetaChunks, kc_total - kc0);
-            }
-            mbar_arrive_expect_tx(full_bar(stage), stage_tx_bytes<kMode, kBf16, kBN>(false, chunks));
-            // A: 128 bytes of each row per stage
-            const int ax = C::kSparse ? kt * (C::kKT / 2) : kt * C::kKT;  // elements
-            tma_load_2d(sa, &tm_a, full_bar(stage), ax, ya, pol_stream);
-            // B: logical K range of the stage, in 128-byte boxes
-            const int box_elems = kBf16 ? 64 : 128;
-#pragma unroll
-            for (int bx = 0; bx < C::kBBoxes; ++bx)
-              tma_load_2d(sb + bx * kBN * 128, &tm_b, full_bar(stage), kt * C::kKT + bx * box_elems,
-                          yb, pol_keep);
-            if (C::kSparse) {
-              const int64_t kc_total = p.K / 128;
-              const uint8_t* src = p.meta + ((int64_t)ta * kc_total + (int64_t)kt * C::kMetaChunks) * 2048;
-              bulk_load(sm, src, chunks * 2048, full_bar(stage), pol_stream);
-            }
+            tma_load_2d(sa, &tm_a2, full_bar(stage), kt * 64, ya, pol_stream);
+            bulk_load(sm, p.meta + ((int64_t)ta * p.num_kt + kt) * 2048, 2048, full_bar(stage),
+                      pol_stream);
           }
-          armed[stage] = (int)phase;
+        } else {
+          const int ax = C::kSparse ? kt * (C::kKT / 2) : kt * C::kKT;  // elements
+          tma_load_2d(sa, &tm_a, full_bar(stage), ax, ya, pol_stream);
+          if (C::kSparse) {
+            const int64_t kc_total = p.K / 128;
+            const int chunks = (int)min((int64_t)C::kMetaChunks, kc_total - (int64_t)kt * C::kMetaChunks);
+            const uint8_t* src = p.meta + ((int64_t)ta * kc_total + (int64_t)kt * C::kMetaChunks) * 2048;
+            bulk_load(sm, src, chunks * 2048, full_bar(stage), pol_stream);
+          }
+        }
+      };
+      auto load_b = [&](int stage, int tb, int kt) {
+        const uint32_t sb = smem_u32(smem + stage * C::kStageBytes) + C::kABytes;
+        const int32_t yb = tb * kBN;
+        if (C::kHybrid) {
+          tma_load_2d(sb, &tm_b, full_bar(stage), kt * 128, yb, pol_keep);
+        } else {
+          const int box_elems = kBf16 ? 64 : 128;
+#pragma unroll
+          for (int bx = 0; bx < C::kBBoxes; ++bx)
+            tma_load_2d(sb + bx * kBN * 128, &tm_b, full_bar(stage), kt * C::kKT + bx * box_elems, yb,
+                        pol_keep);
+        }
+      };
+      auto stage_bytes = [&](int ta, int kt) -> uint32_t {
+        if (C::kHybrid)
+          return is_dense_tile(ta, kt) ? (uint32_t)(C::kABytes + kBN * 128)
+                                       : (uint32_t)(kBlockA * 64 + kBN * 128 + 2048);
+        uint32_t b = C::kABytes + C::kBBytes;
+        if (C::kSparse) {
+          const int64_t kc_total = p.K / 128;
+          b += (uint32_t)min((int64_t)C::kMetaChunks, kc_total - (int64_t)kt * C::kMetaChunks) * 2048;
+        }
+        return b;
+      };
+
+      // 1. weights first: arm the first S stages and start their A loads
+      //    before the dependency wait when A is known not to be in flux
+      int pre = 0;
+      if (p.w_static) {
+        SegIter it;
+        it.init(p, blockIdx.x, grid);
+        int tile, kb, ke, seg;
+        while (pre < S && it.next(p, grid, tile, kb, ke, seg)) {
+          const int ta = tile % p.tiles_a;
+          for (int kt = kb; kt < ke && pre < S; ++kt, ++pre) {
+            mbar_arrive_expect_tx(full_bar(pre), stage_bytes(ta, kt));
+            load_a(pre, ta, kt, true);
+            armed[pre] = 0;
+          }
+        }
+      }
+      if (p.use_pdl) pdl_wait();
+
+      // 2. the main stream
+      int stage = 0;
+      uint32_t phase = 0;
+      int n = 0;
+      bool ok = true;
+      SegIter it;
+      it.init(p, blockIdx.x, grid);
+      int tile, kb, ke, seg;
+      while (ok && it.next(p, grid, tile, kb, ke, seg)) {
+        const int ta = tile % p.tiles_a, tb = tile / p.tiles_a;
+        for (int kt = kb; kt < ke; ++kt, ++n) {
+          if (n < pre) {
+            load_b(stage, tb, kt);  // A already in flight
+          } else {
+            if (!mbar_wait(empty_bar(stage), phase ^ 1, p.timeout_ns, kDevErrWaitEmpty)) {
+              ok = false;
+              *abort_flag = 1;
+              break;
+            }
+            mbar_arrive_expect_tx(full_bar(stage), stage_bytes(ta, kt));
+            load_a(stage, ta, kt, false);
+            load_b(stage, tb, kt);
+            armed[stage] = (int)phase;
+          }
           if (++stage == S) {
             stage = 0;
             phase ^= 1;
@@ -250,9 +348,11 @@ k_gemm(const __grid_constant__ CUtensorMap tm_a,      // A: dense [rows_a x K] o
       uint32_t phase = 0;
       uint32_t acc_i = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
-        int ta, tb, kb, ke;
-        unit_coords(u, ta, tb, kb, ke);
+      SegIter it;
+      it.init(p, blockIdx.x, grid);
+      int tile, kb, ke, seg;
+      while (ok && it.next(p, grid, tile, kb, ke, seg)) {
+        const int ta = tile % p.tiles_a;
         const int buf = acc_i & 1;
         const uint32_t acc_phase = (acc_i >> 1) & 1;
         if (!mbar_wait(acce_bar(buf), acc_phase ^ 1, p.timeout_ns, kDevErrWaitAccEmpty)) {
@@ -339,15 +439,32 @@ k_gemm(const __grid_constant__ CUtensorMap tm_a,      // A: dense [rows_a x K] o
     __syncwarp();
   } else {
     // ------------------------------------------------------------------ epilogue
+    if (p.use_pdl) pdl_wait();                 // B scales and Y may belong to the upstream grid
     const int lg = warp & 3;                   // tensor-memory lane group of this warp
     const int row = lg * 32 + lane;            // accumulator row (lane) within the tile
     const int et = threadIdx.x - 64;           // 0..127
     uint32_t acc_i = 0;
-    for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
-      int ta, tb, kb, ke;
-      unit_coords(u, ta, tb, kb, ke);
+    int cached_tb = -1;
+    SegIter it;
+    it.init(p, blockIdx.x, grid);
+    int tile, kb, ke, seg;
+    while (it.next(p, grid, tile, kb, ke, seg)) {
+      const int ta = tile % p.tiles_a, tb = tile / p.tiles_a;
       const int buf = acc_i & 1;
       const uint32_t acc_phase = (acc_i >> 1) & 1;
+      const int ga = ta * kBlockA + row;     // global A row of this thread
+      const bool a_live = ga < p.rows_a;
+      // scales: loaded before waiting for the accumulator so their latency hides
+      const float sa_v = (p.scale_a != nullptr && a_live) ? __ldg(p.scale_a + ga) : 1.0f;
+      if (tb != cached_tb) {
+        named_bar_sync(1, 128);
+        for (int i = et; i < kBN; i += 128) {
+          const int gb = tb * kBN + i;
+          s_scale_b[i] = (p.scale_b != nullptr && gb < p.rows_b) ? p.scale_b[gb] : 1.0f;
+        }
+        named_bar_sync(1, 128);
+        cached_tb = tb;
+      }
       bool ok = mbar_wait(accf_bar(buf), acc_phase, p.timeout_ns, kDevErrWaitAccFull);
       __syncwarp();
       ok = named_bar_red_and(2, 128, ok);  // all epilogue threads agree
@@ -356,48 +473,87 @@ k_gemm(const __grid_constant__ CUtensorMap tm_a,      // A: dense [rows_a x K] o
         break;
       }
       tc_fence_after_sync();
-      const int ga = ta * kBlockA + row;     // global A row of this thread
-      const bool a_live = ga < p.rows_a;
-      const float sa_v = (p.scale_a != nullptr && a_live) ? p.scale_a[ga] : 1.0f;
       const uint32_t tbase = tmem_base + ((uint32_t)(lg * 32) << 16) + buf * kBN;
-      float* part = p.splits > 1 ? p.ws_partials + (int64_t)u * kBN * 128 : nullptr;
+      const bool full = (kb == 0 && ke == p.num_kt);
+      // stream-K partials: [cta][seg][row][kBN] fp32, each thread's row contiguous
+      float* part = full ? nullptr
+                         : p.ws_partials + (((int64_t)blockIdx.x * p.maxseg + seg) * 128 + row) * kBN;
+
+      // Scales and stores 16 consecutive accumulator columns starting at c0
+      // with 16-byte vector stores.  Rows of Y are 16-byte aligned (checked
+      // on the host); a vector that crosses the end of a row is stored per
+      // element.
+      uint8_t* wtile = s_epi + (warp - 2) * 2048;  // this warp's staging tile
+      const int eb = p.out_f32 ? 4 : 2;
+      const int per_vec = 16 / eb;                   // elements per 16-byte vector
+      auto store16 = [&](const float (&v)[16], int c0) {
+        const int gb0 = tb * kBN + c0;
+        if (kAIsW) {
+          // lane = n (output feature), column = m (token).  Stage the warp's
+          // 32 n x 16 m block transposed, then write each output row's 32
+          // consecutive n as 16-byte vectors.
+          const int n0 = ta * kBlockA + lg * 32;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float y = v[i] * sa_v * s_scale_b[c0 + i];
+            if (p.out_f32) reinterpret_cast<float*>(wtile)[i * 32 + lane] = y;
+            else reinterpret_cast<__nv_bfloat16*>(wtile)[i * 32 + lane] = __float2bfloat16_rn(y);
+          }
+          __syncwarp();
+          const int vec_per_row = 32 / per_vec;
+          for (int q = lane; q < 16 * vec_per_row; q += 32) {
+            const int i = q / vec_per_row, sg = q - i * vec_per_row;
+            const int m = gb0 + i;
+            const int n = n0 + sg * per_vec;
+            if (m >= p.rows_b || n >= p.rows_a) continue;
+            uint8_t* dst = static_cast<uint8_t*>(p.Y) + ((int64_t)m * p.ldy + n) * eb;
+            const uint8_t* src = wtile + (i * 32 + sg * per_vec) * eb;
+            if (n + per_vec <= p.rows_a) {
+              *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
+            } else {
+              for (int e = 0; e < p.rows_a - n; ++e)
+                for (int b = 0; b < eb; ++b) dst[e * eb + b] = src[e * eb + b];
+            }
+          }
+          __syncwarp();
+        } else {
+          // lane = m (token), column = n (output feature): this thread's 16
+          // consecutive n of row ga
+          if (!a_live) return;
+          alignas(16) uint8_t buf[64];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float y = v[i] * sa_v * s_scale_b[c0 + i];
+            if (p.out_f32) reinterpret_cast<float*>(buf)[i] = y;
+            else reinterpret_cast<__nv_bfloat16*>(buf)[i] = __float2bfloat16_rn(y);
+          }
+          uint8_t* dst = static_cast<uint8_t*>(p.Y) + ((int64_t)ga * p.ldy + gb0) * eb;
+          if (gb0 + 16 <= p.rows_b) {
+            for (int q = 0; q < 16 / per_vec; ++q)
+              reinterpret_cast<uint4*>(dst)[q] = reinterpret_cast<const uint4*>(buf)[q];
+          } else {
+            for (int e = 0; e < p.rows_b - gb0; ++e)
+              for (int b = 0; b < eb; ++b) dst[e * eb + b] = buf[e * eb + b];
+          }
+        }
+      };
+
 #pragma unroll 1
       for (int c0 = 0; c0 < kBN; c0 += 16) {
         uint32_t r[16];
         tmem_ld_x16(tbase + c0, r);
         tmem_ld_wait();
         if (part != nullptr) {
+          float4* q = reinterpret_cast<float4*>(part + c0);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) __stcg(part + (c0 + i) * 128 + row, __uint_as_float(r[i]));
+          for (int j = 0; j < 4; ++j)
+            __stcg(q + j, make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                      __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3])));
         } else {
-          const int gb0 = tb * kBN + c0;
-          if (kAIsW) {
-            // lane = n (output feature), column = m (token)
+          float v[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int m = gb0 + i;
-              if (m < p.rows_b && a_live) {
-                float v = __uint_as_float(r[i]) * sa_v;
-                if (p.scale_b != nullptr) v *= p.scale_b[m];
-                if (p.out_f32) static_cast<float*>(p.Y)[(int64_t)m * p.ldy + ga] = v;
-                else static_cast<__nv_bfloat16*>(p.Y)[(int64_t)m * p.ldy + ga] = __float2bfloat16_rn(v);
-              }
-            }
-          } else {
-            // lane = m (token), column = n (output feature)
-            if (a_live) {
-#pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                const int n = gb0 + i;
-                if (n < p.rows_b) {
-                  float v = __uint_as_float(r[i]) * sa_v;
-                  if (p.scale_b != nullptr) v *= p.scale_b[n];
-                  if (p.out_f32) static_cast<float*>(p.Y)[(int64_t)ga * p.ldy + n] = v;
-                  else static_cast<__nv_bfloat16*>(p.Y)[(int64_t)ga * p.ldy + n] = __float2bfloat16_rn(v);
-                }
-              }
-            }
-          }
+          for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+          store16(v, c0);
         }
       }
       tc_fence_before_sync();
@@ -405,39 +561,36 @@ k_gemm(const __grid_constant__ CUtensorMap tm_a,      // A: dense [rows_a x K] o
       ++acc_i;
 
       if (part != nullptr) {
-        // split-K: the last unit of this tile to arrive sums all partials in
-        // slot order (deterministic) and writes the output.
-        const int tile = u / p.splits;
-        __threadfence();
-        named_bar_sync(1, 128);
+        // The contributors of this tile are the CTAs whose iteration ranges
+        // cover it; the last to arrive sums all partials in contributor order.
+        const int c_first = sk_owner(p, grid, (int64_t)tile * p.num_kt);
+        const int c_last = sk_owner(p, grid, (int64_t)(tile + 1) * p.num_kt - 1);
+        const unsigned int count = (unsigned int)(c_last - c_first + 1);
+        named_bar_sync(1, 128);  // every partial store of this CTA precedes the ticket
         if (et == 0) {
-          const unsigned int old = atomicAdd(&p.ws_counters[tile], 1u);
-          *last_flag = (old == (unsigned int)(p.splits - 1)) ? 1 : 0;
+          const unsigned int old = atom_add_acq_rel_gpu(&p.ws_counters[tile], 1u);
+          *last_flag = (old == count - 1) ? 1 : 0;
         }
         named_bar_sync(1, 128);
         if (*last_flag) {
-          __threadfence();
-          const float* base = p.ws_partials + (int64_t)tile * p.splits * kBN * 128;
 #pragma unroll 1
-          for (int c = 0; c < kBN; ++c) {
-            const int gb = tb * kBN + c;
-            float v = 0.0f;
-            for (int s = 0; s < p.splits; ++s) v += __ldcg(base + ((int64_t)s * kBN + c) * 128 + row);
-            if (kAIsW) {
-              if (gb < p.rows_b && a_live) {
-                v *= sa_v;
-                if (p.scale_b != nullptr) v *= p.scale_b[gb];
-                if (p.out_f32) static_cast<float*>(p.Y)[(int64_t)gb * p.ldy + ga] = v;
-                else static_cast<__nv_bfloat16*>(p.Y)[(int64_t)gb * p.ldy + ga] = __float2bfloat16_rn(v);
-              }
-            } else {
-              if (gb < p.rows_b && a_live) {
-                v *= sa_v;
-                if (p.scale_b != nullptr) v *= p.scale_b[gb];
-                if (p.out_f32) static_cast<float*>(p.Y)[(int64_t)ga * p.ldy + gb] = v;
-                else static_cast<__nv_bfloat16*>(p.Y)[(int64_t)ga * p.ldy + gb] = __float2bfloat16_rn(v);
-              }
+          for (int c0 = 0; c0 < kBN; c0 += 16) {
+            float v[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[i] = 0.0f;
+            for (int c = c_first; c <= c_last; ++c) {
+              // the contributor's segment index for this tile
+              const int64_t it0 = (int64_t)c * p.total_iters / grid;
+              const int sj = tile - (int)(it0 / p.num_kt);
+              const float4* q = reinterpret_cast<const float4*>(
+                  p.ws_partials + (((int64_t)c * p.maxseg + sj) * 128 + row) * kBN + c0);
+              const float4 a0 = __ldcg(q), a1 = __ldcg(q + 1), a2 = __ldcg(q + 2), a3 = __ldcg(q + 3);
+              v[0] += a0.x; v[1] += a0.y; v[2] += a0.z; v[3] += a0.w;
+              v[4] += a1.x; v[5] += a1.y; v[6] += a1.z; v[7] += a1.w;
+              v[8] += a2.x; v[9] += a2.y; v[10] += a2.z; v[11] += a2.w;
+              v[12] += a3.x; v[13] += a3.y; v[14] += a3.z; v[15] += a3.w;
             }
+            store16(v, c0);
           }
           if (et == 0) p.ws_counters[tile] = 0u;  // ready for the next call
         }

@@ -92,6 +92,8 @@ k_prune_compress(const uint16_t* __restrict__ src, int64_t rows, int64_t K, int6
                  const float* __restrict__ amax_in, const uint8_t* __restrict__ tile_mask,
                  void* __restrict__ dense_out) {
   __shared__ __align__(16) uint8_t canon[kChunkRows][16];
+  pdl_launch_dependents();
+  pdl_wait();  // src may be written by the upstream grid
   const int64_t KC = K / kChunkK;
   const int64_t RB = (rows + kChunkRows - 1) / kChunkRows;
   const int64_t n_chunks = RB * KC;
@@ -203,47 +205,102 @@ __global__ void k_finalize_scales(float* __restrict__ s, int64_t rows) {
 }
 
 // ---------------------------------------------------------------------------
-// Per-row (per-token) E4M3 quantization: one CTA per row.  Pass 1 reduces
-// the amax, pass 2 re-reads the row (L1/L2 resident) and writes codes.
+// Per-row (per-token) E4M3 quantization of a group of matrices: one CTA per
+// row.  Rows of up to kQuantThreads * kQuantRegVecs * 8 elements are read
+// once into registers (amax, then codes from the registers); longer rows are
+// read twice (the second read hits L1/L2).
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256)
-k_quantize_rows_e4m3(const uint16_t* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
-                     uint8_t* __restrict__ q, float* __restrict__ scales) {
-  __shared__ uint32_t red[8];
-  for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
-    const uint4* p = reinterpret_cast<const uint4*>(src + row * ld);
-    uint32_t m = 0;
-    for (int64_t i = threadIdx.x; i < K / 8; i += blockDim.x) {
-      const uint4 v = __ldg(p + i);
-      m = max(m, max(max(v.x & 0x7FFFu, v.x >> 16 & 0x7FFFu), max(v.y & 0x7FFFu, v.y >> 16 & 0x7FFFu)));
-      m = max(m, max(max(v.z & 0x7FFFu, v.z >> 16 & 0x7FFFu), max(v.w & 0x7FFFu, v.w >> 16 & 0x7FFFu)));
+constexpr int kQuantThreads = 512;
+constexpr int kQuantRegVecs = 8;
+constexpr int kMaxQuantItems = 32;
+
+struct QuantItem {
+  const uint16_t* src;
+  int64_t rows, K, ld;
+  uint8_t* q;
+  float* scales;
+};
+
+struct QuantGroup {
+  QuantItem item[kMaxQuantItems];
+  int64_t row_start[kMaxQuantItems + 1];  // prefix sums of rows
+  int n;
+};
+
+__device__ __forceinline__ uint32_t amax_bits8(const uint4 v) {
+  uint32_t m = max(max(v.x & 0x7FFFu, v.x >> 16 & 0x7FFFu), max(v.y & 0x7FFFu, v.y >> 16 & 0x7FFFu));
+  return max(m, max(max(v.z & 0x7FFFu, v.z >> 16 & 0x7FFFu), max(v.w & 0x7FFFu, v.w >> 16 & 0x7FFFu)));
+}
+
+__device__ __forceinline__ uint2 e4m3_codes8(const uint4 v, float inv) {
+  const uint32_t e[8] = {v.x & 0xFFFFu, v.x >> 16, v.y & 0xFFFFu, v.y >> 16,
+                         v.z & 0xFFFFu, v.z >> 16, v.w & 0xFFFFu, v.w >> 16};
+  uint32_t lo = 0, hi = 0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) lo |= (uint32_t)e4m3_of(__fmul_rn(bf16_bits_to_float(e[j]), inv)) << (8 * j);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) hi |= (uint32_t)e4m3_of(__fmul_rn(bf16_bits_to_float(e[4 + j]), inv)) << (8 * j);
+  return make_uint2(lo, hi);
+}
+
+// Block-wide max of one value per thread (all threads get the result).
+__device__ __forceinline__ uint32_t block_max(uint32_t m, uint32_t* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    uint32_t t = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0u;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) t = max(t, __shfl_xor_sync(0xFFFFFFFFu, t, o));
+    if (threadIdx.x == 0) red[32] = t;
+  }
+  __syncthreads();
+  const uint32_t r = red[32];
+  __syncthreads();  // red may be reused by the next row
+  return r;
+}
+
+__global__ void __launch_bounds__(kQuantThreads)
+k_quantize_rows_e4m3(const __grid_constant__ QuantGroup g) {
+  __shared__ uint32_t red[33];
+  pdl_launch_dependents();
+  pdl_wait();  // the activations may be written by the upstream grid
+  const int64_t total = g.row_start[g.n];
+  for (int64_t gr = blockIdx.x; gr < total; gr += gridDim.x) {
+    int i = 0;
+    while (gr >= g.row_start[i + 1]) ++i;
+    const QuantItem& it = g.item[i];
+    const int64_t row = gr - g.row_start[i];
+    const uint4* p = reinterpret_cast<const uint4*>(it.src + row * it.ld);
+    uint8_t* q = it.q + row * it.K;
+    const int64_t nv = it.K / 8;
+    if (nv <= (int64_t)kQuantThreads * kQuantRegVecs) {
+      uint4 reg[kQuantRegVecs];
+      uint32_t m = 0;
+#pragma unroll
+      for (int j = 0; j < kQuantRegVecs; ++j) {
+        const int64_t idx = threadIdx.x + (int64_t)j * kQuantThreads;
+        reg[j] = idx < nv ? __ldg(p + idx) : make_uint4(0, 0, 0, 0);
+        m = max(m, amax_bits8(reg[j]));
+      }
+      const float amax = bf16_bits_to_float(block_max(m, red));
+      const float inv = e4m3_inv_scale(amax);
+      if (threadIdx.x == 0) it.scales[row] = amax == 0.0f ? 1.0f : __fdiv_rn(amax, 448.0f);
+#pragma unroll
+      for (int j = 0; j < kQuantRegVecs; ++j) {
+        const int64_t idx = threadIdx.x + (int64_t)j * kQuantThreads;
+        if (idx < nv) *reinterpret_cast<uint2*>(q + idx * 8) = e4m3_codes8(reg[j], inv);
+      }
+    } else {
+      uint32_t m = 0;
+      for (int64_t idx = threadIdx.x; idx < nv; idx += kQuantThreads) m = max(m, amax_bits8(__ldg(p + idx)));
+      const float amax = bf16_bits_to_float(block_max(m, red));
+      const float inv = e4m3_inv_scale(amax);
+      if (threadIdx.x == 0) it.scales[row] = amax == 0.0f ? 1.0f : __fdiv_rn(amax, 448.0f);
+      for (int64_t idx = threadIdx.x; idx < nv; idx += kQuantThreads)
+        *reinterpret_cast<uint2*>(q + idx * 8) = e4m3_codes8(__ldg(p + idx), inv);
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
-    __syncthreads();
-    if (threadIdx.x < 32) {
-      uint32_t t = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0u;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) t = max(t, __shfl_xor_sync(0xFFFFFFFFu, t, o));
-      if (threadIdx.x == 0) red[0] = t;
-    }
-    __syncthreads();
-    const float amax = bf16_bits_to_float(red[0]);
-    const float inv = e4m3_inv_scale(amax);
-    if (threadIdx.x == 0) scales[row] = amax == 0.0f ? 1.0f : __fdiv_rn(amax, 448.0f);
-    for (int64_t i = threadIdx.x; i < K / 8; i += blockDim.x) {
-      const uint4 v = __ldg(p + i);
-      const uint32_t e[8] = {v.x & 0xFFFFu, v.x >> 16, v.y & 0xFFFFu, v.y >> 16,
-                             v.z & 0xFFFFu, v.z >> 16, v.w & 0xFFFFu, v.w >> 16};
-      uint32_t lo = 0, hi = 0;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) lo |= (uint32_t)e4m3_of(__fmul_rn(bf16_bits_to_float(e[j]), inv)) << (8 * j);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) hi |= (uint32_t)e4m3_of(__fmul_rn(bf16_bits_to_float(e[4 + j]), inv)) << (8 * j);
-      *reinterpret_cast<uint2*>(q + row * K + i * 8) = make_uint2(lo, hi);
-    }
-    __syncthreads();
   }
 }
 

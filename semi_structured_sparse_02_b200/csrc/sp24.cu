@@ -123,8 +123,11 @@ struct Plan {
   bool a_is_w;
   int bn;
   int kt;          // logical K per stage
-  int stage_a_bytes;
-  int num_kt, tiles_a, tiles_b, splits, num_units;
+  int num_kt, tiles_a, tiles_b;
+  int sched;       // kSchedDataParallel / kSchedStreamK
+  int grid;
+  int maxseg;      // stream-K partial slots per CTA
+  int64_t total_iters;
   size_t ws_bytes;
 };
 
@@ -141,40 +144,32 @@ int stage_k(int mode, bool bf16) {
   return bf16 ? 64 : 128;
 }
 
-size_t split_ws_bytes(const Plan& pl) {
-  if (pl.splits <= 1) return 0;
-  const size_t part = (size_t)pl.num_units * pl.bn * 128 * sizeof(float);
+size_t sk_ws_bytes(const Plan& pl) {
+  const size_t part = (size_t)pl.grid * pl.maxseg * pl.bn * 128 * sizeof(float);
   const size_t cnt = ((size_t)pl.tiles_a * pl.tiles_b * sizeof(unsigned int) + 255) & ~(size_t)255;
   return part + cnt;
 }
 
-// Splits the K range of each output tile so that the persistent grid's
-// waves are balanced (decode shapes have fewer tiles than SMs).
-void choose_splits(Plan& pl, int sms, size_t ws_cap) {
+// Work schedule: with at least two tiles per SM the CTAs take whole tiles
+// round-robin; with fewer (the decode shapes) the tiles' K-iterations are
+// split evenly over the SMs (stream-K), which needs a workspace for the
+// partial sums.  Without enough workspace the whole-tile schedule is used.
+void choose_schedule(Plan& pl, int sms, size_t ws_cap) {
   const int64_t tiles = (int64_t)pl.tiles_a * pl.tiles_b;
-  pl.splits = 1;
-  if (tiles < 2 * sms) {
-    double best = 1e300;
-    const int max_s = std::min(pl.num_kt, 64);
-    for (int s = 1; s <= max_s; ++s) {
-      const int64_t units = tiles * s;
-      const int64_t waves = (units + sms - 1) / sms;
-      const int64_t kt_per = (pl.num_kt + s - 1) / s;
-      const double per_unit = (double)kt_per * pl.stage_a_bytes +
-                              (s > 1 ? 2.0 * pl.bn * 128 * 4 : 0.0);
-      const double cost = (double)waves * per_unit;
-      Plan t = pl;
-      t.splits = s;
-      t.num_units = (int)units;
-      if (split_ws_bytes(t) > ws_cap) break;
-      if (cost < best * 0.999) {
-        best = cost;
-        pl.splits = s;
-      }
-    }
+  pl.total_iters = tiles * pl.num_kt;
+  pl.sched = kSchedDataParallel;
+  pl.grid = (int)std::min<int64_t>(tiles, sms);
+  pl.maxseg = 0;
+  pl.ws_bytes = 0;
+  if (tiles < 2 * (int64_t)sms && pl.num_kt > 1) {
+    Plan t = pl;
+    t.sched = kSchedStreamK;
+    t.grid = (int)std::min<int64_t>(t.total_iters, sms);
+    const int64_t per_cta = (t.total_iters + t.grid - 1) / t.grid;
+    t.maxseg = (int)((per_cta + t.num_kt - 1) / t.num_kt) + 1;
+    t.ws_bytes = sk_ws_bytes(t);
+    if (t.ws_bytes <= ws_cap) pl = t;
   }
-  pl.num_units = (int)(tiles * pl.splits);
-  pl.ws_bytes = split_ws_bytes(pl);
 }
 
 // ---------------------------------------------------------------------------
@@ -271,7 +266,7 @@ int validate_gemm(const sp24_gemm_args* a) {
   if (a->ldx < a->K || a->ldy < a->N) return SP24_ERR_INVALID_ARG;
   if (!aligned16(a->X) || !aligned16(a->W)) return SP24_ERR_ALIGNMENT;
   if ((a->ldx * eb) % 16 != 0 || (a->ldw * eb) % 16 != 0) return SP24_ERR_ALIGNMENT;
-  if ((reinterpret_cast<uintptr_t>(a->Y) % ob) != 0) return SP24_ERR_ALIGNMENT;
+  if (!aligned16(a->Y) || (a->ldy * ob) % 16 != 0) return SP24_ERR_ALIGNMENT;
   return SP24_OK;
 }
 
@@ -286,10 +281,22 @@ Plan plan_gemm(const sp24_gemm_args* a, int sms, size_t ws_cap) {
   pl.num_kt = (int)((a->K + pl.kt - 1) / pl.kt);
   pl.tiles_a = (int)((a->N + kBlockA - 1) / kBlockA);
   pl.tiles_b = (int)((a->M + pl.bn - 1) / pl.bn);
-  // bytes of the streamed operand per stage (A tile + metadata)
-  pl.stage_a_bytes = kBlockA * 128 + (pl.mode == kModeDense ? 0 : 2048 * (pl.bf16 ? 1 : 2));
-  choose_splits(pl, sms, ws_cap);
+  choose_schedule(pl, sms, ws_cap);
   return pl;
+}
+
+void fill_sched(GemmParams& p, const Plan& pl, void* workspace) {
+  p.num_kt = pl.num_kt;
+  p.tiles_a = pl.tiles_a;
+  p.tiles_b = pl.tiles_b;
+  p.sched = pl.sched;
+  p.maxseg = pl.maxseg;
+  p.total_iters = pl.total_iters;
+  if (pl.sched == kSchedStreamK) {
+    p.ws_partials = static_cast<float*>(workspace);
+    p.ws_counters = reinterpret_cast<unsigned int*>(
+        static_cast<uint8_t*>(workspace) + (size_t)pl.grid * pl.maxseg * pl.bn * 128 * sizeof(float));
+  }
 }
 
 int run_gemm(const sp24_gemm_args* a, cudaStream_t stream) {
@@ -323,27 +330,36 @@ int run_gemm(const sp24_gemm_args* a, cudaStream_t stream) {
   p.rows_a = (int32_t)a->N;
   p.rows_b = (int32_t)a->M;
   p.K = (int32_t)a->K;
-  p.num_kt = pl.num_kt;
-  p.tiles_a = pl.tiles_a;
-  p.tiles_b = pl.tiles_b;
-  p.splits = pl.splits;
-  p.num_units = pl.num_units;
+  fill_sched(p, pl, a->workspace);
   p.out_f32 = a->out_dtype == SP24_F32;
   p.use_pdl = 1;
+  p.w_static = (a->flags & SP24_GEMM_W_STATIC) ? 1 : 0;
   p.meta = static_cast<const uint8_t*>(a->W_meta);
   p.tile_mask = a->tile_dense_mask;
   p.scale_a = a->in_dtype == SP24_E4M3 ? a->w_scales : nullptr;
   p.scale_b = a->in_dtype == SP24_E4M3 ? a->x_scales : nullptr;
   p.Y = a->Y;
   p.ldy = a->ldy;
-  if (pl.splits > 1) {
-    p.ws_partials = static_cast<float*>(a->workspace);
-    p.ws_counters = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(a->workspace) +
-                                                    (size_t)pl.num_units * pl.bn * 128 * sizeof(float));
-  }
   p.timeout_ns = g_timeout_ns.load();
-  const int grid = std::min(pl.num_units, di.sms);
-  return dispatch_gemm(pl, ta, ta2, tb, p, grid, stream);
+  return dispatch_gemm(pl, ta, ta2, tb, p, pl.grid, stream);
+}
+
+// Launch with programmatic dependent launch allowed (the kernel itself waits
+// on the upstream grid before touching dependent memory).
+template <typename... KArgs, typename... Args>
+int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+               Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return launch_result(cudaLaunchKernelEx(&cfg, kernel, args...));
 }
 
 }  // namespace
@@ -422,16 +438,33 @@ int sp24_decompress(const void* values, const void* meta, int64_t rows, int64_t 
 
 int sp24_quantize_e4m3_rows(const void* src, int64_t rows, int64_t K, int64_t ld, void* q,
                             float* scales, void* stream) {
-  if (src == nullptr || q == nullptr || scales == nullptr) return SP24_ERR_NULL;
-  if (rows < 1 || K < 1 || ld < K) return SP24_ERR_INVALID_ARG;
-  if (K % 16 != 0 || ld % 8 != 0 || !aligned16(src) || !aligned16(q)) return SP24_ERR_ALIGNMENT;
+  sp24_quant_item item = {src, rows, K, ld, q, scales};
+  return sp24_quantize_e4m3_rows_grouped(&item, 1, stream);
+}
+
+int sp24_quantize_e4m3_rows_grouped(const sp24_quant_item* items, int n_items, void* stream) {
+  if (items == nullptr) return SP24_ERR_NULL;
+  if (n_items < 1 || n_items > kMaxQuantItems) return SP24_ERR_INVALID_ARG;
+  QuantGroup g;
+  memset(&g, 0, sizeof g);
+  g.n = n_items;
+  g.row_start[0] = 0;
+  for (int i = 0; i < n_items; ++i) {
+    const sp24_quant_item& it = items[i];
+    if (it.src_dev == nullptr || it.q_dev == nullptr || it.scales_dev == nullptr) return SP24_ERR_NULL;
+    if (it.rows < 1 || it.K < 1 || it.ld < it.K) return SP24_ERR_INVALID_ARG;
+    if (it.K % 16 != 0 || it.ld % 8 != 0 || !aligned16(it.src_dev) || !aligned16(it.q_dev))
+      return SP24_ERR_ALIGNMENT;
+    g.item[i] = QuantItem{static_cast<const uint16_t*>(it.src_dev), it.rows, it.K, it.ld,
+                          static_cast<uint8_t*>(it.q_dev), it.scales_dev};
+    g.row_start[i + 1] = g.row_start[i] + it.rows;
+  }
   DeviceInfo di;
   int st = current_device_info(&di);
   if (st != SP24_OK) return st;
-  const int grid = (int)std::min<int64_t>(rows, (int64_t)di.sms * 8);
-  k_quantize_rows_e4m3<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const uint16_t*>(src), rows, K, ld, static_cast<uint8_t*>(q), scales);
-  return launch_result(cudaGetLastError());
+  const int grid = (int)std::min<int64_t>(g.row_start[n_items], (int64_t)di.sms * 4);
+  return launch_pdl(k_quantize_rows_e4m3, dim3(grid), dim3(kQuantThreads), 0,
+                    static_cast<cudaStream_t>(stream), g);
 }
 
 size_t sp24_gemm_workspace_bytes(const sp24_gemm_args* a) {
@@ -464,6 +497,7 @@ int sp24_prune_compress_activations_fused(const void* X, int64_t M, int64_t K, i
   if (K % 128 != 0) return SP24_ERR_NOT_2_4;
   if ((x_values == nullptr) != (x_meta == nullptr)) return SP24_ERR_NULL;
   if (ldx % 8 != 0 || ldw % 8 != 0 || !aligned16(X) || !aligned16(W)) return SP24_ERR_ALIGNMENT;
+  if (!aligned16(Y) || (ldy * (out_dtype == SP24_F32 ? 4 : 2)) % 16 != 0) return SP24_ERR_ALIGNMENT;
   if (x_values == nullptr) {
     if (workspace == nullptr) return SP24_ERR_WORKSPACE;
     if (workspace_bytes < sp24_activations_workspace_bytes(M, K)) return SP24_ERR_WORKSPACE;
@@ -478,10 +512,11 @@ int sp24_prune_compress_activations_fused(const void* X, int64_t M, int64_t K, i
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int64_t chunks = ((M + 127) / 128) * (K / 128);
   const int grid = (int)std::min<int64_t>(chunks, (int64_t)di.sms * 4);
-  k_prune_compress<false><<<grid, kPruneThreads, 0, s>>>(static_cast<const uint16_t*>(X), M, K, ldx,
-                                                         x_values, static_cast<uint8_t*>(x_meta), nullptr,
-                                                         nullptr, nullptr);
-  if ((st = launch_result(cudaGetLastError())) != SP24_OK) return st;
+  st = launch_pdl(k_prune_compress<false>, dim3(grid), dim3(kPruneThreads), 0, s,
+                  static_cast<const uint16_t*>(X), M, K, ldx, x_values, static_cast<uint8_t*>(x_meta),
+                  static_cast<const float*>(nullptr), static_cast<const uint8_t*>(nullptr),
+                  static_cast<void*>(nullptr));
+  if (st != SP24_OK) return st;
 
   // GEMM with X (compressed) as the sparse operand A and W dense as B.
   Plan pl;
@@ -493,8 +528,7 @@ int sp24_prune_compress_activations_fused(const void* X, int64_t M, int64_t K, i
   pl.num_kt = (int)(K / 128);
   pl.tiles_a = (int)((M + 127) / 128);
   pl.tiles_b = (int)((N + 127) / 128);
-  pl.splits = 1;
-  pl.num_units = pl.tiles_a * pl.tiles_b;
+  choose_schedule(pl, di.sms, 0);  // whole tiles: no workspace for partial sums
   CUtensorMap ta, tb;
   bool ok = make_map(&ta, x_values, 2, K / 2, M, (K / 2) * 2, 64, kBlockA, CU_TENSOR_MAP_SWIZZLE_128B);
   ok &= make_map(&tb, W, 2, K, N, ldw * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
@@ -504,19 +538,14 @@ int sp24_prune_compress_activations_fused(const void* X, int64_t M, int64_t K, i
   p.rows_a = (int32_t)M;
   p.rows_b = (int32_t)N;
   p.K = (int32_t)K;
-  p.num_kt = pl.num_kt;
-  p.tiles_a = pl.tiles_a;
-  p.tiles_b = pl.tiles_b;
-  p.splits = 1;
-  p.num_units = pl.num_units;
+  fill_sched(p, pl, nullptr);
   p.out_f32 = out_dtype == SP24_F32;
   p.use_pdl = 1;
   p.meta = static_cast<const uint8_t*>(x_meta);
   p.Y = Y;
   p.ldy = ldy;
   p.timeout_ns = g_timeout_ns.load();
-  const int ggrid = std::min(pl.num_units, di.sms);
-  return dispatch_gemm(pl, ta, ta, tb, p, ggrid, s);
+  return dispatch_gemm(pl, ta, ta, tb, p, pl.grid, s);
 }
 
 int sp24_select_tactic(const sp24_gemm_args* sparse_args, const sp24_gemm_args* dense_args, int warmup,

@@ -32,6 +32,7 @@ SP24_ERR_WORKSPACE = 9
 
 BF16, E4M3, F32 = 0, 1, 2
 SPARSE, DENSE = 0, 1
+GEMM_W_STATIC = 1
 
 
 class Sp24Error(RuntimeError):
@@ -51,6 +52,14 @@ class GemmArgs(ctypes.Structure):
         ("tile_dense_mask", ctypes.c_void_p), ("W_dense_tiles", ctypes.c_void_p),
         ("Y", ctypes.c_void_p), ("ldy", ctypes.c_int64),
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+        ("flags", ctypes.c_uint32),
+    ]
+
+
+class QuantItem(ctypes.Structure):
+    _fields_ = [
+        ("src", ctypes.c_void_p), ("rows", ctypes.c_int64), ("K", ctypes.c_int64),
+        ("ld", ctypes.c_int64), ("q", ctypes.c_void_p), ("scales", ctypes.c_void_p),
     ]
 
 
@@ -84,6 +93,7 @@ def lib() -> ctypes.CDLL:
         "sp24_prune_compress": (I, [P, I64, I64, I64, I, P, P, P, P, P, P]),
         "sp24_decompress": (I, [P, P, I64, I64, I, P, P]),
         "sp24_quantize_e4m3_rows": (I, [P, I64, I64, I64, P, P, P]),
+        "sp24_quantize_e4m3_rows_grouped": (I, [ctypes.POINTER(QuantItem), I, P]),
         "sp24_gemm_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(GemmArgs)]),
         "sp24_gemm": (I, [ctypes.POINTER(GemmArgs), P]),
         "sp24_activations_workspace_bytes": (ctypes.c_size_t, [I64, I64]),
@@ -183,6 +193,25 @@ def quantize_e4m3_rows(src: torch.Tensor, q: torch.Tensor, scales: torch.Tensor,
                                          _stream(stream)), "sp24_quantize_e4m3_rows")
 
 
+class QuantGroup:
+    """A prepared grouped per-token quantization (the item array and the
+    tensors it points at are kept alive with it)."""
+
+    def __init__(self, pairs):
+        # pairs: list of (src bf16 [rows x K], q e4m3 [rows x K], scales fp32 [rows])
+        self.items = (QuantItem * len(pairs))()
+        self._keep = []
+        for i, (src, q, sc) in enumerate(pairs):
+            rows, K = src.shape
+            self.items[i] = QuantItem(src.data_ptr(), rows, K, src.stride(0), q.data_ptr(),
+                                      sc.data_ptr())
+            self._keep += [src, q, sc]
+
+    def __call__(self, stream=None):
+        _check(lib().sp24_quantize_e4m3_rows_grouped(self.items, len(self.items), _stream(stream)),
+               "sp24_quantize_e4m3_rows_grouped")
+
+
 # ---------------------------------------------------------------------------
 # GEMM
 # ---------------------------------------------------------------------------
@@ -191,7 +220,7 @@ def gemm_args(X: torch.Tensor, W: torch.Tensor, Y: torch.Tensor, K: int, tactic:
               W_meta: Optional[torch.Tensor] = None, x_scales: Optional[torch.Tensor] = None,
               w_scales: Optional[torch.Tensor] = None, tile_mask: Optional[torch.Tensor] = None,
               W_dense_tiles: Optional[torch.Tensor] = None,
-              workspace: Optional[torch.Tensor] = None) -> GemmArgs:
+              workspace: Optional[torch.Tensor] = None, flags: int = 0) -> GemmArgs:
     """Y [M x N] = X [M x K] * W^T; W is [N x K] (dense) or values [N x K/2]."""
     a = GemmArgs()
     a.M, a.N, a.K = X.shape[0], Y.shape[1], K
@@ -206,6 +235,7 @@ def gemm_args(X: torch.Tensor, W: torch.Tensor, Y: torch.Tensor, K: int, tactic:
     a.tile_dense_mask = tile_mask.data_ptr() if tile_mask is not None else None
     a.W_dense_tiles = W_dense_tiles.data_ptr() if W_dense_tiles is not None else None
     a.Y, a.ldy = Y.data_ptr(), Y.stride(0)
+    a.flags = flags
     if workspace is not None:
         a.workspace = workspace.data_ptr()
         a.workspace_bytes = workspace.numel() * workspace.element_size()

@@ -101,6 +101,21 @@ def test_gemm_validation():
     assert L.sp24_gemm_workspace_bytes(ctypes.byref(gemm_args(M=0))) == 0
 
 
+def test_grouped_quantize_validation():
+    f = L.sp24_quantize_e4m3_rows_grouped
+    assert f(None, 1, None) == sp24.SP24_ERR_NULL
+    items = (sp24.QuantItem * 2)()
+    items[0] = sp24.QuantItem(FAKE, 4, 256, 256, FAKE, FAKE)
+    items[1] = sp24.QuantItem(FAKE, 4, 256, 256, None, FAKE)
+    assert f(items, 0, None) == sp24.SP24_ERR_INVALID_ARG
+    assert f(items, 33, None) == sp24.SP24_ERR_INVALID_ARG
+    assert f(items, 2, None) == sp24.SP24_ERR_NULL
+    items[1] = sp24.QuantItem(FAKE, 4, 250, 256, FAKE, FAKE)
+    assert f(items, 2, None) == sp24.SP24_ERR_ALIGNMENT
+    items[1] = sp24.QuantItem(FAKE, 0, 256, 256, FAKE, FAKE)
+    assert f(items, 2, None) == sp24.SP24_ERR_INVALID_ARG
+
+
 def test_activation_and_selector_validation():
     f = L.sp24_prune_compress_activations_fused
     assert f(None, 16, 256, 256, FAKE, 256, 256, FAKE, 256, sp24.BF16, None, None, None, 0, None) \

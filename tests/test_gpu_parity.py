@@ -114,6 +114,22 @@ def test_quantize_rows_e4m3_bit_exact(rows, K):
     assert np.array_equal(s.cpu().numpy(), s_ref)
 
 
+def test_grouped_quantize_matches_oracle_per_matrix():
+    shapes = [(1, 5120), (8, 25600), (32, 256), (128, 4096), (3, 33024)]  # last: two-pass path
+    pairs, refs = [], []
+    for i, (rows, K) in enumerate(shapes):
+        X = inputs.normal_bf16((rows, K), 1.0, seed=50 + i)
+        refs.append(orc.quantize_rows_e4m3(X))
+        pairs.append((dev_bf16(X), torch.empty(rows, K, dtype=torch.uint8, device="cuda"),
+                      torch.empty(rows, dtype=torch.float32, device="cuda")))
+    g = sp24.QuantGroup(pairs)
+    g()
+    torch.cuda.synchronize()
+    for (src, q, s), (q_ref, s_ref) in zip(pairs, refs):
+        assert np.array_equal(u8(q), q_ref)
+        assert np.array_equal(s.cpu().numpy(), s_ref)
+
+
 # ---------------------------------------------------------------------------
 # GEMM (kernels 2 and 3)
 # ---------------------------------------------------------------------------
@@ -128,7 +144,7 @@ GEMM_SHAPES = [
 ]
 
 
-def run_gemm(X_bits, W_bits, e4, tactic, out_f32, mask=None):
+def run_gemm(X_bits, W_bits, e4, tactic, out_f32, mask=None, use_ws=True, flags=0):
     M, K = X_bits.shape
     N = W_bits.shape[0]
     xq, xs, X_hat = oracle_x(X_bits, e4)
@@ -154,7 +170,8 @@ def run_gemm(X_bits, W_bits, e4, tactic, out_f32, mask=None):
             W_hat = orc.bf16_bits_to_f64(W_bits)
         a = sp24.gemm_args(Xd, Wd, Y, K, sp24.DENSE, x_scales=dev(xs) if e4 else None,
                            w_scales=dev(ws_) if e4 else None)
-    ws = workspace_for(a)
+    a.flags = flags
+    ws = workspace_for(a) if use_ws else None
     sp24.set_workspace(a, ws)
     sp24.gemm(a)
     torch.cuda.synchronize()
@@ -181,13 +198,36 @@ def test_dense_gemm_ragged_n(M, N, K):
         check_tolerance(y, y_ref, a_ref, "dense ragged")
 
 
-def test_split_k_is_deterministic_and_leaves_counters_zero():
+@pytest.mark.parametrize("M,N,K", [(8, 1024, 4096), (1, 384, 512), (40, 256, 1280), (128, 640, 2048)])
+@pytest.mark.parametrize("e4", [False, True])
+def test_whole_tile_schedule_without_workspace(M, N, K, e4):
+    X, W = inputs.linear_pair(M, N, K, seed=3 * M + N)
+    y, y_ref, a_ref, _, ws = run_gemm(X, W, e4, sp24.SPARSE, True, use_ws=False)
+    assert ws is None
+    check_tolerance(y, y_ref, a_ref, "whole tiles")
+
+
+@pytest.mark.parametrize("tactic", [sp24.SPARSE, sp24.DENSE])
+def test_stream_k_is_deterministic_and_reusable(tactic):
+    # three calls on one workspace: identical bits each time (fixed summation
+    # order) -- a counter left non-zero would break the second or third call
     X, W = inputs.linear_pair(8, 1024, 4096, seed=77)
-    y1, y_ref, a_ref, args, ws = run_gemm(X, W, True, sp24.SPARSE, True)
-    assert ws is not None  # this decode shape runs split-K
-    sp24.gemm(args)
-    torch.cuda.synchronize()
-    check_tolerance(y1, y_ref, a_ref, "split-K")
+    y1, y_ref, a_ref, args, ws = run_gemm(X, W, True, tactic, True, flags=sp24.GEMM_W_STATIC)
+    assert ws is not None  # this decode shape takes the stream-K schedule
+    check_tolerance(y1, y_ref, a_ref, "stream-K")
+    Y = args._keep[2]
+    for _ in range(2):
+        Y.zero_()
+        sp24.gemm(args)
+        torch.cuda.synchronize()
+        assert np.array_equal(Y.cpu().numpy(), y1.astype(np.float32))
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 5120, 5120), (32, 2560, 25600), (128, 1280, 5120)])
+def test_w_static_prefetch_parity(M, N, K):
+    X, W = inputs.linear_pair(M, N, K, seed=M + 11)
+    y, y_ref, a_ref, _, _ = run_gemm(X, W, True, sp24.SPARSE, False, flags=sp24.GEMM_W_STATIC)
+    check_tolerance(y, y_ref, a_ref, "w_static")
 
 
 @pytest.mark.parametrize("M", [1, 16, 200])
