@@ -189,12 +189,14 @@ typedef struct sp24_gemm_args {
 
 /* Bytes of workspace the call would use for its stream-K schedule (0 if the
  * shape needs none).  Shapes with fewer than two output tiles per SM split
- * the tiles' K range evenly over all SMs and sum the partials in a fixed
- * order; with a smaller or missing workspace the call falls back to whole
- * tiles per CTA (same results up to fp32 summation order, fewer SMs busy).
- * The workspace must be zero-filled once before its first use; every call
- * that returns SP24_OK leaves its counter words at zero again.  Calls that
- * share a workspace must not overlap on the GPU. */
+ * the tiles' K range evenly over all SMs; the parts of a split tile are added
+ * with fp32 atomics into a per-tile accumulator in the workspace, so their
+ * fp32 summation order (and the last bits of those outputs) can vary from
+ * run to run.  With a smaller or missing workspace the call falls back to
+ * whole tiles per CTA (fewer SMs busy on such shapes).  The workspace must
+ * be zero-filled once before its first use; every call that returns SP24_OK
+ * leaves it zero again.  Calls that share a workspace must not overlap on
+ * the GPU. */
 size_t sp24_gemm_workspace_bytes(const sp24_gemm_args *args);
 
 /* Y = s_x[m] * s_w[n] * sum_k x[m,k] * w[n,k] (scales only for E4M3), fp32

@@ -13,8 +13,12 @@
 // Work schedule.  "Data-parallel": each CTA takes whole output tiles
 // round-robin.  "Stream-K" (few tiles, e.g. decode): the tiles' K-iterations
 // are laid end to end and every CTA streams one equal contiguous range of
-// them, so every SM moves the same number of bytes; a tile split between CTAs
-// is summed by whichever contributor finishes last, in contributor order.
+// them, so every SM moves the same number of bytes.  The contributors of a
+// tile split between CTAs add their fp32 partial sums into one accumulator
+// tile with vector atomics (red.global.add.v4.f32, no waiting on the L2
+// round trip); the last one to take a ticket scales, converts and stores the
+// tile and zeroes the accumulator for the next call.  The fp32 addition
+// order of a split tile therefore varies between runs.
 //
 // Kernel chaining.  Every CTA triggers the dependent grid at once
 // (programmatic dependent launch).  With p.w_static the producer starts
@@ -47,7 +51,6 @@ struct GemmParams {
   int32_t num_kt;             // K-stages per tile
   int32_t tiles_a, tiles_b;
   int32_t sched;              // kSchedDataParallel / kSchedStreamK
-  int32_t maxseg;             // stream-K: partial slots per CTA
   int64_t total_iters;        // stream-K: tiles * num_kt
   int32_t out_f32;            // 1: fp32 output, 0: bf16
   int32_t use_pdl;            // wait on the upstream grid before dependent loads
@@ -58,7 +61,7 @@ struct GemmParams {
   const float* scale_b;       // per-B-row scale (E4M3) or null
   void* Y;
   int64_t ldy;
-  float* ws_partials;         // stream-K partials [grid][maxseg][128 rows][BN]
+  float* ws_accum;            // stream-K fp32 accumulators [tiles][128 rows][BN]
   unsigned int* ws_counters;  // stream-K arrival counters [tiles]
   uint64_t timeout_ns;
 };
@@ -111,8 +114,14 @@ __device__ __forceinline__ bool named_bar_red_and(int id, int count, bool pred) 
   return out != 0;
 }
 
+// fp32 vector atomic add (fire and forget).
+__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+
 // GPU-scope acquire-release fetch-add: publishes (with the preceding CTA
-// barrier) the CTA's partial stores and acquires the other contributors'.
+// barrier) the CTA's partial adds and acquires the other contributors'.
 __device__ __forceinline__ unsigned int atom_add_acq_rel_gpu(unsigned int* p, unsigned int v) {
   unsigned int old;
   asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
@@ -475,9 +484,8 @@ k_gemm(const __grid_constant__ CUtensorMap tm_a,      // A: dense [rows_a x K] o
       tc_fence_after_sync();
       const uint32_t tbase = tmem_base + ((uint32_t)(lg * 32) << 16) + buf * kBN;
       const bool full = (kb == 0 && ke == p.num_kt);
-      // stream-K partials: [cta][seg][row][kBN] fp32, each thread's row contiguous
-      float* part = full ? nullptr
-                         : p.ws_partials + (((int64_t)blockIdx.x * p.maxseg + seg) * 128 + row) * kBN;
+      // stream-K accumulator row of this thread: [tile][row][kBN] fp32
+      float* part = full ? nullptr : p.ws_accum + ((int64_t)tile * 128 + row) * kBN;
 
       // Scales and stores 16 consecutive accumulator columns starting at c0
       // with 16-byte vector stores.  Rows of Y are 16-byte aligned (checked
@@ -544,11 +552,10 @@ k_gemm(const __grid_constant__ CUtensorMap tm_a,      // A: dense [rows_a x K] o
         tmem_ld_x16(tbase + c0, r);
         tmem_ld_wait();
         if (part != nullptr) {
-          float4* q = reinterpret_cast<float4*>(part + c0);
 #pragma unroll
           for (int j = 0; j < 4; ++j)
-            __stcg(q + j, make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
-                                      __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3])));
+            red_add_v4(part + c0 + 4 * j, __uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                       __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
         } else {
           float v[16];
 #pragma unroll
@@ -562,35 +569,38 @@ k_gemm(const __grid_constant__ CUtensorMap tm_a,      // A: dense [rows_a x K] o
 
       if (part != nullptr) {
         // The contributors of this tile are the CTAs whose iteration ranges
-        // cover it; the last to arrive sums all partials in contributor order.
+        // cover it; the last to take a ticket finishes the tile.
         const int c_first = sk_owner(p, grid, (int64_t)tile * p.num_kt);
         const int c_last = sk_owner(p, grid, (int64_t)(tile + 1) * p.num_kt - 1);
         const unsigned int count = (unsigned int)(c_last - c_first + 1);
-        named_bar_sync(1, 128);  // every partial store of this CTA precedes the ticket
+        named_bar_sync(1, 128);  // every partial add of this CTA precedes the ticket
         if (et == 0) {
           const unsigned int old = atom_add_acq_rel_gpu(&p.ws_counters[tile], 1u);
           *last_flag = (old == count - 1) ? 1 : 0;
         }
         named_bar_sync(1, 128);
         if (*last_flag) {
+          // all loads of a 64-column block in flight at once, then store and
+          // zero the accumulator for the next call
+          constexpr int kFix = kBN < 64 ? kBN : 64;
 #pragma unroll 1
-          for (int c0 = 0; c0 < kBN; c0 += 16) {
-            float v[16];
+          for (int cb = 0; cb < kBN; cb += kFix) {
+            float4 q[kFix / 4];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) v[i] = 0.0f;
-            for (int c = c_first; c <= c_last; ++c) {
-              // the contributor's segment index for this tile
-              const int64_t it0 = (int64_t)c * p.total_iters / grid;
-              const int sj = tile - (int)(it0 / p.num_kt);
-              const float4* q = reinterpret_cast<const float4*>(
-                  p.ws_partials + (((int64_t)c * p.maxseg + sj) * 128 + row) * kBN + c0);
-              const float4 a0 = __ldcg(q), a1 = __ldcg(q + 1), a2 = __ldcg(q + 2), a3 = __ldcg(q + 3);
-              v[0] += a0.x; v[1] += a0.y; v[2] += a0.z; v[3] += a0.w;
-              v[4] += a1.x; v[5] += a1.y; v[6] += a1.z; v[7] += a1.w;
-              v[8] += a2.x; v[9] += a2.y; v[10] += a2.z; v[11] += a2.w;
-              v[12] += a3.x; v[13] += a3.y; v[14] += a3.z; v[15] += a3.w;
+            for (int j = 0; j < kFix / 4; ++j) q[j] = __ldcg(reinterpret_cast<const float4*>(part + cb) + j);
+#pragma unroll
+            for (int j = 0; j < kFix / 4; ++j)
+              __stcg(reinterpret_cast<float4*>(part + cb) + j, make_float4(0.f, 0.f, 0.f, 0.f));
+#pragma unroll
+            for (int c0 = 0; c0 < kFix; c0 += 16) {
+              float v[16];
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const float4 t = q[c0 / 4 + j];
+                v[4 * j] = t.x; v[4 * j + 1] = t.y; v[4 * j + 2] = t.z; v[4 * j + 3] = t.w;
+              }
+              store16(v, cb + c0);
             }
-            store16(v, c0);
           }
           if (et == 0) p.ws_counters[tile] = 0u;  // ready for the next call
         }

@@ -126,7 +126,6 @@ struct Plan {
   int num_kt, tiles_a, tiles_b;
   int sched;       // kSchedDataParallel / kSchedStreamK
   int grid;
-  int maxseg;      // stream-K partial slots per CTA
   int64_t total_iters;
   size_t ws_bytes;
 };
@@ -144,10 +143,13 @@ int stage_k(int mode, bool bf16) {
   return bf16 ? 64 : 128;
 }
 
+size_t sk_accum_bytes(const Plan& pl) {
+  return (size_t)pl.tiles_a * pl.tiles_b * pl.bn * 128 * sizeof(float);
+}
+
 size_t sk_ws_bytes(const Plan& pl) {
-  const size_t part = (size_t)pl.grid * pl.maxseg * pl.bn * 128 * sizeof(float);
   const size_t cnt = ((size_t)pl.tiles_a * pl.tiles_b * sizeof(unsigned int) + 255) & ~(size_t)255;
-  return part + cnt;
+  return sk_accum_bytes(pl) + cnt;
 }
 
 // Work schedule: with at least two tiles per SM the CTAs take whole tiles
@@ -159,14 +161,11 @@ void choose_schedule(Plan& pl, int sms, size_t ws_cap) {
   pl.total_iters = tiles * pl.num_kt;
   pl.sched = kSchedDataParallel;
   pl.grid = (int)std::min<int64_t>(tiles, sms);
-  pl.maxseg = 0;
   pl.ws_bytes = 0;
   if (tiles < 2 * (int64_t)sms && pl.num_kt > 1) {
     Plan t = pl;
     t.sched = kSchedStreamK;
     t.grid = (int)std::min<int64_t>(t.total_iters, sms);
-    const int64_t per_cta = (t.total_iters + t.grid - 1) / t.grid;
-    t.maxseg = (int)((per_cta + t.num_kt - 1) / t.num_kt) + 1;
     t.ws_bytes = sk_ws_bytes(t);
     if (t.ws_bytes <= ws_cap) pl = t;
   }
@@ -290,12 +289,10 @@ void fill_sched(GemmParams& p, const Plan& pl, void* workspace) {
   p.tiles_a = pl.tiles_a;
   p.tiles_b = pl.tiles_b;
   p.sched = pl.sched;
-  p.maxseg = pl.maxseg;
   p.total_iters = pl.total_iters;
   if (pl.sched == kSchedStreamK) {
-    p.ws_partials = static_cast<float*>(workspace);
-    p.ws_counters = reinterpret_cast<unsigned int*>(
-        static_cast<uint8_t*>(workspace) + (size_t)pl.grid * pl.maxseg * pl.bn * 128 * sizeof(float));
+    p.ws_accum = static_cast<float*>(workspace);
+    p.ws_counters = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(workspace) + sk_accum_bytes(pl));
   }
 }
 

@@ -208,9 +208,11 @@ def test_whole_tile_schedule_without_workspace(M, N, K, e4):
 
 
 @pytest.mark.parametrize("tactic", [sp24.SPARSE, sp24.DENSE])
-def test_stream_k_is_deterministic_and_reusable(tactic):
-    # three calls on one workspace: identical bits each time (fixed summation
-    # order) -- a counter left non-zero would break the second or third call
+def test_stream_k_workspace_is_reusable(tactic):
+    # three calls on one workspace: every call leaves the accumulators and
+    # counters zero, so each one is within tolerance on its own (a residue
+    # would add a whole partial sum); the split tiles' fp32 addition order may
+    # differ between calls, so they agree to fp32 rounding
     X, W = inputs.linear_pair(8, 1024, 4096, seed=77)
     y1, y_ref, a_ref, args, ws = run_gemm(X, W, True, tactic, True, flags=sp24.GEMM_W_STATIC)
     assert ws is not None  # this decode shape takes the stream-K schedule
@@ -220,7 +222,10 @@ def test_stream_k_is_deterministic_and_reusable(tactic):
         Y.zero_()
         sp24.gemm(args)
         torch.cuda.synchronize()
-        assert np.array_equal(Y.cpu().numpy(), y1.astype(np.float32))
+        y = Y.cpu().numpy().astype(np.float64)
+        check_tolerance(y, y_ref, a_ref, "stream-K repeat")
+        assert np.allclose(y, y1, rtol=1e-5, atol=1e-5 * np.abs(y1).max())
+    assert int(ws.view(torch.int32).abs().sum().item()) == 0  # accumulators and counters zero
 
 
 @pytest.mark.parametrize("M,N,K", [(1, 5120, 5120), (32, 2560, 25600), (128, 1280, 5120)])
