@@ -152,22 +152,30 @@ size_t sk_ws_bytes(const Plan& pl) {
   return sk_accum_bytes(pl) + cnt;
 }
 
-// Work schedule: with at least two tiles per SM the CTAs take whole tiles
-// round-robin; with fewer (the decode shapes) the tiles' K-iterations are
-// split evenly over the SMs (stream-K), which needs a workspace for the
-// partial sums.  Without enough workspace the whole-tile schedule is used.
+// Work schedule, from a cost model in units of one K-stage of one SM
+// (streaming one stage of weights takes about the same time on every SM
+// when all SMs stream):
+//   whole tiles round-robin: ceil(tiles / SMs) * stages per tile
+//   stream-K:                ceil(tiles * stages / SMs) + the cost of finishing
+//                            the split tiles (fp32 atomics into an accumulator,
+//                            then one pass over it), which grows with the tile
+//                            width BN: about 2 + BN^2 / 800 stage-equivalents.
+// Stream-K needs a workspace for the accumulators; without enough of it the
+// whole-tile schedule is used.
 void choose_schedule(Plan& pl, int sms, size_t ws_cap) {
   const int64_t tiles = (int64_t)pl.tiles_a * pl.tiles_b;
   pl.total_iters = tiles * pl.num_kt;
   pl.sched = kSchedDataParallel;
   pl.grid = (int)std::min<int64_t>(tiles, sms);
   pl.ws_bytes = 0;
-  if (tiles < 2 * (int64_t)sms && pl.num_kt > 1) {
+  if (pl.num_kt > 1 && tiles < 4 * (int64_t)sms) {
+    const double cost_dp = (double)((tiles + sms - 1) / sms) * pl.num_kt;
+    const double cost_sk = (double)((pl.total_iters + sms - 1) / sms) + 2.0 + pl.bn * pl.bn / 800.0;
     Plan t = pl;
     t.sched = kSchedStreamK;
     t.grid = (int)std::min<int64_t>(t.total_iters, sms);
     t.ws_bytes = sk_ws_bytes(t);
-    if (t.ws_bytes <= ws_cap) pl = t;
+    if (cost_sk < cost_dp && t.ws_bytes <= ws_cap) pl = t;
   }
 }
 
