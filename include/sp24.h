@@ -206,6 +206,28 @@ size_t sp24_gemm_workspace_bytes(const sp24_gemm_args *args);
  * (bf16) / K % 16 == 0 (e4m3); any M, N >= 1. */
 int sp24_gemm(const sp24_gemm_args *args, void *stream);
 
+/* The GEMM for callers that cannot allocate device memory: code that runs
+ * where cudaMalloc is unavailable or unwanted, for instance inside a stream
+ * capture that must not allocate, in an allocator-free runtime, or under a
+ * caller that owns every byte of device memory and has none to lend.  It
+ * behaves like sp24_gemm but takes its stream-K scratch from a fixed 8 MiB
+ * array inside this library (args->workspace and args->workspace_bytes are
+ * ignored) and never allocates or frees anything.
+ * Not from the pages: they have no counterpart; this is an operational
+ * variant of sp24_gemm.
+ *  - The first call on each device looks up the array's device address (with
+ *    that device current) and caches it; make that first call before any
+ *    stream capture.
+ *  - Shapes whose schedule needs more than sp24_gemm_noalloc_max_scratch_bytes()
+ *    of scratch return SP24_ERR_WORKSPACE.
+ *  - Every call clears the part of the array it uses (a memset on `stream`)
+ *    and shares the same array: calls that overlap on the GPU race with each
+ *    other (on one device, issue them on one stream or order them). */
+int sp24_gemm_noalloc(const sp24_gemm_args *args, void *stream);
+
+/* Size of the fixed scratch array sp24_gemm_noalloc draws on. */
+size_t sp24_gemm_noalloc_max_scratch_bytes(void);
+
 /* ---------------------------------------------------------------------- */
 /* Online activation prune + compress fused ahead of the GEMM (kernel 4)   */
 /* ---------------------------------------------------------------------- */

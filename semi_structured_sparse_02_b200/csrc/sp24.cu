@@ -367,6 +367,39 @@ int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cud
   return launch_result(cudaLaunchKernelEx(&cfg, kernel, args...));
 }
 
+// ---------------------------------------------------------------------------
+// Scratch for sp24_gemm_noalloc: a fixed device array in this library, so
+// that callers that must not allocate device memory still get the stream-K
+// schedule.  Every GPU that loads the library holds it until exit.
+// ---------------------------------------------------------------------------
+constexpr size_t kStaticScratchBytes = (size_t)8 << 20;  // 8 MiB
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+void* g_scratch_addr[kMaxDevices] = {};
+std::mutex g_scratch_mu;
+
+// The scratch array's device address on the current device.  In host code
+// the array's name is only a host-side stand-in, so the address is looked up
+// once per device, with that device current, and cached.
+int static_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return SP24_ERR_UNSUPPORTED_DEVICE;
+  }
+  std::lock_guard<std::mutex> lk(g_scratch_mu);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_static_scratch) != cudaSuccess || ptr == nullptr) {
+      cudaGetLastError();
+      return SP24_ERR_CUDA;
+    }
+    g_scratch_addr[dev] = ptr;
+  }
+  *out = g_scratch_addr[dev];
+  return SP24_OK;
+}
+
 }  // namespace
 }  // namespace sp24
 
@@ -485,6 +518,31 @@ int sp24_gemm(const sp24_gemm_args* a, void* stream) {
   if (st != SP24_OK) return st;
   return run_gemm(a, static_cast<cudaStream_t>(stream));
 }
+
+int sp24_gemm_noalloc(const sp24_gemm_args* a, void* stream) {
+  int st = validate_gemm(a);
+  if (st != SP24_OK) return st;
+  DeviceInfo di;
+  if ((st = current_device_info(&di)) != SP24_OK) return st;
+  // The same schedule sp24_gemm picks with an unlimited workspace.
+  const Plan pl = plan_gemm(a, di.sms, (size_t)-1);
+  if (pl.ws_bytes > kStaticScratchBytes) return SP24_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  if ((st = static_scratch(&scratch)) != SP24_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // the accumulators and counters must start at zero; the array keeps
+  // whatever the previous call on this device left in it
+  if (pl.ws_bytes > 0 && cudaMemsetAsync(scratch, 0, pl.ws_bytes, s) != cudaSuccess) {
+    cudaGetLastError();
+    return SP24_ERR_CUDA;
+  }
+  sp24_gemm_args b = *a;
+  b.workspace = scratch;
+  b.workspace_bytes = kStaticScratchBytes;
+  return run_gemm(&b, s);
+}
+
+size_t sp24_gemm_noalloc_max_scratch_bytes(void) { return kStaticScratchBytes; }
 
 size_t sp24_activations_workspace_bytes(int64_t M, int64_t K) {
   if (M < 1 || K < 128) return 0;

@@ -96,6 +96,8 @@ def lib() -> ctypes.CDLL:
         "sp24_quantize_e4m3_rows_grouped": (I, [ctypes.POINTER(QuantItem), I, P]),
         "sp24_gemm_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(GemmArgs)]),
         "sp24_gemm": (I, [ctypes.POINTER(GemmArgs), P]),
+        "sp24_gemm_noalloc": (I, [ctypes.POINTER(GemmArgs), P]),
+        "sp24_gemm_noalloc_max_scratch_bytes": (ctypes.c_size_t, []),
         "sp24_activations_workspace_bytes": (ctypes.c_size_t, [I64, I64]),
         "sp24_prune_compress_activations_fused": (I, [P, I64, I64, I64, P, I64, I64, P, I64, I,
                                                       P, P, P, ctypes.c_size_t, P]),
@@ -262,6 +264,16 @@ def gemm_workspace_bytes(args: GemmArgs) -> int:
 
 def gemm(args: GemmArgs, stream=None):
     _check(lib().sp24_gemm(ctypes.byref(args), _stream(stream)), "sp24_gemm")
+
+
+def gemm_noalloc(args: GemmArgs, stream=None):
+    """sp24_gemm without any device allocation: stream-K scratch comes from a
+    fixed array in the library (args.workspace is ignored)."""
+    _check(lib().sp24_gemm_noalloc(ctypes.byref(args), _stream(stream)), "sp24_gemm_noalloc")
+
+
+def gemm_noalloc_max_scratch_bytes() -> int:
+    return lib().sp24_gemm_noalloc_max_scratch_bytes()
 
 
 def activations_workspace_bytes(M: int, K: int) -> int:
