@@ -62,6 +62,27 @@ def gemm_bytes(M, N, K):
     return N * K // 2 + N * K // 8 + 4 * N + M * K + 4 * M + 2 * M * N
 
 
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_step_traffic.md")
+GEMM_SOURCE = os.path.join(ROOT, "semi_structured_sparse_02_b200", "csrc", "gemm.cuh")
+
+
+def recorded_traffic():
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary, if it was taken on the current GEMM source (else None)."""
+    import hashlib
+    import re
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    txt = open(TRAFFIC_FILE).read()
+    sha = re.search(r"gemm_source_sha256:\s*([0-9a-f]{64})", txt)
+    val = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", txt)
+    if not sha or not val:
+        return None
+    if hashlib.sha256(open(GEMM_SOURCE, "rb").read()).hexdigest() != sha.group(1):
+        return None
+    return int(val.group(1))
+
+
 def quant_bytes(M, K):
     return 2 * M * K + M * K + 4 * M
 
@@ -367,7 +388,7 @@ def run_product(args, rank, world, local_rank):
             "peak_source": peak_src,
             "unit": "GB/s",
             "frac": round(achieved / hbm_peak, 4),
-            "traffic": None,
+            "traffic": recorded_traffic(),
             "bytes_per_launch": int(bytes_per_launch),
             "us_per_launch": round(t_gemm_launch * 1e6, 3),
         },
