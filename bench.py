@@ -5,7 +5,9 @@ Workload (one step): for M in {1, 8, 32, 128} and (N, K) in {(5120,5120),
 (25600,5120), (5120,25600), (10240,5120)}: cast the bf16 activations X [M x K]
 to E4M3 per token, then Y [M x N] = X * W^T with W pruned 2:4 along K and
 stored as E4M3 values + metadata with one fp32 scale per output channel
-(16 independent GEMMs; the 16 casts run as one grouped launch: 17 launches).  W ~ N(0, 0.02^2), X ~ N(0, 1), seeded.
+(16 independent GEMMs).  The 16 casts run as one grouped launch and the 16
+GEMMs as three grouped launches, one per token-count class (M in {1, 8}, 32,
+128): 4 launches per step.  W ~ N(0, 0.02^2), X ~ N(0, 1), seeded.
 Each of the 16 GEMMs reads its own copy of W (852 MB of distinct weights per
 step, far above the 126 MB L2), so no weight is served from L2.
 
@@ -213,24 +215,35 @@ def run_product(args, rank, world, local_rank):
 
     stream = torch.cuda.Stream(device=dev)
     # the per-token e4m3 casts of the 16 independent activation matrices run
-    # as one grouped launch; then the 16 GEMMs (chained by programmatic
-    # dependent launch, each streaming its weights while the previous kernel
-    # drains)
+    # as one grouped launch; then the GEMMs run as grouped launches, one per
+    # (tactic, token-count class): M in {1, 8} share one, M = 32 and M = 128
+    # one each.  Launches are chained by programmatic dependent launch, each
+    # streaming its weights while the previous kernel drains.
     quant_all = sp24.QuantGroup([(it["X"], it["xq"], it["xs"]) for it in inst])
+
+    def make_groups(pick):
+        """Grouped launches for the tactic pick(it) of every GEMM."""
+        by = {}
+        for it in inst:
+            t = pick(it)
+            a = it["a_sp"] if t == "sparse" else it["a_dn"]
+            by.setdefault((t, sp24.m_class(it["M"])), []).append(a)
+        return [sp24.GemmGroup(v) for _, v in sorted(by.items())]
+
+    groups = {"sparse": make_groups(lambda it: "sparse"), "dense": make_groups(lambda it: "dense")}
 
     def step(kind):
         quant_all()
-        for it in inst:
-            if kind == "sparse":
+        if kind == "ungrouped":
+            for it in inst:
                 sp24.gemm(it["a_sp"])
-            elif kind == "dense":
-                sp24.gemm(it["a_dn"])
-            elif kind == "selected":
-                sp24.gemm(it["a_sp"] if it["tactic"] == "sparse" else it["a_dn"])
+            return
+        for grp in groups[kind]:
+            grp()
 
     def gemm_only():
-        for it in inst:
-            sp24.gemm(it["a_sp"])
+        for grp in groups["sparse"]:
+            grp()
 
     # tactic selection per GEMM (untimed), on the benchmark stream
     with torch.cuda.stream(stream):
@@ -244,16 +257,18 @@ def run_product(args, rank, world, local_rank):
     if args.manifest and rank == 0:
         with open(args.manifest, "w") as f:
             f.write(manifest.dumps(man))
+    groups["selected"] = make_groups(lambda it: it["tactic"])
 
     # eager warm-up (sets kernel attributes), then capture the graphs
+    kinds = ("sparse", "dense", "selected", "ungrouped", "gemm_only")
     with torch.cuda.stream(stream):
-        for kind in ("sparse", "dense", "selected"):
+        for kind in kinds[:-1]:
             step(kind)
         gemm_only()
     torch.cuda.synchronize()
     graphs = {}
     launches = {}
-    for kind in ("sparse", "dense", "selected", "gemm_only"):
+    for kind in kinds:
         g = torch.cuda.CUDAGraph()
         c0 = sp24.launch_count()
         with torch.cuda.graph(g, stream=stream):
@@ -311,6 +326,7 @@ def run_product(args, rank, world, local_rank):
     ms_dense = time_graph(graphs["dense"], K_steps, W_warm)
     ms_sel = time_graph(graphs["selected"], K_steps, W_warm)
     ms_gemm = time_graph(graphs["gemm_only"], K_steps, W_warm)
+    ms_ungrouped = time_graph(graphs["ungrouped"], K_steps, W_warm)
 
     # end to end through the public API: pinned host X in, host Y out, eager calls
     X_host = torch.empty(x_elems, dtype=torch.bfloat16, pin_memory=True)
@@ -342,8 +358,9 @@ def run_product(args, rank, world, local_rank):
     step_flops = sum(2.0 * M * N * K for M, N, K in gemms)
     t_step = ms_sparse / K_steps / 1e3
     value = replicas.aggregate_rate(step_bytes, t_step, world) / 1e9
-    t_gemm_launch = ms_gemm / K_steps / 1e3 / len(gemms)
-    bytes_per_launch = gemm_bytes_total / len(gemms)
+    n_gemm_launches = launches["gemm_only"]
+    t_gemm_launch = ms_gemm / K_steps / 1e3 / n_gemm_launches
+    bytes_per_launch = gemm_bytes_total / n_gemm_launches
     peaks_path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(peaks_path):
         peaks = json.load(open(peaks_path))
@@ -373,15 +390,18 @@ def run_product(args, rank, world, local_rank):
             "parallelism": "replicas" if world > 1 else "single-gpu",
             "l2": L2_NOTE,
             "timing": "CUDA graph of one step replayed K times; CUDA events on the replay stream",
-            "step": "one grouped per-token e4m3 cast of the 16 activation matrices, then 16 GEMMs",
+            "step": ("one grouped per-token e4m3 cast of the 16 activation matrices, then the 16 "
+                     "GEMMs as %d grouped launches (one per token-count class: M in {1,8}, 32, 128)"
+                     % len(groups["sparse"])),
         },
         "tflops": round(world * step_flops / t_step / 1e12, 3),
         "speedup_vs_dense": round(ms_dense / ms_sparse, 4),
         "ms_per_step_dense": round(ms_dense / K_steps, 5),
         "ms_per_step_selected": round(ms_sel / K_steps, 5),
+        "ms_per_step_ungrouped": round(ms_ungrouped / K_steps, 5),
         "tactics": man["metrics"],
         "roofline": {
-            "kernel": "k_gemm sparse e4m3 (tcgen05.mma.sp)",
+            "kernel": "k_gemm sparse e4m3 (tcgen05.mma.sp), grouped launch",
             "bound": "hbm",
             "achieved": round(achieved, 1),
             "peak": hbm_peak,
@@ -399,8 +419,9 @@ def run_product(args, rank, world, local_rank):
             "h2d_bytes_per_step": x_elems * 2,
             "d2h_bytes_per_step": y_elems * 2,
             "ms_per_step": round(ms_e2e / e2e_steps, 5),
-            "how": "eager public-API calls (one sp24_quantize_e4m3_rows_grouped + 16 sp24_gemm) "
-                   "with one pinned H2D copy of X and one D2H copy of Y per step",
+            "how": "eager public-API calls (one sp24_quantize_e4m3_rows_grouped + %d "
+                   "sp24_gemm_grouped) with one pinned H2D copy of X and one D2H copy of Y per step"
+                   % len(groups["sparse"]),
         },
         "gpu_launches": launches["sparse"] * K_steps,
     }

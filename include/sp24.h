@@ -206,6 +206,21 @@ size_t sp24_gemm_workspace_bytes(const sp24_gemm_args *args);
  * (bf16) / K % 16 == 0 (e4m3); any M, N >= 1. */
 int sp24_gemm(const sp24_gemm_args *args, void *stream);
 
+/* Up to 16 independent GEMMs in one persistent launch (a grouped GEMM: the
+ * projections that share an input, experts, or any batch of independent
+ * problems).  Same results as sp24_gemm on each.  The work of all problems
+ * is scheduled together, so the weights of the whole group stream without a
+ * launch, ramp or tail between problems.  All problems must share in_dtype,
+ * out_dtype and tactic, use no hybrid mask, and have M in the same class
+ * (1-16, 17-32, 33-64, >64); otherwise SP24_ERR_INVALID_ARG.  Each args'
+ * own workspace fields are ignored: the group uses `workspace` (size from
+ * sp24_gemm_grouped_workspace_bytes, same zero-fill rule as sp24_gemm).
+ * SP24_GEMM_W_STATIC applies when every problem sets it. */
+int sp24_gemm_grouped(const sp24_gemm_args *args, int n, void *workspace_dev, size_t workspace_bytes,
+                      void *stream);
+
+size_t sp24_gemm_grouped_workspace_bytes(const sp24_gemm_args *args, int n);
+
 /* The GEMM for callers that cannot allocate device memory: code that runs
  * where cudaMalloc is unavailable or unwanted, for instance inside a stream
  * capture that must not allocate, in an allocator-free runtime, or under a

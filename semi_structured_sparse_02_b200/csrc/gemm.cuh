@@ -1,6 +1,7 @@
 // gemm.cuh -- kernels 2 and 3: persistent, warp-specialized tcgen05 GEMM for
 // sm_100a.  One template covers the dense MMA, the 2:4 sparse MMA
-// (tcgen05.mma.sp, metadata in tensor memory) and the hybrid tile mix.
+// (tcgen05.mma.sp, metadata in tensor memory) and the hybrid tile mix, for
+// one problem or a group of up to kMaxGroup independent problems.
 //
 //   warp 0       TMA producer: A tile, B tile(s) and metadata chunk(s) of each
 //                K-stage into a STAGES-deep shared-memory ring (mbarriers).
@@ -8,20 +9,21 @@
 //                shared -> tensor memory) and tcgen05.mma into one of two fp32
 //                accumulators in tensor memory, then tcgen05.commit.
 //   warps 2..5   epilogue: tcgen05.ld of the accumulator, scales, output
-//                store; or a stream-K partial store + last-arriver reduction.
+//                store; or a stream-K partial add + last-arriver finish.
 //
 // Work schedule.  "Data-parallel": each CTA takes whole output tiles
-// round-robin.  "Stream-K" (few tiles, e.g. decode): the tiles' K-iterations
-// are laid end to end and every CTA streams one equal contiguous range of
-// them, so every SM moves the same number of bytes.  The contributors of a
-// tile split between CTAs add their fp32 partial sums into one accumulator
-// tile with vector atomics (red.global.add.v4.f32, no waiting on the L2
-// round trip); the last one to take a ticket scales, converts and stores the
-// tile and zeroes the accumulator for the next call.  The fp32 addition
-// order of a split tile therefore varies between runs.
+// round-robin over the tiles of all problems.  "Stream-K" (few tiles, e.g.
+// decode): the K-iterations of all tiles of all problems are laid end to end
+// and every CTA streams one equal contiguous range of them, so every SM moves
+// the same number of bytes and a group streams without gaps between problems.
+// The contributors of a tile split between CTAs add their fp32 partial sums
+// into one accumulator tile with vector atomics (red.global.add.v4.f32, no
+// waiting on the L2 round trip); the last one to take a ticket scales,
+// converts and stores the tile and zeroes the accumulator for the next call.
+// The fp32 addition order of a split tile therefore varies between runs.
 //
 // Kernel chaining.  Every CTA triggers the dependent grid at once
-// (programmatic dependent launch).  With p.w_static the producer starts
+// (programmatic dependent launch).  With w_static the producer starts
 // streaming the A operand (weights + metadata) before waiting on the
 // upstream grid; everything the upstream grid may write (B, scales of B,
 // the output) is touched only after griddepcontrol.wait.
@@ -44,17 +46,17 @@ enum GemmSched : int { kSchedDataParallel = 0, kSchedStreamK = 1 };
 
 constexpr int kGemmThreads = 192;
 constexpr int kBlockA = 128;  // MMA M: rows of A per tile
+constexpr int kMaxGroup = 16; // problems per grouped launch
 
-struct GemmParams {
+// One problem of a (possibly grouped) launch.
+struct GemmProblem {
   int32_t rows_a, rows_b;     // A rows (tile_a dim), B rows (tile_b dim)
   int32_t K;                  // logical reduction length
   int32_t num_kt;             // K-stages per tile
   int32_t tiles_a, tiles_b;
-  int32_t sched;              // kSchedDataParallel / kSchedStreamK
-  int64_t total_iters;        // stream-K: tiles * num_kt
-  int32_t out_f32;            // 1: fp32 output, 0: bf16
-  int32_t use_pdl;            // wait on the upstream grid before dependent loads
-  int32_t w_static;           // A operand is not written by the upstream grid
+  int32_t tile_begin;         // first global tile index of this problem
+  int32_t pad0;
+  int64_t iter_begin;         // first global stream-K iteration of this problem
   const uint8_t* meta;        // metadata image of A (sparse / hybrid)
   const uint8_t* tile_mask;   // hybrid: [tiles_a x K/128]
   const float* scale_a;       // per-A-row scale (E4M3) or null
@@ -63,7 +65,28 @@ struct GemmParams {
   int64_t ldy;
   float* ws_accum;            // stream-K fp32 accumulators [tiles][128 rows][BN]
   unsigned int* ws_counters;  // stream-K arrival counters [tiles]
+};
+
+struct GemmParams {
+  int32_t n_prob;
+  int32_t sched;              // kSchedDataParallel / kSchedStreamK
+  int64_t total_iters;        // stream-K: sum over problems of tiles * num_kt
+  int32_t total_tiles;        // sum over problems of tiles
+  int32_t out_f32;            // 1: fp32 output, 0: bf16
+  int32_t use_pdl;            // wait on the upstream grid before dependent loads
+  int32_t w_static;           // A operands are not written by the upstream grid
   uint64_t timeout_ns;
+};
+
+// Everything a launch needs, passed by value (tensor maps must live in
+// parameter, constant or global memory for TMA).
+template <int kMaxProb>
+struct GemmLaunch {
+  CUtensorMap tm_a[kMaxProb];   // A: dense [rows_a x K] or values [rows_a x K/2]
+  CUtensorMap tm_a2[kMaxProb];  // hybrid: values map (64-byte swizzle)
+  CUtensorMap tm_b[kMaxProb];   // B: [rows_b x K]
+  GemmProblem prob[kMaxProb];
+  GemmParams p;
 };
 
 // Compile-time geometry of one configuration.
@@ -129,55 +152,61 @@ __device__ __forceinline__ unsigned int atom_add_acq_rel_gpu(unsigned int* p, un
 }
 
 // ---------------------------------------------------------------------------
-// Work segments: a (tile, k-begin, k-end) range; j numbers the segments of
-// one CTA.  Every role of a CTA walks the same sequence.
+// Work segments: a (problem, tile, k-begin, k-end) range; seg numbers the
+// segments of one CTA.  Every role of a CTA walks the same sequence.
 // ---------------------------------------------------------------------------
+template <int kMaxProb>
 struct SegIter {
-  int64_t it, it1;    // stream-K iteration cursor and end
-  int tile_dp;        // data-parallel tile cursor
+  int64_t it, it1;    // stream-K global iteration cursor and end
+  int tile_g;         // data-parallel global tile cursor
+  int pr;             // problem cursor (only moves forward)
   int j;
-  __device__ __forceinline__ void init(const GemmParams& p, int cta, int grid) {
+  __device__ __forceinline__ void init(const GemmLaunch<kMaxProb>& g, int cta, int grid) {
     j = 0;
-    if (p.sched == kSchedStreamK) {
-      it = (int64_t)cta * p.total_iters / grid;
-      it1 = (int64_t)(cta + 1) * p.total_iters / grid;
+    pr = 0;
+    if (g.p.sched == kSchedStreamK) {
+      it = (int64_t)cta * g.p.total_iters / grid;
+      it1 = (int64_t)(cta + 1) * g.p.total_iters / grid;
     } else {
-      tile_dp = cta;
+      tile_g = cta;
     }
   }
-  __device__ __forceinline__ bool next(const GemmParams& p, int grid, int& tile, int& kb, int& ke,
-                                       int& seg) {
-    if (p.sched == kSchedStreamK) {
+  __device__ __forceinline__ bool next(const GemmLaunch<kMaxProb>& g, int grid, int& prob, int& tile,
+                                       int& kb, int& ke, int& seg) {
+    if (g.p.sched == kSchedStreamK) {
       if (it >= it1) return false;
-      tile = (int)(it / p.num_kt);
-      kb = (int)(it - (int64_t)tile * p.num_kt);
-      ke = (int)min((int64_t)p.num_kt, (int64_t)kb + (it1 - it));
+      while (pr + 1 < g.p.n_prob && it >= g.prob[pr + 1].iter_begin) ++pr;
+      const GemmProblem& P = g.prob[pr];
+      const int64_t local = it - P.iter_begin;
+      tile = (int)(local / P.num_kt);
+      kb = (int)(local - (int64_t)tile * P.num_kt);
+      ke = (int)min((int64_t)P.num_kt, (int64_t)kb + (it1 - it));
       it += ke - kb;
     } else {
-      if (tile_dp >= p.tiles_a * p.tiles_b) return false;
-      tile = tile_dp;
+      if (tile_g >= g.p.total_tiles) return false;
+      while (pr + 1 < g.p.n_prob && tile_g >= g.prob[pr + 1].tile_begin) ++pr;
+      tile = tile_g - g.prob[pr].tile_begin;
       kb = 0;
-      ke = p.num_kt;
-      tile_dp += grid;
+      ke = g.prob[pr].num_kt;
+      tile_g += grid;
     }
+    prob = pr;
     seg = j++;
     return true;
   }
 };
 
-// The CTA whose stream-K range holds iteration i.
-__device__ __forceinline__ int sk_owner(const GemmParams& p, int grid, int64_t i) {
-  return (int)(((i + 1) * grid - 1) / p.total_iters);
+// The CTA whose stream-K range holds global iteration i.
+__device__ __forceinline__ int sk_owner(int64_t total_iters, int grid, int64_t i) {
+  return (int)(((i + 1) * grid - 1) / total_iters);
 }
 
-template <int kMode, bool kBf16, int kBN, bool kAIsW>
+template <int kMode, bool kBf16, int kBN, bool kAIsW, int kMaxProb>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-k_gemm(const __grid_constant__ CUtensorMap tm_a,      // A: dense [rows_a x K] or values [rows_a x K/2]
-       const __grid_constant__ CUtensorMap tm_a2,     // hybrid: values map (64-byte swizzle)
-       const __grid_constant__ CUtensorMap tm_b,      // B: [rows_b x K]
-       const GemmParams p) {
+k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
   using C = GemmCfg<kMode, kBf16, kBN>;
   constexpr int S = C::kStages;
+  const GemmParams& p = g.p;
 
   // the next kernel in the stream may launch now; it waits for our completion
   // (griddepcontrol.wait) before it reads anything we write
@@ -218,9 +247,6 @@ k_gemm(const __grid_constant__ CUtensorMap tm_a,      // A: dense [rows_a x K] o
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
-    tma_prefetch_desc(&tm_a);
-    tma_prefetch_desc(&tm_b);
-    if (C::kHybrid) tma_prefetch_desc(&tm_a2);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
@@ -231,8 +257,12 @@ k_gemm(const __grid_constant__ CUtensorMap tm_a,      // A: dense [rows_a x K] o
   tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
 
-  auto is_dense_tile = [&](int ta, int kt) -> bool {
-    return p.tile_mask[(int64_t)ta * p.num_kt + kt] != 0;
+  auto is_dense_tile = [&](const GemmProblem& P, int ta, int kt) -> bool {
+    return P.tile_mask[(int64_t)ta * P.num_kt + kt] != 0;
+  };
+  // metadata chunks (128 K positions each) of stage kt of problem P
+  auto meta_chunks = [&](const GemmProblem& P, int kt) -> int {
+    return (int)min((int64_t)C::kMetaChunks, (int64_t)(P.K / 128) - (int64_t)kt * C::kMetaChunks);
   };
 
   if (warp == 0) {
@@ -243,68 +273,71 @@ k_gemm(const __grid_constant__ CUtensorMap tm_a,      // A: dense [rows_a x K] o
       int armed[S];
       for (int s = 0; s < S; ++s) armed[s] = -1;
 
-      // the A-operand (and metadata) part of one stage; returns its bytes
-      auto load_a = [&](int stage, int ta, int kt, bool arm_only_a) -> void {
-        (void)arm_only_a;
+      // the A-operand (and metadata) part of one stage
+      auto load_a = [&](int stage, int pr, int ta, int kt) {
+        const GemmProblem& P = g.prob[pr];
         const uint32_t sa = smem_u32(smem + stage * C::kStageBytes);
         const uint32_t sm = sa + C::kABytes + C::kBBytes;
         const int32_t ya = ta * kBlockA;
         if (C::kHybrid) {
-          if (is_dense_tile(ta, kt)) {
-            tma_load_2d(sa, &tm_a, full_bar(stage), kt * 128, ya, pol_stream);
+          if (is_dense_tile(P, ta, kt)) {
+            tma_load_2d(sa, &g.tm_a[pr], full_bar(stage), kt * 128, ya, pol_stream);
           } else {
-            tma_load_2d(sa, &tm_a2, full_bar(stage), kt * 64, ya, pol_stream);
-            bulk_load(sm, p.meta + ((int64_t)ta * p.num_kt + kt) * 2048, 2048, full_bar(stage),
+            tma_load_2d(sa, &g.tm_a2[pr], full_bar(stage), kt * 64, ya, pol_stream);
+            bulk_load(sm, P.meta + ((int64_t)ta * P.num_kt + kt) * 2048, 2048, full_bar(stage),
                       pol_stream);
           }
         } else {
           const int ax = C::kSparse ? kt * (C::kKT / 2) : kt * C::kKT;  // elements
-          tma_load_2d(sa, &tm_a, full_bar(stage), ax, ya, pol_stream);
+          tma_load_2d(sa, &g.tm_a[pr], full_bar(stage), ax, ya, pol_stream);
           if (C::kSparse) {
-            const int64_t kc_total = p.K / 128;
-            const int chunks = (int)min((int64_t)C::kMetaChunks, kc_total - (int64_t)kt * C::kMetaChunks);
-            const uint8_t* src = p.meta + ((int64_t)ta * kc_total + (int64_t)kt * C::kMetaChunks) * 2048;
-            bulk_load(sm, src, chunks * 2048, full_bar(stage), pol_stream);
+            const int64_t kc_total = P.K / 128;
+            const uint8_t* src = P.meta + ((int64_t)ta * kc_total + (int64_t)kt * C::kMetaChunks) * 2048;
+            bulk_load(sm, src, meta_chunks(P, kt) * 2048, full_bar(stage), pol_stream);
           }
         }
       };
-      auto load_b = [&](int stage, int tb, int kt) {
+      auto load_b = [&](int stage, int pr, int tb, int kt) {
         const uint32_t sb = smem_u32(smem + stage * C::kStageBytes) + C::kABytes;
         const int32_t yb = tb * kBN;
         if (C::kHybrid) {
-          tma_load_2d(sb, &tm_b, full_bar(stage), kt * 128, yb, pol_keep);
+          tma_load_2d(sb, &g.tm_b[pr], full_bar(stage), kt * 128, yb, pol_keep);
         } else {
           const int box_elems = kBf16 ? 64 : 128;
 #pragma unroll
           for (int bx = 0; bx < C::kBBoxes; ++bx)
-            tma_load_2d(sb + bx * kBN * 128, &tm_b, full_bar(stage), kt * C::kKT + bx * box_elems, yb,
-                        pol_keep);
+            tma_load_2d(sb + bx * kBN * 128, &g.tm_b[pr], full_bar(stage), kt * C::kKT + bx * box_elems,
+                        yb, pol_keep);
         }
       };
-      auto stage_bytes = [&](int ta, int kt) -> uint32_t {
+      auto stage_bytes = [&](int pr, int ta, int kt) -> uint32_t {
+        const GemmProblem& P = g.prob[pr];
         if (C::kHybrid)
-          return is_dense_tile(ta, kt) ? (uint32_t)(C::kABytes + kBN * 128)
-                                       : (uint32_t)(kBlockA * 64 + kBN * 128 + 2048);
+          return is_dense_tile(P, ta, kt) ? (uint32_t)(C::kABytes + kBN * 128)
+                                          : (uint32_t)(kBlockA * 64 + kBN * 128 + 2048);
         uint32_t b = C::kABytes + C::kBBytes;
-        if (C::kSparse) {
-          const int64_t kc_total = p.K / 128;
-          b += (uint32_t)min((int64_t)C::kMetaChunks, kc_total - (int64_t)kt * C::kMetaChunks) * 2048;
-        }
+        if (C::kSparse) b += (uint32_t)meta_chunks(P, kt) * 2048;
         return b;
       };
 
       // 1. weights first: arm the first S stages and start their A loads
       //    before the dependency wait when A is known not to be in flux
       int pre = 0;
+      int last_pr = -1;
       if (p.w_static) {
-        SegIter it;
-        it.init(p, blockIdx.x, grid);
-        int tile, kb, ke, seg;
-        while (pre < S && it.next(p, grid, tile, kb, ke, seg)) {
-          const int ta = tile % p.tiles_a;
+        SegIter<kMaxProb> it;
+        it.init(g, blockIdx.x, grid);
+        int pr, tile, kb, ke, seg;
+        while (pre < S && it.next(g, grid, pr, tile, kb, ke, seg)) {
+          if (pr != last_pr) {
+            tma_prefetch_desc(&g.tm_a[pr]);
+            if (C::kHybrid) tma_prefetch_desc(&g.tm_a2[pr]);
+            last_pr = pr;
+          }
+          const int ta = tile % g.prob[pr].tiles_a;
           for (int kt = kb; kt < ke && pre < S; ++kt, ++pre) {
-            mbar_arrive_expect_tx(full_bar(pre), stage_bytes(ta, kt));
-            load_a(pre, ta, kt, true);
+            mbar_arrive_expect_tx(full_bar(pre), stage_bytes(pr, ta, kt));
+            load_a(pre, pr, ta, kt);
             armed[pre] = 0;
           }
         }
@@ -316,23 +349,30 @@ k_gemm(const __grid_constant__ CUtensorMap tm_a,      // A: dense [rows_a x K] o
       uint32_t phase = 0;
       int n = 0;
       bool ok = true;
-      SegIter it;
-      it.init(p, blockIdx.x, grid);
-      int tile, kb, ke, seg;
-      while (ok && it.next(p, grid, tile, kb, ke, seg)) {
-        const int ta = tile % p.tiles_a, tb = tile / p.tiles_a;
+      last_pr = -1;
+      SegIter<kMaxProb> it;
+      it.init(g, blockIdx.x, grid);
+      int pr, tile, kb, ke, seg;
+      while (ok && it.next(g, grid, pr, tile, kb, ke, seg)) {
+        if (pr != last_pr) {
+          tma_prefetch_desc(&g.tm_a[pr]);
+          tma_prefetch_desc(&g.tm_b[pr]);
+          if (C::kHybrid) tma_prefetch_desc(&g.tm_a2[pr]);
+          last_pr = pr;
+        }
+        const int ta = tile % g.prob[pr].tiles_a, tb = tile / g.prob[pr].tiles_a;
         for (int kt = kb; kt < ke; ++kt, ++n) {
           if (n < pre) {
-            load_b(stage, tb, kt);  // A already in flight
+            load_b(stage, pr, tb, kt);  // A already in flight
           } else {
             if (!mbar_wait(empty_bar(stage), phase ^ 1, p.timeout_ns, kDevErrWaitEmpty)) {
               ok = false;
               *abort_flag = 1;
               break;
             }
-            mbar_arrive_expect_tx(full_bar(stage), stage_bytes(ta, kt));
-            load_a(stage, ta, kt, false);
-            load_b(stage, tb, kt);
+            mbar_arrive_expect_tx(full_bar(stage), stage_bytes(pr, ta, kt));
+            load_a(stage, pr, ta, kt);
+            load_b(stage, pr, tb, kt);
             armed[stage] = (int)phase;
           }
           if (++stage == S) {
@@ -357,11 +397,12 @@ k_gemm(const __grid_constant__ CUtensorMap tm_a,      // A: dense [rows_a x K] o
       uint32_t phase = 0;
       uint32_t acc_i = 0;
       bool ok = true;
-      SegIter it;
-      it.init(p, blockIdx.x, grid);
-      int tile, kb, ke, seg;
-      while (ok && it.next(p, grid, tile, kb, ke, seg)) {
-        const int ta = tile % p.tiles_a;
+      SegIter<kMaxProb> it;
+      it.init(g, blockIdx.x, grid);
+      int pr, tile, kb, ke, seg;
+      while (ok && it.next(g, grid, pr, tile, kb, ke, seg)) {
+        const GemmProblem& P = g.prob[pr];
+        const int ta = tile % P.tiles_a;
         const int buf = acc_i & 1;
         const uint32_t acc_phase = (acc_i >> 1) & 1;
         if (!mbar_wait(acce_bar(buf), acc_phase ^ 1, p.timeout_ns, kDevErrWaitAccEmpty)) {
@@ -384,7 +425,7 @@ k_gemm(const __grid_constant__ CUtensorMap tm_a,      // A: dense [rows_a x K] o
           const uint32_t mcol = meta_col0 + stage * C::kMetaCols;
           const bool first = kt == kb;
           if (C::kHybrid) {
-            if (is_dense_tile(ta, kt)) {
+            if (is_dense_tile(P, ta, kt)) {
 #pragma unroll
               for (int j = 0; j < 4; ++j) {
                 const uint64_t da = smem_desc(sa + j * 32, 16, 1024, kLayoutSw128);
@@ -401,8 +442,7 @@ k_gemm(const __grid_constant__ CUtensorMap tm_a,      // A: dense [rows_a x K] o
               }
             }
           } else if (C::kSparse) {
-            const int kc_total = p.K / 128;
-            const int chunks = min(C::kMetaChunks, kc_total - kt * C::kMetaChunks);
+            const int chunks = meta_chunks(P, kt);
             for (int c = 0; c < chunks; ++c)
               tc_cp_128x128b(tmem_base + mcol + 4 * c, smem_desc(sm + c * 2048, 16, 128, kLayoutNone));
             const int n_mma = kBf16 ? 4 : 2 * chunks;
@@ -453,25 +493,30 @@ k_gemm(const __grid_constant__ CUtensorMap tm_a,      // A: dense [rows_a x K] o
     const int row = lg * 32 + lane;            // accumulator row (lane) within the tile
     const int et = threadIdx.x - 64;           // 0..127
     uint32_t acc_i = 0;
-    int cached_tb = -1;
-    SegIter it;
-    it.init(p, blockIdx.x, grid);
-    int tile, kb, ke, seg;
-    while (it.next(p, grid, tile, kb, ke, seg)) {
-      const int ta = tile % p.tiles_a, tb = tile / p.tiles_a;
+    int cached_pr = -1, cached_tb = -1;
+    uint8_t* wtile = s_epi + (warp - 2) * 2048;  // this warp's staging tile
+    const int eb = p.out_f32 ? 4 : 2;
+    const int per_vec = 16 / eb;                   // elements per 16-byte vector
+    SegIter<kMaxProb> it;
+    it.init(g, blockIdx.x, grid);
+    int pr, tile, kb, ke, seg;
+    while (it.next(g, grid, pr, tile, kb, ke, seg)) {
+      const GemmProblem& P = g.prob[pr];
+      const int ta = tile % P.tiles_a, tb = tile / P.tiles_a;
       const int buf = acc_i & 1;
       const uint32_t acc_phase = (acc_i >> 1) & 1;
       const int ga = ta * kBlockA + row;     // global A row of this thread
-      const bool a_live = ga < p.rows_a;
+      const bool a_live = ga < P.rows_a;
       // scales: loaded before waiting for the accumulator so their latency hides
-      const float sa_v = (p.scale_a != nullptr && a_live) ? __ldg(p.scale_a + ga) : 1.0f;
-      if (tb != cached_tb) {
+      const float sa_v = (P.scale_a != nullptr && a_live) ? __ldg(P.scale_a + ga) : 1.0f;
+      if (pr != cached_pr || tb != cached_tb) {
         named_bar_sync(1, 128);
         for (int i = et; i < kBN; i += 128) {
           const int gb = tb * kBN + i;
-          s_scale_b[i] = (p.scale_b != nullptr && gb < p.rows_b) ? p.scale_b[gb] : 1.0f;
+          s_scale_b[i] = (P.scale_b != nullptr && gb < P.rows_b) ? P.scale_b[gb] : 1.0f;
         }
         named_bar_sync(1, 128);
+        cached_pr = pr;
         cached_tb = tb;
       }
       bool ok = mbar_wait(accf_bar(buf), acc_phase, p.timeout_ns, kDevErrWaitAccFull);
@@ -483,17 +528,14 @@ k_gemm(const __grid_constant__ CUtensorMap tm_a,      // A: dense [rows_a x K] o
       }
       tc_fence_after_sync();
       const uint32_t tbase = tmem_base + ((uint32_t)(lg * 32) << 16) + buf * kBN;
-      const bool full = (kb == 0 && ke == p.num_kt);
+      const bool full = (kb == 0 && ke == P.num_kt);
       // stream-K accumulator row of this thread: [tile][row][kBN] fp32
-      float* part = full ? nullptr : p.ws_accum + ((int64_t)tile * 128 + row) * kBN;
+      float* part = full ? nullptr : P.ws_accum + ((int64_t)tile * 128 + row) * kBN;
 
       // Scales and stores 16 consecutive accumulator columns starting at c0
       // with 16-byte vector stores.  Rows of Y are 16-byte aligned (checked
       // on the host); a vector that crosses the end of a row is stored per
       // element.
-      uint8_t* wtile = s_epi + (warp - 2) * 2048;  // this warp's staging tile
-      const int eb = p.out_f32 ? 4 : 2;
-      const int per_vec = 16 / eb;                   // elements per 16-byte vector
       auto store16 = [&](const float (&v)[16], int c0) {
         const int gb0 = tb * kBN + c0;
         if (kAIsW) {
@@ -513,13 +555,13 @@ k_gemm(const __grid_constant__ CUtensorMap tm_a,      // A: dense [rows_a x K] o
             const int i = q / vec_per_row, sg = q - i * vec_per_row;
             const int m = gb0 + i;
             const int n = n0 + sg * per_vec;
-            if (m >= p.rows_b || n >= p.rows_a) continue;
-            uint8_t* dst = static_cast<uint8_t*>(p.Y) + ((int64_t)m * p.ldy + n) * eb;
+            if (m >= P.rows_b || n >= P.rows_a) continue;
+            uint8_t* dst = static_cast<uint8_t*>(P.Y) + ((int64_t)m * P.ldy + n) * eb;
             const uint8_t* src = wtile + (i * 32 + sg * per_vec) * eb;
-            if (n + per_vec <= p.rows_a) {
+            if (n + per_vec <= P.rows_a) {
               *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
             } else {
-              for (int e = 0; e < p.rows_a - n; ++e)
+              for (int e = 0; e < P.rows_a - n; ++e)
                 for (int b = 0; b < eb; ++b) dst[e * eb + b] = src[e * eb + b];
             }
           }
@@ -528,20 +570,20 @@ k_gemm(const __grid_constant__ CUtensorMap tm_a,      // A: dense [rows_a x K] o
           // lane = m (token), column = n (output feature): this thread's 16
           // consecutive n of row ga
           if (!a_live) return;
-          alignas(16) uint8_t buf[64];
+          alignas(16) uint8_t vbuf[64];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const float y = v[i] * sa_v * s_scale_b[c0 + i];
-            if (p.out_f32) reinterpret_cast<float*>(buf)[i] = y;
-            else reinterpret_cast<__nv_bfloat16*>(buf)[i] = __float2bfloat16_rn(y);
+            if (p.out_f32) reinterpret_cast<float*>(vbuf)[i] = y;
+            else reinterpret_cast<__nv_bfloat16*>(vbuf)[i] = __float2bfloat16_rn(y);
           }
-          uint8_t* dst = static_cast<uint8_t*>(p.Y) + ((int64_t)ga * p.ldy + gb0) * eb;
-          if (gb0 + 16 <= p.rows_b) {
+          uint8_t* dst = static_cast<uint8_t*>(P.Y) + ((int64_t)ga * P.ldy + gb0) * eb;
+          if (gb0 + 16 <= P.rows_b) {
             for (int q = 0; q < 16 / per_vec; ++q)
-              reinterpret_cast<uint4*>(dst)[q] = reinterpret_cast<const uint4*>(buf)[q];
+              reinterpret_cast<uint4*>(dst)[q] = reinterpret_cast<const uint4*>(vbuf)[q];
           } else {
-            for (int e = 0; e < p.rows_b - gb0; ++e)
-              for (int b = 0; b < eb; ++b) dst[e * eb + b] = buf[e * eb + b];
+            for (int e = 0; e < P.rows_b - gb0; ++e)
+              for (int b = 0; b < eb; ++b) dst[e * eb + b] = vbuf[e * eb + b];
           }
         }
       };
@@ -570,12 +612,13 @@ k_gemm(const __grid_constant__ CUtensorMap tm_a,      // A: dense [rows_a x K] o
       if (part != nullptr) {
         // The contributors of this tile are the CTAs whose iteration ranges
         // cover it; the last to take a ticket finishes the tile.
-        const int c_first = sk_owner(p, grid, (int64_t)tile * p.num_kt);
-        const int c_last = sk_owner(p, grid, (int64_t)(tile + 1) * p.num_kt - 1);
+        const int64_t i0 = P.iter_begin + (int64_t)tile * P.num_kt;
+        const int c_first = sk_owner(p.total_iters, grid, i0);
+        const int c_last = sk_owner(p.total_iters, grid, i0 + P.num_kt - 1);
         const unsigned int count = (unsigned int)(c_last - c_first + 1);
         named_bar_sync(1, 128);  // every partial add of this CTA precedes the ticket
         if (et == 0) {
-          const unsigned int old = atom_add_acq_rel_gpu(&p.ws_counters[tile], 1u);
+          const unsigned int old = atom_add_acq_rel_gpu(&P.ws_counters[tile], 1u);
           *last_flag = (old == count - 1) ? 1 : 0;
         }
         named_bar_sync(1, 128);
@@ -602,7 +645,7 @@ k_gemm(const __grid_constant__ CUtensorMap tm_a,      // A: dense [rows_a x K] o
               store16(v, cb + c0);
             }
           }
-          if (et == 0) p.ws_counters[tile] = 0u;  // ready for the next call
+          if (et == 0) P.ws_counters[tile] = 0u;  // ready for the next call
         }
         named_bar_sync(1, 128);
       }

@@ -115,7 +115,8 @@ bool make_map(CUtensorMap* map, const void* base, int elem_bytes, uint64_t inner
 }
 
 // ---------------------------------------------------------------------------
-// GEMM planning
+// GEMM planning (one problem, or a group of independent problems launched
+// together)
 // ---------------------------------------------------------------------------
 struct Plan {
   int mode;        // kModeDense / kModeSparse / kModeHybrid
@@ -123,10 +124,12 @@ struct Plan {
   bool a_is_w;
   int bn;
   int kt;          // logical K per stage
-  int num_kt, tiles_a, tiles_b;
+  int n;           // problems
+  int num_kt[kMaxGroup], tiles_a[kMaxGroup], tiles_b[kMaxGroup];
   int sched;       // kSchedDataParallel / kSchedStreamK
   int grid;
   int64_t total_iters;
+  int total_tiles;
   size_t ws_bytes;
 };
 
@@ -144,18 +147,18 @@ int stage_k(int mode, bool bf16) {
 }
 
 size_t sk_accum_bytes(const Plan& pl) {
-  return (size_t)pl.tiles_a * pl.tiles_b * pl.bn * 128 * sizeof(float);
+  return (size_t)pl.total_tiles * pl.bn * 128 * sizeof(float);
 }
 
 size_t sk_ws_bytes(const Plan& pl) {
-  const size_t cnt = ((size_t)pl.tiles_a * pl.tiles_b * sizeof(unsigned int) + 255) & ~(size_t)255;
+  const size_t cnt = ((size_t)pl.total_tiles * sizeof(unsigned int) + 255) & ~(size_t)255;
   return sk_accum_bytes(pl) + cnt;
 }
 
 // Work schedule, from a cost model in units of one K-stage of one SM
 // (streaming one stage of weights takes about the same time on every SM
 // when all SMs stream):
-//   whole tiles round-robin: ceil(tiles / SMs) * stages per tile
+//   whole tiles round-robin: ceil(tiles / SMs) * stages of the longest tile
 //   stream-K:                ceil(tiles * stages / SMs) + the cost of finishing
 //                            the split tiles (fp32 atomics into an accumulator,
 //                            then one pass over it), which grows with the tile
@@ -163,35 +166,52 @@ size_t sk_ws_bytes(const Plan& pl) {
 // Stream-K needs a workspace for the accumulators; without enough of it the
 // whole-tile schedule is used.
 void choose_schedule(Plan& pl, int sms, size_t ws_cap) {
-  const int64_t tiles = (int64_t)pl.tiles_a * pl.tiles_b;
-  pl.total_iters = tiles * pl.num_kt;
+  int64_t tiles = 0, iters = 0;
+  for (int i = 0; i < pl.n; ++i) {
+    const int64_t t = (int64_t)pl.tiles_a[i] * pl.tiles_b[i];
+    tiles += t;
+    iters += t * pl.num_kt[i];
+  }
+  pl.total_tiles = (int)tiles;
+  pl.total_iters = iters;
   pl.sched = kSchedDataParallel;
   pl.grid = (int)std::min<int64_t>(tiles, sms);
   pl.ws_bytes = 0;
-  if (pl.num_kt > 1 && tiles < 4 * (int64_t)sms) {
-    const double cost_dp = (double)((tiles + sms - 1) / sms) * pl.num_kt;
-    const double cost_sk = (double)((pl.total_iters + sms - 1) / sms) + 2.0 + pl.bn * pl.bn / 800.0;
-    Plan t = pl;
-    t.sched = kSchedStreamK;
-    t.grid = (int)std::min<int64_t>(t.total_iters, sms);
-    t.ws_bytes = sk_ws_bytes(t);
-    if (cost_sk < cost_dp && t.ws_bytes <= ws_cap) pl = t;
+  // A single problem with many tiles balances well in whole tiles.  In a
+  // group the tiles differ in length, so the round-robin deal is costed as
+  // the most-loaded CTA's stage count.
+  if (iters <= tiles || (pl.n == 1 && tiles >= 4 * (int64_t)sms)) return;
+  double cost_dp;
+  if (pl.n == 1) {
+    cost_dp = (double)((tiles + sms - 1) / sms) * pl.num_kt[0];
+  } else {
+    std::vector<int64_t> load((size_t)pl.grid, 0);
+    int64_t tg = 0;
+    for (int i = 0; i < pl.n; ++i)
+      for (int64_t t = 0; t < (int64_t)pl.tiles_a[i] * pl.tiles_b[i]; ++t, ++tg)
+        load[(size_t)(tg % pl.grid)] += pl.num_kt[i];
+    cost_dp = (double)*std::max_element(load.begin(), load.end());
   }
+  const double cost_sk = (double)((iters + sms - 1) / sms) + 2.0 + pl.bn * pl.bn / 800.0;
+  Plan t = pl;
+  t.sched = kSchedStreamK;
+  t.grid = (int)std::min<int64_t>(iters, sms);
+  t.ws_bytes = sk_ws_bytes(t);
+  if (cost_sk < cost_dp && t.ws_bytes <= ws_cap) pl = t;
 }
 
 // ---------------------------------------------------------------------------
 // kernel launch for one instantiation
 // ---------------------------------------------------------------------------
-template <int kMode, bool kBf16, int kBN, bool kAIsW>
-int launch_gemm_inst(const CUtensorMap& ta, const CUtensorMap& ta2, const CUtensorMap& tb,
-                     const GemmParams& p, int grid, cudaStream_t stream) {
+template <int kMode, bool kBf16, int kBN, bool kAIsW, int kMaxProb>
+int launch_gemm_inst(const GemmLaunch<kMaxProb>& gl, int grid, cudaStream_t stream) {
   using C = GemmCfg<kMode, kBf16, kBN>;
   static std::atomic<uint64_t> attr_set{0};
   int dev = 0;
   cudaGetDevice(&dev);
   const uint64_t bit = 1ull << (dev & 63);
   if (!(attr_set.load() & bit)) {
-    if (cudaFuncSetAttribute(k_gemm<kMode, kBf16, kBN, kAIsW>,
+    if (cudaFuncSetAttribute(k_gemm<kMode, kBf16, kBN, kAIsW, kMaxProb>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess) {
       cudaGetLastError();
       return SP24_ERR_CUDA;
@@ -207,37 +227,45 @@ int launch_gemm_inst(const CUtensorMap& ta, const CUtensorMap& ta2, const CUtens
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = p.use_pdl ? 1 : 0;
-  return launch_result(cudaLaunchKernelEx(&cfg, k_gemm<kMode, kBf16, kBN, kAIsW>, ta, ta2, tb, p));
+  cfg.numAttrs = gl.p.use_pdl ? 1 : 0;
+  return launch_result(cudaLaunchKernelEx(&cfg, k_gemm<kMode, kBf16, kBN, kAIsW, kMaxProb>, gl));
 }
 
-template <int kMode, bool kBf16, bool kAIsW>
-int launch_gemm_bn(int bn, const CUtensorMap& ta, const CUtensorMap& ta2, const CUtensorMap& tb,
-                   const GemmParams& p, int grid, cudaStream_t s) {
+template <int kMode, bool kBf16, bool kAIsW, int kMaxProb>
+int launch_gemm_bn(int bn, const GemmLaunch<kMaxProb>& gl, int grid, cudaStream_t s) {
   switch (bn) {
-    case 16: return launch_gemm_inst<kMode, kBf16, 16, kAIsW>(ta, ta2, tb, p, grid, s);
-    case 32: return launch_gemm_inst<kMode, kBf16, 32, kAIsW>(ta, ta2, tb, p, grid, s);
-    case 64: return launch_gemm_inst<kMode, kBf16, 64, kAIsW>(ta, ta2, tb, p, grid, s);
-    case 128: return launch_gemm_inst<kMode, kBf16, 128, kAIsW>(ta, ta2, tb, p, grid, s);
+    case 16: return launch_gemm_inst<kMode, kBf16, 16, kAIsW, kMaxProb>(gl, grid, s);
+    case 32: return launch_gemm_inst<kMode, kBf16, 32, kAIsW, kMaxProb>(gl, grid, s);
+    case 64: return launch_gemm_inst<kMode, kBf16, 64, kAIsW, kMaxProb>(gl, grid, s);
+    case 128: return launch_gemm_inst<kMode, kBf16, 128, kAIsW, kMaxProb>(gl, grid, s);
     default: return SP24_ERR_INVALID_ARG;
   }
 }
 
-int dispatch_gemm(const Plan& pl, const CUtensorMap& ta, const CUtensorMap& ta2, const CUtensorMap& tb,
-                  const GemmParams& p, int grid, cudaStream_t s) {
+int dispatch_gemm(const Plan& pl, const GemmLaunch<1>& gl, cudaStream_t s) {
   if (!pl.a_is_w) {
     if (pl.mode == kModeSparse && pl.bf16 && pl.bn == 128)
-      return launch_gemm_inst<kModeSparse, true, 128, false>(ta, ta2, tb, p, grid, s);
+      return launch_gemm_inst<kModeSparse, true, 128, false, 1>(gl, pl.grid, s);
     return SP24_ERR_DTYPE;
   }
   if (pl.mode == kModeSparse)
-    return pl.bf16 ? launch_gemm_bn<kModeSparse, true, true>(pl.bn, ta, ta2, tb, p, grid, s)
-                   : launch_gemm_bn<kModeSparse, false, true>(pl.bn, ta, ta2, tb, p, grid, s);
+    return pl.bf16 ? launch_gemm_bn<kModeSparse, true, true, 1>(pl.bn, gl, pl.grid, s)
+                   : launch_gemm_bn<kModeSparse, false, true, 1>(pl.bn, gl, pl.grid, s);
   if (pl.mode == kModeDense)
-    return pl.bf16 ? launch_gemm_bn<kModeDense, true, true>(pl.bn, ta, ta2, tb, p, grid, s)
-                   : launch_gemm_bn<kModeDense, false, true>(pl.bn, ta, ta2, tb, p, grid, s);
+    return pl.bf16 ? launch_gemm_bn<kModeDense, true, true, 1>(pl.bn, gl, pl.grid, s)
+                   : launch_gemm_bn<kModeDense, false, true, 1>(pl.bn, gl, pl.grid, s);
   if (pl.mode == kModeHybrid && !pl.bf16)
-    return launch_gemm_bn<kModeHybrid, false, true>(pl.bn, ta, ta2, tb, p, grid, s);
+    return launch_gemm_bn<kModeHybrid, false, true, 1>(pl.bn, gl, pl.grid, s);
+  return SP24_ERR_DTYPE;
+}
+
+int dispatch_gemm_group(const Plan& pl, const GemmLaunch<kMaxGroup>& gl, cudaStream_t s) {
+  if (pl.mode == kModeSparse)
+    return pl.bf16 ? launch_gemm_bn<kModeSparse, true, true, kMaxGroup>(pl.bn, gl, pl.grid, s)
+                   : launch_gemm_bn<kModeSparse, false, true, kMaxGroup>(pl.bn, gl, pl.grid, s);
+  if (pl.mode == kModeDense)
+    return pl.bf16 ? launch_gemm_bn<kModeDense, true, true, kMaxGroup>(pl.bn, gl, pl.grid, s)
+                   : launch_gemm_bn<kModeDense, false, true, kMaxGroup>(pl.bn, gl, pl.grid, s);
   return SP24_ERR_DTYPE;
 }
 
@@ -277,31 +305,107 @@ int validate_gemm(const sp24_gemm_args* a) {
   return SP24_OK;
 }
 
-Plan plan_gemm(const sp24_gemm_args* a, int sms, size_t ws_cap) {
+int args_mode(const sp24_gemm_args* a) {
+  return a->tactic == SP24_TACTIC_DENSE ? kModeDense : (a->tile_dense_mask ? kModeHybrid : kModeSparse);
+}
+
+// Plans one launch over n (validated, mutually compatible) problems.
+Plan plan_group(const sp24_gemm_args* const* a, int n, int sms, size_t ws_cap) {
   Plan pl;
-  pl.bf16 = a->in_dtype == SP24_BF16;
+  memset(&pl, 0, sizeof pl);
+  pl.bf16 = a[0]->in_dtype == SP24_BF16;
   pl.a_is_w = true;
-  pl.mode = a->tactic == SP24_TACTIC_DENSE ? kModeDense
-                                           : (a->tile_dense_mask ? kModeHybrid : kModeSparse);
-  pl.bn = pick_bn(a->M);
+  pl.mode = args_mode(a[0]);
+  pl.bn = pick_bn(a[0]->M);
   pl.kt = stage_k(pl.mode, pl.bf16);
-  pl.num_kt = (int)((a->K + pl.kt - 1) / pl.kt);
-  pl.tiles_a = (int)((a->N + kBlockA - 1) / kBlockA);
-  pl.tiles_b = (int)((a->M + pl.bn - 1) / pl.bn);
+  pl.n = n;
+  for (int i = 0; i < n; ++i) {
+    pl.num_kt[i] = (int)((a[i]->K + pl.kt - 1) / pl.kt);
+    pl.tiles_a[i] = (int)((a[i]->N + kBlockA - 1) / kBlockA);
+    pl.tiles_b[i] = (int)((a[i]->M + pl.bn - 1) / pl.bn);
+  }
   choose_schedule(pl, sms, ws_cap);
   return pl;
 }
 
-void fill_sched(GemmParams& p, const Plan& pl, void* workspace) {
-  p.num_kt = pl.num_kt;
-  p.tiles_a = pl.tiles_a;
-  p.tiles_b = pl.tiles_b;
-  p.sched = pl.sched;
-  p.total_iters = pl.total_iters;
-  if (pl.sched == kSchedStreamK) {
-    p.ws_accum = static_cast<float*>(workspace);
-    p.ws_counters = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(workspace) + sk_accum_bytes(pl));
+Plan plan_gemm(const sp24_gemm_args* a, int sms, size_t ws_cap) { return plan_group(&a, 1, sms, ws_cap); }
+
+// Tensor maps and problem record of problem i of a launch.
+template <int kMaxProb>
+bool fill_problem(GemmLaunch<kMaxProb>& gl, int i, const sp24_gemm_args* a, const Plan& pl,
+                  int64_t iter_begin, int tile_begin, float* accum, unsigned int* counters) {
+  const int eb = dtype_bytes(a->in_dtype);
+  const int box_elems = 128 / eb;  // 128 bytes
+  bool ok = true;
+  if (pl.mode == kModeDense) {
+    ok &= make_map(&gl.tm_a[i], a->W, eb, a->K, a->N, a->ldw * eb, box_elems, kBlockA,
+                   CU_TENSOR_MAP_SWIZZLE_128B);
+    gl.tm_a2[i] = gl.tm_a[i];
+  } else if (pl.mode == kModeSparse) {
+    ok &= make_map(&gl.tm_a[i], a->W, eb, a->K / 2, a->N, a->ldw * eb, box_elems, kBlockA,
+                   CU_TENSOR_MAP_SWIZZLE_128B);
+    gl.tm_a2[i] = gl.tm_a[i];
+  } else {
+    ok &= make_map(&gl.tm_a[i], a->W_dense_tiles, 1, a->K, a->N, a->K, 128, kBlockA,
+                   CU_TENSOR_MAP_SWIZZLE_128B);
+    ok &= make_map(&gl.tm_a2[i], a->W, 1, a->K / 2, a->N, a->ldw, 64, kBlockA, CU_TENSOR_MAP_SWIZZLE_64B);
   }
+  ok &= make_map(&gl.tm_b[i], a->X, eb, a->K, a->M, a->ldx * eb, box_elems, pl.bn,
+                 CU_TENSOR_MAP_SWIZZLE_128B);
+  GemmProblem& P = gl.prob[i];
+  memset(&P, 0, sizeof P);
+  P.rows_a = (int32_t)a->N;
+  P.rows_b = (int32_t)a->M;
+  P.K = (int32_t)a->K;
+  P.num_kt = pl.num_kt[i];
+  P.tiles_a = pl.tiles_a[i];
+  P.tiles_b = pl.tiles_b[i];
+  P.tile_begin = tile_begin;
+  P.iter_begin = iter_begin;
+  P.meta = static_cast<const uint8_t*>(a->W_meta);
+  P.tile_mask = a->tile_dense_mask;
+  P.scale_a = a->in_dtype == SP24_E4M3 ? a->w_scales : nullptr;
+  P.scale_b = a->in_dtype == SP24_E4M3 ? a->x_scales : nullptr;
+  P.Y = a->Y;
+  P.ldy = a->ldy;
+  P.ws_accum = accum;
+  P.ws_counters = counters;
+  return ok;
+}
+
+// Fills a launch for n problems with the plan's schedule and workspace.
+template <int kMaxProb>
+int build_launch(GemmLaunch<kMaxProb>& gl, const sp24_gemm_args* const* a, int n, const Plan& pl,
+                 void* workspace, bool w_static) {
+  memset(&gl, 0, sizeof gl);
+  int64_t iter = 0;
+  int tile = 0;
+  float* accum = static_cast<float*>(workspace);
+  unsigned int* counters =
+      pl.sched == kSchedStreamK
+          ? reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(workspace) + sk_accum_bytes(pl))
+          : nullptr;
+  for (int i = 0; i < n; ++i) {
+    const int tiles = pl.tiles_a[i] * pl.tiles_b[i];
+    const bool sk = pl.sched == kSchedStreamK;
+    if (!fill_problem(gl, i, a[i], pl, iter, tile, sk ? accum : nullptr, sk ? counters : nullptr))
+      return SP24_ERR_CUDA;
+    if (sk) {
+      accum += (size_t)tiles * pl.bn * 128;
+      counters += tiles;
+    }
+    iter += (int64_t)tiles * pl.num_kt[i];
+    tile += tiles;
+  }
+  gl.p.n_prob = n;
+  gl.p.sched = pl.sched;
+  gl.p.total_iters = pl.total_iters;
+  gl.p.total_tiles = pl.total_tiles;
+  gl.p.out_f32 = a[0]->out_dtype == SP24_F32;
+  gl.p.use_pdl = 1;
+  gl.p.w_static = w_static ? 1 : 0;
+  gl.p.timeout_ns = g_timeout_ns.load();
+  return SP24_OK;
 }
 
 int run_gemm(const sp24_gemm_args* a, cudaStream_t stream) {
@@ -310,43 +414,26 @@ int run_gemm(const sp24_gemm_args* a, cudaStream_t stream) {
   if (st != SP24_OK) return st;
   size_t ws_cap = a->workspace != nullptr ? a->workspace_bytes : 0;
   if (a->workspace != nullptr && !aligned16(a->workspace)) return SP24_ERR_ALIGNMENT;
-  Plan pl = plan_gemm(a, di.sms, ws_cap);
-  const int eb = dtype_bytes(a->in_dtype);
-  const int box_elems = 128 / eb;  // 128 bytes
-  CUtensorMap ta, ta2, tb;
-  bool ok = true;
-  if (pl.mode == kModeDense) {
-    ok &= make_map(&ta, a->W, eb, a->K, a->N, a->ldw * eb, box_elems, kBlockA,
-                   CU_TENSOR_MAP_SWIZZLE_128B);
-    ta2 = ta;
-  } else if (pl.mode == kModeSparse) {
-    ok &= make_map(&ta, a->W, eb, a->K / 2, a->N, a->ldw * eb, box_elems, kBlockA,
-                   CU_TENSOR_MAP_SWIZZLE_128B);
-    ta2 = ta;
-  } else {
-    ok &= make_map(&ta, a->W_dense_tiles, 1, a->K, a->N, a->K, 128, kBlockA, CU_TENSOR_MAP_SWIZZLE_128B);
-    ok &= make_map(&ta2, a->W, 1, a->K / 2, a->N, a->ldw, 64, kBlockA, CU_TENSOR_MAP_SWIZZLE_64B);
-  }
-  ok &= make_map(&tb, a->X, eb, a->K, a->M, a->ldx * eb, box_elems, pl.bn, CU_TENSOR_MAP_SWIZZLE_128B);
-  if (!ok) return SP24_ERR_CUDA;
+  const Plan pl = plan_gemm(a, di.sms, ws_cap);
+  GemmLaunch<1> gl;
+  if ((st = build_launch(gl, &a, 1, pl, a->workspace, (a->flags & SP24_GEMM_W_STATIC) != 0)) != SP24_OK)
+    return st;
+  return dispatch_gemm(pl, gl, stream);
+}
 
-  GemmParams p;
-  memset(&p, 0, sizeof p);
-  p.rows_a = (int32_t)a->N;
-  p.rows_b = (int32_t)a->M;
-  p.K = (int32_t)a->K;
-  fill_sched(p, pl, a->workspace);
-  p.out_f32 = a->out_dtype == SP24_F32;
-  p.use_pdl = 1;
-  p.w_static = (a->flags & SP24_GEMM_W_STATIC) ? 1 : 0;
-  p.meta = static_cast<const uint8_t*>(a->W_meta);
-  p.tile_mask = a->tile_dense_mask;
-  p.scale_a = a->in_dtype == SP24_E4M3 ? a->w_scales : nullptr;
-  p.scale_b = a->in_dtype == SP24_E4M3 ? a->x_scales : nullptr;
-  p.Y = a->Y;
-  p.ldy = a->ldy;
-  p.timeout_ns = g_timeout_ns.load();
-  return dispatch_gemm(pl, ta, ta2, tb, p, pl.grid, stream);
+// Checks that n problems can share one grouped launch.
+int validate_group(const sp24_gemm_args* a, int n) {
+  if (a == nullptr) return SP24_ERR_NULL;
+  if (n < 1 || n > kMaxGroup) return SP24_ERR_INVALID_ARG;
+  for (int i = 0; i < n; ++i) {
+    int st = validate_gemm(&a[i]);
+    if (st != SP24_OK) return st;
+    if (a[i].tile_dense_mask != nullptr) return SP24_ERR_INVALID_ARG;
+    if (a[i].in_dtype != a[0].in_dtype || a[i].out_dtype != a[0].out_dtype ||
+        a[i].tactic != a[0].tactic || pick_bn(a[i].M) != pick_bn(a[0].M))
+      return SP24_ERR_INVALID_ARG;
+  }
+  return SP24_OK;
 }
 
 // Launch with programmatic dependent launch allowed (the kernel itself waits
@@ -519,6 +606,34 @@ int sp24_gemm(const sp24_gemm_args* a, void* stream) {
   return run_gemm(a, static_cast<cudaStream_t>(stream));
 }
 
+size_t sp24_gemm_grouped_workspace_bytes(const sp24_gemm_args* args, int n) {
+  if (validate_group(args, n) != SP24_OK) return 0;
+  DeviceInfo di;
+  if (current_device_info(&di) != SP24_OK) return 0;
+  const sp24_gemm_args* ptrs[kMaxGroup];
+  for (int i = 0; i < n; ++i) ptrs[i] = &args[i];
+  return plan_group(ptrs, n, di.sms, (size_t)-1).ws_bytes;
+}
+
+int sp24_gemm_grouped(const sp24_gemm_args* args, int n, void* workspace, size_t workspace_bytes,
+                      void* stream) {
+  int st = validate_group(args, n);
+  if (st != SP24_OK) return st;
+  if (workspace != nullptr && !aligned16(workspace)) return SP24_ERR_ALIGNMENT;
+  DeviceInfo di;
+  if ((st = current_device_info(&di)) != SP24_OK) return st;
+  const sp24_gemm_args* ptrs[kMaxGroup];
+  bool w_static = true;
+  for (int i = 0; i < n; ++i) {
+    ptrs[i] = &args[i];
+    w_static = w_static && (args[i].flags & SP24_GEMM_W_STATIC) != 0;
+  }
+  const Plan pl = plan_group(ptrs, n, di.sms, workspace != nullptr ? workspace_bytes : 0);
+  static thread_local GemmLaunch<kMaxGroup> gl;  // large: keep it off the stack
+  if ((st = build_launch(gl, ptrs, n, pl, workspace, w_static)) != SP24_OK) return st;
+  return dispatch_gemm_group(pl, gl, static_cast<cudaStream_t>(stream));
+}
+
 int sp24_gemm_noalloc(const sp24_gemm_args* a, void* stream) {
   int st = validate_gemm(a);
   if (st != SP24_OK) return st;
@@ -583,32 +698,41 @@ int sp24_prune_compress_activations_fused(const void* X, int64_t M, int64_t K, i
 
   // GEMM with X (compressed) as the sparse operand A and W dense as B.
   Plan pl;
+  memset(&pl, 0, sizeof pl);
   pl.mode = kModeSparse;
   pl.bf16 = true;
   pl.a_is_w = false;
   pl.bn = 128;
   pl.kt = 128;
-  pl.num_kt = (int)(K / 128);
-  pl.tiles_a = (int)((M + 127) / 128);
-  pl.tiles_b = (int)((N + 127) / 128);
+  pl.n = 1;
+  pl.num_kt[0] = (int)(K / 128);
+  pl.tiles_a[0] = (int)((M + 127) / 128);
+  pl.tiles_b[0] = (int)((N + 127) / 128);
   choose_schedule(pl, di.sms, 0);  // whole tiles: no workspace for partial sums
-  CUtensorMap ta, tb;
-  bool ok = make_map(&ta, x_values, 2, K / 2, M, (K / 2) * 2, 64, kBlockA, CU_TENSOR_MAP_SWIZZLE_128B);
-  ok &= make_map(&tb, W, 2, K, N, ldw * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  GemmLaunch<1> gl;
+  memset(&gl, 0, sizeof gl);
+  bool ok = make_map(&gl.tm_a[0], x_values, 2, K / 2, M, (K / 2) * 2, 64, kBlockA, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= make_map(&gl.tm_b[0], W, 2, K, N, ldw * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok) return SP24_ERR_CUDA;
-  GemmParams p;
-  memset(&p, 0, sizeof p);
-  p.rows_a = (int32_t)M;
-  p.rows_b = (int32_t)N;
-  p.K = (int32_t)K;
-  fill_sched(p, pl, nullptr);
-  p.out_f32 = out_dtype == SP24_F32;
-  p.use_pdl = 1;
-  p.meta = static_cast<const uint8_t*>(x_meta);
-  p.Y = Y;
-  p.ldy = ldy;
-  p.timeout_ns = g_timeout_ns.load();
-  return dispatch_gemm(pl, ta, ta, tb, p, pl.grid, s);
+  gl.tm_a2[0] = gl.tm_a[0];
+  GemmProblem& P = gl.prob[0];
+  P.rows_a = (int32_t)M;
+  P.rows_b = (int32_t)N;
+  P.K = (int32_t)K;
+  P.num_kt = pl.num_kt[0];
+  P.tiles_a = pl.tiles_a[0];
+  P.tiles_b = pl.tiles_b[0];
+  P.meta = static_cast<const uint8_t*>(x_meta);
+  P.Y = Y;
+  P.ldy = ldy;
+  gl.p.n_prob = 1;
+  gl.p.sched = pl.sched;
+  gl.p.total_iters = pl.total_iters;
+  gl.p.total_tiles = pl.total_tiles;
+  gl.p.out_f32 = out_dtype == SP24_F32;
+  gl.p.use_pdl = 1;
+  gl.p.timeout_ns = g_timeout_ns.load();
+  return dispatch_gemm(pl, gl, s);
 }
 
 int sp24_select_tactic(const sp24_gemm_args* sparse_args, const sp24_gemm_args* dense_args, int warmup,

@@ -98,6 +98,8 @@ def lib() -> ctypes.CDLL:
         "sp24_gemm": (I, [ctypes.POINTER(GemmArgs), P]),
         "sp24_gemm_noalloc": (I, [ctypes.POINTER(GemmArgs), P]),
         "sp24_gemm_noalloc_max_scratch_bytes": (ctypes.c_size_t, []),
+        "sp24_gemm_grouped": (I, [ctypes.POINTER(GemmArgs), I, P, ctypes.c_size_t, P]),
+        "sp24_gemm_grouped_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(GemmArgs), I]),
         "sp24_activations_workspace_bytes": (ctypes.c_size_t, [I64, I64]),
         "sp24_prune_compress_activations_fused": (I, [P, I64, I64, I64, P, I64, I64, P, I64, I,
                                                       P, P, P, ctypes.c_size_t, P]),
@@ -270,6 +272,48 @@ def gemm_noalloc(args: GemmArgs, stream=None):
     """sp24_gemm without any device allocation: stream-K scratch comes from a
     fixed array in the library (args.workspace is ignored)."""
     _check(lib().sp24_gemm_noalloc(ctypes.byref(args), _stream(stream)), "sp24_gemm_noalloc")
+
+
+class GemmGroup:
+    """Up to 16 independent GEMMs run by one sp24_gemm_grouped launch.
+
+    The argument array is built once; `workspace` (zero-filled, reusable
+    across calls on one stream) is allocated here when the group's schedule
+    needs one.  The GemmArgs objects (and the tensors they keep alive) are
+    held for the group's lifetime."""
+
+    def __init__(self, args_list, workspace: Optional[torch.Tensor] = None,
+                 allocate_workspace: bool = True):
+        self.args_list = list(args_list)
+        n = len(self.args_list)
+        self.arr = (GemmArgs * n)(*self.args_list)
+        self.n = n
+        need = lib().sp24_gemm_grouped_workspace_bytes(self.arr, n)
+        if workspace is None and need > 0 and allocate_workspace:
+            workspace = torch.zeros(need, dtype=torch.uint8, device=torch.cuda.current_device())
+        self.workspace = workspace
+        self.ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+
+    def workspace_bytes(self) -> int:
+        return lib().sp24_gemm_grouped_workspace_bytes(self.arr, self.n)
+
+    def __call__(self, stream=None):
+        _check(lib().sp24_gemm_grouped(self.arr, self.n, _ptr(self.workspace), self.ws_bytes,
+                                       _stream(stream)), "sp24_gemm_grouped")
+
+
+def m_class(M: int) -> int:
+    """The token-count class of a GEMM (1-16, 17-32, 33-64, >64); only GEMMs of
+    one class share a grouped launch."""
+    return 16 if M <= 16 else 32 if M <= 32 else 64 if M <= 64 else 128
+
+
+def gemm_grouped(args_list, workspace: Optional[torch.Tensor] = None, stream=None) -> GemmGroup:
+    """Runs the GEMMs of args_list in one grouped launch; returns the group
+    so that it can be called again."""
+    g = GemmGroup(args_list, workspace)
+    g(stream)
+    return g
 
 
 def gemm_noalloc_max_scratch_bytes() -> int:

@@ -133,3 +133,34 @@ def test_activation_and_selector_validation():
         == sp24.SP24_ERR_INVALID_ARG
     # values [16 x 128] bf16 (4096 B, 256-aligned) + one row block x 2 chunks of image
     assert sp24.activations_workspace_bytes(16, 256) == 4096 + 2 * 2048
+
+
+def test_grouped_gemm_validation():
+    f = L.sp24_gemm_grouped
+    assert f(None, 1, None, 0, None) == sp24.SP24_ERR_NULL
+    arr = (sp24.GemmArgs * 17)(*[gemm_args() for _ in range(17)])
+    assert f(arr, 0, None, 0, None) == sp24.SP24_ERR_INVALID_ARG
+    assert f(arr, 17, None, 0, None) == sp24.SP24_ERR_INVALID_ARG   # at most 16 problems
+    arr[1] = gemm_args(in_dtype=sp24.E4M3, x_scales=FAKE, w_scales=FAKE)
+    assert f(arr, 2, None, 0, None) == sp24.SP24_ERR_INVALID_ARG    # mixed input dtypes
+    arr[1] = gemm_args(out_dtype=sp24.F32)
+    assert f(arr, 2, None, 0, None) == sp24.SP24_ERR_INVALID_ARG    # mixed output dtypes
+    arr[1] = gemm_args(tactic=sp24.DENSE)
+    assert f(arr, 2, None, 0, None) == sp24.SP24_ERR_INVALID_ARG    # mixed tactics
+    arr[1] = gemm_args(M=17)
+    assert f(arr, 2, None, 0, None) == sp24.SP24_ERR_INVALID_ARG    # M classes 1-16 and 17-32
+    arr[1] = gemm_args(M=9, N=512, K=1024)
+    assert f(arr, 2, FAKE + 8, 1024, None) == sp24.SP24_ERR_ALIGNMENT
+    arr[1] = gemm_args(X=None)
+    assert f(arr, 2, None, 0, None) == sp24.SP24_ERR_NULL           # each problem validated
+    e4 = dict(in_dtype=sp24.E4M3, x_scales=FAKE, w_scales=FAKE)
+    arr[0] = gemm_args(mask=FAKE, dense=FAKE, **e4)
+    arr[1] = gemm_args(**e4)
+    assert f(arr, 2, None, 0, None) == sp24.SP24_ERR_INVALID_ARG    # no hybrid tiles in a group
+    assert L.sp24_gemm_grouped_workspace_bytes(arr, 2) == 0
+
+
+@pytest.mark.skipif(not NO_GPU, reason="only meaningful without a device")
+def test_grouped_gemm_without_device():
+    arr = (sp24.GemmArgs * 2)(gemm_args(), gemm_args(M=3, N=512, K=512))
+    assert L.sp24_gemm_grouped(arr, 2, None, 0, None) == sp24.SP24_ERR_UNSUPPORTED_DEVICE

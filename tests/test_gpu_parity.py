@@ -144,7 +144,9 @@ GEMM_SHAPES = [
 ]
 
 
-def run_gemm(X_bits, W_bits, e4, tactic, out_f32, mask=None, use_ws=True, flags=0):
+def prepare_gemm(X_bits, W_bits, e4, tactic, out_f32, mask=None, flags=0):
+    """Device operands from the oracle's own compression and quantization, the
+    argument block, and the oracle's fp64 product with its error scale."""
     M, K = X_bits.shape
     N = W_bits.shape[0]
     xq, xs, X_hat = oracle_x(X_bits, e4)
@@ -171,12 +173,17 @@ def run_gemm(X_bits, W_bits, e4, tactic, out_f32, mask=None, use_ws=True, flags=
         a = sp24.gemm_args(Xd, Wd, Y, K, sp24.DENSE, x_scales=dev(xs) if e4 else None,
                            w_scales=dev(ws_) if e4 else None)
     a.flags = flags
+    y_ref, a_ref = orc.gemm_f64(X_hat, W_hat)
+    return a, Y, y_ref, a_ref
+
+
+def run_gemm(X_bits, W_bits, e4, tactic, out_f32, mask=None, use_ws=True, flags=0):
+    a, Y, y_ref, a_ref = prepare_gemm(X_bits, W_bits, e4, tactic, out_f32, mask, flags)
     ws = workspace_for(a) if use_ws else None
     sp24.set_workspace(a, ws)
     sp24.gemm(a)
     torch.cuda.synchronize()
     assert sp24.last_device_error() == sp24.SP24_OK
-    y_ref, a_ref = orc.gemm_f64(X_hat, W_hat)
     return Y.float().cpu().numpy().astype(np.float64), y_ref, a_ref, a, ws
 
 
@@ -233,6 +240,84 @@ def test_w_static_prefetch_parity(M, N, K):
     X, W = inputs.linear_pair(M, N, K, seed=M + 11)
     y, y_ref, a_ref, _, _ = run_gemm(X, W, True, sp24.SPARSE, False, flags=sp24.GEMM_W_STATIC)
     check_tolerance(y, y_ref, a_ref, "w_static")
+
+
+# Grouped launches: independent problems of one M class, different N and K,
+# with ragged token counts; each output is checked against the oracle.
+GROUPS = {
+    "decode": [(8, 1024, 4096), (5, 384, 512), (16, 640, 2048), (1, 256, 1280)],
+    "m32": [(17, 512, 1024), (32, 256, 3072), (20, 1152, 256)],
+    "m64": [(40, 256, 1280), (64, 768, 512)],
+    "m128": [(130, 512, 768), (256, 384, 384), (65, 128, 2560)],
+}
+
+
+def run_group(shapes, e4, tactic, out_f32, use_ws=True, flags=0, seed=0):
+    items = []
+    for i, (M, N, K) in enumerate(shapes):
+        X, W = inputs.linear_pair(M, N, K, seed=seed + 31 * i + M, outliers=True)
+        items.append(prepare_gemm(X, W, e4, tactic, out_f32, flags=flags))
+    grp = sp24.GemmGroup([it[0] for it in items], allocate_workspace=use_ws)
+    grp()
+    torch.cuda.synchronize()
+    assert sp24.last_device_error() == sp24.SP24_OK
+    return grp, items
+
+
+def check_group(items, what):
+    for i, (_, Y, y_ref, a_ref) in enumerate(items):
+        y = Y.float().cpu().numpy().astype(np.float64)
+        check_tolerance(y, y_ref, a_ref, "%s problem %d" % (what, i))
+
+
+@pytest.mark.parametrize("group", sorted(GROUPS))
+@pytest.mark.parametrize("e4", [False, True])
+@pytest.mark.parametrize("tactic", [sp24.SPARSE, sp24.DENSE])
+def test_grouped_gemm_parity(group, e4, tactic):
+    for out_f32 in (True, False):
+        _, items = run_group(GROUPS[group], e4, tactic, out_f32, seed=len(group))
+        check_group(items, "group %s e4=%s tactic=%d f32=%s" % (group, e4, tactic, out_f32))
+
+
+@pytest.mark.parametrize("e4", [False, True])
+def test_grouped_gemm_whole_tiles_without_workspace(e4):
+    grp, items = run_group(GROUPS["decode"], e4, sp24.SPARSE, True, use_ws=False)
+    assert grp.workspace_bytes() > 0  # stream-K would have been chosen with a workspace
+    check_group(items, "grouped whole tiles")
+
+
+def test_grouped_gemm_sixteen_problems_w_static_reusable():
+    # the largest group: 16 decode projections of mixed sizes, weights marked
+    # static; three calls on one workspace, which ends zero after each
+    shapes = [(1 + (i % 16), 128 * (1 + i % 5), 256 * (1 + (i * 7) % 9)) for i in range(16)]
+    grp, items = run_group(shapes, True, sp24.SPARSE, True, flags=sp24.GEMM_W_STATIC, seed=5)
+    check_group(items, "16 problems")
+    first = [it[1].clone() for it in items]
+    for _ in range(2):
+        for it in items:
+            it[1].zero_()
+        grp()
+        torch.cuda.synchronize()
+        check_group(items, "16 problems repeat")
+        for it, y1 in zip(items, first):
+            y1 = y1.cpu().numpy().astype(np.float64)
+            assert np.allclose(it[1].cpu().numpy(), y1, rtol=1e-5, atol=1e-5 * np.abs(y1).max())
+    if grp.workspace is not None:
+        assert int(grp.workspace.view(torch.int32).abs().sum().item()) == 0
+
+
+def test_group_of_one_matches_single_gemm():
+    X, W = inputs.linear_pair(8, 1024, 4096, seed=123)
+    a, Y, y_ref, a_ref = prepare_gemm(X, W, True, sp24.SPARSE, True)
+    sp24.gemm_grouped([a])
+    torch.cuda.synchronize()
+    yg = Y.cpu().numpy().astype(np.float64)
+    check_tolerance(yg, y_ref, a_ref, "group of one")
+    sp24.set_workspace(a, workspace_for(a))
+    Y.zero_()
+    sp24.gemm(a)
+    torch.cuda.synchronize()
+    assert np.allclose(Y.cpu().numpy(), yg, rtol=1e-5, atol=1e-5 * np.abs(yg).max())
 
 
 @pytest.mark.parametrize("M", [1, 16, 200])
