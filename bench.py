@@ -47,6 +47,11 @@ def parse():
     p.add_argument("--manifest", default="", help="write the tactic audit manifest here")
     p.add_argument("--cpu-rows", type=int, default=256,
                    help="weight rows per GEMM in the CPU-baseline sample")
+    p.add_argument("--config", default="decode",
+                   choices=["decode", "tiny", "prefill", "activation", "hybrid", "prune"],
+                   help="decode (default): the headline step line.  The others time the other "
+                        "workloads of the hot path, one JSON line each, eager calls with an L2 "
+                        "flush before every timed call")
     p.add_argument("--case", default="",
                    help="M,N,K[,bf16|e4m3[,sparse|dense]]: time one GEMM of the decode/prefill "
                         "family in isolation (used for profiler captures) instead of the step")
@@ -542,32 +547,237 @@ def run_case(args):
     if n:
         sp24.set_workspace(a, torch.zeros(n, dtype=torch.uint8, device=dev))
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # > L2: evicts W between calls
-    for _ in range(args.warmup):
-        sp24.gemm(a)
-    torch.cuda.synchronize()
-    ts = []
-    for _ in range(args.steps):
-        flush.zero_()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record()
-        sp24.gemm(a)
-        e1.record()
-        torch.cuda.synchronize()
-        ts.append(e0.elapsed_time(e1) * 1e3)
+    t, _ = _time_calls(lambda: sp24.gemm(a), args.steps, args.warmup, flush)
     eb = 1 if e4 else 2
     wbytes = N * K * eb // 2 + N * K // 8 if sparse else N * K * eb
     byts = wbytes + M * K * eb + 2 * M * N
-    t = float(np.median(ts))
     print(json.dumps({"case": args.case, "us_median": round(t, 3), "GBps": round(byts / t / 1e3, 1),
                       "TFLOPS": round(2.0 * M * N * K / t / 1e6, 2),
                       "workspace_bytes": n}), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# the other workloads (--config): one JSON line each
+# ---------------------------------------------------------------------------
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        pk = json.load(open(path))
+        return float(pk["hbm_gbs"]), float(pk["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+def _flush_l2(buf):
+    """Evicts L2 by reading a buffer twice its size.  A read leaves clean lines
+    behind; a memset would leave ~126 MB of dirty lines whose write-back
+    lands inside the next timed call."""
+    buf.max()
+
+
+def _time_calls(fn, reps, warmup, flush):
+    """Median and min device time (us) of fn(), each call after an L2 flush.
+
+    All reps are enqueued before one synchronize, so the host runs ahead of
+    the device and no host-side launch latency lands between the events."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    torch.cuda._sleep(1_000_000)  # the device waits ~0.5 ms while the host enqueues the reps
+    ev = []
+    for _ in range(reps):
+        _flush_l2(flush)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        ev.append((e0, e1))
+    torch.cuda.synchronize()
+    ts = [e0.elapsed_time(e1) * 1e3 for e0, e1 in ev]
+    return float(np.median(ts)), float(np.min(ts))
+
+
+def _bf16_dev(bits, dev):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+
+def _roofline(flops, byts, t_us, tflops_peak, hbm):
+    t_roof = max(flops / (tflops_peak * 1e12), byts / (hbm * 1e9)) * 1e6
+    bound = "tensor" if flops / (tflops_peak * 1e12) >= byts / (hbm * 1e9) else "hbm"
+    return dict(bound=bound, t_roofline_us=round(t_roof, 3), frac=round(t_roof / t_us, 4))
+
+
+class _Linear:
+    """One linear layer's device operands in every form the suite times."""
+
+    def __init__(self, W_bits, M, e4, dev, x_seed, mask=None):
+        import torch
+
+        from semi_structured_sparse_02_b200 import inputs, sp24
+        N, K = W_bits.shape
+        self.M, self.N, self.K, self.e4 = M, N, K, e4
+        W = _bf16_dev(W_bits, dev)
+        X = _bf16_dev(inputs.normal_bf16((M, K), 1.0, seed=x_seed), dev)
+        vdt = torch.uint8 if e4 else torch.bfloat16
+        self.vals = torch.empty(N, K // 2, dtype=vdt, device=dev)
+        self.meta = torch.empty(sp24.meta_bytes(N, K), dtype=torch.uint8, device=dev)
+        self.wsc = torch.empty(N, dtype=torch.float32, device=dev) if e4 else None
+        self.mask = self.dense_tiles = None
+        if mask is not None:
+            self.mask = torch.from_numpy(mask).to(dev)
+            self.dense_tiles = torch.empty(N, K, dtype=torch.uint8, device=dev)
+        sp24.prune_compress(W, sp24.E4M3 if e4 else sp24.BF16, self.vals, self.meta,
+                            row_scales=self.wsc, tile_mask=self.mask, dense_tiles=self.dense_tiles)
+        if e4:
+            self.wd = torch.empty(N, K, dtype=torch.uint8, device=dev)
+            self.wdsc = torch.empty(N, dtype=torch.float32, device=dev)
+            sp24.quantize_e4m3_rows(W, self.wd, self.wdsc)
+            self.x = torch.empty(M, K, dtype=torch.uint8, device=dev)
+            self.xs = torch.empty(M, dtype=torch.float32, device=dev)
+            sp24.quantize_e4m3_rows(X, self.x, self.xs)
+        else:
+            self.wd, self.wdsc, self.x, self.xs = W, None, X, None
+        del W, X
+        self.Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        self.sp = sp24.gemm_args(self.x, self.vals, self.Y, K, sp24.SPARSE, W_meta=self.meta,
+                                 x_scales=self.xs, w_scales=self.wsc, tile_mask=self.mask,
+                                 W_dense_tiles=self.dense_tiles)
+        self.dn = sp24.gemm_args(self.x, self.wd, self.Y, K, sp24.DENSE, x_scales=self.xs,
+                                 w_scales=self.wdsc)
+        for a in (self.sp, self.dn):
+            n = sp24.gemm_workspace_bytes(a)
+            if n:
+                sp24.set_workspace(a, torch.zeros(n, dtype=torch.uint8, device=dev))
+
+    def sparse_bytes(self):
+        eb = 1 if self.e4 else 2
+        M, N, K = self.M, self.N, self.K
+        return N * K * eb // 2 + N * K // 8 + (4 * N if self.e4 else 0) + M * K * eb + \
+            (4 * M if self.e4 else 0) + 2 * M * N
+
+    def dense_bytes(self):
+        eb = 1 if self.e4 else 2
+        M, N, K = self.M, self.N, self.K
+        return N * K * eb + (4 * N if self.e4 else 0) + M * K * eb + (4 * M if self.e4 else 0) + 2 * M * N
+
+
+def run_config(args):
+    """Times one of the non-headline workloads and prints one JSON line."""
+    import torch
+
+    from semi_structured_sparse_02_b200 import inputs, manifest, sp24
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    sp24.lib()
+    hbm, bf16_tf, src = _peaks()
+    # dense-equivalent flops; sparse peaks are twice the dense ones, e4m3 twice bf16
+    peak = {("sparse", False): 2 * bf16_tf, ("dense", False): bf16_tf,
+            ("sparse", True): 4 * bf16_tf, ("dense", True): 2 * bf16_tf}
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    reps, warm = max(5, min(args.steps, 30)), max(3, args.warmup)
+    rows = []
+    out = {"config": args.config, "unit_note": "us = median device time per call (CUDA events), "
+           "L2 flushed before every call; TFLOPS = 2*M*N*K / t (dense-equivalent)",
+           "peaks": {"hbm_gbs": hbm, "bf16_dense_tflops": bf16_tf, "source": src,
+                     "sparse": "2x dense (2:4), e4m3 2x bf16 (nominal ratios)"}}
+
+    def gemm_row(L, label, extra=None):
+        t_sp, t_sp_min = _time_calls(lambda: sp24.gemm(L.sp), reps, warm, flush)
+        t_dn, t_dn_min = _time_calls(lambda: sp24.gemm(L.dn), reps, warm, flush)
+        F = 2.0 * L.M * L.N * L.K
+        r = dict(gemm=label, M=L.M, N=L.N, K=L.K, dtype="e4m3" if L.e4 else "bf16",
+                 us_sparse=round(t_sp, 2), us_dense=round(t_dn, 2),
+                 tflops_sparse=round(F / t_sp / 1e6, 1), tflops_dense=round(F / t_dn / 1e6, 1),
+                 gbs_sparse=round(L.sparse_bytes() / t_sp / 1e3, 1),
+                 speedup_vs_dense=round(t_dn / t_sp, 3),
+                 roofline_sparse=_roofline(F, L.sparse_bytes(), t_sp, peak[("sparse", L.e4)], hbm),
+                 roofline_dense=_roofline(F, L.dense_bytes(), t_dn, peak[("dense", L.e4)], hbm))
+        if extra:
+            r.update(extra)
+        rows.append(r)
+        print(json.dumps(r), file=sys.stderr, flush=True)
+
+    if args.config == "tiny":
+        X, W = inputs.tiny(0)
+        L = _Linear(W, 16, False, dev, 0)
+        L.x.copy_(_bf16_dev(X, dev))
+        gemm_row(L, "tiny")
+    elif args.config == "prefill":
+        for i, (N, K) in enumerate(inputs.PREFILL_NK):
+            W = inputs.weights_with_outliers(N, K, seed=3 + i)
+            for e4 in (False, True):
+                for M in inputs.PREFILL_M:
+                    L = _Linear(W, M, e4, dev, x_seed=3000 + M + i)
+                    gemm_row(L, "prefill")
+                    del L
+                    torch.cuda.empty_cache()
+    elif args.config == "hybrid":
+        records = {}
+        for e4 in (True,):
+            for gi, (name, N, K) in enumerate(inputs.HYBRID_NK):
+                W = inputs.normal_bf16((N, K), 0.02, seed=5 + gi)
+                mask = inputs.hybrid_mask(N, K, seed=gi)
+                for M in inputs.HYBRID_M:
+                    L = _Linear(W, M, e4, dev, x_seed=5000 + M + gi, mask=mask)
+                    rec = sp24.select_tactic(L.sp, L.dn, warmup=3, iters=15)
+                    records["%s_M%d" % (name, M)] = rec
+                    gemm_row(L, name, dict(selected=rec["selected"], dense_tiles=0.25))
+                    del L
+                    torch.cuda.empty_cache()
+        out["tactics"] = manifest.build_manifest(records, revision="synthetic-seeded")["metrics"]
+    elif args.config == "activation":
+        M, K, N = inputs.ACT_SHAPE["M"], inputs.ACT_SHAPE["K"], inputs.ACT_SHAPE["N"]
+        X = _bf16_dev(inputs.student_t_bf16((M, K), 3.0, seed=4), dev)
+        W = _bf16_dev(inputs.normal_bf16((N, K), 0.02, seed=4), dev)
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(sp24.activations_workspace_bytes(M, K), dtype=torch.uint8, device=dev)
+        t_f, t_f_min = _time_calls(lambda: sp24.prune_compress_activations_fused(X, W, Y, workspace=ws),
+                                   reps, warm, flush)
+        dn = sp24.gemm_args(X, W, Y, K, sp24.DENSE)
+        t_d, t_d_min = _time_calls(lambda: sp24.gemm(dn), reps, warm, flush)
+        F = 2.0 * M * N * K
+        byts = 2 * M * K + 1.125 * M * K + 1.125 * M * K + 2 * N * K + 2 * M * N
+        rows.append(dict(gemm="activation", M=M, N=N, K=K, dtype="bf16",
+                         us_fused=round(t_f, 2), us_dense=round(t_d, 2),
+                         tflops_fused=round(F / t_f / 1e6, 1), tflops_dense=round(F / t_d / 1e6, 1),
+                         speedup_vs_dense=round(t_d / t_f, 3),
+                         roofline_fused=_roofline(F, byts, t_f, peak[("sparse", False)], hbm),
+                         roofline_dense=_roofline(F, 2 * M * K + 2 * N * K + 2 * M * N, t_d,
+                                                  peak[("dense", False)], hbm),
+                         note="fused = prune+compress of X every call, then the sparse GEMM with X as "
+                              "the sparse operand; dense = the in-build dense GEMM on unpruned X"))
+    elif args.config == "prune":
+        shapes = [("decode", N, K, True) for N, K in inputs.DECODE_NK] + \
+                 [("prefill", N, K, False) for N, K in inputs.PREFILL_NK] + \
+                 [("hybrid", N, K, True) for _, N, K in inputs.HYBRID_NK]
+        for name, N, K, e4 in shapes:
+            W = _bf16_dev(inputs.normal_bf16((N, K), 0.02, seed=N + K), dev)
+            vals = torch.empty(N, K // 2, dtype=torch.uint8 if e4 else torch.bfloat16, device=dev)
+            meta = torch.empty(sp24.meta_bytes(N, K), dtype=torch.uint8, device=dev)
+            sc = torch.empty(N, dtype=torch.float32, device=dev) if e4 else None
+            t, t_min = _time_calls(lambda: sp24.prune_compress(W, sp24.E4M3 if e4 else sp24.BF16,
+                                                               vals, meta, row_scales=sc),
+                                   reps, warm, flush)
+            # algorithmic: read bf16 W once, write values + metadata (+ scales)
+            byts = 2 * N * K + N * K * (1 if e4 else 2) // 2 + N * K // 8 + (4 * N if e4 else 0)
+            rows.append(dict(weights=name, N=N, K=K, out="e4m3" if e4 else "bf16", us=round(t, 2),
+                             gbs=round(byts / t / 1e3, 1), frac_hbm=round(byts / t / 1e3 / hbm, 4)))
+            print(json.dumps(rows[-1]), file=sys.stderr, flush=True)
+            del W, vals, meta, sc
+    out["rows"] = rows
+    print(json.dumps(out), flush=True)
+
 
 
 def main():
     args = parse()
     if args.case:
         run_case(args)
+        return
+    if args.config != "decode":
+        run_config(args)
         return
     from semi_structured_sparse_02_b200 import replicas
     rank, world, local_rank = replicas.env_ranks()

@@ -187,6 +187,13 @@ typedef struct sp24_gemm_args {
  * launch).  X, x_scales and Y are always ordered after it. */
 #define SP24_GEMM_W_STATIC 1u
 
+/* Shapes with M >= 256 tokens and N >= 256 output features (no hybrid mask)
+ * run on CTA pairs: one tcgen05 MMA over two SMs computes a 256 x 256 output
+ * tile, each SM loading half of both operands (no workspace).  This flag
+ * keeps such a call on the one-CTA kernel (128-row tiles); results agree to
+ * the tolerance of the method, not bit for bit. */
+#define SP24_GEMM_SINGLE_CTA 2u
+
 /* Bytes of workspace the call would use for its stream-K schedule (0 if the
  * shape needs none).  Shapes with fewer than two output tiles per SM split
  * the tiles' K range evenly over all SMs; the parts of a split tile are added
@@ -290,7 +297,12 @@ typedef struct sp24_tactic_record {
  * the dense median; a tie or an ineligible sparse call selects DENSE
  * ("Sparse Tactic Audit": latency is the sole criterion; every fallback is
  * logged with its reason).  Synchronizes `stream`.  Both argument sets must
- * describe the same M, N, K and output buffer semantics. */
+ * describe the same M, N, K and output buffer semantics.
+ * Each timed call runs on a cold L2 (the library reads a buffer of twice the
+ * L2 size before it; that buffer is allocated on the first call per device
+ * and kept until exit), and the device is kept busy (a bounded spin kernel)
+ * while the host enqueues the timed sequence, so host launch latency is not
+ * timed. */
 int sp24_select_tactic(const sp24_gemm_args *sparse_args, const sp24_gemm_args *dense_args,
                        int warmup, int iters, sp24_tactic_record *out, void *stream);
 

@@ -1,0 +1,376 @@
+// gemm_wide.cuh -- the large-M GEMM: a CTA pair (cluster of two, tcgen05
+// cta_group::2) computes a 256 x 256 output tile with one MMA stream.
+//
+// Why a pair.  A single CTA's 128 x 128 tile needs about 195 bytes of operand
+// per clock at the sparse tensor rate (A 16 KB + B 32 KB + metadata 2 KB per
+// 128-deep bf16 stage), above what one SM can pull from L2, and the N = 128
+// MMA itself issues at only ~62% of the N = 256 rate.  In a pair each CTA
+// holds 128 rows of A (weights) and 128 rows of B (tokens); the pair's MMA is
+// M = 256 (A rows of both CTAs) by N = 256 (B rows of both CTAs), so every
+// CTA computes a 128 x 256 block while loading only half of B: 50 KB per
+// 128 x 256 x 128 stage, ~98 bytes per clock at the sparse rate.
+//
+//   warp 0       both CTAs: TMA producer for the CTA's own A, B and metadata
+//                halves; completion is counted on rank 0's stage barrier
+//                (which expects both halves).  No multicast.
+//   warp 1       both CTAs allocate tensor memory (pair allocation); rank 0,
+//                lane 0 issues tcgen05.cp (metadata, both CTAs) and the pair
+//                MMAs, then commits to the stage / accumulator barriers of
+//                both CTAs.
+//   warps 2..5   both CTAs: epilogue of the CTA's 128 accumulator rows.
+//
+// Tensor memory (512 columns per CTA).  Dense: two 256-column accumulators.
+// Sparse: the metadata needs columns too, so the second accumulator starts at
+// column 224 and overlaps the first by 32 columns; the metadata slots take
+// columns 480..511.  The epilogue drains a tile's 32 overlapping columns
+// first and then releases the accumulator, so the next tile's MMAs (which
+// only conflict in those columns) start while the rest is drained.  Draining
+// tile i's overlap implies tile i-1 is fully drained (the epilogue is
+// sequential), so one release per tile covers both accumulators.
+//
+// Work schedule: whole 256 x 256 tiles, round-robin over the pairs, A tile
+// index fastest (consecutive pairs share a B tile, all pairs share A in L2).
+#pragma once
+
+#include "gemm.cuh"
+
+namespace sp24 {
+
+struct WideLaunch {
+  CUtensorMap tm_a;     // A: dense [rows_a x K] or values [rows_a x K/2]; 128-byte box x 128 rows, SW128
+  CUtensorMap tm_b;     // B: [rows_b x K]; 128-byte box x 128 rows, SW128
+  CUtensorMap tm_meta;  // metadata image viewed as [chunks * 8 rows x 256 B]; box 256 B x 8 * chunks rows
+  int32_t rows_a, rows_b, K, num_kt;
+  int32_t tiles_a, tiles_b;  // 256-row tiles
+  int32_t total_tiles, meta_blocks;  // metadata row blocks (128 rows) that exist
+  int32_t out_f32, use_pdl;
+  const float* scale_a;
+  const float* scale_b;
+  void* Y;
+  int64_t ldy;
+  uint64_t timeout_ns;
+};
+
+template <int kMode, bool kBf16>
+struct WideCfg {
+  static constexpr bool kSparse = kMode == kModeSparse;
+  static constexpr int kKT = kSparse ? (kBf16 ? 128 : 256) : (kBf16 ? 64 : 128);  // logical K per stage
+  static constexpr int kABytes = 128 * 128;
+  static constexpr int kBBoxes = kSparse ? 2 : 1;
+  static constexpr int kBBytes = 128 * 128 * kBBoxes;
+  static constexpr int kMetaChunks = kSparse ? (kBf16 ? 1 : 2) : 0;
+  static constexpr int kMetaBytes = kMetaChunks * 2048;
+  static constexpr int kStageBytes = kABytes + kBBytes + kMetaBytes;  // per CTA
+  static constexpr int kStages = kSparse ? 4 : 6;
+  static constexpr int kMetaCols = kMetaChunks * 4;
+  static constexpr int kOverlap = kSparse ? 32 : 0;
+  static constexpr int kAcc1 = 256 - kOverlap;       // first column of the second accumulator
+  static constexpr int kMetaCol0 = 512 - kOverlap;   // metadata slots (sparse)
+  static_assert(!kSparse || kStages * kMetaCols <= kOverlap, "metadata slots overflow");
+  static constexpr int kBarOffset = kStages * kStageBytes;
+  static constexpr int kScaleOffset = kBarOffset + 256;
+  static constexpr int kEpiOffset = kScaleOffset + 256 * 4;
+  static constexpr int kSmemBytes = kEpiOffset + 4 * 2048 + 1024;  // + alignment slack
+  static_assert(kSmemBytes <= 232448, "shared memory overflow");
+};
+
+template <int kMode, bool kBf16, bool kAIsW>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+k_gemm_wide(const __grid_constant__ WideLaunch g) {
+  using C = WideCfg<kMode, kBf16>;
+  constexpr int S = C::kStages;
+  pdl_launch_dependents();
+
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOffset);
+  // bars[0..S): full (used in rank 0), [S..2S): empty, [2S..2S+2): acc_full,
+  // [2S+2..2S+4): acc_empty (used in rank 0), [2S+4]: drain
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* s_scale_b = reinterpret_cast<float*>(smem + C::kScaleOffset);
+  uint8_t* s_epi = smem + C::kEpiOffset;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = blockIdx.x >> 1;
+  const int n_pairs = gridDim.x >> 1;
+
+  auto bar_u32 = [&](int i) { return smem_u32(&bars[i]); };
+  const int kFull = 0, kEmpty = S, kAccFull = 2 * S, kAccEmpty = 2 * S + 2, kDrain = 2 * S + 4;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(bar_u32(kFull + s), 1);
+      mbar_init(bar_u32(kEmpty + s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar_u32(kAccFull + b), 1);
+      mbar_init(bar_u32(kAccEmpty + b), 8);  // 4 epilogue warps in each of the 2 CTAs
+    }
+    mbar_init(bar_u32(kDrain), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_slot), 512);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  cluster_sync();  // both CTAs' barriers initialized and tensor memory allocated
+  tc_fence_after_sync();
+  const uint32_t tmem_base = *tmem_slot;
+
+  auto meta_chunks = [&](int kt) -> int {
+    return (int)min((int64_t)C::kMetaChunks, (int64_t)(g.K / 128) - (int64_t)kt * C::kMetaChunks);
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ producer (both CTAs)
+    if (lane == 0) {
+      if (g.use_pdl) pdl_wait();
+      const uint32_t full0 = mapa_shared(bar_u32(kFull), 0);  // rank 0's stage barriers
+      const int box_elems = kBf16 ? 64 : 128;                // 128 bytes of B per box row
+      const int kc_total = g.K / 128;
+      int armed[S];
+      for (int s = 0; s < S; ++s) armed[s] = -1;
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = pair; ok && tile < g.total_tiles; tile += n_pairs) {
+        const int ta = tile % g.tiles_a, tb = tile / g.tiles_a;
+        const int ya = ta * 256 + (int)rank * 128;
+        const int yb = tb * 256 + (int)rank * 128;
+        int rb = ta * 2 + (int)rank;        // metadata row block of this CTA's A rows
+        if (rb >= g.meta_blocks) rb = 0;    // rows past the end: A is zero-filled; any valid metadata
+        for (int kt = 0; kt < g.num_kt; ++kt) {
+          if (!mbar_wait(bar_u32(kEmpty + stage), phase ^ 1, g.timeout_ns, kDevErrWaitEmpty)) {
+            ok = false;
+            *abort_flag = 1;
+            break;
+          }
+          if (rank == 0) {
+            mbar_arrive_expect_tx(bar_u32(kFull + stage), 2u * C::kStageBytes);
+            armed[stage] = (int)phase;
+          }
+          const uint32_t sa = smem_u32(smem + stage * C::kStageBytes);
+          const uint32_t fb = full0 + 8u * stage;
+          const int ax = C::kSparse ? kt * (C::kKT / 2) : kt * C::kKT;
+          tma_load_2d_pair(sa, &g.tm_a, fb, ax, ya);
+#pragma unroll
+          for (int bx = 0; bx < C::kBBoxes; ++bx)
+            tma_load_2d_pair(sa + C::kABytes + bx * 16384, &g.tm_b, fb, kt * C::kKT + bx * box_elems, yb);
+          if (C::kSparse)
+            tma_load_2d_pair(sa + C::kABytes + C::kBBytes, &g.tm_meta, fb, 0,
+                             (rb * kc_total + kt * C::kMetaChunks) * 8);
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      // rank 0: wait (bounded) until every armed stage has landed
+      for (int s = 0; s < S; ++s)
+        if (armed[s] >= 0) mbar_wait(bar_u32(kFull + s), (uint32_t)armed[s], g.timeout_ns, kDevErrWaitFull);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer (rank 0)
+    if (rank == 0 && lane == 0) {
+      const uint32_t idesc = make_idesc(C::kSparse, kBf16, 256, 256);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int j = 0;
+      for (int tile = pair; ok && tile < g.total_tiles; tile += n_pairs, ++j) {
+        const int b = j & 1;
+        // the accumulator: sparse waits for tile j-1's overlap release (which
+        // implies tile j-2 is drained); dense waits for tile j-2's release
+        if (C::kSparse ? j >= 1 : j >= 2) {
+          const int jr = C::kSparse ? j - 1 : j - 2;
+          if (!mbar_wait(bar_u32(kAccEmpty + (jr & 1)), (uint32_t)((jr >> 1) & 1), g.timeout_ns,
+                         kDevErrWaitAccEmpty)) {
+            ok = false;
+            *abort_flag = 1;
+            break;
+          }
+        }
+        tc_fence_after_sync();
+        const uint32_t d = tmem_base + (b ? (uint32_t)C::kAcc1 : 0u);
+        for (int kt = 0; kt < g.num_kt; ++kt) {
+          if (!mbar_wait(bar_u32(kFull + stage), phase, g.timeout_ns, kDevErrWaitFull)) {
+            ok = false;
+            *abort_flag = 1;
+            break;
+          }
+          tc_fence_after_sync();
+          const uint32_t sa = smem_u32(smem + stage * C::kStageBytes);
+          const uint32_t sb = sa + C::kABytes;
+          const uint32_t sm = sb + C::kBBytes;
+          const bool first = kt == 0;
+          if (C::kSparse) {
+            const uint32_t mcol = C::kMetaCol0 + stage * C::kMetaCols;
+            const int chunks = meta_chunks(kt);
+            for (int c = 0; c < chunks; ++c)
+              tc_cp_128x128b_pair(tmem_base + mcol + 4 * c, smem_desc(sm + c * 2048, 16, 128, kLayoutNone));
+            const int n_mma = kBf16 ? 4 : 2 * chunks;
+            for (int q = 0; q < n_mma; ++q) {
+              const uint64_t da = smem_desc(sa + q * 32, 16, 1024, kLayoutSw128);
+              const uint64_t db = smem_desc(sb + (q >> 1) * 16384 + (q & 1) * 64, 16, 1024, kLayoutSw128);
+              const uint32_t acc = (first && q == 0) ? 0u : 1u;
+              if (kBf16) {
+                const uint32_t col = mcol + q;
+                mma_sp_bf16_pair(d, da, db, tmem_base + (col & ~1u), idesc | (col & 1u), acc);
+              } else {
+                const uint32_t col = mcol + 4 * (q >> 1) + 2 * (q & 1);
+                mma_sp_f8_pair(d, da, db, tmem_base + col, idesc, acc);
+              }
+            }
+          } else {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint64_t da = smem_desc(sa + q * 32, 16, 1024, kLayoutSw128);
+              const uint64_t db = smem_desc(sb + q * 32, 16, 1024, kLayoutSw128);
+              if (kBf16) mma_bf16_pair(d, da, db, idesc, (first && q == 0) ? 0u : 1u);
+              else mma_f8_pair(d, da, db, idesc, (first && q == 0) ? 0u : 1u);
+            }
+          }
+          tc_commit_pair(bar_u32(kEmpty + stage), 0x3);  // frees the stage in both CTAs
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        tc_commit_pair(bar_u32(kAccFull + b), 0x3);
+      }
+      tc_commit_pair(bar_u32(kDrain), 0x1);
+      mbar_wait(bar_u32(kDrain), 0, g.timeout_ns, kDevErrWaitDrain);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------------ epilogue (both CTAs)
+    if (g.use_pdl) pdl_wait();  // Y and the B scales may belong to the upstream grid
+    const int lg = warp & 3;
+    const int row = lg * 32 + lane;   // accumulator lane of this thread
+    const int et = threadIdx.x - 64;  // 0..127
+    const uint32_t acc_empty0 = mapa_shared(bar_u32(kAccEmpty), 0);
+    uint8_t* wtile = s_epi + (warp - 2) * 2048;
+    const int eb = g.out_f32 ? 4 : 2;
+    const int per_vec = 16 / eb;
+    int j = 0;
+    for (int tile = pair; tile < g.total_tiles; tile += n_pairs, ++j) {
+      const int ta = tile % g.tiles_a, tb = tile / g.tiles_a;
+      const int b = j & 1;
+      const int ga = ta * 256 + (int)rank * 128 + row;  // A row of this thread
+      const float sa_v = (g.scale_a != nullptr && ga < g.rows_a) ? __ldg(g.scale_a + ga) : 1.0f;
+      named_bar_sync(1, 128);  // the previous tile's stores are done with the B scales
+      for (int i = et; i < 256; i += 128) {
+        const int gb = tb * 256 + i;
+        s_scale_b[i] = (g.scale_b != nullptr && gb < g.rows_b) ? g.scale_b[gb] : 1.0f;
+      }
+      named_bar_sync(1, 128);
+      bool ok = mbar_wait(bar_u32(kAccFull + b), (uint32_t)((j >> 1) & 1), g.timeout_ns, kDevErrWaitAccFull);
+      __syncwarp();
+      ok = named_bar_red_and(2, 128, ok);
+      if (!ok) {
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after_sync();
+      const uint32_t tbase = tmem_base + ((uint32_t)(lg * 32) << 16) + (b ? (uint32_t)C::kAcc1 : 0u);
+
+      // scales and stores 16 accumulator columns starting at c0
+      auto store16 = [&](const float (&v)[16], int c0) {
+        const int gb0 = tb * 256 + c0;
+        if (kAIsW) {
+          // lane = output feature n, column = token m: stage the warp's
+          // 32 n x 16 m block transposed, then write 16-byte vectors of n
+          const int n0 = ta * 256 + (int)rank * 128 + lg * 32;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float y = v[i] * sa_v * s_scale_b[c0 + i];
+            if (g.out_f32) reinterpret_cast<float*>(wtile)[i * 32 + lane] = y;
+            else reinterpret_cast<__nv_bfloat16*>(wtile)[i * 32 + lane] = __float2bfloat16_rn(y);
+          }
+          __syncwarp();
+          const int vec_per_row = 32 / per_vec;
+          for (int q = lane; q < 16 * vec_per_row; q += 32) {
+            const int i = q / vec_per_row, sg = q - i * vec_per_row;
+            const int m = gb0 + i;
+            const int n = n0 + sg * per_vec;
+            if (m >= g.rows_b || n >= g.rows_a) continue;
+            uint8_t* dst = static_cast<uint8_t*>(g.Y) + ((int64_t)m * g.ldy + n) * eb;
+            const uint8_t* src = wtile + (i * 32 + sg * per_vec) * eb;
+            if (n + per_vec <= g.rows_a) {
+              *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
+            } else {
+              for (int e = 0; e < g.rows_a - n; ++e)
+                for (int k = 0; k < eb; ++k) dst[e * eb + k] = src[e * eb + k];
+            }
+          }
+          __syncwarp();
+        } else {
+          // lane = token m, column = output feature n: 16 consecutive n of row ga
+          if (ga >= g.rows_a) return;
+          alignas(16) uint8_t vbuf[64];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float y = v[i] * sa_v * s_scale_b[c0 + i];
+            if (g.out_f32) reinterpret_cast<float*>(vbuf)[i] = y;
+            else reinterpret_cast<__nv_bfloat16*>(vbuf)[i] = __float2bfloat16_rn(y);
+          }
+          uint8_t* dst = static_cast<uint8_t*>(g.Y) + ((int64_t)ga * g.ldy + gb0) * eb;
+          if (gb0 + 16 <= g.rows_b) {
+            for (int q = 0; q < 16 / per_vec; ++q)
+              reinterpret_cast<uint4*>(dst)[q] = reinterpret_cast<const uint4*>(vbuf)[q];
+          } else {
+            for (int e = 0; e < g.rows_b - gb0; ++e)
+              for (int k = 0; k < eb; ++k) dst[e * eb + k] = vbuf[e * eb + k];
+          }
+        }
+      };
+      auto drain = [&](int c_begin, int c_end) {
+#pragma unroll 1
+        for (int c0 = c_begin; c0 < c_end; c0 += 16) {
+          uint32_t r[16];
+          tmem_ld_x16(tbase + c0, r);
+          tmem_ld_wait();
+          float v[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+          store16(v, c0);
+        }
+      };
+      auto release = [&]() {
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(acc_empty0 + 8u * b);
+      };
+      if (C::kSparse) {
+        // the columns shared with the other accumulator first, then release
+        const int ov0 = b ? 0 : 256 - C::kOverlap;
+        drain(ov0, ov0 + C::kOverlap);
+        release();
+        if (b) drain(C::kOverlap, 256);
+        else drain(0, 256 - C::kOverlap);
+      } else {
+        drain(0, 256);
+        release();
+      }
+    }
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  cluster_sync();  // neither CTA leaves while its peer may still use its memory
+  if (warp == 1) {
+    tc_fence_after_sync();
+    tmem_dealloc_pair(tmem_base, 512);
+  }
+}
+
+}  // namespace sp24

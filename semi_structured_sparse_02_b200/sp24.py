@@ -33,6 +33,7 @@ SP24_ERR_WORKSPACE = 9
 BF16, E4M3, F32 = 0, 1, 2
 SPARSE, DENSE = 0, 1
 GEMM_W_STATIC = 1
+GEMM_SINGLE_CTA = 2
 
 
 class Sp24Error(RuntimeError):

@@ -379,6 +379,98 @@ def test_activation_fused_parity(M, N, K):
 
 
 # ---------------------------------------------------------------------------
+# CTA-pair kernel (M >= 256 and N >= 256): 256 x 256 tiles on two SMs
+# ---------------------------------------------------------------------------
+PAIR_SHAPES = [
+    (256, 256, 256),     # one pair tile
+    (512, 384, 1024),    # second row tile half past N: zero-filled A rows, clamped metadata
+    (300, 640, 768),     # ragged token count
+    (260, 256, 384),     # e4m3: the last 256-deep stage holds one 128-deep chunk
+    (1024, 1024, 2048),  # 16 tiles, deep K
+]
+
+
+@pytest.mark.parametrize("M,N,K", PAIR_SHAPES)
+@pytest.mark.parametrize("e4", [False, True])
+@pytest.mark.parametrize("tactic", [sp24.SPARSE, sp24.DENSE])
+def test_pair_kernel_parity(M, N, K, e4, tactic):
+    X, W = inputs.linear_pair(M, N, K, seed=7 * M + N + K, outliers=True)
+    for out_f32 in (True, False):
+        y, y_ref, a_ref, args, ws = run_gemm(X, W, e4, tactic, out_f32)
+        assert ws is None  # the pair kernel needs no workspace
+        check_tolerance(y, y_ref, a_ref, "pair M%d N%d K%d e4=%s tactic=%d f32=%s"
+                        % (M, N, K, e4, tactic, out_f32))
+    # the one-CTA kernel on the same operands agrees to the same tolerance
+    y1, _, _, _, _ = run_gemm(X, W, e4, tactic, True, flags=sp24.GEMM_SINGLE_CTA)
+    check_tolerance(y1, y_ref, a_ref, "single-CTA M%d N%d K%d" % (M, N, K))
+
+
+@pytest.mark.parametrize("e4", [False, True])
+def test_pair_kernel_many_tiles_per_pair_sampled(e4):
+    # 4096 x 4096 output = 256 tiles over at most 74 pairs: every pair runs
+    # several tiles, cycling both accumulators (and, sparse, their overlap)
+    M, N, K = 4096, 4096, 512
+    X, W = inputs.linear_pair(M, N, K, seed=99, outliers=True)
+    for tactic in (sp24.SPARSE, sp24.DENSE):
+        a, Y, _, _ = _prepare_large(X, W, e4, tactic)
+        sp24.gemm(a)
+        torch.cuda.synchronize()
+        assert sp24.last_device_error() == sp24.SP24_OK
+        g = np.random.default_rng(3)
+        ms = np.concatenate([g.choice(M, size=40, replace=False), [0, 255, 256, M - 1]])
+        ns = np.concatenate([g.choice(N, size=40, replace=False), [0, 255, 256, N - 1]])
+        W_hat = _w_hat(W[ns], e4, tactic)
+        _, _, X_hat = oracle_x(X[ms], e4)
+        y_ref, a_ref = orc.gemm_f64_sampled(X_hat, W_hat, np.arange(ms.size), np.arange(ns.size))
+        y_gpu = Y.float().cpu().numpy().astype(np.float64)[np.ix_(ms, ns)].diagonal()
+        check_tolerance(y_gpu, y_ref, a_ref, "pair many tiles e4=%s tactic=%d" % (e4, tactic))
+
+
+def _w_hat(W_rows, e4, tactic):
+    if tactic == sp24.SPARSE:
+        return OracleSparseW(W_rows, e4m3=e4).W_hat
+    if e4:
+        wq, s = orc.quantize_rows_e4m3(W_rows)
+        return orc.e4m3_decode(wq) * s.astype(np.float64)[:, None]
+    return orc.bf16_bits_to_f64(W_rows)
+
+
+def _prepare_large(X_bits, W_bits, e4, tactic):
+    """Device operands from the library's own prune / quantize (bit-exact to
+    the oracle, checked elsewhere), for sizes where the oracle's full
+    compression would be slow."""
+    M, K = X_bits.shape
+    N = W_bits.shape[0]
+    Wd = dev_bf16(W_bits)
+    ws_ = torch.empty(N, dtype=torch.float32, device="cuda") if e4 else None
+    if tactic == sp24.SPARSE:
+        Wv = torch.empty(N, K // 2, dtype=torch.uint8 if e4 else torch.bfloat16, device="cuda")
+        meta = torch.empty(sp24.meta_bytes(N, K), dtype=torch.uint8, device="cuda")
+        sp24.prune_compress(Wd, sp24.E4M3 if e4 else sp24.BF16, Wv, meta, row_scales=ws_)
+    else:
+        meta = None
+        if e4:
+            Wv = torch.empty(N, K, dtype=torch.uint8, device="cuda")
+            sp24.quantize_e4m3_rows(Wd, Wv, ws_)
+        else:
+            Wv = Wd
+    if e4:
+        Xd = torch.empty(M, K, dtype=torch.uint8, device="cuda")
+        xs = torch.empty(M, dtype=torch.float32, device="cuda")
+        sp24.quantize_e4m3_rows(dev_bf16(X_bits), Xd, xs)
+    else:
+        Xd, xs = dev_bf16(X_bits), None
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    a = sp24.gemm_args(Xd, Wv, Y, K, tactic, W_meta=meta, x_scales=xs, w_scales=ws_)
+    return a, Y, None, None
+
+
+@pytest.mark.parametrize("M,N,K", [(512, 384, 512), (300, 256, 1024)])
+def test_activation_fused_pair_kernel(M, N, K):
+    test_activation_fused_parity(M, N, K)
+
+
+# ---------------------------------------------------------------------------
 # full-size configurations, sampled outputs
 # ---------------------------------------------------------------------------
 
