@@ -54,7 +54,8 @@ def parse():
                         "flush before every timed call")
     p.add_argument("--case", default="",
                    help="M,N,K[,bf16|e4m3[,sparse|dense]]: time one GEMM of the decode/prefill "
-                        "family in isolation (used for profiler captures) instead of the step")
+                        "family in isolation (used for profiler captures) instead of the step; "
+                        "group:M1,M2,...: one grouped launch of the decode GEMMs for those M")
     return p.parse_args()
 
 
@@ -508,11 +509,52 @@ def run_reference(args, world):
     print(json.dumps(line), flush=True)
 
 
+def run_group_case(args):
+    """One grouped launch of the decode GEMMs for the token counts listed after
+    "group:" (e.g. group:1,8), e4m3 sparse weights marked static; eager calls,
+    CUDA-event timing (for profiler captures)."""
+    import torch
+
+    from semi_structured_sparse_02_b200 import inputs, sp24
+    dev = torch.device("cuda", 0)
+    Ms = [int(v) for v in args.case.split(":", 1)[1].split(",")]
+    keep, argl = [], []
+    for M in Ms:
+        for i, (N, K) in enumerate(inputs.DECODE_NK):
+            W = torch.from_numpy(inputs.normal_bf16((N, K), 0.02, seed=N + K).view(np.int16)).view(
+                torch.bfloat16).to(dev)
+            X = torch.from_numpy(inputs.normal_bf16((M, K), 1.0, seed=M + i).view(np.int16)).view(
+                torch.bfloat16).to(dev)
+            vals = torch.empty(N, K // 2, dtype=torch.uint8, device=dev)
+            meta = torch.empty(sp24.meta_bytes(N, K), dtype=torch.uint8, device=dev)
+            wsc = torch.empty(N, dtype=torch.float32, device=dev)
+            sp24.prune_compress(W, sp24.E4M3, vals, meta, row_scales=wsc)
+            xq = torch.empty(M, K, dtype=torch.uint8, device=dev)
+            xs = torch.empty(M, dtype=torch.float32, device=dev)
+            sp24.quantize_e4m3_rows(X, xq, xs)
+            Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+            argl.append(sp24.gemm_args(xq, vals, Y, K, sp24.SPARSE, W_meta=meta, x_scales=xs, w_scales=wsc,
+                                       flags=sp24.GEMM_W_STATIC))
+            keep.append((W, X))
+            del W
+    del keep
+    grp = sp24.GemmGroup(argl)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    t, _ = _time_calls(lambda: grp(), args.steps, args.warmup, flush)
+    byts = sum(gemm_bytes(a.M, a.N, a.K) for a in argl)
+    print(json.dumps({"case": args.case, "gemms": len(argl), "us_median": round(t, 3),
+                      "GBps": round(byts / t / 1e3, 1), "bytes": byts,
+                      "workspace_bytes": grp.ws_bytes}), flush=True)
+
+
 def run_case(args):
     """One GEMM shape, eager calls, CUDA-event timing (for profiler captures)."""
     import torch
 
     from semi_structured_sparse_02_b200 import inputs, sp24
+    if args.case.startswith("group:"):
+        run_group_case(args)
+        return
     f = args.case.split(",")
     M, N, K = int(f[0]), int(f[1]), int(f[2])
     e4 = (f[3] if len(f) > 3 else "e4m3") == "e4m3"

@@ -194,6 +194,12 @@ typedef struct sp24_gemm_args {
  * the tolerance of the method, not bit for bit. */
 #define SP24_GEMM_SINGLE_CTA 2u
 
+/* For M <= 255 (and N >= 256, no hybrid mask): run 256-row weight tiles on
+ * CTA pairs (M = 256 pair MMA, each SM loading half of the tile) instead of
+ * 128-row tiles on single CTAs.  In a grouped call it applies when every
+ * problem sets it.  Same results to the method's tolerance. */
+#define SP24_GEMM_CTA_PAIR 4u
+
 /* Bytes of workspace the call would use for its stream-K schedule (0 if the
  * shape needs none).  Shapes with fewer than two output tiles per SM split
  * the tiles' K range evenly over all SMs; the parts of a split tile are added

@@ -37,6 +37,8 @@
 
 #include <cuda_bf16.h>
 
+#include <type_traits>
+
 #include "sp24_device.cuh"
 
 namespace sp24 {
@@ -55,7 +57,7 @@ struct GemmProblem {
   int32_t num_kt;             // K-stages per tile
   int32_t tiles_a, tiles_b;
   int32_t tile_begin;         // first global tile index of this problem
-  int32_t pad0;
+  int32_t meta_blocks;        // 128-row blocks of the metadata image (pair tiles clamp to it)
   int64_t iter_begin;         // first global stream-K iteration of this problem
   const uint8_t* meta;        // metadata image of A (sparse / hybrid)
   const uint8_t* tile_mask;   // hybrid: [tiles_a x K/128]
@@ -89,16 +91,21 @@ struct GemmLaunch {
   GemmParams p;
 };
 
-// Compile-time geometry of one configuration.
-template <int kMode, bool kBf16, int kBN>
+// Compile-time geometry of one configuration.  kPair: the tile's 256 A rows
+// are split over a CTA pair (tcgen05 cta_group::2); each CTA holds 128 A rows
+// and kBN/2 of the kBN B rows, and the pair's MMA is M = 256 by N = kBN.
+template <int kMode, bool kBf16, int kBN, bool kPair = false>
 struct GemmCfg {
   static constexpr bool kSparse = kMode == kModeSparse;
   static constexpr bool kHybrid = kMode == kModeHybrid;
+  static_assert(!(kPair && kHybrid), "hybrid tiles run on single CTAs");
+  static constexpr int kRowsA = kPair ? 2 * kBlockA : kBlockA;  // A rows per tile
+  static constexpr int kBRows = kPair ? kBN / 2 : kBN;          // B rows per CTA
   // logical K per stage
   static constexpr int kKT = kHybrid ? 128 : (kSparse ? (kBf16 ? 128 : 256) : (kBf16 ? 64 : 128));
   static constexpr int kABytes = kBlockA * 128;                 // A tile (dense or sparse)
   static constexpr int kBBoxes = kSparse ? 2 : 1;               // 128-byte-wide B boxes
-  static constexpr int kBBytes = kBN * 128 * kBBoxes;
+  static constexpr int kBBytes = kBRows * 128 * kBBoxes;
   static constexpr int kMetaChunks = kSparse ? (kBf16 ? 1 : 2) : (kHybrid ? 1 : 0);
   static constexpr int kMetaBytes = kMetaChunks * 2048;
   static constexpr int kStageBytes = kABytes + kBBytes + kMetaBytes;
@@ -196,16 +203,17 @@ struct SegIter {
   }
 };
 
-// The CTA whose stream-K range holds global iteration i.
+// The unit (CTA or CTA pair) whose stream-K range holds global iteration i.
 __device__ __forceinline__ int sk_owner(int64_t total_iters, int grid, int64_t i) {
   return (int)(((i + 1) * grid - 1) / total_iters);
 }
 
-template <int kMode, bool kBf16, int kBN, bool kAIsW, int kMaxProb>
+template <int kMode, bool kBf16, int kBN, bool kAIsW, int kMaxProb, bool kPair = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
-  using C = GemmCfg<kMode, kBf16, kBN>;
+  using C = GemmCfg<kMode, kBf16, kBN, kPair>;
   constexpr int S = C::kStages;
+  static_assert(!kPair || kAIsW, "pairs split the weight rows");
   const GemmParams& p = g.p;
 
   // the next kernel in the stream may launch now; it waits for our completion
@@ -218,7 +226,7 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
                                              ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOffset);
   // bars[0..S): full, [S..2S): empty, [2S..2S+2): acc_full, [2S+2..2S+4): acc_empty,
-  // [2S+4]: drain
+  // [2S+4]: drain.  In a pair the full, acc_empty and drain barriers of rank 0 are used.
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* last_flag = reinterpret_cast<int*>(tmem_slot + 2);
@@ -227,7 +235,10 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int grid = gridDim.x;
+  // scheduling units: CTAs, or CTA pairs
+  const uint32_t rank = kPair ? cluster_ctarank() : 0u;
+  const int unit = kPair ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int units = kPair ? (int)(gridDim.x >> 1) : (int)gridDim.x;
 
   auto full_bar = [&](int s) { return smem_u32(&bars[s]); };
   auto empty_bar = [&](int s) { return smem_u32(&bars[S + s]); };
@@ -242,18 +253,24 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(accf_bar(b), 1);
-      mbar_init(acce_bar(b), 128);
+      mbar_init(acce_bar(b), kPair ? 8 : 4);  // one arrive per epilogue warp (of both CTAs)
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
-    tmem_relinquish();
+    if (kPair) {
+      tmem_alloc_pair(smem_u32(tmem_slot), C::kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before_sync();
   __syncthreads();
+  if (kPair) cluster_sync();  // the peer's barriers and tensor memory are ready
   tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
 
@@ -272,13 +289,19 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
       const uint64_t pol_keep = policy_evict_last();     // B: re-read by many CTAs
       int armed[S];
       for (int s = 0; s < S; ++s) armed[s] = -1;
+      // the barrier a copy completes on (rank 0's in a pair)
+      auto fbar = [&](int stage) { return kPair ? mapa_shared(full_bar(stage), 0) : full_bar(stage); };
+      auto load2d = [&](uint32_t dst, const CUtensorMap* map, int stage, int32_t x, int32_t y, uint64_t pol) {
+        if (kPair) tma_load_2d_pair_hint(dst, map, fbar(stage), x, y, pol);
+        else tma_load_2d(dst, map, full_bar(stage), x, y, pol);
+      };
 
       // the A-operand (and metadata) part of one stage
       auto load_a = [&](int stage, int pr, int ta, int kt) {
         const GemmProblem& P = g.prob[pr];
         const uint32_t sa = smem_u32(smem + stage * C::kStageBytes);
         const uint32_t sm = sa + C::kABytes + C::kBBytes;
-        const int32_t ya = ta * kBlockA;
+        const int32_t ya = ta * C::kRowsA + (int32_t)rank * kBlockA;
         if (C::kHybrid) {
           if (is_dense_tile(P, ta, kt)) {
             tma_load_2d(sa, &g.tm_a[pr], full_bar(stage), kt * 128, ya, pol_stream);
@@ -289,35 +312,51 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
           }
         } else {
           const int ax = C::kSparse ? kt * (C::kKT / 2) : kt * C::kKT;  // elements
-          tma_load_2d(sa, &g.tm_a[pr], full_bar(stage), ax, ya, pol_stream);
+          load2d(sa, &g.tm_a[pr], stage, ax, ya, pol_stream);
           if (C::kSparse) {
             const int64_t kc_total = P.K / 128;
-            const uint8_t* src = P.meta + ((int64_t)ta * kc_total + (int64_t)kt * C::kMetaChunks) * 2048;
-            bulk_load(sm, src, meta_chunks(P, kt) * 2048, full_bar(stage), pol_stream);
+            if (kPair) {
+              // metadata through the 2-D map over the image (8 rows of 256 B per
+              // chunk); rows past the end take block 0 (their A rows are zero)
+              int rb = ta * 2 + (int)rank;
+              if (rb >= P.meta_blocks) rb = 0;
+              load2d(sm, &g.tm_a2[pr], stage, 0, (int32_t)((rb * kc_total + (int64_t)kt * C::kMetaChunks) * 8),
+                     pol_stream);
+            } else {
+              const uint8_t* src = P.meta + ((int64_t)ta * kc_total + (int64_t)kt * C::kMetaChunks) * 2048;
+              bulk_load(sm, src, meta_chunks(P, kt) * 2048, full_bar(stage), pol_stream);
+            }
           }
         }
       };
       auto load_b = [&](int stage, int pr, int tb, int kt) {
         const uint32_t sb = smem_u32(smem + stage * C::kStageBytes) + C::kABytes;
-        const int32_t yb = tb * kBN;
+        const int32_t yb = tb * kBN + (int32_t)rank * C::kBRows;
         if (C::kHybrid) {
           tma_load_2d(sb, &g.tm_b[pr], full_bar(stage), kt * 128, yb, pol_keep);
         } else {
           const int box_elems = kBf16 ? 64 : 128;
 #pragma unroll
           for (int bx = 0; bx < C::kBBoxes; ++bx)
-            tma_load_2d(sb + bx * kBN * 128, &g.tm_b[pr], full_bar(stage), kt * C::kKT + bx * box_elems,
-                        yb, pol_keep);
+            load2d(sb + bx * C::kBRows * 128, &g.tm_b[pr], stage, kt * C::kKT + bx * box_elems, yb, pol_keep);
         }
       };
+      // bytes that complete one stage (both CTAs' halves in a pair)
       auto stage_bytes = [&](int pr, int ta, int kt) -> uint32_t {
         const GemmProblem& P = g.prob[pr];
         if (C::kHybrid)
           return is_dense_tile(P, ta, kt) ? (uint32_t)(C::kABytes + kBN * 128)
                                           : (uint32_t)(kBlockA * 64 + kBN * 128 + 2048);
+        if (kPair) return 2u * (uint32_t)C::kStageBytes;  // metadata boxes are always whole
         uint32_t b = C::kABytes + C::kBBytes;
         if (C::kSparse) b += (uint32_t)meta_chunks(P, kt) * 2048;
         return b;
+      };
+      auto arm = [&](int stage, uint32_t bytes, int ph) {
+        if (rank == 0) {
+          mbar_arrive_expect_tx(full_bar(stage), bytes);
+          armed[stage] = ph;
+        }
       };
 
       // 1. weights first: arm the first S stages and start their A loads
@@ -326,19 +365,18 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
       int last_pr = -1;
       if (p.w_static) {
         SegIter<kMaxProb> it;
-        it.init(g, blockIdx.x, grid);
+        it.init(g, unit, units);
         int pr, tile, kb, ke, seg;
-        while (pre < S && it.next(g, grid, pr, tile, kb, ke, seg)) {
+        while (pre < S && it.next(g, units, pr, tile, kb, ke, seg)) {
           if (pr != last_pr) {
             tma_prefetch_desc(&g.tm_a[pr]);
-            if (C::kHybrid) tma_prefetch_desc(&g.tm_a2[pr]);
+            if (C::kHybrid || (kPair && C::kSparse)) tma_prefetch_desc(&g.tm_a2[pr]);
             last_pr = pr;
           }
           const int ta = tile % g.prob[pr].tiles_a;
           for (int kt = kb; kt < ke && pre < S; ++kt, ++pre) {
-            mbar_arrive_expect_tx(full_bar(pre), stage_bytes(pr, ta, kt));
+            arm(pre, stage_bytes(pr, ta, kt), 0);
             load_a(pre, pr, ta, kt);
-            armed[pre] = 0;
           }
         }
       }
@@ -351,13 +389,13 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
       bool ok = true;
       last_pr = -1;
       SegIter<kMaxProb> it;
-      it.init(g, blockIdx.x, grid);
+      it.init(g, unit, units);
       int pr, tile, kb, ke, seg;
-      while (ok && it.next(g, grid, pr, tile, kb, ke, seg)) {
+      while (ok && it.next(g, units, pr, tile, kb, ke, seg)) {
         if (pr != last_pr) {
           tma_prefetch_desc(&g.tm_a[pr]);
           tma_prefetch_desc(&g.tm_b[pr]);
-          if (C::kHybrid) tma_prefetch_desc(&g.tm_a2[pr]);
+          if (C::kHybrid || (kPair && C::kSparse)) tma_prefetch_desc(&g.tm_a2[pr]);
           last_pr = pr;
         }
         const int ta = tile % g.prob[pr].tiles_a, tb = tile / g.prob[pr].tiles_a;
@@ -370,10 +408,9 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
               *abort_flag = 1;
               break;
             }
-            mbar_arrive_expect_tx(full_bar(stage), stage_bytes(pr, ta, kt));
+            arm(stage, stage_bytes(pr, ta, kt), (int)phase);
             load_a(stage, pr, ta, kt);
             load_b(stage, pr, tb, kt);
-            armed[stage] = (int)phase;
           }
           if (++stage == S) {
             stage = 0;
@@ -381,26 +418,30 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
           }
         }
       }
-      // wait (bounded) until every copy this thread started has landed
+      // wait (bounded) until every copy counted on this CTA's barriers has landed
       for (int s = 0; s < S; ++s)
         if (armed[s] >= 0) mbar_wait(full_bar(s), (uint32_t)armed[s], p.timeout_ns, kDevErrWaitFull);
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc = make_idesc(C::kSparse, kBf16, kBlockA, kBN);
+    // ------------------------------------------------------------------ MMA issuer (rank 0 in a pair)
+    if (lane == 0 && rank == 0) {
+      const uint32_t idesc = make_idesc(C::kSparse, kBf16, C::kRowsA, kBN);
       const uint32_t idesc_dense = make_idesc(false, kBf16, kBlockA, kBN);
-      const uint32_t idesc_sp = make_idesc(true, kBf16, kBlockA, kBN);
+      const uint32_t idesc_sp = make_idesc(true, kBf16, C::kRowsA, kBN);
       const uint32_t meta_col0 = C::kAccCols;
+      const uint32_t s0 = smem_u32(smem);
+      const uint64_t da0 = smem_desc(s0, 16, 1024, kLayoutSw128);
+      const uint64_t db0 = smem_desc(s0 + C::kABytes, 16, 1024, kLayoutSw128);
+      const uint64_t dm0 = smem_desc(s0 + C::kABytes + C::kBBytes, 16, 128, kLayoutNone);
       int stage = 0;
       uint32_t phase = 0;
       uint32_t acc_i = 0;
       bool ok = true;
       SegIter<kMaxProb> it;
-      it.init(g, blockIdx.x, grid);
+      it.init(g, unit, units);
       int pr, tile, kb, ke, seg;
-      while (ok && it.next(g, grid, pr, tile, kb, ke, seg)) {
+      while (ok && it.next(g, units, pr, tile, kb, ke, seg)) {
         const GemmProblem& P = g.prob[pr];
         const int ta = tile % P.tiles_a;
         const int buf = acc_i & 1;
@@ -442,47 +483,74 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
               }
             }
           } else if (C::kSparse) {
-            const int chunks = meta_chunks(P, kt);
-            for (int c = 0; c < chunks; ++c)
-              tc_cp_128x128b(tmem_base + mcol + 4 * c, smem_desc(sm + c * 2048, 16, 128, kLayoutNone));
-            const int n_mma = kBf16 ? 4 : 2 * chunks;
-            for (int j = 0; j < n_mma; ++j) {
-              const uint64_t da = smem_desc(sa + j * 32, 16, 1024, kLayoutSw128);
-              const uint64_t db = smem_desc(sb + (j >> 1) * kBN * 128 + (j & 1) * 64, 16, 1024,
-                                            kLayoutSw128);
-              const uint32_t acc = (first && j == 0) ? 0u : 1u;
-              if (kBf16) {
-                // one 32-bit metadata column per k-block; the selector picks
-                // the odd column of an even-aligned pair
-                const uint32_t col = mcol + j;
-                mma_sp_bf16(d, da, db, tmem_base + (col & ~1u), idesc_sp | (col & 1u), acc);
-              } else {
-                // two metadata columns per k-block
-                const uint32_t col = mcol + 4 * (j >> 1) + 2 * (j & 1);
-                mma_sp_f8(d, da, db, tmem_base + col, idesc_sp, acc);
+            // descriptors of this stage: the stage-0 descriptors plus the
+            // stage offset (the address field counts 16-byte units)
+            const uint64_t so = (uint64_t)((uint32_t)stage * (uint32_t)(C::kStageBytes >> 4));
+            const uint64_t da = da0 + so, db = db0 + so, dm = dm0 + so;
+            auto issue = [&](auto chunks_c) {
+              constexpr int kChunks = decltype(chunks_c)::value;
+#pragma unroll
+              for (int c = 0; c < kChunks; ++c) {
+                if (kPair) tc_cp_128x128b_pair(tmem_base + mcol + 4 * c, dm + (uint64_t)(c * (2048 >> 4)));
+                else tc_cp_128x128b(tmem_base + mcol + 4 * c, dm + (uint64_t)(c * (2048 >> 4)));
               }
-            }
+              constexpr int kMmas = kBf16 ? 4 : 2 * kChunks;
+#pragma unroll
+              for (int j = 0; j < kMmas; ++j) {
+                const uint64_t a_d = da + (uint64_t)(j * (32 >> 4));
+                const uint64_t b_d = db + (uint64_t)(((j >> 1) * C::kBRows * 128 + (j & 1) * 64) >> 4);
+                const uint32_t acc = (first && j == 0) ? 0u : 1u;
+                if (kBf16) {
+                  // one 32-bit metadata column per k-block; the selector picks
+                  // the odd column of an even-aligned pair
+                  const uint32_t col = mcol + j;
+                  if (kPair) mma_sp_bf16_pair(d, a_d, b_d, tmem_base + (col & ~1u), idesc_sp | (col & 1u), acc);
+                  else mma_sp_bf16(d, a_d, b_d, tmem_base + (col & ~1u), idesc_sp | (col & 1u), acc);
+                } else {
+                  // two metadata columns per k-block
+                  const uint32_t col = mcol + 4 * (j >> 1) + 2 * (j & 1);
+                  if (kPair) mma_sp_f8_pair(d, a_d, b_d, tmem_base + col, idesc_sp, acc);
+                  else mma_sp_f8(d, a_d, b_d, tmem_base + col, idesc_sp, acc);
+                }
+              }
+            };
+            // a stage is whole except, for e4m3, a last stage of one 128-deep chunk
+            if (kBf16 || C::kMetaChunks == 1 || meta_chunks(P, kt) == C::kMetaChunks)
+              issue(std::integral_constant<int, C::kMetaChunks>{});
+            else
+              issue(std::integral_constant<int, 1>{});
           } else {
+            const uint64_t so = (uint64_t)((uint32_t)stage * (uint32_t)(C::kStageBytes >> 4));
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-              const uint64_t da = smem_desc(sa + j * 32, 16, 1024, kLayoutSw128);
-              const uint64_t db = smem_desc(sb + j * 32, 16, 1024, kLayoutSw128);
-              if (kBf16) mma_bf16(d, da, db, idesc, (first && j == 0) ? 0u : 1u);
-              else mma_f8(d, da, db, idesc, (first && j == 0) ? 0u : 1u);
+              const uint64_t da = da0 + so + (uint64_t)(j * (32 >> 4));
+              const uint64_t db = db0 + so + (uint64_t)(j * (32 >> 4));
+              const uint32_t acc = (first && j == 0) ? 0u : 1u;
+              if (kPair) {
+                if (kBf16) mma_bf16_pair(d, da, db, idesc, acc);
+                else mma_f8_pair(d, da, db, idesc, acc);
+              } else {
+                if (kBf16) mma_bf16(d, da, db, idesc, acc);
+                else mma_f8(d, da, db, idesc, acc);
+              }
             }
           }
-          tc_commit(empty_bar(stage));  // frees the stage once these MMAs are done
+          // frees the stage (in both CTAs of a pair) once these MMAs are done
+          if (kPair) tc_commit_pair(empty_bar(stage), 0x3);
+          else tc_commit(empty_bar(stage));
           if (++stage == S) {
             stage = 0;
             phase ^= 1;
           }
         }
         if (!ok) break;
-        tc_commit(accf_bar(buf));
+        if (kPair) tc_commit_pair(accf_bar(buf), 0x3);
+        else tc_commit(accf_bar(buf));
         ++acc_i;
       }
       // drain: every MMA and copy issued above has completed
-      tc_commit(drain_bar);
+      if (kPair) tc_commit_pair(drain_bar, 0x1);
+      else tc_commit(drain_bar);
       mbar_wait(drain_bar, 0, p.timeout_ns, kDevErrWaitDrain);
     }
     __syncwarp();
@@ -490,7 +558,7 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
     // ------------------------------------------------------------------ epilogue
     if (p.use_pdl) pdl_wait();                 // B scales and Y may belong to the upstream grid
     const int lg = warp & 3;                   // tensor-memory lane group of this warp
-    const int row = lg * 32 + lane;            // accumulator row (lane) within the tile
+    const int row = lg * 32 + lane;            // accumulator row (lane) within the CTA's half
     const int et = threadIdx.x - 64;           // 0..127
     uint32_t acc_i = 0;
     int cached_pr = -1, cached_tb = -1;
@@ -498,14 +566,14 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
     const int eb = p.out_f32 ? 4 : 2;
     const int per_vec = 16 / eb;                   // elements per 16-byte vector
     SegIter<kMaxProb> it;
-    it.init(g, blockIdx.x, grid);
+    it.init(g, unit, units);
     int pr, tile, kb, ke, seg;
-    while (it.next(g, grid, pr, tile, kb, ke, seg)) {
+    while (it.next(g, units, pr, tile, kb, ke, seg)) {
       const GemmProblem& P = g.prob[pr];
       const int ta = tile % P.tiles_a, tb = tile / P.tiles_a;
       const int buf = acc_i & 1;
       const uint32_t acc_phase = (acc_i >> 1) & 1;
-      const int ga = ta * kBlockA + row;     // global A row of this thread
+      const int ga = ta * C::kRowsA + (int)rank * kBlockA + row;  // global A row of this thread
       const bool a_live = ga < P.rows_a;
       // scales: loaded before waiting for the accumulator so their latency hides
       const float sa_v = (P.scale_a != nullptr && a_live) ? __ldg(P.scale_a + ga) : 1.0f;
@@ -529,8 +597,9 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
       tc_fence_after_sync();
       const uint32_t tbase = tmem_base + ((uint32_t)(lg * 32) << 16) + buf * kBN;
       const bool full = (kb == 0 && ke == P.num_kt);
-      // stream-K accumulator row of this thread: [tile][row][kBN] fp32
-      float* part = full ? nullptr : P.ws_accum + ((int64_t)tile * 128 + row) * kBN;
+      // stream-K accumulator row of this thread: [tile][pair half][row][kBN] fp32
+      const int64_t slot = (int64_t)tile * (kPair ? 2 : 1) + (int64_t)rank;
+      float* part = full ? nullptr : P.ws_accum + (slot * 128 + row) * kBN;
 
       // Scales and stores 16 consecutive accumulator columns starting at c0
       // with 16-byte vector stores.  Rows of Y are 16-byte aligned (checked
@@ -542,7 +611,7 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
           // lane = n (output feature), column = m (token).  Stage the warp's
           // 32 n x 16 m block transposed, then write each output row's 32
           // consecutive n as 16-byte vectors.
-          const int n0 = ta * kBlockA + lg * 32;
+          const int n0 = ta * C::kRowsA + (int)rank * kBlockA + lg * 32;
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const float y = v[i] * sa_v * s_scale_b[c0 + i];
@@ -605,20 +674,27 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
           store16(v, c0);
         }
       }
+      // the accumulator may be overwritten now (one arrive per warp; rank
+      // 0's barrier in a pair)
       tc_fence_before_sync();
-      mbar_arrive(acce_bar(buf));  // accumulator may be overwritten now
+      __syncwarp();
+      if (lane == 0) {
+        if (kPair) mbar_arrive_cluster(mapa_shared(acce_bar(buf), 0));
+        else mbar_arrive(acce_bar(buf));
+      }
       ++acc_i;
 
       if (part != nullptr) {
-        // The contributors of this tile are the CTAs whose iteration ranges
-        // cover it; the last to take a ticket finishes the tile.
+        // The contributors of this tile are the units whose iteration ranges
+        // cover it; the last to take a ticket finishes the tile (each half of
+        // a pair tile separately).
         const int64_t i0 = P.iter_begin + (int64_t)tile * P.num_kt;
-        const int c_first = sk_owner(p.total_iters, grid, i0);
-        const int c_last = sk_owner(p.total_iters, grid, i0 + P.num_kt - 1);
+        const int c_first = sk_owner(p.total_iters, units, i0);
+        const int c_last = sk_owner(p.total_iters, units, i0 + P.num_kt - 1);
         const unsigned int count = (unsigned int)(c_last - c_first + 1);
         named_bar_sync(1, 128);  // every partial add of this CTA precedes the ticket
         if (et == 0) {
-          const unsigned int old = atom_add_acq_rel_gpu(&P.ws_counters[tile], 1u);
+          const unsigned int old = atom_add_acq_rel_gpu(&P.ws_counters[slot], 1u);
           *last_flag = (old == count - 1) ? 1 : 0;
         }
         named_bar_sync(1, 128);
@@ -645,7 +721,7 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
               store16(v, cb + c0);
             }
           }
-          if (et == 0) P.ws_counters[tile] = 0u;  // ready for the next call
+          if (et == 0) P.ws_counters[slot] = 0u;  // ready for the next call
         }
         named_bar_sync(1, 128);
       }
@@ -654,9 +730,11 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
 
   tc_fence_before_sync();
   __syncthreads();
+  if (kPair) cluster_sync();  // neither CTA leaves while its peer may still use its memory
   if (warp == 1) {
     tc_fence_after_sync();
-    tmem_dealloc(tmem_base, C::kTmemCols);
+    if (kPair) tmem_dealloc_pair(tmem_base, C::kTmemCols);
+    else tmem_dealloc(tmem_base, C::kTmemCols);
   }
 }
 

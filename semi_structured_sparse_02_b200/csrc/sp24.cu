@@ -35,9 +35,12 @@ struct DeviceInfo {
   int checked = 0;
   int ok = 0;
   int sms = 0;
+  int pairs = 0;  // co-resident CTA pairs of the GEMM kernel
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
+
+int device_pairs(int dev);
 
 int current_device_info(DeviceInfo* out) {
   int dev = 0;
@@ -58,6 +61,7 @@ int current_device_info(DeviceInfo* out) {
     d.checked = 1;
     d.ok = (major == 10 && minor == 0);
     d.sms = sms;
+    d.pairs = d.ok ? device_pairs(dev) : 0;
   }
   if (!d.ok) return SP24_ERR_UNSUPPORTED_DEVICE;
   *out = d;
@@ -124,6 +128,7 @@ struct Plan {
   int mode;        // kModeDense / kModeSparse / kModeHybrid
   bool bf16;
   bool a_is_w;
+  bool pair;       // tiles of 256 weight rows on CTA pairs (cta_group::2)
   int bn;
   int kt;          // logical K per stage
   int n;           // problems
@@ -148,18 +153,19 @@ int stage_k(int mode, bool bf16) {
   return bf16 ? 64 : 128;
 }
 
-size_t sk_accum_bytes(const Plan& pl) {
-  return (size_t)pl.total_tiles * pl.bn * 128 * sizeof(float);
-}
+// stream-K accumulator slots: one per tile, or one per half of a pair tile
+size_t sk_slots(const Plan& pl) { return (size_t)pl.total_tiles * (pl.pair ? 2 : 1); }
+
+size_t sk_accum_bytes(const Plan& pl) { return sk_slots(pl) * pl.bn * 128 * sizeof(float); }
 
 size_t sk_ws_bytes(const Plan& pl) {
-  const size_t cnt = ((size_t)pl.total_tiles * sizeof(unsigned int) + 255) & ~(size_t)255;
+  const size_t cnt = (sk_slots(pl) * sizeof(unsigned int) + 255) & ~(size_t)255;
   return sk_accum_bytes(pl) + cnt;
 }
 
-// Work schedule, from a cost model in units of one K-stage of one SM
-// (streaming one stage of weights takes about the same time on every SM
-// when all SMs stream):
+// Work schedule, from a cost model in units of one K-stage of one scheduling
+// unit (an SM, or a CTA pair; streaming one stage of weights takes about the
+// same time on every unit when all units stream):
 //   whole tiles round-robin: ceil(tiles / SMs) * stages of the longest tile
 //   stream-K:                ceil(tiles * stages / SMs) + the cost of finishing
 //                            the split tiles (fp32 atomics into an accumulator,
@@ -205,15 +211,15 @@ void choose_schedule(Plan& pl, int sms, size_t ws_cap) {
 // ---------------------------------------------------------------------------
 // kernel launch for one instantiation
 // ---------------------------------------------------------------------------
-template <int kMode, bool kBf16, int kBN, bool kAIsW, int kMaxProb>
+template <int kMode, bool kBf16, int kBN, bool kAIsW, int kMaxProb, bool kPair = false>
 int launch_gemm_inst(const GemmLaunch<kMaxProb>& gl, int grid, cudaStream_t stream) {
-  using C = GemmCfg<kMode, kBf16, kBN>;
+  using C = GemmCfg<kMode, kBf16, kBN, kPair>;
   static std::atomic<uint64_t> attr_set{0};
   int dev = 0;
   cudaGetDevice(&dev);
   const uint64_t bit = 1ull << (dev & 63);
   if (!(attr_set.load() & bit)) {
-    if (cudaFuncSetAttribute(k_gemm<kMode, kBf16, kBN, kAIsW, kMaxProb>,
+    if (cudaFuncSetAttribute(k_gemm<kMode, kBf16, kBN, kAIsW, kMaxProb, kPair>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess) {
       cudaGetLastError();
       return SP24_ERR_CUDA;
@@ -221,16 +227,27 @@ int launch_gemm_inst(const GemmLaunch<kMaxProb>& gl, int grid, cudaStream_t stre
     attr_set.fetch_or(bit);
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
+  cfg.gridDim = dim3(kPair ? 2 * grid : grid);
   cfg.blockDim = dim3(kGemmThreads);
   cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (gl.p.use_pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  if (kPair) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = 2;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = gl.p.use_pdl ? 1 : 0;
-  return launch_result(cudaLaunchKernelEx(&cfg, k_gemm<kMode, kBf16, kBN, kAIsW, kMaxProb>, gl));
+  cfg.numAttrs = na;
+  return launch_result(cudaLaunchKernelEx(&cfg, k_gemm<kMode, kBf16, kBN, kAIsW, kMaxProb, kPair>, gl));
 }
 
 template <int kMode, bool kBf16, bool kAIsW, int kMaxProb>
@@ -244,7 +261,67 @@ int launch_gemm_bn(int bn, const GemmLaunch<kMaxProb>& gl, int grid, cudaStream_
   }
 }
 
+// Pair tiles (grid = pairs).  The sparse e4m3 pair MMA needs N >= 32.
+template <int kMode, bool kBf16, int kMaxProb>
+int launch_gemm_pair_bn(int bn, const GemmLaunch<kMaxProb>& gl, int pairs, cudaStream_t s) {
+  constexpr bool kNo16 = kMode == kModeSparse && !kBf16;
+  switch (bn) {
+    case 16:
+      if (kNo16) return SP24_ERR_INVALID_ARG;
+      return launch_gemm_inst<kMode, kBf16, kNo16 ? 32 : 16, true, kMaxProb, true>(gl, pairs, s);
+    case 32: return launch_gemm_inst<kMode, kBf16, 32, true, kMaxProb, true>(gl, pairs, s);
+    case 64: return launch_gemm_inst<kMode, kBf16, 64, true, kMaxProb, true>(gl, pairs, s);
+    case 128: return launch_gemm_inst<kMode, kBf16, 128, true, kMaxProb, true>(gl, pairs, s);
+    default: return SP24_ERR_INVALID_ARG;
+  }
+}
+
+template <int kMaxProb>
+int dispatch_pair(const Plan& pl, const GemmLaunch<kMaxProb>& gl, cudaStream_t s) {
+  if (pl.mode == kModeSparse)
+    return pl.bf16 ? launch_gemm_pair_bn<kModeSparse, true, kMaxProb>(pl.bn, gl, pl.grid, s)
+                   : launch_gemm_pair_bn<kModeSparse, false, kMaxProb>(pl.bn, gl, pl.grid, s);
+  if (pl.mode == kModeDense)
+    return pl.bf16 ? launch_gemm_pair_bn<kModeDense, true, kMaxProb>(pl.bn, gl, pl.grid, s)
+                   : launch_gemm_pair_bn<kModeDense, false, kMaxProb>(pl.bn, gl, pl.grid, s);
+  return SP24_ERR_DTYPE;
+}
+
+// How many CTA pairs of the GEMM kernel can be resident at once on the
+// current device (clusters are placed within a GPC, so this can be below
+// SMs / 2).  Every instantiation holds one CTA per SM, so one query serves all.
+int device_pairs(int dev) {
+  static std::atomic<int> cached[kMaxDevices];
+  if (dev < 0 || dev >= kMaxDevices) return 0;
+  int n = cached[dev].load();
+  if (n > 0) return n;
+  using C = GemmCfg<kModeSparse, false, 32, true>;
+  auto fn = k_gemm<kModeSparse, false, 32, true, 1, true>;
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  cudaLaunchConfig_t q = {};
+  q.gridDim = dim3(2);
+  q.blockDim = dim3(kGemmThreads);
+  q.dynamicSmemBytes = C::kSmemBytes;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  q.attrs = attr;
+  q.numAttrs = 1;
+  if (cudaOccupancyMaxActiveClusters(&n, fn, &q) != cudaSuccess || n < 1) {
+    cudaGetLastError();
+    return 0;
+  }
+  cached[dev].store(n);
+  return n;
+}
+
 int dispatch_gemm(const Plan& pl, const GemmLaunch<1>& gl, cudaStream_t s) {
+  if (pl.pair) return dispatch_pair(pl, gl, s);
   if (!pl.a_is_w) {
     if (pl.mode == kModeSparse && pl.bf16 && pl.bn == 128)
       return launch_gemm_inst<kModeSparse, true, 128, false, 1>(gl, pl.grid, s);
@@ -262,6 +339,7 @@ int dispatch_gemm(const Plan& pl, const GemmLaunch<1>& gl, cudaStream_t s) {
 }
 
 int dispatch_gemm_group(const Plan& pl, const GemmLaunch<kMaxGroup>& gl, cudaStream_t s) {
+  if (pl.pair) return dispatch_pair(pl, gl, s);
   if (pl.mode == kModeSparse)
     return pl.bf16 ? launch_gemm_bn<kModeSparse, true, true, kMaxGroup>(pl.bn, gl, pl.grid, s)
                    : launch_gemm_bn<kModeSparse, false, true, kMaxGroup>(pl.bn, gl, pl.grid, s);
@@ -312,7 +390,21 @@ int args_mode(const sp24_gemm_args* a) {
 }
 
 // Plans one launch over n (validated, mutually compatible) problems.
-Plan plan_group(const sp24_gemm_args* const* a, int n, int sms, size_t ws_cap) {
+// Token-count-limited launches (M <= 255) run on CTA pairs only when every
+// problem asks for it (SP24_GEMM_CTA_PAIR) and has at least 256 weight rows.
+// A pair's M = 256 MMA moves twice the weight bytes per tcgen05 instruction,
+// but only one of its two SMs issues, so in this weight-streaming regime pairs
+// and single CTAs reach about the same rate (single CTAs measured slightly
+// ahead), and single CTAs stay the default.
+bool want_pair(const sp24_gemm_args* const* a, int n, int mode, int pairs) {
+  if (mode == kModeHybrid || pairs < 1) return false;
+  for (int i = 0; i < n; ++i)
+    if (a[i]->N < 256 || (a[i]->flags & SP24_GEMM_CTA_PAIR) == 0 || (a[i]->flags & SP24_GEMM_SINGLE_CTA) != 0)
+      return false;
+  return true;
+}
+
+Plan plan_group(const sp24_gemm_args* const* a, int n, const DeviceInfo& di, size_t ws_cap) {
   Plan pl;
   memset(&pl, 0, sizeof pl);
   pl.bf16 = a[0]->in_dtype == SP24_BF16;
@@ -321,16 +413,19 @@ Plan plan_group(const sp24_gemm_args* const* a, int n, int sms, size_t ws_cap) {
   pl.bn = pick_bn(a[0]->M);
   pl.kt = stage_k(pl.mode, pl.bf16);
   pl.n = n;
+  pl.pair = want_pair(a, n, pl.mode, di.pairs);
+  if (pl.pair && pl.mode == kModeSparse && !pl.bf16 && pl.bn < 32) pl.bn = 32;  // sparse e4m3 pair: N >= 32
+  const int rows_a = pl.pair ? 2 * kBlockA : kBlockA;
   for (int i = 0; i < n; ++i) {
     pl.num_kt[i] = (int)((a[i]->K + pl.kt - 1) / pl.kt);
-    pl.tiles_a[i] = (int)((a[i]->N + kBlockA - 1) / kBlockA);
+    pl.tiles_a[i] = (int)((a[i]->N + rows_a - 1) / rows_a);
     pl.tiles_b[i] = (int)((a[i]->M + pl.bn - 1) / pl.bn);
   }
-  choose_schedule(pl, sms, ws_cap);
+  choose_schedule(pl, pl.pair ? di.pairs : di.sms, ws_cap);
   return pl;
 }
 
-Plan plan_gemm(const sp24_gemm_args* a, int sms, size_t ws_cap) { return plan_group(&a, 1, sms, ws_cap); }
+Plan plan_gemm(const sp24_gemm_args* a, const DeviceInfo& di, size_t ws_cap) { return plan_group(&a, 1, di, ws_cap); }
 
 // Tensor maps and problem record of problem i of a launch.
 template <int kMaxProb>
@@ -346,16 +441,25 @@ bool fill_problem(GemmLaunch<kMaxProb>& gl, int i, const sp24_gemm_args* a, cons
   } else if (pl.mode == kModeSparse) {
     ok &= make_map(&gl.tm_a[i], a->W, eb, a->K / 2, a->N, a->ldw * eb, box_elems, kBlockA,
                    CU_TENSOR_MAP_SWIZZLE_128B);
-    gl.tm_a2[i] = gl.tm_a[i];
+    if (pl.pair) {
+      // the metadata image as rows of 256 bytes (8 per 2048-byte chunk), read
+      // by TMA so that both CTAs of a pair count on one barrier
+      const int chunks = pl.bf16 ? 1 : 2;
+      const uint64_t meta_rows = (uint64_t)((a->N + 127) / 128) * (uint64_t)(a->K / 128) * 8;
+      ok &= make_map(&gl.tm_a2[i], a->W_meta, 1, 256, meta_rows, 256, 256, 8 * chunks, CU_TENSOR_MAP_SWIZZLE_NONE);
+    } else {
+      gl.tm_a2[i] = gl.tm_a[i];
+    }
   } else {
     ok &= make_map(&gl.tm_a[i], a->W_dense_tiles, 1, a->K, a->N, a->K, 128, kBlockA,
                    CU_TENSOR_MAP_SWIZZLE_128B);
     ok &= make_map(&gl.tm_a2[i], a->W, 1, a->K / 2, a->N, a->ldw, 64, kBlockA, CU_TENSOR_MAP_SWIZZLE_64B);
   }
-  ok &= make_map(&gl.tm_b[i], a->X, eb, a->K, a->M, a->ldx * eb, box_elems, pl.bn,
+  ok &= make_map(&gl.tm_b[i], a->X, eb, a->K, a->M, a->ldx * eb, box_elems, pl.pair ? pl.bn / 2 : pl.bn,
                  CU_TENSOR_MAP_SWIZZLE_128B);
   GemmProblem& P = gl.prob[i];
   memset(&P, 0, sizeof P);
+  P.meta_blocks = (int32_t)((a->N + 127) / 128);
   P.rows_a = (int32_t)a->N;
   P.rows_b = (int32_t)a->M;
   P.K = (int32_t)a->K;
@@ -393,8 +497,9 @@ int build_launch(GemmLaunch<kMaxProb>& gl, const sp24_gemm_args* const* a, int n
     if (!fill_problem(gl, i, a[i], pl, iter, tile, sk ? accum : nullptr, sk ? counters : nullptr))
       return SP24_ERR_CUDA;
     if (sk) {
-      accum += (size_t)tiles * pl.bn * 128;
-      counters += tiles;
+      const size_t slots = (size_t)tiles * (pl.pair ? 2 : 1);
+      accum += slots * pl.bn * 128;
+      counters += slots;
     }
     iter += (int64_t)tiles * pl.num_kt[i];
     tile += tiles;
@@ -527,7 +632,7 @@ int run_gemm(const sp24_gemm_args* a, cudaStream_t stream) {
   if (st != SP24_OK) return st;
   size_t ws_cap = a->workspace != nullptr ? a->workspace_bytes : 0;
   if (a->workspace != nullptr && !aligned16(a->workspace)) return SP24_ERR_ALIGNMENT;
-  const Plan pl = plan_gemm(a, di.sms, ws_cap);
+  const Plan pl = plan_gemm(a, di, ws_cap);
   GemmLaunch<1> gl;
   if ((st = build_launch(gl, &a, 1, pl, a->workspace, (a->flags & SP24_GEMM_W_STATIC) != 0)) != SP24_OK)
     return st;
@@ -765,7 +870,7 @@ int sp24_quantize_e4m3_rows_grouped(const sp24_quant_item* items, int n_items, v
   DeviceInfo di;
   int st = current_device_info(&di);
   if (st != SP24_OK) return st;
-  const int grid = (int)std::min<int64_t>(g.row_start[n_items], (int64_t)di.sms * 4);
+  const int grid = (int)std::min<int64_t>(g.row_start[n_items], (int64_t)di.sms * kQuantCtasPerSm);
   return launch_pdl(k_quantize_rows_e4m3, dim3(grid), dim3(kQuantThreads), 0,
                     static_cast<cudaStream_t>(stream), g);
 }
@@ -775,7 +880,7 @@ size_t sp24_gemm_workspace_bytes(const sp24_gemm_args* a) {
   DeviceInfo di;
   if (current_device_info(&di) != SP24_OK) return 0;
   if (use_pair(a->N, a->M, a->tile_dense_mask != nullptr, a->flags)) return 0;
-  Plan pl = plan_gemm(a, di.sms, (size_t)-1);
+  Plan pl = plan_gemm(a, di, (size_t)-1);
   return pl.ws_bytes;
 }
 
@@ -791,7 +896,7 @@ size_t sp24_gemm_grouped_workspace_bytes(const sp24_gemm_args* args, int n) {
   if (current_device_info(&di) != SP24_OK) return 0;
   const sp24_gemm_args* ptrs[kMaxGroup];
   for (int i = 0; i < n; ++i) ptrs[i] = &args[i];
-  return plan_group(ptrs, n, di.sms, (size_t)-1).ws_bytes;
+  return plan_group(ptrs, n, di, (size_t)-1).ws_bytes;
 }
 
 int sp24_gemm_grouped(const sp24_gemm_args* args, int n, void* workspace, size_t workspace_bytes,
@@ -807,7 +912,7 @@ int sp24_gemm_grouped(const sp24_gemm_args* args, int n, void* workspace, size_t
     ptrs[i] = &args[i];
     w_static = w_static && (args[i].flags & SP24_GEMM_W_STATIC) != 0;
   }
-  const Plan pl = plan_group(ptrs, n, di.sms, workspace != nullptr ? workspace_bytes : 0);
+  const Plan pl = plan_group(ptrs, n, di, workspace != nullptr ? workspace_bytes : 0);
   static thread_local GemmLaunch<kMaxGroup> gl;  // large: keep it off the stack
   if ((st = build_launch(gl, ptrs, n, pl, workspace, w_static)) != SP24_OK) return st;
   return dispatch_gemm_group(pl, gl, static_cast<cudaStream_t>(stream));
@@ -819,7 +924,7 @@ int sp24_gemm_noalloc(const sp24_gemm_args* a, void* stream) {
   DeviceInfo di;
   if ((st = current_device_info(&di)) != SP24_OK) return st;
   // The same schedule sp24_gemm picks with an unlimited workspace.
-  const Plan pl = plan_gemm(a, di.sms, (size_t)-1);
+  const Plan pl = plan_gemm(a, di, (size_t)-1);
   if (pl.ws_bytes > kStaticScratchBytes) return SP24_ERR_WORKSPACE;
   void* scratch = nullptr;
   if ((st = static_scratch(&scratch)) != SP24_OK) return st;

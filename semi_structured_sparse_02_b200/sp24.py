@@ -34,6 +34,7 @@ BF16, E4M3, F32 = 0, 1, 2
 SPARSE, DENSE = 0, 1
 GEMM_W_STATIC = 1
 GEMM_SINGLE_CTA = 2
+GEMM_CTA_PAIR = 4
 
 
 class Sp24Error(RuntimeError):

@@ -306,6 +306,17 @@ def test_grouped_gemm_sixteen_problems_w_static_reusable():
         assert int(grp.workspace.view(torch.int32).abs().sum().item()) == 0
 
 
+@pytest.mark.parametrize("e4", [False, True])
+def test_grouped_gemm_cta_pairs(e4):
+    # the decode group on CTA pairs (ragged N: 384 and 640 leave the second
+    # CTA of the last pair tile past the end)
+    shapes = [(8, 1024, 4096), (5, 384, 512), (16, 640, 2048), (1, 256, 1280)]
+    flags = sp24.GEMM_CTA_PAIR | sp24.GEMM_W_STATIC
+    for use_ws in (True, False):
+        _, items = run_group(shapes, e4, sp24.SPARSE, True, use_ws=use_ws, flags=flags, seed=17)
+        check_group(items, "pair group ws=%s" % use_ws)
+
+
 def test_group_of_one_matches_single_gemm():
     X, W = inputs.linear_pair(8, 1024, 4096, seed=123)
     a, Y, y_ref, a_ref = prepare_gemm(X, W, True, sp24.SPARSE, True)
@@ -403,6 +414,22 @@ def test_pair_kernel_parity(M, N, K, e4, tactic):
     # the one-CTA kernel on the same operands agrees to the same tolerance
     y1, _, _, _, _ = run_gemm(X, W, e4, tactic, True, flags=sp24.GEMM_SINGLE_CTA)
     check_tolerance(y1, y_ref, a_ref, "single-CTA M%d N%d K%d" % (M, N, K))
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 384, 2048), (8, 1024, 4096), (16, 2560, 1280), (40, 640, 768),
+                                   (128, 1280, 5120)])
+@pytest.mark.parametrize("e4", [False, True])
+@pytest.mark.parametrize("tactic", [sp24.SPARSE, sp24.DENSE])
+def test_decode_pair_tiles_and_single_cta_agree(M, N, K, e4, tactic):
+    # with GEMM_CTA_PAIR, M <= 255 and N >= 256 run 256-row tiles on CTA pairs
+    # (stream-K when the tiles are few); the default one-CTA tiles must agree
+    # to the same tolerance
+    X, W = inputs.linear_pair(M, N, K, seed=M * 3 + N, outliers=True)
+    pair = sp24.GEMM_CTA_PAIR
+    for flags in (0, sp24.GEMM_W_STATIC, pair, pair | sp24.GEMM_W_STATIC):
+        y, y_ref, a_ref, _, _ = run_gemm(X, W, e4, tactic, True, flags=flags)
+        check_tolerance(y, y_ref, a_ref, "decode M%d N%d K%d e4=%s tactic=%d flags=%d"
+                        % (M, N, K, e4, tactic, flags))
 
 
 @pytest.mark.parametrize("e4", [False, True])
