@@ -201,15 +201,17 @@ typedef struct sp24_gemm_args {
 #define SP24_GEMM_CTA_PAIR 4u
 
 /* Bytes of workspace the call would use for its stream-K schedule (0 if the
- * shape needs none).  Shapes with fewer than two output tiles per SM split
- * the tiles' K range evenly over all SMs; the parts of a split tile are added
- * with fp32 atomics into a per-tile accumulator in the workspace, so their
- * fp32 summation order (and the last bits of those outputs) can vary from
- * run to run.  With a smaller or missing workspace the call falls back to
- * whole tiles per CTA (fewer SMs busy on such shapes).  The workspace must
- * be zero-filled once before its first use; every call that returns SP24_OK
- * leaves it zero again.  Calls that share a workspace must not overlap on
- * the GPU. */
+ * shape needs none).  Shapes with few output tiles per SM may split the
+ * tiles' K range evenly over all SMs (a cost model decides); a split tile is
+ * finished by the contributor that arrives last, which adds the others'
+ * fp32 partial tiles (stored in the workspace) to its own.  Which
+ * contributor finishes can vary from run to run, and with it the fp32
+ * summation order (the last bits of those outputs).  With a smaller or
+ * missing workspace the call falls back to whole tiles per CTA (fewer SMs
+ * busy on such shapes).  The workspace must be zero-filled once before its
+ * first use; every call that returns SP24_OK leaves its state (the leading
+ * sp24_gemm_workspace_state_bytes) zero again.  Calls that share a workspace
+ * must not overlap on the GPU. */
 size_t sp24_gemm_workspace_bytes(const sp24_gemm_args *args);
 
 /* Y = s_x[m] * s_w[n] * sum_k x[m,k] * w[n,k] (scales only for E4M3), fp32
@@ -231,6 +233,14 @@ int sp24_gemm(const sp24_gemm_args *args, void *stream);
  * SP24_GEMM_W_STATIC applies when every problem sets it. */
 int sp24_gemm_grouped(const sp24_gemm_args *args, int n, void *workspace_dev, size_t workspace_bytes,
                       void *stream);
+
+/* Leading bytes of the workspace that hold the stream-K state (arrival
+ * counters and partial-tile flags): zero before the first call, and zero
+ * again after every call that returns SP24_OK.  The rest of the workspace
+ * holds partial tiles whose contents never matter between calls.  0 when the
+ * call's schedule needs no workspace. */
+size_t sp24_gemm_workspace_state_bytes(const sp24_gemm_args *args);
+size_t sp24_gemm_grouped_workspace_state_bytes(const sp24_gemm_args *args, int n);
 
 size_t sp24_gemm_grouped_workspace_bytes(const sp24_gemm_args *args, int n);
 

@@ -16,11 +16,13 @@
 // decode): the K-iterations of all tiles of all problems are laid end to end
 // and every CTA streams one equal contiguous range of them, so every SM moves
 // the same number of bytes and a group streams without gaps between problems.
-// The contributors of a tile split between CTAs add their fp32 partial sums
-// into one accumulator tile with vector atomics (red.global.add.v4.f32, no
-// waiting on the L2 round trip); the last one to take a ticket scales,
-// converts and stores the tile and zeroes the accumulator for the next call.
-// The fp32 addition order of a split tile therefore varies between runs.
+// A tile split between CTAs is finished by whichever contributor takes the
+// last ticket: every other contributor stores its fp32 partial tile with
+// plain stores into a slot of its own (a unit has at most two split tiles,
+// its first and its last segment) and raises a flag; the last one adds those
+// partials to its own accumulator as it drains tensor memory, stores Y and
+// clears the flags and the ticket for the next call.  Which contributor
+// finishes varies between runs, and with it the fp32 addition order.
 //
 // Kernel chaining.  Every CTA triggers the dependent grid at once
 // (programmatic dependent launch).  With w_static the producer starts
@@ -65,8 +67,7 @@ struct GemmProblem {
   const float* scale_b;       // per-B-row scale (E4M3) or null
   void* Y;
   int64_t ldy;
-  float* ws_accum;            // stream-K fp32 accumulators [tiles][128 rows][BN]
-  unsigned int* ws_counters;  // stream-K arrival counters [tiles]
+  unsigned int* ws_counters;  // stream-K arrival counters [tiles (x2 halves in a pair)]
 };
 
 struct GemmParams {
@@ -78,6 +79,8 @@ struct GemmParams {
   int32_t use_pdl;            // wait on the upstream grid before dependent loads
   int32_t w_static;           // A operands are not written by the upstream grid
   uint64_t timeout_ns;
+  float* sk_slots;            // stream-K partial tiles [units][pair half][2][128 rows][BN] fp32
+  unsigned int* sk_flags;     // "partial stored" flags [units][pair half][2]
 };
 
 // Everything a launch needs, passed by value (tensor maps must live in
@@ -148,6 +151,15 @@ __device__ __forceinline__ bool named_bar_red_and(int id, int count, bool pred) 
 __device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
                : "memory");
+}
+
+__device__ __forceinline__ void st_release_gpu(unsigned int* p, unsigned int v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int* p) {
+  unsigned int v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
 }
 
 // GPU-scope acquire-release fetch-add: publishes (with the preceding CTA
@@ -597,9 +609,6 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
       tc_fence_after_sync();
       const uint32_t tbase = tmem_base + ((uint32_t)(lg * 32) << 16) + buf * kBN;
       const bool full = (kb == 0 && ke == P.num_kt);
-      // stream-K accumulator row of this thread: [tile][pair half][row][kBN] fp32
-      const int64_t slot = (int64_t)tile * (kPair ? 2 : 1) + (int64_t)rank;
-      float* part = full ? nullptr : P.ws_accum + (slot * 128 + row) * kBN;
 
       // Scales and stores 16 consecutive accumulator columns starting at c0
       // with 16-byte vector stores.  Rows of Y are 16-byte aligned (checked
@@ -657,74 +666,139 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
         }
       };
 
+      // the accumulator may be overwritten now (one arrive per warp; rank
+      // 0's barrier in a pair)
+      auto release_acc = [&]() {
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) {
+          if (kPair) mbar_arrive_cluster(mapa_shared(acce_bar(buf), 0));
+          else mbar_arrive(acce_bar(buf));
+        }
+      };
+
+      if (full) {
 #pragma unroll 1
-      for (int c0 = 0; c0 < kBN; c0 += 16) {
-        uint32_t r[16];
-        tmem_ld_x16(tbase + c0, r);
-        tmem_ld_wait();
-        if (part != nullptr) {
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            red_add_v4(part + c0 + 4 * j, __uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
-                       __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
-        } else {
+        for (int c0 = 0; c0 < kBN; c0 += 16) {
+          uint32_t r[16];
+          tmem_ld_x16(tbase + c0, r);
+          tmem_ld_wait();
           float v[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
           store16(v, c0);
         }
-      }
-      // the accumulator may be overwritten now (one arrive per warp; rank
-      // 0's barrier in a pair)
-      tc_fence_before_sync();
-      __syncwarp();
-      if (lane == 0) {
-        if (kPair) mbar_arrive_cluster(mapa_shared(acce_bar(buf), 0));
-        else mbar_arrive(acce_bar(buf));
-      }
-      ++acc_i;
-
-      if (part != nullptr) {
-        // The contributors of this tile are the units whose iteration ranges
-        // cover it; the last to take a ticket finishes the tile (each half of
-        // a pair tile separately).
+        release_acc();
+      } else {
+        // a split tile: its contributors are the units whose ranges cover it
         const int64_t i0 = P.iter_begin + (int64_t)tile * P.num_kt;
         const int c_first = sk_owner(p.total_iters, units, i0);
         const int c_last = sk_owner(p.total_iters, units, i0 + P.num_kt - 1);
         const unsigned int count = (unsigned int)(c_last - c_first + 1);
-        named_bar_sync(1, 128);  // every partial add of this CTA precedes the ticket
+        const int64_t cslot = (int64_t)tile * (kPair ? 2 : 1) + (int64_t)rank;
+        // slot s of unit u: 0 for the unit's first segment, 1 for its last
+        auto slot_idx = [&](int u, int sidx) { return ((int64_t)u * (kPair ? 2 : 1) + (int64_t)rank) * 2 + sidx; };
+        // the other contributor v's segment of this tile is v's first one
+        // exactly when v's range starts inside the tile
+        auto slot_of = [&](int v) { return ((int64_t)v * p.total_iters / units) >= i0 ? 0 : 1; };
+        named_bar_sync(1, 128);
         if (et == 0) {
-          const unsigned int old = atom_add_acq_rel_gpu(&P.ws_counters[slot], 1u);
+          const unsigned int old = atom_add_acq_rel_gpu(&P.ws_counters[cslot], 1u);
           *last_flag = (old == count - 1) ? 1 : 0;
         }
         named_bar_sync(1, 128);
-        if (*last_flag) {
-          // all loads of a 64-column block in flight at once, then store and
-          // zero the accumulator for the next call
+        if (!*last_flag) {
+          // store the partial tile (plain stores), then raise the flag
+          const int64_t my = slot_idx(unit, seg == 0 ? 0 : 1);
+          float* dst = p.sk_slots + (my * 128 + row) * kBN;
+#pragma unroll 1
+          for (int c0 = 0; c0 < kBN; c0 += 16) {
+            uint32_t r[16];
+            tmem_ld_x16(tbase + c0, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              __stcg(reinterpret_cast<float4*>(dst + c0) + j,
+                     make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                 __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3])));
+          }
+          release_acc();
+          named_bar_sync(1, 128);  // every store of the tile precedes the flag
+          if (et == 0) {
+            __threadfence();
+            st_release_gpu(p.sk_flags + my, 1u);
+          }
+        } else {
+          // wait (bounded) for the other contributors' flags
+          bool ok2 = true;
+          if (et == 0) {
+            for (int v = c_first; v <= c_last && ok2; ++v) {
+              if (v == unit) continue;
+              const unsigned int* f = p.sk_flags + slot_idx(v, slot_of(v));
+              if (ld_acquire_gpu(f) == 0u) {
+                const uint64_t t0 = globaltimer_ns();
+                while (ld_acquire_gpu(f) == 0u) {
+                  if (globaltimer_ns() - t0 > p.timeout_ns) {
+                    record_dev_error(kDevErrWaitCounter);
+                    ok2 = false;
+                    break;
+                  }
+                }
+              }
+            }
+            *last_flag = ok2 ? 1 : 2;
+          }
+          named_bar_sync(1, 128);
+          const bool have = *last_flag == 1;
+          // our accumulator plus the others' partials, 64 columns at a time
           constexpr int kFix = kBN < 64 ? kBN : 64;
 #pragma unroll 1
           for (int cb = 0; cb < kBN; cb += kFix) {
             float4 q[kFix / 4];
 #pragma unroll
-            for (int j = 0; j < kFix / 4; ++j) q[j] = __ldcg(reinterpret_cast<const float4*>(part + cb) + j);
+            for (int j = 0; j < kFix / 4; ++j) q[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (have) {
+              for (int v = c_first; v <= c_last; ++v) {
+                if (v == unit) continue;
+                const float* src = p.sk_slots + (slot_idx(v, slot_of(v)) * 128 + row) * kBN + cb;
+                float4 t[kFix / 4];
 #pragma unroll
-            for (int j = 0; j < kFix / 4; ++j)
-              __stcg(reinterpret_cast<float4*>(part + cb) + j, make_float4(0.f, 0.f, 0.f, 0.f));
+                for (int j = 0; j < kFix / 4; ++j) t[j] = __ldcg(reinterpret_cast<const float4*>(src) + j);
+#pragma unroll
+                for (int j = 0; j < kFix / 4; ++j) {
+                  q[j].x += t[j].x; q[j].y += t[j].y; q[j].z += t[j].z; q[j].w += t[j].w;
+                }
+              }
+            }
 #pragma unroll
             for (int c0 = 0; c0 < kFix; c0 += 16) {
+              uint32_t r[16];
+              tmem_ld_x16(tbase + cb + c0, r);
+              tmem_ld_wait();
               float v[16];
 #pragma unroll
               for (int j = 0; j < 4; ++j) {
                 const float4 t = q[c0 / 4 + j];
-                v[4 * j] = t.x; v[4 * j + 1] = t.y; v[4 * j + 2] = t.z; v[4 * j + 3] = t.w;
+                v[4 * j] = __uint_as_float(r[4 * j]) + t.x;
+                v[4 * j + 1] = __uint_as_float(r[4 * j + 1]) + t.y;
+                v[4 * j + 2] = __uint_as_float(r[4 * j + 2]) + t.z;
+                v[4 * j + 3] = __uint_as_float(r[4 * j + 3]) + t.w;
               }
               store16(v, cb + c0);
             }
           }
-          if (et == 0) P.ws_counters[slot] = 0u;  // ready for the next call
+          release_acc();
+          named_bar_sync(1, 128);  // every read of the partials precedes the reset
+          if (et == 0) {
+            // ready for the next call
+            for (int v = c_first; v <= c_last; ++v)
+              if (v != unit) p.sk_flags[slot_idx(v, slot_of(v))] = 0u;
+            P.ws_counters[cslot] = 0u;
+          }
+          if (!have) *abort_flag = 1;
         }
-        named_bar_sync(1, 128);
       }
+      ++acc_i;
     }
   }
 

@@ -9,6 +9,7 @@
 #include <atomic>
 #include <chrono>
 #include <cmath>
+#include <cstddef>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -153,15 +154,20 @@ int stage_k(int mode, bool bf16) {
   return bf16 ? 64 : 128;
 }
 
-// stream-K accumulator slots: one per tile, or one per half of a pair tile
-size_t sk_slots(const Plan& pl) { return (size_t)pl.total_tiles * (pl.pair ? 2 : 1); }
+// Stream-K workspace: two partial-tile slots per scheduling unit (and pair
+// half), a flag per slot, and an arrival counter per tile (and pair half).
+size_t sk_slot_count(const Plan& pl) { return (size_t)pl.grid * (pl.pair ? 2 : 1) * 2; }
+size_t round256(size_t b) { return (b + 255) & ~(size_t)255; }
+size_t sk_slots_bytes(const Plan& pl) { return round256(sk_slot_count(pl) * pl.bn * 128 * sizeof(float)); }
+size_t sk_flags_bytes(const Plan& pl) { return round256(sk_slot_count(pl) * sizeof(unsigned int)); }
 
-size_t sk_accum_bytes(const Plan& pl) { return sk_slots(pl) * pl.bn * 128 * sizeof(float); }
-
-size_t sk_ws_bytes(const Plan& pl) {
-  const size_t cnt = (sk_slots(pl) * sizeof(unsigned int) + 255) & ~(size_t)255;
-  return sk_accum_bytes(pl) + cnt;
+size_t sk_counters_bytes(const Plan& pl) {
+  return round256((size_t)pl.total_tiles * (pl.pair ? 2 : 1) * sizeof(unsigned int));
 }
+// Layout: [counters][flags][partial-tile slots]; the first two are the state
+// that must be zero between calls.
+size_t sk_state_bytes(const Plan& pl) { return sk_counters_bytes(pl) + sk_flags_bytes(pl); }
+size_t sk_ws_bytes(const Plan& pl) { return sk_state_bytes(pl) + sk_slots_bytes(pl); }
 
 // Work schedule, from a cost model in units of one K-stage of one scheduling
 // unit (an SM, or a CTA pair; streaming one stage of weights takes about the
@@ -430,7 +436,7 @@ Plan plan_gemm(const sp24_gemm_args* a, const DeviceInfo& di, size_t ws_cap) { r
 // Tensor maps and problem record of problem i of a launch.
 template <int kMaxProb>
 bool fill_problem(GemmLaunch<kMaxProb>& gl, int i, const sp24_gemm_args* a, const Plan& pl,
-                  int64_t iter_begin, int tile_begin, float* accum, unsigned int* counters) {
+                  int64_t iter_begin, int tile_begin, unsigned int* counters) {
   const int eb = dtype_bytes(a->in_dtype);
   const int box_elems = 128 / eb;  // 128 bytes
   bool ok = true;
@@ -474,7 +480,6 @@ bool fill_problem(GemmLaunch<kMaxProb>& gl, int i, const sp24_gemm_args* a, cons
   P.scale_b = a->in_dtype == SP24_E4M3 ? a->x_scales : nullptr;
   P.Y = a->Y;
   P.ldy = a->ldy;
-  P.ws_accum = accum;
   P.ws_counters = counters;
   return ok;
 }
@@ -486,24 +491,18 @@ int build_launch(GemmLaunch<kMaxProb>& gl, const sp24_gemm_args* const* a, int n
   memset(&gl, 0, sizeof gl);
   int64_t iter = 0;
   int tile = 0;
-  float* accum = static_cast<float*>(workspace);
-  unsigned int* counters =
-      pl.sched == kSchedStreamK
-          ? reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(workspace) + sk_accum_bytes(pl))
-          : nullptr;
+  const bool sk = pl.sched == kSchedStreamK;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  unsigned int* counters = sk ? reinterpret_cast<unsigned int*>(ws) : nullptr;
   for (int i = 0; i < n; ++i) {
     const int tiles = pl.tiles_a[i] * pl.tiles_b[i];
-    const bool sk = pl.sched == kSchedStreamK;
-    if (!fill_problem(gl, i, a[i], pl, iter, tile, sk ? accum : nullptr, sk ? counters : nullptr))
-      return SP24_ERR_CUDA;
-    if (sk) {
-      const size_t slots = (size_t)tiles * (pl.pair ? 2 : 1);
-      accum += slots * pl.bn * 128;
-      counters += slots;
-    }
+    if (!fill_problem(gl, i, a[i], pl, iter, tile, sk ? counters : nullptr)) return SP24_ERR_CUDA;
+    if (sk) counters += (size_t)tiles * (pl.pair ? 2 : 1);
     iter += (int64_t)tiles * pl.num_kt[i];
     tile += tiles;
   }
+  gl.p.sk_flags = sk ? reinterpret_cast<unsigned int*>(ws + sk_counters_bytes(pl)) : nullptr;
+  gl.p.sk_slots = sk ? reinterpret_cast<float*>(ws + sk_state_bytes(pl)) : nullptr;
   gl.p.n_prob = n;
   gl.p.sched = pl.sched;
   gl.p.total_iters = pl.total_iters;
@@ -514,6 +513,82 @@ int build_launch(GemmLaunch<kMaxProb>& gl, const sp24_gemm_args* const* a, int n
   gl.p.timeout_ns = g_timeout_ns.load();
   return SP24_OK;
 }
+
+// ---------------------------------------------------------------------------
+// Launch cache.  Planning a GEMM and encoding its tensor maps costs the host
+// ~2-5 us per map; a repeated call with byte-identical arguments (the common
+// case for a model's static layers) reuses the filled launch instead.  The
+// key is every byte of the argument blocks plus the device, the workspace and
+// the wait bound, so a hit launches exactly what a miss would have built.
+// ---------------------------------------------------------------------------
+struct LaunchKey {
+  int dev;
+  int n;
+  uint64_t timeout;
+  const void* ws;
+  size_t ws_bytes;
+  sp24_gemm_args a[kMaxGroup];
+};
+
+template <class Value, int kEntries>
+struct LaunchCache {
+  struct Entry {
+    bool valid = false;
+    size_t key_bytes = 0;
+    LaunchKey key;
+    Value val;
+  };
+  std::mutex mu;
+  Entry e[kEntries];
+  int next = 0;
+
+  static size_t key_size(int n) { return offsetof(LaunchKey, a) + (size_t)n * sizeof(sp24_gemm_args); }
+
+  // Runs fn(value) on a cached value for this key (true), or returns false.
+  template <class Fn>
+  bool find(const LaunchKey& k, Fn&& fn) {
+    const size_t kb = key_size(k.n);
+    std::lock_guard<std::mutex> lk(mu);
+    for (auto& x : e)
+      if (x.valid && x.key_bytes == kb && memcmp(&x.key, &k, kb) == 0) {
+        fn(x.val);
+        return true;
+      }
+    return false;
+  }
+  void put(const LaunchKey& k, const Value& v) {
+    std::lock_guard<std::mutex> lk(mu);
+    Entry& x = e[next];
+    next = (next + 1) % kEntries;
+    x.key_bytes = key_size(k.n);
+    memcpy(&x.key, &k, x.key_bytes);
+    x.val = v;
+    x.valid = true;
+  }
+};
+
+LaunchKey make_key(const sp24_gemm_args* a, int n, const void* ws, size_t ws_bytes) {
+  LaunchKey k;
+  memset(&k, 0, sizeof k);
+  cudaGetDevice(&k.dev);
+  k.n = n;
+  k.timeout = g_timeout_ns.load();
+  k.ws = ws;
+  k.ws_bytes = ws_bytes;
+  memcpy(k.a, a, (size_t)n * sizeof(sp24_gemm_args));
+  return k;
+}
+
+struct SingleLaunch {
+  Plan pl;
+  GemmLaunch<1> gl;
+};
+struct GroupLaunch {
+  Plan pl;
+  GemmLaunch<kMaxGroup> gl;
+};
+LaunchCache<SingleLaunch, 32> g_cache_single;
+LaunchCache<GroupLaunch, 16> g_cache_group;
 
 // ---------------------------------------------------------------------------
 // The CTA-pair kernel (256 x 256 tiles) for large token counts
@@ -632,11 +707,14 @@ int run_gemm(const sp24_gemm_args* a, cudaStream_t stream) {
   if (st != SP24_OK) return st;
   size_t ws_cap = a->workspace != nullptr ? a->workspace_bytes : 0;
   if (a->workspace != nullptr && !aligned16(a->workspace)) return SP24_ERR_ALIGNMENT;
-  const Plan pl = plan_gemm(a, di, ws_cap);
-  GemmLaunch<1> gl;
-  if ((st = build_launch(gl, &a, 1, pl, a->workspace, (a->flags & SP24_GEMM_W_STATIC) != 0)) != SP24_OK)
+  const LaunchKey key = make_key(a, 1, nullptr, 0);
+  if (g_cache_single.find(key, [&](const SingleLaunch& v) { st = dispatch_gemm(v.pl, v.gl, stream); })) return st;
+  static thread_local SingleLaunch v;
+  v.pl = plan_gemm(a, di, ws_cap);
+  if ((st = build_launch(v.gl, &a, 1, v.pl, a->workspace, (a->flags & SP24_GEMM_W_STATIC) != 0)) != SP24_OK)
     return st;
-  return dispatch_gemm(pl, gl, stream);
+  g_cache_single.put(key, v);
+  return dispatch_gemm(v.pl, v.gl, stream);
 }
 
 // Checks that n problems can share one grouped launch.
@@ -884,6 +962,15 @@ size_t sp24_gemm_workspace_bytes(const sp24_gemm_args* a) {
   return pl.ws_bytes;
 }
 
+size_t sp24_gemm_workspace_state_bytes(const sp24_gemm_args* a) {
+  if (validate_gemm(a) != SP24_OK) return 0;
+  DeviceInfo di;
+  if (current_device_info(&di) != SP24_OK) return 0;
+  if (use_pair(a->N, a->M, a->tile_dense_mask != nullptr, a->flags)) return 0;
+  const Plan pl = plan_gemm(a, di, (size_t)-1);
+  return pl.sched == kSchedStreamK ? sk_state_bytes(pl) : 0;
+}
+
 int sp24_gemm(const sp24_gemm_args* a, void* stream) {
   int st = validate_gemm(a);
   if (st != SP24_OK) return st;
@@ -899,6 +986,16 @@ size_t sp24_gemm_grouped_workspace_bytes(const sp24_gemm_args* args, int n) {
   return plan_group(ptrs, n, di, (size_t)-1).ws_bytes;
 }
 
+size_t sp24_gemm_grouped_workspace_state_bytes(const sp24_gemm_args* args, int n) {
+  if (validate_group(args, n) != SP24_OK) return 0;
+  DeviceInfo di;
+  if (current_device_info(&di) != SP24_OK) return 0;
+  const sp24_gemm_args* ptrs[kMaxGroup];
+  for (int i = 0; i < n; ++i) ptrs[i] = &args[i];
+  const Plan pl = plan_group(ptrs, n, di, (size_t)-1);
+  return pl.sched == kSchedStreamK ? sk_state_bytes(pl) : 0;
+}
+
 int sp24_gemm_grouped(const sp24_gemm_args* args, int n, void* workspace, size_t workspace_bytes,
                       void* stream) {
   int st = validate_group(args, n);
@@ -912,10 +1009,14 @@ int sp24_gemm_grouped(const sp24_gemm_args* args, int n, void* workspace, size_t
     ptrs[i] = &args[i];
     w_static = w_static && (args[i].flags & SP24_GEMM_W_STATIC) != 0;
   }
-  const Plan pl = plan_group(ptrs, n, di, workspace != nullptr ? workspace_bytes : 0);
-  static thread_local GemmLaunch<kMaxGroup> gl;  // large: keep it off the stack
-  if ((st = build_launch(gl, ptrs, n, pl, workspace, w_static)) != SP24_OK) return st;
-  return dispatch_gemm_group(pl, gl, static_cast<cudaStream_t>(stream));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const LaunchKey key = make_key(args, n, workspace, workspace_bytes);
+  if (g_cache_group.find(key, [&](const GroupLaunch& v) { st = dispatch_gemm_group(v.pl, v.gl, s); })) return st;
+  static thread_local GroupLaunch v;  // large: keep it off the stack
+  v.pl = plan_group(ptrs, n, di, workspace != nullptr ? workspace_bytes : 0);
+  if ((st = build_launch(v.gl, ptrs, n, v.pl, workspace, w_static)) != SP24_OK) return st;
+  g_cache_group.put(key, v);
+  return dispatch_gemm_group(v.pl, v.gl, s);
 }
 
 int sp24_gemm_noalloc(const sp24_gemm_args* a, void* stream) {
@@ -929,9 +1030,9 @@ int sp24_gemm_noalloc(const sp24_gemm_args* a, void* stream) {
   void* scratch = nullptr;
   if ((st = static_scratch(&scratch)) != SP24_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // the accumulators and counters must start at zero; the array keeps
-  // whatever the previous call on this device left in it
-  if (pl.ws_bytes > 0 && cudaMemsetAsync(scratch, 0, pl.ws_bytes, s) != cudaSuccess) {
+  // the flags and counters must start at zero; the array keeps whatever
+  // the previous call on this device left in it
+  if (pl.ws_bytes > 0 && cudaMemsetAsync(scratch, 0, sk_state_bytes(pl), s) != cudaSuccess) {
     cudaGetLastError();
     return SP24_ERR_CUDA;
   }

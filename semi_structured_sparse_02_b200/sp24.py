@@ -102,6 +102,8 @@ def lib() -> ctypes.CDLL:
         "sp24_gemm_noalloc_max_scratch_bytes": (ctypes.c_size_t, []),
         "sp24_gemm_grouped": (I, [ctypes.POINTER(GemmArgs), I, P, ctypes.c_size_t, P]),
         "sp24_gemm_grouped_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(GemmArgs), I]),
+        "sp24_gemm_workspace_state_bytes": (ctypes.c_size_t, [ctypes.POINTER(GemmArgs)]),
+        "sp24_gemm_grouped_workspace_state_bytes": (ctypes.c_size_t, [ctypes.POINTER(GemmArgs), I]),
         "sp24_activations_workspace_bytes": (ctypes.c_size_t, [I64, I64]),
         "sp24_prune_compress_activations_fused": (I, [P, I64, I64, I64, P, I64, I64, P, I64, I,
                                                       P, P, P, ctypes.c_size_t, P]),
@@ -266,6 +268,10 @@ def gemm_workspace_bytes(args: GemmArgs) -> int:
     return lib().sp24_gemm_workspace_bytes(ctypes.byref(args))
 
 
+def gemm_workspace_state_bytes(args: GemmArgs) -> int:
+    return lib().sp24_gemm_workspace_state_bytes(ctypes.byref(args))
+
+
 def gemm(args: GemmArgs, stream=None):
     _check(lib().sp24_gemm(ctypes.byref(args), _stream(stream)), "sp24_gemm")
 
@@ -298,6 +304,9 @@ class GemmGroup:
 
     def workspace_bytes(self) -> int:
         return lib().sp24_gemm_grouped_workspace_bytes(self.arr, self.n)
+
+    def workspace_state_bytes(self) -> int:
+        return lib().sp24_gemm_grouped_workspace_state_bytes(self.arr, self.n)
 
     def __call__(self, stream=None):
         _check(lib().sp24_gemm_grouped(self.arr, self.n, _ptr(self.workspace), self.ws_bytes,

@@ -232,7 +232,9 @@ def test_stream_k_workspace_is_reusable(tactic):
         y = Y.cpu().numpy().astype(np.float64)
         check_tolerance(y, y_ref, a_ref, "stream-K repeat")
         assert np.allclose(y, y1, rtol=1e-5, atol=1e-5 * np.abs(y1).max())
-    assert int(ws.view(torch.int32).abs().sum().item()) == 0  # accumulators and counters zero
+    nstate = sp24.gemm_workspace_state_bytes(args)
+    assert 0 < nstate <= ws.numel()
+    assert int(ws[:nstate].view(torch.int32).abs().sum().item()) == 0  # counters and flags zero
 
 
 @pytest.mark.parametrize("M,N,K", [(1, 5120, 5120), (32, 2560, 25600), (128, 1280, 5120)])
@@ -303,7 +305,8 @@ def test_grouped_gemm_sixteen_problems_w_static_reusable():
             y1 = y1.cpu().numpy().astype(np.float64)
             assert np.allclose(it[1].cpu().numpy(), y1, rtol=1e-5, atol=1e-5 * np.abs(y1).max())
     if grp.workspace is not None:
-        assert int(grp.workspace.view(torch.int32).abs().sum().item()) == 0
+        nstate = grp.workspace_state_bytes()
+        assert int(grp.workspace[:nstate].view(torch.int32).abs().sum().item()) == 0
 
 
 @pytest.mark.parametrize("e4", [False, True])
@@ -315,6 +318,35 @@ def test_grouped_gemm_cta_pairs(e4):
     for use_ws in (True, False):
         _, items = run_group(shapes, e4, sp24.SPARSE, True, use_ws=use_ws, flags=flags, seed=17)
         check_group(items, "pair group ws=%s" % use_ws)
+
+
+def test_launch_cache_tells_argument_sets_apart():
+    # repeated calls with identical arguments reuse a cached launch; any
+    # changed field (here the output pointer, then the workspace) must not
+    X, W = inputs.linear_pair(8, 1024, 4096, seed=321)
+    a, Y1, y_ref, a_ref = prepare_gemm(X, W, True, sp24.SPARSE, True)
+    for _ in range(2):
+        Y1.zero_()
+        sp24.gemm(a)
+        torch.cuda.synchronize()
+        check_tolerance(Y1.cpu().numpy().astype(np.float64), y_ref, a_ref, "cached call")
+    Y2 = torch.zeros_like(Y1)
+    b = sp24.gemm_args(a._keep[0], a._keep[1], Y2, 4096, sp24.SPARSE, W_meta=a._keep[3], x_scales=a._keep[4],
+                       w_scales=a._keep[5])
+    Y1.zero_()
+    sp24.gemm(b)
+    torch.cuda.synchronize()
+    assert float(Y1.abs().max()) == 0.0
+    check_tolerance(Y2.cpu().numpy().astype(np.float64), y_ref, a_ref, "new output pointer")
+    ws = workspace_for(b)
+    assert ws is not None
+    sp24.set_workspace(b, ws)  # stream-K schedule now: a different launch
+    Y2.zero_()
+    sp24.gemm(b)
+    torch.cuda.synchronize()
+    check_tolerance(Y2.cpu().numpy().astype(np.float64), y_ref, a_ref, "with workspace")
+    nstate = sp24.gemm_workspace_state_bytes(b)
+    assert int(ws[:nstate].view(torch.int32).abs().sum().item()) == 0
 
 
 def test_group_of_one_matches_single_gemm():
