@@ -575,8 +575,13 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
     uint32_t acc_i = 0;
     int cached_pr = -1, cached_tb = -1;
     uint8_t* wtile = s_epi + (warp - 2) * 2048;  // this warp's staging tile
-    const int eb = p.out_f32 ? 4 : 2;
-    const int per_vec = 16 / eb;                   // elements per 16-byte vector
+    // values read once into registers: the tcgen05 and barrier asm statements
+    // below clobber memory, which would otherwise force the parameter-struct
+    // fields to be re-read after each of them
+    const bool out_f32 = p.out_f32 != 0;
+    const int64_t total_iters = p.total_iters;
+    float* const sk_slots = p.sk_slots;
+    unsigned int* const sk_flags = p.sk_flags;
     SegIter<kMaxProb> it;
     it.init(g, unit, units);
     int pr, tile, kb, ke, seg;
@@ -586,14 +591,17 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
       const int buf = acc_i & 1;
       const uint32_t acc_phase = (acc_i >> 1) & 1;
       const int ga = ta * C::kRowsA + (int)rank * kBlockA + row;  // global A row of this thread
-      const bool a_live = ga < P.rows_a;
+      const int rows_a = P.rows_a, rows_b = P.rows_b;
+      uint8_t* const Yb = static_cast<uint8_t*>(P.Y);
+      const int64_t ldy = P.ldy;
+      const bool a_live = ga < rows_a;
       // scales: loaded before waiting for the accumulator so their latency hides
       const float sa_v = (P.scale_a != nullptr && a_live) ? __ldg(P.scale_a + ga) : 1.0f;
       if (pr != cached_pr || tb != cached_tb) {
         named_bar_sync(1, 128);
         for (int i = et; i < kBN; i += 128) {
           const int gb = tb * kBN + i;
-          s_scale_b[i] = (P.scale_b != nullptr && gb < P.rows_b) ? P.scale_b[gb] : 1.0f;
+          s_scale_b[i] = (P.scale_b != nullptr && gb < rows_b) ? P.scale_b[gb] : 1.0f;
         }
         named_bar_sync(1, 128);
         cached_pr = pr;
@@ -613,34 +621,46 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
       // Scales and stores 16 consecutive accumulator columns starting at c0
       // with 16-byte vector stores.  Rows of Y are 16-byte aligned (checked
       // on the host); a vector that crosses the end of a row is stored per
-      // element.
-      auto store16 = [&](const float (&v)[16], int c0) {
+      // element.  EB (output bytes) is a compile-time constant so that the
+      // index arithmetic is shifts and masks: this code runs on one warp per
+      // sub-partition, where every dependent instruction shows in the time.
+      auto store16 = [&](auto eb_c, const float (&v)[16], int c0) {
+        constexpr int EB = decltype(eb_c)::value;
+        constexpr int PV = 16 / EB;   // elements per 16-byte vector
         const int gb0 = tb * kBN + c0;
+        float sc[16];
+#pragma unroll
+        for (int i = 0; i < 16; i += 4) {
+          const float4 t = *reinterpret_cast<const float4*>(s_scale_b + c0 + i);
+          sc[i] = t.x * sa_v; sc[i + 1] = t.y * sa_v; sc[i + 2] = t.z * sa_v; sc[i + 3] = t.w * sa_v;
+        }
         if (kAIsW) {
           // lane = n (output feature), column = m (token).  Stage the warp's
           // 32 n x 16 m block transposed, then write each output row's 32
           // consecutive n as 16-byte vectors.
+          constexpr int VPR = 32 / PV;  // vectors per row of 32 n
           const int n0 = ta * C::kRowsA + (int)rank * kBlockA + lg * 32;
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const float y = v[i] * sa_v * s_scale_b[c0 + i];
-            if (p.out_f32) reinterpret_cast<float*>(wtile)[i * 32 + lane] = y;
+            const float y = v[i] * sc[i];
+            if (EB == 4) reinterpret_cast<float*>(wtile)[i * 32 + lane] = y;
             else reinterpret_cast<__nv_bfloat16*>(wtile)[i * 32 + lane] = __float2bfloat16_rn(y);
           }
           __syncwarp();
-          const int vec_per_row = 32 / per_vec;
-          for (int q = lane; q < 16 * vec_per_row; q += 32) {
-            const int i = q / vec_per_row, sg = q - i * vec_per_row;
+#pragma unroll
+          for (int it = 0; it < 16 * VPR / 32; ++it) {
+            const int q = lane + 32 * it;
+            const int i = q / VPR, sg = q % VPR;
             const int m = gb0 + i;
-            const int n = n0 + sg * per_vec;
-            if (m >= P.rows_b || n >= P.rows_a) continue;
-            uint8_t* dst = static_cast<uint8_t*>(P.Y) + ((int64_t)m * P.ldy + n) * eb;
-            const uint8_t* src = wtile + (i * 32 + sg * per_vec) * eb;
-            if (n + per_vec <= P.rows_a) {
-              *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
-            } else {
-              for (int e = 0; e < P.rows_a - n; ++e)
-                for (int b = 0; b < eb; ++b) dst[e * eb + b] = src[e * eb + b];
+            const int n = n0 + sg * PV;
+            if (m < rows_b && n < rows_a) {
+              uint8_t* dst = Yb + ((int64_t)m * ldy + n) * EB;
+              const uint8_t* src = wtile + (i * 32 + sg * PV) * EB;
+              if (n + PV <= rows_a) {
+                *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
+              } else {
+                for (int e = 0; e < (rows_a - n) * EB; ++e) dst[e] = src[e];
+              }
             }
           }
           __syncwarp();
@@ -648,22 +668,41 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
           // lane = m (token), column = n (output feature): this thread's 16
           // consecutive n of row ga
           if (!a_live) return;
-          alignas(16) uint8_t vbuf[64];
+          constexpr int NW = 16 * EB / 4;  // 32-bit words of output
+          uint32_t w[NW];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float y = v[i] * sa_v * s_scale_b[c0 + i];
-            if (p.out_f32) reinterpret_cast<float*>(vbuf)[i] = y;
-            else reinterpret_cast<__nv_bfloat16*>(vbuf)[i] = __float2bfloat16_rn(y);
+          for (int j = 0; j < NW; ++j) {
+            if (EB == 4) {
+              w[j] = __float_as_uint(v[j] * sc[j]);
+            } else {
+              const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * j] * sc[2 * j], v[2 * j + 1] * sc[2 * j + 1]);
+              w[j] = *reinterpret_cast<const uint32_t*>(&h);
+            }
           }
-          uint8_t* dst = static_cast<uint8_t*>(P.Y) + ((int64_t)ga * P.ldy + gb0) * eb;
-          if (gb0 + 16 <= P.rows_b) {
-            for (int q = 0; q < 16 / per_vec; ++q)
-              reinterpret_cast<uint4*>(dst)[q] = reinterpret_cast<const uint4*>(vbuf)[q];
+          uint8_t* dst = Yb + ((int64_t)ga * ldy + gb0) * EB;
+          if (gb0 + 16 <= rows_b) {
+#pragma unroll
+            for (int q = 0; q < NW / 4; ++q)
+              reinterpret_cast<uint4*>(dst)[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
           } else {
-            for (int e = 0; e < P.rows_b - gb0; ++e)
-              for (int b = 0; b < eb; ++b) dst[e * eb + b] = vbuf[e * eb + b];
+#pragma unroll
+            for (int j = 0; j < NW; ++j) {
+              // whole 32-bit words inside the row (for bf16 a word holds two
+              // outputs; a row of odd length ends in a half word)
+              const int e0 = j * 4 / EB;  // first output of word j
+              if (e0 >= rows_b - gb0) break;
+              if (EB == 4 || e0 + 1 < rows_b - gb0) {
+                reinterpret_cast<uint32_t*>(dst)[j] = w[j];
+              } else {
+                reinterpret_cast<uint16_t*>(dst)[2 * j] = (uint16_t)(w[j] & 0xFFFFu);
+              }
+            }
           }
         }
+      };
+      auto store16_any = [&](const float (&v)[16], int c0) {
+        if (out_f32) store16(std::integral_constant<int, 4>{}, v, c0);
+        else store16(std::integral_constant<int, 2>{}, v, c0);
       };
 
       // the accumulator may be overwritten now (one arrive per warp; rank
@@ -686,21 +725,21 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
           float v[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
-          store16(v, c0);
+          store16_any(v, c0);
         }
         release_acc();
       } else {
         // a split tile: its contributors are the units whose ranges cover it
         const int64_t i0 = P.iter_begin + (int64_t)tile * P.num_kt;
-        const int c_first = sk_owner(p.total_iters, units, i0);
-        const int c_last = sk_owner(p.total_iters, units, i0 + P.num_kt - 1);
+        const int c_first = sk_owner(total_iters, units, i0);
+        const int c_last = sk_owner(total_iters, units, i0 + P.num_kt - 1);
         const unsigned int count = (unsigned int)(c_last - c_first + 1);
         const int64_t cslot = (int64_t)tile * (kPair ? 2 : 1) + (int64_t)rank;
         // slot s of unit u: 0 for the unit's first segment, 1 for its last
         auto slot_idx = [&](int u, int sidx) { return ((int64_t)u * (kPair ? 2 : 1) + (int64_t)rank) * 2 + sidx; };
         // the other contributor v's segment of this tile is v's first one
         // exactly when v's range starts inside the tile
-        auto slot_of = [&](int v) { return ((int64_t)v * p.total_iters / units) >= i0 ? 0 : 1; };
+        auto slot_of = [&](int v) { return ((int64_t)v * total_iters / units) >= i0 ? 0 : 1; };
         named_bar_sync(1, 128);
         if (et == 0) {
           const unsigned int old = atom_add_acq_rel_gpu(&P.ws_counters[cslot], 1u);
@@ -710,7 +749,7 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
         if (!*last_flag) {
           // store the partial tile (plain stores), then raise the flag
           const int64_t my = slot_idx(unit, seg == 0 ? 0 : 1);
-          float* dst = p.sk_slots + (my * 128 + row) * kBN;
+          float* dst = sk_slots + (my * 128 + row) * kBN;
 #pragma unroll 1
           for (int c0 = 0; c0 < kBN; c0 += 16) {
             uint32_t r[16];
@@ -726,7 +765,7 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
           named_bar_sync(1, 128);  // every store of the tile precedes the flag
           if (et == 0) {
             __threadfence();
-            st_release_gpu(p.sk_flags + my, 1u);
+            st_release_gpu(sk_flags + my, 1u);
           }
         } else {
           // wait (bounded) for the other contributors' flags
@@ -734,7 +773,7 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
           if (et == 0) {
             for (int v = c_first; v <= c_last && ok2; ++v) {
               if (v == unit) continue;
-              const unsigned int* f = p.sk_flags + slot_idx(v, slot_of(v));
+              const unsigned int* f = sk_flags + slot_idx(v, slot_of(v));
               if (ld_acquire_gpu(f) == 0u) {
                 const uint64_t t0 = globaltimer_ns();
                 while (ld_acquire_gpu(f) == 0u) {
@@ -760,7 +799,7 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
             if (have) {
               for (int v = c_first; v <= c_last; ++v) {
                 if (v == unit) continue;
-                const float* src = p.sk_slots + (slot_idx(v, slot_of(v)) * 128 + row) * kBN + cb;
+                const float* src = sk_slots + (slot_idx(v, slot_of(v)) * 128 + row) * kBN + cb;
                 float4 t[kFix / 4];
 #pragma unroll
                 for (int j = 0; j < kFix / 4; ++j) t[j] = __ldcg(reinterpret_cast<const float4*>(src) + j);
@@ -784,7 +823,7 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
                 v[4 * j + 2] = __uint_as_float(r[4 * j + 2]) + t.z;
                 v[4 * j + 3] = __uint_as_float(r[4 * j + 3]) + t.w;
               }
-              store16(v, cb + c0);
+              store16_any(v, cb + c0);
             }
           }
           release_acc();
@@ -792,7 +831,7 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
           if (et == 0) {
             // ready for the next call
             for (int v = c_first; v <= c_last; ++v)
-              if (v != unit) p.sk_flags[slot_idx(v, slot_of(v))] = 0u;
+              if (v != unit) sk_flags[slot_idx(v, slot_of(v))] = 0u;
             P.ws_counters[cslot] = 0u;
           }
           if (!have) *abort_flag = 1;

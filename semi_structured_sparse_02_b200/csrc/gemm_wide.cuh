@@ -259,18 +259,24 @@ k_gemm_wide(const __grid_constant__ WideLaunch g) {
     const int et = threadIdx.x - 64;  // 0..127
     const uint32_t acc_empty0 = mapa_shared(bar_u32(kAccEmpty), 0);
     uint8_t* wtile = s_epi + (warp - 2) * 2048;
-    const int eb = g.out_f32 ? 4 : 2;
-    const int per_vec = 16 / eb;
+    // values read once into registers (the asm statements below clobber
+    // memory, which would force parameter fields to be re-read after each)
+    const bool out_f32 = g.out_f32 != 0;
+    const int rows_a = g.rows_a, rows_b = g.rows_b, tiles_a = g.tiles_a, total_tiles = g.total_tiles;
+    uint8_t* const Yb = static_cast<uint8_t*>(g.Y);
+    const int64_t ldy = g.ldy;
+    const float* const scale_a = g.scale_a;
+    const float* const scale_b = g.scale_b;
     int j = 0;
-    for (int tile = pair; tile < g.total_tiles; tile += n_pairs, ++j) {
-      const int ta = tile % g.tiles_a, tb = tile / g.tiles_a;
+    for (int tile = pair; tile < total_tiles; tile += n_pairs, ++j) {
+      const int ta = tile % tiles_a, tb = tile / tiles_a;
       const int b = j & 1;
       const int ga = ta * 256 + (int)rank * 128 + row;  // A row of this thread
-      const float sa_v = (g.scale_a != nullptr && ga < g.rows_a) ? __ldg(g.scale_a + ga) : 1.0f;
+      const float sa_v = (scale_a != nullptr && ga < rows_a) ? __ldg(scale_a + ga) : 1.0f;
       named_bar_sync(1, 128);  // the previous tile's stores are done with the B scales
       for (int i = et; i < 256; i += 128) {
         const int gb = tb * 256 + i;
-        s_scale_b[i] = (g.scale_b != nullptr && gb < g.rows_b) ? g.scale_b[gb] : 1.0f;
+        s_scale_b[i] = (scale_b != nullptr && gb < rows_b) ? scale_b[gb] : 1.0f;
       }
       named_bar_sync(1, 128);
       bool ok = mbar_wait(bar_u32(kAccFull + b), (uint32_t)((j >> 1) & 1), g.timeout_ns, kDevErrWaitAccFull);
@@ -283,55 +289,80 @@ k_gemm_wide(const __grid_constant__ WideLaunch g) {
       tc_fence_after_sync();
       const uint32_t tbase = tmem_base + ((uint32_t)(lg * 32) << 16) + (b ? (uint32_t)C::kAcc1 : 0u);
 
-      // scales and stores 16 accumulator columns starting at c0
-      auto store16 = [&](const float (&v)[16], int c0) {
+      // scales and stores 16 accumulator columns starting at c0; EB (output
+      // bytes) is a compile-time constant so the index arithmetic is shifts
+      auto store16 = [&](auto eb_c, const float (&v)[16], int c0) {
+        constexpr int EB = decltype(eb_c)::value;
+        constexpr int PV = 16 / EB;  // elements per 16-byte vector
         const int gb0 = tb * 256 + c0;
+        float sc[16];
+#pragma unroll
+        for (int i = 0; i < 16; i += 4) {
+          const float4 t = *reinterpret_cast<const float4*>(s_scale_b + c0 + i);
+          sc[i] = t.x * sa_v; sc[i + 1] = t.y * sa_v; sc[i + 2] = t.z * sa_v; sc[i + 3] = t.w * sa_v;
+        }
         if (kAIsW) {
           // lane = output feature n, column = token m: stage the warp's
           // 32 n x 16 m block transposed, then write 16-byte vectors of n
+          constexpr int VPR = 32 / PV;
           const int n0 = ta * 256 + (int)rank * 128 + lg * 32;
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const float y = v[i] * sa_v * s_scale_b[c0 + i];
-            if (g.out_f32) reinterpret_cast<float*>(wtile)[i * 32 + lane] = y;
+            const float y = v[i] * sc[i];
+            if (EB == 4) reinterpret_cast<float*>(wtile)[i * 32 + lane] = y;
             else reinterpret_cast<__nv_bfloat16*>(wtile)[i * 32 + lane] = __float2bfloat16_rn(y);
           }
           __syncwarp();
-          const int vec_per_row = 32 / per_vec;
-          for (int q = lane; q < 16 * vec_per_row; q += 32) {
-            const int i = q / vec_per_row, sg = q - i * vec_per_row;
+#pragma unroll
+          for (int it = 0; it < 16 * VPR / 32; ++it) {
+            const int q = lane + 32 * it;
+            const int i = q / VPR, sg = q % VPR;
             const int m = gb0 + i;
-            const int n = n0 + sg * per_vec;
-            if (m >= g.rows_b || n >= g.rows_a) continue;
-            uint8_t* dst = static_cast<uint8_t*>(g.Y) + ((int64_t)m * g.ldy + n) * eb;
-            const uint8_t* src = wtile + (i * 32 + sg * per_vec) * eb;
-            if (n + per_vec <= g.rows_a) {
-              *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
-            } else {
-              for (int e = 0; e < g.rows_a - n; ++e)
-                for (int k = 0; k < eb; ++k) dst[e * eb + k] = src[e * eb + k];
+            const int n = n0 + sg * PV;
+            if (m < rows_b && n < rows_a) {
+              uint8_t* dst = Yb + ((int64_t)m * ldy + n) * EB;
+              const uint8_t* src = wtile + (i * 32 + sg * PV) * EB;
+              if (n + PV <= rows_a) {
+                *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
+              } else {
+                for (int e = 0; e < (rows_a - n) * EB; ++e) dst[e] = src[e];
+              }
             }
           }
           __syncwarp();
         } else {
           // lane = token m, column = output feature n: 16 consecutive n of row ga
-          if (ga >= g.rows_a) return;
-          alignas(16) uint8_t vbuf[64];
+          if (ga >= rows_a) return;
+          constexpr int NW = 16 * EB / 4;
+          uint32_t w[NW];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float y = v[i] * sa_v * s_scale_b[c0 + i];
-            if (g.out_f32) reinterpret_cast<float*>(vbuf)[i] = y;
-            else reinterpret_cast<__nv_bfloat16*>(vbuf)[i] = __float2bfloat16_rn(y);
+          for (int j = 0; j < NW; ++j) {
+            if (EB == 4) {
+              w[j] = __float_as_uint(v[j] * sc[j]);
+            } else {
+              const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * j] * sc[2 * j], v[2 * j + 1] * sc[2 * j + 1]);
+              w[j] = *reinterpret_cast<const uint32_t*>(&h);
+            }
           }
-          uint8_t* dst = static_cast<uint8_t*>(g.Y) + ((int64_t)ga * g.ldy + gb0) * eb;
-          if (gb0 + 16 <= g.rows_b) {
-            for (int q = 0; q < 16 / per_vec; ++q)
-              reinterpret_cast<uint4*>(dst)[q] = reinterpret_cast<const uint4*>(vbuf)[q];
+          uint8_t* dst = Yb + ((int64_t)ga * ldy + gb0) * EB;
+          if (gb0 + 16 <= rows_b) {
+#pragma unroll
+            for (int q = 0; q < NW / 4; ++q)
+              reinterpret_cast<uint4*>(dst)[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
           } else {
-            for (int e = 0; e < g.rows_b - gb0; ++e)
-              for (int k = 0; k < eb; ++k) dst[e * eb + k] = vbuf[e * eb + k];
+#pragma unroll
+            for (int j = 0; j < NW; ++j) {
+              const int e0 = j * 4 / EB;  // first output of word j
+              if (e0 >= rows_b - gb0) break;
+              if (EB == 4 || e0 + 1 < rows_b - gb0) reinterpret_cast<uint32_t*>(dst)[j] = w[j];
+              else reinterpret_cast<uint16_t*>(dst)[2 * j] = (uint16_t)(w[j] & 0xFFFFu);
+            }
           }
         }
+      };
+      auto store16_any = [&](const float (&v)[16], int c0) {
+        if (out_f32) store16(std::integral_constant<int, 4>{}, v, c0);
+        else store16(std::integral_constant<int, 2>{}, v, c0);
       };
       auto drain = [&](int c_begin, int c_end) {
 #pragma unroll 1
@@ -342,7 +373,7 @@ k_gemm_wide(const __grid_constant__ WideLaunch g) {
           float v[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
-          store16(v, c0);
+          store16_any(v, c0);
         }
       };
       auto release = [&]() {
