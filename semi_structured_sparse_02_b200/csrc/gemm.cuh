@@ -749,7 +749,9 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
         if (!*last_flag) {
           // store the partial tile (plain stores), then raise the flag
           const int64_t my = slot_idx(unit, seg == 0 ? 0 : 1);
-          float* dst = sk_slots + (my * 128 + row) * kBN;
+          // slot layout: float4 (col / 4) of row r at index (col / 4) * 128 + r,
+          // so each warp store covers 512 contiguous bytes
+          float4* dst = reinterpret_cast<float4*>(sk_slots + my * 128 * kBN) + row;
 #pragma unroll 1
           for (int c0 = 0; c0 < kBN; c0 += 16) {
             uint32_t r[16];
@@ -757,7 +759,7 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
             tmem_ld_wait();
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-              __stcg(reinterpret_cast<float4*>(dst + c0) + j,
+              __stcg(dst + (c0 / 4 + j) * 128,
                      make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
                                  __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3])));
           }
@@ -799,10 +801,10 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
             if (have) {
               for (int v = c_first; v <= c_last; ++v) {
                 if (v == unit) continue;
-                const float* src = sk_slots + (slot_idx(v, slot_of(v)) * 128 + row) * kBN + cb;
+                const float4* src = reinterpret_cast<const float4*>(sk_slots + slot_idx(v, slot_of(v)) * 128 * kBN) + row;
                 float4 t[kFix / 4];
 #pragma unroll
-                for (int j = 0; j < kFix / 4; ++j) t[j] = __ldcg(reinterpret_cast<const float4*>(src) + j);
+                for (int j = 0; j < kFix / 4; ++j) t[j] = __ldcg(src + (cb / 4 + j) * 128);
 #pragma unroll
                 for (int j = 0; j < kFix / 4; ++j) {
                   q[j].x += t[j].x; q[j].y += t[j].y; q[j].z += t[j].z; q[j].w += t[j].w;
