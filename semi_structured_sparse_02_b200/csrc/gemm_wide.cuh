@@ -32,6 +32,8 @@
 // index fastest (consecutive pairs share a B tile, all pairs share A in L2).
 #pragma once
 
+#include <type_traits>
+
 #include "gemm.cuh"
 
 namespace sp24 {
@@ -135,19 +137,22 @@ k_gemm_wide(const __grid_constant__ WideLaunch g) {
       const uint32_t full0 = mapa_shared(bar_u32(kFull), 0);  // rank 0's stage barriers
       const int box_elems = kBf16 ? 64 : 128;                // 128 bytes of B per box row
       const int kc_total = g.K / 128;
+      // parameter fields in registers (the asm below clobbers memory)
+      const int num_kt = g.num_kt, total_tiles = g.total_tiles, tiles_a = g.tiles_a, meta_blocks = g.meta_blocks;
+      const uint64_t timeout_ns = g.timeout_ns;
       int armed[S];
       for (int s = 0; s < S; ++s) armed[s] = -1;
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int tile = pair; ok && tile < g.total_tiles; tile += n_pairs) {
-        const int ta = tile % g.tiles_a, tb = tile / g.tiles_a;
+      for (int tile = pair; ok && tile < total_tiles; tile += n_pairs) {
+        const int ta = tile % tiles_a, tb = tile / tiles_a;
         const int ya = ta * 256 + (int)rank * 128;
         const int yb = tb * 256 + (int)rank * 128;
         int rb = ta * 2 + (int)rank;        // metadata row block of this CTA's A rows
-        if (rb >= g.meta_blocks) rb = 0;    // rows past the end: A is zero-filled; any valid metadata
-        for (int kt = 0; kt < g.num_kt; ++kt) {
-          if (!mbar_wait(bar_u32(kEmpty + stage), phase ^ 1, g.timeout_ns, kDevErrWaitEmpty)) {
+        if (rb >= meta_blocks) rb = 0;    // rows past the end: A is zero-filled; any valid metadata
+        for (int kt = 0; kt < num_kt; ++kt) {
+          if (!mbar_wait(bar_u32(kEmpty + stage), phase ^ 1, timeout_ns, kDevErrWaitEmpty)) {
             ok = false;
             *abort_flag = 1;
             break;
@@ -174,24 +179,30 @@ k_gemm_wide(const __grid_constant__ WideLaunch g) {
       }
       // rank 0: wait (bounded) until every armed stage has landed
       for (int s = 0; s < S; ++s)
-        if (armed[s] >= 0) mbar_wait(bar_u32(kFull + s), (uint32_t)armed[s], g.timeout_ns, kDevErrWaitFull);
+        if (armed[s] >= 0) mbar_wait(bar_u32(kFull + s), (uint32_t)armed[s], timeout_ns, kDevErrWaitFull);
     }
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer (rank 0)
     if (rank == 0 && lane == 0) {
       const uint32_t idesc = make_idesc(C::kSparse, kBf16, 256, 256);
+      const uint32_t s0 = smem_u32(smem);
+      const uint64_t da0 = smem_desc(s0, 16, 1024, kLayoutSw128);
+      const uint64_t db0 = smem_desc(s0 + C::kABytes, 16, 1024, kLayoutSw128);
+      const uint64_t dm0 = smem_desc(s0 + C::kABytes + C::kBBytes, 16, 128, kLayoutNone);
+      const int num_kt = g.num_kt, total_tiles = g.total_tiles;
+      const uint64_t timeout_ns = g.timeout_ns;
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
       int j = 0;
-      for (int tile = pair; ok && tile < g.total_tiles; tile += n_pairs, ++j) {
+      for (int tile = pair; ok && tile < total_tiles; tile += n_pairs, ++j) {
         const int b = j & 1;
         // the accumulator: sparse waits for tile j-1's overlap release (which
         // implies tile j-2 is drained); dense waits for tile j-2's release
         if (C::kSparse ? j >= 1 : j >= 2) {
           const int jr = C::kSparse ? j - 1 : j - 2;
-          if (!mbar_wait(bar_u32(kAccEmpty + (jr & 1)), (uint32_t)((jr >> 1) & 1), g.timeout_ns,
+          if (!mbar_wait(bar_u32(kAccEmpty + (jr & 1)), (uint32_t)((jr >> 1) & 1), timeout_ns,
                          kDevErrWaitAccEmpty)) {
             ok = false;
             *abort_flag = 1;
@@ -200,42 +211,52 @@ k_gemm_wide(const __grid_constant__ WideLaunch g) {
         }
         tc_fence_after_sync();
         const uint32_t d = tmem_base + (b ? (uint32_t)C::kAcc1 : 0u);
-        for (int kt = 0; kt < g.num_kt; ++kt) {
-          if (!mbar_wait(bar_u32(kFull + stage), phase, g.timeout_ns, kDevErrWaitFull)) {
+        for (int kt = 0; kt < num_kt; ++kt) {
+          if (!mbar_wait(bar_u32(kFull + stage), phase, timeout_ns, kDevErrWaitFull)) {
             ok = false;
             *abort_flag = 1;
             break;
           }
           tc_fence_after_sync();
-          const uint32_t sa = smem_u32(smem + stage * C::kStageBytes);
-          const uint32_t sb = sa + C::kABytes;
-          const uint32_t sm = sb + C::kBBytes;
+          // this stage's descriptors: the stage-0 ones plus the stage offset
+          // (the address field counts 16-byte units); the issuing thread is
+          // on the critical path, so the loops below are fully unrolled
+          const uint64_t so = (uint64_t)((uint32_t)stage * (uint32_t)(C::kStageBytes >> 4));
+          const uint64_t da = da0 + so, db = db0 + so, dm = dm0 + so;
           const bool first = kt == 0;
           if (C::kSparse) {
             const uint32_t mcol = C::kMetaCol0 + stage * C::kMetaCols;
-            const int chunks = meta_chunks(kt);
-            for (int c = 0; c < chunks; ++c)
-              tc_cp_128x128b_pair(tmem_base + mcol + 4 * c, smem_desc(sm + c * 2048, 16, 128, kLayoutNone));
-            const int n_mma = kBf16 ? 4 : 2 * chunks;
-            for (int q = 0; q < n_mma; ++q) {
-              const uint64_t da = smem_desc(sa + q * 32, 16, 1024, kLayoutSw128);
-              const uint64_t db = smem_desc(sb + (q >> 1) * 16384 + (q & 1) * 64, 16, 1024, kLayoutSw128);
-              const uint32_t acc = (first && q == 0) ? 0u : 1u;
-              if (kBf16) {
-                const uint32_t col = mcol + q;
-                mma_sp_bf16_pair(d, da, db, tmem_base + (col & ~1u), idesc | (col & 1u), acc);
-              } else {
-                const uint32_t col = mcol + 4 * (q >> 1) + 2 * (q & 1);
-                mma_sp_f8_pair(d, da, db, tmem_base + col, idesc, acc);
+            auto issue = [&](auto chunks_c) {
+              constexpr int kChunks = decltype(chunks_c)::value;
+#pragma unroll
+              for (int c = 0; c < kChunks; ++c)
+                tc_cp_128x128b_pair(tmem_base + mcol + 4 * c, dm + (uint64_t)(c * (2048 >> 4)));
+              constexpr int kMmas = kBf16 ? 4 : 2 * kChunks;
+#pragma unroll
+              for (int q = 0; q < kMmas; ++q) {
+                const uint64_t a_d = da + (uint64_t)(q * (32 >> 4));
+                const uint64_t b_d = db + (uint64_t)(((q >> 1) * 16384 + (q & 1) * 64) >> 4);
+                const uint32_t acc = (first && q == 0) ? 0u : 1u;
+                if (kBf16) {
+                  const uint32_t col = mcol + q;
+                  mma_sp_bf16_pair(d, a_d, b_d, tmem_base + (col & ~1u), idesc | (col & 1u), acc);
+                } else {
+                  const uint32_t col = mcol + 4 * (q >> 1) + 2 * (q & 1);
+                  mma_sp_f8_pair(d, a_d, b_d, tmem_base + col, idesc, acc);
+                }
               }
-            }
+            };
+            if (kBf16 || C::kMetaChunks == 1 || meta_chunks(kt) == C::kMetaChunks)
+              issue(std::integral_constant<int, C::kMetaChunks>{});
+            else
+              issue(std::integral_constant<int, 1>{});
           } else {
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-              const uint64_t da = smem_desc(sa + q * 32, 16, 1024, kLayoutSw128);
-              const uint64_t db = smem_desc(sb + q * 32, 16, 1024, kLayoutSw128);
-              if (kBf16) mma_bf16_pair(d, da, db, idesc, (first && q == 0) ? 0u : 1u);
-              else mma_f8_pair(d, da, db, idesc, (first && q == 0) ? 0u : 1u);
+              const uint64_t a_d = da + (uint64_t)(q * (32 >> 4));
+              const uint64_t b_d = db + (uint64_t)(q * (32 >> 4));
+              if (kBf16) mma_bf16_pair(d, a_d, b_d, idesc, (first && q == 0) ? 0u : 1u);
+              else mma_f8_pair(d, a_d, b_d, idesc, (first && q == 0) ? 0u : 1u);
             }
           }
           tc_commit_pair(bar_u32(kEmpty + stage), 0x3);  // frees the stage in both CTAs
