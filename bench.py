@@ -790,6 +790,32 @@ def run_config(args):
                                                   peak[("dense", False)], hbm),
                          note="fused = prune+compress of X every call, then the sparse GEMM with X as "
                               "the sparse operand; dense = the in-build dense GEMM on unpruned X"))
+        # the same at the FP8 floor: X pruned and cast to e4m3 per token every call, W e4m3 per channel
+        Wq = torch.empty(N, K, dtype=torch.uint8, device=dev)
+        wsc = torch.empty(N, dtype=torch.float32, device=dev)
+        sp24.quantize_e4m3_rows(W, Wq, wsc)
+        ws8 = torch.empty(sp24.activations_e4m3_workspace_bytes(M, K), dtype=torch.uint8, device=dev)
+        t_f8, _ = _time_calls(lambda: sp24.prune_compress_activations_fused_e4m3(X, Wq, wsc, Y, workspace=ws8),
+                              reps, warm, flush)
+        Xq = torch.empty(M, K, dtype=torch.uint8, device=dev)
+        xsc = torch.empty(M, dtype=torch.float32, device=dev)
+        dn8 = sp24.gemm_args(Xq, Wq, Y, K, sp24.DENSE, x_scales=xsc, w_scales=wsc)
+
+        def dense8():
+            sp24.quantize_e4m3_rows(X, Xq, xsc)
+            sp24.gemm(dn8)
+        t_d8, _ = _time_calls(dense8, reps, warm, flush)
+        t_d8g, _ = _time_calls(lambda: sp24.gemm(dn8), reps, warm, flush)
+        byts8 = 2 * M * K + (0.625 * M * K + 4 * M) * 2 + N * K + 4 * N + 2 * M * N
+        rows.append(dict(gemm="activation_e4m3", M=M, N=N, K=K, dtype="e4m3",
+                         us_fused=round(t_f8, 2), us_dense=round(t_d8, 2), us_dense_gemm_only=round(t_d8g, 2),
+                         tflops_fused=round(F / t_f8 / 1e6, 1), tflops_dense=round(F / t_d8 / 1e6, 1),
+                         speedup_vs_dense=round(t_d8 / t_f8, 3),
+                         roofline_fused=_roofline(F, byts8, t_f8, peak[("sparse", True)], hbm),
+                         roofline_dense=_roofline(F, 3 * M * K + N * K + 2 * M * N, t_d8, peak[("dense", True)], hbm),
+                         note="fused = prune + per-token e4m3 cast of X every call (row amax, prune/cast, "
+                              "scale passes), then the e4m3 sparse GEMM with X as the sparse operand; dense = "
+                              "per-token e4m3 cast of unpruned X plus the in-build dense e4m3 GEMM"))
     elif args.config == "prune":
         shapes = [("decode", N, K, True) for N, K in inputs.DECODE_NK] + \
                  [("prefill", N, K, False) for N, K in inputs.PREFILL_NK] + \

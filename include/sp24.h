@@ -291,6 +291,25 @@ int sp24_prune_compress_activations_fused(const void *X_dev, int64_t M, int64_t 
                                           void *workspace_dev, size_t workspace_bytes,
                                           void *stream);
 
+/* The online-activation path at the FP8 floor: per call, X (bf16 [M x K])
+ * is pruned 2:4 along K on its bf16 magnitudes (same rule as
+ * sp24_prune_compress), the kept values are cast to E4M3 with one fp32 scale
+ * per token (row amax / 448, the rule of sp24_quantize_e4m3_rows), and then
+ * Y [M x N] = X_sparse * Wq^T with Wq the dense E4M3 weights [N x K] and
+ * their per-output-channel scales w_scales [N] (from sp24_quantize_e4m3_rows).
+ * (The activation prune "optionally fuses FP8 or INT8 quantization":
+ * 2:4-versus-quantization paper, section 3.5.)  x_values (E4M3 [M x K/2]),
+ * x_meta (image, sp24_meta_bytes(M, K)) and x_scales ([M] fp32) receive the
+ * compressed activations when given (all three or none); otherwise workspace
+ * must hold sp24_activations_e4m3_workspace_bytes(M, K) bytes.  ldw is in
+ * bytes and a multiple of 16.  Same errors as the bf16 path. */
+size_t sp24_activations_e4m3_workspace_bytes(int64_t M, int64_t K);
+int sp24_prune_compress_activations_fused_e4m3(const void *X_dev, int64_t M, int64_t K, int64_t ldx,
+                                               const void *Wq_dev, const float *w_scales_dev, int64_t N,
+                                               int64_t ldw, void *Y_dev, int64_t ldy, sp24_dtype out_dtype,
+                                               void *x_values_dev, void *x_meta_dev, float *x_scales_dev,
+                                               void *workspace_dev, size_t workspace_bytes, void *stream);
+
 /* ---------------------------------------------------------------------- */
 /* Tactic selection (kernel 5)                                             */
 /* ---------------------------------------------------------------------- */

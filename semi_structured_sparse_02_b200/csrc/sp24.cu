@@ -329,8 +329,9 @@ int device_pairs(int dev) {
 int dispatch_gemm(const Plan& pl, const GemmLaunch<1>& gl, cudaStream_t s) {
   if (pl.pair) return dispatch_pair(pl, gl, s);
   if (!pl.a_is_w) {
-    if (pl.mode == kModeSparse && pl.bf16 && pl.bn == 128)
-      return launch_gemm_inst<kModeSparse, true, 128, false, 1>(gl, pl.grid, s);
+    if (pl.mode == kModeSparse && pl.bn == 128)
+      return pl.bf16 ? launch_gemm_inst<kModeSparse, true, 128, false, 1>(gl, pl.grid, s)
+                     : launch_gemm_inst<kModeSparse, false, 128, false, 1>(gl, pl.grid, s);
     return SP24_ERR_DTYPE;
   }
   if (pl.mode == kModeSparse)
@@ -685,7 +686,9 @@ int run_wide(int mode, bool bf16, bool a_is_w, const void* A, int64_t lda, const
   wl.ldy = ldy;
   wl.timeout_ns = g_timeout_ns.load();
   if (!a_is_w) {
-    if (sparse && bf16) return launch_wide_inst<kModeSparse, true, false>(wl, stream);
+    if (sparse)
+      return bf16 ? launch_wide_inst<kModeSparse, true, false>(wl, stream)
+                  : launch_wide_inst<kModeSparse, false, false>(wl, stream);
     return SP24_ERR_DTYPE;
   }
   if (sparse)
@@ -715,6 +718,58 @@ int run_gemm(const sp24_gemm_args* a, cudaStream_t stream) {
     return st;
   g_cache_single.put(key, v);
   return dispatch_gemm(v.pl, v.gl, stream);
+}
+
+// The GEMM of the online-activation path: X (compressed, M rows) is the
+// sparse operand A, W (dense, N rows) is B, Y [M x N].
+int run_activation_gemm(bool bf16, const void* x_values, const void* x_meta, const float* x_scales,
+                        const void* W, int64_t ldw, const float* w_scales, int64_t M, int64_t N, int64_t K,
+                        void* Y, int64_t ldy, bool out_f32, const DeviceInfo& di, cudaStream_t s) {
+  if (use_pair(M, N, false, 0))
+    return run_wide(kModeSparse, bf16, false, x_values, K / 2, x_meta, W, ldw, M, N, K, x_scales, w_scales, Y,
+                    ldy, out_f32, s);
+  const int eb = bf16 ? 2 : 1;
+  const int box_elems = 128 / eb;
+  Plan pl;
+  memset(&pl, 0, sizeof pl);
+  pl.mode = kModeSparse;
+  pl.bf16 = bf16;
+  pl.a_is_w = false;
+  pl.bn = 128;
+  pl.kt = stage_k(kModeSparse, bf16);
+  pl.n = 1;
+  pl.num_kt[0] = (int)((K + pl.kt - 1) / pl.kt);
+  pl.tiles_a[0] = (int)((M + 127) / 128);
+  pl.tiles_b[0] = (int)((N + 127) / 128);
+  choose_schedule(pl, di.sms, 0);  // whole tiles: no workspace for partial sums
+  GemmLaunch<1> gl;
+  memset(&gl, 0, sizeof gl);
+  bool ok = make_map(&gl.tm_a[0], x_values, eb, K / 2, M, (K / 2) * eb, box_elems, kBlockA,
+                     CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= make_map(&gl.tm_b[0], W, eb, K, N, ldw * eb, box_elems, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!ok) return SP24_ERR_CUDA;
+  gl.tm_a2[0] = gl.tm_a[0];
+  GemmProblem& P = gl.prob[0];
+  P.rows_a = (int32_t)M;
+  P.rows_b = (int32_t)N;
+  P.K = (int32_t)K;
+  P.num_kt = pl.num_kt[0];
+  P.tiles_a = pl.tiles_a[0];
+  P.tiles_b = pl.tiles_b[0];
+  P.meta_blocks = (int32_t)((M + 127) / 128);
+  P.meta = static_cast<const uint8_t*>(x_meta);
+  P.scale_a = x_scales;
+  P.scale_b = w_scales;
+  P.Y = Y;
+  P.ldy = ldy;
+  gl.p.n_prob = 1;
+  gl.p.sched = pl.sched;
+  gl.p.total_iters = pl.total_iters;
+  gl.p.total_tiles = pl.total_tiles;
+  gl.p.out_f32 = out_f32 ? 1 : 0;
+  gl.p.use_pdl = 1;
+  gl.p.timeout_ns = g_timeout_ns.load();
+  return dispatch_gemm(pl, gl, s);
 }
 
 // Checks that n problems can share one grouped launch.
@@ -1050,6 +1105,57 @@ size_t sp24_activations_workspace_bytes(int64_t M, int64_t K) {
   return vals + sp24_meta_bytes(M, K);
 }
 
+size_t sp24_activations_e4m3_workspace_bytes(int64_t M, int64_t K) {
+  if (M < 1 || K < 128) return 0;
+  const size_t vals = ((size_t)M * (size_t)(K / 2) + 255) & ~(size_t)255;
+  const size_t meta = (sp24_meta_bytes(M, K) + 255) & ~(size_t)255;
+  return vals + meta + (size_t)M * sizeof(float);
+}
+
+int sp24_prune_compress_activations_fused_e4m3(const void* X, int64_t M, int64_t K, int64_t ldx, const void* Wq,
+                                               const float* w_scales, int64_t N, int64_t ldw, void* Y, int64_t ldy,
+                                               sp24_dtype out_dtype, void* x_values, void* x_meta, float* x_scales,
+                                               void* workspace, size_t workspace_bytes, void* stream) {
+  if (X == nullptr || Wq == nullptr || w_scales == nullptr || Y == nullptr) return SP24_ERR_NULL;
+  if (out_dtype != SP24_BF16 && out_dtype != SP24_F32) return SP24_ERR_DTYPE;
+  if (M < 1 || N < 1 || K < 128 || ldx < K || ldw < K || ldy < N) return SP24_ERR_INVALID_ARG;
+  if (K % 128 != 0) return SP24_ERR_NOT_2_4;
+  const bool have_v = x_values != nullptr, have_m = x_meta != nullptr, have_s = x_scales != nullptr;
+  if (have_v != have_m || have_v != have_s) return SP24_ERR_NULL;
+  if (ldx % 8 != 0 || ldw % 16 != 0 || !aligned16(X) || !aligned16(Wq)) return SP24_ERR_ALIGNMENT;
+  if (!aligned16(Y) || (ldy * (out_dtype == SP24_F32 ? 4 : 2)) % 16 != 0) return SP24_ERR_ALIGNMENT;
+  if (!have_v) {
+    if (workspace == nullptr) return SP24_ERR_WORKSPACE;
+    if (workspace_bytes < sp24_activations_e4m3_workspace_bytes(M, K)) return SP24_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return SP24_ERR_ALIGNMENT;
+    uint8_t* w = static_cast<uint8_t*>(workspace);
+    x_values = w;
+    w += ((size_t)M * (size_t)(K / 2) + 255) & ~(size_t)255;
+    x_meta = w;
+    w += (sp24_meta_bytes(M, K) + 255) & ~(size_t)255;
+    x_scales = reinterpret_cast<float*>(w);
+  }
+  if (!aligned16(x_values) || !aligned16(x_meta)) return SP24_ERR_ALIGNMENT;
+  DeviceInfo di;
+  int st = current_device_info(&di);
+  if (st != SP24_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // per-token amax, prune + compress + quantize with it, then amax -> scale
+  const uint16_t* x16 = static_cast<const uint16_t*>(X);
+  const int agrid = (int)std::min<int64_t>((M + 7) / 8, (int64_t)di.sms * 8);
+  k_row_amax<<<agrid, 256, 0, s>>>(x16, M, K, ldx, x_scales);
+  if ((st = launch_result(cudaGetLastError())) != SP24_OK) return st;
+  const int64_t chunks = ((M + 127) / 128) * (K / 128);
+  const int grid = (int)std::min<int64_t>(chunks, (int64_t)di.sms * 4);
+  k_prune_compress<true><<<grid, kPruneThreads, 0, s>>>(x16, M, K, ldx, x_values, static_cast<uint8_t*>(x_meta),
+                                                        x_scales, nullptr, nullptr);
+  if ((st = launch_result(cudaGetLastError())) != SP24_OK) return st;
+  k_finalize_scales<<<(int)((M + 255) / 256), 256, 0, s>>>(x_scales, M);
+  if ((st = launch_result(cudaGetLastError())) != SP24_OK) return st;
+  return run_activation_gemm(false, x_values, x_meta, x_scales, Wq, ldw, w_scales, M, N, K, Y, ldy,
+                             out_dtype == SP24_F32, di, s);
+}
+
 int sp24_prune_compress_activations_fused(const void* X, int64_t M, int64_t K, int64_t ldx,
                                           const void* W, int64_t N, int64_t ldw, void* Y, int64_t ldy,
                                           sp24_dtype out_dtype, void* x_values, void* x_meta,
@@ -1082,45 +1188,8 @@ int sp24_prune_compress_activations_fused(const void* X, int64_t M, int64_t K, i
   if (st != SP24_OK) return st;
 
   // GEMM with X (compressed) as the sparse operand A and W dense as B.
-  if (use_pair(M, N, false, 0))
-    return run_wide(kModeSparse, true, false, x_values, K / 2, x_meta, W, ldw, M, N, K, nullptr, nullptr, Y,
-                    ldy, out_dtype == SP24_F32, s);
-  Plan pl;
-  memset(&pl, 0, sizeof pl);
-  pl.mode = kModeSparse;
-  pl.bf16 = true;
-  pl.a_is_w = false;
-  pl.bn = 128;
-  pl.kt = 128;
-  pl.n = 1;
-  pl.num_kt[0] = (int)(K / 128);
-  pl.tiles_a[0] = (int)((M + 127) / 128);
-  pl.tiles_b[0] = (int)((N + 127) / 128);
-  choose_schedule(pl, di.sms, 0);  // whole tiles: no workspace for partial sums
-  GemmLaunch<1> gl;
-  memset(&gl, 0, sizeof gl);
-  bool ok = make_map(&gl.tm_a[0], x_values, 2, K / 2, M, (K / 2) * 2, 64, kBlockA, CU_TENSOR_MAP_SWIZZLE_128B);
-  ok &= make_map(&gl.tm_b[0], W, 2, K, N, ldw * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
-  if (!ok) return SP24_ERR_CUDA;
-  gl.tm_a2[0] = gl.tm_a[0];
-  GemmProblem& P = gl.prob[0];
-  P.rows_a = (int32_t)M;
-  P.rows_b = (int32_t)N;
-  P.K = (int32_t)K;
-  P.num_kt = pl.num_kt[0];
-  P.tiles_a = pl.tiles_a[0];
-  P.tiles_b = pl.tiles_b[0];
-  P.meta = static_cast<const uint8_t*>(x_meta);
-  P.Y = Y;
-  P.ldy = ldy;
-  gl.p.n_prob = 1;
-  gl.p.sched = pl.sched;
-  gl.p.total_iters = pl.total_iters;
-  gl.p.total_tiles = pl.total_tiles;
-  gl.p.out_f32 = out_dtype == SP24_F32;
-  gl.p.use_pdl = 1;
-  gl.p.timeout_ns = g_timeout_ns.load();
-  return dispatch_gemm(pl, gl, s);
+  return run_activation_gemm(true, x_values, x_meta, nullptr, W, ldw, nullptr, M, N, K, Y, ldy,
+                             out_dtype == SP24_F32, di, s);
 }
 
 int sp24_select_tactic(const sp24_gemm_args* sparse_args, const sp24_gemm_args* dense_args, int warmup,

@@ -107,6 +107,9 @@ def lib() -> ctypes.CDLL:
         "sp24_activations_workspace_bytes": (ctypes.c_size_t, [I64, I64]),
         "sp24_prune_compress_activations_fused": (I, [P, I64, I64, I64, P, I64, I64, P, I64, I,
                                                       P, P, P, ctypes.c_size_t, P]),
+        "sp24_activations_e4m3_workspace_bytes": (ctypes.c_size_t, [I64, I64]),
+        "sp24_prune_compress_activations_fused_e4m3": (I, [P, I64, I64, I64, P, P, I64, I64, P, I64, I,
+                                                           P, P, P, P, ctypes.c_size_t, P]),
         "sp24_select_tactic": (I, [ctypes.POINTER(GemmArgs), ctypes.POINTER(GemmArgs), I, I,
                                    ctypes.POINTER(TacticRecord), P]),
         "sp24_status_string": (ctypes.c_char_p, [I]),
@@ -346,6 +349,26 @@ def prune_compress_activations_fused(X: torch.Tensor, W: torch.Tensor, Y: torch.
         _ptr(X), M, K, X.stride(0), _ptr(W), N, W.stride(0), _ptr(Y), Y.stride(0),
         dtype_code(Y.dtype), _ptr(x_values), _ptr(x_meta), _ptr(workspace), ws_bytes,
         _stream(stream)), "sp24_prune_compress_activations_fused")
+
+
+def activations_e4m3_workspace_bytes(M: int, K: int) -> int:
+    return lib().sp24_activations_e4m3_workspace_bytes(M, K)
+
+
+def prune_compress_activations_fused_e4m3(X: torch.Tensor, Wq: torch.Tensor, w_scales: torch.Tensor,
+                                          Y: torch.Tensor, x_values: Optional[torch.Tensor] = None,
+                                          x_meta: Optional[torch.Tensor] = None,
+                                          x_scales: Optional[torch.Tensor] = None,
+                                          workspace: Optional[torch.Tensor] = None, stream=None):
+    """X bf16 [M x K] pruned 2:4 and cast to e4m3 per token each call, then
+    Y = X_sparse * Wq^T with Wq e4m3 [N x K] (per-channel scales)."""
+    M, K = X.shape
+    N = Wq.shape[0]
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().sp24_prune_compress_activations_fused_e4m3(
+        _ptr(X), M, K, X.stride(0), _ptr(Wq), _ptr(w_scales), N, Wq.stride(0), _ptr(Y), Y.stride(0),
+        dtype_code(Y.dtype), _ptr(x_values), _ptr(x_meta), _ptr(x_scales), _ptr(workspace), ws_bytes,
+        _stream(stream)), "sp24_prune_compress_activations_fused_e4m3")
 
 
 def select_tactic(sparse_args: Optional[GemmArgs], dense_args: GemmArgs, warmup: int = 3,

@@ -164,3 +164,22 @@ def test_grouped_gemm_validation():
 def test_grouped_gemm_without_device():
     arr = (sp24.GemmArgs * 2)(gemm_args(), gemm_args(M=3, N=512, K=512))
     assert L.sp24_gemm_grouped(arr, 2, None, 0, None) == sp24.SP24_ERR_UNSUPPORTED_DEVICE
+
+
+def test_activation_e4m3_validation():
+    f = L.sp24_prune_compress_activations_fused_e4m3
+    ok = dict(X=FAKE, M=16, K=256, ldx=256, W=FAKE, ws=FAKE, N=256, ldw=256, Y=FAKE, ldy=256, out=sp24.BF16,
+              xv=FAKE, xm=FAKE, xs=FAKE, work=None, wbytes=0)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return f(a["X"], a["M"], a["K"], a["ldx"], a["W"], a["ws"], a["N"], a["ldw"], a["Y"], a["ldy"], a["out"],
+                 a["xv"], a["xm"], a["xs"], a["work"], a["wbytes"], None)
+    assert call(ws=None) == sp24.SP24_ERR_NULL                  # weight scales required
+    assert call(xs=None) == sp24.SP24_ERR_NULL                  # all three outputs or none
+    assert call(xv=None, xm=None, xs=None) == sp24.SP24_ERR_WORKSPACE
+    assert call(K=192, ldx=192, ldw=192) == sp24.SP24_ERR_NOT_2_4
+    assert call(ldw=264) == sp24.SP24_ERR_ALIGNMENT             # e4m3 rows: 16-byte multiple
+    assert call(out=sp24.E4M3) == sp24.SP24_ERR_DTYPE
+    # values [16 x 128] e4m3 (2048 B) + image (one row block x 2 chunks) + 16 scales
+    assert sp24.activations_e4m3_workspace_bytes(16, 256) == 2048 + 2 * 2048 + 16 * 4

@@ -524,6 +524,37 @@ def _prepare_large(X_bits, W_bits, e4, tactic):
     return a, Y, None, None
 
 
+@pytest.mark.parametrize("M,N,K", [(128, 384, 512), (200, 256, 1280), (1, 128, 128), (512, 384, 512),
+                                   (300, 640, 768)])
+def test_activation_fused_e4m3_parity(M, N, K):
+    # X pruned 2:4 and cast to e4m3 per token on every call; the compressed
+    # activations are bit-exact to the oracle's, Y within tolerance
+    X = inputs.student_t_bf16((M, K), 3.0, seed=M + 7 * K)
+    W = inputs.normal_bf16((N, K), 0.02, seed=N + 1)
+    wq, wsc = orc.quantize_rows_e4m3(W)
+    Y = torch.empty(M, N, dtype=torch.float32, device="cuda")
+    xv = torch.empty(M, K // 2, dtype=torch.uint8, device="cuda")
+    xm = torch.empty(sp24.meta_bytes(M, K), dtype=torch.uint8, device="cuda")
+    xs = torch.empty(M, dtype=torch.float32, device="cuda")
+    sp24.prune_compress_activations_fused_e4m3(dev_bf16(X), dev(wq), dev(wsc), Y, x_values=xv, x_meta=xm,
+                                               x_scales=xs)
+    torch.cuda.synchronize()
+    assert sp24.last_device_error() == sp24.SP24_OK
+    ref = OracleSparseW(X, e4m3=True)  # the oracle's prune + per-row e4m3 cast, applied to X's rows
+    assert np.array_equal(u8(xv), ref.values)
+    assert np.array_equal(u8(xm), ref.image)
+    assert np.array_equal(xs.cpu().numpy().view(np.uint32), ref.scales.view(np.uint32))
+    W_hat = orc.e4m3_decode(wq) * wsc.astype(np.float64)[:, None]
+    y_ref, a_ref = orc.gemm_f64(ref.W_hat, W_hat)
+    check_tolerance(Y.cpu().numpy().astype(np.float64), y_ref, a_ref, "activations e4m3 M%d N%d K%d" % (M, N, K))
+    # workspace variant, bf16 output
+    ws = torch.empty(sp24.activations_e4m3_workspace_bytes(M, K), dtype=torch.uint8, device="cuda")
+    Y2 = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    sp24.prune_compress_activations_fused_e4m3(dev_bf16(X), dev(wq), dev(wsc), Y2, workspace=ws)
+    torch.cuda.synchronize()
+    check_tolerance(Y2.float().cpu().numpy().astype(np.float64), y_ref, a_ref, "activations e4m3 ws")
+
+
 @pytest.mark.parametrize("M,N,K", [(512, 384, 512), (300, 256, 1024)])
 def test_activation_fused_pair_kernel(M, N, K):
     test_activation_fused_parity(M, N, K)
