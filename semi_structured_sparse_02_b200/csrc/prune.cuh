@@ -41,6 +41,30 @@ __device__ __forceinline__ uint32_t prune_group4(uint32_t a0, uint32_t a1, uint3
   return (uint32_t)i0 | ((uint32_t)i1 << 2);
 }
 
+// The same rule on full bf16 bit patterns, returning the two kept values
+// (ascending index) by selects rather than by indexing, which would put the
+// group in local memory.
+__device__ __forceinline__ uint32_t prune_pick4(uint32_t x0, uint32_t x1, uint32_t x2, uint32_t x3,
+                                                uint32_t& kept0, uint32_t& kept1) {
+  const uint32_t a0 = x0 & 0x7FFFu, a1 = x1 & 0x7FFFu, a2 = x2 & 0x7FFFu, a3 = x3 & 0x7FFFu;
+  const int l0 = (a1 > a0) + (a2 > a0) + (a3 > a0);
+  const int l1 = (a0 >= a1) + (a2 > a1) + (a3 > a1);
+  const int l2 = (a0 >= a2) + (a1 >= a2) + (a3 > a2);
+  const int l3 = (a0 >= a3) + (a1 >= a3) + (a2 >= a3);
+  const bool k0 = l0 < 2, k1 = l1 < 2, k2 = l2 < 2, k3 = l3 < 2;
+  const uint32_t i0 = k0 ? 0u : (k1 ? 1u : 2u);
+  const uint32_t i1 = k3 ? 3u : (k2 ? 2u : 1u);
+  kept0 = k0 ? x0 : (k1 ? x1 : x2);
+  kept1 = k3 ? x3 : (k2 ? x2 : x1);
+  return i0 | (i1 << 2);
+}
+
+// Two E4M3 codes (round to nearest even, saturating) in the low 16 bits:
+// lo in bits 0..7, hi in bits 8..15.
+__device__ __forceinline__ uint32_t e4m3x2_of(float lo, float hi) {
+  return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3);
+}
+
 __device__ __forceinline__ uint8_t e4m3_of(float v) {
   return (uint8_t)__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3);
 }
@@ -92,6 +116,7 @@ k_prune_compress(const uint16_t* __restrict__ src, int64_t rows, int64_t K, int6
                  const float* __restrict__ amax_in, const uint8_t* __restrict__ tile_mask,
                  void* __restrict__ dense_out) {
   __shared__ __align__(16) uint8_t canon[kChunkRows][16];
+  __shared__ float s_inv[kChunkRows];  // E4M3: 448 / amax of each row of the chunk
   pdl_launch_dependents();
   pdl_wait();  // src may be written by the upstream grid
   const int64_t KC = K / kChunkK;
@@ -102,6 +127,14 @@ k_prune_compress(const uint16_t* __restrict__ src, int64_t rows, int64_t K, int6
   for (int64_t c = blockIdx.x; c < n_chunks; c += gridDim.x) {
     const int64_t rb = c / KC, kc = c % KC;
     const bool dense_tile = tile_mask != nullptr && tile_mask[c] != 0;
+    if (kOutE4M3) {
+      // one correctly rounded division per row of the chunk, not per element
+      if (threadIdx.x < kChunkRows) {
+        const int64_t row = rb * kChunkRows + threadIdx.x;
+        s_inv[threadIdx.x] = row < rows ? e4m3_inv_scale(amax_in[row]) : 0.0f;
+      }
+      __syncthreads();
+    }
     for (int i = threadIdx.x; i < kChunkRows * 16; i += kPruneThreads) {
       const int rl = i >> 4, seg = i & 15;
       const int64_t row = rb * kChunkRows + rl;
@@ -109,58 +142,40 @@ k_prune_compress(const uint16_t* __restrict__ src, int64_t rows, int64_t K, int6
       uint4 v = make_uint4(0, 0, 0, 0);
       const bool live = row < rows;
       if (live) v = __ldg(reinterpret_cast<const uint4*>(src + row * ld + k0));
-      const uint32_t e[8] = {v.x & 0xFFFFu, v.x >> 16, v.y & 0xFFFFu, v.y >> 16,
-                             v.z & 0xFFFFu, v.z >> 16, v.w & 0xFFFFu, v.w >> 16};
-      float inv = 0.0f;
-      if (kOutE4M3 && live) inv = e4m3_inv_scale(amax_in[row]);
-      uint32_t nib[2];
-      uint32_t kept[4];
+      const uint32_t e0 = v.x & 0xFFFFu, e1 = v.x >> 16, e2 = v.y & 0xFFFFu, e3 = v.y >> 16;
+      const uint32_t e4 = v.z & 0xFFFFu, e5 = v.z >> 16, e6 = v.w & 0xFFFFu, e7 = v.w >> 16;
+      const float inv = kOutE4M3 ? s_inv[rl] : 0.0f;
+      uint32_t nib0, nib1, k00 = 0, k01 = 0, k10 = 0, k11 = 0;
       if (dense_tile) {
-        nib[0] = nib[1] = 0x4u;
-        kept[0] = kept[1] = kept[2] = kept[3] = 0u;
+        nib0 = nib1 = 0x4u;
         if (live) {
           if (kOutE4M3) {
-            uint32_t q0 = 0, q1 = 0;
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              q0 |= (uint32_t)e4m3_of(__fmul_rn(bf16_bits_to_float(e[j]), inv)) << (8 * j);
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              q1 |= (uint32_t)e4m3_of(__fmul_rn(bf16_bits_to_float(e[4 + j]), inv)) << (8 * j);
-            *reinterpret_cast<uint2*>(static_cast<uint8_t*>(dense_out) + row * K + k0) =
-                make_uint2(q0, q1);
+            const uint32_t q0 = e4m3x2_of(__fmul_rn(bf16_bits_to_float(e0), inv), __fmul_rn(bf16_bits_to_float(e1), inv)) |
+                                (e4m3x2_of(__fmul_rn(bf16_bits_to_float(e2), inv), __fmul_rn(bf16_bits_to_float(e3), inv)) << 16);
+            const uint32_t q1 = e4m3x2_of(__fmul_rn(bf16_bits_to_float(e4), inv), __fmul_rn(bf16_bits_to_float(e5), inv)) |
+                                (e4m3x2_of(__fmul_rn(bf16_bits_to_float(e6), inv), __fmul_rn(bf16_bits_to_float(e7), inv)) << 16);
+            *reinterpret_cast<uint2*>(static_cast<uint8_t*>(dense_out) + row * K + k0) = make_uint2(q0, q1);
           } else {
             *reinterpret_cast<uint4*>(static_cast<uint16_t*>(dense_out) + row * K + k0) = v;
           }
         }
       } else {
-#pragma unroll
-        for (int g = 0; g < 2; ++g) {
-          const uint32_t* x = e + 4 * g;
-          int i0, i1;
-          nib[g] = prune_group4(x[0] & 0x7FFFu, x[1] & 0x7FFFu, x[2] & 0x7FFFu, x[3] & 0x7FFFu,
-                                i0, i1);
-          kept[2 * g + 0] = x[i0];
-          kept[2 * g + 1] = x[i1];
-        }
+        nib0 = prune_pick4(e0, e1, e2, e3, k00, k01);
+        nib1 = prune_pick4(e4, e5, e6, e7, k10, k11);
       }
       if (live) {
         if (kOutE4M3) {
           uint32_t q = 0;
-          if (!dense_tile) {
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              q |= (uint32_t)e4m3_of(__fmul_rn(bf16_bits_to_float(kept[j]), inv)) << (8 * j);
-          }
-          *reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(values) + row * half_k + kc * 64 +
-                                       seg * 4) = q;
+          if (!dense_tile)
+            q = e4m3x2_of(__fmul_rn(bf16_bits_to_float(k00), inv), __fmul_rn(bf16_bits_to_float(k01), inv)) |
+                (e4m3x2_of(__fmul_rn(bf16_bits_to_float(k10), inv), __fmul_rn(bf16_bits_to_float(k11), inv)) << 16);
+          *reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(values) + row * half_k + kc * 64 + seg * 4) = q;
         } else {
-          *reinterpret_cast<uint2*>(static_cast<uint16_t*>(values) + row * half_k + kc * 64 +
-                                    seg * 4) =
-              make_uint2(kept[0] | (kept[1] << 16), kept[2] | (kept[3] << 16));
+          *reinterpret_cast<uint2*>(static_cast<uint16_t*>(values) + row * half_k + kc * 64 + seg * 4) =
+              make_uint2(k00 | (k01 << 16), k10 | (k11 << 16));
         }
       }
-      canon[rl][seg] = (uint8_t)(nib[0] | (nib[1] << 4));
+      canon[rl][seg] = (uint8_t)(nib0 | (nib1 << 4));
     }
     __syncthreads();
     if (threadIdx.x < kChunkRows) {

@@ -941,7 +941,7 @@ int sp24_prune_compress(const void* src, int64_t rows, int64_t K, int64_t ld, sp
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const uint16_t* src16 = static_cast<const uint16_t*>(src);
   const int64_t chunks = ((rows + 127) / 128) * (K / 128);
-  const int grid = (int)std::min<int64_t>(chunks, (int64_t)di.sms * 4);
+  const int grid = (int)std::min<int64_t>(chunks, (int64_t)di.sms * 8);
   uint8_t* meta8 = static_cast<uint8_t*>(meta);
   if (out_dtype == SP24_BF16) {
     k_prune_compress<false><<<grid, kPruneThreads, 0, s>>>(src16, rows, K, ld, values, meta8, nullptr,
@@ -970,7 +970,7 @@ int sp24_decompress(const void* values, const void* meta, int64_t rows, int64_t 
   if (st != SP24_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int64_t chunks = ((rows + 127) / 128) * (K / 128);
-  const int grid = (int)std::min<int64_t>(chunks, (int64_t)di.sms * 4);
+  const int grid = (int)std::min<int64_t>(chunks, (int64_t)di.sms * 8);
   const uint8_t* m8 = static_cast<const uint8_t*>(meta);
   if (dtype == SP24_BF16) k_decompress<false><<<grid, kPruneThreads, 0, s>>>(values, m8, rows, K, dst);
   else k_decompress<true><<<grid, kPruneThreads, 0, s>>>(values, m8, rows, K, dst);
@@ -1146,7 +1146,7 @@ int sp24_prune_compress_activations_fused_e4m3(const void* X, int64_t M, int64_t
   k_row_amax<<<agrid, 256, 0, s>>>(x16, M, K, ldx, x_scales);
   if ((st = launch_result(cudaGetLastError())) != SP24_OK) return st;
   const int64_t chunks = ((M + 127) / 128) * (K / 128);
-  const int grid = (int)std::min<int64_t>(chunks, (int64_t)di.sms * 4);
+  const int grid = (int)std::min<int64_t>(chunks, (int64_t)di.sms * 8);
   k_prune_compress<true><<<grid, kPruneThreads, 0, s>>>(x16, M, K, ldx, x_values, static_cast<uint8_t*>(x_meta),
                                                         x_scales, nullptr, nullptr);
   if ((st = launch_result(cudaGetLastError())) != SP24_OK) return st;
@@ -1180,7 +1180,7 @@ int sp24_prune_compress_activations_fused(const void* X, int64_t M, int64_t K, i
   if (st != SP24_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int64_t chunks = ((M + 127) / 128) * (K / 128);
-  const int grid = (int)std::min<int64_t>(chunks, (int64_t)di.sms * 4);
+  const int grid = (int)std::min<int64_t>(chunks, (int64_t)di.sms * 8);
   st = launch_pdl(k_prune_compress<false>, dim3(grid), dim3(kPruneThreads), 0, s,
                   static_cast<const uint16_t*>(X), M, K, ldx, x_values, static_cast<uint8_t*>(x_meta),
                   static_cast<const float*>(nullptr), static_cast<const uint8_t*>(nullptr),
