@@ -58,6 +58,7 @@ def lib() -> ctypes.CDLL:
             "orc_gemm_f64_sampled": (None, [P, P, I64, P, P, I64, P, P]),
             "orc_gemm_sparse_f64": (None, [P, I64, I64, P, P, I64, P]),
             "orc_bf16_to_double": (ctypes.c_double, [ctypes.c_uint16]),
+            "orc_energy_loss": (None, [P, I64, I64, I64, P, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -164,6 +165,20 @@ def prune_compress_e4m3(W_bits: np.ndarray, mask: Optional[np.ndarray] = None):
     lib().orc_prune_compress_e4m3(_p(W), rows, K, K, _p(m), _p(values), _p(meta),
                                   _p(scales), _p(dense))
     return values, meta, scales, dense
+
+
+def energy_loss(W_bits: np.ndarray):
+    """2:4 energy loss [P4 sections 1 and 5]: (per-row dropped energy, per-row
+    total energy, per-row share, tensor share).  A row (or tensor) with no
+    energy has share 0 (reading)."""
+    W = np.ascontiguousarray(W_bits, dtype=np.uint16)
+    rows, K = W.shape
+    dropped = np.empty(rows, np.float64)
+    total = np.empty(rows, np.float64)
+    lib().orc_energy_loss(_p(W), rows, K, K, _p(dropped), _p(total))
+    share = np.where(total > 0, dropped / np.where(total > 0, total, 1.0), 0.0)
+    t = total.sum()
+    return dropped, total, share, (dropped.sum() / t if t > 0 else 0.0)
 
 
 def decompress(values: np.ndarray, meta_canon: np.ndarray, rows: int, K: int) -> np.ndarray:

@@ -471,3 +471,34 @@ void orc_e4m3_encode_array(const double *x, int64_t n, uint8_t *q)
 {
     for (int64_t i = 0; i < n; ++i) q[i] = orc_e4m3_encode(x[i]);
 }
+
+/* ------------------------------------------------------------------ */
+/* 2:4 energy loss  [P4 section 1 and section 5, "The energy that 2:4  */
+/*    removes": the share of a tensor's energy carried by the two      */
+/*    values that 2:4 drops from each group of four]                   */
+/* ------------------------------------------------------------------ */
+
+/* For each row: the energy (sum of squares) of the values the 2:4 prune
+ * drops, and the energy of the whole row, both in fp64 (a bf16 square is
+ * exact in fp64).  The share is dropped / total, per row and summed over
+ * rows for the tensor.  The dropped positions are those orc_prune_group
+ * does not keep. */
+void orc_energy_loss(const uint16_t *src, int64_t rows, int64_t K, int64_t ld,
+                     double *row_dropped, double *row_total)
+{
+    for (int64_t r = 0; r < rows; ++r) {
+        double dropped = 0.0, total = 0.0;
+        for (int64_t g = 0; g < K / 4; ++g) {
+            const uint16_t *v = src + r * ld + 4 * g;
+            int i0, i1;
+            orc_prune_group(v, &i0, &i1);
+            for (int i = 0; i < 4; ++i) {
+                const double x = orc_bf16_to_double(v[i]);
+                total += x * x;
+                if (i != i0 && i != i1) dropped += x * x;
+            }
+        }
+        row_dropped[r] = dropped;
+        row_total[r] = total;
+    }
+}

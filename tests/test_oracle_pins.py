@@ -340,3 +340,50 @@ def test_manifest_example_arithmetic_and_tactic_rule():
     assert orc.select_tactic([1.0, 1.5, 9.0], [2.0, 2.0, 2.0])[0] == "sparse"
     cov = orc.sparse_gpu_time_coverage([("sparse", 0.684), ("dense", 0.316)])
     assert abs(cov - m["sparse_gpu_time_coverage"]) < 1e-12
+
+
+# ---------------------------------------------------------------------------
+# 2:4 energy loss: the page's worked example, closed forms, brute force
+# ---------------------------------------------------------------------------
+
+def test_energy_loss_worked_example():
+    # the page's group keeps 0.42 and 0.31 and drops -0.18 and 0.07: the
+    # dropped share is (0.18^2 + 0.07^2) / (sum of all four squares), here
+    # on the bf16 values of the four numbers
+    g = json.load(open(os.path.join(GOLDEN, "worked_example.json")))
+    v = bf16(g["dense"])
+    x = [float(t) for t in torch.from_numpy(v.view(np.int16)).view(torch.bfloat16).float()]
+    dropped, total, share, tensor = orc.energy_loss(v.reshape(1, 4))
+    assert dropped[0] == x[1] ** 2 + x[2] ** 2
+    assert total[0] == sum(t * t for t in x)
+    assert share[0] == pytest.approx(0.0373 / 0.3098, rel=2e-2)  # the decimal values, before bf16 rounding
+    assert tensor == share[0]
+
+
+def test_energy_loss_closed_forms():
+    # equal magnitudes in every group: exactly half the energy is dropped
+    row = bf16(np.tile([1.5, -1.5, 1.5, -1.5], 16)).reshape(2, 32)
+    _, _, share, tensor = orc.energy_loss(row)
+    assert share.tolist() == [0.5, 0.5] and tensor == 0.5
+    # two zeros in every group (an already 2:4 tensor): nothing is dropped
+    row = bf16(np.tile([0.0, 3.0, 0.0, -2.0], 8)).reshape(1, 32)
+    assert orc.energy_loss(row)[2][0] == 0.0
+    # a row of zeros has no energy: share 0 (reading)
+    assert orc.energy_loss(np.zeros((1, 8), np.uint16))[2][0] == 0.0
+    # scaling by a power of two scales both energies alike: the share is unchanged
+    W = inputs.normal_bf16((4, 64), 1.0, seed=11)
+    W2 = bf16(torch.from_numpy(W.view(np.int16)).view(torch.bfloat16).float().numpy() * 8.0)
+    assert np.array_equal(orc.energy_loss(W)[2], orc.energy_loss(W2)[2])
+
+
+def test_energy_loss_brute_force_by_sorting():
+    # independent of the prune rule: in every group the two smallest squares
+    # are dropped (ties do not matter for the energy)
+    W = inputs.student_t_bf16((6, 128), 3.0, seed=5)
+    x = torch.from_numpy(W.view(np.int16)).view(torch.bfloat16).double().numpy()
+    sq = np.sort((x.reshape(6, 32, 4)) ** 2, axis=2)
+    dropped = sq[:, :, :2].sum(axis=(1, 2))
+    total = (x ** 2).sum(axis=1)
+    d, t, share, tensor = orc.energy_loss(W)
+    assert np.allclose(d, dropped, rtol=1e-14, atol=0) and np.allclose(t, total, rtol=1e-14, atol=0)
+    assert tensor == pytest.approx(dropped.sum() / total.sum(), rel=1e-14)
