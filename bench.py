@@ -833,6 +833,15 @@ def run_config(args):
             rows.append(dict(weights=name, N=N, K=K, out="e4m3" if e4 else "bf16", us=round(t, 2),
                              gbs=round(byts / t / 1e3, 1), frac_hbm=round(byts / t / 1e3 / hbm, 4)))
             print(json.dumps(rows[-1]), file=sys.stderr, flush=True)
+            # the 2:4 energy-loss diagnostic on the same weights: reads 2 B per element
+            share = torch.empty(N, dtype=torch.float64, device=dev)
+            sums = torch.empty(2, dtype=torch.float64, device=dev)
+            te, _ = _time_calls(lambda: sp24.energy_loss(W, share, sums), reps, warm, flush)
+            eb_ = 2 * N * K + 8 * N
+            rows.append(dict(energy_loss=name, N=N, K=K, us=round(te, 2), gbs=round(eb_ / te / 1e3, 1),
+                             frac_hbm=round(eb_ / te / 1e3 / hbm, 4),
+                             e24=round(float(sums[0] / sums[1]), 5)))
+            del share, sums
             del W, vals, meta, sc
     out["rows"] = rows
     print(json.dumps(out), flush=True)

@@ -310,6 +310,21 @@ int sp24_prune_compress_activations_fused_e4m3(const void *X_dev, int64_t M, int
                                                void *x_values_dev, void *x_meta_dev, float *x_scales_dev,
                                                void *workspace_dev, size_t workspace_bytes, void *stream);
 
+/* The 2:4 energy loss e_2:4 of a bf16 matrix [rows x K] (row-major, ld
+ * elements): the share of the energy (sum of squares) carried by the two
+ * values that the 2:4 prune of sp24_prune_compress drops from every group of
+ * four along K ("the 2:4 energy loss": 2:4-versus-quantization paper,
+ * section 1 and section 5, "The energy that 2:4 removes"), as a cheap
+ * diagnostic next to the prune.  row_share_dev [rows] (fp64, may be NULL)
+ * receives each row's share (0 for a row with no energy); sums_dev [2] (fp64,
+ * may be NULL) receives the dropped and the total energy of the whole
+ * tensor, so e_2:4 = sums[0] / sums[1] (the call zeroes sums first; the
+ * atomic accumulation order varies, within fp64 rounding).  At least one
+ * output is required.  K must be a multiple of 8, ld a multiple of 8, src
+ * 16-byte aligned.  Asynchronous on `stream`. */
+int sp24_energy_loss(const void *src_dev, int64_t rows, int64_t K, int64_t ld, double *row_share_dev,
+                     double *sums_dev, void *stream);
+
 /* ---------------------------------------------------------------------- */
 /* Tactic selection (kernel 5)                                             */
 /* ---------------------------------------------------------------------- */

@@ -210,6 +210,65 @@ k_row_amax(const uint16_t* __restrict__ src, int64_t rows, int64_t K, int64_t ld
   }
 }
 
+// ---------------------------------------------------------------------------
+// 2:4 energy loss: per row, the energy (sum of squares, fp64: a bf16 square
+// is exact) of the two values of each group that the prune drops, and of the
+// whole row.  One warp per row; the row share goes to row_share (if given)
+// and both energies are added into sums[0] (dropped) and sums[1] (total).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+k_energy_loss(const uint16_t* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
+              double* __restrict__ row_share, double* __restrict__ sums) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int64_t n_warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t row = warp; row < rows; row += n_warps) {
+    double dropped = 0.0, total = 0.0;
+    const uint4* p = reinterpret_cast<const uint4*>(src + row * ld);
+    const int64_t nv = K / 8;
+    auto fold = [&](const uint4& v) {
+      const uint32_t e[8] = {v.x & 0xFFFFu, v.x >> 16, v.y & 0xFFFFu, v.y >> 16,
+                             v.z & 0xFFFFu, v.z >> 16, v.w & 0xFFFFu, v.w >> 16};
+#pragma unroll
+      for (int g = 0; g < 2; ++g) {
+        uint32_t k0, k1;
+        prune_pick4(e[4 * g], e[4 * g + 1], e[4 * g + 2], e[4 * g + 3], k0, k1);
+        double all = 0.0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const double x = (double)bf16_bits_to_float(e[4 * g + j]);
+          all += x * x;
+        }
+        const double a = (double)bf16_bits_to_float(k0), b = (double)bf16_bits_to_float(k1);
+        total += all;
+        dropped += all - (a * a + b * b);
+      }
+    };
+    // four 16-byte loads in flight per lane, then the remainder
+    int64_t i = lane;
+    for (; i + 96 < nv; i += 128) {
+      uint4 v[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) v[j] = __ldg(p + i + 32 * j);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) fold(v[j]);
+    }
+    for (; i < nv; i += 32) fold(__ldg(p + i));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      dropped += __shfl_xor_sync(0xFFFFFFFFu, dropped, o);
+      total += __shfl_xor_sync(0xFFFFFFFFu, total, o);
+    }
+    if (lane == 0) {
+      if (row_share != nullptr) row_share[row] = total > 0.0 ? dropped / total : 0.0;
+      if (sums != nullptr) {
+        atomicAdd(sums, dropped);
+        atomicAdd(sums + 1, total);
+      }
+    }
+  }
+}
+
 // scale = amax / 448 (correctly rounded), 1 when amax == 0; in place.
 __global__ void k_finalize_scales(float* __restrict__ s, int64_t rows) {
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;

@@ -1099,6 +1099,26 @@ int sp24_gemm_noalloc(const sp24_gemm_args* a, void* stream) {
 
 size_t sp24_gemm_noalloc_max_scratch_bytes(void) { return kStaticScratchBytes; }
 
+int sp24_energy_loss(const void* src, int64_t rows, int64_t K, int64_t ld, double* row_share, double* sums,
+                     void* stream) {
+  if (src == nullptr) return SP24_ERR_NULL;
+  if (row_share == nullptr && sums == nullptr) return SP24_ERR_NULL;
+  if (rows < 1 || K < 8 || ld < K) return SP24_ERR_INVALID_ARG;
+  if (K % 8 != 0) return SP24_ERR_NOT_2_4;
+  if (ld % 8 != 0 || !aligned16(src)) return SP24_ERR_ALIGNMENT;
+  DeviceInfo di;
+  int st = current_device_info(&di);
+  if (st != SP24_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (sums != nullptr && cudaMemsetAsync(sums, 0, 2 * sizeof(double), s) != cudaSuccess) {
+    cudaGetLastError();
+    return SP24_ERR_CUDA;
+  }
+  const int grid = (int)std::min<int64_t>((rows + 7) / 8, (int64_t)di.sms * 8);
+  k_energy_loss<<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(src), rows, K, ld, row_share, sums);
+  return launch_result(cudaGetLastError());
+}
+
 size_t sp24_activations_workspace_bytes(int64_t M, int64_t K) {
   if (M < 1 || K < 128) return 0;
   const size_t vals = ((size_t)M * (size_t)(K / 2) * 2 + 255) & ~(size_t)255;

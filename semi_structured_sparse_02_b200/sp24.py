@@ -108,6 +108,7 @@ def lib() -> ctypes.CDLL:
         "sp24_prune_compress_activations_fused": (I, [P, I64, I64, I64, P, I64, I64, P, I64, I,
                                                       P, P, P, ctypes.c_size_t, P]),
         "sp24_activations_e4m3_workspace_bytes": (ctypes.c_size_t, [I64, I64]),
+        "sp24_energy_loss": (I, [P, I64, I64, I64, P, P, P]),
         "sp24_prune_compress_activations_fused_e4m3": (I, [P, I64, I64, I64, P, P, I64, I64, P, I64, I,
                                                            P, P, P, P, ctypes.c_size_t, P]),
         "sp24_select_tactic": (I, [ctypes.POINTER(GemmArgs), ctypes.POINTER(GemmArgs), I, I,
@@ -349,6 +350,15 @@ def prune_compress_activations_fused(X: torch.Tensor, W: torch.Tensor, Y: torch.
         _ptr(X), M, K, X.stride(0), _ptr(W), N, W.stride(0), _ptr(Y), Y.stride(0),
         dtype_code(Y.dtype), _ptr(x_values), _ptr(x_meta), _ptr(workspace), ws_bytes,
         _stream(stream)), "sp24_prune_compress_activations_fused")
+
+
+def energy_loss(src: torch.Tensor, row_share: Optional[torch.Tensor] = None,
+                sums: Optional[torch.Tensor] = None, stream=None):
+    """2:4 energy loss of a bf16 matrix: per-row share (fp64 [rows]) and/or the
+    tensor's dropped and total energy (fp64 [2])."""
+    rows, K = src.shape
+    _check(lib().sp24_energy_loss(_ptr(src), rows, K, src.stride(0), _ptr(row_share), _ptr(sums),
+                                  _stream(stream)), "sp24_energy_loss")
 
 
 def activations_e4m3_workspace_bytes(M: int, K: int) -> int:

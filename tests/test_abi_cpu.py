@@ -183,3 +183,13 @@ def test_activation_e4m3_validation():
     assert call(out=sp24.E4M3) == sp24.SP24_ERR_DTYPE
     # values [16 x 128] e4m3 (2048 B) + image (one row block x 2 chunks) + 16 scales
     assert sp24.activations_e4m3_workspace_bytes(16, 256) == 2048 + 2 * 2048 + 16 * 4
+
+
+def test_energy_loss_validation():
+    f = L.sp24_energy_loss
+    assert f(None, 4, 64, 64, FAKE, None, None) == sp24.SP24_ERR_NULL
+    assert f(FAKE, 4, 64, 64, None, None, None) == sp24.SP24_ERR_NULL      # one output at least
+    assert f(FAKE, 0, 64, 64, FAKE, None, None) == sp24.SP24_ERR_INVALID_ARG
+    assert f(FAKE, 4, 60, 60, FAKE, None, None) == sp24.SP24_ERR_NOT_2_4
+    assert f(FAKE, 4, 64, 68, FAKE, None, None) == sp24.SP24_ERR_ALIGNMENT
+    assert f(FAKE + 8, 4, 64, 64, FAKE, None, None) == sp24.SP24_ERR_ALIGNMENT

@@ -561,6 +561,36 @@ def test_activation_fused_pair_kernel(M, N, K):
 
 
 # ---------------------------------------------------------------------------
+# 2:4 energy loss (diagnostic next to the prune)
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("rows,K,dist", [(1, 256, "normal"), (200, 1024, "student"), (5120, 5120, "normal"),
+                                         (37, 4096, "student")])
+def test_energy_loss_matches_oracle(rows, K, dist):
+    if dist == "normal":
+        W = inputs.normal_bf16((rows, K), 0.02, seed=rows + K)
+    else:
+        W = inputs.student_t_bf16((rows, K), 3.0, seed=rows + K)
+    W[0, : min(K, 64)] = 0  # a stretch of zeros (kept zeros)
+    share = torch.empty(rows, dtype=torch.float64, device="cuda")
+    sums = torch.full((2,), 7.0, dtype=torch.float64, device="cuda")  # the call zeroes it
+    sp24.energy_loss(dev_bf16(W), share, sums)
+    torch.cuda.synchronize()
+    d, t, sh, e = orc.energy_loss(W)
+    assert np.allclose(share.cpu().numpy(), sh, rtol=1e-12, atol=1e-15)
+    s = sums.cpu().numpy()
+    assert s[0] == pytest.approx(d.sum(), rel=1e-12) and s[1] == pytest.approx(t.sum(), rel=1e-12)
+    assert s[0] / s[1] == pytest.approx(e, rel=1e-12)
+
+
+def test_energy_loss_zero_rows():
+    W = np.zeros((3, 64), np.uint16)
+    share = torch.full((3,), 5.0, dtype=torch.float64, device="cuda")
+    sp24.energy_loss(dev_bf16(W), share, None)
+    torch.cuda.synchronize()
+    assert share.cpu().numpy().tolist() == [0.0, 0.0, 0.0]
+
+
+# ---------------------------------------------------------------------------
 # full-size configurations, sampled outputs
 # ---------------------------------------------------------------------------
 
