@@ -286,7 +286,8 @@ __global__ void k_finalize_scales(float* __restrict__ s, int64_t rows) {
 // ---------------------------------------------------------------------------
 constexpr int kQuantThreads = 256;
 constexpr int kQuantRegVecs = 4;
-constexpr int kQuantCtasPerSm = 6;  // resident per SM at the register use of this kernel
+constexpr int kQuantPassVecs = 8;   // loads in flight per thread on long rows
+constexpr int kQuantCtasPerSm = 5;  // resident per SM at the register use of this kernel
 constexpr int kMaxQuantItems = 32;
 
 struct QuantItem {
@@ -368,31 +369,31 @@ k_quantize_rows_e4m3(const __grid_constant__ QuantGroup g) {
         if (idx < nv) *reinterpret_cast<uint2*>(q + idx * 8) = e4m3_codes8(reg[j], inv);
       }
     } else {
-      // long rows: an amax pass with kQuantRegVecs loads in flight per
+      // long rows: an amax pass with kQuantPassVecs loads in flight per
       // thread, then a second pass (served from L2) that writes the codes
       uint32_t m = 0;
-      for (int64_t base = threadIdx.x; base < nv; base += (int64_t)kQuantThreads * kQuantRegVecs) {
-        uint4 v[kQuantRegVecs];
+      for (int64_t base = threadIdx.x; base < nv; base += (int64_t)kQuantThreads * kQuantPassVecs) {
+        uint4 v[kQuantPassVecs];
 #pragma unroll
-        for (int j = 0; j < kQuantRegVecs; ++j) {
+        for (int j = 0; j < kQuantPassVecs; ++j) {
           const int64_t idx = base + (int64_t)j * kQuantThreads;
           v[j] = idx < nv ? __ldg(p + idx) : make_uint4(0, 0, 0, 0);
         }
 #pragma unroll
-        for (int j = 0; j < kQuantRegVecs; ++j) m = max(m, amax_bits8(v[j]));
+        for (int j = 0; j < kQuantPassVecs; ++j) m = max(m, amax_bits8(v[j]));
       }
       const float amax = bf16_bits_to_float(block_max(m, red));
       const float inv = e4m3_inv_scale(amax);
       if (threadIdx.x == 0) it.scales[row] = amax == 0.0f ? 1.0f : __fdiv_rn(amax, 448.0f);
-      for (int64_t base = threadIdx.x; base < nv; base += (int64_t)kQuantThreads * kQuantRegVecs) {
-        uint4 v[kQuantRegVecs];
+      for (int64_t base = threadIdx.x; base < nv; base += (int64_t)kQuantThreads * kQuantPassVecs) {
+        uint4 v[kQuantPassVecs];
 #pragma unroll
-        for (int j = 0; j < kQuantRegVecs; ++j) {
+        for (int j = 0; j < kQuantPassVecs; ++j) {
           const int64_t idx = base + (int64_t)j * kQuantThreads;
           v[j] = idx < nv ? __ldg(p + idx) : make_uint4(0, 0, 0, 0);
         }
 #pragma unroll
-        for (int j = 0; j < kQuantRegVecs; ++j) {
+        for (int j = 0; j < kQuantPassVecs; ++j) {
           const int64_t idx = base + (int64_t)j * kQuantThreads;
           if (idx < nv) *reinterpret_cast<uint2*>(q + idx * 8) = e4m3_codes8(v[j], inv);
         }

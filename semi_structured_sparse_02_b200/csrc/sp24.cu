@@ -986,19 +986,27 @@ int sp24_quantize_e4m3_rows(const void* src, int64_t rows, int64_t K, int64_t ld
 int sp24_quantize_e4m3_rows_grouped(const sp24_quant_item* items, int n_items, void* stream) {
   if (items == nullptr) return SP24_ERR_NULL;
   if (n_items < 1 || n_items > kMaxQuantItems) return SP24_ERR_INVALID_ARG;
-  QuantGroup g;
-  memset(&g, 0, sizeof g);
-  g.n = n_items;
-  g.row_start[0] = 0;
   for (int i = 0; i < n_items; ++i) {
     const sp24_quant_item& it = items[i];
     if (it.src_dev == nullptr || it.q_dev == nullptr || it.scales_dev == nullptr) return SP24_ERR_NULL;
     if (it.rows < 1 || it.K < 1 || it.ld < it.K) return SP24_ERR_INVALID_ARG;
     if (it.K % 16 != 0 || it.ld % 8 != 0 || !aligned16(it.src_dev) || !aligned16(it.q_dev))
       return SP24_ERR_ALIGNMENT;
-    g.item[i] = QuantItem{static_cast<const uint16_t*>(it.src_dev), it.rows, it.K, it.ld,
+  }
+  // longest rows first: their CTAs are the slowest, so they start in the
+  // first wave (the items are independent, so their order is free)
+  int order[kMaxQuantItems];
+  for (int i = 0; i < n_items; ++i) order[i] = i;
+  std::stable_sort(order, order + n_items, [&](int x, int y) { return items[x].K > items[y].K; });
+  QuantGroup g;
+  memset(&g, 0, sizeof g);
+  g.n = n_items;
+  g.row_start[0] = 0;
+  for (int j = 0; j < n_items; ++j) {
+    const sp24_quant_item& it = items[order[j]];
+    g.item[j] = QuantItem{static_cast<const uint16_t*>(it.src_dev), it.rows, it.K, it.ld,
                           static_cast<uint8_t*>(it.q_dev), it.scales_dev};
-    g.row_start[i + 1] = g.row_start[i] + it.rows;
+    g.row_start[j + 1] = g.row_start[j] + it.rows;
   }
   DeviceInfo di;
   int st = current_device_info(&di);
