@@ -446,6 +446,9 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
       const uint64_t da0 = smem_desc(s0, 16, 1024, kLayoutSw128);
       const uint64_t db0 = smem_desc(s0 + C::kABytes, 16, 1024, kLayoutSw128);
       const uint64_t dm0 = smem_desc(s0 + C::kABytes + C::kBBytes, 16, 128, kLayoutNone);
+      // both chunks of an e4m3 stage as one 128 x 256-bit copy: the second
+      // chunk is the second core matrix along the row, 2048 bytes on
+      const uint64_t dm2 = smem_desc(s0 + C::kABytes + C::kBBytes, 2048, 128, kLayoutNone);
       int stage = 0;
       uint32_t phase = 0;
       uint32_t acc_i = 0;
@@ -498,13 +501,15 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
             // descriptors of this stage: the stage-0 descriptors plus the
             // stage offset (the address field counts 16-byte units)
             const uint64_t so = (uint64_t)((uint32_t)stage * (uint32_t)(C::kStageBytes >> 4));
-            const uint64_t da = da0 + so, db = db0 + so, dm = dm0 + so;
+            const uint64_t da = da0 + so, db = db0 + so;
             auto issue = [&](auto chunks_c) {
               constexpr int kChunks = decltype(chunks_c)::value;
-#pragma unroll
-              for (int c = 0; c < kChunks; ++c) {
-                if (kPair) tc_cp_128x128b_pair(tmem_base + mcol + 4 * c, dm + (uint64_t)(c * (2048 >> 4)));
-                else tc_cp_128x128b(tmem_base + mcol + 4 * c, dm + (uint64_t)(c * (2048 >> 4)));
+              if (kChunks == 2) {
+                if (kPair) tc_cp_128x256b_pair(tmem_base + mcol, dm2 + so);
+                else tc_cp_128x256b(tmem_base + mcol, dm2 + so);
+              } else {
+                if (kPair) tc_cp_128x128b_pair(tmem_base + mcol, dm0 + so);
+                else tc_cp_128x128b(tmem_base + mcol, dm0 + so);
               }
               constexpr int kMmas = kBf16 ? 4 : 2 * kChunks;
 #pragma unroll

@@ -190,6 +190,8 @@ k_gemm_wide(const __grid_constant__ WideLaunch g) {
       const uint64_t da0 = smem_desc(s0, 16, 1024, kLayoutSw128);
       const uint64_t db0 = smem_desc(s0 + C::kABytes, 16, 1024, kLayoutSw128);
       const uint64_t dm0 = smem_desc(s0 + C::kABytes + C::kBBytes, 16, 128, kLayoutNone);
+      // e4m3: the stage's two metadata chunks as one 128 x 256-bit copy
+      const uint64_t dm2 = smem_desc(s0 + C::kABytes + C::kBBytes, 2048, 128, kLayoutNone);
       const int num_kt = g.num_kt, total_tiles = g.total_tiles;
       const uint64_t timeout_ns = g.timeout_ns;
       int stage = 0;
@@ -222,15 +224,14 @@ k_gemm_wide(const __grid_constant__ WideLaunch g) {
           // (the address field counts 16-byte units); the issuing thread is
           // on the critical path, so the loops below are fully unrolled
           const uint64_t so = (uint64_t)((uint32_t)stage * (uint32_t)(C::kStageBytes >> 4));
-          const uint64_t da = da0 + so, db = db0 + so, dm = dm0 + so;
+          const uint64_t da = da0 + so, db = db0 + so;
           const bool first = kt == 0;
           if (C::kSparse) {
             const uint32_t mcol = C::kMetaCol0 + stage * C::kMetaCols;
             auto issue = [&](auto chunks_c) {
               constexpr int kChunks = decltype(chunks_c)::value;
-#pragma unroll
-              for (int c = 0; c < kChunks; ++c)
-                tc_cp_128x128b_pair(tmem_base + mcol + 4 * c, dm + (uint64_t)(c * (2048 >> 4)));
+              if (kChunks == 2) tc_cp_128x256b_pair(tmem_base + mcol, dm2 + so);
+              else tc_cp_128x128b_pair(tmem_base + mcol, dm0 + so);
               constexpr int kMmas = kBf16 ? 4 : 2 * kChunks;
 #pragma unroll
               for (int q = 0; q < kMmas; ++q) {

@@ -219,6 +219,11 @@ __device__ __forceinline__ void mma_sp_f8(uint32_t d, uint64_t a, uint64_t b, ui
 __device__ __forceinline__ void tc_cp_128x128b(uint32_t taddr, uint64_t sdesc) {
   asm volatile("tcgen05.cp.cta_group::1.128x128b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
+// Two 128x128b metadata chunks in one copy: 128 lanes x 256 bits, the two
+// 16-byte halves of each lane's row being core matrices LBO bytes apart.
+__device__ __forceinline__ void tc_cp_128x256b(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
 
 // Tensor memory -> registers: each thread of the warp reads its own lane
 // (warp w reads lanes 32*(w%4) .. +31), 16 consecutive 32-bit columns.
@@ -340,6 +345,9 @@ __device__ __forceinline__ void tc_commit_pair(uint32_t bar, uint16_t mask) {
 }
 __device__ __forceinline__ void tc_cp_128x128b_pair(uint32_t taddr, uint64_t sdesc) {
   asm volatile("tcgen05.cp.cta_group::2.128x128b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+__device__ __forceinline__ void tc_cp_128x256b_pair(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.128x256b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 __device__ __forceinline__ void mma_bf16_pair(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
                                               uint32_t acc) {
