@@ -142,7 +142,8 @@ def prune_compress_bf16(W_bits: np.ndarray):
 
 
 def prune_compress_bf16_hybrid(W_bits: np.ndarray, mask: np.ndarray):
-    """Hybrid bf16: (values, meta_canon, dense_out) with dense tiles copied."""
+    """Hybrid bf16: (values, meta_canon, dense_out); dense_out is the hybrid
+    matrix in dense form (dense tiles unpruned, sparse tiles pruned)."""
     W = np.ascontiguousarray(W_bits, dtype=np.uint16)
     rows, K = W.shape
     values = np.empty((rows, K // 2), np.uint16)
@@ -154,7 +155,10 @@ def prune_compress_bf16_hybrid(W_bits: np.ndarray, mask: np.ndarray):
 
 
 def prune_compress_e4m3(W_bits: np.ndarray, mask: Optional[np.ndarray] = None):
-    """Return (values_q [rows,K/2], meta_canon, scales [rows] f32, dense_q [rows,K])."""
+    """Return (values_q [rows,K/2], meta_canon, scales [rows] f32, dense_q [rows,K]).
+    With a mask, dense_q is the hybrid matrix in dense form (dense tiles
+    quantized unpruned, sparse tiles their kept codes and zero bytes); without
+    one it stays zero."""
     W = np.ascontiguousarray(W_bits, dtype=np.uint16)
     rows, K = W.shape
     values = np.empty((rows, K // 2), np.uint8)

@@ -262,8 +262,11 @@ void orc_quantize_rows_e4m3(const uint16_t *src, int64_t rows, int64_t K, int64_
  * PATCH abstracts]: when tile_dense_mask is not NULL it holds one byte per
  * 128 x 128 tile (row-block major, ceil(rows/128) x K/128); a non-zero byte
  * keeps that tile dense.  A dense tile's values are quantized unpruned into
- * dense_q ([rows x K], other tiles untouched); its slots in values are 0 and
- * its canonical nibbles are 0x4 (indices 0 and 1).
+ * dense_q ([rows x K]); its slots in values are 0 and its canonical nibbles
+ * are 0x4 (indices 0 and 1).  With a mask, dense_q is the whole hybrid matrix
+ * in dense form: a sparse tile holds its kept codes at their positions and
+ * zero bytes at the dropped ones (reading R11).  Without a mask dense_q is
+ * not written.
  * values_q: [rows x K/2]; meta_canon: [rows x K/8]; scales: [rows]. */
 void orc_prune_compress_e4m3(const uint16_t *src, int64_t rows, int64_t K, int64_t ld,
                              const uint8_t *tile_dense_mask,
@@ -301,6 +304,11 @@ void orc_prune_compress_e4m3(const uint16_t *src, int64_t rows, int64_t K, int64
                     orc_e4m3_encode((double)mul_f32(bf16_to_float(v[i0]), inv));
                 values_q[r * (K / 2) + 2 * g + 1] =
                     orc_e4m3_encode((double)mul_f32(bf16_to_float(v[i1]), inv));
+                if (tile_dense_mask) {
+                    for (int i = 0; i < 4; ++i) dense_q[r * K + 4 * g + i] = 0;
+                    dense_q[r * K + 4 * g + i0] = values_q[r * (K / 2) + 2 * g + 0];
+                    dense_q[r * K + 4 * g + i1] = values_q[r * (K / 2) + 2 * g + 1];
+                }
             }
             meta_canon[r * (K / 8) + g / 2] |= (uint8_t)(nib << ((g % 2) * 4));
         }
@@ -308,7 +316,9 @@ void orc_prune_compress_e4m3(const uint16_t *src, int64_t rows, int64_t K, int64
 }
 
 /* Same hybrid treatment for bf16 output: dense tiles are copied unpruned
- * into dense_out ([rows x K]); their value slots are 0 and nibbles 0x4. */
+ * into dense_out ([rows x K]); their value slots are 0 and nibbles 0x4.
+ * Sparse tiles appear in dense_out pruned: kept values at their positions,
+ * +0 at the dropped ones (reading R11). */
 void orc_prune_compress_bf16_hybrid(const uint16_t *src, int64_t rows, int64_t K, int64_t ld,
                                     const uint8_t *tile_dense_mask,
                                     uint16_t *values, uint8_t *meta_canon, uint16_t *dense_out)
@@ -332,6 +342,9 @@ void orc_prune_compress_bf16_hybrid(const uint16_t *src, int64_t rows, int64_t K
                 nib = orc_prune_group(v, &i0, &i1);
                 values[r * (K / 2) + 2 * g + 0] = v[i0];
                 values[r * (K / 2) + 2 * g + 1] = v[i1];
+                for (int i = 0; i < 4; ++i) dense_out[r * K + 4 * g + i] = 0;
+                dense_out[r * K + 4 * g + i0] = v[i0];
+                dense_out[r * K + 4 * g + i1] = v[i1];
             }
             meta_canon[r * (K / 8) + g / 2] |= (uint8_t)(nib << ((g % 2) * 4));
         }

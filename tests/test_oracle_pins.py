@@ -313,6 +313,7 @@ def test_hybrid_dense_tiles_and_sparse_tiles():
     vq, mq, sq, dq = orc.prune_compress_e4m3(W, mask)
     vq0, mq0, sq0, _ = orc.prune_compress_e4m3(W)
     q_dense, s_dense = orc.quantize_rows_e4m3(W)
+    pruned0 = orc.decompress(vq0, mq0, rows, K)  # the all-sparse matrix in dense form
     assert np.array_equal(sq, sq0) and np.array_equal(sq, s_dense)
     for rb in range(2):
         for kt in range(4):
@@ -325,7 +326,16 @@ def test_hybrid_dense_tiles_and_sparse_tiles():
             else:
                 assert np.array_equal(vq[rs, vs], vq0[rs, vs])
                 assert np.array_equal(mq[rs, ms_], mq0[rs, ms_])
-                assert np.all(dq[rs, ks] == 0)
+                # a sparse tile appears in the dense image pruned: exactly the
+                # round trip of its compressed form, two zero bytes per group
+                assert np.array_equal(dq[rs, ks], pruned0[rs, ks])
+                assert np.all((dq[rs, ks].reshape(128, 32, 4) == 0).sum(axis=2) >= 2)
+    # bf16 output: the dense image is the original at dense tiles and the
+    # plain 2:4 prune elsewhere
+    vb, mb, db = orc.prune_compress_bf16_hybrid(W, mask)
+    pruned_b, _, _ = orc.prune_compress_bf16(W)
+    dm = np.kron(mask, np.ones((128, 128), np.uint8)).astype(bool)
+    assert np.array_equal(db, np.where(dm, W, pruned_b))
 
 
 # ---------------------------------------------------------------------------
