@@ -625,7 +625,10 @@ def _time_calls(fn, reps, warmup, flush):
     for _ in range(warmup):
         fn()
     torch.cuda.synchronize()
-    torch.cuda._sleep(1_000_000)  # the device waits ~0.5 ms while the host enqueues the reps
+    # the device waits (~0.1 ms per rep) while the host enqueues the reps, so
+    # no host launch latency lands between a call's events even when one
+    # call plus its flush takes less device time than the host takes to issue it
+    torch.cuda._sleep(200_000 * reps)
     ev = []
     for _ in range(reps):
         _flush_l2(flush)

@@ -119,8 +119,11 @@ size_t sp24_meta_bytes(int64_t rows, int64_t K);
  *               SlideSparse page).  A dense tile is written unpruned (quantized
  *               with the row scale for E4M3) into dense_tiles_dev; its value
  *               slots are written as 0 and its metadata nibbles as 0x4.
- *   dense_tiles_dev  [rows x K] of out_dtype, contiguous; only dense tiles are
- *               written.  Required when the mask is given.
+ *   dense_tiles_dev  [rows x K] of out_dtype, contiguous: the hybrid matrix in
+ *               dense form.  Dense tiles hold their values unpruned, sparse
+ *               tiles their kept values in place and zeros at the dropped
+ *               positions.  Required when the mask is given; not written
+ *               without one.
  * Requirements: rows >= 1, K % 128 == 0, ld >= K, ld % 8 == 0.
  */
 int sp24_prune_compress(const void *src_dev, int64_t rows, int64_t K, int64_t ld,
@@ -173,7 +176,12 @@ typedef struct sp24_gemm_args {
     const float *w_scales;    /* device fp32 [N]; E4M3 only (per output channel) */
     const uint8_t *tile_dense_mask; /* device; SPARSE E4M3 only: NULL or the
                                  [N/128 x K/128] hybrid tile mask                */
-    const void *W_dense_tiles;/* device [N x K] pitch K; read only at dense tiles */
+    const void *W_dense_tiles;/* device [N x K] pitch K: W in dense form as
+                                 sp24_prune_compress writes it for a hybrid
+                                 mask (sparse tiles pruned).  The one-CTA
+                                 kernel reads dense tiles from it; a CTA pair
+                                 (M, N >= 256) also reads a sparse tile from it
+                                 at K-steps where the other half is dense    */
     void *Y;                  /* device, [M x N] row pitch ldy                   */
     int64_t ldy;
     void *workspace;          /* device stream-K workspace (see below) or NULL   */

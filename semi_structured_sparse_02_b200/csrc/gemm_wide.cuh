@@ -30,6 +30,15 @@
 //
 // Work schedule: whole 256 x 256 tiles, round-robin over the pairs, A tile
 // index fastest (consecutive pairs share a B tile, all pairs share A in L2).
+//
+// Hybrid weights (E4M3, a dense/sparse flag per 128 x 128 tile of A): the
+// two CTAs of a pair hold two different 128-row blocks, and one pair MMA
+// serves both, so each 128-deep K-step runs dense when either block's tile is
+// dense there and sparse otherwise.  A dense step loads both halves from the
+// dense-form copy of A (where a sparse tile is stored pruned), a sparse step
+// the compressed values and metadata.  The producer warp reads the tile's
+// flags into shared memory when it starts a tile; the stage kind goes to the
+// MMA thread through shared memory, ordered by the stage barrier.
 #pragma once
 
 #include <type_traits>
@@ -42,6 +51,8 @@ struct WideLaunch {
   CUtensorMap tm_a;     // A: dense [rows_a x K] or values [rows_a x K/2]; 128-byte box x 128 rows, SW128
   CUtensorMap tm_b;     // B: [rows_b x K]; 128-byte box x 128 rows, SW128
   CUtensorMap tm_meta;  // metadata image viewed as [chunks * 8 rows x 256 B]; box 256 B x 8 * chunks rows
+  CUtensorMap tm_a2;    // hybrid: values [rows_a x K/2]; 64-byte box x 128 rows, SW64 (tm_a: dense form)
+  const uint8_t* tile_mask;  // hybrid: [ceil(rows_a/128) x K/128] dense flags
   int32_t rows_a, rows_b, K, num_kt;
   int32_t tiles_a, tiles_b;  // 256-row tiles
   int32_t total_tiles, meta_blocks;  // metadata row blocks (128 rows) that exist
@@ -56,23 +67,29 @@ struct WideLaunch {
 template <int kMode, bool kBf16>
 struct WideCfg {
   static constexpr bool kSparse = kMode == kModeSparse;
-  static constexpr int kKT = kSparse ? (kBf16 ? 128 : 256) : (kBf16 ? 64 : 128);  // logical K per stage
-  static constexpr int kABytes = 128 * 128;
+  static constexpr bool kHybrid = kMode == kModeHybrid;  // E4M3 only
+  static constexpr bool kUsesMeta = kSparse || kHybrid;
+  static_assert(!kHybrid || !kBf16, "hybrid tiles are E4M3");
+  // logical K per stage; a hybrid stage is one 128-deep tile column
+  static constexpr int kKT = kSparse ? (kBf16 ? 128 : 256) : (kHybrid ? 128 : (kBf16 ? 64 : 128));
+  static constexpr int kABytes = 128 * 128;  // hybrid: dense 128 x 128 B, or sparse 128 x 64 B
   static constexpr int kBBoxes = kSparse ? 2 : 1;
   static constexpr int kBBytes = 128 * 128 * kBBoxes;
-  static constexpr int kMetaChunks = kSparse ? (kBf16 ? 1 : 2) : 0;
+  static constexpr int kMetaChunks = kSparse ? (kBf16 ? 1 : 2) : (kHybrid ? 1 : 0);
   static constexpr int kMetaBytes = kMetaChunks * 2048;
   static constexpr int kStageBytes = kABytes + kBBytes + kMetaBytes;  // per CTA
   static constexpr int kStages = kSparse ? 4 : 6;
   static constexpr int kMetaCols = kMetaChunks * 4;
-  static constexpr int kOverlap = kSparse ? 32 : 0;
+  static constexpr int kOverlap = kUsesMeta ? 32 : 0;
   static constexpr int kAcc1 = 256 - kOverlap;       // first column of the second accumulator
   static constexpr int kMetaCol0 = 512 - kOverlap;   // metadata slots (sparse)
-  static_assert(!kSparse || kStages * kMetaCols <= kOverlap, "metadata slots overflow");
+  static_assert(!kUsesMeta || kStages * kMetaCols <= kOverlap, "metadata slots overflow");
   static constexpr int kBarOffset = kStages * kStageBytes;
   static constexpr int kScaleOffset = kBarOffset + 256;
   static constexpr int kEpiOffset = kScaleOffset + 256 * 4;
-  static constexpr int kSmemBytes = kEpiOffset + 4 * 2048 + 1024;  // + alignment slack
+  static constexpr int kMaxHybridKt = 2048;  // hybrid: K / 128 limit (one flag byte per K-step)
+  static constexpr int kKindOffset = kEpiOffset + 4 * 2048;
+  static constexpr int kSmemBytes = kKindOffset + (kHybrid ? kMaxHybridKt : 0) + 1024;  // + alignment slack
   static_assert(kSmemBytes <= 232448, "shared memory overflow");
 };
 
@@ -91,6 +108,10 @@ k_gemm_wide(const __grid_constant__ WideLaunch g) {
   // [2S+2..2S+4): acc_empty (used in rank 0), [2S+4]: drain
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  // hybrid: the kind of each stage in flight (1 = dense), producer -> MMA
+  volatile uint8_t* s_kind = reinterpret_cast<volatile uint8_t*>(tmem_slot + 2);
+  // hybrid: the dense flag of every K-step of the producer's current tile
+  volatile uint8_t* s_tile_kind = smem + C::kKindOffset;
   float* s_scale_b = reinterpret_cast<float*>(smem + C::kScaleOffset);
   uint8_t* s_epi = smem + C::kEpiOffset;
 
@@ -130,7 +151,73 @@ k_gemm_wide(const __grid_constant__ WideLaunch g) {
     return (int)min((int64_t)C::kMetaChunks, (int64_t)(g.K / 128) - (int64_t)kt * C::kMetaChunks);
   };
 
-  if (warp == 0) {
+  if (warp == 0 && C::kHybrid) {
+    // ------------------------------------------------------------------ hybrid producer (both CTAs)
+    // the whole warp reads a tile's dense flags; lane 0 issues the copies
+    if (g.use_pdl) pdl_wait();
+    const uint32_t full0 = mapa_shared(bar_u32(kFull), 0);
+    const int num_kt = g.num_kt, total_tiles = g.total_tiles, tiles_a = g.tiles_a, meta_blocks = g.meta_blocks;
+    const uint64_t timeout_ns = g.timeout_ns;
+    const uint8_t* const mask = g.tile_mask;
+    constexpr uint32_t kDenseTx = 2u * (128 * 128 + 128 * 128);          // A dense + B, both CTAs
+    constexpr uint32_t kSparseTx = 2u * (128 * 64 + 128 * 128 + 2048);   // A values + B + metadata
+    int armed[S];
+    for (int s = 0; s < S; ++s) armed[s] = -1;
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int tile = pair; tile < total_tiles; tile += n_pairs) {
+      const int ta = tile % tiles_a, tb = tile / tiles_a;
+      const int rb0 = ta * 2, rb1 = ta * 2 + 1;  // the pair's two 128-row blocks
+      __syncwarp();  // lane 0 has finished with the previous tile's flags
+      for (int kt = lane; kt < num_kt; kt += 32) {
+        // a row block past the end of A counts as sparse (its rows are zero)
+        const bool d = mask[(int64_t)rb0 * num_kt + kt] != 0 ||
+                       (rb1 < meta_blocks && mask[(int64_t)rb1 * num_kt + kt] != 0);
+        s_tile_kind[kt] = d ? 1 : 0;
+      }
+      __syncwarp();
+      if (lane == 0) {
+        const int ya = ta * 256 + (int)rank * 128;
+        const int yb = tb * 256 + (int)rank * 128;
+        int rb = rb0 + (int)rank;
+        if (rb >= meta_blocks) rb = 0;  // rows past the end: A is zero-filled; any valid metadata
+        for (int kt = 0; kt < num_kt; ++kt) {
+          if (!mbar_wait(bar_u32(kEmpty + stage), phase ^ 1, timeout_ns, kDevErrWaitEmpty)) {
+            ok = false;
+            *abort_flag = 1;
+            break;
+          }
+          const bool dense = s_tile_kind[kt] != 0;
+          if (rank == 0) {
+            s_kind[stage] = dense ? 1 : 0;  // published by the arrive below (release)
+            mbar_arrive_expect_tx(bar_u32(kFull + stage), dense ? kDenseTx : kSparseTx);
+            armed[stage] = (int)phase;
+          }
+          const uint32_t sa = smem_u32(smem + stage * C::kStageBytes);
+          const uint32_t fb = full0 + 8u * stage;
+          if (dense) {
+            tma_load_2d_pair(sa, &g.tm_a, fb, kt * 128, ya);
+          } else {
+            tma_load_2d_pair(sa, &g.tm_a2, fb, kt * 64, ya);
+            tma_load_2d_pair(sa + C::kABytes + C::kBBytes, &g.tm_meta, fb, 0, (rb * num_kt + kt) * 8);
+          }
+          tma_load_2d_pair(sa + C::kABytes, &g.tm_b, fb, kt * 128, yb);
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
+    }
+    // rank 0: wait (bounded) until every armed stage has landed
+    if (lane == 0)
+      for (int s = 0; s < S; ++s)
+        if (armed[s] >= 0) mbar_wait(bar_u32(kFull + s), (uint32_t)armed[s], timeout_ns, kDevErrWaitFull);
+    __syncwarp();
+  } else if (warp == 0) {
     // ------------------------------------------------------------------ producer (both CTAs)
     if (lane == 0) {
       if (g.use_pdl) pdl_wait();
@@ -186,12 +273,16 @@ k_gemm_wide(const __grid_constant__ WideLaunch g) {
     // ------------------------------------------------------------------ MMA issuer (rank 0)
     if (rank == 0 && lane == 0) {
       const uint32_t idesc = make_idesc(C::kSparse, kBf16, 256, 256);
+      const uint32_t idesc_dense = make_idesc(false, kBf16, 256, 256);  // hybrid dense K-steps
+      const uint32_t idesc_sp = make_idesc(true, kBf16, 256, 256);      // hybrid sparse K-steps
       const uint32_t s0 = smem_u32(smem);
       const uint64_t da0 = smem_desc(s0, 16, 1024, kLayoutSw128);
       const uint64_t db0 = smem_desc(s0 + C::kABytes, 16, 1024, kLayoutSw128);
       const uint64_t dm0 = smem_desc(s0 + C::kABytes + C::kBBytes, 16, 128, kLayoutNone);
       // e4m3: the stage's two metadata chunks as one 128 x 256-bit copy
       const uint64_t dm2 = smem_desc(s0 + C::kABytes + C::kBBytes, 2048, 128, kLayoutNone);
+      // hybrid sparse K-steps: A is 128 rows x 64 bytes, 64-byte swizzle
+      const uint64_t dsp0 = smem_desc(s0, 16, 512, kLayoutSw64);
       const int num_kt = g.num_kt, total_tiles = g.total_tiles;
       const uint64_t timeout_ns = g.timeout_ns;
       int stage = 0;
@@ -202,8 +293,8 @@ k_gemm_wide(const __grid_constant__ WideLaunch g) {
         const int b = j & 1;
         // the accumulator: sparse waits for tile j-1's overlap release (which
         // implies tile j-2 is drained); dense waits for tile j-2's release
-        if (C::kSparse ? j >= 1 : j >= 2) {
-          const int jr = C::kSparse ? j - 1 : j - 2;
+        if (C::kUsesMeta ? j >= 1 : j >= 2) {
+          const int jr = C::kUsesMeta ? j - 1 : j - 2;
           if (!mbar_wait(bar_u32(kAccEmpty + (jr & 1)), (uint32_t)((jr >> 1) & 1), timeout_ns,
                          kDevErrWaitAccEmpty)) {
             ok = false;
@@ -226,7 +317,21 @@ k_gemm_wide(const __grid_constant__ WideLaunch g) {
           const uint64_t so = (uint64_t)((uint32_t)stage * (uint32_t)(C::kStageBytes >> 4));
           const uint64_t da = da0 + so, db = db0 + so;
           const bool first = kt == 0;
-          if (C::kSparse) {
+          if (C::kHybrid) {
+            const uint32_t mcol = C::kMetaCol0 + stage * C::kMetaCols;
+            if (s_kind[stage] != 0) {
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                mma_f8_pair(d, da + (uint64_t)(q * (32 >> 4)), db + (uint64_t)(q * (32 >> 4)), idesc_dense,
+                            (first && q == 0) ? 0u : 1u);
+            } else {
+              tc_cp_128x128b_pair(tmem_base + mcol, dm0 + so);
+#pragma unroll
+              for (int q = 0; q < 2; ++q)
+                mma_sp_f8_pair(d, dsp0 + so + (uint64_t)(q * (32 >> 4)), db + (uint64_t)(q * (64 >> 4)),
+                               tmem_base + mcol + 2 * q, idesc_sp, (first && q == 0) ? 0u : 1u);
+            }
+          } else if (C::kSparse) {
             const uint32_t mcol = C::kMetaCol0 + stage * C::kMetaCols;
             auto issue = [&](auto chunks_c) {
               constexpr int kChunks = decltype(chunks_c)::value;
@@ -403,7 +508,7 @@ k_gemm_wide(const __grid_constant__ WideLaunch g) {
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(acc_empty0 + 8u * b);
       };
-      if (C::kSparse) {
+      if (C::kUsesMeta) {
         // the columns shared with the other accumulator first, then release
         const int ov0 = b ? 0 : 256 - C::kOverlap;
         drain(ov0, ov0 + C::kOverlap);

@@ -164,15 +164,30 @@ k_prune_compress(const uint16_t* __restrict__ src, int64_t rows, int64_t K, int6
         nib1 = prune_pick4(e4, e5, e6, e7, k10, k11);
       }
       if (live) {
+        // a hybrid matrix's dense-form array also holds its sparse tiles,
+        // pruned: kept values at their positions, zeros at the dropped ones
+        const bool dense_form = tile_mask != nullptr && !dense_tile;
+        const uint32_t i00 = nib0 & 3u, i01 = nib0 >> 2, i10 = nib1 & 3u, i11 = nib1 >> 2;
         if (kOutE4M3) {
           uint32_t q = 0;
           if (!dense_tile)
             q = e4m3x2_of(__fmul_rn(bf16_bits_to_float(k00), inv), __fmul_rn(bf16_bits_to_float(k01), inv)) |
                 (e4m3x2_of(__fmul_rn(bf16_bits_to_float(k10), inv), __fmul_rn(bf16_bits_to_float(k11), inv)) << 16);
           *reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(values) + row * half_k + kc * 64 + seg * 4) = q;
+          if (dense_form) {
+            const uint32_t d0 = ((q & 0xFFu) << (8 * i00)) | (((q >> 8) & 0xFFu) << (8 * i01));
+            const uint32_t d1 = (((q >> 16) & 0xFFu) << (8 * i10)) | ((q >> 24) << (8 * i11));
+            *reinterpret_cast<uint2*>(static_cast<uint8_t*>(dense_out) + row * K + k0) = make_uint2(d0, d1);
+          }
         } else {
           *reinterpret_cast<uint2*>(static_cast<uint16_t*>(values) + row * half_k + kc * 64 + seg * 4) =
               make_uint2(k00 | (k01 << 16), k10 | (k11 << 16));
+          if (dense_form) {
+            const uint64_t d0 = ((uint64_t)k00 << (16 * i00)) | ((uint64_t)k01 << (16 * i01));
+            const uint64_t d1 = ((uint64_t)k10 << (16 * i10)) | ((uint64_t)k11 << (16 * i11));
+            *reinterpret_cast<uint4*>(static_cast<uint16_t*>(dense_out) + row * K + k0) =
+                make_uint4((uint32_t)d0, (uint32_t)(d0 >> 32), (uint32_t)d1, (uint32_t)(d1 >> 32));
+          }
         }
       }
       canon[rl][seg] = (uint8_t)(nib0 | (nib1 << 4));

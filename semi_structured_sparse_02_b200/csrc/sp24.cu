@@ -595,10 +595,17 @@ LaunchCache<GroupLaunch, 16> g_cache_group;
 // The CTA-pair kernel (256 x 256 tiles) for large token counts
 // ---------------------------------------------------------------------------
 // A GEMM takes the pair kernel when both output dimensions span at least one
-// 256-row tile and no hybrid mask is given, unless SP24_GEMM_SINGLE_CTA asks
-// for the one-CTA kernel.
-bool use_pair(int64_t rows_a, int64_t rows_b, bool hybrid, uint32_t flags) {
-  return !hybrid && rows_a >= 256 && rows_b >= 256 && (flags & SP24_GEMM_SINGLE_CTA) == 0;
+// 256-row tile, unless SP24_GEMM_SINGLE_CTA asks for the one-CTA kernel.
+// Hybrid weights take it from 512 tokens on (and while K / 128 fits the
+// kernel's per-tile flag buffer): at 256 tokens the one-CTA kernel, whose
+// K-steps need not agree across two row blocks, measured ~10% faster.
+bool use_pair(int64_t rows_a, int64_t rows_b, int64_t K, bool hybrid, uint32_t flags) {
+  if (rows_a < 256 || rows_b < 256 || (flags & SP24_GEMM_SINGLE_CTA) != 0) return false;
+  if (!hybrid) return true;
+  return rows_b >= 512 && K / 128 <= WideCfg<kModeHybrid, false>::kMaxHybridKt;
+}
+bool args_use_pair(const sp24_gemm_args* a) {
+  return use_pair(a->N, a->M, a->K, a->tile_dense_mask != nullptr, a->flags);
 }
 
 // Launches one instantiation on min(tiles, co-resident pairs) pairs; the
@@ -644,26 +651,38 @@ int launch_wide_inst(const WideLaunch& wl, cudaStream_t stream) {
   return launch_result(cudaLaunchKernelEx(&cfg, k_gemm_wide<kMode, kBf16, kAIsW>, wl));
 }
 
-// Fills and launches the pair kernel.  A = rows_a x K (values when sparse,
-// with its metadata image), B = rows_b x K dense.
+// Fills and launches the pair kernel.  A = rows_a x K (values when sparse or
+// hybrid, with its metadata image; hybrid adds A's dense form, pitch K, and
+// the tile mask), B = rows_b x K dense.
 int run_wide(int mode, bool bf16, bool a_is_w, const void* A, int64_t lda, const void* A_meta,
-             const void* B, int64_t ldb, int64_t rows_a, int64_t rows_b, int64_t K, const float* scale_a,
-             const float* scale_b, void* Y, int64_t ldy, bool out_f32, cudaStream_t stream) {
+             const void* A_dense, const uint8_t* A_mask, const void* B, int64_t ldb, int64_t rows_a,
+             int64_t rows_b, int64_t K, const float* scale_a, const float* scale_b, void* Y, int64_t ldy,
+             bool out_f32, cudaStream_t stream) {
   DeviceInfo di;
   int st = current_device_info(&di);
   if (st != SP24_OK) return st;
   const int eb = bf16 ? 2 : 1;
   const int box_elems = 128 / eb;
   const bool sparse = mode == kModeSparse;
-  const int kt = sparse ? (bf16 ? 128 : 256) : (bf16 ? 64 : 128);
+  const bool hybrid = mode == kModeHybrid;
+  if (hybrid && (bf16 || !a_is_w)) return SP24_ERR_DTYPE;
+  const int kt = sparse ? (bf16 ? 128 : 256) : (hybrid ? 128 : (bf16 ? 64 : 128));
   static thread_local WideLaunch wl;
   memset(&wl, 0, sizeof wl);
-  bool ok = make_map(&wl.tm_a, A, eb, sparse ? K / 2 : K, rows_a, lda * eb, box_elems, 128,
-                     CU_TENSOR_MAP_SWIZZLE_128B);
+  bool ok = true;
+  if (hybrid) {
+    // dense K-steps read A's dense form, sparse ones the compressed values
+    ok &= make_map(&wl.tm_a, A_dense, 1, K, rows_a, K, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok &= make_map(&wl.tm_a2, A, 1, K / 2, rows_a, lda, 64, 128, CU_TENSOR_MAP_SWIZZLE_64B);
+  } else {
+    ok &= make_map(&wl.tm_a, A, eb, sparse ? K / 2 : K, rows_a, lda * eb, box_elems, 128,
+                   CU_TENSOR_MAP_SWIZZLE_128B);
+    wl.tm_a2 = wl.tm_a;
+  }
   ok &= make_map(&wl.tm_b, B, eb, K, rows_b, ldb * eb, box_elems, 128, CU_TENSOR_MAP_SWIZZLE_128B);
   const int meta_blocks = (int)((rows_a + 127) / 128);
-  if (sparse) {
-    const int chunks = bf16 ? 1 : 2;
+  if (sparse || hybrid) {
+    const int chunks = (bf16 || hybrid) ? 1 : 2;
     const uint64_t meta_rows = (uint64_t)meta_blocks * (uint64_t)(K / 128) * 8;  // 256-byte rows
     ok &= make_map(&wl.tm_meta, A_meta, 1, 256, meta_rows, 256, 256, 8 * chunks, CU_TENSOR_MAP_SWIZZLE_NONE);
   } else {
@@ -685,6 +704,8 @@ int run_wide(int mode, bool bf16, bool a_is_w, const void* A, int64_t lda, const
   wl.Y = Y;
   wl.ldy = ldy;
   wl.timeout_ns = g_timeout_ns.load();
+  wl.tile_mask = A_mask;
+  if (hybrid) return launch_wide_inst<kModeHybrid, false, true>(wl, stream);
   if (!a_is_w) {
     if (sparse)
       return bf16 ? launch_wide_inst<kModeSparse, true, false>(wl, stream)
@@ -699,11 +720,11 @@ int run_wide(int mode, bool bf16, bool a_is_w, const void* A, int64_t lda, const
 }
 
 int run_gemm(const sp24_gemm_args* a, cudaStream_t stream) {
-  if (use_pair(a->N, a->M, a->tile_dense_mask != nullptr, a->flags)) {
+  if (args_use_pair(a)) {
     const bool e4 = a->in_dtype == SP24_E4M3;
-    return run_wide(a->tactic == SP24_TACTIC_DENSE ? kModeDense : kModeSparse, !e4, true, a->W, a->ldw,
-                    a->W_meta, a->X, a->ldx, a->N, a->M, a->K, e4 ? a->w_scales : nullptr,
-                    e4 ? a->x_scales : nullptr, a->Y, a->ldy, a->out_dtype == SP24_F32, stream);
+    return run_wide(args_mode(a), !e4, true, a->W, a->ldw, a->W_meta, a->W_dense_tiles, a->tile_dense_mask,
+                    a->X, a->ldx, a->N, a->M, a->K, e4 ? a->w_scales : nullptr, e4 ? a->x_scales : nullptr,
+                    a->Y, a->ldy, a->out_dtype == SP24_F32, stream);
   }
   DeviceInfo di;
   int st = current_device_info(&di);
@@ -725,8 +746,9 @@ int run_gemm(const sp24_gemm_args* a, cudaStream_t stream) {
 int run_activation_gemm(bool bf16, const void* x_values, const void* x_meta, const float* x_scales,
                         const void* W, int64_t ldw, const float* w_scales, int64_t M, int64_t N, int64_t K,
                         void* Y, int64_t ldy, bool out_f32, const DeviceInfo& di, cudaStream_t s) {
-  if (use_pair(M, N, false, 0))
-    return run_wide(kModeSparse, bf16, false, x_values, K / 2, x_meta, W, ldw, M, N, K, x_scales, w_scales, Y,
+  if (use_pair(M, N, K, false, 0))
+    return run_wide(kModeSparse, bf16, false, x_values, K / 2, x_meta, nullptr, nullptr, W, ldw, M, N, K,
+                    x_scales, w_scales, Y,
                     ldy, out_f32, s);
   const int eb = bf16 ? 2 : 1;
   const int box_elems = 128 / eb;
@@ -1020,7 +1042,7 @@ size_t sp24_gemm_workspace_bytes(const sp24_gemm_args* a) {
   if (validate_gemm(a) != SP24_OK) return 0;
   DeviceInfo di;
   if (current_device_info(&di) != SP24_OK) return 0;
-  if (use_pair(a->N, a->M, a->tile_dense_mask != nullptr, a->flags)) return 0;
+  if (args_use_pair(a)) return 0;
   Plan pl = plan_gemm(a, di, (size_t)-1);
   return pl.ws_bytes;
 }
@@ -1029,7 +1051,7 @@ size_t sp24_gemm_workspace_state_bytes(const sp24_gemm_args* a) {
   if (validate_gemm(a) != SP24_OK) return 0;
   DeviceInfo di;
   if (current_device_info(&di) != SP24_OK) return 0;
-  if (use_pair(a->N, a->M, a->tile_dense_mask != nullptr, a->flags)) return 0;
+  if (args_use_pair(a)) return 0;
   const Plan pl = plan_gemm(a, di, (size_t)-1);
   return pl.sched == kSchedStreamK ? sk_state_bytes(pl) : 0;
 }

@@ -372,6 +372,70 @@ def test_hybrid_gemm_parity(M):
     check_tolerance(y, y_ref, a_ref, "hybrid")
 
 
+def _pair_mask(kind, N, K, seed):
+    RB, KT = N // 128, K // 128
+    if kind == "random":
+        return inputs.hybrid_mask(N, K, seed=seed)
+    if kind == "all_dense":
+        return np.ones((RB, KT), np.uint8)
+    if kind == "all_sparse":
+        return np.zeros((RB, KT), np.uint8)
+    if kind == "odd_blocks":   # every pair mixed: the second half dense, the first sparse
+        m = np.zeros((RB, KT), np.uint8)
+        m[1::2, :] = 1
+        return m
+    if kind == "checker":      # mixed, dense-first and dense-second K-steps interleaved
+        return ((np.arange(RB)[:, None] + np.arange(KT)[None, :]) % 2).astype(np.uint8)
+    raise ValueError(kind)
+
+
+HYBRID_PAIR_SHAPES = [
+    (512, 512, 1024),
+    (600, 384, 640),    # ragged token tile; the last weight tile's second half is past the end
+    (520, 768, 2048),
+]
+
+
+@pytest.mark.parametrize("M,N,K", HYBRID_PAIR_SHAPES)
+@pytest.mark.parametrize("kind", ["random", "all_dense", "all_sparse", "odd_blocks", "checker"])
+def test_hybrid_gemm_pair_parity(M, N, K, kind):
+    """M >= 512, N >= 256: hybrid weights on CTA pairs, where a K-step runs dense when
+    either half of the pair is dense there.  Checked against the oracle and
+    against the one-CTA kernel."""
+    X, W = inputs.linear_pair(M, N, K, seed=M + N + K + 7, outliers=True)
+    mask = _pair_mask(kind, N, K, seed=M + K)
+    y, y_ref, a_ref, _, _ = run_gemm(X, W, True, sp24.SPARSE, True, mask=mask)
+    check_tolerance(y, y_ref, a_ref, "hybrid pair %s M%d N%d K%d" % (kind, M, N, K))
+    y1, _, _, _, _ = run_gemm(X, W, True, sp24.SPARSE, True, mask=mask, flags=sp24.GEMM_SINGLE_CTA)
+    scale = np.abs(y_ref).max()
+    assert np.allclose(y, y1, rtol=1e-5, atol=1e-5 * scale)
+
+
+def test_hybrid_pair_gemm_on_gpu_pruned_weights():
+    """The device prune writes the dense-form array the pair kernel reads at
+    mixed K-steps; the whole chain against the oracle."""
+    M, N, K = 512, 640, 1536
+    X, W = inputs.linear_pair(M, N, K, seed=17, outliers=True)
+    mask = inputs.hybrid_mask(N, K, seed=17)
+    ref = OracleSparseW(W, e4m3=True, mask=mask)
+    vals = torch.empty(N, K // 2, dtype=torch.uint8, device="cuda")
+    meta = torch.empty(sp24.meta_bytes(N, K), dtype=torch.uint8, device="cuda")
+    dense = torch.empty(N, K, dtype=torch.uint8, device="cuda")
+    sc = torch.empty(N, dtype=torch.float32, device="cuda")
+    sp24.prune_compress(dev_bf16(W), sp24.E4M3, vals, meta, row_scales=sc, tile_mask=dev(mask), dense_tiles=dense)
+    torch.cuda.synchronize()
+    assert np.array_equal(u8(dense), ref.dense)
+    xq, xs, X_hat = oracle_x(X, True)
+    Y = torch.empty(M, N, dtype=torch.float32, device="cuda")
+    a = sp24.gemm_args(dev(xq), vals, Y, K, sp24.SPARSE, W_meta=meta, x_scales=dev(xs), w_scales=sc,
+                       tile_mask=dev(mask), W_dense_tiles=dense)
+    sp24.gemm(a)
+    torch.cuda.synchronize()
+    assert sp24.last_device_error() == sp24.SP24_OK
+    y_ref, a_ref = orc.gemm_f64(X_hat, ref.W_hat)
+    check_tolerance(Y.cpu().numpy().astype(np.float64), y_ref, a_ref, "hybrid pair, device-pruned W")
+
+
 def test_gemm_with_gpu_pruned_weights_end_to_end():
     M, N, K = 32, 640, 2048
     X, W = inputs.linear_pair(M, N, K, seed=9, outliers=True)
