@@ -195,9 +195,13 @@ typedef struct sp24_gemm_args {
  * launch).  X, x_scales and Y are always ordered after it. */
 #define SP24_GEMM_W_STATIC 1u
 
-/* Shapes with M >= 256 tokens and N >= 256 output features (no hybrid mask)
- * run on CTA pairs: one tcgen05 MMA over two SMs computes a 256 x 256 output
- * tile, each SM loading half of both operands (no workspace).  This flag
+/* Shapes with M >= 256 tokens and N >= 256 output features run on CTA
+ * pairs: one tcgen05 MMA over two SMs computes a 256 x 256 output tile, each
+ * SM loading half of both operands (no workspace).  With a hybrid mask they
+ * do so only when the 256 x 256 tiles are at least as many as the pairs that
+ * fit on the device at once (a pair's K-step runs dense when either of its
+ * two row blocks is dense there, which costs more than the one-CTA kernel's
+ * per-tile choice unless the one-CTA kernel is short of tiles).  This flag
  * keeps such a call on the one-CTA kernel (128-row tiles); results agree to
  * the tolerance of the method, not bit for bit. */
 #define SP24_GEMM_SINGLE_CTA 2u
@@ -205,7 +209,8 @@ typedef struct sp24_gemm_args {
 /* For M <= 255 (and N >= 256, no hybrid mask): run 256-row weight tiles on
  * CTA pairs (M = 256 pair MMA, each SM loading half of the tile) instead of
  * 128-row tiles on single CTAs.  In a grouped call it applies when every
- * problem sets it.  Same results to the method's tolerance. */
+ * problem sets it.  With a hybrid mask and M, N >= 256: take the CTA-pair
+ * kernel whatever the tile count.  Same results to the method's tolerance. */
 #define SP24_GEMM_CTA_PAIR 4u
 
 /* Bytes of workspace the call would use for its stream-K schedule (0 if the

@@ -418,6 +418,69 @@ k_quantize_rows_e4m3(const __grid_constant__ QuantGroup g) {
 }
 
 // ---------------------------------------------------------------------------
+// Per-row E4M3 quantization, one HBM read per element: rows are cut into
+// warp segments of up to kQWarpVecs 16-byte vectors per lane, held in
+// registers from the load to the store.  A row takes w = ceil(K/8 / (32 *
+// kQWarpVecs)) warps; a CTA of kQWarps warps takes floor(kQWarps / w) rows of
+// one matrix, so a 25600-wide row fills one CTA and 5120-wide rows go five to
+// a CTA.  The row amax is combined across its warps in shared memory.  Same
+// arithmetic as k_quantize_rows_e4m3 (bit-identical codes and scales).
+// ---------------------------------------------------------------------------
+constexpr int kQWarps = 16;
+constexpr int kQWarpVecs = 7;
+constexpr int kQSegVecs = 32 * kQWarpVecs;      // vectors of one warp segment
+constexpr int kQMaxVecs = kQWarps * kQSegVecs;  // longest row (vectors) this kernel takes
+
+struct QuantSegGroup {
+  QuantItem item[kMaxQuantItems];
+  int32_t cta_start[kMaxQuantItems + 1];  // prefix sums of CTAs per item
+  int32_t warps_per_row[kMaxQuantItems];
+  int32_t rows_per_cta[kMaxQuantItems];
+  int n;
+};
+
+__global__ void __launch_bounds__(kQWarps * 32, 2)
+k_quantize_rows_e4m3_seg(const __grid_constant__ QuantSegGroup g) {
+  __shared__ uint32_t s_amax[kQWarps];
+  pdl_launch_dependents();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x < kQWarps) s_amax[threadIdx.x] = 0u;
+  int i = 0;
+  while ((int)blockIdx.x >= g.cta_start[i + 1]) ++i;
+  const QuantItem& it = g.item[i];
+  const int w = g.warps_per_row[i], r = g.rows_per_cta[i];
+  const int slot = warp / w, seg = warp - slot * w;
+  const int64_t row = (int64_t)((int)blockIdx.x - g.cta_start[i]) * r + slot;
+  const bool active = slot < r && row < it.rows;
+  const int64_t nv = it.K / 8;
+  pdl_wait();  // the activations may be written by the upstream grid
+  uint4 reg[kQWarpVecs];
+  uint32_t m = 0;
+  const uint4* p = reinterpret_cast<const uint4*>(it.src + (active ? row : 0) * it.ld);
+#pragma unroll
+  for (int j = 0; j < kQWarpVecs; ++j) {
+    const int64_t idx = (int64_t)seg * kQSegVecs + j * 32 + lane;
+    reg[j] = (active && idx < nv) ? __ldg(p + idx) : make_uint4(0, 0, 0, 0);
+    m = max(m, amax_bits8(reg[j]));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  __syncthreads();  // s_amax initialized
+  if (active && lane == 0) atomicMax(&s_amax[slot], m);
+  __syncthreads();
+  if (!active) return;
+  const float amax = bf16_bits_to_float(s_amax[slot]);
+  const float inv = e4m3_inv_scale(amax);
+  if (seg == 0 && lane == 0) it.scales[row] = amax == 0.0f ? 1.0f : __fdiv_rn(amax, 448.0f);
+  uint8_t* q = it.q + row * it.K;
+#pragma unroll
+  for (int j = 0; j < kQWarpVecs; ++j) {
+    const int64_t idx = (int64_t)seg * kQSegVecs + j * 32 + lane;
+    if (idx < nv) *reinterpret_cast<uint2*>(q + idx * 8) = e4m3_codes8(reg[j], inv);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Decompress: scatter values back using the metadata image.
 // ---------------------------------------------------------------------------
 // Nibble of (row-in-block r, group g in chunk) inside one image chunk.

@@ -596,13 +596,21 @@ LaunchCache<GroupLaunch, 16> g_cache_group;
 // ---------------------------------------------------------------------------
 // A GEMM takes the pair kernel when both output dimensions span at least one
 // 256-row tile, unless SP24_GEMM_SINGLE_CTA asks for the one-CTA kernel.
-// Hybrid weights take it from 512 tokens on (and while K / 128 fits the
-// kernel's per-tile flag buffer): at 256 tokens the one-CTA kernel, whose
-// K-steps need not agree across two row blocks, measured ~10% faster.
+// Hybrid weights (while K / 128 fits the kernel's per-tile flag buffer) take
+// it when its 256 x 256 tiles fill the co-resident pairs, or when
+// SP24_GEMM_CTA_PAIR asks: a pair's K-step runs dense when either of its two
+// row blocks is dense there, so with fewer tiles the one-CTA kernel (per-tile
+// choice, stream-K over every SM) measured faster (e.g. 6144 x 4096 at 256
+// tokens: 22.6 against 24.5 us; 24576 x 4096 at 256 tokens: 49 against 41).
 bool use_pair(int64_t rows_a, int64_t rows_b, int64_t K, bool hybrid, uint32_t flags) {
   if (rows_a < 256 || rows_b < 256 || (flags & SP24_GEMM_SINGLE_CTA) != 0) return false;
   if (!hybrid) return true;
-  return rows_b >= 512 && K / 128 <= WideCfg<kModeHybrid, false>::kMaxHybridKt;
+  if (K / 128 > WideCfg<kModeHybrid, false>::kMaxHybridKt) return false;
+  if ((flags & SP24_GEMM_CTA_PAIR) != 0) return true;
+  DeviceInfo di;
+  if (current_device_info(&di) != SP24_OK) return false;
+  const int64_t tiles = ((rows_a + 255) / 256) * ((rows_b + 255) / 256);
+  return tiles >= (int64_t)di.pairs;
 }
 bool args_use_pair(const sp24_gemm_args* a) {
   return use_pair(a->N, a->M, a->K, a->tile_dense_mask != nullptr, a->flags);
@@ -1020,6 +1028,32 @@ int sp24_quantize_e4m3_rows_grouped(const sp24_quant_item* items, int n_items, v
   int order[kMaxQuantItems];
   for (int i = 0; i < n_items; ++i) order[i] = i;
   std::stable_sort(order, order + n_items, [&](int x, int y) { return items[x].K > items[y].K; });
+  DeviceInfo di;
+  int st = current_device_info(&di);
+  if (st != SP24_OK) return st;
+  bool seg_ok = true;
+  for (int i = 0; i < n_items; ++i) seg_ok &= items[i].K / 8 <= kQMaxVecs;
+  if (seg_ok) {
+    // every row fits in registers: warp segments, one read per element
+    QuantSegGroup sg;
+    memset(&sg, 0, sizeof sg);
+    sg.n = n_items;
+    int64_t ctas = 0;
+    for (int j = 0; j < n_items; ++j) {
+      const sp24_quant_item& it = items[order[j]];
+      sg.item[j] = QuantItem{static_cast<const uint16_t*>(it.src_dev), it.rows, it.K, it.ld,
+                             static_cast<uint8_t*>(it.q_dev), it.scales_dev};
+      const int w = (int)((it.K / 8 + kQSegVecs - 1) / kQSegVecs);
+      sg.warps_per_row[j] = w;
+      sg.rows_per_cta[j] = kQWarps / w;
+      sg.cta_start[j] = (int32_t)ctas;
+      ctas += (it.rows + sg.rows_per_cta[j] - 1) / sg.rows_per_cta[j];
+      if (ctas > INT32_MAX / 2) return SP24_ERR_INVALID_ARG;
+    }
+    sg.cta_start[n_items] = (int32_t)ctas;
+    return launch_pdl(k_quantize_rows_e4m3_seg, dim3((unsigned)ctas), dim3(kQWarps * 32), 0,
+                      static_cast<cudaStream_t>(stream), sg);
+  }
   QuantGroup g;
   memset(&g, 0, sizeof g);
   g.n = n_items;
@@ -1030,9 +1064,6 @@ int sp24_quantize_e4m3_rows_grouped(const sp24_quant_item* items, int n_items, v
                           static_cast<uint8_t*>(it.q_dev), it.scales_dev};
     g.row_start[j + 1] = g.row_start[j] + it.rows;
   }
-  DeviceInfo di;
-  int st = current_device_info(&di);
-  if (st != SP24_OK) return st;
   const int grid = (int)std::min<int64_t>(g.row_start[n_items], (int64_t)di.sms * kQuantCtasPerSm);
   return launch_pdl(k_quantize_rows_e4m3, dim3(grid), dim3(kQuantThreads), 0,
                     static_cast<cudaStream_t>(stream), g);

@@ -101,7 +101,11 @@ def test_prune_hybrid_tiles_bit_exact(e4):
         assert np.array_equal(bits16(dense), ref.dense)
 
 
-@pytest.mark.parametrize("rows,K", [(1, 5120), (16, 256), (128, 4096), (7, 25600)])
+# register-resident warp segments up to 28672 wide (one warp per 1792 elements:
+# 37 x 1792 packs 16 rows per CTA with a ragged last CTA, 28672 fills 16 warps);
+# the two-pass kernel beyond (30720)
+@pytest.mark.parametrize("rows,K", [(1, 5120), (16, 256), (128, 4096), (7, 25600), (37, 1792), (2, 28672),
+                                    (3, 30720)])
 def test_quantize_rows_e4m3_bit_exact(rows, K):
     X = inputs.normal_bf16((rows, K), 1.0, seed=rows * 3 + K)
     X[0, :] = 0  # an all-zero token: scale 1, codes 0
@@ -114,8 +118,11 @@ def test_quantize_rows_e4m3_bit_exact(rows, K):
     assert np.array_equal(s.cpu().numpy(), s_ref)
 
 
-def test_grouped_quantize_matches_oracle_per_matrix():
-    shapes = [(1, 5120), (8, 25600), (32, 256), (128, 4096), (3, 33024)]  # last: two-pass path
+@pytest.mark.parametrize("shapes", [
+    [(1, 5120), (8, 25600), (32, 256), (128, 4096), (5, 28672)],   # warp-segment kernel
+    [(1, 5120), (8, 25600), (32, 256), (128, 4096), (3, 33024)],   # a row too long for it: two-pass kernel
+])
+def test_grouped_quantize_matches_oracle_per_matrix(shapes):
     pairs, refs = [], []
     for i, (rows, K) in enumerate(shapes):
         X = inputs.normal_bf16((rows, K), 1.0, seed=50 + i)
@@ -390,8 +397,8 @@ def _pair_mask(kind, N, K, seed):
 
 
 HYBRID_PAIR_SHAPES = [
-    (512, 512, 1024),
-    (600, 384, 640),    # ragged token tile; the last weight tile's second half is past the end
+    (256, 512, 1024),
+    (300, 384, 640),    # ragged token tile; the last weight tile's second half is past the end
     (520, 768, 2048),
 ]
 
@@ -399,12 +406,13 @@ HYBRID_PAIR_SHAPES = [
 @pytest.mark.parametrize("M,N,K", HYBRID_PAIR_SHAPES)
 @pytest.mark.parametrize("kind", ["random", "all_dense", "all_sparse", "odd_blocks", "checker"])
 def test_hybrid_gemm_pair_parity(M, N, K, kind):
-    """M >= 512, N >= 256: hybrid weights on CTA pairs, where a K-step runs dense when
-    either half of the pair is dense there.  Checked against the oracle and
-    against the one-CTA kernel."""
+    """Hybrid weights on CTA pairs (forced: these shapes have fewer tiles than
+    the device has pairs), where a K-step runs dense when either half of the
+    pair is dense there.  Checked against the oracle and against the one-CTA
+    kernel."""
     X, W = inputs.linear_pair(M, N, K, seed=M + N + K + 7, outliers=True)
     mask = _pair_mask(kind, N, K, seed=M + K)
-    y, y_ref, a_ref, _, _ = run_gemm(X, W, True, sp24.SPARSE, True, mask=mask)
+    y, y_ref, a_ref, _, _ = run_gemm(X, W, True, sp24.SPARSE, True, mask=mask, flags=sp24.GEMM_CTA_PAIR)
     check_tolerance(y, y_ref, a_ref, "hybrid pair %s M%d N%d K%d" % (kind, M, N, K))
     y1, _, _, _, _ = run_gemm(X, W, True, sp24.SPARSE, True, mask=mask, flags=sp24.GEMM_SINGLE_CTA)
     scale = np.abs(y_ref).max()
@@ -429,6 +437,7 @@ def test_hybrid_pair_gemm_on_gpu_pruned_weights():
     Y = torch.empty(M, N, dtype=torch.float32, device="cuda")
     a = sp24.gemm_args(dev(xq), vals, Y, K, sp24.SPARSE, W_meta=meta, x_scales=dev(xs), w_scales=sc,
                        tile_mask=dev(mask), W_dense_tiles=dense)
+    a.flags = sp24.GEMM_CTA_PAIR
     sp24.gemm(a)
     torch.cuda.synchronize()
     assert sp24.last_device_error() == sp24.SP24_OK
