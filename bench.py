@@ -228,13 +228,17 @@ def run_product(args, rank, world, local_rank):
     quant_all = sp24.QuantGroup([(it["X"], it["xq"], it["xs"]) for it in inst])
 
     def make_groups(pick):
-        """Grouped launches for the tactic pick(it) of every GEMM."""
+        """Grouped launches for the tactic pick(it) of every GEMM.  The GEMMs
+        are independent and all their inputs come from the cast before the
+        first group, so every group after the first is marked as following
+        an independent GEMM launch: its CTAs start as SMs free up instead of
+        waiting for the previous group to finish."""
         by = {}
         for it in inst:
             t = pick(it)
             a = it["a_sp"] if t == "sparse" else it["a_dn"]
             by.setdefault((t, sp24.m_class(it["M"])), []).append(a)
-        return [sp24.GemmGroup(v) for _, v in sorted(by.items())]
+        return [sp24.GemmGroup(v, after_independent=i > 0) for i, (_, v) in enumerate(sorted(by.items()))]
 
     groups = {"sparse": make_groups(lambda it: "sparse"), "dense": make_groups(lambda it: "dense")}
 

@@ -213,6 +213,19 @@ typedef struct sp24_gemm_args {
  * kernel whatever the tile count.  Same results to the method's tolerance. */
 #define SP24_GEMM_CTA_PAIR 4u
 
+/* The kernel that precedes this call in the stream is an sp24 GEMM call that
+ * is independent of it: neither call writes anything the other reads or
+ * writes (inputs, outputs, workspace), and every input of this call was
+ * complete when that preceding call began (it waited for its own upstream
+ * kernel).  The call then starts its work as soon as SMs free up, without
+ * waiting for the preceding GEMM to finish, and waits for it only before
+ * exiting, so that its own completion still implies the preceding call's.
+ * Ignored by the CTA-pair (256 x 256 tile) kernel, which always waits.  In a
+ * grouped call it applies when every problem sets it.  Meant for chains of
+ * independent GEMMs after one producer, such as a layer's projections after
+ * one activation cast. */
+#define SP24_GEMM_AFTER_INDEPENDENT 8u
+
 /* Bytes of workspace the call would use for its stream-K schedule (0 if the
  * shape needs none).  Shapes with few output tiles per SM may split the
  * tiles' K range evenly over all SMs (a cost model decides); a split tile is

@@ -78,6 +78,7 @@ struct GemmParams {
   int32_t out_f32;            // 1: fp32 output, 0: bf16
   int32_t use_pdl;            // wait on the upstream grid before dependent loads
   int32_t w_static;           // A operands are not written by the upstream grid
+  int32_t after_independent;  // the upstream grid is an independent GEMM: wait for it only at the end
   uint64_t timeout_ns;
   float* sk_slots;            // stream-K partial tiles [units][pair half][2][128 rows][BN] fp32
   unsigned int* sk_flags;     // "partial stored" flags [units][pair half][2]
@@ -228,9 +229,15 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
   static_assert(!kPair || kAIsW, "pairs split the weight rows");
   const GemmParams& p = g.p;
 
-  // the next kernel in the stream may launch now; it waits for our completion
-  // (griddepcontrol.wait) before it reads anything we write
-  pdl_launch_dependents();
+  // Programmatic dependent launch.  A launch that depends on its upstream
+  // grid lets the next kernel launch only after every thread has seen the
+  // upstream complete (wait, then trigger), so a next kernel that is
+  // independent of this one may skip its own wait and still find this
+  // launch's inputs complete.  A launch after an independent GEMM triggers at
+  // once and waits only before exiting (its completion then implies the
+  // upstream's).
+  const bool wait_first = p.use_pdl && !p.after_independent;
+  if (!wait_first) pdl_launch_dependents();
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte alignment for the swizzled tiles
@@ -296,6 +303,10 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
 
   if (warp == 0) {
     // ------------------------------------------------------------------ producer
+    if (lane != 0 && wait_first) {
+      pdl_wait();
+      pdl_launch_dependents();
+    }
     if (lane == 0) {
       const uint64_t pol_stream = policy_evict_first();  // A: read once
       const uint64_t pol_keep = policy_evict_last();     // B: re-read by many CTAs
@@ -392,7 +403,10 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
           }
         }
       }
-      if (p.use_pdl) pdl_wait();
+      if (wait_first) {
+        pdl_wait();
+        pdl_launch_dependents();
+      }
 
       // 2. the main stream
       int stage = 0;
@@ -437,6 +451,10 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer (rank 0 in a pair)
+    if (wait_first) {  // nothing to issue before the producer's dependent loads anyway
+      pdl_wait();
+      pdl_launch_dependents();
+    }
     if (lane == 0 && rank == 0) {
       const uint32_t idesc = make_idesc(C::kSparse, kBf16, C::kRowsA, kBN);
       const uint32_t idesc_dense = make_idesc(false, kBf16, kBlockA, kBN);
@@ -573,7 +591,10 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
     __syncwarp();
   } else {
     // ------------------------------------------------------------------ epilogue
-    if (p.use_pdl) pdl_wait();                 // B scales and Y may belong to the upstream grid
+    if (wait_first) {                          // B scales and Y may belong to the upstream grid
+      pdl_wait();
+      pdl_launch_dependents();
+    }
     const int lg = warp & 3;                   // tensor-memory lane group of this warp
     const int row = lg * 32 + lane;            // accumulator row (lane) within the CTA's half
     const int et = threadIdx.x - 64;           // 0..127
@@ -850,6 +871,9 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
 
   tc_fence_before_sync();
   __syncthreads();
+  // after an independent GEMM: complete only once it has (stream order of
+  // completion for whatever follows)
+  if (p.use_pdl && p.after_independent) pdl_wait();
   if (kPair) cluster_sync();  // neither CTA leaves while its peer may still use its memory
   if (warp == 1) {
     tc_fence_after_sync();

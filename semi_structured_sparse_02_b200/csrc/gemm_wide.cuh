@@ -98,7 +98,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 k_gemm_wide(const __grid_constant__ WideLaunch g) {
   using C = WideCfg<kMode, kBf16>;
   constexpr int S = C::kStages;
-  pdl_launch_dependents();
+  // programmatic dependent launch: every thread waits for the upstream grid
+  // before it triggers the next launch, so a next GEMM that is independent of
+  // this one may skip its own wait and still find this launch's inputs
+  // complete
+  if (!g.use_pdl) pdl_launch_dependents();
+  auto wait_upstream = [&]() {
+    if (g.use_pdl) {
+      pdl_wait();
+      pdl_launch_dependents();
+    }
+  };
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -154,7 +164,7 @@ k_gemm_wide(const __grid_constant__ WideLaunch g) {
   if (warp == 0 && C::kHybrid) {
     // ------------------------------------------------------------------ hybrid producer (both CTAs)
     // the whole warp reads a tile's dense flags; lane 0 issues the copies
-    if (g.use_pdl) pdl_wait();
+    wait_upstream();
     const uint32_t full0 = mapa_shared(bar_u32(kFull), 0);
     const int num_kt = g.num_kt, total_tiles = g.total_tiles, tiles_a = g.tiles_a, meta_blocks = g.meta_blocks;
     const uint64_t timeout_ns = g.timeout_ns;
@@ -219,8 +229,9 @@ k_gemm_wide(const __grid_constant__ WideLaunch g) {
     __syncwarp();
   } else if (warp == 0) {
     // ------------------------------------------------------------------ producer (both CTAs)
+    if (lane != 0) wait_upstream();
     if (lane == 0) {
-      if (g.use_pdl) pdl_wait();
+      wait_upstream();
       const uint32_t full0 = mapa_shared(bar_u32(kFull), 0);  // rank 0's stage barriers
       const int box_elems = kBf16 ? 64 : 128;                // 128 bytes of B per box row
       const int kc_total = g.K / 128;
@@ -271,6 +282,7 @@ k_gemm_wide(const __grid_constant__ WideLaunch g) {
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer (rank 0)
+    wait_upstream();  // nothing to issue before the producer's loads anyway
     if (rank == 0 && lane == 0) {
       const uint32_t idesc = make_idesc(C::kSparse, kBf16, 256, 256);
       const uint32_t idesc_dense = make_idesc(false, kBf16, 256, 256);  // hybrid dense K-steps
@@ -380,7 +392,7 @@ k_gemm_wide(const __grid_constant__ WideLaunch g) {
     __syncwarp();
   } else {
     // ------------------------------------------------------------------ epilogue (both CTAs)
-    if (g.use_pdl) pdl_wait();  // Y and the B scales may belong to the upstream grid
+    wait_upstream();  // Y and the B scales may belong to the upstream grid
     const int lg = warp & 3;
     const int row = lg * 32 + lane;   // accumulator lane of this thread
     const int et = threadIdx.x - 64;  // 0..127

@@ -511,6 +511,9 @@ int build_launch(GemmLaunch<kMaxProb>& gl, const sp24_gemm_args* const* a, int n
   gl.p.out_f32 = a[0]->out_dtype == SP24_F32;
   gl.p.use_pdl = 1;
   gl.p.w_static = w_static ? 1 : 0;
+  bool indep = true;
+  for (int i = 0; i < n; ++i) indep = indep && (a[i]->flags & SP24_GEMM_AFTER_INDEPENDENT) != 0;
+  gl.p.after_independent = indep ? 1 : 0;
   gl.p.timeout_ns = g_timeout_ns.load();
   return SP24_OK;
 }

@@ -35,6 +35,7 @@ SPARSE, DENSE = 0, 1
 GEMM_W_STATIC = 1
 GEMM_SINGLE_CTA = 2
 GEMM_CTA_PAIR = 4
+GEMM_AFTER_INDEPENDENT = 8
 
 
 class Sp24Error(RuntimeError):
@@ -295,10 +296,15 @@ class GemmGroup:
     held for the group's lifetime."""
 
     def __init__(self, args_list, workspace: Optional[torch.Tensor] = None,
-                 allocate_workspace: bool = True):
+                 allocate_workspace: bool = True, after_independent: bool = False):
         self.args_list = list(args_list)
         n = len(self.args_list)
         self.arr = (GemmArgs * n)(*self.args_list)
+        if after_independent:
+            # the launch before this one in the stream is an independent GEMM
+            # group (GEMM_AFTER_INDEPENDENT); set on this group's copies only
+            for i in range(n):
+                self.arr[i].flags |= GEMM_AFTER_INDEPENDENT
         self.n = n
         need = lib().sp24_gemm_grouped_workspace_bytes(self.arr, n)
         if workspace is None and need > 0 and allocate_workspace:

@@ -295,6 +295,58 @@ def test_grouped_gemm_whole_tiles_without_workspace(e4):
     check_group(items, "grouped whole tiles")
 
 
+def test_independent_group_chain_after_one_cast():
+    """A per-token cast, then three grouped launches of independent GEMMs on one
+    stream, the second and third flagged as following an independent GEMM
+    launch (they start before the previous group finishes and wait for it only
+    before exiting).  Every iteration casts different activations and writes
+    its own outputs, with no host synchronization in between, so a group that
+    read its activations before the cast finished would show the previous
+    iteration's values."""
+    classes = [[(1, 512, 1024), (8, 384, 2048)], [(32, 640, 1024)], [(128, 512, 1536), (100, 256, 1024)]]
+    iters = 4
+    torch.cuda.synchronize()
+    shapes = [sh for cl in classes for sh in cl]
+    Ws = [OracleSparseW(inputs.normal_bf16((N, K), 0.02, seed=100 + j), e4m3=True) for j, (_, N, K) in enumerate(shapes)]
+    Wd = [(dev(w.values), dev(w.image), dev(w.scales)) for w in Ws]
+    srcs = [[inputs.normal_bf16((M, K), 1.0, seed=1000 * t + j) for j, (M, _, K) in enumerate(shapes)]
+            for t in range(iters)]
+    xb = [[dev_bf16(x) for x in it] for it in srcs]
+    xq = [torch.empty(M, K, dtype=torch.uint8, device="cuda") for (M, _, K) in shapes]
+    xs = [torch.empty(M, dtype=torch.float32, device="cuda") for (M, _, _) in shapes]
+    Ys = [[torch.empty(M, N, dtype=torch.float32, device="cuda") for (M, N, _) in shapes] for _ in range(iters)]
+    # groups (and their workspaces) built first, so that the launches below
+    # follow one another directly in the stream
+    casts, groups = [], []
+    for t in range(iters):
+        casts.append(sp24.QuantGroup([(xb[t][j], xq[j], xs[j]) for j in range(len(shapes))]))
+        j0, gt = 0, []
+        for c, cl in enumerate(classes):
+            args = []
+            for j in range(j0, j0 + len(cl)):
+                v, m, sc = Wd[j]
+                args.append(sp24.gemm_args(xq[j], v, Ys[t][j], shapes[j][2], sp24.SPARSE, W_meta=m,
+                                           x_scales=xs[j], w_scales=sc, flags=sp24.GEMM_W_STATIC))
+            gt.append(sp24.GemmGroup(args, after_independent=c > 0))
+            j0 += len(cl)
+        groups.append(gt)
+    torch.cuda.synchronize()
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        for t in range(iters):
+            casts[t](stream)
+            for grp in groups[t]:
+                grp(stream)
+    torch.cuda.synchronize()
+    assert sp24.last_device_error() == sp24.SP24_OK
+    for t in range(iters):
+        for j, (M, N, K) in enumerate(shapes):
+            _, _, X_hat = oracle_x(srcs[t][j], True)
+            y_ref, a_ref = orc.gemm_f64(X_hat, Ws[j].W_hat)
+            check_tolerance(Ys[t][j].cpu().numpy().astype(np.float64), y_ref, a_ref,
+                            "iteration %d problem %d" % (t, j))
+
+
 def test_grouped_gemm_sixteen_problems_w_static_reusable():
     # the largest group: 16 decode projections of mixed sizes, weights marked
     # static; three calls on one workspace, which ends zero after each
