@@ -193,3 +193,16 @@ def test_energy_loss_validation():
     assert f(FAKE, 4, 60, 60, FAKE, None, None) == sp24.SP24_ERR_NOT_2_4
     assert f(FAKE, 4, 64, 68, FAKE, None, None) == sp24.SP24_ERR_ALIGNMENT
     assert f(FAKE + 8, 4, 64, 64, FAKE, None, None) == sp24.SP24_ERR_ALIGNMENT
+
+
+def test_binding_constants_match_the_header():
+    """The Python binding's enum and flag values are the header's."""
+    import os
+    import re
+    hdr = open(os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "sp24.h")).read()
+    defines = {m.group(1): int(m.group(2)) for m in re.finditer(r"#define\s+SP24_(GEMM_\w+)\s+(\d+)u", hdr)}
+    assert defines == {"GEMM_W_STATIC": sp24.GEMM_W_STATIC, "GEMM_SINGLE_CTA": sp24.GEMM_SINGLE_CTA,
+                       "GEMM_CTA_PAIR": sp24.GEMM_CTA_PAIR, "GEMM_AFTER_INDEPENDENT": sp24.GEMM_AFTER_INDEPENDENT}
+    # flag bits are distinct
+    vals = list(defines.values())
+    assert all(v & (v - 1) == 0 for v in vals) and len(set(vals)) == len(vals)
