@@ -53,8 +53,9 @@ def parse():
                         "workloads of the hot path, one JSON line each, eager calls with an L2 "
                         "flush before every timed call")
     p.add_argument("--case", default="",
-                   help="M,N,K[,bf16|e4m3[,sparse|dense]]: time one GEMM of the decode/prefill "
-                        "family in isolation (used for profiler captures) instead of the step; "
+                   help="M,N,K[,bf16|e4m3[,sparse|dense|hybrid]]: time one GEMM of the decode/prefill "
+                        "family in isolation (used for profiler captures) instead of the step; hybrid = "
+                        "e4m3 2:4 weights with 25%% dense 128 x 128 tiles; "
                         "group:M1,M2,...: one grouped launch of the decode GEMMs for those M")
     return p.parse_args()
 
@@ -562,18 +563,26 @@ def run_case(args):
     f = args.case.split(",")
     M, N, K = int(f[0]), int(f[1]), int(f[2])
     e4 = (f[3] if len(f) > 3 else "e4m3") == "e4m3"
-    sparse = (f[4] if len(f) > 4 else "sparse") == "sparse"
+    tactic = f[4] if len(f) > 4 else "sparse"
+    assert tactic in ("sparse", "dense", "hybrid"), tactic
+    hybrid = tactic == "hybrid"  # 2:4 weights with 25% dense 128 x 128 tiles (seeded), e4m3 only
+    assert e4 or not hybrid, "hybrid tiles are e4m3"
+    sparse = tactic != "dense"
     dev = torch.device("cuda", 0)
     W = torch.from_numpy(inputs.normal_bf16((N, K), 0.02, seed=N + K).view(np.int16)).view(
         torch.bfloat16).to(dev)
     X = torch.from_numpy(inputs.normal_bf16((M, K), 1.0, seed=M).view(np.int16)).view(
         torch.bfloat16).to(dev)
-    wsc = xs = meta = None
+    wsc = xs = meta = mask = dense = None
     if sparse:
         Wv = torch.empty(N, K // 2, dtype=torch.uint8 if e4 else torch.bfloat16, device=dev)
         meta = torch.empty(sp24.meta_bytes(N, K), dtype=torch.uint8, device=dev)
         wsc = torch.empty(N, dtype=torch.float32, device=dev) if e4 else None
-        sp24.prune_compress(W, sp24.E4M3 if e4 else sp24.BF16, Wv, meta, row_scales=wsc)
+        if hybrid:
+            mask = torch.from_numpy(inputs.hybrid_mask(N, K, seed=0)).to(dev)
+            dense = torch.empty(N, K, dtype=torch.uint8, device=dev)
+        sp24.prune_compress(W, sp24.E4M3 if e4 else sp24.BF16, Wv, meta, row_scales=wsc, tile_mask=mask,
+                            dense_tiles=dense)
     elif e4:
         Wv = torch.empty(N, K, dtype=torch.uint8, device=dev)
         wsc = torch.empty(N, dtype=torch.float32, device=dev)
@@ -588,7 +597,7 @@ def run_case(args):
         Xq = X
     Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
     a = sp24.gemm_args(Xq, Wv, Y, K, sp24.SPARSE if sparse else sp24.DENSE, W_meta=meta,
-                       x_scales=xs, w_scales=wsc)
+                       x_scales=xs, w_scales=wsc, tile_mask=mask, W_dense_tiles=dense)
     n = sp24.gemm_workspace_bytes(a)
     if n:
         sp24.set_workspace(a, torch.zeros(n, dtype=torch.uint8, device=dev))
@@ -596,6 +605,8 @@ def run_case(args):
     t, _ = _time_calls(lambda: sp24.gemm(a), args.steps, args.warmup, flush)
     eb = 1 if e4 else 2
     wbytes = N * K * eb // 2 + N * K // 8 if sparse else N * K * eb
+    if hybrid:  # a dense tile reads its dense form instead of its (zero) compressed slots
+        wbytes = int(0.75 * wbytes + 0.25 * N * K)
     byts = wbytes + M * K * eb + 2 * M * N
     print(json.dumps({"case": args.case, "us_median": round(t, 3), "GBps": round(byts / t / 1e3, 1),
                       "TFLOPS": round(2.0 * M * N * K / t / 1e6, 2),

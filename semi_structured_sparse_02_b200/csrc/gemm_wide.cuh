@@ -28,8 +28,12 @@
 // tile i's overlap implies tile i-1 is fully drained (the epilogue is
 // sequential), so one release per tile covers both accumulators.
 //
-// Work schedule: whole 256 x 256 tiles, round-robin over the pairs, A tile
-// index fastest (consecutive pairs share a B tile, all pairs share A in L2).
+// Work schedule: whole 256 x 256 tiles, round-robin over the pairs.  By
+// default the A tile index runs fastest (consecutive pairs share a B tile; A
+// is re-read from L2 for every B tile).  When A is the larger operand and B
+// fits comfortably in L2 (b_fastest, chosen on the host), the B index runs
+// fastest instead, so that each A tile streams from HBM once and B is the
+// operand re-read from L2.
 //
 // Hybrid weights (E4M3, a dense/sparse flag per 128 x 128 tile of A): the
 // two CTAs of a pair hold two different 128-row blocks, and one pair MMA
@@ -56,6 +60,7 @@ struct WideLaunch {
   int32_t rows_a, rows_b, K, num_kt;
   int32_t tiles_a, tiles_b;  // 256-row tiles
   int32_t total_tiles, meta_blocks;  // metadata row blocks (128 rows) that exist
+  int32_t b_fastest;                 // tile order: B tile index fastest (else A)
   int32_t out_f32, use_pdl;
   const float* scale_a;
   const float* scale_b;
@@ -167,6 +172,8 @@ k_gemm_wide(const __grid_constant__ WideLaunch g) {
     wait_upstream();
     const uint32_t full0 = mapa_shared(bar_u32(kFull), 0);
     const int num_kt = g.num_kt, total_tiles = g.total_tiles, tiles_a = g.tiles_a, meta_blocks = g.meta_blocks;
+    const int tiles_b = g.tiles_b;
+    const bool b_fastest = g.b_fastest != 0;
     const uint64_t timeout_ns = g.timeout_ns;
     const uint8_t* const mask = g.tile_mask;
     constexpr uint32_t kDenseTx = 2u * (128 * 128 + 128 * 128);          // A dense + B, both CTAs
@@ -177,7 +184,8 @@ k_gemm_wide(const __grid_constant__ WideLaunch g) {
     uint32_t phase = 0;
     bool ok = true;
     for (int tile = pair; tile < total_tiles; tile += n_pairs) {
-      const int ta = tile % tiles_a, tb = tile / tiles_a;
+      const int ta = b_fastest ? tile / tiles_b : tile % tiles_a;
+      const int tb = b_fastest ? tile % tiles_b : tile / tiles_a;
       const int rb0 = ta * 2, rb1 = ta * 2 + 1;  // the pair's two 128-row blocks
       __syncwarp();  // lane 0 has finished with the previous tile's flags
       for (int kt = lane; kt < num_kt; kt += 32) {
@@ -237,6 +245,8 @@ k_gemm_wide(const __grid_constant__ WideLaunch g) {
       const int kc_total = g.K / 128;
       // parameter fields in registers (the asm below clobbers memory)
       const int num_kt = g.num_kt, total_tiles = g.total_tiles, tiles_a = g.tiles_a, meta_blocks = g.meta_blocks;
+      const int tiles_b = g.tiles_b;
+      const bool b_fastest = g.b_fastest != 0;
       const uint64_t timeout_ns = g.timeout_ns;
       int armed[S];
       for (int s = 0; s < S; ++s) armed[s] = -1;
@@ -244,7 +254,8 @@ k_gemm_wide(const __grid_constant__ WideLaunch g) {
       uint32_t phase = 0;
       bool ok = true;
       for (int tile = pair; ok && tile < total_tiles; tile += n_pairs) {
-        const int ta = tile % tiles_a, tb = tile / tiles_a;
+        const int ta = b_fastest ? tile / tiles_b : tile % tiles_a;
+        const int tb = b_fastest ? tile % tiles_b : tile / tiles_a;
         const int ya = ta * 256 + (int)rank * 128;
         const int yb = tb * 256 + (int)rank * 128;
         int rb = ta * 2 + (int)rank;        // metadata row block of this CTA's A rows
@@ -402,13 +413,16 @@ k_gemm_wide(const __grid_constant__ WideLaunch g) {
     // memory, which would force parameter fields to be re-read after each)
     const bool out_f32 = g.out_f32 != 0;
     const int rows_a = g.rows_a, rows_b = g.rows_b, tiles_a = g.tiles_a, total_tiles = g.total_tiles;
+    const int tiles_b = g.tiles_b;
+    const bool b_fastest = g.b_fastest != 0;
     uint8_t* const Yb = static_cast<uint8_t*>(g.Y);
     const int64_t ldy = g.ldy;
     const float* const scale_a = g.scale_a;
     const float* const scale_b = g.scale_b;
     int j = 0;
     for (int tile = pair; tile < total_tiles; tile += n_pairs, ++j) {
-      const int ta = tile % tiles_a, tb = tile / tiles_a;
+      const int ta = b_fastest ? tile / tiles_b : tile % tiles_a;
+      const int tb = b_fastest ? tile % tiles_b : tile / tiles_a;
       const int b = j & 1;
       const int ga = ta * 256 + (int)rank * 128 + row;  // A row of this thread
       const float sa_v = (scale_a != nullptr && ga < rows_a) ? __ldg(scale_a + ga) : 1.0f;

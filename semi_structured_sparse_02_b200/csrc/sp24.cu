@@ -708,6 +708,18 @@ int run_wide(int mode, bool bf16, bool a_is_w, const void* A, int64_t lda, const
   wl.tiles_b = (int32_t)((rows_b + 255) / 256);
   wl.total_tiles = wl.tiles_a * wl.tiles_b;
   wl.meta_blocks = meta_blocks;
+  // tile order: with A running fastest, all of A is re-read (from L2 if it
+  // fits) for every B tile.  When A is the larger operand and B fits easily
+  // in L2, run B fastest instead so that each A tile streams from HBM once
+  // (e.g. 24576 x 4096 hybrid weights, ~160 MB with their dense form, against
+  // 4096 e4m3 tokens, 17 MB: DRAM reads measured ~6x the weight bytes with A
+  // fastest).
+  {
+    const double a_bytes = (double)rows_a * (double)K *
+                           (hybrid ? 1.0 + 0.5 + 0.125 : sparse ? (double)eb / 2 + 0.125 : (double)eb);
+    const double b_bytes = (double)rows_b * (double)K * eb;
+    wl.b_fastest = (a_bytes > b_bytes && b_bytes <= 32.0 * 1024 * 1024) ? 1 : 0;
+  }
   wl.out_f32 = out_f32 ? 1 : 0;
   wl.use_pdl = 1;
   wl.scale_a = scale_a;

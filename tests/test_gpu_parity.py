@@ -783,6 +783,135 @@ def test_prefill_full_size_sampled(e4):
     check_tolerance(y_gpu, y_ref, a_ref, "prefill e4=%s" % e4)
 
 
+def test_decode_step_full_size_grouped_sampled():
+    """The decode step as the benchmark times it: 16 GEMMs (M in 1, 8, 32, 128
+    times the four weight shapes, e4m3 2:4 weights), one grouped per-token cast,
+    then one grouped launch per token-count class, weights marked static, the
+    second and third groups chained after the first as independent launches.
+    Sampled outputs of every GEMM against the oracle."""
+    g = np.random.default_rng(7)
+    Wb = {}
+    for (N, K) in inputs.DECODE_NK:
+        W = inputs.normal_bf16((N, K), 0.02, seed=N + K)
+        vals = torch.empty(N, K // 2, dtype=torch.uint8, device="cuda")
+        meta = torch.empty(sp24.meta_bytes(N, K), dtype=torch.uint8, device="cuda")
+        sc = torch.empty(N, dtype=torch.float32, device="cuda")
+        sp24.prune_compress(dev_bf16(W), sp24.E4M3, vals, meta, row_scales=sc)
+        Wb[(N, K)] = (W, vals, meta, sc)
+    items = []
+    for M in inputs.DECODE_M:
+        for i, (N, K) in enumerate(inputs.DECODE_NK):
+            X = inputs.normal_bf16((M, K), 1.0, seed=M * 10 + i)
+            xq = torch.empty(M, K, dtype=torch.uint8, device="cuda")
+            xs = torch.empty(M, dtype=torch.float32, device="cuda")
+            Y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+            _, vals, meta, sc = Wb[(N, K)]
+            a = sp24.gemm_args(xq, vals, Y, K, sp24.SPARSE, W_meta=meta, x_scales=xs, w_scales=sc,
+                               flags=sp24.GEMM_W_STATIC)
+            items.append(dict(M=M, N=N, K=K, X=X, Xd=dev_bf16(X), xq=xq, xs=xs, Y=Y, a=a))
+    cast = sp24.QuantGroup([(it["Xd"], it["xq"], it["xs"]) for it in items])
+    by = {}
+    for it in items:
+        by.setdefault(sp24.m_class(it["M"]), []).append(it["a"])
+    groups = [sp24.GemmGroup(v, after_independent=i > 0) for i, (_, v) in enumerate(sorted(by.items()))]
+    assert len(groups) == 3
+    torch.cuda.synchronize()
+    for _ in range(2):  # the second pass runs on workspaces the first left at zero
+        cast()
+        for grp in groups:
+            grp()
+    torch.cuda.synchronize()
+    assert sp24.last_device_error() == sp24.SP24_OK
+    for it in items:
+        M, N, K = it["M"], it["N"], it["K"]
+        ns = g.choice(N, size=24, replace=False)
+        ms = g.integers(0, M, size=24)
+        ref = OracleSparseW(Wb[(N, K)][0][ns], e4m3=True)
+        _, _, X_hat = oracle_x(it["X"], True)
+        y_ref, a_ref = orc.gemm_f64_sampled(X_hat, ref.W_hat, ms, np.arange(ns.size))
+        y_gpu = it["Y"].float().cpu().numpy().astype(np.float64)[ms, ns]
+        check_tolerance(y_gpu, y_ref, a_ref, "decode step M%d %dx%d" % (M, N, K))
+
+
+@pytest.mark.parametrize("name,M", [("gate_up", 4096), ("qkv", 16)])
+def test_hybrid_full_size_sampled(name, M):
+    """Hybrid weights (25% dense 128 x 128 tiles, e4m3) at full size: gate_up at
+    4096 tokens runs on CTA pairs, qkv at 16 tokens on single CTAs.  The
+    weights are pruned on the device; the oracle checks two whole 128-row
+    blocks (their tile flags carried along) against 16 sampled tokens."""
+    N, K = {n: (N_, K_) for n, N_, K_ in inputs.HYBRID_NK}[name]
+    W = inputs.normal_bf16((N, K), 0.02, seed=N + 3)
+    X = inputs.normal_bf16((M, K), 1.0, seed=M + 3)
+    mask = inputs.hybrid_mask(N, K, seed=5)
+    vals = torch.empty(N, K // 2, dtype=torch.uint8, device="cuda")
+    meta = torch.empty(sp24.meta_bytes(N, K), dtype=torch.uint8, device="cuda")
+    dense = torch.empty(N, K, dtype=torch.uint8, device="cuda")
+    sc = torch.empty(N, dtype=torch.float32, device="cuda")
+    sp24.prune_compress(dev_bf16(W), sp24.E4M3, vals, meta, row_scales=sc, tile_mask=dev(mask), dense_tiles=dense)
+    xq = torch.empty(M, K, dtype=torch.uint8, device="cuda")
+    xs = torch.empty(M, dtype=torch.float32, device="cuda")
+    sp24.quantize_e4m3_rows(dev_bf16(X), xq, xs)
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    a = sp24.gemm_args(xq, vals, Y, K, sp24.SPARSE, W_meta=meta, x_scales=xs, w_scales=sc,
+                       tile_mask=dev(mask), W_dense_tiles=dense)
+    sp24.set_workspace(a, workspace_for(a))
+    sp24.gemm(a)
+    torch.cuda.synchronize()
+    assert sp24.last_device_error() == sp24.SP24_OK
+    g = np.random.default_rng(11)
+    rbs = np.sort(g.choice(N // 128, size=2, replace=False))
+    rows = np.concatenate([np.arange(128 * rb, 128 * rb + 128) for rb in rbs])
+    ref = OracleSparseW(W[rows], e4m3=True, mask=mask[rbs])
+    ms = np.sort(g.choice(M, size=min(M, 16), replace=False))
+    _, _, X_hat = oracle_x(X[ms], True)
+    y_ref, a_ref = orc.gemm_f64(X_hat, ref.W_hat)
+    y_gpu = Y.float().cpu().numpy().astype(np.float64)[np.ix_(ms, rows)]
+    check_tolerance(y_gpu, y_ref, a_ref, "hybrid %s M%d" % (name, M))
+
+
+@pytest.mark.parametrize("e4", [False, True])
+def test_activation_full_size_sampled(e4):
+    """The online activation path at its full size (X 8192 x 4096 Student-t,
+    W 12288 x 4096): compressed X of sampled rows and of the first row block's
+    metadata bit-exact, sampled outputs within tolerance."""
+    M, K, N = inputs.ACT_SHAPE["M"], inputs.ACT_SHAPE["K"], inputs.ACT_SHAPE["N"]
+    X = inputs.student_t_bf16((M, K), 3.0, seed=4)
+    W = inputs.normal_bf16((N, K), 0.02, seed=4)
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    xm = torch.empty(sp24.meta_bytes(M, K), dtype=torch.uint8, device="cuda")
+    xv = torch.empty(M, K // 2, dtype=torch.uint8 if e4 else torch.bfloat16, device="cuda")
+    if e4:
+        wq, wsc = orc.quantize_rows_e4m3(W)
+        xs = torch.empty(M, dtype=torch.float32, device="cuda")
+        sp24.prune_compress_activations_fused_e4m3(dev_bf16(X), dev(wq), dev(wsc), Y, x_values=xv, x_meta=xm,
+                                                   x_scales=xs)
+    else:
+        sp24.prune_compress_activations_fused(dev_bf16(X), dev_bf16(W), Y, x_values=xv, x_meta=xm)
+    torch.cuda.synchronize()
+    assert sp24.last_device_error() == sp24.SP24_OK
+    g = np.random.default_rng(13)
+    ms = np.sort(g.choice(M, size=32, replace=False))
+    ns = np.sort(g.choice(N, size=32, replace=False))
+    img0 = u8(xm)[:(K // 128) * 2048]  # row block 0's chunks come first in the image
+    if e4:
+        ref = OracleSparseW(X[ms], e4m3=True)
+        assert np.array_equal(u8(xv)[ms], ref.values)
+        assert np.array_equal(xs.cpu().numpy()[ms].view(np.uint32), ref.scales.view(np.uint32))
+        assert np.array_equal(img0, OracleSparseW(X[:128], e4m3=True).image)
+        W_hat = orc.e4m3_decode(wq[ns]) * wsc[ns].astype(np.float64)[:, None]
+        X_hat = ref.W_hat
+    else:
+        pruned, vals, canon = orc.prune_compress_bf16(X[ms])
+        assert np.array_equal(bits16(xv)[ms], vals)
+        _, _, canon0 = orc.prune_compress_bf16(X[:128])
+        assert np.array_equal(img0, orc.meta_image(canon0, 128, K, False))
+        W_hat = orc.bf16_bits_to_f64(W[ns])
+        X_hat = orc.bf16_bits_to_f64(pruned)
+    y_ref, a_ref = orc.gemm_f64(X_hat, W_hat)
+    y_gpu = Y.float().cpu().numpy().astype(np.float64)[np.ix_(ms, ns)]
+    check_tolerance(y_gpu, y_ref, a_ref, "activations full size e4=%s" % e4)
+
+
 # ---------------------------------------------------------------------------
 # tactic selector (kernel 5) and the bounded wait
 # ---------------------------------------------------------------------------
