@@ -59,6 +59,18 @@ def lib() -> ctypes.CDLL:
             "orc_gemm_sparse_f64": (None, [P, I64, I64, P, P, I64, P]),
             "orc_bf16_to_double": (ctypes.c_double, [ctypes.c_uint16]),
             "orc_energy_loss": (None, [P, I64, I64, I64, P, P]),
+            "orc_e2m1_decode": (ctypes.c_double, [ctypes.c_uint8]),
+            "orc_e2m1_encode": (ctypes.c_uint8, [ctypes.c_double]),
+            "orc_prune_pairs8": (ctypes.c_int, [P, P, P]),
+            "orc_prune_pairs_bf16": (None, [P, I64, I64, I64, P]),
+            "orc_nvfp4_tensor_scale": (ctypes.c_float, [ctypes.c_float]),
+            "orc_nvfp4_block_code": (ctypes.c_uint8, [ctypes.c_float, ctypes.c_float]),
+            "orc_nvfp4_code": (ctypes.c_uint8, [ctypes.c_float, ctypes.c_uint8, ctypes.c_float]),
+            "orc_nvfp4_48_compress": (None, [P, I64, I64, I64, P, P, P, P]),
+            "orc_nvfp4_48_dequant": (None, [P, P, P, ctypes.c_float, I64, I64, P]),
+            "orc_nvfp4_quantize": (None, [P, I64, I64, I64, P, P, P]),
+            "orc_nvfp4_dequant": (None, [P, P, ctypes.c_float, I64, I64, P]),
+            "orc_energy_loss_48": (None, [P, I64, I64, I64, P, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -273,3 +285,104 @@ def sparse_gpu_time_coverage(selected_times):
     tot = sum(t for _, t in selected_times)
     sp = sum(t for tac, t in selected_times if tac == "sparse")
     return sp / tot if tot > 0 else 0.0
+
+
+# ---------------------------------------------------------------------------
+# pairwise 4:8 sparsity with NVFP4 values  [P4 section 2 "Quantization";
+# section 6.2 "What pairwise 4:8 costs on Blackwell"]
+# ---------------------------------------------------------------------------
+
+def e2m1_decode(codes: np.ndarray) -> np.ndarray:
+    """Values of E2M1 codes (low 4 bits: sign, two exponent bits, mantissa)."""
+    table = np.array([lib().orc_e2m1_decode(c) for c in range(16)], np.float64)
+    return table[np.asarray(codes, dtype=np.uint8) & 0xF]
+
+
+def e2m1_encode(x) -> np.ndarray:
+    """Round to nearest E2M1 (ties to the even code, saturating to 6)."""
+    xs = np.asarray(x, dtype=np.float64)
+    return np.array([lib().orc_e2m1_encode(float(v)) for v in xs.ravel()], np.uint8).reshape(xs.shape)
+
+
+def prune_pairs8(v_bits: Sequence[int]):
+    """(nibble, p0, p1) for one group of eight bf16 bit patterns."""
+    a = np.ascontiguousarray(np.asarray(v_bits, dtype=np.uint16))
+    p0 = ctypes.c_int()
+    p1 = ctypes.c_int()
+    nib = lib().orc_prune_pairs8(_p(a), ctypes.byref(p0), ctypes.byref(p1))
+    return nib, p0.value, p1.value
+
+
+def prune_pairs_bf16(W_bits: np.ndarray) -> np.ndarray:
+    """The pairwise 4:8 pruned matrix (bf16 bits, dropped positions +0)."""
+    W = np.ascontiguousarray(W_bits, dtype=np.uint16)
+    rows, K = W.shape
+    out = np.empty((rows, K), np.uint16)
+    lib().orc_prune_pairs_bf16(_p(W), rows, K, K, _p(out))
+    return out
+
+
+def nvfp4_tensor_scale(amax: float) -> float:
+    return float(lib().orc_nvfp4_tensor_scale(ctypes.c_float(amax)))
+
+
+def nvfp4_block_code(amax_b: float, s_t: float) -> int:
+    return int(lib().orc_nvfp4_block_code(ctypes.c_float(amax_b), ctypes.c_float(s_t)))
+
+
+def nvfp4_code(v: float, b: int, s_t: float) -> int:
+    return int(lib().orc_nvfp4_code(ctypes.c_float(v), ctypes.c_uint8(b), ctypes.c_float(s_t)))
+
+
+def nvfp4_48_compress(W_bits: np.ndarray):
+    """Sparse pairwise 4:8 NVFP4 operand: (values [rows, K/4] packed codes,
+    meta [rows, K/16] canonical nibbles, block scales [rows, K/32] E4M3
+    codes, tensor scale)."""
+    W = np.ascontiguousarray(W_bits, dtype=np.uint16)
+    rows, K = W.shape
+    assert K % 32 == 0
+    values = np.empty((rows, K // 4), np.uint8)
+    meta = np.empty((rows, K // 16), np.uint8)
+    scales = np.empty((rows, K // 32), np.uint8)
+    st = ctypes.c_float()
+    lib().orc_nvfp4_48_compress(_p(W), rows, K, K, _p(values), _p(meta), _p(scales), ctypes.byref(st))
+    return values, meta, scales, float(st.value)
+
+
+def nvfp4_48_dequant(values, meta, scales, tensor_scale: float, rows: int, K: int) -> np.ndarray:
+    out = np.empty((rows, K), np.float64)
+    lib().orc_nvfp4_48_dequant(_p(np.ascontiguousarray(values)), _p(np.ascontiguousarray(meta)),
+                               _p(np.ascontiguousarray(scales)), ctypes.c_float(tensor_scale), rows, K, _p(out))
+    return out
+
+
+def nvfp4_quantize(W_bits: np.ndarray):
+    """Dense NVFP4: (codes [rows, K/2] packed, block scales [rows, K/16], tensor scale)."""
+    W = np.ascontiguousarray(W_bits, dtype=np.uint16)
+    rows, K = W.shape
+    assert K % 16 == 0
+    codes = np.empty((rows, K // 2), np.uint8)
+    scales = np.empty((rows, K // 16), np.uint8)
+    st = ctypes.c_float()
+    lib().orc_nvfp4_quantize(_p(W), rows, K, K, _p(codes), _p(scales), ctypes.byref(st))
+    return codes, scales, float(st.value)
+
+
+def nvfp4_dequant(codes, scales, tensor_scale: float, rows: int, K: int) -> np.ndarray:
+    out = np.empty((rows, K), np.float64)
+    lib().orc_nvfp4_dequant(_p(np.ascontiguousarray(codes)), _p(np.ascontiguousarray(scales)),
+                            ctypes.c_float(tensor_scale), rows, K, _p(out))
+    return out
+
+
+def energy_loss_48(W_bits: np.ndarray):
+    """Pairwise 4:8 energy loss: (per-row dropped, per-row total, per-row
+    share, tensor share), as energy_loss for 2:4."""
+    W = np.ascontiguousarray(W_bits, dtype=np.uint16)
+    rows, K = W.shape
+    dropped = np.empty(rows, np.float64)
+    total = np.empty(rows, np.float64)
+    lib().orc_energy_loss_48(_p(W), rows, K, K, _p(dropped), _p(total))
+    share = np.where(total > 0, dropped / np.where(total > 0, total, 1.0), 0.0)
+    tensor = float(dropped.sum() / total.sum()) if total.sum() > 0 else 0.0
+    return dropped, total, share, tensor

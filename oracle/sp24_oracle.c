@@ -515,3 +515,254 @@ void orc_energy_loss(const uint16_t *src, int64_t rows, int64_t K, int64_t ld,
         row_total[r] = total;
     }
 }
+
+/* ================================================================== */
+/* Pairwise 4:8 sparsity with NVFP4 values  [P4 section 2             */
+/*    "Quantization" (NVFP4: E2M1 values, one E4M3 scale per 16        */
+/*    elements, one per-tensor scale) and section 6.2 "What pairwise   */
+/*    4:8 costs on Blackwell" (in each group of eight elements two of  */
+/*    the four adjacent pairs are kept; the sparse block-scaled GEMM   */
+/*    carries one scale per 32 positions of the reduction axis)]       */
+/*  [EXT] OCP microscaling formats specification, E2M1 encoding (one   */
+/*    sign bit, two exponent bits with bias 1, one mantissa bit, no    */
+/*    infinities or NaN, largest finite 6).                            */
+/* Readings (listed in the design notes): R14 a pair's weight is its   */
+/* energy x0^2 + x1^2 (exact in fp64 from bf16), the two heaviest of   */
+/* the four pairs are kept, ties to the lower pair index; R15 the      */
+/* scale arithmetic below, each step one correctly rounded fp32        */
+/* operation; R16 block and tensor scales of the sparse operand come   */
+/* from the kept values; R17 the storage layout below.                 */
+/* ================================================================== */
+
+/* E2M1 code (low 4 bits): sign bit 3, exponent bits 2..1, mantissa bit 0. */
+double orc_e2m1_decode(uint8_t q)
+{
+    int s = (q >> 3) & 1;
+    int e = (q >> 1) & 3;
+    int m = q & 1;
+    double mag = (e == 0) ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+    return s ? -mag : mag;
+}
+
+/* Round to nearest E2M1, ties to the even code (mantissa bit 0), magnitudes
+ * above 6 saturate to 6; the sign is kept (a negative value that rounds to
+ * zero gives the negative-zero code).  A plain scan of the eight magnitudes. */
+uint8_t orc_e2m1_encode(double x)
+{
+    uint8_t sign = (x < 0.0 || (x == 0.0 && signbit(x))) ? 0x8 : 0x0;
+    double a = fabs(x);
+    int best = 0;
+    double best_d = INFINITY;
+    for (int c = 0; c < 8; ++c) {
+        double d = fabs(a - orc_e2m1_decode((uint8_t)c));
+        if (d < best_d || (d == best_d && (c & 1) == 0)) {
+            best = c;
+            best_d = d;
+        }
+    }
+    if (a > 6.0) best = 7;
+    return (uint8_t)(sign | best);
+}
+
+/* The pair rule on one group of eight bf16 values: pair j holds elements
+ * 2j and 2j+1; pair j is kept iff fewer than two pairs beat it, where i
+ * beats j when e_i > e_j, or e_i == e_j and i < j.  Returns the canonical
+ * nibble p0 | p1 << 2 (p0 < p1). */
+int orc_prune_pairs8(const uint16_t v[8], int *p0, int *p1)
+{
+    double e[4];
+    for (int j = 0; j < 4; ++j) {
+        double a = orc_bf16_to_double(v[2 * j]), b = orc_bf16_to_double(v[2 * j + 1]);
+        e[j] = a * a + b * b;
+    }
+    int kept[2];
+    int nk = 0;
+    for (int j = 0; j < 4; ++j) {
+        int beaten_by = 0;
+        for (int i = 0; i < 4; ++i) {
+            if (i == j) continue;
+            if (e[i] > e[j] || (e[i] == e[j] && i < j)) beaten_by++;
+        }
+        if (beaten_by < 2) kept[nk++] = j;
+    }
+    *p0 = kept[0];
+    *p1 = kept[1];
+    return kept[0] | (kept[1] << 2);
+}
+
+/* The 4:8 pruned matrix in bf16 (dropped positions +0).  K % 8 == 0. */
+void orc_prune_pairs_bf16(const uint16_t *src, int64_t rows, int64_t K, int64_t ld, uint16_t *pruned)
+{
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t g = 0; g < K / 8; ++g) {
+            const uint16_t *v = src + r * ld + 8 * g;
+            int p0, p1;
+            orc_prune_pairs8(v, &p0, &p1);
+            for (int i = 0; i < 8; ++i)
+                pruned[r * K + 8 * g + i] = (i / 2 == p0 || i / 2 == p1) ? v[i] : (uint16_t)0;
+        }
+}
+
+/* Per-tensor scale from the tensor amax (R15): amax / (448 * 6), 1 for 0. */
+float orc_nvfp4_tensor_scale(float amax)
+{
+    return amax == 0.0f ? 1.0f : div_f32(amax, 2688.0f);
+}
+
+/* Block scale code from the block amax (R15): E4M3(amax / (6 * s_t)). */
+uint8_t orc_nvfp4_block_code(float amax_b, float s_t)
+{
+    return orc_e4m3_encode((double)div_f32(amax_b, mul_f32(6.0f, s_t)));
+}
+
+/* E2M1 code of v under block code b and tensor scale s_t (R15): the
+ * effective scale is S = decode(b) * s_t in fp32 and the code rounds v / S
+ * (one fp32 division); a zero scale gives code 0. */
+uint8_t orc_nvfp4_code(float v, uint8_t b, float s_t)
+{
+    float S = mul_f32((float)orc_e4m3_decode(b), s_t);
+    if (S == 0.0f) return 0;
+    return orc_e2m1_encode((double)div_f32(v, S));
+}
+
+static void put_nibble(uint8_t *base, int64_t idx, uint8_t nib)
+{
+    if (idx % 2 == 0) base[idx / 2] = (uint8_t)((base[idx / 2] & 0xF0) | (nib & 0xF));
+    else base[idx / 2] = (uint8_t)((base[idx / 2] & 0x0F) | ((nib & 0xF) << 4));
+}
+
+static uint8_t get_nibble(const uint8_t *base, int64_t idx)
+{
+    return (uint8_t)((base[idx / 2] >> ((idx % 2) * 4)) & 0xF);
+}
+
+/* Sparse operand, pairwise 4:8 with NVFP4 values (R16, R17).  K % 32 == 0.
+ *   values:   [rows x K/4] bytes, the kept elements in ascending position,
+ *             two E2M1 codes per byte (the earlier element in the low nibble)
+ *   meta:     [rows x K/16] bytes, one canonical nibble p0 | p1 << 2 per
+ *             group of eight, the even group in the low nibble
+ *   scales:   [rows x K/32] E4M3 block codes, one per 32 positions of K
+ *             (16 kept values)
+ *   *tensor_scale: the fp32 per-tensor scale.
+ * The tensor amax and each block amax run over the kept values. */
+void orc_nvfp4_48_compress(const uint16_t *src, int64_t rows, int64_t K, int64_t ld,
+                           uint8_t *values, uint8_t *meta, uint8_t *scales, float *tensor_scale)
+{
+    float amax_t = 0.0f;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t g = 0; g < K / 8; ++g) {
+            const uint16_t *v = src + r * ld + 8 * g;
+            int p0, p1;
+            orc_prune_pairs8(v, &p0, &p1);
+            const int pos[4] = {2 * p0, 2 * p0 + 1, 2 * p1, 2 * p1 + 1};
+            for (int i = 0; i < 4; ++i) {
+                float a = fabsf(bf16_to_float(v[pos[i]]));
+                if (a > amax_t) amax_t = a;
+            }
+        }
+    const float s_t = orc_nvfp4_tensor_scale(amax_t);
+    *tensor_scale = s_t;
+    memset(values, 0, (size_t)(rows * (K / 4)));
+    memset(meta, 0, (size_t)(rows * (K / 16)));
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t blk = 0; blk < K / 32; ++blk) {
+            float kept[16];
+            int nk = 0;
+            for (int64_t g = 4 * blk; g < 4 * blk + 4; ++g) {
+                const uint16_t *v = src + r * ld + 8 * g;
+                int p0, p1;
+                int nib = orc_prune_pairs8(v, &p0, &p1);
+                put_nibble(meta + r * (K / 16), g, (uint8_t)nib);
+                const int pos[4] = {2 * p0, 2 * p0 + 1, 2 * p1, 2 * p1 + 1};
+                for (int i = 0; i < 4; ++i) kept[nk++] = bf16_to_float(v[pos[i]]);
+            }
+            float amax_b = 0.0f;
+            for (int i = 0; i < 16; ++i)
+                if (fabsf(kept[i]) > amax_b) amax_b = fabsf(kept[i]);
+            const uint8_t b = orc_nvfp4_block_code(amax_b, s_t);
+            scales[r * (K / 32) + blk] = b;
+            for (int i = 0; i < 16; ++i)
+                put_nibble(values + r * (K / 4), 16 * blk + i, orc_nvfp4_code(kept[i], b, s_t));
+        }
+}
+
+/* The dequantized dense matrix of a 4:8 NVFP4 operand (fp64, [rows x K]):
+ * each kept code times its block scale times the tensor scale, zeros at
+ * the dropped positions. */
+void orc_nvfp4_48_dequant(const uint8_t *values, const uint8_t *meta, const uint8_t *scales,
+                          float tensor_scale, int64_t rows, int64_t K, double *out)
+{
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t k = 0; k < K; ++k) out[r * K + k] = 0.0;
+        for (int64_t g = 0; g < K / 8; ++g) {
+            const uint8_t nib = get_nibble(meta + r * (K / 16), g);
+            const int p0 = nib & 3, p1 = (nib >> 2) & 3;
+            const int pos[4] = {2 * p0, 2 * p0 + 1, 2 * p1, 2 * p1 + 1};
+            const double sb = orc_e4m3_decode(scales[r * (K / 32) + g / 4]) * (double)tensor_scale;
+            for (int i = 0; i < 4; ++i)
+                out[r * K + 8 * g + pos[i]] = orc_e2m1_decode(get_nibble(values + r * (K / 4), 4 * g + i)) * sb;
+        }
+    }
+}
+
+/* Dense NVFP4 (the dense side at the same floor): one E4M3 block code per
+ * 16 elements along K, the tensor scale from the whole matrix (R15).
+ *   codes: [rows x K/2] bytes, two E2M1 codes per byte; scales: [rows x K/16]. */
+void orc_nvfp4_quantize(const uint16_t *src, int64_t rows, int64_t K, int64_t ld,
+                        uint8_t *codes, uint8_t *scales, float *tensor_scale)
+{
+    float amax_t = 0.0f;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t k = 0; k < K; ++k) {
+            float a = fabsf(bf16_to_float(src[r * ld + k]));
+            if (a > amax_t) amax_t = a;
+        }
+    const float s_t = orc_nvfp4_tensor_scale(amax_t);
+    *tensor_scale = s_t;
+    memset(codes, 0, (size_t)(rows * (K / 2)));
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t blk = 0; blk < K / 16; ++blk) {
+            float amax_b = 0.0f;
+            for (int i = 0; i < 16; ++i) {
+                float a = fabsf(bf16_to_float(src[r * ld + 16 * blk + i]));
+                if (a > amax_b) amax_b = a;
+            }
+            const uint8_t b = orc_nvfp4_block_code(amax_b, s_t);
+            scales[r * (K / 16) + blk] = b;
+            for (int i = 0; i < 16; ++i)
+                put_nibble(codes + r * (K / 2), 16 * blk + i,
+                           orc_nvfp4_code(bf16_to_float(src[r * ld + 16 * blk + i]), b, s_t));
+        }
+}
+
+/* The dequantized matrix of a dense NVFP4 operand (fp64, [rows x K]). */
+void orc_nvfp4_dequant(const uint8_t *codes, const uint8_t *scales, float tensor_scale,
+                       int64_t rows, int64_t K, double *out)
+{
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t k = 0; k < K; ++k)
+            out[r * K + k] = orc_e2m1_decode(get_nibble(codes + r * (K / 2), k)) *
+                             orc_e4m3_decode(scales[r * (K / 16) + k / 16]) * (double)tensor_scale;
+}
+
+/* 4:8 pairwise energy loss per row, as orc_energy_loss for 2:4: the energy
+ * of the values the pair rule drops and of the whole row (fp64). */
+void orc_energy_loss_48(const uint16_t *src, int64_t rows, int64_t K, int64_t ld,
+                        double *row_dropped, double *row_total)
+{
+    for (int64_t r = 0; r < rows; ++r) {
+        double dropped = 0.0, total = 0.0;
+        for (int64_t g = 0; g < K / 8; ++g) {
+            const uint16_t *v = src + r * ld + 8 * g;
+            int p0, p1;
+            orc_prune_pairs8(v, &p0, &p1);
+            for (int i = 0; i < 8; ++i) {
+                const double x = orc_bf16_to_double(v[i]);
+                total += x * x;
+                if (i / 2 != p0 && i / 2 != p1) dropped += x * x;
+            }
+        }
+        row_dropped[r] = dropped;
+        row_total[r] = total;
+    }
+}

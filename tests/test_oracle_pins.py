@@ -397,3 +397,158 @@ def test_energy_loss_brute_force_by_sorting():
     d, t, share, tensor = orc.energy_loss(W)
     assert np.allclose(d, dropped, rtol=1e-14, atol=0) and np.allclose(t, total, rtol=1e-14, atol=0)
     assert tensor == pytest.approx(dropped.sum() / total.sum(), rel=1e-14)
+
+
+# ---------------------------------------------------------------------------
+# pairwise 4:8 sparsity with NVFP4 values (the next row after the 2:4 path)
+# ---------------------------------------------------------------------------
+
+# E2M1 magnitudes as tabulated in the OCP microscaling specification
+E2M1_MAGNITUDES = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+
+
+def test_e2m1_table_ties_to_even_and_saturation():
+    vals = orc.e2m1_decode(np.arange(16))
+    assert list(vals[:8]) == E2M1_MAGNITUDES
+    assert list(-vals[8:]) == E2M1_MAGNITUDES and all(np.signbit(vals[8:]))
+    # representable values are fixed points
+    for c, m in enumerate(E2M1_MAGNITUDES):
+        assert orc.e2m1_encode([m])[0] == c
+        assert orc.e2m1_encode([-m])[0] == c | 8
+    # midpoints go to the neighbour whose code is even (mantissa bit 0)
+    mids = {0.25: 0.0, 0.75: 1.0, 1.25: 1.0, 1.75: 2.0, 2.5: 2.0, 3.5: 4.0, 5.0: 4.0}
+    for x, want in mids.items():
+        assert orc.e2m1_decode(orc.e2m1_encode([x]))[0] == want
+        assert orc.e2m1_decode(orc.e2m1_encode([-x]))[0] == -want
+    # off-midpoint values go to the nearest; beyond 6 saturates
+    for x in (0.26, 0.74, 1.26, 2.49, 2.51, 4.9, 5.1, 6.0, 6.5, 1e6):
+        got = orc.e2m1_decode(orc.e2m1_encode([x]))[0]
+        near = min(E2M1_MAGNITUDES, key=lambda m: abs(m - min(x, 6.0)))
+        assert got == near, (x, got)
+    # monotone on a fine grid
+    grid = np.linspace(-7, 7, 2801)
+    dec = orc.e2m1_decode(orc.e2m1_encode(grid))
+    assert np.all(np.diff(dec) >= 0)
+
+
+def _pair_group(energies_as_values, signs=(1, 1, 1, 1), split=False):
+    """Eight bf16 values whose pair j carries the given value (as one element,
+    or split over both elements when split)."""
+    v = []
+    for j, x in enumerate(energies_as_values):
+        a = signs[j] * float(x)
+        v.extend([0.0, a] if split else [a, 0.0])
+    return bf16(np.array(v, np.float32))
+
+
+def test_pair_rule_brute_force_all_tie_patterns():
+    """Every ordering (with ties) of the four pair weights, against the rule
+    written as a stable sort: the two heaviest pairs, ties to the lower pair."""
+    for pattern in itertools.product(range(4), repeat=4):
+        for signs in ((1, 1, 1, 1), (-1, 1, -1, 1)):
+            for split in (False, True):
+                g = _pair_group(pattern, signs, split)
+                nib, p0, p1 = orc.prune_pairs8(g)
+                order = sorted(range(4), key=lambda j: (-pattern[j] ** 2, j))
+                want = sorted(order[:2])
+                assert [p0, p1] == want, (pattern, signs, split)
+                assert nib == want[0] | (want[1] << 2)
+
+
+def test_pair_rule_weighs_energy_not_the_largest_element():
+    # pair 0 holds the largest element (3) but less energy (9) than pairs 1
+    # and 2 (2.25^2 * 2 = 10.125 each): the energy reading drops it
+    g = bf16(np.array([3.0, 0.0, 2.25, 2.25, 2.25, 2.25, 0.5, 0.5], np.float32))
+    nib, p0, p1 = orc.prune_pairs8(g)
+    assert (p0, p1) == (1, 2)
+
+
+def test_pairwise_48_keeps_four_aligned_elements():
+    W = inputs.normal_bf16((64, 256), 1.0, seed=21)
+    P = orc.prune_pairs_bf16(W)
+    kept = (P != 0).reshape(64, 32, 4, 2)
+    # whole pairs only, two pairs per group of eight
+    assert np.all(kept[..., 0] == kept[..., 1])
+    assert np.all(kept[..., 0].sum(axis=2) == 2)
+    assert np.array_equal(P[P != 0], W[P != 0])
+
+
+def test_pairwise_48_energy_closed_form_on_gaussian_data():
+    """A pair of N(0,1) values has chi-square(2) energy, exponential with mean
+    2; dropping the lighter two of four drops 2/4 + (2/4 + 2/3) = 5/3 of the
+    group's expected 8, i.e. 5/24.  The pages put pairs at about one and a half
+    times the energy that element-wise 2:4 removes from Gaussian data."""
+    W = inputs.normal_bf16((2048, 1024), 1.0, seed=22)
+    _, _, _, e48 = orc.energy_loss_48(W)
+    _, _, _, e24 = orc.energy_loss(W)
+    assert abs(e48 - 5.0 / 24.0) < 2e-3
+    assert 1.4 < e48 / e24 < 1.7
+
+
+def test_energy_loss_48_brute_force_by_sorting():
+    W = inputs.normal_bf16((8, 64), 1.0, seed=23)
+    dropped, total, share, tensor = orc.energy_loss_48(W)
+    x = W.view(np.uint16).astype(np.uint32) << 16
+    xf = x.view(np.float32).astype(np.float64).reshape(8, 8, 4, 2)
+    e = (xf ** 2).sum(axis=3)                            # pair energies [rows, groups, 4]
+    drop = np.sort(e, axis=2)[:, :, :2].sum(axis=(1, 2))  # the two lightest pairs per group
+    assert np.allclose(dropped, drop, rtol=0, atol=1e-12)
+    assert np.allclose(total, (xf ** 2).sum(axis=(1, 2, 3)), rtol=0, atol=1e-12)
+
+
+def test_nvfp4_scales_closed_forms():
+    amax = np.float32(3.75)
+    st = orc.nvfp4_tensor_scale(float(amax))
+    assert np.float32(st) == amax / np.float32(2688.0)   # 448 * 6
+    assert orc.nvfp4_tensor_scale(0.0) == 1.0
+    # the tensor's own amax gets the largest block code, 448
+    b = orc.nvfp4_block_code(float(amax), st)
+    assert orc.e4m3_decode(np.array([b], np.uint8))[0] == 448.0
+    # the block's largest value lands on the E2M1 code of 6: the E4M3 scale is
+    # off by at most 1/16, so |v| / S stays within [5.6, 6.5]
+    g = np.random.default_rng(24)
+    for _ in range(200):
+        amax_b = np.float32(g.uniform(1e-3, 3.75))
+        bb = orc.nvfp4_block_code(float(amax_b), st)
+        assert orc.e2m1_decode(np.array([orc.nvfp4_code(float(amax_b), bb, st)]))[0] == 6.0
+    assert orc.nvfp4_block_code(0.0, st) == 0 and orc.nvfp4_code(1.0, 0, st) == 0
+
+
+def test_nvfp4_48_operand_round_trip_and_error_bound():
+    rows, K = 32, 256
+    W = inputs.normal_bf16((rows, K), 0.02, seed=25)
+    vals, meta, scales, st = orc.nvfp4_48_compress(W)
+    assert vals.shape == (rows, K // 4) and meta.shape == (rows, K // 16) and scales.shape == (rows, K // 32)
+    # metadata: the pair rule's nibbles, even group in the low nibble
+    for r in (0, 7, 31):
+        for grp in (0, 5, K // 8 - 1):
+            nib = orc.prune_pairs8(W[r, 8 * grp:8 * grp + 8])[0]
+            assert (meta[r, grp // 2] >> (4 * (grp % 2))) & 0xF == nib
+    P = orc.bf16_bits_to_f64(orc.prune_pairs_bf16(W))
+    D = orc.nvfp4_48_dequant(vals, meta, scales, st, rows, K)
+    assert np.all(D[P == 0] == 0)                        # nothing at the dropped positions
+    S = orc.e4m3_decode(scales).astype(np.float64) * st  # effective scale per 32 positions
+    Sfull = np.repeat(S, 32, axis=1)
+    # E2M1 gaps are at most 2 (between 4 and 6), so the error is at most one scale
+    assert np.all(np.abs(D - P) <= Sfull * (1.0 + 1e-12))
+    # storage: 4-bit codes for half the positions, a nibble per 8, a byte per 32
+    assert (vals.nbytes + meta.nbytes + scales.nbytes) * 8 / (rows * K) == 2.75
+
+
+def test_dense_nvfp4_costs_4_5_bits_and_bounds_error():
+    """Dense NVFP4 (E4M3 scale per 16 elements) costs 4.5 bits per element
+    before the per-tensor scale, the figure the pages use for it."""
+    rows, K = 16, 128
+    W = inputs.normal_bf16((rows, K), 0.02, seed=26)
+    codes, scales, st = orc.nvfp4_quantize(W)
+    assert (codes.nbytes + scales.nbytes) * 8 / (rows * K) == 4.5
+    D = orc.nvfp4_dequant(codes, scales, st, rows, K)
+    X = orc.bf16_bits_to_f64(W)
+    S = np.repeat(orc.e4m3_decode(scales).astype(np.float64) * st, 16, axis=1)
+    assert np.all(np.abs(D - X) <= S * (1.0 + 1e-12))
+    # every block's largest magnitude is represented by the E2M1 code of 6
+    c = np.stack([codes & 0xF, codes >> 4], axis=2).reshape(rows, K)
+    for r in range(rows):
+        for blk in range(K // 16):
+            i = np.argmax(np.abs(X[r, 16 * blk:16 * blk + 16]))
+            assert orc.e2m1_decode(np.array([c[r, 16 * blk + i]]))[0] in (6.0, -6.0)
