@@ -1,5 +1,6 @@
 /*
- * sp24_oracle.c -- CPU oracle for 2:4 semi-structured sparsity.
+ * sp24_oracle.c -- CPU oracle for 2:4 semi-structured sparsity (and, at the
+ * end, the pairwise 4:8 sparse NVFP4 format that comes next).
  *
  * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the
  * benchmark's CPU-baseline leg may load this file's library.  The CUDA
