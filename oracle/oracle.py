@@ -68,8 +68,8 @@ def lib() -> ctypes.CDLL:
             "orc_nvfp4_code": (ctypes.c_uint8, [ctypes.c_float, ctypes.c_uint8, ctypes.c_float]),
             "orc_nvfp4_48_compress": (None, [P, I64, I64, I64, P, P, P, P]),
             "orc_nvfp4_48_dequant": (None, [P, P, P, ctypes.c_float, I64, I64, P]),
-            "orc_nvfp4_quantize": (None, [P, I64, I64, I64, P, P, P]),
-            "orc_nvfp4_dequant": (None, [P, P, ctypes.c_float, I64, I64, P]),
+            "orc_nvfp4_quantize_blocks": (None, [P, I64, I64, I64, ctypes.c_int, P, P, P]),
+            "orc_nvfp4_dequant_blocks": (None, [P, P, ctypes.c_float, I64, I64, ctypes.c_int, P]),
             "orc_energy_loss_48": (None, [P, I64, I64, I64, P, P]),
         }
         for name, (res, args) in sig.items():
@@ -356,22 +356,24 @@ def nvfp4_48_dequant(values, meta, scales, tensor_scale: float, rows: int, K: in
     return out
 
 
-def nvfp4_quantize(W_bits: np.ndarray):
-    """Dense NVFP4: (codes [rows, K/2] packed, block scales [rows, K/16], tensor scale)."""
+def nvfp4_quantize(W_bits: np.ndarray, block: int = 16):
+    """Dense NVFP4: (codes [rows, K/2] packed, block scales [rows, K/block],
+    tensor scale).  block 16 is dense NVFP4; block 32 is the dense operand of
+    the sparse block-scaled GEMM (one scale per 32 positions of K)."""
     W = np.ascontiguousarray(W_bits, dtype=np.uint16)
     rows, K = W.shape
-    assert K % 16 == 0
+    assert K % block == 0
     codes = np.empty((rows, K // 2), np.uint8)
-    scales = np.empty((rows, K // 16), np.uint8)
+    scales = np.empty((rows, K // block), np.uint8)
     st = ctypes.c_float()
-    lib().orc_nvfp4_quantize(_p(W), rows, K, K, _p(codes), _p(scales), ctypes.byref(st))
+    lib().orc_nvfp4_quantize_blocks(_p(W), rows, K, K, block, _p(codes), _p(scales), ctypes.byref(st))
     return codes, scales, float(st.value)
 
 
-def nvfp4_dequant(codes, scales, tensor_scale: float, rows: int, K: int) -> np.ndarray:
+def nvfp4_dequant(codes, scales, tensor_scale: float, rows: int, K: int, block: int = 16) -> np.ndarray:
     out = np.empty((rows, K), np.float64)
-    lib().orc_nvfp4_dequant(_p(np.ascontiguousarray(codes)), _p(np.ascontiguousarray(scales)),
-                            ctypes.c_float(tensor_scale), rows, K, _p(out))
+    lib().orc_nvfp4_dequant_blocks(_p(np.ascontiguousarray(codes)), _p(np.ascontiguousarray(scales)),
+                                   ctypes.c_float(tensor_scale), rows, K, block, _p(out))
     return out
 
 

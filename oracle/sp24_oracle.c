@@ -706,11 +706,13 @@ void orc_nvfp4_48_dequant(const uint8_t *values, const uint8_t *meta, const uint
     }
 }
 
-/* Dense NVFP4 (the dense side at the same floor): one E4M3 block code per
- * 16 elements along K, the tensor scale from the whole matrix (R15).
- *   codes: [rows x K/2] bytes, two E2M1 codes per byte; scales: [rows x K/16]. */
-void orc_nvfp4_quantize(const uint16_t *src, int64_t rows, int64_t K, int64_t ld,
-                        uint8_t *codes, uint8_t *scales, float *tensor_scale)
+/* Dense NVFP4 with one E4M3 block code per `block` elements along K (16: the
+ * dense NVFP4 operand; 32: the dense operand of the sparse block-scaled GEMM,
+ * which carries one scale per 32 positions of the reduction axis), the tensor
+ * scale from the whole matrix (R15).  K % block == 0.
+ *   codes: [rows x K/2] bytes, two E2M1 codes per byte; scales: [rows x K/block]. */
+void orc_nvfp4_quantize_blocks(const uint16_t *src, int64_t rows, int64_t K, int64_t ld, int block,
+                               uint8_t *codes, uint8_t *scales, float *tensor_scale)
 {
     float amax_t = 0.0f;
     for (int64_t r = 0; r < rows; ++r)
@@ -722,28 +724,28 @@ void orc_nvfp4_quantize(const uint16_t *src, int64_t rows, int64_t K, int64_t ld
     *tensor_scale = s_t;
     memset(codes, 0, (size_t)(rows * (K / 2)));
     for (int64_t r = 0; r < rows; ++r)
-        for (int64_t blk = 0; blk < K / 16; ++blk) {
+        for (int64_t blk = 0; blk < K / block; ++blk) {
             float amax_b = 0.0f;
-            for (int i = 0; i < 16; ++i) {
-                float a = fabsf(bf16_to_float(src[r * ld + 16 * blk + i]));
+            for (int i = 0; i < block; ++i) {
+                float a = fabsf(bf16_to_float(src[r * ld + block * blk + i]));
                 if (a > amax_b) amax_b = a;
             }
             const uint8_t b = orc_nvfp4_block_code(amax_b, s_t);
-            scales[r * (K / 16) + blk] = b;
-            for (int i = 0; i < 16; ++i)
-                put_nibble(codes + r * (K / 2), 16 * blk + i,
-                           orc_nvfp4_code(bf16_to_float(src[r * ld + 16 * blk + i]), b, s_t));
+            scales[r * (K / block) + blk] = b;
+            for (int i = 0; i < block; ++i)
+                put_nibble(codes + r * (K / 2), block * blk + i,
+                           orc_nvfp4_code(bf16_to_float(src[r * ld + block * blk + i]), b, s_t));
         }
 }
 
 /* The dequantized matrix of a dense NVFP4 operand (fp64, [rows x K]). */
-void orc_nvfp4_dequant(const uint8_t *codes, const uint8_t *scales, float tensor_scale,
-                       int64_t rows, int64_t K, double *out)
+void orc_nvfp4_dequant_blocks(const uint8_t *codes, const uint8_t *scales, float tensor_scale,
+                              int64_t rows, int64_t K, int block, double *out)
 {
     for (int64_t r = 0; r < rows; ++r)
         for (int64_t k = 0; k < K; ++k)
             out[r * K + k] = orc_e2m1_decode(get_nibble(codes + r * (K / 2), k)) *
-                             orc_e4m3_decode(scales[r * (K / 16) + k / 16]) * (double)tensor_scale;
+                             orc_e4m3_decode(scales[r * (K / block) + k / block]) * (double)tensor_scale;
 }
 
 /* 4:8 pairwise energy loss per row, as orc_energy_loss for 2:4: the energy

@@ -552,3 +552,31 @@ def test_dense_nvfp4_costs_4_5_bits_and_bounds_error():
         for blk in range(K // 16):
             i = np.argmax(np.abs(X[r, 16 * blk:16 * blk + 16]))
             assert orc.e2m1_decode(np.array([c[r, 16 * blk + i]]))[0] in (6.0, -6.0)
+
+
+def test_nvfp4_32_blocks_for_the_sparse_gemms_dense_operand():
+    """The dense operand of the sparse block-scaled GEMM carries one scale per
+    32 positions of K: 4.25 bits per element, the same codes as 16-element
+    blocks wherever both blocks of 16 share the larger block's scale, and
+    the same error bound."""
+    rows, K = 8, 256
+    X = inputs.normal_bf16((rows, K), 1.0, seed=27)
+    c32, s32, st = orc.nvfp4_quantize(X, block=32)
+    assert s32.shape == (rows, K // 32) and (c32.nbytes + s32.nbytes) * 8 / (rows * K) == 4.25
+    D = orc.nvfp4_dequant(c32, s32, st, rows, K, block=32)
+    S = np.repeat(orc.e4m3_decode(s32).astype(np.float64) * st, 32, axis=1)
+    assert np.all(np.abs(D - orc.bf16_bits_to_f64(X)) <= S * (1.0 + 1e-12))
+    # a 32-block's scale equals the 16-block scale of whichever half holds its amax
+    c16, s16, st16 = orc.nvfp4_quantize(X, block=16)
+    assert st16 == st
+    assert np.array_equal(s32, np.maximum(s16[:, 0::2], s16[:, 1::2]))
+    # the sparse GEMM in the oracle is the fp64 product of the dequantized operands;
+    # with a 4:8 weight whose pruned entries the product never sees
+    W = inputs.normal_bf16((16, K), 0.02, seed=28)
+    v, m, sw, stw = orc.nvfp4_48_compress(W)
+    Wd = orc.nvfp4_48_dequant(v, m, sw, stw, 16, K)
+    Y, A = orc.gemm_f64(D, Wd)
+    P = orc.prune_pairs_bf16(W) != 0
+    Y2 = np.array([[np.sum(D[i][P[j]] * Wd[j][P[j]]) for j in range(16)] for i in range(rows)])
+    assert np.allclose(Y, Y2, rtol=1e-12, atol=1e-15)
+
