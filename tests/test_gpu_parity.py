@@ -443,7 +443,7 @@ def _pair_mask(kind, N, K, seed):
         m = np.zeros((RB, KT), np.uint8)
         m[1::2, :] = 1
         return m
-    if kind == "checker":      # mixed, dense-first and dense-second K-steps interleaved
+    if kind == "checkerboard":  # mixed, dense-first and dense-second K-steps interleaved
         return ((np.arange(RB)[:, None] + np.arange(KT)[None, :]) % 2).astype(np.uint8)
     raise ValueError(kind)
 
@@ -456,7 +456,7 @@ HYBRID_PAIR_SHAPES = [
 
 
 @pytest.mark.parametrize("M,N,K", HYBRID_PAIR_SHAPES)
-@pytest.mark.parametrize("kind", ["random", "all_dense", "all_sparse", "odd_blocks", "checker"])
+@pytest.mark.parametrize("kind", ["random", "all_dense", "all_sparse", "odd_blocks", "checkerboard"])
 def test_hybrid_gemm_pair_parity(M, N, K, kind):
     """Hybrid weights on CTA pairs (forced: these shapes have fewer tiles than
     the device has pairs), where a K-step runs dense when either half of the
