@@ -580,3 +580,35 @@ def test_nvfp4_32_blocks_for_the_sparse_gemms_dense_operand():
     Y2 = np.array([[np.sum(D[i][P[j]] * Wd[j][P[j]]) for j in range(16)] for i in range(rows)])
     assert np.allclose(Y, Y2, rtol=1e-12, atol=1e-15)
 
+
+
+def test_nvfp4_48_packing_and_kept_value_scales():
+    """R16/R17 by hand on one row of 32 positions: the kept values in ascending
+    position, two codes per byte (earlier element low), one nibble per group of
+    eight, and scales from the kept values only."""
+    # heavy pairs (1, 3) in groups 0 and 2, (0, 2) in groups 1 and 3, light
+    # pairs elsewhere; then an 8.0 makes pair 0 the heaviest of group 0
+    row = np.zeros(32, np.float32)
+    for g in range(4):
+        kept = (1, 3) if g % 2 == 0 else (0, 2)
+        for p in range(4):
+            a, b = 8 * g + 2 * p, 8 * g + 2 * p + 1
+            if p in kept:
+                row[a], row[b] = 2.0 + p, -(1.0 + p)
+            else:
+                row[a], row[b] = 0.25, 0.125
+    row[0] = 8.0   # pair 0 of group 0: energy 64 + 1/64, above pair 1 (13) and pair 3 (41): pairs (0, 3) kept
+    W = bf16(row[None, :])
+    vals, meta, scales, st = orc.nvfp4_48_compress(W)
+    nibs = [(meta[0, g // 2] >> (4 * (g % 2))) & 0xF for g in range(4)]
+    assert nibs == [0 | (3 << 2), 0 | (2 << 2), 1 | (3 << 2), 0 | (2 << 2)]
+    kept_vals = []
+    for g, nib in enumerate(nibs):
+        p0, p1 = nib & 3, nib >> 2
+        kept_vals += [row[8 * g + 2 * p0], row[8 * g + 2 * p0 + 1], row[8 * g + 2 * p1], row[8 * g + 2 * p1 + 1]]
+    amax = max(abs(v) for v in kept_vals)
+    assert np.float32(st) == np.float32(amax) / np.float32(2688.0)
+    codes = [(vals[0, i // 2] >> (4 * (i % 2))) & 0xF for i in range(16)]
+    b = int(scales[0, 0])
+    assert codes == [orc.nvfp4_code(float(v), b, st) for v in kept_vals]
+    assert b == orc.nvfp4_block_code(float(amax), st)
