@@ -18,7 +18,12 @@
  *
  * Conventions for every call:
  *  - Pointers named *_dev are DEVICE pointers; the caller allocates and frees
- *    every buffer.  The library allocates nothing on the device.
+ *    every buffer it passes.  The library's own device memory is limited to
+ *    two documented items: the fixed scratch array of sp24_gemm_noalloc (a
+ *    static array, held by every GPU that loads the library), and the L2
+ *    flush buffer of sp24_select_tactic (twice the L2 size, allocated on the
+ *    selector's first call on a device and kept until exit).  No other call
+ *    allocates device memory.
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *    stream).  Every call is asynchronous on that stream unless stated.
  *  - Argument errors are returned synchronously, before any launch.  A failed
@@ -252,8 +257,10 @@ int sp24_gemm(const sp24_gemm_args *args, void *stream);
  * problems).  Same results as sp24_gemm on each.  The work of all problems
  * is scheduled together, so the weights of the whole group stream without a
  * launch, ramp or tail between problems.  All problems must share in_dtype,
- * out_dtype and tactic, use no hybrid mask, and have M in the same class
- * (1-16, 17-32, 33-64, >64); otherwise SP24_ERR_INVALID_ARG.  Each args'
+ * out_dtype and tactic, either all carry a hybrid tile mask or none does, and
+ * have M in the same class (1-16, 17-32, 33-64, >64); otherwise
+ * SP24_ERR_INVALID_ARG.  Hybrid problems run 128-row tiles on single CTAs
+ * (each 128-deep K-step dense or sparse as its tile's flag says).  Each args'
  * own workspace fields are ignored: the group uses `workspace` (size from
  * sp24_gemm_grouped_workspace_bytes, same zero-fill rule as sp24_gemm).
  * SP24_GEMM_W_STATIC applies when every problem sets it. */
@@ -282,11 +289,15 @@ size_t sp24_gemm_grouped_workspace_bytes(const sp24_gemm_args *args, int n);
  *  - The first call on each device looks up the array's device address (with
  *    that device current) and caches it; make that first call before any
  *    stream capture.
- *  - Shapes whose schedule needs more than sp24_gemm_noalloc_max_scratch_bytes()
- *    of scratch return SP24_ERR_WORKSPACE.
- *  - Every call clears the part of the array it uses (a memset on `stream`)
- *    and shares the same array: calls that overlap on the GPU race with each
- *    other (on one device, issue them on one stream or order them). */
+ *  - The schedule is the one sp24_gemm picks when given a workspace of
+ *    sp24_gemm_noalloc_max_scratch_bytes(): a shape whose stream-K schedule
+ *    would need more scratch than that runs whole tiles per CTA (no scratch),
+ *    and shapes on the CTA-pair kernel (M, N >= 256) use none.  A plan that
+ *    still needed more than the array would return SP24_ERR_WORKSPACE.
+ *  - A call whose schedule uses scratch clears the part of the array that
+ *    must start at zero (a memset on `stream`); every call shares the same
+ *    array, so calls that overlap on the GPU race with each other (on one
+ *    device, issue them on one stream or order them). */
 int sp24_gemm_noalloc(const sp24_gemm_args *args, void *stream);
 
 /* Size of the fixed scratch array sp24_gemm_noalloc draws on. */

@@ -249,6 +249,9 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* last_flag = reinterpret_cast<int*>(tmem_slot + 2);
+  // hybrid: the kind of each stage in flight (1 = dense), producer -> MMA
+  // thread, published by the stage barrier's arrive
+  volatile uint8_t* s_kind = reinterpret_cast<volatile uint8_t*>(tmem_slot + 3);
   float* s_scale_b = reinterpret_cast<float*>(smem + C::kScaleOffset);
   uint8_t* s_epi = smem + C::kEpiOffset;
 
@@ -293,15 +296,122 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
   tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
 
-  auto is_dense_tile = [&](const GemmProblem& P, int ta, int kt) -> bool {
-    return P.tile_mask[(int64_t)ta * P.num_kt + kt] != 0;
-  };
   // metadata chunks (128 K positions each) of stage kt of problem P
   auto meta_chunks = [&](const GemmProblem& P, int kt) -> int {
     return (int)min((int64_t)C::kMetaChunks, (int64_t)(P.K / 128) - (int64_t)kt * C::kMetaChunks);
   };
 
-  if (warp == 0) {
+  if (warp == 0 && C::kHybrid) {
+    // ------------------------------------------------------------------ hybrid producer
+    // The whole warp walks the segments.  Every 32 K-stages of a segment the
+    // lanes read the next 32 dense flags of the tile in parallel (one ballot),
+    // so a flag costs no dependent global load per stage; lane 0 issues the
+    // copies and publishes each stage's kind to the MMA thread in s_kind
+    // before arming the stage's barrier (the arrive releases it).
+    const uint64_t pol_stream = policy_evict_first();
+    const uint64_t pol_keep = policy_evict_last();
+    constexpr uint32_t kDenseTx = (uint32_t)(C::kABytes + kBN * 128);
+    constexpr uint32_t kSparseTx = (uint32_t)(kBlockA * 64 + kBN * 128 + 2048);
+    int armed[S];
+    for (int s = 0; s < S; ++s) armed[s] = -1;
+    auto flag_word = [&](const GemmProblem& P, int ta, int k0, int ke) -> uint32_t {
+      const int k = k0 + lane;
+      const bool d = k < ke && P.tile_mask[(int64_t)ta * P.num_kt + k] != 0;
+      return __ballot_sync(0xFFFFFFFFu, d);
+    };
+    auto load_a = [&](int stage, const GemmProblem& P, int pr, int ta, int kt, bool dense) {
+      const uint32_t sa = smem_u32(smem + stage * C::kStageBytes);
+      const int32_t ya = ta * kBlockA;
+      if (dense) {
+        tma_load_2d(sa, &g.tm_a[pr], full_bar(stage), kt * 128, ya, pol_stream);
+      } else {
+        tma_load_2d(sa, &g.tm_a2[pr], full_bar(stage), kt * 64, ya, pol_stream);
+        bulk_load(sa + C::kABytes + C::kBBytes, P.meta + ((int64_t)ta * P.num_kt + kt) * 2048, 2048,
+                  full_bar(stage), pol_stream);
+      }
+    };
+    auto arm = [&](int stage, bool dense, int ph) {
+      s_kind[stage] = dense ? 1 : 0;
+      mbar_arrive_expect_tx(full_bar(stage), dense ? kDenseTx : kSparseTx);
+      armed[stage] = ph;
+    };
+    // 1. static weights: the first S stages' A copies before the dependency wait
+    int pre = 0;
+    if (p.w_static) {
+      SegIter<kMaxProb> it;
+      it.init(g, unit, units);
+      int pr, tile, kb, ke, seg;
+      while (pre < S && it.next(g, units, pr, tile, kb, ke, seg)) {
+        const GemmProblem& P = g.prob[pr];
+        const int ta = tile % P.tiles_a;
+        const int take = min(ke - kb, S - pre);  // <= S <= 8 stages: one flag word
+        const uint32_t fl = flag_word(P, ta, kb, kb + take);
+        if (lane == 0) {
+          tma_prefetch_desc(&g.tm_a[pr]);
+          tma_prefetch_desc(&g.tm_a2[pr]);
+          for (int i = 0; i < take; ++i) {
+            const bool dense = (fl >> i) & 1u;
+            arm(pre + i, dense, 0);
+            load_a(pre + i, P, pr, ta, kb + i, dense);
+          }
+        }
+        pre += take;
+      }
+    }
+    if (wait_first) {
+      pdl_wait();
+      pdl_launch_dependents();
+    }
+    // 2. the main stream
+    int stage = 0;
+    uint32_t phase = 0;
+    int n = 0;
+    bool ok = true;
+    SegIter<kMaxProb> it;
+    it.init(g, unit, units);
+    int pr, tile, kb, ke, seg;
+    while (ok && it.next(g, units, pr, tile, kb, ke, seg)) {
+      const GemmProblem& P = g.prob[pr];
+      const int ta = tile % P.tiles_a, tb = tile / P.tiles_a;
+      if (lane == 0) {
+        tma_prefetch_desc(&g.tm_a[pr]);
+        tma_prefetch_desc(&g.tm_a2[pr]);
+        tma_prefetch_desc(&g.tm_b[pr]);
+      }
+      uint32_t fl = 0;
+      for (int kt = kb; kt < ke; ++kt) {
+        if (((kt - kb) & 31) == 0) fl = flag_word(P, ta, kt, ke);
+        if (lane == 0) {
+          const bool dense = (fl >> ((kt - kb) & 31)) & 1u;
+          if (n >= pre) {
+            if (!mbar_wait(empty_bar(stage), phase ^ 1, p.timeout_ns, kDevErrWaitEmpty)) {
+              ok = false;
+              *abort_flag = 1;
+            } else {
+              arm(stage, dense, (int)phase);
+              load_a(stage, P, pr, ta, kt, dense);
+            }
+          }
+          if (ok) {
+            tma_load_2d(smem_u32(smem + stage * C::kStageBytes) + C::kABytes, &g.tm_b[pr], full_bar(stage),
+                        kt * 128, tb * kBN, pol_keep);
+            ++n;
+            if (++stage == S) {
+              stage = 0;
+              phase ^= 1;
+            }
+          }
+        }
+        ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
+        if (!ok) break;
+      }
+    }
+    // wait (bounded) until every copy counted on this CTA's barriers has landed
+    if (lane == 0)
+      for (int s = 0; s < S; ++s)
+        if (armed[s] >= 0) mbar_wait(full_bar(s), (uint32_t)armed[s], p.timeout_ns, kDevErrWaitFull);
+    __syncwarp();
+  } else if (warp == 0) {
     // ------------------------------------------------------------------ producer
     if (lane != 0 && wait_first) {
       pdl_wait();
@@ -325,15 +435,7 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
         const uint32_t sa = smem_u32(smem + stage * C::kStageBytes);
         const uint32_t sm = sa + C::kABytes + C::kBBytes;
         const int32_t ya = ta * C::kRowsA + (int32_t)rank * kBlockA;
-        if (C::kHybrid) {
-          if (is_dense_tile(P, ta, kt)) {
-            tma_load_2d(sa, &g.tm_a[pr], full_bar(stage), kt * 128, ya, pol_stream);
-          } else {
-            tma_load_2d(sa, &g.tm_a2[pr], full_bar(stage), kt * 64, ya, pol_stream);
-            bulk_load(sm, P.meta + ((int64_t)ta * P.num_kt + kt) * 2048, 2048, full_bar(stage),
-                      pol_stream);
-          }
-        } else {
+        {
           const int ax = C::kSparse ? kt * (C::kKT / 2) : kt * C::kKT;  // elements
           load2d(sa, &g.tm_a[pr], stage, ax, ya, pol_stream);
           if (C::kSparse) {
@@ -355,9 +457,7 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
       auto load_b = [&](int stage, int pr, int tb, int kt) {
         const uint32_t sb = smem_u32(smem + stage * C::kStageBytes) + C::kABytes;
         const int32_t yb = tb * kBN + (int32_t)rank * C::kBRows;
-        if (C::kHybrid) {
-          tma_load_2d(sb, &g.tm_b[pr], full_bar(stage), kt * 128, yb, pol_keep);
-        } else {
+        {
           const int box_elems = kBf16 ? 64 : 128;
 #pragma unroll
           for (int bx = 0; bx < C::kBBoxes; ++bx)
@@ -367,9 +467,6 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
       // bytes that complete one stage (both CTAs' halves in a pair)
       auto stage_bytes = [&](int pr, int ta, int kt) -> uint32_t {
         const GemmProblem& P = g.prob[pr];
-        if (C::kHybrid)
-          return is_dense_tile(P, ta, kt) ? (uint32_t)(C::kABytes + kBN * 128)
-                                          : (uint32_t)(kBlockA * 64 + kBN * 128 + 2048);
         if (kPair) return 2u * (uint32_t)C::kStageBytes;  // metadata boxes are always whole
         uint32_t b = C::kABytes + C::kBBytes;
         if (C::kSparse) b += (uint32_t)meta_chunks(P, kt) * 2048;
@@ -393,7 +490,7 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
         while (pre < S && it.next(g, units, pr, tile, kb, ke, seg)) {
           if (pr != last_pr) {
             tma_prefetch_desc(&g.tm_a[pr]);
-            if (C::kHybrid || (kPair && C::kSparse)) tma_prefetch_desc(&g.tm_a2[pr]);
+            if (kPair && C::kSparse) tma_prefetch_desc(&g.tm_a2[pr]);
             last_pr = pr;
           }
           const int ta = tile % g.prob[pr].tiles_a;
@@ -421,7 +518,7 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
         if (pr != last_pr) {
           tma_prefetch_desc(&g.tm_a[pr]);
           tma_prefetch_desc(&g.tm_b[pr]);
-          if (C::kHybrid || (kPair && C::kSparse)) tma_prefetch_desc(&g.tm_a2[pr]);
+          if (kPair && C::kSparse) tma_prefetch_desc(&g.tm_a2[pr]);
           last_pr = pr;
         }
         const int ta = tile % g.prob[pr].tiles_a, tb = tile / g.prob[pr].tiles_a;
@@ -476,7 +573,6 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
       int pr, tile, kb, ke, seg;
       while (ok && it.next(g, units, pr, tile, kb, ke, seg)) {
         const GemmProblem& P = g.prob[pr];
-        const int ta = tile % P.tiles_a;
         const int buf = acc_i & 1;
         const uint32_t acc_phase = (acc_i >> 1) & 1;
         if (!mbar_wait(acce_bar(buf), acc_phase ^ 1, p.timeout_ns, kDevErrWaitAccEmpty)) {
@@ -499,7 +595,7 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
           const uint32_t mcol = meta_col0 + stage * C::kMetaCols;
           const bool first = kt == kb;
           if (C::kHybrid) {
-            if (is_dense_tile(P, ta, kt)) {
+            if (s_kind[stage] != 0) {
 #pragma unroll
               for (int j = 0; j < 4; ++j) {
                 const uint64_t da = smem_desc(sa + j * 32, 16, 1024, kLayoutSw128);

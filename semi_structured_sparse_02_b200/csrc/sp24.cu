@@ -353,6 +353,8 @@ int dispatch_gemm_group(const Plan& pl, const GemmLaunch<kMaxGroup>& gl, cudaStr
   if (pl.mode == kModeDense)
     return pl.bf16 ? launch_gemm_bn<kModeDense, true, true, kMaxGroup>(pl.bn, gl, pl.grid, s)
                    : launch_gemm_bn<kModeDense, false, true, kMaxGroup>(pl.bn, gl, pl.grid, s);
+  if (pl.mode == kModeHybrid && !pl.bf16)
+    return launch_gemm_bn<kModeHybrid, false, true, kMaxGroup>(pl.bn, gl, pl.grid, s);
   return SP24_ERR_DTYPE;
 }
 
@@ -824,7 +826,8 @@ int validate_group(const sp24_gemm_args* a, int n) {
   for (int i = 0; i < n; ++i) {
     int st = validate_gemm(&a[i]);
     if (st != SP24_OK) return st;
-    if (a[i].tile_dense_mask != nullptr) return SP24_ERR_INVALID_ARG;
+    // hybrid weights group with hybrid weights only (one kernel mode per launch)
+    if ((a[i].tile_dense_mask != nullptr) != (a[0].tile_dense_mask != nullptr)) return SP24_ERR_INVALID_ARG;
     if (a[i].in_dtype != a[0].in_dtype || a[i].out_dtype != a[0].out_dtype ||
         a[i].tactic != a[0].tactic || pick_bn(a[i].M) != pick_bn(a[0].M))
       return SP24_ERR_INVALID_ARG;
@@ -1155,15 +1158,18 @@ int sp24_gemm_noalloc(const sp24_gemm_args* a, void* stream) {
   if (st != SP24_OK) return st;
   DeviceInfo di;
   if ((st = current_device_info(&di)) != SP24_OK) return st;
-  // The same schedule sp24_gemm picks with an unlimited workspace.
-  const Plan pl = plan_gemm(a, di, (size_t)-1);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // the CTA-pair kernel takes no scratch at all
+  if (args_use_pair(a)) return run_gemm(a, s);
+  // The schedule sp24_gemm picks with a workspace as large as the array:
+  // stream-K only where its scratch fits, whole tiles otherwise.
+  const Plan pl = plan_gemm(a, di, kStaticScratchBytes);
   if (pl.ws_bytes > kStaticScratchBytes) return SP24_ERR_WORKSPACE;
   void* scratch = nullptr;
   if ((st = static_scratch(&scratch)) != SP24_OK) return st;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   // the flags and counters must start at zero; the array keeps whatever
   // the previous call on this device left in it
-  if (pl.ws_bytes > 0 && cudaMemsetAsync(scratch, 0, sk_state_bytes(pl), s) != cudaSuccess) {
+  if (pl.sched == kSchedStreamK && cudaMemsetAsync(scratch, 0, sk_state_bytes(pl), s) != cudaSuccess) {
     cudaGetLastError();
     return SP24_ERR_CUDA;
   }

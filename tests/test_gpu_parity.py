@@ -431,6 +431,55 @@ def test_hybrid_gemm_parity(M):
     check_tolerance(y, y_ref, a_ref, "hybrid")
 
 
+# Grouped launches of hybrid weights (one-CTA tiles): a token-count class of
+# qkv / o / gate_up / down-like shapes.  K = 5120 gives 40 K-steps per tile, so
+# a segment spans more than one 32-step word of dense flags.
+HYBRID_GROUPS = {
+    "decode": [(1, 768, 512), (16, 512, 1024), (5, 1536, 512), (9, 256, 5120)],
+    "m128": [(256, 768, 512), (200, 512, 1536), (70, 384, 5120)],
+}
+
+
+def _group_mask(kind, N, K, seed):
+    RB, KT = N // 128, K // 128
+    if kind == "random":
+        return inputs.hybrid_mask(N, K, seed=seed)
+    if kind == "all_dense":
+        return np.ones((RB, KT), np.uint8)
+    return ((np.arange(RB)[:, None] + np.arange(KT)[None, :]) % 2).astype(np.uint8)
+
+
+@pytest.mark.parametrize("group", sorted(HYBRID_GROUPS))
+@pytest.mark.parametrize("use_ws", [True, False])
+@pytest.mark.parametrize("kind", ["random", "all_dense", "checkerboard"])
+def test_grouped_hybrid_gemm_parity(group, use_ws, kind):
+    shapes = HYBRID_GROUPS[group]
+    items = []
+    for i, (M, N, K) in enumerate(shapes):
+        X, W = inputs.linear_pair(M, N, K, seed=17 * i + M + K, outliers=True)
+        mask = _group_mask(kind, N, K, seed=i + M)
+        items.append(prepare_gemm(X, W, True, sp24.SPARSE, True, mask=mask, flags=sp24.GEMM_W_STATIC))
+    grp = sp24.GemmGroup([it[0] for it in items], allocate_workspace=use_ws)
+    if use_ws and group == "decode":
+        assert grp.ws_bytes > 0  # the stream-K schedule
+    for call in range(2):  # the second call reuses the workspace the first left zeroed
+        for it in items:
+            it[1].fill_(float("nan"))
+        grp()
+        torch.cuda.synchronize()
+        assert sp24.last_device_error() == sp24.SP24_OK
+        check_group(items, "hybrid group %s ws=%s %s call %d" % (group, use_ws, kind, call))
+
+
+def test_grouped_rejects_mixed_hybrid_and_plain_weights():
+    X, W = inputs.linear_pair(8, 256, 512, seed=3)
+    plain = prepare_gemm(X, W, True, sp24.SPARSE, True)[0]
+    hyb = prepare_gemm(X, W, True, sp24.SPARSE, True, mask=inputs.hybrid_mask(256, 512, seed=1))[0]
+    arr = (sp24.GemmArgs * 2)(plain, hyb)
+    st = sp24.lib().sp24_gemm_grouped(arr, 2, None, 0, None)
+    assert st == sp24.SP24_ERR_INVALID_ARG
+
+
 def _pair_mask(kind, N, K, seed):
     RB, KT = N // 128, K // 128
     if kind == "random":
