@@ -71,6 +71,8 @@ def lib() -> ctypes.CDLL:
             "orc_nvfp4_quantize_blocks": (None, [P, I64, I64, I64, ctypes.c_int, P, P, P]),
             "orc_nvfp4_dequant_blocks": (None, [P, P, ctypes.c_float, I64, I64, ctypes.c_int, P]),
             "orc_energy_loss_48": (None, [P, I64, I64, I64, P, P]),
+            "orc_nvfp4_48_meta_image": (None, [P, I64, I64, P]),
+            "orc_nvfp4_scale_image": (None, [P, I64, I64, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -374,6 +376,26 @@ def nvfp4_dequant(codes, scales, tensor_scale: float, rows: int, K: int, block: 
     out = np.empty((rows, K), np.float64)
     lib().orc_nvfp4_dequant_blocks(_p(np.ascontiguousarray(codes)), _p(np.ascontiguousarray(scales)),
                                    ctypes.c_float(tensor_scale), rows, K, block, _p(out))
+    return out
+
+
+def nvfp4_48_meta_image(meta: np.ndarray, rows: int, K: int) -> np.ndarray:
+    """The 4:8 metadata image the block-scaled GEMM copies to tensor memory
+    (layout spec): 2048-byte chunks of 128 rows x 256 positions of K."""
+    assert K % 256 == 0
+    out = np.empty(((rows + 127) // 128) * (K // 256) * 2048, np.uint8)
+    lib().orc_nvfp4_48_meta_image(_p(np.ascontiguousarray(meta, dtype=np.uint8)), rows, K, _p(out))
+    return out
+
+
+def nvfp4_scale_image(scales: np.ndarray, rows: int) -> np.ndarray:
+    """The block-scale image (layout spec): 512-byte chunks of 128 rows x 4
+    consecutive scale blocks."""
+    sc = np.ascontiguousarray(scales, dtype=np.uint8)
+    nblk = sc.shape[1]
+    assert nblk % 4 == 0
+    out = np.empty(((rows + 127) // 128) * 128 * nblk, np.uint8)
+    lib().orc_nvfp4_scale_image(_p(sc), rows, nblk, _p(out))
     return out
 
 

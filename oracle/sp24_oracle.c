@@ -748,6 +748,46 @@ void orc_nvfp4_dequant_blocks(const uint8_t *codes, const uint8_t *scales, float
                              orc_e4m3_decode(scales[r * (K / block) + k / block]) * (double)tensor_scale;
 }
 
+/* Device images of the NVFP4 operands for the block-scaled tensor-core MMA
+ * (layout spec; parity pinned by layout spec and by the GPU GEMM that reads
+ * them through the tensor cores, as for the 2:4 metadata image).
+ *
+ * 4:8 metadata image: 2048-byte chunks, one per (128-row block rb, 256
+ * positions of K kc) at byte (rb * K/256 + kc) * 2048; image row L (16 bytes
+ * at 16 L) is row 128 rb + L's canonical metadata bytes [16 kc, 16 kc + 16)
+ * (32 group nibbles, the even group low); rows past the end hold 0x44 bytes
+ * (pairs 0 and 1 in every group).  K % 256 == 0. */
+void orc_nvfp4_48_meta_image(const uint8_t *meta, int64_t rows, int64_t K, uint8_t *image)
+{
+    int64_t RB = (rows + 127) / 128, KC = K / 256;
+    for (int64_t rb = 0; rb < RB; ++rb)
+        for (int64_t kc = 0; kc < KC; ++kc)
+            for (int L = 0; L < 128; ++L) {
+                uint8_t *dst = image + (rb * KC + kc) * 2048 + 16 * L;
+                int64_t r = rb * 128 + L;
+                for (int b = 0; b < 16; ++b)
+                    dst[b] = r < rows ? meta[r * (K / 16) + 16 * kc + b] : (uint8_t)0x44;
+            }
+}
+
+/* Scale image: 512-byte chunks, one per (128-row block rb, four consecutive
+ * scale blocks kq) at byte (rb * nblk/4 + kq) * 512; the code of row
+ * r = 128 rb + 32 q + l (0 <= l < 32), block 4 kq + j sits at byte
+ * 16 l + 4 q + j of the chunk; rows past the end hold 0.  nblk % 4 == 0. */
+void orc_nvfp4_scale_image(const uint8_t *scales, int64_t rows, int64_t nblk, uint8_t *image)
+{
+    int64_t RB = (rows + 127) / 128, KQ = nblk / 4;
+    for (int64_t rb = 0; rb < RB; ++rb)
+        for (int64_t kq = 0; kq < KQ; ++kq)
+            for (int q = 0; q < 4; ++q)
+                for (int l = 0; l < 32; ++l) {
+                    int64_t r = rb * 128 + 32 * q + l;
+                    for (int j = 0; j < 4; ++j)
+                        image[(rb * KQ + kq) * 512 + 16 * l + 4 * q + j] =
+                            r < rows ? scales[r * nblk + 4 * kq + j] : (uint8_t)0;
+                }
+}
+
 /* 4:8 pairwise energy loss per row, as orc_energy_loss for 2:4: the energy
  * of the values the pair rule drops and of the whole row (fp64). */
 void orc_energy_loss_48(const uint16_t *src, int64_t rows, int64_t K, int64_t ld,

@@ -612,3 +612,40 @@ def test_nvfp4_48_packing_and_kept_value_scales():
     b = int(scales[0, 0])
     assert codes == [orc.nvfp4_code(float(v), b, st) for v in kept_vals]
     assert b == orc.nvfp4_block_code(float(amax), st)
+
+
+# ---------------------------------------------------------------------------
+# NVFP4 device images (layout spec): pinned by hand-derived positions and by
+# being permutations of the canonical bytes plus fixed padding
+# ---------------------------------------------------------------------------
+
+def test_nvfp4_48_meta_image_positions_and_padding():
+    rows, K = 200, 512
+    g = np.random.default_rng(4)
+    meta = g.integers(0, 256, size=(rows, K // 16), dtype=np.uint8)
+    img = orc.nvfp4_48_meta_image(meta, rows, K)
+    assert img.size == 2 * (K // 256) * 2048
+    # row 5, positions 256..511 (chunk kc = 1): image row 5 of chunk (rb 0, kc 1)
+    assert bytes(img[1 * 2048 + 16 * 5: 1 * 2048 + 16 * 6]) == bytes(meta[5, 16:32])
+    # row 130 = block 1, image row 2, chunk (1, 0) at (1 * 2 + 0) * 2048
+    assert bytes(img[2 * 2048 + 32: 2 * 2048 + 48]) == bytes(meta[130, 0:16])
+    # rows past the end hold pairs 0 and 1 in every group
+    assert (img[2 * 2048 + 16 * 72: 3 * 2048] == 0x44).all()
+    # a permutation of the canonical bytes plus the padding
+    live = np.concatenate([img[(rb * 2 + kc) * 2048 + 16 * L:(rb * 2 + kc) * 2048 + 16 * L + 16]
+                           for rb in range(2) for L in range(128) if rb * 128 + L < rows for kc in range(2)])
+    assert sorted(live.tolist()) == sorted(meta.ravel().tolist())
+
+
+def test_nvfp4_scale_image_positions_and_padding():
+    rows, nblk = 150, 8
+    sc = np.random.default_rng(9).integers(1, 256, size=(rows, nblk), dtype=np.uint8)
+    img = orc.nvfp4_scale_image(sc, rows)
+    assert img.size == 256 * nblk
+    # row 37 = 32 * 1 + 5 (q 1, l 5) of block 0, scale block 6 (kq 1, j 2)
+    assert img[(0 * 2 + 1) * 512 + 16 * 5 + 4 * 1 + 2] == sc[37, 6]
+    # row 140 = block 1, 32 * 0 + 12, scale block 3 (kq 0, j 3)
+    assert img[(1 * 2 + 0) * 512 + 16 * 12 + 0 + 3] == sc[140, 3]
+    # rows 150..255 hold 0; the live bytes are a permutation of the codes
+    assert (img != 0).sum() == rows * nblk
+    assert sorted(img[img != 0].tolist()) == sorted(sc.ravel().tolist())
