@@ -692,6 +692,81 @@ def run_group_case(args):
                       "workspace_bytes": grp.ws_bytes}), flush=True)
 
 
+def run_other_case(args):
+    """prune:N,K,bf16|e4m3 -- the weight prune / compress of N x K;
+    act:M,N,K,bf16|e4m3 -- the online-activation path (prune of X every call,
+    then the sparse GEMM); nv:M,N,K,sparse|dense -- the NVFP4 GEMM (pairwise
+    4:8 or dense), X cast to NVFP4 once.  Eager calls, CUDA-event timing, L2
+    flushed before each call (for profiler captures)."""
+    import torch
+
+    from semi_structured_sparse_02_b200 import inputs, sp24
+    dev = torch.device("cuda", 0)
+    kind, rest = args.case.split(":", 1)
+    f = rest.split(",")
+    T = Timer(dev, args.steps, args.warmup, 0.0)
+    if kind == "prune":
+        N, K, e4 = int(f[0]), int(f[1]), (f[2] if len(f) > 2 else "bf16") == "e4m3"
+        W = _bf16_dev(inputs.normal_bf16((N, K), 0.02, seed=N + K), dev)
+        vals = torch.empty(N, K // 2, dtype=torch.uint8 if e4 else torch.bfloat16, device=dev)
+        meta = torch.empty(sp24.meta_bytes(N, K), dtype=torch.uint8, device=dev)
+        sc = torch.empty(N, dtype=torch.float32, device=dev) if e4 else None
+        t, _, _ = T.calls(lambda: sp24.prune_compress(W, sp24.E4M3 if e4 else sp24.BF16, vals, meta, row_scales=sc))
+        byts = 2 * N * K + N * K * (1 if e4 else 2) // 2 + N * K // 8
+        print(json.dumps({"case": args.case, "us_median": round(t, 3), "GBps": round(byts / t / 1e3, 1)}), flush=True)
+    elif kind == "act":
+        M, N, K, e4 = int(f[0]), int(f[1]), int(f[2]), (f[3] if len(f) > 3 else "bf16") == "e4m3"
+        X = _bf16_dev(inputs.student_t_bf16((M, K), 3.0, seed=4), dev)
+        W = _bf16_dev(inputs.normal_bf16((N, K), 0.02, seed=4), dev)
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        if e4:
+            Wq = torch.empty(N, K, dtype=torch.uint8, device=dev)
+            wsc = torch.empty(N, dtype=torch.float32, device=dev)
+            sp24.quantize_e4m3_rows(W, Wq, wsc)
+            ws = torch.empty(sp24.activations_e4m3_workspace_bytes(M, K), dtype=torch.uint8, device=dev)
+            fn = lambda: sp24.prune_compress_activations_fused_e4m3(X, Wq, wsc, Y, workspace=ws)  # noqa: E731
+        else:
+            ws = torch.empty(sp24.activations_workspace_bytes(M, K), dtype=torch.uint8, device=dev)
+            fn = lambda: sp24.prune_compress_activations_fused(X, W, Y, workspace=ws)  # noqa: E731
+        t, _, _ = T.calls(fn)
+        print(json.dumps({"case": args.case, "us_median": round(t, 3),
+                          "TFLOPS": round(2.0 * M * N * K / t / 1e6, 1)}), flush=True)
+    elif kind == "nv":
+        M, N, K = int(f[0]), int(f[1]), int(f[2])
+        sparse = (f[3] if len(f) > 3 else "sparse") == "sparse"
+        blk = 32 if sparse else 16
+        W = _bf16_dev(inputs.normal_bf16((N, K), 0.02, seed=N + K), dev)
+        X = _bf16_dev(inputs.normal_bf16((M, K), 1.0, seed=M), dev)
+        xc = torch.empty(M, K // 2, dtype=torch.uint8, device=dev)
+        xs = torch.empty(sp24.nvfp4_scales_bytes(M, K, blk), dtype=torch.uint8, device=dev)
+        xts = torch.empty(1, dtype=torch.float32, device=dev)
+        sp24.quantize_nvfp4(X, blk, xc, xs, xts)
+        wts = torch.empty(1, dtype=torch.float32, device=dev)
+        ws_ = torch.empty(sp24.nvfp4_scales_bytes(N, K, blk), dtype=torch.uint8, device=dev)
+        meta = None
+        if sparse:
+            wv = torch.empty(N, K // 4, dtype=torch.uint8, device=dev)
+            meta = torch.empty(sp24.nvfp4_48_meta_bytes(N, K), dtype=torch.uint8, device=dev)
+            sp24.prune_compress_nvfp4_48(W, wv, meta, ws_, wts)
+        else:
+            wv = torch.empty(N, K // 2, dtype=torch.uint8, device=dev)
+            sp24.quantize_nvfp4(W, 16, wv, ws_, wts)
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        a = sp24.nvfp4_gemm_args(xc, xs, xts, wv, ws_, wts, Y, K, sp24.SPARSE if sparse else sp24.DENSE, W_meta=meta)
+        n = sp24.gemm_nvfp4_workspace_bytes(a)
+        if n:
+            wsp = torch.zeros(n, dtype=torch.uint8, device=dev)
+            a.workspace, a.workspace_bytes = wsp.data_ptr(), n
+            a._keep.append(wsp)
+        t, _, _ = T.calls(lambda: sp24.gemm_nvfp4(a))
+        wbytes = N * K * (0.25 + 1 / 16 + 1 / 32) if sparse else N * K * (0.5 + 1 / 16)
+        byts = wbytes + M * K * (0.5 + 1 / blk) + 2 * M * N
+        print(json.dumps({"case": args.case, "us_median": round(t, 3), "GBps": round(byts / t / 1e3, 1),
+                          "TFLOPS": round(2.0 * M * N * K / t / 1e6, 1), "workspace_bytes": n}), flush=True)
+    else:
+        raise SystemExit("unknown case kind %r" % kind)
+
+
 def run_case(args):
     """One GEMM shape, eager calls, CUDA-event timing (for profiler captures)."""
     import torch
@@ -699,6 +774,9 @@ def run_case(args):
     from semi_structured_sparse_02_b200 import inputs, sp24
     if args.case.startswith("group:"):
         run_group_case(args)
+        return
+    if args.case.split(":", 1)[0] in ("prune", "act", "nv"):
+        run_other_case(args)
         return
     f = args.case.split(",")
     M, N, K = int(f[0]), int(f[1]), int(f[2])

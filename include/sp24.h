@@ -363,6 +363,89 @@ int sp24_energy_loss(const void *src_dev, int64_t rows, int64_t K, int64_t ld, d
                      double *sums_dev, void *stream);
 
 /* ---------------------------------------------------------------------- */
+/* Pairwise 4:8 sparse NVFP4 (the Blackwell sparse FP4 format)             */
+/* ---------------------------------------------------------------------- */
+/* NVFP4: E2M1 values (two per byte, the earlier element in the low nibble),
+ * one unsigned E4M3 scale per block of positions along K, one fp32 scale per
+ * tensor ("Quantization", section 2 of the 2:4-versus-quantization paper,
+ * paperpeel.com/paper/2610.28947).  The pairwise 4:8 pattern keeps two of the
+ * four adjacent pairs in every group of eight along K, and the sparse
+ * block-scaled GEMM carries one scale per 32 positions of K (section 6.2,
+ * "What pairwise 4:8 costs on Blackwell").
+ * Readings where the pages are silent: the two pairs of largest energy
+ * x0^2 + x1^2 survive (ties to the lower pair index); tensor scale
+ * s_t = amax / 2688 (1 for amax 0); block code b = E4M3(amax_b / (6 s_t));
+ * value code = E2M1(v / (decode(b) * s_t)), each step one correctly rounded
+ * fp32 operation, E2M1 rounding to nearest even and saturating at 6 (a zero
+ * block scale gives code 0); for the sparse operand both amaxes run over the
+ * kept values.
+ * Device layouts:
+ *  - sparse values [rows x K/4] bytes (kept elements in ascending position);
+ *    dense codes [rows x K/2] bytes;
+ *  - 4:8 metadata image: 2048-byte chunks, one per (128-row block rb, 256
+ *    positions kc) at (rb * K/256 + kc) * 2048; image row L (16 bytes at 16 L)
+ *    holds row 128 rb + L's 32 group nibbles p0 | p1 << 2 (p0 < p1 the kept
+ *    pairs) in order, the even group low; rows past the end hold 0x44;
+ *  - scale image: 512-byte chunks, one per (128-row block rb, four
+ *    consecutive scale blocks kq) at (rb * nblk/4 + kq) * 512, the code of row
+ *    128 rb + 32 q + l, block 4 kq + j at byte 16 l + 4 q + j; rows past the
+ *    end hold 0 (the order in which the tensor core reads scales from tensor
+ *    memory after a 32 x 128-bit, four-quarter copy). */
+
+size_t sp24_nvfp4_48_values_bytes(int64_t rows, int64_t K);      /* rows * K/4            */
+size_t sp24_nvfp4_48_meta_bytes(int64_t rows, int64_t K);        /* ceil(rows/128)*K/256*2048 */
+size_t sp24_nvfp4_codes_bytes(int64_t rows, int64_t K);          /* rows * K/2            */
+size_t sp24_nvfp4_scales_bytes(int64_t rows, int64_t K, int block); /* ceil(rows/128)*128*K/block */
+
+/* Pairwise 4:8 prune + NVFP4 cast of a bf16 matrix (weights, offline):
+ * values, metadata image, scale image (one code per 32 positions) and the
+ * tensor scale (device fp32; it holds the amax bits during the call).  Four
+ * stream-ordered steps on `stream`: zero the tensor scale, tensor amax of the
+ * kept values, prune + cast, amax -> scale.  Requirements: rows >= 1,
+ * K % 256 == 0, ld >= K, ld % 8 == 0, all pointers 16-byte aligned. */
+int sp24_prune_compress_nvfp4_48(const void *src_dev, int64_t rows, int64_t K, int64_t ld,
+                                 void *values_dev, void *meta_dev, void *scales_dev, float *tensor_scale_dev,
+                                 void *stream);
+
+/* Dense NVFP4 cast of a bf16 matrix with one scale per `block` positions
+ * (16: dense NVFP4; 32: the dense operand of the sparse 4:8 GEMM): codes,
+ * scale image and tensor scale, as above (amax over every value).
+ * Requirements: K % (4 * block) == 0, block in {16, 32}. */
+int sp24_quantize_nvfp4(const void *src_dev, int64_t rows, int64_t K, int64_t ld, int block,
+                        void *codes_dev, void *scales_dev, float *tensor_scale_dev, void *stream);
+
+typedef struct sp24_nvfp4_gemm_args {
+    int64_t M, N, K;          /* Y [M x N] = X [M x K] * W [N x K]^T           */
+    sp24_tactic tactic;       /* SPARSE: W pairwise 4:8; DENSE: W dense NVFP4 */
+    sp24_dtype out_dtype;     /* SP24_BF16 or SP24_F32                         */
+    const void *X;            /* device, NVFP4 codes [M x K/2] (contiguous)    */
+    const void *x_scales;     /* device, scale image of X: one code per 32
+                                 positions (SPARSE) or per 16 (DENSE)          */
+    const float *x_tensor_scale; /* device, 1 float                           */
+    const void *W;            /* device; SPARSE: values [N x K/4]; DENSE: codes [N x K/2] */
+    const void *W_meta;       /* device; SPARSE: 4:8 metadata image of W       */
+    const void *w_scales;     /* device, scale image of W (per 32 / per 16)    */
+    const float *w_tensor_scale; /* device, 1 float                           */
+    void *Y;                  /* device, [M x N] row pitch ldy                 */
+    int64_t ldy;
+    void *workspace;          /* stream-K workspace (as sp24_gemm) or NULL     */
+    size_t workspace_bytes;
+    uint32_t flags;           /* SP24_GEMM_W_STATIC, SP24_GEMM_AFTER_INDEPENDENT */
+} sp24_nvfp4_gemm_args;
+
+/* Workspace of sp24_gemm_nvfp4's stream-K schedule (0 if none), with the
+ * zero-fill rule of sp24_gemm_workspace_bytes. */
+size_t sp24_gemm_nvfp4_workspace_bytes(const sp24_nvfp4_gemm_args *args);
+
+/* Y = s_x * s_w * sum_k x[m,k] w[n,k] (block scales applied inside the
+ * block-scaled tensor-core MMA, fp32 accumulation in tensor memory; tensor
+ * scales in the epilogue).  SPARSE: tcgen05.mma.sp kind::mxf4nvf4 with the
+ * 4:8 metadata; DENSE: the same kind, dense.  One persistent launch (128-row
+ * weight tiles on single CTAs).  Requirements: K % 256 == 0, every pointer
+ * 16-byte aligned, ldy * out bytes % 16 == 0. */
+int sp24_gemm_nvfp4(const sp24_nvfp4_gemm_args *args, void *stream);
+
+/* ---------------------------------------------------------------------- */
 /* Tactic selection (kernel 5)                                             */
 /* ---------------------------------------------------------------------- */
 

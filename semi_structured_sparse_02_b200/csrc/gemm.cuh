@@ -45,7 +45,10 @@
 
 namespace sp24 {
 
-enum GemmMode : int { kModeDense = 0, kModeSparse = 1, kModeHybrid = 2 };
+// kModeNvSparse / kModeNvDense: block-scaled NVFP4 operands (kind::mxf4nvf4):
+// A pairwise 4:8 sparse (values, metadata image, scales per 32 positions) or
+// dense (scales per 16), B dense NVFP4, one fp32 tensor scale per operand.
+enum GemmMode : int { kModeDense = 0, kModeSparse = 1, kModeHybrid = 2, kModeNvSparse = 3, kModeNvDense = 4 };
 enum GemmSched : int { kSchedDataParallel = 0, kSchedStreamK = 1 };
 
 constexpr int kGemmThreads = 192;
@@ -63,8 +66,10 @@ struct GemmProblem {
   int64_t iter_begin;         // first global stream-K iteration of this problem
   const uint8_t* meta;        // metadata image of A (sparse / hybrid)
   const uint8_t* tile_mask;   // hybrid: [tiles_a x K/128]
-  const float* scale_a;       // per-A-row scale (E4M3) or null
-  const float* scale_b;       // per-B-row scale (E4M3) or null
+  const float* scale_a;       // per-A-row scale (E4M3), tensor scale (NVFP4) or null
+  const float* scale_b;       // per-B-row scale (E4M3), tensor scale (NVFP4) or null
+  const uint8_t* sfa;         // NVFP4: scale image of A
+  const uint8_t* sfb;         // NVFP4: scale image of B
   void* Y;
   int64_t ldy;
   unsigned int* ws_counters;  // stream-K arrival counters [tiles (x2 halves in a pair)]
@@ -89,7 +94,8 @@ struct GemmParams {
 template <int kMaxProb>
 struct GemmLaunch {
   CUtensorMap tm_a[kMaxProb];   // A: dense [rows_a x K] or values [rows_a x K/2]
-  CUtensorMap tm_a2[kMaxProb];  // hybrid: values map (64-byte swizzle)
+  CUtensorMap tm_a2[kMaxProb];  // hybrid: values map (64-byte boxes, 64-byte swizzle)
+  CUtensorMap tm_a3[kMaxProb];  // hybrid: values map (128-byte boxes, 128-byte swizzle)
   CUtensorMap tm_b[kMaxProb];   // B: [rows_b x K]
   GemmProblem prob[kMaxProb];
   GemmParams p;
@@ -102,22 +108,32 @@ template <int kMode, bool kBf16, int kBN, bool kPair = false>
 struct GemmCfg {
   static constexpr bool kSparse = kMode == kModeSparse;
   static constexpr bool kHybrid = kMode == kModeHybrid;
-  static_assert(!(kPair && kHybrid), "hybrid tiles run on single CTAs");
+  static constexpr bool kNvSparse = kMode == kModeNvSparse;
+  static constexpr bool kNv = kNvSparse || kMode == kModeNvDense;
+  static_assert(!(kPair && (kHybrid || kNv)), "hybrid and NVFP4 tiles run on single CTAs");
   static constexpr int kRowsA = kPair ? 2 * kBlockA : kBlockA;  // A rows per tile
   static constexpr int kBRows = kPair ? kBN / 2 : kBN;          // B rows per CTA
-  // logical K per stage
-  static constexpr int kKT = kHybrid ? 128 : (kSparse ? (kBf16 ? 128 : 256) : (kBf16 ? 64 : 128));
-  static constexpr int kABytes = kBlockA * 128;                 // A tile (dense or sparse)
-  static constexpr int kBBoxes = kSparse ? 2 : 1;               // 128-byte-wide B boxes
+  // logical K per stage (NVFP4: 128 bytes of A per row, four MMAs)
+  // (hybrid: two 128 x 128 tile columns per stage, each dense or sparse)
+  static constexpr int kKT = kNv ? (kNvSparse ? 512 : 256)
+                                 : kHybrid ? 256 : (kSparse ? (kBf16 ? 128 : 256) : (kBf16 ? 64 : 128));
+  // A tile (dense or sparse); hybrid: two 16 KB slots, one per tile column
+  static constexpr int kABytes = kBlockA * 128 * (kHybrid ? 2 : 1);
+  static constexpr int kBBoxes = (kSparse || kNvSparse || kHybrid) ? 2 : 1;  // 128-byte-wide B boxes
   static constexpr int kBBytes = kBRows * 128 * kBBoxes;
-  static constexpr int kMetaChunks = kSparse ? (kBf16 ? 1 : 2) : (kHybrid ? 1 : 0);
+  static constexpr int kMetaChunks = kSparse ? (kBf16 ? 1 : 2) : ((kHybrid || kNvSparse) ? 2 : 0);
   static constexpr int kMetaBytes = kMetaChunks * 2048;
-  static constexpr int kStageBytes = kABytes + kBBytes + kMetaBytes;
+  // NVFP4: four 512-byte scale chunks of A, then four of B (one per MMA)
+  static constexpr int kSfBytes = kNv ? 4096 : 0;
+  static constexpr int kSfChunkK = kNvSparse ? 128 : 64;        // logical K of one scale chunk
+  static constexpr int kStageBytes = kABytes + kBBytes + kMetaBytes + kSfBytes;
   static constexpr int kSmemBudget = 212 * 1024;
   static constexpr int kStagesRaw = kSmemBudget / kStageBytes;
   static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
   static_assert(kStages >= 2, "stage too large");
-  static constexpr int kMetaCols = kMetaChunks * 4;              // tensor-memory columns per stage
+  // tensor-memory columns per stage: metadata, then (NVFP4) 16 of A scales
+  // and 16 of B scales
+  static constexpr int kMetaCols = kMetaChunks * 4 + (kNv ? 32 : 0);
   static constexpr int kAccCols = 2 * kBN;
   static constexpr int kColsNeeded = kAccCols + kStages * kMetaCols;
   static constexpr int kTmemCols = kColsNeeded <= 32 ? 32 : kColsNeeded <= 64 ? 64 :
@@ -300,39 +316,70 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
   auto meta_chunks = [&](const GemmProblem& P, int kt) -> int {
     return (int)min((int64_t)C::kMetaChunks, (int64_t)(P.K / 128) - (int64_t)kt * C::kMetaChunks);
   };
+  // NVFP4: a last stage that covers only half of kKT (K % kKT == kKT / 2)
+  auto nv_half = [&](const GemmProblem& P, int kt) -> bool {
+    return (int64_t)P.K - (int64_t)kt * C::kKT < C::kKT;
+  };
 
   if (warp == 0 && C::kHybrid) {
     // ------------------------------------------------------------------ hybrid producer
-    // The whole warp walks the segments.  Every 32 K-stages of a segment the
-    // lanes read the next 32 dense flags of the tile in parallel (one ballot),
-    // so a flag costs no dependent global load per stage; lane 0 issues the
-    // copies and publishes each stage's kind to the MMA thread in s_kind
-    // before arming the stage's barrier (the arrive releases it).
+    // A stage covers two 128 x 128 tile columns of A.  Both sparse: one
+    // 128-byte box of compressed values (128-byte swizzle) and both metadata
+    // chunks, as in a plain 2:4 stage.  Otherwise each column separately: a
+    // dense column from A's dense form (16 KB, 128-byte swizzle) into its
+    // slot, a sparse one as a 64-byte box of values (64-byte swizzle) plus its
+    // metadata chunk.  The stage's kind (bit c: column c dense; bit 2: no
+    // second column, K / 128 odd) goes to the MMA thread in s_kind before the
+    // stage's barrier is armed (the arrive releases it).  The whole warp walks
+    // the segments; every 16 stages the lanes read the next 32 dense flags of
+    // the tile row in parallel (one ballot), so no flag costs a dependent
+    // global load.
     const uint64_t pol_stream = policy_evict_first();
     const uint64_t pol_keep = policy_evict_last();
-    constexpr uint32_t kDenseTx = (uint32_t)(C::kABytes + kBN * 128);
-    constexpr uint32_t kSparseTx = (uint32_t)(kBlockA * 64 + kBN * 128 + 2048);
+    constexpr uint32_t kBTx = (uint32_t)C::kBBytes;
     int armed[S];
     for (int s = 0; s < S; ++s) armed[s] = -1;
-    auto flag_word = [&](const GemmProblem& P, int ta, int k0, int ke) -> uint32_t {
-      const int k = k0 + lane;
-      const bool d = k < ke && P.tile_mask[(int64_t)ta * P.num_kt + k] != 0;
+    auto flag_word = [&](const GemmProblem& P, int ta, int c0) -> uint32_t {
+      const int kcols = P.K / 128;
+      const int c = c0 + lane;
+      const bool d = c < kcols && P.tile_mask[(int64_t)ta * kcols + c] != 0;
       return __ballot_sync(0xFFFFFFFFu, d);
     };
-    auto load_a = [&](int stage, const GemmProblem& P, int pr, int ta, int kt, bool dense) {
+    auto stage_kind = [&](const GemmProblem& P, int kt, int i, uint32_t fl) -> uint32_t {
+      const int b = (2 * i) & 31;
+      return ((fl >> b) & 3u) | (2 * kt + 1 >= P.K / 128 ? 4u : 0u);
+    };
+    auto a_bytes = [&](uint32_t kind) -> uint32_t {
+      if (kind == 0) return 16384u + 4096u;
+      uint32_t b = (kind & 1u) ? 16384u : 8192u + 2048u;
+      if (!(kind & 4u)) b += (kind & 2u) ? 16384u : 8192u + 2048u;
+      return b;
+    };
+    auto load_a = [&](int stage, const GemmProblem& P, int pr, int ta, int kt, uint32_t kind) {
       const uint32_t sa = smem_u32(smem + stage * C::kStageBytes);
+      const uint32_t sm = sa + C::kABytes + C::kBBytes;
       const int32_t ya = ta * kBlockA;
-      if (dense) {
-        tma_load_2d(sa, &g.tm_a[pr], full_bar(stage), kt * 128, ya, pol_stream);
-      } else {
-        tma_load_2d(sa, &g.tm_a2[pr], full_bar(stage), kt * 64, ya, pol_stream);
-        bulk_load(sa + C::kABytes + C::kBBytes, P.meta + ((int64_t)ta * P.num_kt + kt) * 2048, 2048,
-                  full_bar(stage), pol_stream);
+      const int64_t chunk0 = (int64_t)ta * (P.K / 128) + 2 * (int64_t)kt;
+      if (kind == 0) {
+        tma_load_2d(sa, &g.tm_a3[pr], full_bar(stage), kt * 128, ya, pol_stream);
+        bulk_load(sm, P.meta + chunk0 * 2048, 4096, full_bar(stage), pol_stream);
+        return;
+      }
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        if (c == 1 && (kind & 4u)) break;
+        const uint32_t slot = sa + c * 16384;
+        if ((kind >> c) & 1u) {
+          tma_load_2d(slot, &g.tm_a[pr], full_bar(stage), (2 * kt + c) * 128, ya, pol_stream);
+        } else {
+          tma_load_2d(slot, &g.tm_a2[pr], full_bar(stage), (2 * kt + c) * 64, ya, pol_stream);
+          bulk_load(sm + c * 2048, P.meta + (chunk0 + c) * 2048, 2048, full_bar(stage), pol_stream);
+        }
       }
     };
-    auto arm = [&](int stage, bool dense, int ph) {
-      s_kind[stage] = dense ? 1 : 0;
-      mbar_arrive_expect_tx(full_bar(stage), dense ? kDenseTx : kSparseTx);
+    auto arm = [&](int stage, uint32_t kind, int ph) {
+      s_kind[stage] = (uint8_t)kind;
+      mbar_arrive_expect_tx(full_bar(stage), a_bytes(kind) + kBTx);
       armed[stage] = ph;
     };
     // 1. static weights: the first S stages' A copies before the dependency wait
@@ -345,14 +392,15 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
         const GemmProblem& P = g.prob[pr];
         const int ta = tile % P.tiles_a;
         const int take = min(ke - kb, S - pre);  // <= S <= 8 stages: one flag word
-        const uint32_t fl = flag_word(P, ta, kb, kb + take);
+        const uint32_t fl = flag_word(P, ta, 2 * kb);
         if (lane == 0) {
           tma_prefetch_desc(&g.tm_a[pr]);
           tma_prefetch_desc(&g.tm_a2[pr]);
+          tma_prefetch_desc(&g.tm_a3[pr]);
           for (int i = 0; i < take; ++i) {
-            const bool dense = (fl >> i) & 1u;
-            arm(pre + i, dense, 0);
-            load_a(pre + i, P, pr, ta, kb + i, dense);
+            const uint32_t kind = stage_kind(P, kb + i, i, fl);
+            arm(pre + i, kind, 0);
+            load_a(pre + i, P, pr, ta, kb + i, kind);
           }
         }
         pre += take;
@@ -376,25 +424,29 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
       if (lane == 0) {
         tma_prefetch_desc(&g.tm_a[pr]);
         tma_prefetch_desc(&g.tm_a2[pr]);
+        tma_prefetch_desc(&g.tm_a3[pr]);
         tma_prefetch_desc(&g.tm_b[pr]);
       }
       uint32_t fl = 0;
       for (int kt = kb; kt < ke; ++kt) {
-        if (((kt - kb) & 31) == 0) fl = flag_word(P, ta, kt, ke);
+        const int i = kt - kb;
+        if ((i & 15) == 0) fl = flag_word(P, ta, 2 * kt);
         if (lane == 0) {
-          const bool dense = (fl >> ((kt - kb) & 31)) & 1u;
           if (n >= pre) {
             if (!mbar_wait(empty_bar(stage), phase ^ 1, p.timeout_ns, kDevErrWaitEmpty)) {
               ok = false;
               *abort_flag = 1;
             } else {
-              arm(stage, dense, (int)phase);
-              load_a(stage, P, pr, ta, kt, dense);
+              const uint32_t kind = stage_kind(P, kt, i & 15, fl);
+              arm(stage, kind, (int)phase);
+              load_a(stage, P, pr, ta, kt, kind);
             }
           }
           if (ok) {
-            tma_load_2d(smem_u32(smem + stage * C::kStageBytes) + C::kABytes, &g.tm_b[pr], full_bar(stage),
-                        kt * 128, tb * kBN, pol_keep);
+            const uint32_t sb = smem_u32(smem + stage * C::kStageBytes) + C::kABytes;
+#pragma unroll
+            for (int bx = 0; bx < 2; ++bx)
+              tma_load_2d(sb + bx * kBN * 128, &g.tm_b[pr], full_bar(stage), kt * 256 + bx * 128, tb * kBN, pol_keep);
             ++n;
             if (++stage == S) {
               stage = 0;
@@ -435,7 +487,17 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
         const uint32_t sa = smem_u32(smem + stage * C::kStageBytes);
         const uint32_t sm = sa + C::kABytes + C::kBBytes;
         const int32_t ya = ta * C::kRowsA + (int32_t)rank * kBlockA;
-        {
+        if (C::kNv) {
+          // 128 bytes of A per row; metadata chunks (sparse) and the four
+          // scale chunks of A's 128-row block at this stage's K
+          load2d(sa, &g.tm_a[pr], stage, kt * 128, ya, pol_stream);
+          const int nsf = nv_half(P, kt) ? 2 : 4;
+          if (C::kNvSparse)
+            bulk_load(sm, P.meta + ((int64_t)ta * (P.K / 256) + 2 * (int64_t)kt) * 2048, (uint32_t)(nsf / 2) * 2048,
+                      full_bar(stage), pol_stream);
+          bulk_load(sm + C::kMetaBytes, P.sfa + ((int64_t)ta * (P.K / C::kSfChunkK) + 4 * (int64_t)kt) * 512,
+                    (uint32_t)nsf * 512, full_bar(stage), pol_stream);
+        } else {
           const int ax = C::kSparse ? kt * (C::kKT / 2) : kt * C::kKT;  // elements
           load2d(sa, &g.tm_a[pr], stage, ax, ya, pol_stream);
           if (C::kSparse) {
@@ -457,7 +519,19 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
       auto load_b = [&](int stage, int pr, int tb, int kt) {
         const uint32_t sb = smem_u32(smem + stage * C::kStageBytes) + C::kABytes;
         const int32_t yb = tb * kBN + (int32_t)rank * C::kBRows;
-        {
+        if (C::kNv) {
+          // kKT / 2 bytes of B per row, then the four scale chunks of the
+          // 128-row block of B that holds this tile (tiles of fewer than 128
+          // rows are the only tile of their operand: the host checks)
+          const GemmProblem& P = g.prob[pr];
+#pragma unroll
+          for (int bx = 0; bx < C::kBBoxes; ++bx)
+            load2d(sb + bx * C::kBRows * 128, &g.tm_b[pr], stage, kt * (C::kKT / 2) + bx * 128, yb, pol_keep);
+          const int nsf = nv_half(P, kt) ? 2 : 4;
+          bulk_load(sb + C::kBBytes + C::kMetaBytes + 2048,
+                    P.sfb + ((int64_t)((tb * kBN) >> 7) * (P.K / C::kSfChunkK) + 4 * (int64_t)kt) * 512,
+                    (uint32_t)nsf * 512, full_bar(stage), pol_keep);
+        } else {
           const int box_elems = kBf16 ? 64 : 128;
 #pragma unroll
           for (int bx = 0; bx < C::kBBoxes; ++bx)
@@ -468,6 +542,10 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
       auto stage_bytes = [&](int pr, int ta, int kt) -> uint32_t {
         const GemmProblem& P = g.prob[pr];
         if (kPair) return 2u * (uint32_t)C::kStageBytes;  // metadata boxes are always whole
+        if (C::kNv) {
+          const uint32_t nsf = nv_half(P, kt) ? 2u : 4u;
+          return (uint32_t)(C::kABytes + C::kBBytes) + (C::kNvSparse ? nsf / 2 * 2048u : 0u) + 2u * nsf * 512u;
+        }
         uint32_t b = C::kABytes + C::kBBytes;
         if (C::kSparse) b += (uint32_t)meta_chunks(P, kt) * 2048;
         return b;
@@ -553,7 +631,8 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
       pdl_launch_dependents();
     }
     if (lane == 0 && rank == 0) {
-      const uint32_t idesc = make_idesc(C::kSparse, kBf16, C::kRowsA, kBN);
+      const uint32_t idesc = C::kNv ? make_idesc_nvf4(C::kNvSparse, kBlockA, kBN)
+                                    : make_idesc(C::kSparse, kBf16, C::kRowsA, kBN);
       const uint32_t idesc_dense = make_idesc(false, kBf16, kBlockA, kBN);
       const uint32_t idesc_sp = make_idesc(true, kBf16, C::kRowsA, kBN);
       const uint32_t meta_col0 = C::kAccCols;
@@ -564,6 +643,11 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
       // both chunks of an e4m3 stage as one 128 x 256-bit copy: the second
       // chunk is the second core matrix along the row, 2048 bytes on
       const uint64_t dm2 = smem_desc(s0 + C::kABytes + C::kBBytes, 2048, 128, kLayoutNone);
+      // NVFP4: the first scale chunk of A (B's follow 2048 bytes on), one
+      // 32-row x 128-bit matrix of 16-byte rows
+      const uint64_t dsf0 = smem_desc(s0 + C::kABytes + C::kBBytes + C::kMetaBytes, 16, 128, kLayoutNone);
+      // hybrid: a sparse tile column's 64-byte rows of values (64-byte swizzle)
+      const uint64_t dsp0 = smem_desc(s0, 16, 512, kLayoutSw64);
       int stage = 0;
       uint32_t phase = 0;
       uint32_t acc_i = 0;
@@ -595,22 +679,73 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
           const uint32_t mcol = meta_col0 + stage * C::kMetaCols;
           const bool first = kt == kb;
           if (C::kHybrid) {
-            if (s_kind[stage] != 0) {
+            const uint32_t kind = s_kind[stage];
+            const uint64_t so = (uint64_t)((uint32_t)stage * (uint32_t)(C::kStageBytes >> 4));
+            uint32_t acc = first ? 0u : 1u;
+            if (kind == 0) {
+              // both columns sparse: the plain 2:4 e4m3 stage
+              tc_cp_128x256b(tmem_base + mcol, dm2 + so);
 #pragma unroll
               for (int j = 0; j < 4; ++j) {
-                const uint64_t da = smem_desc(sa + j * 32, 16, 1024, kLayoutSw128);
-                const uint64_t db = smem_desc(sb + j * 32, 16, 1024, kLayoutSw128);
-                mma_f8(d, da, db, idesc_dense, (first && j == 0) ? 0u : 1u);
+                const uint64_t a_d = da0 + so + (uint64_t)(j * 2);
+                const uint64_t b_d = db0 + so + (uint64_t)(((j >> 1) * kBN * 128 + (j & 1) * 64) >> 4);
+                mma_sp_f8(d, a_d, b_d, tmem_base + mcol + 2 * j, idesc_sp, acc);
+                acc = 1u;
               }
             } else {
-              tc_cp_128x128b(tmem_base + mcol, smem_desc(sm, 16, 128, kLayoutNone));
 #pragma unroll
-              for (int j = 0; j < 2; ++j) {
-                const uint64_t da = smem_desc(sa + j * 32, 16, 512, kLayoutSw64);
-                const uint64_t db = smem_desc(sb + j * 64, 16, 1024, kLayoutSw128);
-                mma_sp_f8(d, da, db, tmem_base + mcol + 2 * j, idesc_sp, (first && j == 0) ? 0u : 1u);
+              for (int c = 0; c < 2; ++c) {
+                if (c == 1 && (kind & 4u)) break;
+                const uint64_t slot = so + (uint64_t)(c * (16384 >> 4));       // A slot of column c
+                const uint64_t bbox = db0 + so + (uint64_t)((c * kBN * 128) >> 4);  // B box of column c
+                if ((kind >> c) & 1u) {
+#pragma unroll
+                  for (int j = 0; j < 4; ++j) {
+                    mma_f8(d, da0 + slot + (uint64_t)(j * 2), bbox + (uint64_t)(j * 2), idesc_dense, acc);
+                    acc = 1u;
+                  }
+                } else {
+                  tc_cp_128x128b(tmem_base + mcol + 4 * c, dm0 + so + (uint64_t)(c * (2048 >> 4)));
+#pragma unroll
+                  for (int j = 0; j < 2; ++j) {
+                    mma_sp_f8(d, dsp0 + slot + (uint64_t)(j * 2), bbox + (uint64_t)(j * 4),
+                              tmem_base + mcol + 4 * c + 2 * j, idesc_sp, acc);
+                    acc = 1u;
+                  }
+                }
               }
             }
+          } else if (C::kNv) {
+            const uint64_t so = (uint64_t)((uint32_t)stage * (uint32_t)(C::kStageBytes >> 4));
+            const uint64_t da = da0 + so, db = db0 + so, dsf = dsf0 + so;
+            const uint32_t scol = mcol + C::kMetaChunks * 4;  // A scales; B scales 16 columns on
+            auto issue = [&](auto mmas_c) {
+              constexpr int kMmas = decltype(mmas_c)::value;
+              if (C::kNvSparse) {
+                if (kMmas == 4) tc_cp_128x256b(tmem_base + mcol, dm2 + so);
+                else tc_cp_128x128b(tmem_base + mcol, dm0 + so);
+              }
+#pragma unroll
+              for (int j = 0; j < kMmas; ++j) {
+                tc_cp_32x128b_x4(tmem_base + scol + 4 * j, dsf + (uint64_t)(32 * j));
+                tc_cp_32x128b_x4(tmem_base + scol + 16 + 4 * j, dsf + (uint64_t)(128 + 32 * j));
+              }
+#pragma unroll
+              for (int j = 0; j < kMmas; ++j) {
+                const uint32_t acc = (first && j == 0) ? 0u : 1u;
+                const uint32_t sfa = tmem_base + scol + 4 * j, sfb = tmem_base + scol + 16 + 4 * j;
+                if (C::kNvSparse) {
+                  // 32 bytes of A (128 logical positions) and 64 bytes of B per MMA
+                  const uint64_t a_d = da + (uint64_t)(j * 2);
+                  const uint64_t b_d = db + (uint64_t)(((j >> 1) * C::kBRows * 128 + (j & 1) * 64) >> 4);
+                  mma_sp_nvf4(d, a_d, b_d, tmem_base + mcol + 2 * j, idesc, sfa, sfb, acc);
+                } else {
+                  mma_nvf4(d, da + (uint64_t)(j * 2), db + (uint64_t)(j * 2), idesc, sfa, sfb, acc);
+                }
+              }
+            };
+            if (nv_half(P, kt)) issue(std::integral_constant<int, 2>{});
+            else issue(std::integral_constant<int, 4>{});
           } else if (C::kSparse) {
             // descriptors of this stage: the stage-0 descriptors plus the
             // stage offset (the address field counts 16-byte units)
@@ -718,12 +853,12 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
       const int64_t ldy = P.ldy;
       const bool a_live = ga < rows_a;
       // scales: loaded before waiting for the accumulator so their latency hides
-      const float sa_v = (P.scale_a != nullptr && a_live) ? __ldg(P.scale_a + ga) : 1.0f;
+      const float sa_v = P.scale_a == nullptr ? 1.0f : C::kNv ? __ldg(P.scale_a) : a_live ? __ldg(P.scale_a + ga) : 1.0f;
       if (pr != cached_pr || tb != cached_tb) {
         named_bar_sync(1, 128);
         for (int i = et; i < kBN; i += 128) {
           const int gb = tb * kBN + i;
-          s_scale_b[i] = (P.scale_b != nullptr && gb < rows_b) ? P.scale_b[gb] : 1.0f;
+          s_scale_b[i] = P.scale_b == nullptr ? 1.0f : C::kNv ? P.scale_b[0] : gb < rows_b ? P.scale_b[gb] : 1.0f;
         }
         named_bar_sync(1, 128);
         cached_pr = pr;

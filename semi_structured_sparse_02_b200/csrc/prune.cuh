@@ -481,6 +481,71 @@ k_quantize_rows_e4m3_seg(const __grid_constant__ QuantSegGroup g) {
 }
 
 // ---------------------------------------------------------------------------
+// Online activations at the FP8 floor in one pass: per-token amax, 2:4 prune
+// on the bf16 magnitudes, E4M3 cast of the kept values with the row scale,
+// the metadata image and the scale, from one HBM read of X.  Rows are held in
+// registers as warp segments (the layout of k_quantize_rows_e4m3_seg: a row
+// takes w warps of kQWarpVecs 16-byte vectors per lane, a CTA floor(16 / w)
+// rows), the row amax is combined across its warps in shared memory.  Each
+// 16-byte vector is two groups: one metadata byte (image row = the row for
+// 8-bit values, byte idx % 16 of chunk idx / 16) and four E4M3 codes.  Same
+// results as k_row_amax + k_prune_compress<true> + k_finalize_scales.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kQWarps * 32, 2)
+k_prune_cast_rows_e4m3(const uint16_t* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
+                       int warps_per_row, int rows_per_cta, uint8_t* __restrict__ values,
+                       uint8_t* __restrict__ meta, float* __restrict__ scales) {
+  __shared__ uint32_t s_amax[kQWarps];
+  pdl_launch_dependents();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x < kQWarps) s_amax[threadIdx.x] = 0u;
+  const int w = warps_per_row, slot = warp / w, seg = warp - slot * w;
+  const int64_t row = (int64_t)blockIdx.x * rows_per_cta + slot;
+  // rows from `rows` to the end of the last 128-row block only get their
+  // metadata (the prune of zeros: positions 0 and 1)
+  const int64_t rows_pad = (rows + kChunkRows - 1) / kChunkRows * kChunkRows;
+  const bool active = slot < rows_per_cta && row < rows_pad;
+  const bool live = active && row < rows;
+  const int64_t nv = K / 8;
+  pdl_wait();  // the activations may be written by the upstream grid
+  uint4 reg[kQWarpVecs];
+  uint32_t m = 0;
+  const uint4* p = reinterpret_cast<const uint4*>(src + (live ? row : 0) * ld);
+#pragma unroll
+  for (int j = 0; j < kQWarpVecs; ++j) {
+    const int64_t idx = (int64_t)seg * kQSegVecs + j * 32 + lane;
+    reg[j] = (live && idx < nv) ? __ldg(p + idx) : make_uint4(0, 0, 0, 0);
+    m = max(m, amax_bits8(reg[j]));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  __syncthreads();  // s_amax initialized
+  if (active && lane == 0) atomicMax(&s_amax[slot], m);
+  __syncthreads();
+  if (!active) return;
+  const float amax = bf16_bits_to_float(s_amax[slot]);
+  const float inv = e4m3_inv_scale(amax);
+  if (live && seg == 0 && lane == 0) scales[row] = amax == 0.0f ? 1.0f : __fdiv_rn(amax, 448.0f);
+  const int64_t KC = K / kChunkK;
+  const int64_t rb = row / kChunkRows, L = row % kChunkRows;
+  uint8_t* vrow = values + row * (K / 2);
+#pragma unroll
+  for (int j = 0; j < kQWarpVecs; ++j) {
+    const int64_t idx = (int64_t)seg * kQSegVecs + j * 32 + lane;
+    if (idx < nv) {
+      const uint4 v = reg[j];
+      uint32_t k00, k01, k10, k11;
+      const uint32_t nib0 = prune_pick4(v.x & 0xFFFFu, v.x >> 16, v.y & 0xFFFFu, v.y >> 16, k00, k01);
+      const uint32_t nib1 = prune_pick4(v.z & 0xFFFFu, v.z >> 16, v.w & 0xFFFFu, v.w >> 16, k10, k11);
+      const uint32_t q = e4m3x2_of(__fmul_rn(bf16_bits_to_float(k00), inv), __fmul_rn(bf16_bits_to_float(k01), inv)) |
+                         (e4m3x2_of(__fmul_rn(bf16_bits_to_float(k10), inv), __fmul_rn(bf16_bits_to_float(k11), inv)) << 16);
+      if (live) *reinterpret_cast<uint32_t*>(vrow + idx * 4) = q;
+      meta[(rb * KC + idx / 16) * kChunkBytes + L * 16 + (idx % 16)] = (uint8_t)(nib0 | (nib1 << 4));
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Decompress: scatter values back using the metadata image.
 // ---------------------------------------------------------------------------
 // Nibble of (row-in-block r, group g in chunk) inside one image chunk.

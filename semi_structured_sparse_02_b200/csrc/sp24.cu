@@ -18,6 +18,7 @@
 #include "sp24.h"
 #include "sp24_device.cuh"
 #include "prune.cuh"
+#include "nvfp4.cuh"
 #include "gemm.cuh"
 #include "gemm_wide.cuh"
 
@@ -149,7 +150,9 @@ int pick_bn(int64_t rows_b) {
 }
 
 int stage_k(int mode, bool bf16) {
-  if (mode == kModeHybrid) return 128;
+  if (mode == kModeNvSparse) return 512;
+  if (mode == kModeNvDense) return 256;
+  if (mode == kModeHybrid) return 256;
   if (mode == kModeSparse) return bf16 ? 128 : 256;
   return bf16 ? 64 : 128;
 }
@@ -342,6 +345,8 @@ int dispatch_gemm(const Plan& pl, const GemmLaunch<1>& gl, cudaStream_t s) {
                    : launch_gemm_bn<kModeDense, false, true, 1>(pl.bn, gl, pl.grid, s);
   if (pl.mode == kModeHybrid && !pl.bf16)
     return launch_gemm_bn<kModeHybrid, false, true, 1>(pl.bn, gl, pl.grid, s);
+  if (pl.mode == kModeNvSparse) return launch_gemm_bn<kModeNvSparse, false, true, 1>(pl.bn, gl, pl.grid, s);
+  if (pl.mode == kModeNvDense) return launch_gemm_bn<kModeNvDense, false, true, 1>(pl.bn, gl, pl.grid, s);
   return SP24_ERR_DTYPE;
 }
 
@@ -460,10 +465,14 @@ bool fill_problem(GemmLaunch<kMaxProb>& gl, int i, const sp24_gemm_args* a, cons
       gl.tm_a2[i] = gl.tm_a[i];
     }
   } else {
+    // hybrid: the dense form (dense tile columns), the values as 64-byte boxes
+    // (one sparse column) and as 128-byte boxes (two sparse columns)
     ok &= make_map(&gl.tm_a[i], a->W_dense_tiles, 1, a->K, a->N, a->K, 128, kBlockA,
                    CU_TENSOR_MAP_SWIZZLE_128B);
     ok &= make_map(&gl.tm_a2[i], a->W, 1, a->K / 2, a->N, a->ldw, 64, kBlockA, CU_TENSOR_MAP_SWIZZLE_64B);
+    ok &= make_map(&gl.tm_a3[i], a->W, 1, a->K / 2, a->N, a->ldw, 128, kBlockA, CU_TENSOR_MAP_SWIZZLE_128B);
   }
+  if (pl.mode != kModeHybrid) gl.tm_a3[i] = gl.tm_a[i];
   ok &= make_map(&gl.tm_b[i], a->X, eb, a->K, a->M, a->ldx * eb, box_elems, pl.pair ? pl.bn / 2 : pl.bn,
                  CU_TENSOR_MAP_SWIZZLE_128B);
   GemmProblem& P = gl.prob[i];
@@ -796,6 +805,7 @@ int run_activation_gemm(bool bf16, const void* x_values, const void* x_meta, con
   ok &= make_map(&gl.tm_b[0], W, eb, K, N, ldw * eb, box_elems, 128, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok) return SP24_ERR_CUDA;
   gl.tm_a2[0] = gl.tm_a[0];
+  gl.tm_a3[0] = gl.tm_a[0];
   GemmProblem& P = gl.prob[0];
   P.rows_a = (int32_t)M;
   P.rows_b = (int32_t)N;
@@ -851,6 +861,89 @@ int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cud
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return launch_result(cudaLaunchKernelEx(&cfg, kernel, args...));
+}
+
+// ---------------------------------------------------------------------------
+// NVFP4 GEMM (block-scaled kind::mxf4nvf4): validation, plan, launch fill
+// ---------------------------------------------------------------------------
+int validate_nvfp4(const sp24_nvfp4_gemm_args* a) {
+  if (a == nullptr) return SP24_ERR_NULL;
+  if (a->M < 1 || a->N < 1 || a->K < 1) return SP24_ERR_INVALID_ARG;
+  if (a->M > INT32_MAX / 2 || a->N > INT32_MAX / 2 || a->K > INT32_MAX / 2) return SP24_ERR_INVALID_ARG;
+  if (a->tactic != SP24_TACTIC_SPARSE && a->tactic != SP24_TACTIC_DENSE) return SP24_ERR_INVALID_ARG;
+  if (a->out_dtype != SP24_BF16 && a->out_dtype != SP24_F32) return SP24_ERR_DTYPE;
+  const bool sparse = a->tactic == SP24_TACTIC_SPARSE;
+  if (a->X == nullptr || a->x_scales == nullptr || a->x_tensor_scale == nullptr || a->W == nullptr ||
+      a->w_scales == nullptr || a->w_tensor_scale == nullptr || a->Y == nullptr || (sparse && a->W_meta == nullptr))
+    return SP24_ERR_NULL;
+  if (a->K % 256 != 0) return sparse ? SP24_ERR_NOT_2_4 : SP24_ERR_ALIGNMENT;
+  if (a->ldy < a->N) return SP24_ERR_INVALID_ARG;
+  const int ob = dtype_bytes(a->out_dtype);
+  if (!aligned16(a->X) || !aligned16(a->x_scales) || !aligned16(a->W) || !aligned16(a->w_scales) ||
+      (sparse && !aligned16(a->W_meta)) || !aligned16(a->Y) || (a->ldy * ob) % 16 != 0)
+    return SP24_ERR_ALIGNMENT;
+  if ((reinterpret_cast<uintptr_t>(a->x_tensor_scale) & 3u) || (reinterpret_cast<uintptr_t>(a->w_tensor_scale) & 3u))
+    return SP24_ERR_ALIGNMENT;
+  return SP24_OK;
+}
+
+// Token tiles (pick_bn) of fewer than 128 rows only occur when the tokens fit
+// one tile, so every tile's B scales start a 128-row chunk of the scale image.
+Plan plan_nvfp4(const sp24_nvfp4_gemm_args* a, const DeviceInfo& di, size_t ws_cap) {
+  Plan pl;
+  memset(&pl, 0, sizeof pl);
+  pl.mode = a->tactic == SP24_TACTIC_SPARSE ? kModeNvSparse : kModeNvDense;
+  pl.bf16 = false;
+  pl.a_is_w = true;
+  pl.bn = pick_bn(a->M);
+  pl.kt = stage_k(pl.mode, false);
+  pl.n = 1;
+  pl.num_kt[0] = (int)((a->K + pl.kt - 1) / pl.kt);
+  pl.tiles_a[0] = (int)((a->N + kBlockA - 1) / kBlockA);
+  pl.tiles_b[0] = (int)((a->M + pl.bn - 1) / pl.bn);
+  choose_schedule(pl, di.sms, ws_cap);
+  return pl;
+}
+
+int build_launch_nvfp4(GemmLaunch<1>& gl, const sp24_nvfp4_gemm_args* a, const Plan& pl) {
+  memset(&gl, 0, sizeof gl);
+  const bool sparse = pl.mode == kModeNvSparse;
+  const uint64_t a_bytes = (uint64_t)(sparse ? a->K / 4 : a->K / 2);  // bytes of a W row
+  bool ok = make_map(&gl.tm_a[0], a->W, 1, a_bytes, a->N, a_bytes, 128, kBlockA, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= make_map(&gl.tm_b[0], a->X, 1, a->K / 2, a->M, a->K / 2, 128, pl.bn, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!ok) return SP24_ERR_CUDA;
+  gl.tm_a2[0] = gl.tm_a[0];
+  gl.tm_a3[0] = gl.tm_a[0];
+  const bool sk = pl.sched == kSchedStreamK;
+  uint8_t* ws = static_cast<uint8_t*>(a->workspace);
+  GemmProblem& P = gl.prob[0];
+  P.rows_a = (int32_t)a->N;
+  P.rows_b = (int32_t)a->M;
+  P.K = (int32_t)a->K;
+  P.num_kt = pl.num_kt[0];
+  P.tiles_a = pl.tiles_a[0];
+  P.tiles_b = pl.tiles_b[0];
+  P.meta_blocks = (int32_t)((a->N + 127) / 128);
+  P.meta = static_cast<const uint8_t*>(a->W_meta);
+  P.sfa = static_cast<const uint8_t*>(a->w_scales);
+  P.sfb = static_cast<const uint8_t*>(a->x_scales);
+  P.scale_a = a->w_tensor_scale;
+  P.scale_b = a->x_tensor_scale;
+  P.Y = a->Y;
+  P.ldy = a->ldy;
+  P.ws_counters = sk ? reinterpret_cast<unsigned int*>(ws) : nullptr;
+  gl.p.sk_flags = sk ? reinterpret_cast<unsigned int*>(ws + sk_counters_bytes(pl)) : nullptr;
+  gl.p.sk_slots = sk ? reinterpret_cast<float*>(ws + sk_state_bytes(pl)) : nullptr;
+  gl.p.n_prob = 1;
+  gl.p.sched = pl.sched;
+  gl.p.total_iters = pl.total_iters;
+  gl.p.total_tiles = pl.total_tiles;
+  gl.p.out_f32 = a->out_dtype == SP24_F32;
+  gl.p.use_pdl = 1;
+  gl.p.w_static = (a->flags & SP24_GEMM_W_STATIC) != 0;
+  gl.p.after_independent = (a->flags & SP24_GEMM_AFTER_INDEPENDENT) != 0;
+  gl.p.timeout_ns = g_timeout_ns.load();
+  return SP24_OK;
 }
 
 // ---------------------------------------------------------------------------
@@ -1201,6 +1294,108 @@ int sp24_energy_loss(const void* src, int64_t rows, int64_t K, int64_t ld, doubl
   return launch_result(cudaGetLastError());
 }
 
+size_t sp24_nvfp4_48_values_bytes(int64_t rows, int64_t K) {
+  return rows < 0 || K < 0 ? 0 : (size_t)rows * (size_t)(K / 4);
+}
+
+size_t sp24_nvfp4_48_meta_bytes(int64_t rows, int64_t K) {
+  return rows < 0 || K < 0 ? 0 : (size_t)((rows + 127) / 128) * (size_t)(K / 256) * 2048;
+}
+
+size_t sp24_nvfp4_codes_bytes(int64_t rows, int64_t K) {
+  return rows < 0 || K < 0 ? 0 : (size_t)rows * (size_t)(K / 2);
+}
+
+size_t sp24_nvfp4_scales_bytes(int64_t rows, int64_t K, int block) {
+  if (rows < 0 || K < 0 || (block != 16 && block != 32)) return 0;
+  return (size_t)((rows + 127) / 128) * 128 * (size_t)(K / block);
+}
+
+int sp24_prune_compress_nvfp4_48(const void* src, int64_t rows, int64_t K, int64_t ld, void* values, void* meta,
+                                 void* scales, float* tensor_scale, void* stream) {
+  if (src == nullptr || values == nullptr || meta == nullptr || scales == nullptr || tensor_scale == nullptr)
+    return SP24_ERR_NULL;
+  if (rows < 1 || K < 256 || ld < K) return SP24_ERR_INVALID_ARG;
+  if (K % 256 != 0) return SP24_ERR_NOT_2_4;
+  if (ld % 8 != 0 || !aligned16(src) || !aligned16(values) || !aligned16(meta) || !aligned16(scales) ||
+      (reinterpret_cast<uintptr_t>(tensor_scale) & 3u))
+    return SP24_ERR_ALIGNMENT;
+  DeviceInfo di;
+  int st = current_device_info(&di);
+  if (st != SP24_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const uint16_t* src16 = static_cast<const uint16_t*>(src);
+  unsigned int* amax = reinterpret_cast<unsigned int*>(tensor_scale);
+  if (cudaMemsetAsync(tensor_scale, 0, sizeof(float), s) != cudaSuccess) {
+    cudaGetLastError();
+    return SP24_ERR_CUDA;
+  }
+  const int64_t groups = rows * (K / 8);
+  const int agrid = (int)std::min<int64_t>((groups + kNvThreads - 1) / kNvThreads, (int64_t)di.sms * 8);
+  k_nvfp4_amax<true><<<agrid, kNvThreads, 0, s>>>(src16, rows, K, ld, amax);
+  if ((st = launch_result(cudaGetLastError())) != SP24_OK) return st;
+  const int64_t chunks = ((rows + 127) / 128) * (K / 256);
+  const int cgrid = (int)std::min<int64_t>(chunks, (int64_t)di.sms * 8);
+  st = launch_pdl(k_nvfp4_48_compress, dim3(cgrid), dim3(kNvThreads), 0, s, src16, rows, K, ld,
+                  static_cast<uint8_t*>(values), static_cast<uint8_t*>(meta), static_cast<uint8_t*>(scales),
+                  static_cast<const unsigned int*>(amax));
+  if (st != SP24_OK) return st;
+  return launch_pdl(k_nvfp4_finalize, dim3(1), dim3(32), 0, s, tensor_scale);
+}
+
+int sp24_quantize_nvfp4(const void* src, int64_t rows, int64_t K, int64_t ld, int block, void* codes, void* scales,
+                        float* tensor_scale, void* stream) {
+  if (src == nullptr || codes == nullptr || scales == nullptr || tensor_scale == nullptr) return SP24_ERR_NULL;
+  if (block != 16 && block != 32) return SP24_ERR_INVALID_ARG;
+  if (rows < 1 || K < 4 * block || ld < K) return SP24_ERR_INVALID_ARG;
+  if (K % (4 * block) != 0) return SP24_ERR_ALIGNMENT;
+  if (ld % 8 != 0 || !aligned16(src) || !aligned16(codes) || !aligned16(scales) ||
+      (reinterpret_cast<uintptr_t>(tensor_scale) & 3u))
+    return SP24_ERR_ALIGNMENT;
+  DeviceInfo di;
+  int st = current_device_info(&di);
+  if (st != SP24_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const uint16_t* src16 = static_cast<const uint16_t*>(src);
+  unsigned int* amax = reinterpret_cast<unsigned int*>(tensor_scale);
+  if (cudaMemsetAsync(tensor_scale, 0, sizeof(float), s) != cudaSuccess) {
+    cudaGetLastError();
+    return SP24_ERR_CUDA;
+  }
+  const int64_t groups = rows * (K / 8);
+  const int agrid = (int)std::min<int64_t>((groups + kNvThreads - 1) / kNvThreads, (int64_t)di.sms * 8);
+  k_nvfp4_amax<false><<<agrid, kNvThreads, 0, s>>>(src16, rows, K, ld, amax);
+  if ((st = launch_result(cudaGetLastError())) != SP24_OK) return st;
+  const int64_t items = ((rows + 127) / 128) * 128 * (K / (4 * block));
+  const int qgrid = (int)std::min<int64_t>((items + kNvThreads - 1) / kNvThreads, (int64_t)di.sms * 8);
+  uint8_t* c8 = static_cast<uint8_t*>(codes);
+  uint8_t* s8 = static_cast<uint8_t*>(scales);
+  const unsigned int* ab = amax;
+  st = block == 16 ? launch_pdl(k_nvfp4_quantize<16>, dim3(qgrid), dim3(kNvThreads), 0, s, src16, rows, K, ld, c8, s8, ab)
+                   : launch_pdl(k_nvfp4_quantize<32>, dim3(qgrid), dim3(kNvThreads), 0, s, src16, rows, K, ld, c8, s8, ab);
+  if (st != SP24_OK) return st;
+  return launch_pdl(k_nvfp4_finalize, dim3(1), dim3(32), 0, s, tensor_scale);
+}
+
+size_t sp24_gemm_nvfp4_workspace_bytes(const sp24_nvfp4_gemm_args* a) {
+  if (validate_nvfp4(a) != SP24_OK) return 0;
+  DeviceInfo di;
+  if (current_device_info(&di) != SP24_OK) return 0;
+  return plan_nvfp4(a, di, (size_t)-1).ws_bytes;
+}
+
+int sp24_gemm_nvfp4(const sp24_nvfp4_gemm_args* a, void* stream) {
+  int st = validate_nvfp4(a);
+  if (st != SP24_OK) return st;
+  if (a->workspace != nullptr && !aligned16(a->workspace)) return SP24_ERR_ALIGNMENT;
+  DeviceInfo di;
+  if ((st = current_device_info(&di)) != SP24_OK) return st;
+  static thread_local SingleLaunch v;
+  v.pl = plan_nvfp4(a, di, a->workspace != nullptr ? a->workspace_bytes : 0);
+  if ((st = build_launch_nvfp4(v.gl, a, v.pl)) != SP24_OK) return st;
+  return dispatch_gemm(v.pl, v.gl, static_cast<cudaStream_t>(stream));
+}
+
 size_t sp24_activations_workspace_bytes(int64_t M, int64_t K) {
   if (M < 1 || K < 128) return 0;
   const size_t vals = ((size_t)M * (size_t)(K / 2) * 2 + 255) & ~(size_t)255;
@@ -1242,8 +1437,20 @@ int sp24_prune_compress_activations_fused_e4m3(const void* X, int64_t M, int64_t
   int st = current_device_info(&di);
   if (st != SP24_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // per-token amax, prune + compress + quantize with it, then amax -> scale
   const uint16_t* x16 = static_cast<const uint16_t*>(X);
+  if (K / 8 <= kQMaxVecs) {
+    // rows that fit in registers: amax, prune, cast, metadata and scale in
+    // one pass over X, chained to the GEMM
+    const int w = (int)((K / 8 + kQSegVecs - 1) / kQSegVecs);
+    const int rpc = kQWarps / w;
+    const int64_t rows_pad = (M + 127) / 128 * 128;
+    st = launch_pdl(k_prune_cast_rows_e4m3, dim3((unsigned)((rows_pad + rpc - 1) / rpc)), dim3(kQWarps * 32), 0, s,
+                    x16, M, K, ldx, w, rpc, static_cast<uint8_t*>(x_values), static_cast<uint8_t*>(x_meta), x_scales);
+    if (st != SP24_OK) return st;
+    return run_activation_gemm(false, x_values, x_meta, x_scales, Wq, ldw, w_scales, M, N, K, Y, ldy,
+                               out_dtype == SP24_F32, di, s);
+  }
+  // longer rows: per-token amax, prune + compress + quantize with it, then amax -> scale
   const int agrid = (int)std::min<int64_t>((M + 7) / 8, (int64_t)di.sms * 8);
   k_row_amax<<<agrid, 256, 0, s>>>(x16, M, K, ldx, x_scales);
   if ((st = launch_result(cudaGetLastError())) != SP24_OK) return st;

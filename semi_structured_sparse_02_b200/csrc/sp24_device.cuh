@@ -214,6 +214,49 @@ __device__ __forceinline__ void mma_sp_f8(uint32_t d, uint64_t a, uint64_t b, ui
       : "memory");
 }
 
+// Block-scaled NVFP4 MMA (kind::mxf4nvf4): E2M1 operands, one unsigned E4M3
+// scale per 16 stored elements of each operand row, read from tensor memory
+// at sfa / sfb (four codes per row per MMA).  Dense: K = 64 per MMA.  Sparse
+// (pairwise 4:8 A, metadata at e): K = 128 logical positions per MMA, so one
+// scale per 32 positions.
+__device__ __forceinline__ void mma_nvf4(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t sfa,
+                                         uint32_t sfb, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%4], [%5], p;\n\t}\n" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(sfa), "r"(sfb), "r"(acc)
+      : "memory");
+}
+__device__ __forceinline__ void mma_sp_nvf4(uint32_t d, uint64_t a, uint64_t b, uint32_t e, uint32_t idesc,
+                                            uint32_t sfa, uint32_t sfb, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %7, 0;\n\t"
+      "tcgen05.mma.sp.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, [%3], %4, [%5], [%6], p;\n\t}\n" ::"r"(d),
+      "l"(a), "l"(b), "r"(e), "r"(idesc), "r"(sfa), "r"(sfb), "r"(acc)
+      : "memory");
+}
+
+// Instruction descriptor of the block-scaled kinds: sparse flag bit 2, A and
+// B formats bits 7..9 / 10..12 (E2M1 = 1 for kind::mxf4nvf4), both K-major,
+// N >> 3 in bits 17..22, scale format bit 23 (0 = unsigned E4M3), M >> 4 in
+// bits 24..28; scale-factor byte selectors (bits 4..5, 29..30) 0.
+__host__ __device__ __forceinline__ uint32_t make_idesc_nvf4(bool sparse, uint32_t M, uint32_t N) {
+  uint32_t d = 0;
+  if (sparse) d |= 1u << 2;
+  d |= 1u << 7;
+  d |= 1u << 10;
+  d |= ((N >> 3) & 0x3Fu) << 17;
+  d |= ((M >> 4) & 0x1Fu) << 24;
+  return d;
+}
+
+// Shared -> tensor memory copy of a 32-row x 128-bit matrix into all four
+// 32-lane quarters: source row i lands in lanes i, 32 + i, 64 + i and 96 + i,
+// four consecutive 32-bit columns (a 512-byte scale chunk).
+__device__ __forceinline__ void tc_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
 // Shared -> tensor memory copy of a 128-row x 128-bit matrix: source row i
 // lands in lane i, four consecutive 32-bit columns.
 __device__ __forceinline__ void tc_cp_128x128b(uint32_t taddr, uint64_t sdesc) {

@@ -59,6 +59,19 @@ class GemmArgs(ctypes.Structure):
     ]
 
 
+class Nvfp4GemmArgs(ctypes.Structure):
+    _fields_ = [
+        ("M", ctypes.c_int64), ("N", ctypes.c_int64), ("K", ctypes.c_int64),
+        ("tactic", ctypes.c_int), ("out_dtype", ctypes.c_int),
+        ("X", ctypes.c_void_p), ("x_scales", ctypes.c_void_p), ("x_tensor_scale", ctypes.c_void_p),
+        ("W", ctypes.c_void_p), ("W_meta", ctypes.c_void_p), ("w_scales", ctypes.c_void_p),
+        ("w_tensor_scale", ctypes.c_void_p),
+        ("Y", ctypes.c_void_p), ("ldy", ctypes.c_int64),
+        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+        ("flags", ctypes.c_uint32),
+    ]
+
+
 class QuantItem(ctypes.Structure):
     _fields_ = [
         ("src", ctypes.c_void_p), ("rows", ctypes.c_int64), ("K", ctypes.c_int64),
@@ -114,6 +127,14 @@ def lib() -> ctypes.CDLL:
                                                            P, P, P, P, ctypes.c_size_t, P]),
         "sp24_select_tactic": (I, [ctypes.POINTER(GemmArgs), ctypes.POINTER(GemmArgs), I, I,
                                    ctypes.POINTER(TacticRecord), P]),
+        "sp24_nvfp4_48_values_bytes": (ctypes.c_size_t, [I64, I64]),
+        "sp24_nvfp4_48_meta_bytes": (ctypes.c_size_t, [I64, I64]),
+        "sp24_nvfp4_codes_bytes": (ctypes.c_size_t, [I64, I64]),
+        "sp24_nvfp4_scales_bytes": (ctypes.c_size_t, [I64, I64, I]),
+        "sp24_prune_compress_nvfp4_48": (I, [P, I64, I64, I64, P, P, P, P, P]),
+        "sp24_quantize_nvfp4": (I, [P, I64, I64, I64, I, P, P, P, P]),
+        "sp24_gemm_nvfp4_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(Nvfp4GemmArgs)]),
+        "sp24_gemm_nvfp4": (I, [ctypes.POINTER(Nvfp4GemmArgs), P]),
         "sp24_status_string": (ctypes.c_char_p, [I]),
         "sp24_last_device_error": (I, []),
         "sp24_clear_device_error": (I, []),
@@ -398,6 +419,75 @@ def select_tactic(sparse_args: Optional[GemmArgs], dense_args: GemmArgs, warmup:
                 iters=rec.iters, eligible=bool(rec.eligible),
                 selected="sparse" if rec.selected == SPARSE else "dense",
                 reason=rec.reason.decode())
+
+
+# ---------------------------------------------------------------------------
+# pairwise 4:8 sparse NVFP4 and dense NVFP4
+# ---------------------------------------------------------------------------
+
+def nvfp4_48_values_bytes(rows: int, K: int) -> int:
+    return lib().sp24_nvfp4_48_values_bytes(rows, K)
+
+
+def nvfp4_48_meta_bytes(rows: int, K: int) -> int:
+    return lib().sp24_nvfp4_48_meta_bytes(rows, K)
+
+
+def nvfp4_codes_bytes(rows: int, K: int) -> int:
+    return lib().sp24_nvfp4_codes_bytes(rows, K)
+
+
+def nvfp4_scales_bytes(rows: int, K: int, block: int) -> int:
+    return lib().sp24_nvfp4_scales_bytes(rows, K, block)
+
+
+def prune_compress_nvfp4_48(src: torch.Tensor, values: torch.Tensor, meta: torch.Tensor, scales: torch.Tensor,
+                            tensor_scale: torch.Tensor, stream=None):
+    """Pairwise 4:8 prune + NVFP4 cast of a bf16 matrix: values [rows, K/4],
+    metadata image, scale image (per 32 positions), tensor scale (fp32 [1])."""
+    rows, K = src.shape
+    _check(lib().sp24_prune_compress_nvfp4_48(_ptr(src), rows, K, src.stride(0), _ptr(values), _ptr(meta),
+                                              _ptr(scales), _ptr(tensor_scale), _stream(stream)),
+           "sp24_prune_compress_nvfp4_48")
+
+
+def quantize_nvfp4(src: torch.Tensor, block: int, codes: torch.Tensor, scales: torch.Tensor,
+                   tensor_scale: torch.Tensor, stream=None):
+    """Dense NVFP4 cast of a bf16 matrix, one scale per `block` (16 or 32)."""
+    rows, K = src.shape
+    _check(lib().sp24_quantize_nvfp4(_ptr(src), rows, K, src.stride(0), block, _ptr(codes), _ptr(scales),
+                                     _ptr(tensor_scale), _stream(stream)), "sp24_quantize_nvfp4")
+
+
+def nvfp4_gemm_args(X: torch.Tensor, x_scales: torch.Tensor, x_ts: torch.Tensor, W: torch.Tensor,
+                    w_scales: torch.Tensor, w_ts: torch.Tensor, Y: torch.Tensor, K: int, tactic: int,
+                    W_meta: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                    flags: int = 0) -> Nvfp4GemmArgs:
+    """Y [M x N] = X * W^T with NVFP4 operands: X codes [M, K/2] (+ scale
+    image, tensor scale); W sparse values [N, K/4] + metadata image, or dense
+    codes [N, K/2] (+ scale image, tensor scale)."""
+    a = Nvfp4GemmArgs()
+    a.M, a.N, a.K = X.shape[0], Y.shape[1], K
+    a.tactic = tactic
+    a.out_dtype = dtype_code(Y.dtype)
+    a.X, a.x_scales, a.x_tensor_scale = X.data_ptr(), x_scales.data_ptr(), x_ts.data_ptr()
+    a.W, a.w_scales, a.w_tensor_scale = W.data_ptr(), w_scales.data_ptr(), w_ts.data_ptr()
+    a.W_meta = W_meta.data_ptr() if W_meta is not None else None
+    a.Y, a.ldy = Y.data_ptr(), Y.stride(0)
+    a.flags = flags
+    if workspace is not None:
+        a.workspace = workspace.data_ptr()
+        a.workspace_bytes = workspace.numel() * workspace.element_size()
+    a._keep = [X, x_scales, x_ts, W, w_scales, w_ts, W_meta, Y, workspace]
+    return a
+
+
+def gemm_nvfp4_workspace_bytes(args: Nvfp4GemmArgs) -> int:
+    return lib().sp24_gemm_nvfp4_workspace_bytes(ctypes.byref(args))
+
+
+def gemm_nvfp4(args: Nvfp4GemmArgs, stream=None):
+    _check(lib().sp24_gemm_nvfp4(ctypes.byref(args), _stream(stream)), "sp24_gemm_nvfp4")
 
 
 # ---------------------------------------------------------------------------

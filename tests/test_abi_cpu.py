@@ -206,3 +206,57 @@ def test_binding_constants_match_the_header():
     # flag bits are distinct
     vals = list(defines.values())
     assert all(v & (v - 1) == 0 for v in vals) and len(set(vals)) == len(vals)
+
+
+def test_nvfp4_sizes():
+    assert sp24.nvfp4_48_values_bytes(256, 512) == 256 * 128          # 2 bits of value per position
+    assert sp24.nvfp4_48_meta_bytes(256, 512) == 2 * 2 * 2048         # 4 bits per 8 positions
+    assert sp24.nvfp4_48_meta_bytes(40, 256) == 2048                  # rows padded to 128
+    assert sp24.nvfp4_codes_bytes(10, 512) == 2560
+    assert sp24.nvfp4_scales_bytes(200, 512, 32) == 256 * 16
+    assert sp24.nvfp4_scales_bytes(200, 512, 16) == 256 * 32
+    assert sp24.nvfp4_scales_bytes(200, 512, 8) == 0
+    # 4:8 NVFP4 stores 2 + 0.5 bits per position of values and metadata
+    # plus 8 bits per 32 positions of scales: 2.75 bits against dense NVFP4's 4.5
+    rows, K = 1024, 4096
+    sparse = sp24.nvfp4_48_values_bytes(rows, K) + sp24.nvfp4_48_meta_bytes(rows, K) + \
+        sp24.nvfp4_scales_bytes(rows, K, 32)
+    dense = sp24.nvfp4_codes_bytes(rows, K) + sp24.nvfp4_scales_bytes(rows, K, 16)
+    assert sparse * 8 == rows * K * 2.75 and dense * 8 == rows * K * 4.5
+
+
+def nvgemm(**kw):
+    a = sp24.Nvfp4GemmArgs()
+    a.M, a.N, a.K = kw.get("M", 16), kw.get("N", 256), kw.get("K", 512)
+    a.tactic = kw.get("tactic", sp24.SPARSE)
+    a.out_dtype = kw.get("out_dtype", sp24.BF16)
+    for f in ("X", "x_scales", "x_tensor_scale", "W", "W_meta", "w_scales", "w_tensor_scale", "Y"):
+        setattr(a, f, kw.get(f, FAKE))
+    a.ldy = kw.get("ldy", a.N)
+    return L.sp24_gemm_nvfp4(ctypes.byref(a), None)
+
+
+def test_nvfp4_validation():
+    assert L.sp24_gemm_nvfp4(None, None) == sp24.SP24_ERR_NULL
+    assert nvgemm(M=0) == sp24.SP24_ERR_INVALID_ARG
+    assert nvgemm(tactic=5) == sp24.SP24_ERR_INVALID_ARG
+    assert nvgemm(out_dtype=sp24.E4M3) == sp24.SP24_ERR_DTYPE
+    assert nvgemm(W_meta=None) == sp24.SP24_ERR_NULL
+    assert nvgemm(tactic=sp24.DENSE, W_meta=None) != sp24.SP24_ERR_NULL  # dense needs no metadata
+    assert nvgemm(x_tensor_scale=None) == sp24.SP24_ERR_NULL
+    assert nvgemm(K=384) == sp24.SP24_ERR_NOT_2_4
+    assert nvgemm(tactic=sp24.DENSE, K=384) == sp24.SP24_ERR_ALIGNMENT
+    assert nvgemm(X=FAKE + 8) == sp24.SP24_ERR_ALIGNMENT
+    assert nvgemm(ldy=100) == sp24.SP24_ERR_INVALID_ARG
+    P = L.sp24_prune_compress_nvfp4_48
+    assert P(None, 128, 512, 512, FAKE, FAKE, FAKE, FAKE, None) == sp24.SP24_ERR_NULL
+    assert P(FAKE, 128, 384, 384, FAKE, FAKE, FAKE, FAKE, None) == sp24.SP24_ERR_NOT_2_4
+    assert P(FAKE, 0, 512, 512, FAKE, FAKE, FAKE, FAKE, None) == sp24.SP24_ERR_INVALID_ARG
+    assert P(FAKE, 128, 512, 516, FAKE, FAKE, FAKE, FAKE, None) == sp24.SP24_ERR_ALIGNMENT
+    Q = L.sp24_quantize_nvfp4
+    assert Q(FAKE, 16, 512, 512, 8, FAKE, FAKE, FAKE, None) == sp24.SP24_ERR_INVALID_ARG
+    assert Q(FAKE, 16, 96, 96, 16, FAKE, FAKE, FAKE, None) == sp24.SP24_ERR_ALIGNMENT
+    assert Q(FAKE, 16, 512, 512, 32, FAKE, FAKE, FAKE + 2, None) == sp24.SP24_ERR_ALIGNMENT
+    if NO_GPU:
+        assert nvgemm() == sp24.SP24_ERR_UNSUPPORTED_DEVICE
+        assert P(FAKE, 128, 512, 512, FAKE, FAKE, FAKE, FAKE, None) == sp24.SP24_ERR_UNSUPPORTED_DEVICE

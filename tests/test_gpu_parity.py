@@ -480,6 +480,30 @@ def test_grouped_rejects_mixed_hybrid_and_plain_weights():
     assert st == sp24.SP24_ERR_INVALID_ARG
 
 
+@pytest.mark.parametrize("M,N,K", [(8, 256, 640), (130, 384, 128), (1, 128, 1152), (33, 512, 1536)])
+@pytest.mark.parametrize("kind", ["random", "checkerboard", "all_dense", "all_sparse", "odd_columns"])
+def test_hybrid_stage_kinds(M, N, K, kind):
+    """One-CTA hybrid stages cover two tile columns: both sparse, both dense,
+    mixed either way, and a single last column when K / 128 is odd."""
+    RB, KT = N // 128, K // 128
+    if kind == "random":
+        mask = inputs.hybrid_mask(N, K, seed=K)
+    elif kind == "checkerboard":
+        mask = ((np.arange(RB)[:, None] + np.arange(KT)[None, :]) % 2).astype(np.uint8)
+    elif kind == "all_dense":
+        mask = np.ones((RB, KT), np.uint8)
+    elif kind == "all_sparse":
+        mask = np.zeros((RB, KT), np.uint8)
+    else:  # every odd column dense: each stage is sparse then dense
+        mask = np.zeros((RB, KT), np.uint8)
+        mask[:, 1::2] = 1
+    X, W = inputs.linear_pair(M, N, K, seed=M + N + K, outliers=True)
+    for use_ws in (True, False):
+        y, y_ref, a_ref, _, _ = run_gemm(X, W, True, sp24.SPARSE, True, mask=mask, use_ws=use_ws,
+                                         flags=sp24.GEMM_W_STATIC | sp24.GEMM_SINGLE_CTA)
+        check_tolerance(y, y_ref, a_ref, "hybrid kinds %s M%d N%d K%d ws=%s" % (kind, M, N, K, use_ws))
+
+
 def _pair_mask(kind, N, K, seed):
     RB, KT = N // 128, K // 128
     if kind == "random":
@@ -699,8 +723,10 @@ def _prepare_large(X_bits, W_bits, e4, tactic):
 
 
 @pytest.mark.parametrize("M,N,K", [(128, 384, 512), (200, 256, 1280), (1, 128, 128), (512, 384, 512),
-                                   (300, 640, 768)])
+                                   (300, 640, 768), (5, 256, 32768)])
 def test_activation_fused_e4m3_parity(M, N, K):
+    # rows up to 28672 wide take the one-pass kernel (row in registers); the
+    # 32768-wide case takes the amax / prune / scale passes
     # X pruned 2:4 and cast to e4m3 per token on every call; the compressed
     # activations are bit-exact to the oracle's, Y within tolerance
     X = inputs.student_t_bf16((M, K), 3.0, seed=M + 7 * K)
@@ -832,6 +858,51 @@ def test_prefill_full_size_sampled(e4):
     check_tolerance(y_gpu, y_ref, a_ref, "prefill e4=%s" % e4)
 
 
+@pytest.mark.parametrize("M,N,K", [(16384, 12288, 4096), (8192, 4096, 12288)])
+@pytest.mark.parametrize("e4", [False, True])
+def test_prefill_largest_shapes_full_size_sampled(M, N, K, e4):
+    """The largest prefill shapes (many 256 x 256 tiles per CTA pair, K up to
+    12288) on device-pruned weights with outliers; sampled outputs against the
+    oracle."""
+    X, W = inputs.linear_pair(M, N, K, seed=M + K, outliers=True)
+    a, Y, _, _ = _prepare_large(X, W, e4, sp24.SPARSE)
+    sp24.gemm(a)
+    torch.cuda.synchronize()
+    assert sp24.last_device_error() == sp24.SP24_OK
+    g = np.random.default_rng(M + N)
+    ms = np.concatenate([g.integers(0, M, size=40), [0, M - 1]])
+    ns = np.concatenate([g.integers(0, N, size=40), [0, N - 1]])
+    W_hat = OracleSparseW(W[ns], e4m3=e4).W_hat
+    _, _, X_hat = oracle_x(X[ms], e4)
+    y_ref, a_ref = orc.gemm_f64_sampled(X_hat, W_hat, np.arange(ms.size), np.arange(ns.size))
+    y_gpu = Y.float().cpu().numpy().astype(np.float64)[ms, ns]
+    check_tolerance(y_gpu, y_ref, a_ref, "prefill M%d N%d K%d e4=%s" % (M, N, K, e4))
+
+
+def test_tiny_configuration_seed0_matches_oracle():
+    """The tiny configuration exactly as specified (X[16 x 256] ~ N(0,1),
+    W[256 x 256] ~ N(0, 0.02^2), seed 0): W pruned and compressed on the
+    device (values and metadata bit-exact to the oracle), then Y = X W^T with
+    fp32 accumulation, bf16 and e4m3, within tolerance of the fp64 oracle."""
+    X, W = inputs.tiny(0)
+    M, K = X.shape
+    N = W.shape[0]
+    vals = torch.empty(N, K // 2, dtype=torch.bfloat16, device="cuda")
+    meta = torch.empty(sp24.meta_bytes(N, K), dtype=torch.uint8, device="cuda")
+    sp24.prune_compress(dev_bf16(W), sp24.BF16, vals, meta)
+    pruned, values, canon = orc.prune_compress_bf16(W)
+    assert np.array_equal(bits16(vals), values)
+    assert np.array_equal(u8(meta), orc.meta_image(canon, N, K, False))
+    assert (values.reshape(N, K // 2).shape == (256, 128))
+    Y = torch.empty(M, N, dtype=torch.float32, device="cuda")
+    sp24.gemm(sp24.gemm_args(dev_bf16(X), vals, Y, K, sp24.SPARSE, W_meta=meta))
+    torch.cuda.synchronize()
+    y_ref, a_ref = orc.gemm_f64(orc.bf16_bits_to_f64(X), orc.bf16_bits_to_f64(pruned))
+    check_tolerance(Y.cpu().numpy().astype(np.float64), y_ref, a_ref, "tiny bf16")
+    y, y_ref, a_ref, _, _ = run_gemm(X, W, True, sp24.SPARSE, True)
+    check_tolerance(y, y_ref, a_ref, "tiny e4m3")
+
+
 def test_decode_step_full_size_grouped_sampled():
     """The decode step as the benchmark times it: 16 GEMMs (M in 1, 8, 32, 128
     times the four weight shapes, e4m3 2:4 weights), one grouped per-token cast,
@@ -882,7 +953,8 @@ def test_decode_step_full_size_grouped_sampled():
         check_tolerance(y_gpu, y_ref, a_ref, "decode step M%d %dx%d" % (M, N, K))
 
 
-@pytest.mark.parametrize("name,M", [("gate_up", 4096), ("qkv", 16)])
+@pytest.mark.parametrize("name,M", [("gate_up", 4096), ("qkv", 16), ("o", 1), ("o", 256), ("down", 1),
+                                    ("down", 256)])
 def test_hybrid_full_size_sampled(name, M):
     """Hybrid weights (25% dense 128 x 128 tiles, e4m3) at full size: gate_up at
     4096 tokens runs on CTA pairs, qkv at 16 tokens on single CTAs.  The
