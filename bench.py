@@ -50,7 +50,7 @@ def parse():
     p.add_argument("--no-configs", action="store_true",
                    help="leave the other workloads' rows (prefill, activations, hybrid) out of the line")
     p.add_argument("--config", default="decode",
-                   choices=["decode", "tiny", "prefill", "activation", "hybrid", "prune"],
+                   choices=["decode", "tiny", "prefill", "activation", "hybrid", "prune", "nvfp4"],
                    help="decode (default): the headline step line.  The others time the other "
                         "workloads of the hot path, one JSON line each, eager calls with an L2 "
                         "flush before every timed call")
@@ -694,8 +694,9 @@ def run_group_case(args):
 
 def run_other_case(args):
     """prune:N,K,bf16|e4m3 -- the weight prune / compress of N x K;
-    act:M,N,K,bf16|e4m3 -- the online-activation path (prune of X every call,
-    then the sparse GEMM); nv:M,N,K,sparse|dense -- the NVFP4 GEMM (pairwise
+    act:M,N,K,bf16|e4m3|ingemm -- the online-activation path (prune of X every
+    call, then the sparse GEMM; ingemm: the prune inside the GEMM kernel);
+    nv:M,N,K,sparse|dense -- the NVFP4 GEMM (pairwise
     4:8 or dense), X cast to NVFP4 once.  Eager calls, CUDA-event timing, L2
     flushed before each call (for profiler captures)."""
     import torch
@@ -725,6 +726,8 @@ def run_other_case(args):
             sp24.quantize_e4m3_rows(W, Wq, wsc)
             ws = torch.empty(sp24.activations_e4m3_workspace_bytes(M, K), dtype=torch.uint8, device=dev)
             fn = lambda: sp24.prune_compress_activations_fused_e4m3(X, Wq, wsc, Y, workspace=ws)  # noqa: E731
+        elif len(f) > 3 and f[3] == "ingemm":
+            fn = lambda: sp24.prune_activations_in_gemm(X, W, Y)  # noqa: E731
         else:
             ws = torch.empty(sp24.activations_workspace_bytes(M, K), dtype=torch.uint8, device=dev)
             fn = lambda: sp24.prune_compress_activations_fused(X, W, Y, workspace=ws)  # noqa: E731
@@ -1084,6 +1087,16 @@ def cfg_activation(dev, T):
                      selected="sparse" if t_f < t_d else "dense", _win=_win(w1, w2),
                      note="fused = prune+compress of X every call, then the sparse GEMM with X as "
                           "the sparse operand; dense = the in-build dense GEMM on unpruned X"))
+    # the prune inside the GEMM kernel (no compressed X in HBM)
+    t_g, _, w3 = T.calls(lambda: sp24.prune_activations_in_gemm(X, W, Y))
+    rows.append(dict(gemm="activation_in_gemm", M=M, N=N, K=K, dtype="bf16",
+                     us_fused=round(t_g, 2), us_dense=round(t_d, 2), us_two_kernel=round(t_f, 2),
+                     tflops_fused=round(F / t_g / 1e6, 1), speedup_vs_dense=round(t_d / t_g, 3),
+                     speedup_vs_two_kernel=round(t_f / t_g, 3),
+                     roofline_fused=_roofline(F, 2 * M * K + 2 * N * K + 2 * M * N, t_g, T.peak(True, False), T.hbm),
+                     selected="sparse" if t_g < t_d else "dense", _win=_win(w3, w2),
+                     note="X pruned and compressed in shared memory by converter warps of the CTA-pair GEMM "
+                          "(re-pruned for every 256-row block of W), no compressed X in HBM"))
     # the same at the FP8 floor: X pruned and cast to e4m3 per token every call, W e4m3 per channel
     Wq = torch.empty(N, K, dtype=torch.uint8, device=dev)
     wsc = torch.empty(N, dtype=torch.float32, device=dev)
@@ -1228,6 +1241,70 @@ def cfg_hybrid_block(dev, T, Ms):
     return rows
 
 
+def cfg_nvfp4(dev, T, shapes):
+    """Pairwise 4:8 sparse NVFP4 against dense NVFP4 (the Blackwell sparse FP4
+    format, 2:4-versus-quantization paper section 6.2) on linear-layer
+    shapes: W pruned and cast offline, X cast to NVFP4 once (outside the
+    timed call), the block-scaled GEMM timed.  Peaks: FP4 4x the measured
+    bf16 dense figure, sparse 2x that (nominal ratios)."""
+    import torch
+
+    from semi_structured_sparse_02_b200 import inputs, sp24
+    rows = []
+    for (M, N, K) in shapes:
+        W = _bf16_dev(inputs.normal_bf16((N, K), 0.02, seed=N + K), dev)
+        X = _bf16_dev(inputs.normal_bf16((M, K), 1.0, seed=M + K), dev)
+        ops = {}
+        for sparse in (True, False):
+            blk = 32 if sparse else 16
+            xc = torch.empty(M, K // 2, dtype=torch.uint8, device=dev)
+            xs = torch.empty(sp24.nvfp4_scales_bytes(M, K, blk), dtype=torch.uint8, device=dev)
+            xts = torch.empty(1, dtype=torch.float32, device=dev)
+            sp24.quantize_nvfp4(X, blk, xc, xs, xts)
+            wts = torch.empty(1, dtype=torch.float32, device=dev)
+            wsc = torch.empty(sp24.nvfp4_scales_bytes(N, K, blk), dtype=torch.uint8, device=dev)
+            meta = None
+            if sparse:
+                wv = torch.empty(N, K // 4, dtype=torch.uint8, device=dev)
+                meta = torch.empty(sp24.nvfp4_48_meta_bytes(N, K), dtype=torch.uint8, device=dev)
+                sp24.prune_compress_nvfp4_48(W, wv, meta, wsc, wts)
+            else:
+                wv = torch.empty(N, K // 2, dtype=torch.uint8, device=dev)
+                sp24.quantize_nvfp4(W, 16, wv, wsc, wts)
+            Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+            a = sp24.nvfp4_gemm_args(xc, xs, xts, wv, wsc, wts, Y, K, sp24.SPARSE if sparse else sp24.DENSE,
+                                     W_meta=meta)
+            n = sp24.gemm_nvfp4_workspace_bytes(a)
+            if n:
+                wsp = torch.zeros(n, dtype=torch.uint8, device=dev)
+                a.workspace, a.workspace_bytes = wsp.data_ptr(), n
+                a._keep.append(wsp)
+            ops[sparse] = a
+        t_sp, _, w1 = T.calls(lambda: sp24.gemm_nvfp4(ops[True]))
+        t_dn, _, w2 = T.calls(lambda: sp24.gemm_nvfp4(ops[False]))
+        F = 2.0 * M * N * K
+        b_sp = N * K * (0.25 + 1 / 16 + 1 / 32) + M * K * (0.5 + 1 / 32) + 2 * M * N
+        b_dn = N * K * (0.5 + 1 / 16) + M * K * (0.5 + 1 / 16) + 2 * M * N
+        rows.append(dict(gemm="nvfp4", M=M, N=N, K=K, dtype="nvfp4",
+                         us_sparse=round(t_sp, 2), us_dense=round(t_dn, 2),
+                         tflops_sparse=round(F / t_sp / 1e6, 1), tflops_dense=round(F / t_dn / 1e6, 1),
+                         gbs_sparse=round(b_sp / t_sp / 1e3, 1), gbs_dense=round(b_dn / t_dn / 1e3, 1),
+                         speedup_vs_dense=round(t_dn / t_sp, 3),
+                         selected="sparse" if t_sp < t_dn else "dense",
+                         roofline_sparse=_roofline(F, b_sp, t_sp, 8 * T.bf16_tf, T.hbm),
+                         roofline_dense=_roofline(F, b_dn, t_dn, 4 * T.bf16_tf, T.hbm),
+                         _win=_win(w1, w2)))
+        print(json.dumps({k: v for k, v in rows[-1].items() if not k.startswith("_")}), file=sys.stderr,
+              flush=True)
+        del ops, W, X
+        torch.cuda.empty_cache()
+    return rows
+
+
+NVFP4_SHAPES = [(8, N, K) for N, K in [(5120, 5120), (25600, 5120), (5120, 25600), (10240, 5120)]] + \
+    [(128, 5120, 25600), (8192, 4096, 4096), (8192, 12288, 4096)]
+
+
 def cfg_prune(dev, T):
     import torch
 
@@ -1300,6 +1377,8 @@ def run_config(args):
         rows = cfg_activation(dev, T)
     elif args.config == "prune":
         rows = cfg_prune(dev, T)
+    elif args.config == "nvfp4":
+        rows = cfg_nvfp4(dev, T, NVFP4_SHAPES)
     time.sleep(0.2)
     sampler.stop()
     out["rows"] = _finish_rows(rows, sampler)
@@ -1311,7 +1390,9 @@ def run_configs_compact(dev):
     """The other workloads in brief, for the default bench line: prefill at
     16384 tokens (every weight shape, bf16 and e4m3), the online-activation
     paths (bf16 and FP8), the hybrid block's GEMMs alone at 1 and 4096 tokens,
-    the hybrid block step at 1, 16 and 256 tokens, and the tiny case.  Each
+    the hybrid block step at 1, 16 and 256 tokens, the tiny case, and
+    pairwise 4:8 NVFP4 against dense NVFP4 at two decode shapes and one
+    prefill shape.  Each
     row: sparse and dense device time, roofline fraction against the measured
     peaks, the selected tactic, and the clocks sampled during its timing."""
     import torch
@@ -1332,6 +1413,8 @@ def run_configs_compact(dev):
     out["hybrid_block"] = cfg_hybrid_block(dev, T, [1, 16, 256])
     torch.cuda.empty_cache()
     out["tiny"] = cfg_tiny(dev, T)
+    torch.cuda.empty_cache()
+    out["nvfp4"] = cfg_nvfp4(dev, T, [(8, 25600, 5120), (128, 5120, 25600), (8192, 4096, 4096)])
     time.sleep(0.2)
     sampler.stop()
     keep = ("gemm", "block_step", "M", "N", "K", "dtype", "us_sparse", "us_dense", "us_fused", "us_hybrid",

@@ -328,6 +328,23 @@ int sp24_prune_compress_activations_fused(const void *X_dev, int64_t M, int64_t 
                                           void *workspace_dev, size_t workspace_bytes,
                                           void *stream);
 
+/* The online-activation path with the prune inside the GEMM: every call, a
+ * CTA-pair GEMM loads raw bf16 X tiles with TMA and prunes + compresses them
+ * in shared memory (converter warps of the GEMM kernel itself, same rule and
+ * layouts as sp24_prune_compress), then Y [M x N] = X_pruned * W^T with W
+ * dense bf16 [N x K], X as the sparse operand.  No compressed copy of X goes
+ * through HBM ("Measuring speed", section 3.5 of the 2:4-versus-quantization
+ * paper: a dynamic operand pays for its own prune; the two-kernel path of
+ * sp24_prune_compress_activations_fused writes and re-reads it).  The prune of
+ * an X tile is repeated for every 256-row block of W it meets.
+ *   x_values_dev / x_meta_dev: NULL (both), or where the compressed X also
+ *   goes ([M x K/2] bf16 and the image of M rows), for inspection.
+ * Requirements: M >= 256, N >= 256, K % 128 == 0, ldx % 8 == 0, ldw % 8 == 0,
+ * 16-byte aligned pointers.  Asynchronous on `stream`. */
+int sp24_prune_activations_in_gemm(const void *X_dev, int64_t M, int64_t K, int64_t ldx, const void *W_dev,
+                                   int64_t N, int64_t ldw, void *Y_dev, int64_t ldy, sp24_dtype out_dtype,
+                                   void *x_values_dev, void *x_meta_dev, void *stream);
+
 /* The online-activation path at the FP8 floor: per call, X (bf16 [M x K])
  * is pruned 2:4 along K on its bf16 magnitudes (same rule as
  * sp24_prune_compress), the kept values are cast to E4M3 with one fp32 scale

@@ -21,6 +21,7 @@
 #include "nvfp4.cuh"
 #include "gemm.cuh"
 #include "gemm_wide.cuh"
+#include "gemm_wide_prune.cuh"
 
 namespace sp24 {
 namespace {
@@ -751,6 +752,71 @@ int run_wide(int mode, bool bf16, bool a_is_w, const void* A, int64_t lda, const
                 : launch_wide_inst<kModeSparse, false, true>(wl, stream);
   return bf16 ? launch_wide_inst<kModeDense, true, true>(wl, stream)
               : launch_wide_inst<kModeDense, false, true>(wl, stream);
+}
+
+// The CTA-pair GEMM that prunes X (bf16) in its producer (no compressed copy
+// of X in HBM unless asked for): Y [M x N] = prune(X) * W^T.
+int run_wide_prune(const void* X, int64_t ldx, const void* W, int64_t ldw, int64_t M, int64_t N, int64_t K, void* Y,
+                   int64_t ldy, bool out_f32, void* x_values_out, void* x_meta_out, cudaStream_t stream) {
+  using C = WidePruneCfg;
+  static std::atomic<int> max_pairs[kMaxDevices];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= kMaxDevices) return SP24_ERR_UNSUPPORTED_DEVICE;
+  const bool emit = x_values_out != nullptr;
+  auto fn = emit ? k_gemm_wide_prune<true> : k_gemm_wide_prune<false>;
+  int pairs_cap = max_pairs[dev].load();
+  if (pairs_cap <= 0) {
+    for (auto f : {k_gemm_wide_prune<true>, k_gemm_wide_prune<false>})
+      if (cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess) {
+        cudaGetLastError();
+        return SP24_ERR_CUDA;
+      }
+    cudaLaunchConfig_t q = {};
+    q.gridDim = dim3(2);
+    q.blockDim = dim3(kPruneGemmThreads);
+    q.dynamicSmemBytes = C::kSmemBytes;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, k_gemm_wide_prune<false>, &q) != cudaSuccess || n < 1) {
+      cudaGetLastError();
+      return SP24_ERR_CUDA;
+    }
+    pairs_cap = n;
+    max_pairs[dev].store(n);
+  }
+  static thread_local WidePruneLaunch wl;
+  memset(&wl, 0, sizeof wl);
+  bool ok = make_map(&wl.tm_x, X, 2, K, M, ldx * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= make_map(&wl.tm_b, W, 2, K, N, ldw * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!ok) return SP24_ERR_CUDA;
+  wl.rows_a = (int32_t)M;
+  wl.rows_b = (int32_t)N;
+  wl.K = (int32_t)K;
+  wl.num_kt = (int32_t)(K / 128);
+  wl.tiles_a = (int32_t)((M + 255) / 256);
+  wl.tiles_b = (int32_t)((N + 255) / 256);
+  wl.total_tiles = wl.tiles_a * wl.tiles_b;
+  // W (the dense operand, re-read for every X tile) fastest when it fits in
+  // L2 easily, so that each X tile is read from HBM once
+  wl.b_fastest = ((double)N * (double)K * 2 <= 32.0 * 1024 * 1024) ? 1 : 0;
+  wl.out_f32 = out_f32 ? 1 : 0;
+  wl.use_pdl = 1;
+  wl.Y = Y;
+  wl.ldy = ldy;
+  wl.x_values_out = static_cast<uint16_t*>(x_values_out);
+  wl.x_meta_out = static_cast<uint8_t*>(x_meta_out);
+  wl.timeout_ns = g_timeout_ns.load();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * std::max(1, std::min(wl.total_tiles, pairs_cap)));
+  cfg.blockDim = dim3(kPruneGemmThreads);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return launch_result(cudaLaunchKernelEx(&cfg, fn, wl));
 }
 
 int run_gemm(const sp24_gemm_args* a, cudaStream_t stream) {
@@ -1499,6 +1565,25 @@ int sp24_prune_compress_activations_fused(const void* X, int64_t M, int64_t K, i
   // GEMM with X (compressed) as the sparse operand A and W dense as B.
   return run_activation_gemm(true, x_values, x_meta, nullptr, W, ldw, nullptr, M, N, K, Y, ldy,
                              out_dtype == SP24_F32, di, s);
+}
+
+int sp24_prune_activations_in_gemm(const void* X, int64_t M, int64_t K, int64_t ldx, const void* W, int64_t N,
+                                   int64_t ldw, void* Y, int64_t ldy, sp24_dtype out_dtype, void* x_values, void* x_meta,
+                                   void* stream) {
+  if (X == nullptr || W == nullptr || Y == nullptr) return SP24_ERR_NULL;
+  if ((x_values == nullptr) != (x_meta == nullptr)) return SP24_ERR_NULL;
+  if (out_dtype != SP24_BF16 && out_dtype != SP24_F32) return SP24_ERR_DTYPE;
+  if (M < 256 || N < 256 || K < 128 || ldx < K || ldw < K || ldy < N) return SP24_ERR_INVALID_ARG;
+  if (M > INT32_MAX / 2 || N > INT32_MAX / 2 || K > INT32_MAX / 2) return SP24_ERR_INVALID_ARG;
+  if (K % 128 != 0) return SP24_ERR_NOT_2_4;
+  if (ldx % 8 != 0 || ldw % 8 != 0 || !aligned16(X) || !aligned16(W)) return SP24_ERR_ALIGNMENT;
+  if (!aligned16(Y) || (ldy * (out_dtype == SP24_F32 ? 4 : 2)) % 16 != 0) return SP24_ERR_ALIGNMENT;
+  if (x_values != nullptr && (!aligned16(x_values) || !aligned16(x_meta))) return SP24_ERR_ALIGNMENT;
+  DeviceInfo di;
+  int st = current_device_info(&di);
+  if (st != SP24_OK) return st;
+  return run_wide_prune(X, ldx, W, ldw, M, N, K, Y, ldy, out_dtype == SP24_F32, x_values, x_meta,
+                        static_cast<cudaStream_t>(stream));
 }
 
 int sp24_select_tactic(const sp24_gemm_args* sparse_args, const sp24_gemm_args* dense_args, int warmup,

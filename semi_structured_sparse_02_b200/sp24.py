@@ -135,6 +135,7 @@ def lib() -> ctypes.CDLL:
         "sp24_quantize_nvfp4": (I, [P, I64, I64, I64, I, P, P, P, P]),
         "sp24_gemm_nvfp4_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(Nvfp4GemmArgs)]),
         "sp24_gemm_nvfp4": (I, [ctypes.POINTER(Nvfp4GemmArgs), P]),
+        "sp24_prune_activations_in_gemm": (I, [P, I64, I64, I64, P, I64, I64, P, I64, I, P, P, P]),
         "sp24_status_string": (ctypes.c_char_p, [I]),
         "sp24_last_device_error": (I, []),
         "sp24_clear_device_error": (I, []),
@@ -377,6 +378,18 @@ def prune_compress_activations_fused(X: torch.Tensor, W: torch.Tensor, Y: torch.
         _ptr(X), M, K, X.stride(0), _ptr(W), N, W.stride(0), _ptr(Y), Y.stride(0),
         dtype_code(Y.dtype), _ptr(x_values), _ptr(x_meta), _ptr(workspace), ws_bytes,
         _stream(stream)), "sp24_prune_compress_activations_fused")
+
+
+def prune_activations_in_gemm(X: torch.Tensor, W: torch.Tensor, Y: torch.Tensor,
+                              x_values: Optional[torch.Tensor] = None, x_meta: Optional[torch.Tensor] = None,
+                              stream=None):
+    """Y = prune(X) * W^T with the prune done inside the GEMM kernel (X, W
+    bf16; x_values / x_meta optionally receive the compressed X)."""
+    M, K = X.shape
+    N = W.shape[0]
+    _check(lib().sp24_prune_activations_in_gemm(
+        _ptr(X), M, K, X.stride(0), _ptr(W), N, W.stride(0), _ptr(Y), Y.stride(0), dtype_code(Y.dtype),
+        _ptr(x_values), _ptr(x_meta), _stream(stream)), "sp24_prune_activations_in_gemm")
 
 
 def energy_loss(src: torch.Tensor, row_share: Optional[torch.Tensor] = None,

@@ -260,3 +260,24 @@ def test_nvfp4_validation():
     if NO_GPU:
         assert nvgemm() == sp24.SP24_ERR_UNSUPPORTED_DEVICE
         assert P(FAKE, 128, 512, 512, FAKE, FAKE, FAKE, FAKE, None) == sp24.SP24_ERR_UNSUPPORTED_DEVICE
+
+
+def test_prune_in_gemm_validation():
+    F = L.sp24_prune_activations_in_gemm
+    ok = dict(X=FAKE, M=512, K=1024, ldx=1024, W=FAKE, N=512, ldw=1024, Y=FAKE, ldy=512, dt=sp24.BF16, xv=None,
+              xm=None)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return F(a["X"], a["M"], a["K"], a["ldx"], a["W"], a["N"], a["ldw"], a["Y"], a["ldy"], a["dt"], a["xv"],
+                 a["xm"], None)
+    assert call(X=None) == sp24.SP24_ERR_NULL
+    assert call(xv=FAKE) == sp24.SP24_ERR_NULL           # values and metadata together
+    assert call(dt=sp24.E4M3) == sp24.SP24_ERR_DTYPE
+    assert call(M=128) == sp24.SP24_ERR_INVALID_ARG       # the CTA-pair kernel: M, N >= 256
+    assert call(N=200, ldy=200) == sp24.SP24_ERR_INVALID_ARG
+    assert call(K=1000, ldx=1000, ldw=1000) == sp24.SP24_ERR_NOT_2_4
+    assert call(ldx=1028) == sp24.SP24_ERR_ALIGNMENT
+    assert call(Y=FAKE + 2) == sp24.SP24_ERR_ALIGNMENT
+    if NO_GPU:
+        assert call() == sp24.SP24_ERR_UNSUPPORTED_DEVICE

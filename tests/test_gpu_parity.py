@@ -1065,3 +1065,58 @@ def test_bounded_wait_expires_without_fault_and_context_survives():
     X, W = inputs.linear_pair(16, 256, 256, seed=0)
     y, y_ref, a_ref, _, _ = run_gemm(X, W, False, sp24.SPARSE, True)
     check_tolerance(y, y_ref, a_ref, "after self test")
+
+
+# ---------------------------------------------------------------------------
+# online activations pruned inside the GEMM (no compressed X in HBM)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("M,N,K", [(256, 256, 128), (300, 384, 640), (512, 768, 1024), (1024, 512, 4096),
+                                   (260, 1280, 256)])
+def test_prune_in_gemm_parity(M, N, K):
+    X = inputs.student_t_bf16((M, K), 3.0, seed=M + 5 * K)
+    X[3, :8] = np.array([0x3F80, 0xBF80, 0x3F80, 0, 0, 0, 0, 0], np.uint16)  # ties, zero group
+    W = inputs.normal_bf16((N, K), 0.02, seed=N + 9)
+    pruned, values, canon = orc.prune_compress_bf16(X)
+    y_ref, a_ref = orc.gemm_f64(orc.bf16_bits_to_f64(pruned), orc.bf16_bits_to_f64(W))
+    Xd, Wd = dev_bf16(X), dev_bf16(W)
+    for emit in (False, True):
+        for out_f32 in (True, False):
+            Y = torch.empty(M, N, dtype=torch.float32 if out_f32 else torch.bfloat16, device="cuda")
+            Y.fill_(float("nan"))
+            xv = torch.empty(M, K // 2, dtype=torch.bfloat16, device="cuda") if emit else None
+            xm = torch.empty(sp24.meta_bytes(M, K), dtype=torch.uint8, device="cuda") if emit else None
+            sp24.prune_activations_in_gemm(Xd, Wd, Y, x_values=xv, x_meta=xm)
+            torch.cuda.synchronize()
+            assert sp24.last_device_error() == sp24.SP24_OK
+            check_tolerance(Y.float().cpu().numpy().astype(np.float64), y_ref, a_ref,
+                            "prune in gemm M%d N%d K%d f32=%s" % (M, N, K, out_f32))
+            if emit:
+                assert np.array_equal(bits16(xv), values), "emitted compressed X"
+                assert np.array_equal(u8(xm), orc.meta_image(canon, M, K, False)), "emitted metadata image"
+
+
+def test_prune_in_gemm_full_size_sampled():
+    """cfg 4 at full size (X 8192 x 4096 Student-t, W 12288 x 4096): sampled
+    outputs against the oracle and against the two-kernel path."""
+    M, K, N = inputs.ACT_SHAPE["M"], inputs.ACT_SHAPE["K"], inputs.ACT_SHAPE["N"]
+    X = inputs.student_t_bf16((M, K), 3.0, seed=4)
+    W = inputs.normal_bf16((N, K), 0.02, seed=4)
+    Xd, Wd = dev_bf16(X), dev_bf16(W)
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    sp24.prune_activations_in_gemm(Xd, Wd, Y)
+    Y2 = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(sp24.activations_workspace_bytes(M, K), dtype=torch.uint8, device="cuda")
+    sp24.prune_compress_activations_fused(Xd, Wd, Y2, workspace=ws)
+    torch.cuda.synchronize()
+    assert sp24.last_device_error() == sp24.SP24_OK
+    g = np.random.default_rng(21)
+    ms = np.concatenate([g.integers(0, M, size=60), [0, M - 1]])
+    ns = np.concatenate([g.integers(0, N, size=60), [0, N - 1]])
+    pruned, _, _ = orc.prune_compress_bf16(X[ms])
+    y_ref, a_ref = orc.gemm_f64_sampled(orc.bf16_bits_to_f64(pruned), orc.bf16_bits_to_f64(W[ns]),
+                                        np.arange(ms.size), np.arange(ns.size))
+    y = Y.float().cpu().numpy().astype(np.float64)[ms, ns]
+    y2 = Y2.float().cpu().numpy().astype(np.float64)[ms, ns]
+    check_tolerance(y, y_ref, a_ref, "prune in gemm, full size")
+    check_tolerance(y, y2, a_ref, "prune in gemm vs two-kernel path")
