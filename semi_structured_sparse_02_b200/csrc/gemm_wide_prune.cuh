@@ -136,6 +136,7 @@ k_gemm_wide_prune(const __grid_constant__ WidePruneLaunch g) {
     wait_upstream();
     if (lane == 0) {
       const uint32_t full0 = mapa_shared(bar_u32(kFull), 0);
+      const uint64_t pol_x = policy_evict_last();  // an X tile is read again for every W tile
       int armed_raw[S];
       for (int s = 0; s < S; ++s) armed_raw[s] = -1;
       int stage = 0;
@@ -157,7 +158,7 @@ k_gemm_wide_prune(const __grid_constant__ WidePruneLaunch g) {
           armed_raw[stage] = (int)phase;
 #pragma unroll
           for (int bx = 0; bx < 2; ++bx)
-            tma_load_2d(sa + bx * 16384, &g.tm_x, bar_u32(kRaw + stage), kt * 128 + bx * 64, ya, 0ull);
+            tma_load_2d(sa + bx * 16384, &g.tm_x, bar_u32(kRaw + stage), kt * 128 + bx * 64, ya, pol_x);
           if (rank == 0) mbar_arrive_expect_tx(bar_u32(kFull + stage), 2u * 32768u);
 #pragma unroll
           for (int bx = 0; bx < 2; ++bx)

@@ -69,8 +69,26 @@ def oracle_x(X_bits: np.ndarray, e4m3: bool):
     return X_bits, None, orc.bf16_bits_to_f64(X_bits)
 
 
+def bf16_half_ulp(y: np.ndarray) -> np.ndarray:
+    """Half the bf16 spacing at |y| (the largest error of rounding a value of
+    that binade to bf16: 8 significant bits, so 2^-8 relative at the bottom
+    of a binade)."""
+    m = np.abs(np.asarray(y, dtype=np.float64))
+    e = np.floor(np.log2(np.where(m > 0, m, 1.0)))
+    return np.where(m > 0, np.exp2(e - 8), 0.0)
+
+
 def check_tolerance(y_gpu: np.ndarray, y: np.ndarray, a: np.ndarray, what: str = ""):
-    ok = orc.within_tolerance(y_gpu, y, a)
+    """|y_gpu - y| <= 2e-3 * a + 1e-6 (the GEMM's bound on its fp32 result),
+    plus, when the output was stored as bf16, the rounding of that cast:
+    half a bf16 spacing of the stored value.  A bf16 output is recognized by
+    every value's fp32 image having zero low 16 bits."""
+    y_gpu = np.asarray(y_gpu, dtype=np.float64)
+    f32 = y_gpu.astype(np.float32)
+    if y_gpu.size and np.all((f32.view(np.uint32) & 0xFFFF) == 0):
+        ok = np.abs(y_gpu - y) <= 2e-3 * a + 1e-6 + bf16_half_ulp(y_gpu)
+    else:
+        ok = orc.within_tolerance(y_gpu, y, a)
     if not ok.all():
         idx = np.argwhere(~ok)[:5]
         det = ["(%s) gpu=%r ref=%r a=%r" % (tuple(i), float(y_gpu[tuple(i)]), float(y[tuple(i)]),
