@@ -337,12 +337,9 @@ k_gemm_wide_prune(const __grid_constant__ WidePruneLaunch g) {
         uint32_t nibs[2] = {0u, 0u};
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-          uint32_t k00, k01, k10, k11;
           const uint4 v = raw[c];
-          const uint32_t n0 = prune_pick4(v.x & 0xFFFFu, v.x >> 16, v.y & 0xFFFFu, v.y >> 16, k00, k01);
-          const uint32_t n1 = prune_pick4(v.z & 0xFFFFu, v.z >> 16, v.w & 0xFFFFu, v.w >> 16, k10, k11);
-          kept[2 * c] = k00 | (k01 << 16);
-          kept[2 * c + 1] = k10 | (k11 << 16);
+          const uint32_t n0 = prune_pick4w(v.x, v.y, kept[2 * c]);
+          const uint32_t n1 = prune_pick4w(v.z, v.w, kept[2 * c + 1]);
           nibs[c >> 2] |= (n0 | (n1 << 4)) << (8 * (c & 3));
         }
         // the compressed row: 128 bytes = 8 chunks, this half's 4 chunks

@@ -22,41 +22,40 @@ constexpr int kPruneThreads = 256;
 
 // ---------------------------------------------------------------------------
 // One group of four: keep the two largest |v| (bf16 magnitude bits compared as
-// integers), ties to the lower index.  Position i loses to j < i when
-// |v_j| >= |v_i| and to j > i when |v_j| > |v_i|; it survives if it loses to
-// fewer than two positions.  Returns the nibble i0 | i1 << 2.
+// integers), ties to the lower index.  Each position gets a composite key,
+// magnitude bits above a tie-break that is larger for a lower index, so the
+// kept pair is the top two of four distinct keys: the larger of the two
+// pair maxima, and the larger of (the smaller pair maximum, the larger pair
+// minimum).  Same positions as counting, for each one, the positions that
+// beat it (a larger magnitude, or an equal one at a lower index) and keeping
+// those beaten fewer than twice.
+//
+// lo = x0 | x1 << 16, hi = x2 | x3 << 16 (bf16 bit patterns).  Returns the
+// nibble i0 | i1 << 2 (i0 < i1) and, in kept, x_i0 | x_i1 << 16.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t prune_group4(uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                                 int& i0, int& i1) {
-  // a* are magnitude keys (bits & 0x7fff)
-  const int l0 = (a1 > a0) + (a2 > a0) + (a3 > a0);
-  const int l1 = (a0 >= a1) + (a2 > a1) + (a3 > a1);
-  const int l2 = (a0 >= a2) + (a1 >= a2) + (a3 > a2);
-  const int l3 = (a0 >= a3) + (a1 >= a3) + (a2 >= a3);
-  const bool k0 = l0 < 2, k1 = l1 < 2, k2 = l2 < 2, k3 = l3 < 2;
-  // exactly two of k0..k3 are set; pick them in ascending order
-  i0 = k0 ? 0 : (k1 ? 1 : 2);
-  i1 = k3 ? 3 : (k2 ? 2 : 1);
-  (void)k1;
-  return (uint32_t)i0 | ((uint32_t)i1 << 2);
+__device__ __forceinline__ uint32_t prune_pick4w(uint32_t lo, uint32_t hi, uint32_t& kept) {
+  const uint32_t k0 = ((lo << 2) & 0x1FFFCu) | 3u;
+  const uint32_t k1 = ((lo >> 14) & 0x1FFFCu) | 2u;
+  const uint32_t k2 = ((hi << 2) & 0x1FFFCu) | 1u;
+  const uint32_t k3 = (hi >> 14) & 0x1FFFCu;
+  const uint32_t m01 = max(k0, k1), n01 = min(k0, k1), m23 = max(k2, k3), n23 = min(k2, k3);
+  const uint32_t top = max(m01, m23);
+  const uint32_t sec = max(min(m01, m23), max(n01, n23));
+  const uint32_t ia = 3u - (top & 3u), ib = 3u - (sec & 3u);
+  const uint32_t i0 = min(ia, ib), i1 = max(ia, ib);
+  // bytes 2i, 2i+1 of {hi:lo} are x_i
+  kept = __byte_perm(lo, hi, i0 * 0x22u + i1 * 0x2200u + 0x1010u);
+  return i0 | (i1 << 2);
 }
 
-// The same rule on full bf16 bit patterns, returning the two kept values
-// (ascending index) by selects rather than by indexing, which would put the
-// group in local memory.
+// The same rule on four separate bf16 bit patterns (low 16 bits of each).
 __device__ __forceinline__ uint32_t prune_pick4(uint32_t x0, uint32_t x1, uint32_t x2, uint32_t x3,
                                                 uint32_t& kept0, uint32_t& kept1) {
-  const uint32_t a0 = x0 & 0x7FFFu, a1 = x1 & 0x7FFFu, a2 = x2 & 0x7FFFu, a3 = x3 & 0x7FFFu;
-  const int l0 = (a1 > a0) + (a2 > a0) + (a3 > a0);
-  const int l1 = (a0 >= a1) + (a2 > a1) + (a3 > a1);
-  const int l2 = (a0 >= a2) + (a1 >= a2) + (a3 > a2);
-  const int l3 = (a0 >= a3) + (a1 >= a3) + (a2 >= a3);
-  const bool k0 = l0 < 2, k1 = l1 < 2, k2 = l2 < 2, k3 = l3 < 2;
-  const uint32_t i0 = k0 ? 0u : (k1 ? 1u : 2u);
-  const uint32_t i1 = k3 ? 3u : (k2 ? 2u : 1u);
-  kept0 = k0 ? x0 : (k1 ? x1 : x2);
-  kept1 = k3 ? x3 : (k2 ? x2 : x1);
-  return i0 | (i1 << 2);
+  uint32_t kept;
+  const uint32_t nib = prune_pick4w(x0 | (x1 << 16), x2 | (x3 << 16), kept);
+  kept0 = kept & 0xFFFFu;
+  kept1 = kept >> 16;
+  return nib;
 }
 
 // Two E4M3 codes (round to nearest even, saturating) in the low 16 bits:
@@ -160,8 +159,10 @@ k_prune_compress(const uint16_t* __restrict__ src, int64_t rows, int64_t K, int6
           }
         }
       } else {
-        nib0 = prune_pick4(e0, e1, e2, e3, k00, k01);
-        nib1 = prune_pick4(e4, e5, e6, e7, k10, k11);
+        uint32_t w0, w1;
+        nib0 = prune_pick4w(v.x, v.y, w0);
+        nib1 = prune_pick4w(v.z, v.w, w1);
+        k00 = w0 & 0xFFFFu; k01 = w0 >> 16; k10 = w1 & 0xFFFFu; k11 = w1 >> 16;
       }
       if (live) {
         // a hybrid matrix's dense-form array also holds its sparse tiles,
@@ -534,11 +535,11 @@ k_prune_cast_rows_e4m3(const uint16_t* __restrict__ src, int64_t rows, int64_t K
     const int64_t idx = (int64_t)seg * kQSegVecs + j * 32 + lane;
     if (idx < nv) {
       const uint4 v = reg[j];
-      uint32_t k00, k01, k10, k11;
-      const uint32_t nib0 = prune_pick4(v.x & 0xFFFFu, v.x >> 16, v.y & 0xFFFFu, v.y >> 16, k00, k01);
-      const uint32_t nib1 = prune_pick4(v.z & 0xFFFFu, v.z >> 16, v.w & 0xFFFFu, v.w >> 16, k10, k11);
-      const uint32_t q = e4m3x2_of(__fmul_rn(bf16_bits_to_float(k00), inv), __fmul_rn(bf16_bits_to_float(k01), inv)) |
-                         (e4m3x2_of(__fmul_rn(bf16_bits_to_float(k10), inv), __fmul_rn(bf16_bits_to_float(k11), inv)) << 16);
+      uint32_t w0, w1;
+      const uint32_t nib0 = prune_pick4w(v.x, v.y, w0);
+      const uint32_t nib1 = prune_pick4w(v.z, v.w, w1);
+      const uint32_t q = e4m3x2_of(__fmul_rn(__uint_as_float(w0 << 16), inv), __fmul_rn(__uint_as_float(w0 & 0xFFFF0000u), inv)) |
+                         (e4m3x2_of(__fmul_rn(__uint_as_float(w1 << 16), inv), __fmul_rn(__uint_as_float(w1 & 0xFFFF0000u), inv)) << 16);
       if (live) *reinterpret_cast<uint32_t*>(vrow + idx * 4) = q;
       meta[(rb * KC + idx / 16) * kChunkBytes + L * 16 + (idx % 16)] = (uint8_t)(nib0 | (nib1 << 4));
     }
