@@ -259,6 +259,11 @@ def run_product(args, rank, world, local_rank):
         return [sp24.GemmGroup(v, after_independent=i > 0) for i, (_, v) in enumerate(sorted(by.items()))]
 
     groups = {"sparse": make_groups(lambda it: "sparse"), "dense": make_groups(lambda it: "dense")}
+    # other groupings of the same 16 GEMMs, timed for comparison: two launches
+    # (tokens 1, 8 and 32 in one, 128 in the other) and one launch of all 16
+    groups["sparse_2"] = [sp24.GemmGroup([it["a_sp"] for it in inst if it["M"] <= 32]),
+                          sp24.GemmGroup([it["a_sp"] for it in inst if it["M"] > 32], after_independent=True)]
+    groups["sparse_1"] = [sp24.GemmGroup([it["a_sp"] for it in inst])]
 
     def step(kind):
         quant_all()
@@ -288,7 +293,7 @@ def run_product(args, rank, world, local_rank):
     groups["selected"] = make_groups(lambda it: it["tactic"])
 
     # eager warm-up (sets kernel attributes), then capture the graphs
-    kinds = ("sparse", "dense", "selected", "ungrouped", "gemm_only")
+    kinds = ("sparse", "dense", "selected", "ungrouped", "sparse_2", "sparse_1", "gemm_only")
     with torch.cuda.stream(stream):
         for kind in kinds[:-1]:
             step(kind)
@@ -355,6 +360,8 @@ def run_product(args, rank, world, local_rank):
     ms_sel = time_graph(graphs["selected"], K_steps, W_warm)
     ms_gemm = time_graph(graphs["gemm_only"], K_steps, W_warm)
     ms_ungrouped = time_graph(graphs["ungrouped"], K_steps, W_warm)
+    ms_two = time_graph(graphs["sparse_2"], K_steps, W_warm)
+    ms_one = time_graph(graphs["sparse_1"], K_steps, W_warm)
 
     # End to end through the public API: every step copies its activations in
     # from pinned host memory and its outputs back out, eager calls.  The
@@ -476,6 +483,8 @@ def run_product(args, rank, world, local_rank):
         "ms_per_step_dense": round(ms_dense / K_steps, 5),
         "ms_per_step_selected": round(ms_sel / K_steps, 5),
         "ms_per_step_ungrouped": round(ms_ungrouped / K_steps, 5),
+        "ms_per_step_two_launches": round(ms_two / K_steps, 5),
+        "ms_per_step_one_launch": round(ms_one / K_steps, 5),
         "tactics": man["metrics"],
         "roofline": {
             "kernel": "k_gemm sparse e4m3 (tcgen05.mma.sp), grouped launch",

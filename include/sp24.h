@@ -257,10 +257,14 @@ int sp24_gemm(const sp24_gemm_args *args, void *stream);
  * problems).  Same results as sp24_gemm on each.  The work of all problems
  * is scheduled together, so the weights of the whole group stream without a
  * launch, ramp or tail between problems.  All problems must share in_dtype,
- * out_dtype and tactic, either all carry a hybrid tile mask or none does, and
- * have M in the same class (1-16, 17-32, 33-64, >64); otherwise
- * SP24_ERR_INVALID_ARG.  Hybrid problems run 128-row tiles on single CTAs
- * (each 128-deep K-step dense or sparse as its tile's flag says).  Each args'
+ * out_dtype and tactic, and either all carry a hybrid tile mask or none
+ * does; otherwise SP24_ERR_INVALID_ARG.  Their token counts may differ: the
+ * launch is built for the widest token tile of the group (16, 32, 64 or 128
+ * tokens by M) and each problem runs its own width, so problems with small M
+ * stream their weights next to wider ones (fewer pipeline stages than a
+ * launch of small-M problems alone).  Hybrid problems run 128-row tiles on
+ * single CTAs, each stage two tile columns, dense or sparse as their flags
+ * say.  Each args'
  * own workspace fields are ignored: the group uses `workspace` (size from
  * sp24_gemm_grouped_workspace_bytes, same zero-fill rule as sp24_gemm).
  * SP24_GEMM_W_STATIC applies when every problem sets it. */

@@ -63,6 +63,7 @@ struct GemmProblem {
   int32_t tiles_a, tiles_b;
   int32_t tile_begin;         // first global tile index of this problem
   int32_t meta_blocks;        // 128-row blocks of the metadata image (pair tiles clamp to it)
+  int32_t bn;                 // token-tile width of this problem (16..kBN, a multiple of 16; kBN in a pair)
   int64_t iter_begin;         // first global stream-K iteration of this problem
   const uint8_t* meta;        // metadata image of A (sparse / hybrid)
   const uint8_t* tile_mask;   // hybrid: [tiles_a x K/128]
@@ -336,7 +337,7 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
     // global load.
     const uint64_t pol_stream = policy_evict_first();
     const uint64_t pol_keep = policy_evict_last();
-    constexpr uint32_t kBTx = (uint32_t)C::kBBytes;
+
     int armed[S];
     for (int s = 0; s < S; ++s) armed[s] = -1;
     auto flag_word = [&](const GemmProblem& P, int ta, int c0) -> uint32_t {
@@ -377,9 +378,9 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
         }
       }
     };
-    auto arm = [&](int stage, uint32_t kind, int ph) {
+    auto arm = [&](int stage, uint32_t kind, int ph, int bn) {
       s_kind[stage] = (uint8_t)kind;
-      mbar_arrive_expect_tx(full_bar(stage), a_bytes(kind) + kBTx);
+      mbar_arrive_expect_tx(full_bar(stage), a_bytes(kind) + (uint32_t)(bn * 128 * 2));
       armed[stage] = ph;
     };
     // 1. static weights: the first S stages' A copies before the dependency wait
@@ -399,7 +400,7 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
           tma_prefetch_desc(&g.tm_a3[pr]);
           for (int i = 0; i < take; ++i) {
             const uint32_t kind = stage_kind(P, kb + i, i, fl);
-            arm(pre + i, kind, 0);
+            arm(pre + i, kind, 0, P.bn);
             load_a(pre + i, P, pr, ta, kb + i, kind);
           }
         }
@@ -438,7 +439,7 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
               *abort_flag = 1;
             } else {
               const uint32_t kind = stage_kind(P, kt, i & 15, fl);
-              arm(stage, kind, (int)phase);
+              arm(stage, kind, (int)phase, P.bn);
               load_a(stage, P, pr, ta, kt, kind);
             }
           }
@@ -446,7 +447,7 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
             const uint32_t sb = smem_u32(smem + stage * C::kStageBytes) + C::kABytes;
 #pragma unroll
             for (int bx = 0; bx < 2; ++bx)
-              tma_load_2d(sb + bx * kBN * 128, &g.tm_b[pr], full_bar(stage), kt * 256 + bx * 128, tb * kBN, pol_keep);
+              tma_load_2d(sb + bx * kBN * 128, &g.tm_b[pr], full_bar(stage), kt * 256 + bx * 128, tb * P.bn, pol_keep);
             ++n;
             if (++stage == S) {
               stage = 0;
@@ -518,7 +519,7 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
       };
       auto load_b = [&](int stage, int pr, int tb, int kt) {
         const uint32_t sb = smem_u32(smem + stage * C::kStageBytes) + C::kABytes;
-        const int32_t yb = tb * kBN + (int32_t)rank * C::kBRows;
+        const int32_t yb = tb * g.prob[pr].bn + (int32_t)rank * C::kBRows;
         if (C::kNv) {
           // kKT / 2 bytes of B per row, then the four scale chunks of the
           // 128-row block of B that holds this tile (tiles of fewer than 128
@@ -529,7 +530,7 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
             load2d(sb + bx * C::kBRows * 128, &g.tm_b[pr], stage, kt * (C::kKT / 2) + bx * 128, yb, pol_keep);
           const int nsf = nv_half(P, kt) ? 2 : 4;
           bulk_load(sb + C::kBBytes + C::kMetaBytes + 2048,
-                    P.sfb + ((int64_t)((tb * kBN) >> 7) * (P.K / C::kSfChunkK) + 4 * (int64_t)kt) * 512,
+                    P.sfb + ((int64_t)((tb * P.bn) >> 7) * (P.K / C::kSfChunkK) + 4 * (int64_t)kt) * 512,
                     (uint32_t)nsf * 512, full_bar(stage), pol_keep);
         } else {
           const int box_elems = kBf16 ? 64 : 128;
@@ -542,11 +543,13 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
       auto stage_bytes = [&](int pr, int ta, int kt) -> uint32_t {
         const GemmProblem& P = g.prob[pr];
         if (kPair) return 2u * (uint32_t)C::kStageBytes;  // metadata boxes are always whole
+        // the B boxes hold this problem's bn rows
+        const uint32_t bbytes = (uint32_t)(P.bn * 128 * C::kBBoxes);
         if (C::kNv) {
           const uint32_t nsf = nv_half(P, kt) ? 2u : 4u;
-          return (uint32_t)(C::kABytes + C::kBBytes) + (C::kNvSparse ? nsf / 2 * 2048u : 0u) + 2u * nsf * 512u;
+          return (uint32_t)C::kABytes + bbytes + (C::kNvSparse ? nsf / 2 * 2048u : 0u) + 2u * nsf * 512u;
         }
-        uint32_t b = C::kABytes + C::kBBytes;
+        uint32_t b = (uint32_t)C::kABytes + bbytes;
         if (C::kSparse) b += (uint32_t)meta_chunks(P, kt) * 2048;
         return b;
       };
@@ -631,10 +634,17 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
       pdl_launch_dependents();
     }
     if (lane == 0 && rank == 0) {
-      const uint32_t idesc = C::kNv ? make_idesc_nvf4(C::kNvSparse, kBlockA, kBN)
-                                    : make_idesc(C::kSparse, kBf16, C::kRowsA, kBN);
-      const uint32_t idesc_dense = make_idesc(false, kBf16, kBlockA, kBN);
-      const uint32_t idesc_sp = make_idesc(true, kBf16, C::kRowsA, kBN);
+      // instruction descriptors for the current problem's token-tile width
+      uint32_t idesc = 0, idesc_dense = 0, idesc_sp = 0;
+      int idesc_bn = -1;
+      auto set_idesc = [&](int bn) {
+        if (bn == idesc_bn) return;
+        idesc_bn = bn;
+        idesc = C::kNv ? make_idesc_nvf4(C::kNvSparse, kBlockA, (uint32_t)bn)
+                       : make_idesc(C::kSparse, kBf16, C::kRowsA, (uint32_t)bn);
+        idesc_dense = make_idesc(false, kBf16, kBlockA, (uint32_t)bn);
+        idesc_sp = make_idesc(true, kBf16, C::kRowsA, (uint32_t)bn);
+      };
       const uint32_t meta_col0 = C::kAccCols;
       const uint32_t s0 = smem_u32(smem);
       const uint64_t da0 = smem_desc(s0, 16, 1024, kLayoutSw128);
@@ -657,6 +667,7 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
       int pr, tile, kb, ke, seg;
       while (ok && it.next(g, units, pr, tile, kb, ke, seg)) {
         const GemmProblem& P = g.prob[pr];
+        set_idesc(kPair ? kBN : P.bn);
         const int buf = acc_i & 1;
         const uint32_t acc_phase = (acc_i >> 1) & 1;
         if (!mbar_wait(acce_bar(buf), acc_phase ^ 1, p.timeout_ns, kDevErrWaitAccEmpty)) {
@@ -845,6 +856,7 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
     while (it.next(g, units, pr, tile, kb, ke, seg)) {
       const GemmProblem& P = g.prob[pr];
       const int ta = tile % P.tiles_a, tb = tile / P.tiles_a;
+      const int bn = kPair ? kBN : P.bn;   // token-tile width of this problem
       const int buf = acc_i & 1;
       const uint32_t acc_phase = (acc_i >> 1) & 1;
       const int ga = ta * C::kRowsA + (int)rank * kBlockA + row;  // global A row of this thread
@@ -856,8 +868,8 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
       const float sa_v = P.scale_a == nullptr ? 1.0f : C::kNv ? __ldg(P.scale_a) : a_live ? __ldg(P.scale_a + ga) : 1.0f;
       if (pr != cached_pr || tb != cached_tb) {
         named_bar_sync(1, 128);
-        for (int i = et; i < kBN; i += 128) {
-          const int gb = tb * kBN + i;
+        for (int i = et; i < bn; i += 128) {
+          const int gb = tb * bn + i;
           s_scale_b[i] = P.scale_b == nullptr ? 1.0f : C::kNv ? P.scale_b[0] : gb < rows_b ? P.scale_b[gb] : 1.0f;
         }
         named_bar_sync(1, 128);
@@ -884,7 +896,7 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
       auto store16 = [&](auto eb_c, const float (&v)[16], int c0) {
         constexpr int EB = decltype(eb_c)::value;
         constexpr int PV = 16 / EB;   // elements per 16-byte vector
-        const int gb0 = tb * kBN + c0;
+        const int gb0 = tb * bn + c0;
         float sc[16];
 #pragma unroll
         for (int i = 0; i < 16; i += 4) {
@@ -975,7 +987,7 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
 
       if (full) {
 #pragma unroll 1
-        for (int c0 = 0; c0 < kBN; c0 += 16) {
+        for (int c0 = 0; c0 < bn; c0 += 16) {
           uint32_t r[16];
           tmem_ld_x16(tbase + c0, r);
           tmem_ld_wait();
@@ -1010,7 +1022,7 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
           // so each warp store covers 512 contiguous bytes
           float4* dst = reinterpret_cast<float4*>(sk_slots + my * 128 * kBN) + row;
 #pragma unroll 1
-          for (int c0 = 0; c0 < kBN; c0 += 16) {
+          for (int c0 = 0; c0 < bn; c0 += 16) {
             uint32_t r[16];
             tmem_ld_x16(tbase + c0, r);
             tmem_ld_wait();
@@ -1051,7 +1063,7 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
           // our accumulator plus the others' partials, 64 columns at a time
           constexpr int kFix = kBN < 64 ? kBN : 64;
 #pragma unroll 1
-          for (int cb = 0; cb < kBN; cb += kFix) {
+          for (int cb = 0; cb < bn; cb += kFix) {
             float4 q[kFix / 4];
 #pragma unroll
             for (int j = 0; j < kFix / 4; ++j) q[j] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -1070,6 +1082,7 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
             }
 #pragma unroll
             for (int c0 = 0; c0 < kFix; c0 += 16) {
+              if (cb + c0 >= bn) break;  // a problem narrower than the kernel's tile
               uint32_t r[16];
               tmem_ld_x16(tbase + cb + c0, r);
               tmem_ld_wait();

@@ -136,6 +136,7 @@ struct Plan {
   int kt;          // logical K per stage
   int n;           // problems
   int num_kt[kMaxGroup], tiles_a[kMaxGroup], tiles_b[kMaxGroup];
+  int bn_i[kMaxGroup];  // token-tile width of each problem (<= bn, the kernel's compile-time width)
   int sched;       // kSchedDataParallel / kSchedStreamK
   int grid;
   int64_t total_iters;
@@ -428,13 +429,17 @@ Plan plan_group(const sp24_gemm_args* const* a, int n, const DeviceInfo& di, siz
   pl.bn = pick_bn(a[0]->M);
   pl.kt = stage_k(pl.mode, pl.bf16);
   pl.n = n;
+  // the kernel's tile width is the widest class in the group; each problem
+  // runs its own class's width (a pair runs the kernel's)
+  for (int i = 1; i < n; ++i) pl.bn = std::max(pl.bn, pick_bn(a[i]->M));
   pl.pair = want_pair(a, n, pl.mode, di.pairs);
   if (pl.pair && pl.mode == kModeSparse && !pl.bf16 && pl.bn < 32) pl.bn = 32;  // sparse e4m3 pair: N >= 32
   const int rows_a = pl.pair ? 2 * kBlockA : kBlockA;
   for (int i = 0; i < n; ++i) {
+    pl.bn_i[i] = pl.pair ? pl.bn : pick_bn(a[i]->M);
     pl.num_kt[i] = (int)((a[i]->K + pl.kt - 1) / pl.kt);
     pl.tiles_a[i] = (int)((a[i]->N + rows_a - 1) / rows_a);
-    pl.tiles_b[i] = (int)((a[i]->M + pl.bn - 1) / pl.bn);
+    pl.tiles_b[i] = (int)((a[i]->M + pl.bn_i[i] - 1) / pl.bn_i[i]);
   }
   choose_schedule(pl, pl.pair ? di.pairs : di.sms, ws_cap);
   return pl;
@@ -474,10 +479,11 @@ bool fill_problem(GemmLaunch<kMaxProb>& gl, int i, const sp24_gemm_args* a, cons
     ok &= make_map(&gl.tm_a3[i], a->W, 1, a->K / 2, a->N, a->ldw, 128, kBlockA, CU_TENSOR_MAP_SWIZZLE_128B);
   }
   if (pl.mode != kModeHybrid) gl.tm_a3[i] = gl.tm_a[i];
-  ok &= make_map(&gl.tm_b[i], a->X, eb, a->K, a->M, a->ldx * eb, box_elems, pl.pair ? pl.bn / 2 : pl.bn,
+  ok &= make_map(&gl.tm_b[i], a->X, eb, a->K, a->M, a->ldx * eb, box_elems, pl.pair ? pl.bn / 2 : pl.bn_i[i],
                  CU_TENSOR_MAP_SWIZZLE_128B);
   GemmProblem& P = gl.prob[i];
   memset(&P, 0, sizeof P);
+  P.bn = pl.bn_i[i];
   P.meta_blocks = (int32_t)((a->N + 127) / 128);
   P.rows_a = (int32_t)a->N;
   P.rows_b = (int32_t)a->M;
@@ -880,6 +886,7 @@ int run_activation_gemm(bool bf16, const void* x_values, const void* x_meta, con
   P.tiles_a = pl.tiles_a[0];
   P.tiles_b = pl.tiles_b[0];
   P.meta_blocks = (int32_t)((M + 127) / 128);
+  P.bn = pl.bn;
   P.meta = static_cast<const uint8_t*>(x_meta);
   P.scale_a = x_scales;
   P.scale_b = w_scales;
@@ -904,8 +911,7 @@ int validate_group(const sp24_gemm_args* a, int n) {
     if (st != SP24_OK) return st;
     // hybrid weights group with hybrid weights only (one kernel mode per launch)
     if ((a[i].tile_dense_mask != nullptr) != (a[0].tile_dense_mask != nullptr)) return SP24_ERR_INVALID_ARG;
-    if (a[i].in_dtype != a[0].in_dtype || a[i].out_dtype != a[0].out_dtype ||
-        a[i].tactic != a[0].tactic || pick_bn(a[i].M) != pick_bn(a[0].M))
+    if (a[i].in_dtype != a[0].in_dtype || a[i].out_dtype != a[0].out_dtype || a[i].tactic != a[0].tactic)
       return SP24_ERR_INVALID_ARG;
   }
   return SP24_OK;
@@ -990,6 +996,7 @@ int build_launch_nvfp4(GemmLaunch<1>& gl, const sp24_nvfp4_gemm_args* a, const P
   P.tiles_a = pl.tiles_a[0];
   P.tiles_b = pl.tiles_b[0];
   P.meta_blocks = (int32_t)((a->N + 127) / 128);
+  P.bn = pl.bn;
   P.meta = static_cast<const uint8_t*>(a->W_meta);
   P.sfa = static_cast<const uint8_t*>(a->w_scales);
   P.sfb = static_cast<const uint8_t*>(a->x_scales);

@@ -346,8 +346,9 @@ class GemmGroup:
 
 
 def m_class(M: int) -> int:
-    """The token-count class of a GEMM (1-16, 17-32, 33-64, >64); only GEMMs of
-    one class share a grouped launch."""
+    """The token-count class of a GEMM (1-16, 17-32, 33-64, >64): the token
+    tile width it runs with.  A grouped launch may mix classes; it is built
+    for the widest."""
     return 16 if M <= 16 else 32 if M <= 32 else 64 if M <= 64 else 128
 
 

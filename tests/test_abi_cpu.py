@@ -147,8 +147,9 @@ def test_grouped_gemm_validation():
     assert f(arr, 2, None, 0, None) == sp24.SP24_ERR_INVALID_ARG    # mixed output dtypes
     arr[1] = gemm_args(tactic=sp24.DENSE)
     assert f(arr, 2, None, 0, None) == sp24.SP24_ERR_INVALID_ARG    # mixed tactics
-    arr[1] = gemm_args(M=17)
-    assert f(arr, 2, None, 0, None) == sp24.SP24_ERR_INVALID_ARG    # M classes 1-16 and 17-32
+    if NO_GPU:  # token classes may differ within a group: validation passes (no device here)
+        arr[1] = gemm_args(M=17)
+        assert f(arr, 2, None, 0, None) == sp24.SP24_ERR_UNSUPPORTED_DEVICE
     arr[1] = gemm_args(M=9, N=512, K=1024)
     assert f(arr, 2, FAKE + 8, 1024, None) == sp24.SP24_ERR_ALIGNMENT
     arr[1] = gemm_args(X=None)
@@ -156,7 +157,7 @@ def test_grouped_gemm_validation():
     e4 = dict(in_dtype=sp24.E4M3, x_scales=FAKE, w_scales=FAKE)
     arr[0] = gemm_args(mask=FAKE, dense=FAKE, **e4)
     arr[1] = gemm_args(**e4)
-    assert f(arr, 2, None, 0, None) == sp24.SP24_ERR_INVALID_ARG    # no hybrid tiles in a group
+    assert f(arr, 2, None, 0, None) == sp24.SP24_ERR_INVALID_ARG    # hybrid and plain weights in one group
     assert L.sp24_gemm_grouped_workspace_bytes(arr, 2) == 0
 
 

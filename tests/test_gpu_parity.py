@@ -288,6 +288,25 @@ def test_grouped_gemm_parity(group, e4, tactic):
         check_group(items, "group %s e4=%s tactic=%d f32=%s" % (group, e4, tactic, out_f32))
 
 
+# Groups whose problems come from different token-count classes: the launch
+# takes the widest class's tile, each problem runs its own width.
+MIXED_GROUPS = {
+    "to32": [(1, 512, 1024), (8, 384, 2048), (32, 640, 1024), (20, 256, 512)],
+    "to128": [(1, 256, 1024), (16, 384, 512), (32, 512, 1536), (128, 640, 1024), (100, 256, 2048)],
+}
+
+
+@pytest.mark.parametrize("group", sorted(MIXED_GROUPS))
+@pytest.mark.parametrize("e4", [False, True])
+@pytest.mark.parametrize("tactic", [sp24.SPARSE, sp24.DENSE])
+@pytest.mark.parametrize("use_ws", [True, False])
+def test_grouped_gemm_mixed_token_classes(group, e4, tactic, use_ws):
+    for out_f32 in (True, False):
+        _, items = run_group(MIXED_GROUPS[group], e4, tactic, out_f32, use_ws=use_ws, seed=len(group) + 5,
+                             flags=sp24.GEMM_W_STATIC)
+        check_group(items, "mixed group %s e4=%s tactic=%d ws=%s f32=%s" % (group, e4, tactic, use_ws, out_f32))
+
+
 @pytest.mark.parametrize("e4", [False, True])
 def test_grouped_gemm_whole_tiles_without_workspace(e4):
     grp, items = run_group(GROUPS["decode"], e4, sp24.SPARSE, True, use_ws=False)
@@ -469,6 +488,21 @@ def test_grouped_hybrid_gemm_parity(group, use_ws, kind):
         torch.cuda.synchronize()
         assert sp24.last_device_error() == sp24.SP24_OK
         check_group(items, "hybrid group %s ws=%s %s call %d" % (group, use_ws, kind, call))
+
+
+def test_grouped_hybrid_mixed_token_classes():
+    shapes = [(1, 768, 512), (16, 512, 1024), (32, 256, 5120), (100, 384, 640)]
+    items = []
+    for i, (M, N, K) in enumerate(shapes):
+        X, W = inputs.linear_pair(M, N, K, seed=29 * i + M + K, outliers=True)
+        items.append(prepare_gemm(X, W, True, sp24.SPARSE, False, mask=inputs.hybrid_mask(N, K, seed=i),
+                                  flags=sp24.GEMM_W_STATIC))
+    for use_ws in (True, False):
+        grp = sp24.GemmGroup([it[0] for it in items], allocate_workspace=use_ws)
+        grp()
+        torch.cuda.synchronize()
+        assert sp24.last_device_error() == sp24.SP24_OK
+        check_group(items, "hybrid mixed classes ws=%s" % use_ws)
 
 
 def test_grouped_rejects_mixed_hybrid_and_plain_weights():
