@@ -239,31 +239,31 @@ def run_product(args, rank, world, local_rank):
 
     stream = torch.cuda.Stream(device=dev)
     # the per-token e4m3 casts of the 16 independent activation matrices run
-    # as one grouped launch; then the GEMMs run as grouped launches, one per
-    # (tactic, token-count class): M in {1, 8} share one, M = 32 and M = 128
-    # one each.  Launches are chained by programmatic dependent launch, each
+    # as one grouped launch; then the 16 GEMMs run as one grouped launch per
+    # tactic (each problem multiplies its own token-tile width inside the
+    # widest one).  Launches are chained by programmatic dependent launch, each
     # streaming its weights while the previous kernel drains.
     quant_all = sp24.QuantGroup([(it["X"], it["xq"], it["xs"]) for it in inst])
 
-    def make_groups(pick, items=None):
-        """Grouped launches for the tactic pick(it) of every GEMM.  The GEMMs
-        are independent and all their inputs come from the cast before the
-        first group, so every group after the first is marked as following
+    def make_groups(pick, items=None, by_class=False):
+        """Grouped launches for the tactic pick(it) of every GEMM, one per
+        tactic (or, with by_class, one per tactic and token-count class).  The
+        GEMMs are independent and all their inputs come from the cast before
+        the first group, so every group after the first is marked as following
         an independent GEMM launch: its CTAs start as SMs free up instead of
         waiting for the previous group to finish."""
         by = {}
         for it in (inst if items is None else items):
             t = pick(it)
             a = it["a_sp"] if t == "sparse" else it["a_dn"]
-            by.setdefault((t, sp24.m_class(it["M"])), []).append(a)
+            by.setdefault((t, sp24.m_class(it["M"]) if by_class else 0), []).append(a)
         return [sp24.GemmGroup(v, after_independent=i > 0) for i, (_, v) in enumerate(sorted(by.items()))]
 
     groups = {"sparse": make_groups(lambda it: "sparse"), "dense": make_groups(lambda it: "dense")}
-    # other groupings of the same 16 GEMMs, timed for comparison: two launches
-    # (tokens 1, 8 and 32 in one, 128 in the other) and one launch of all 16
-    groups["sparse_2"] = [sp24.GemmGroup([it["a_sp"] for it in inst if it["M"] <= 32]),
-                          sp24.GemmGroup([it["a_sp"] for it in inst if it["M"] > 32], after_independent=True)]
-    groups["sparse_1"] = [sp24.GemmGroup([it["a_sp"] for it in inst])]
+    # the same 16 GEMMs as three launches, one per token-count class
+    # (M in {1, 8}, 32, 128), each with its own token-tile width, for comparison
+    groups["sparse_by_class"] = make_groups(lambda it: "sparse", by_class=True)
+    groups["dense_by_class"] = make_groups(lambda it: "dense", by_class=True)
 
     def step(kind):
         quant_all()
@@ -293,7 +293,7 @@ def run_product(args, rank, world, local_rank):
     groups["selected"] = make_groups(lambda it: it["tactic"])
 
     # eager warm-up (sets kernel attributes), then capture the graphs
-    kinds = ("sparse", "dense", "selected", "ungrouped", "sparse_2", "sparse_1", "gemm_only")
+    kinds = ("sparse", "dense", "selected", "ungrouped", "sparse_by_class", "dense_by_class", "gemm_only")
     with torch.cuda.stream(stream):
         for kind in kinds[:-1]:
             step(kind)
@@ -360,8 +360,8 @@ def run_product(args, rank, world, local_rank):
     ms_sel = time_graph(graphs["selected"], K_steps, W_warm)
     ms_gemm = time_graph(graphs["gemm_only"], K_steps, W_warm)
     ms_ungrouped = time_graph(graphs["ungrouped"], K_steps, W_warm)
-    ms_two = time_graph(graphs["sparse_2"], K_steps, W_warm)
-    ms_one = time_graph(graphs["sparse_1"], K_steps, W_warm)
+    ms_cls = time_graph(graphs["sparse_by_class"], K_steps, W_warm)
+    ms_cls_dense = time_graph(graphs["dense_by_class"], K_steps, W_warm)
 
     # End to end through the public API: every step copies its activations in
     # from pinned host memory and its outputs back out, eager calls.  The
@@ -476,18 +476,18 @@ def run_product(args, rank, world, local_rank):
         "config": bench_config(world),
         "timing": "CUDA graph of one step replayed K times; CUDA events on the replay stream",
         "step": ("one grouped per-token e4m3 cast of the 16 activation matrices, then the 16 "
-                 "GEMMs as %d grouped launches (one per token-count class: M in {1,8}, 32, 128)"
+                 "GEMMs as %d grouped launch (token tiles of 16, 32 and 128 rows in one launch)"
                  % len(groups["sparse"])),
         "tflops": round(world * step_flops / t_step / 1e12, 3),
         "speedup_vs_dense": round(ms_dense / ms_sparse, 4),
         "ms_per_step_dense": round(ms_dense / K_steps, 5),
         "ms_per_step_selected": round(ms_sel / K_steps, 5),
         "ms_per_step_ungrouped": round(ms_ungrouped / K_steps, 5),
-        "ms_per_step_two_launches": round(ms_two / K_steps, 5),
-        "ms_per_step_one_launch": round(ms_one / K_steps, 5),
+        "ms_per_step_by_token_class": round(ms_cls / K_steps, 5),
+        "ms_per_step_dense_by_token_class": round(ms_cls_dense / K_steps, 5),
         "tactics": man["metrics"],
         "roofline": {
-            "kernel": "k_gemm sparse e4m3 (tcgen05.mma.sp), grouped launch",
+            "kernel": "k_gemm sparse e4m3 (tcgen05.mma.sp), one grouped launch of the 16 GEMMs",
             "bound": "hbm",
             "achieved": round(achieved, 1),
             "peak": hbm_peak,

@@ -1,5 +1,6 @@
 // gemm_wide.cuh -- the large-M GEMM: a CTA pair (cluster of two, tcgen05
-// cta_group::2) computes a 256 x 256 output tile with one MMA stream.
+// cta_group::2) computes a 256 x 256 output tile (256 x 240 when A carries
+// sparsity metadata) with one MMA stream.
 //
 // Why a pair.  A single CTA's 128 x 128 tile needs about 195 bytes of operand
 // per clock at the sparse tensor rate (A 16 KB + B 32 KB + metadata 2 KB per
@@ -20,15 +21,16 @@
 //   warps 2..5   both CTAs: epilogue of the CTA's 128 accumulator rows.
 //
 // Tensor memory (512 columns per CTA).  Dense: two 256-column accumulators.
-// Sparse: the metadata needs columns too, so the second accumulator starts at
-// column 224 and overlaps the first by 32 columns; the metadata slots take
-// columns 480..511.  The epilogue drains a tile's 32 overlapping columns
-// first and then releases the accumulator, so the next tile's MMAs (which
-// only conflict in those columns) start while the rest is drained.  Draining
-// tile i's overlap implies tile i-1 is fully drained (the epilogue is
-// sequential), so one release per tile covers both accumulators.
+// Sparse and hybrid: the metadata needs columns too, so the tile is 240 B
+// rows wide (the MMA's N = 240, 120 B rows per CTA): the accumulators start at
+// columns 0 and 256 as in the dense kernel, and the metadata slots take the
+// 16 columns after each (240..255 and 496..511).  Both kinds keep two whole
+// accumulators, so a tile's MMAs start while the previous tile is drained.  (Two 256-column accumulators that share 32 columns with the
+// metadata would make every tile's first MMA wait for the previous tile's
+// last one and for the epilogue to drain the shared columns: a measured
+// ~1.7 us per tile.)
 //
-// Work schedule: whole 256 x 256 tiles, round-robin over the pairs.  By
+// Work schedule: whole tiles, round-robin over the pairs.  By
 // default the A tile index runs fastest (consecutive pairs share a B tile; A
 // is re-read from L2 for every B tile).  When A is the larger operand and B
 // fits comfortably in L2 (b_fastest, chosen on the host), the B index runs
@@ -53,12 +55,12 @@ namespace sp24 {
 
 struct WideLaunch {
   CUtensorMap tm_a;     // A: dense [rows_a x K] or values [rows_a x K/2]; 128-byte box x 128 rows, SW128
-  CUtensorMap tm_b;     // B: [rows_b x K]; 128-byte box x 128 rows, SW128
+  CUtensorMap tm_b;     // B: [rows_b x K]; 128-byte box x kBHalf rows (128, or 120 with metadata), SW128
   CUtensorMap tm_meta;  // metadata image viewed as [chunks * 8 rows x 256 B]; box 256 B x 8 * chunks rows
   CUtensorMap tm_a2;    // hybrid: values [rows_a x K/2]; 64-byte box x 128 rows, SW64 (tm_a: dense form)
   const uint8_t* tile_mask;  // hybrid: [ceil(rows_a/128) x K/128] dense flags
   int32_t rows_a, rows_b, K, num_kt;
-  int32_t tiles_a, tiles_b;  // 256-row tiles
+  int32_t tiles_a, tiles_b;  // 256-row tiles of A, kBN-row tiles of B
   int32_t total_tiles, meta_blocks;  // metadata row blocks (128 rows) that exist
   int32_t b_fastest;                 // tile order: B tile index fastest (else A)
   int32_t out_f32, use_pdl;
@@ -79,16 +81,24 @@ struct WideCfg {
   static constexpr int kKT = kSparse ? (kBf16 ? 128 : 256) : (kHybrid ? 128 : (kBf16 ? 64 : 128));
   static constexpr int kABytes = 128 * 128;  // hybrid: dense 128 x 128 B, or sparse 128 x 64 B
   static constexpr int kBBoxes = kSparse ? 2 : 1;
-  static constexpr int kBBytes = 128 * 128 * kBBoxes;
+  static constexpr int kBN = kUsesMeta ? 240 : 256;  // B rows of a pair tile (the MMA's N)
+  static constexpr int kBHalf = kBN / 2;             // B rows per CTA
+  static constexpr int kBBoxBytes = kBHalf * 128;    // one 128-byte-wide box of B
+  static constexpr int kBBytes = 128 * 128 * kBBoxes;  // boxes at 16 KB strides (1024-byte aligned)
   static constexpr int kMetaChunks = kSparse ? (kBf16 ? 1 : 2) : (kHybrid ? 1 : 0);
   static constexpr int kMetaBytes = kMetaChunks * 2048;
   static constexpr int kStageBytes = kABytes + kBBytes + kMetaBytes;  // per CTA
+  static constexpr uint32_t kStageTx = kABytes + kBBoxes * kBBoxBytes + kMetaBytes;  // bytes a stage receives
   static constexpr int kStages = kSparse ? 4 : 6;
   static constexpr int kMetaCols = kMetaChunks * 4;
-  static constexpr int kOverlap = kUsesMeta ? 32 : 0;
-  static constexpr int kAcc1 = 256 - kOverlap;       // first column of the second accumulator
-  static constexpr int kMetaCol0 = 512 - kOverlap;   // metadata slots (sparse)
-  static_assert(!kUsesMeta || kStages * kMetaCols <= kOverlap, "metadata slots overflow");
+  static constexpr int kAcc1 = 256;  // first column of the second accumulator
+  // metadata slots (sparse, hybrid): stage s in the gap after the first
+  // accumulator, then in the gap after the second
+  static constexpr int kSlotsPerGap = kUsesMeta ? (256 - kBN) / kMetaCols : 0;
+  static_assert(!kUsesMeta || kStages <= 2 * kSlotsPerGap, "metadata slots overflow");
+  __host__ __device__ static constexpr uint32_t meta_col(int s) {
+    return s < kSlotsPerGap ? (uint32_t)(kBN + s * kMetaCols) : (uint32_t)(256 + kBN + (s - kSlotsPerGap) * kMetaCols);
+  }
   static constexpr int kBarOffset = kStages * kStageBytes;
   static constexpr int kScaleOffset = kBarOffset + 256;
   static constexpr int kEpiOffset = kScaleOffset + 256 * 4;
@@ -176,8 +186,8 @@ k_gemm_wide(const __grid_constant__ WideLaunch g) {
     const bool b_fastest = g.b_fastest != 0;
     const uint64_t timeout_ns = g.timeout_ns;
     const uint8_t* const mask = g.tile_mask;
-    constexpr uint32_t kDenseTx = 2u * (128 * 128 + 128 * 128);          // A dense + B, both CTAs
-    constexpr uint32_t kSparseTx = 2u * (128 * 64 + 128 * 128 + 2048);   // A values + B + metadata
+    constexpr uint32_t kDenseTx = 2u * (128 * 128 + C::kBBoxBytes);          // A dense + B, both CTAs
+    constexpr uint32_t kSparseTx = 2u * (128 * 64 + C::kBBoxBytes + 2048);   // A values + B + metadata
     int armed[S];
     for (int s = 0; s < S; ++s) armed[s] = -1;
     int stage = 0;
@@ -197,7 +207,7 @@ k_gemm_wide(const __grid_constant__ WideLaunch g) {
       __syncwarp();
       if (lane == 0) {
         const int ya = ta * 256 + (int)rank * 128;
-        const int yb = tb * 256 + (int)rank * 128;
+        const int yb = tb * C::kBN + (int)rank * C::kBHalf;
         int rb = rb0 + (int)rank;
         if (rb >= meta_blocks) rb = 0;  // rows past the end: A is zero-filled; any valid metadata
         for (int kt = 0; kt < num_kt; ++kt) {
@@ -257,7 +267,7 @@ k_gemm_wide(const __grid_constant__ WideLaunch g) {
         const int ta = b_fastest ? tile / tiles_b : tile % tiles_a;
         const int tb = b_fastest ? tile % tiles_b : tile / tiles_a;
         const int ya = ta * 256 + (int)rank * 128;
-        const int yb = tb * 256 + (int)rank * 128;
+        const int yb = tb * C::kBN + (int)rank * C::kBHalf;
         int rb = ta * 2 + (int)rank;        // metadata row block of this CTA's A rows
         if (rb >= meta_blocks) rb = 0;    // rows past the end: A is zero-filled; any valid metadata
         for (int kt = 0; kt < num_kt; ++kt) {
@@ -267,7 +277,7 @@ k_gemm_wide(const __grid_constant__ WideLaunch g) {
             break;
           }
           if (rank == 0) {
-            mbar_arrive_expect_tx(bar_u32(kFull + stage), 2u * C::kStageBytes);
+            mbar_arrive_expect_tx(bar_u32(kFull + stage), 2u * C::kStageTx);
             armed[stage] = (int)phase;
           }
           const uint32_t sa = smem_u32(smem + stage * C::kStageBytes);
@@ -295,9 +305,9 @@ k_gemm_wide(const __grid_constant__ WideLaunch g) {
     // ------------------------------------------------------------------ MMA issuer (rank 0)
     wait_upstream();  // nothing to issue before the producer's loads anyway
     if (rank == 0 && lane == 0) {
-      const uint32_t idesc = make_idesc(C::kSparse, kBf16, 256, 256);
-      const uint32_t idesc_dense = make_idesc(false, kBf16, 256, 256);  // hybrid dense K-steps
-      const uint32_t idesc_sp = make_idesc(true, kBf16, 256, 256);      // hybrid sparse K-steps
+      const uint32_t idesc = make_idesc(C::kSparse, kBf16, 256, C::kBN);
+      const uint32_t idesc_dense = make_idesc(false, kBf16, 256, C::kBN);  // hybrid dense K-steps
+      const uint32_t idesc_sp = make_idesc(true, kBf16, 256, C::kBN);      // hybrid sparse K-steps
       const uint32_t s0 = smem_u32(smem);
       const uint64_t da0 = smem_desc(s0, 16, 1024, kLayoutSw128);
       const uint64_t db0 = smem_desc(s0 + C::kABytes, 16, 1024, kLayoutSw128);
@@ -314,10 +324,9 @@ k_gemm_wide(const __grid_constant__ WideLaunch g) {
       int j = 0;
       for (int tile = pair; ok && tile < total_tiles; tile += n_pairs, ++j) {
         const int b = j & 1;
-        // the accumulator: sparse waits for tile j-1's overlap release (which
-        // implies tile j-2 is drained); dense waits for tile j-2's release
-        if (C::kUsesMeta ? j >= 1 : j >= 2) {
-          const int jr = C::kUsesMeta ? j - 1 : j - 2;
+        // accumulator b is free once tile j-2 (the last one that used it) is drained
+        if (j >= 2) {
+          const int jr = j - 2;
           if (!mbar_wait(bar_u32(kAccEmpty + (jr & 1)), (uint32_t)((jr >> 1) & 1), timeout_ns,
                          kDevErrWaitAccEmpty)) {
             ok = false;
@@ -341,7 +350,7 @@ k_gemm_wide(const __grid_constant__ WideLaunch g) {
           const uint64_t da = da0 + so, db = db0 + so;
           const bool first = kt == 0;
           if (C::kHybrid) {
-            const uint32_t mcol = C::kMetaCol0 + stage * C::kMetaCols;
+            const uint32_t mcol = C::meta_col(stage);
             if (s_kind[stage] != 0) {
 #pragma unroll
               for (int q = 0; q < 4; ++q)
@@ -355,7 +364,7 @@ k_gemm_wide(const __grid_constant__ WideLaunch g) {
                                tmem_base + mcol + 2 * q, idesc_sp, (first && q == 0) ? 0u : 1u);
             }
           } else if (C::kSparse) {
-            const uint32_t mcol = C::kMetaCol0 + stage * C::kMetaCols;
+            const uint32_t mcol = C::meta_col(stage);
             auto issue = [&](auto chunks_c) {
               constexpr int kChunks = decltype(chunks_c)::value;
               if (kChunks == 2) tc_cp_128x256b_pair(tmem_base + mcol, dm2 + so);
@@ -427,8 +436,8 @@ k_gemm_wide(const __grid_constant__ WideLaunch g) {
       const int ga = ta * 256 + (int)rank * 128 + row;  // A row of this thread
       const float sa_v = (scale_a != nullptr && ga < rows_a) ? __ldg(scale_a + ga) : 1.0f;
       named_bar_sync(1, 128);  // the previous tile's stores are done with the B scales
-      for (int i = et; i < 256; i += 128) {
-        const int gb = tb * 256 + i;
+      for (int i = et; i < C::kBN; i += 128) {
+        const int gb = tb * C::kBN + i;
         s_scale_b[i] = (scale_b != nullptr && gb < rows_b) ? scale_b[gb] : 1.0f;
       }
       named_bar_sync(1, 128);
@@ -447,7 +456,7 @@ k_gemm_wide(const __grid_constant__ WideLaunch g) {
       auto store16 = [&](auto eb_c, const float (&v)[16], int c0) {
         constexpr int EB = decltype(eb_c)::value;
         constexpr int PV = 16 / EB;  // elements per 16-byte vector
-        const int gb0 = tb * 256 + c0;
+        const int gb0 = tb * C::kBN + c0;
         float sc[16];
 #pragma unroll
         for (int i = 0; i < 16; i += 4) {
@@ -534,17 +543,8 @@ k_gemm_wide(const __grid_constant__ WideLaunch g) {
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(acc_empty0 + 8u * b);
       };
-      if (C::kUsesMeta) {
-        // the columns shared with the other accumulator first, then release
-        const int ov0 = b ? 0 : 256 - C::kOverlap;
-        drain(ov0, ov0 + C::kOverlap);
-        release();
-        if (b) drain(C::kOverlap, 256);
-        else drain(0, 256 - C::kOverlap);
-      } else {
-        drain(0, 256);
-        release();
-      }
+      drain(0, C::kBN);
+      release();
     }
   }
 

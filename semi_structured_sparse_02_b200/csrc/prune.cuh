@@ -34,18 +34,23 @@ constexpr int kPruneThreads = 256;
 // nibble i0 | i1 << 2 (i0 < i1) and, in kept, x_i0 | x_i1 << 16.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t prune_pick4w(uint32_t lo, uint32_t hi, uint32_t& kept) {
-  const uint32_t k0 = ((lo << 2) & 0x1FFFCu) | 3u;
-  const uint32_t k1 = ((lo >> 14) & 0x1FFFCu) | 2u;
-  const uint32_t k2 = ((hi << 2) & 0x1FFFCu) | 1u;
-  const uint32_t k3 = (hi >> 14) & 0x1FFFCu;
+  // keys: magnitude bits at 17..31 (the sign shifted out or masked off),
+  // code 3 - i in bits 0..1.  Multiply-adds by powers of two build them and
+  // the index arithmetic below on the FMA pipe, leaving the integer ALU pipe
+  // (this loop's limit) the masks, the six min/max and the byte permute.
+  const uint32_t k0 = mad_u32(lo, 131072u, 3u);
+  const uint32_t k1 = (mad_u32(lo, 2u, 0u) & 0xFFFE0000u) | 2u;
+  const uint32_t k2 = mad_u32(hi, 131072u, 1u);
+  const uint32_t k3 = mad_u32(hi, 2u, 0u) & 0xFFFE0000u;
   const uint32_t m01 = max(k0, k1), n01 = min(k0, k1), m23 = max(k2, k3), n23 = min(k2, k3);
   const uint32_t top = max(m01, m23);
   const uint32_t sec = max(min(m01, m23), max(n01, n23));
-  const uint32_t ia = 3u - (top & 3u), ib = 3u - (sec & 3u);
-  const uint32_t i0 = min(ia, ib), i1 = max(ia, ib);
+  // the smaller position has the larger code: i0 = 3 - max code, i1 = 3 - min code
+  const uint32_t ct = top & 3u, cs = sec & 3u;
+  const uint32_t i0 = max(ct, cs) ^ 3u, i1 = min(ct, cs) ^ 3u;
   // bytes 2i, 2i+1 of {hi:lo} are x_i
-  kept = __byte_perm(lo, hi, i0 * 0x22u + i1 * 0x2200u + 0x1010u);
-  return i0 | (i1 << 2);
+  kept = __byte_perm(lo, hi, mad_u32(i1, 0x2200u, mad_u32(i0, 0x22u, 0x1010u)));
+  return mad_u32(i1, 4u, i0);
 }
 
 // The same rule on four separate bf16 bit patterns (low 16 bits of each).
@@ -319,10 +324,17 @@ struct QuantGroup {
   int n;
 };
 
-__device__ __forceinline__ uint32_t amax_bits8(const uint4 v) {
-  uint32_t m = max(max(v.x & 0x7FFFu, v.x >> 16 & 0x7FFFu), max(v.y & 0x7FFFu, v.y >> 16 & 0x7FFFu));
-  return max(m, max(max(v.z & 0x7FFFu, v.z >> 16 & 0x7FFFu), max(v.w & 0x7FFFu, v.w >> 16 & 0x7FFFu)));
+// Running maximum of the magnitude bits of eight bf16 values, as two 16-bit
+// lanes (packed max, one mask per word); amax_lanes_reduce folds the lanes.
+__device__ __forceinline__ uint32_t amax_lanes8(uint32_t m2, const uint4 v) {
+  const uint32_t a = max_u16x2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu);
+  const uint32_t b = max_u16x2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu);
+  return max_u16x2(m2, max_u16x2(a, b));
 }
+
+__device__ __forceinline__ uint32_t amax_lanes_reduce(uint32_t m2) { return max(m2 & 0xFFFFu, m2 >> 16); }
+
+__device__ __forceinline__ uint32_t amax_bits8(const uint4 v) { return amax_lanes_reduce(amax_lanes8(0u, v)); }
 
 __device__ __forceinline__ uint2 e4m3_codes8(const uint4 v, float inv) {
   const uint32_t e[8] = {v.x & 0xFFFFu, v.x >> 16, v.y & 0xFFFFu, v.y >> 16,
@@ -510,14 +522,15 @@ k_prune_cast_rows_e4m3(const uint16_t* __restrict__ src, int64_t rows, int64_t K
   const int64_t nv = K / 8;
   pdl_wait();  // the activations may be written by the upstream grid
   uint4 reg[kQWarpVecs];
-  uint32_t m = 0;
-  const uint4* p = reinterpret_cast<const uint4*>(src + (live ? row : 0) * ld);
+  uint32_t m2 = 0;
+  const int64_t idx0 = (int64_t)seg * kQSegVecs + lane;  // vector j of this thread: idx0 + 32 j
+  const uint4* p = reinterpret_cast<const uint4*>(src + (live ? row : 0) * ld) + idx0;
 #pragma unroll
   for (int j = 0; j < kQWarpVecs; ++j) {
-    const int64_t idx = (int64_t)seg * kQSegVecs + j * 32 + lane;
-    reg[j] = (live && idx < nv) ? __ldg(p + idx) : make_uint4(0, 0, 0, 0);
-    m = max(m, amax_bits8(reg[j]));
+    reg[j] = (live && idx0 + j * 32 < nv) ? __ldg(p + j * 32) : make_uint4(0, 0, 0, 0);
+    m2 = amax_lanes8(m2, reg[j]);
   }
+  uint32_t m = amax_lanes_reduce(m2);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
   __syncthreads();  // s_amax initialized
@@ -529,19 +542,24 @@ k_prune_cast_rows_e4m3(const uint16_t* __restrict__ src, int64_t rows, int64_t K
   if (live && seg == 0 && lane == 0) scales[row] = amax == 0.0f ? 1.0f : __fdiv_rn(amax, 448.0f);
   const int64_t KC = K / kChunkK;
   const int64_t rb = row / kChunkRows, L = row % kChunkRows;
-  uint8_t* vrow = values + row * (K / 2);
+  // vector idx of the row: 4 value bytes at idx * 4, its metadata byte in
+  // chunk idx / 16 at L * 16 + idx % 16; idx0 % 16 == lane % 16 since the
+  // warp segment length is a multiple of 32, so vector j's byte is 2 chunks on
+  uint32_t* vrow = reinterpret_cast<uint32_t*>(values + row * (K / 2)) + idx0;
+  uint8_t* mrow = meta + (rb * KC + idx0 / 16) * kChunkBytes + L * 16 + (lane & 15);
 #pragma unroll
   for (int j = 0; j < kQWarpVecs; ++j) {
-    const int64_t idx = (int64_t)seg * kQSegVecs + j * 32 + lane;
-    if (idx < nv) {
+    if (idx0 + j * 32 < nv) {
       const uint4 v = reg[j];
       uint32_t w0, w1;
       const uint32_t nib0 = prune_pick4w(v.x, v.y, w0);
       const uint32_t nib1 = prune_pick4w(v.z, v.w, w1);
-      const uint32_t q = e4m3x2_of(__fmul_rn(__uint_as_float(w0 << 16), inv), __fmul_rn(__uint_as_float(w0 & 0xFFFF0000u), inv)) |
-                         (e4m3x2_of(__fmul_rn(__uint_as_float(w1 << 16), inv), __fmul_rn(__uint_as_float(w1 & 0xFFFF0000u), inv)) << 16);
-      if (live) *reinterpret_cast<uint32_t*>(vrow + idx * 4) = q;
-      meta[(rb * KC + idx / 16) * kChunkBytes + L * 16 + (idx % 16)] = (uint8_t)(nib0 | (nib1 << 4));
+      const uint32_t q0 = e4m3x2_of(__fmul_rn(__uint_as_float(mad_u32(w0, 65536u, 0u)), inv),
+                                    __fmul_rn(__uint_as_float(w0 & 0xFFFF0000u), inv));
+      const uint32_t q1 = e4m3x2_of(__fmul_rn(__uint_as_float(mad_u32(w1, 65536u, 0u)), inv),
+                                    __fmul_rn(__uint_as_float(w1 & 0xFFFF0000u), inv));
+      if (live) vrow[j * 32] = mad_u32(q1, 65536u, q0);
+      mrow[j * 2 * kChunkBytes] = (uint8_t)mad_u32(nib1, 16u, nib0);
     }
   }
 }

@@ -613,7 +613,7 @@ LaunchCache<SingleLaunch, 32> g_cache_single;
 LaunchCache<GroupLaunch, 16> g_cache_group;
 
 // ---------------------------------------------------------------------------
-// The CTA-pair kernel (256 x 256 tiles) for large token counts
+// The CTA-pair kernel (256 x 256 tiles, 256 x 240 with metadata) for large token counts
 // ---------------------------------------------------------------------------
 // A GEMM takes the pair kernel when both output dimensions span at least one
 // 256-row tile, unless SP24_GEMM_SINGLE_CTA asks for the one-CTA kernel.
@@ -623,6 +623,10 @@ LaunchCache<GroupLaunch, 16> g_cache_group;
 // row blocks is dense there, so with fewer tiles the one-CTA kernel (per-tile
 // choice, stream-K over every SM) measured faster (e.g. 6144 x 4096 at 256
 // tokens: 22.6 against 24.5 us; 24576 x 4096 at 256 tokens: 49 against 41).
+static_assert(WideCfg<kModeSparse, true>::kBN == WideCfg<kModeSparse, false>::kBN &&
+                  WideCfg<kModeHybrid, false>::kBN == WideCfg<kModeSparse, false>::kBN &&
+                  WideCfg<kModeDense, true>::kBN == WideCfg<kModeDense, false>::kBN,
+              "one pair-tile width per kind of A");
 bool use_pair(int64_t rows_a, int64_t rows_b, int64_t K, bool hybrid, uint32_t flags) {
   if (rows_a < 256 || rows_b < 256 || (flags & SP24_GEMM_SINGLE_CTA) != 0) return false;
   if (!hybrid) return true;
@@ -630,7 +634,8 @@ bool use_pair(int64_t rows_a, int64_t rows_b, int64_t K, bool hybrid, uint32_t f
   if ((flags & SP24_GEMM_CTA_PAIR) != 0) return true;
   DeviceInfo di;
   if (current_device_info(&di) != SP24_OK) return false;
-  const int64_t tiles = ((rows_a + 255) / 256) * ((rows_b + 255) / 256);
+  constexpr int bn = WideCfg<kModeHybrid, false>::kBN;
+  const int64_t tiles = ((rows_a + 255) / 256) * ((rows_b + bn - 1) / bn);
   return tiles >= (int64_t)di.pairs;
 }
 bool args_use_pair(const sp24_gemm_args* a) {
@@ -708,7 +713,10 @@ int run_wide(int mode, bool bf16, bool a_is_w, const void* A, int64_t lda, const
                    CU_TENSOR_MAP_SWIZZLE_128B);
     wl.tm_a2 = wl.tm_a;
   }
-  ok &= make_map(&wl.tm_b, B, eb, K, rows_b, ldb * eb, box_elems, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  // with metadata the pair tile is 240 B rows (two accumulators and the
+  // metadata slots fill tensor memory), else 256
+  const int bn = (sparse || hybrid) ? WideCfg<kModeSparse, false>::kBN : WideCfg<kModeDense, false>::kBN;
+  ok &= make_map(&wl.tm_b, B, eb, K, rows_b, ldb * eb, box_elems, (uint32_t)(bn / 2), CU_TENSOR_MAP_SWIZZLE_128B);
   const int meta_blocks = (int)((rows_a + 127) / 128);
   if (sparse || hybrid) {
     const int chunks = (bf16 || hybrid) ? 1 : 2;
@@ -723,7 +731,7 @@ int run_wide(int mode, bool bf16, bool a_is_w, const void* A, int64_t lda, const
   wl.K = (int32_t)K;
   wl.num_kt = (int32_t)((K + kt - 1) / kt);
   wl.tiles_a = (int32_t)((rows_a + 255) / 256);
-  wl.tiles_b = (int32_t)((rows_b + 255) / 256);
+  wl.tiles_b = (int32_t)((rows_b + bn - 1) / bn);
   wl.total_tiles = wl.tiles_a * wl.tiles_b;
   wl.meta_blocks = meta_blocks;
   // tile order: with A running fastest, all of A is re-read (from L2 if it
