@@ -233,11 +233,12 @@ typedef struct sp24_gemm_args {
 
 /* Bytes of workspace the call would use for its stream-K schedule (0 if the
  * shape needs none).  Shapes with few output tiles per SM may split the
- * tiles' K range evenly over all SMs (a cost model decides); a split tile is
- * finished by the contributor that arrives last, which adds the others'
- * fp32 partial tiles (stored in the workspace) to its own.  Which
- * contributor finishes can vary from run to run, and with it the fp32
- * summation order (the last bits of those outputs).  With a smaller or
+ * tiles' K range over all SMs (a cost model decides; the ranges are cut by
+ * estimated cost, so SMs that stream wider token tiles get fewer K-stages);
+ * a split tile is finished by the SM holding its first K-stage, which adds
+ * the others' fp32 partial tiles (stored in the workspace) to its own.  The
+ * split, and with it the fp32 summation order, is fixed by the shapes and the
+ * device: repeated calls give identical results.  With a smaller or
  * missing workspace the call falls back to whole tiles per CTA (fewer SMs
  * busy on such shapes).  The workspace must be zero-filled once before its
  * first use; every call that returns SP24_OK leaves its state (the leading
@@ -271,8 +272,8 @@ int sp24_gemm(const sp24_gemm_args *args, void *stream);
 int sp24_gemm_grouped(const sp24_gemm_args *args, int n, void *workspace_dev, size_t workspace_bytes,
                       void *stream);
 
-/* Leading bytes of the workspace that hold the stream-K state (arrival
- * counters and partial-tile flags): zero before the first call, and zero
+/* Leading bytes of the workspace that hold the stream-K state (the
+ * partial-tile flags): zero before the first call, and zero
  * again after every call that returns SP24_OK.  The rest of the workspace
  * holds partial tiles whose contents never matter between calls.  0 when the
  * call's schedule needs no workspace. */

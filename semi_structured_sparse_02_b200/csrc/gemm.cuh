@@ -54,6 +54,7 @@ enum GemmSched : int { kSchedDataParallel = 0, kSchedStreamK = 1 };
 constexpr int kGemmThreads = 192;
 constexpr int kBlockA = 128;  // MMA M: rows of A per tile
 constexpr int kMaxGroup = 16; // problems per grouped launch
+constexpr int kMaxSkUnits = 160;  // stream-K scheduling units (SMs or CTA pairs) a launch may have
 
 // One problem of a (possibly grouped) launch.
 struct GemmProblem {
@@ -73,7 +74,6 @@ struct GemmProblem {
   const uint8_t* sfb;         // NVFP4: scale image of B
   void* Y;
   int64_t ldy;
-  unsigned int* ws_counters;  // stream-K arrival counters [tiles (x2 halves in a pair)]
 };
 
 struct GemmParams {
@@ -86,8 +86,11 @@ struct GemmParams {
   int32_t w_static;           // A operands are not written by the upstream grid
   int32_t after_independent;  // the upstream grid is an independent GEMM: wait for it only at the end
   uint64_t timeout_ns;
-  float* sk_slots;            // stream-K partial tiles [units][pair half][2][128 rows][BN] fp32
-  unsigned int* sk_flags;     // "partial stored" flags [units][pair half][2]
+  float* sk_slots;            // stream-K partial tiles [units][pair half][128 rows][BN] fp32
+  unsigned int* sk_flags;     // "partial stored" flags [units][pair half]
+  // stream-K: unit u takes global K-stages [sk_bound[u], sk_bound[u + 1]),
+  // ranges cut so that every unit gets the same weighted stage cost
+  int64_t sk_bound[kMaxSkUnits + 1];
 };
 
 // Everything a launch needs, passed by value (tensor maps must live in
@@ -202,8 +205,8 @@ struct SegIter {
     j = 0;
     pr = 0;
     if (g.p.sched == kSchedStreamK) {
-      it = (int64_t)cta * g.p.total_iters / grid;
-      it1 = (int64_t)(cta + 1) * g.p.total_iters / grid;
+      it = g.p.sk_bound[cta];
+      it1 = g.p.sk_bound[cta + 1];
     } else {
       tile_g = cta;
     }
@@ -233,9 +236,16 @@ struct SegIter {
   }
 };
 
-// The unit (CTA or CTA pair) whose stream-K range holds global iteration i.
-__device__ __forceinline__ int sk_owner(int64_t total_iters, int grid, int64_t i) {
-  return (int)(((i + 1) * grid - 1) / total_iters);
+// The unit (CTA or CTA pair) whose stream-K range holds global iteration i:
+// the last unit whose range starts at or before i (binary search).
+__device__ __forceinline__ int sk_owner(const GemmParams& p, int units, int64_t i) {
+  int lo = 0, hi = units - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (p.sk_bound[mid] <= i) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
 }
 
 template <int kMode, bool kBf16, int kBN, bool kAIsW, int kMaxProb, bool kPair = false>
@@ -847,7 +857,6 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
     // below clobber memory, which would otherwise force the parameter-struct
     // fields to be re-read after each of them
     const bool out_f32 = p.out_f32 != 0;
-    const int64_t total_iters = p.total_iters;
     float* const sk_slots = p.sk_slots;
     unsigned int* const sk_flags = p.sk_flags;
     SegIter<kMaxProb> it;
@@ -876,16 +885,54 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
         cached_pr = pr;
         cached_tb = tb;
       }
+      const bool full = (kb == 0 && ke == P.num_kt);
+      // A split tile is finished by the unit that holds its first K-stage:
+      // that unit's range ends inside the tile, so the tile is its last
+      // segment, and every other contributor's segment of it lies at the
+      // start of (or spans) that contributor's range.  The finisher waits
+      // (bounded) for the others' partials before its own accumulator, so
+      // the wait overlaps its last MMAs.
+      const bool finisher = !full && kb == 0;
+      int64_t i0 = 0;
+      int c_first = 0, c_last = 0;
+      if (!full) {
+        i0 = P.iter_begin + (int64_t)tile * P.num_kt;
+        c_first = sk_owner(p, units, i0);
+        c_last = sk_owner(p, units, i0 + P.num_kt - 1);
+      }
+      // the partial slot of unit u (one per unit: a unit stores at most one
+      // partial, for its first segment)
+      auto slot_idx = [&](int u) { return (int64_t)u * (kPair ? 2 : 1) + (int64_t)rank; };
+      // a unit with an empty range (possible when the ranges are cut by
+      // cost) contributes nothing
+      auto live = [&](int u) { return p.sk_bound[u] < p.sk_bound[u + 1]; };
+      if (finisher && et == 0) {
+        bool ok2 = true;
+        for (int v = c_first + 1; v <= c_last && ok2; ++v) {
+          if (!live(v)) continue;
+          const unsigned int* f = sk_flags + slot_idx(v);
+          if (ld_acquire_gpu(f) == 0u) {
+            const uint64_t t0 = globaltimer_ns();
+            while (ld_acquire_gpu(f) == 0u) {
+              if (globaltimer_ns() - t0 > p.timeout_ns) {
+                record_dev_error(kDevErrWaitCounter);
+                ok2 = false;
+                break;
+              }
+            }
+          }
+        }
+        *last_flag = ok2 ? 1 : 2;
+      }
       bool ok = mbar_wait(accf_bar(buf), acc_phase, p.timeout_ns, kDevErrWaitAccFull);
       __syncwarp();
-      ok = named_bar_red_and(2, 128, ok);  // all epilogue threads agree
+      ok = named_bar_red_and(2, 128, ok);  // all epilogue threads agree (and see last_flag)
       if (!ok) {
         *abort_flag = 1;
         break;
       }
       tc_fence_after_sync();
       const uint32_t tbase = tmem_base + ((uint32_t)(lg * 32) << 16) + buf * kBN;
-      const bool full = (kb == 0 && ke == P.num_kt);
 
       // Scales and stores 16 consecutive accumulator columns starting at c0
       // with 16-byte vector stores.  Rows of Y are 16-byte aligned (checked
@@ -997,117 +1044,76 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
           store16_any(v, c0);
         }
         release_acc();
-      } else {
-        // a split tile: its contributors are the units whose ranges cover it
-        const int64_t i0 = P.iter_begin + (int64_t)tile * P.num_kt;
-        const int c_first = sk_owner(total_iters, units, i0);
-        const int c_last = sk_owner(total_iters, units, i0 + P.num_kt - 1);
-        const unsigned int count = (unsigned int)(c_last - c_first + 1);
-        const int64_t cslot = (int64_t)tile * (kPair ? 2 : 1) + (int64_t)rank;
-        // slot s of unit u: 0 for the unit's first segment, 1 for its last
-        auto slot_idx = [&](int u, int sidx) { return ((int64_t)u * (kPair ? 2 : 1) + (int64_t)rank) * 2 + sidx; };
-        // the other contributor v's segment of this tile is v's first one
-        // exactly when v's range starts inside the tile
-        auto slot_of = [&](int v) { return ((int64_t)v * total_iters / units) >= i0 ? 0 : 1; };
-        named_bar_sync(1, 128);
+      } else if (!finisher) {
+        // store the partial tile (plain stores), then raise the flag
+        // slot layout: float4 (col / 4) of row r at index (col / 4) * 128 + r,
+        // so each warp store covers 512 contiguous bytes
+        const int64_t my = slot_idx(unit);
+        float4* dst = reinterpret_cast<float4*>(sk_slots + my * 128 * kBN) + row;
+#pragma unroll 1
+        for (int c0 = 0; c0 < bn; c0 += 16) {
+          uint32_t r[16];
+          tmem_ld_x16(tbase + c0, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            __stcg(dst + (c0 / 4 + j) * 128,
+                   make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                               __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3])));
+        }
+        release_acc();
+        named_bar_sync(1, 128);  // every store of the tile precedes the flag
         if (et == 0) {
-          const unsigned int old = atom_add_acq_rel_gpu(&P.ws_counters[cslot], 1u);
-          *last_flag = (old == count - 1) ? 1 : 0;
+          __threadfence();
+          st_release_gpu(sk_flags + my, 1u);
         }
-        named_bar_sync(1, 128);
-        if (!*last_flag) {
-          // store the partial tile (plain stores), then raise the flag
-          const int64_t my = slot_idx(unit, seg == 0 ? 0 : 1);
-          // slot layout: float4 (col / 4) of row r at index (col / 4) * 128 + r,
-          // so each warp store covers 512 contiguous bytes
-          float4* dst = reinterpret_cast<float4*>(sk_slots + my * 128 * kBN) + row;
+      } else {
+        // the finisher: our accumulator plus the others' partials, 64
+        // columns at a time
+        const bool have = *last_flag == 1;
+        constexpr int kFix = kBN < 64 ? kBN : 64;
 #pragma unroll 1
-          for (int c0 = 0; c0 < bn; c0 += 16) {
+        for (int cb = 0; cb < bn; cb += kFix) {
+          float4 q[kFix / 4];
+#pragma unroll
+          for (int j = 0; j < kFix / 4; ++j) q[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (have) {
+            for (int v = c_first + 1; v <= c_last; ++v) {
+              if (!live(v)) continue;
+              const float4* src = reinterpret_cast<const float4*>(sk_slots + slot_idx(v) * 128 * kBN) + row;
+              float4 t[kFix / 4];
+#pragma unroll
+              for (int j = 0; j < kFix / 4; ++j) t[j] = __ldcg(src + (cb / 4 + j) * 128);
+#pragma unroll
+              for (int j = 0; j < kFix / 4; ++j) {
+                q[j].x += t[j].x; q[j].y += t[j].y; q[j].z += t[j].z; q[j].w += t[j].w;
+              }
+            }
+          }
+#pragma unroll
+          for (int c0 = 0; c0 < kFix; c0 += 16) {
+            if (cb + c0 >= bn) break;  // a problem narrower than the kernel's tile
             uint32_t r[16];
-            tmem_ld_x16(tbase + c0, r);
+            tmem_ld_x16(tbase + cb + c0, r);
             tmem_ld_wait();
+            float v[16];
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-              __stcg(dst + (c0 / 4 + j) * 128,
-                     make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
-                                 __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3])));
-          }
-          release_acc();
-          named_bar_sync(1, 128);  // every store of the tile precedes the flag
-          if (et == 0) {
-            __threadfence();
-            st_release_gpu(sk_flags + my, 1u);
-          }
-        } else {
-          // wait (bounded) for the other contributors' flags
-          bool ok2 = true;
-          if (et == 0) {
-            for (int v = c_first; v <= c_last && ok2; ++v) {
-              if (v == unit) continue;
-              const unsigned int* f = sk_flags + slot_idx(v, slot_of(v));
-              if (ld_acquire_gpu(f) == 0u) {
-                const uint64_t t0 = globaltimer_ns();
-                while (ld_acquire_gpu(f) == 0u) {
-                  if (globaltimer_ns() - t0 > p.timeout_ns) {
-                    record_dev_error(kDevErrWaitCounter);
-                    ok2 = false;
-                    break;
-                  }
-                }
-              }
+            for (int j = 0; j < 4; ++j) {
+              const float4 t = q[c0 / 4 + j];
+              v[4 * j] = __uint_as_float(r[4 * j]) + t.x;
+              v[4 * j + 1] = __uint_as_float(r[4 * j + 1]) + t.y;
+              v[4 * j + 2] = __uint_as_float(r[4 * j + 2]) + t.z;
+              v[4 * j + 3] = __uint_as_float(r[4 * j + 3]) + t.w;
             }
-            *last_flag = ok2 ? 1 : 2;
+            store16_any(v, cb + c0);
           }
-          named_bar_sync(1, 128);
-          const bool have = *last_flag == 1;
-          // our accumulator plus the others' partials, 64 columns at a time
-          constexpr int kFix = kBN < 64 ? kBN : 64;
-#pragma unroll 1
-          for (int cb = 0; cb < bn; cb += kFix) {
-            float4 q[kFix / 4];
-#pragma unroll
-            for (int j = 0; j < kFix / 4; ++j) q[j] = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (have) {
-              for (int v = c_first; v <= c_last; ++v) {
-                if (v == unit) continue;
-                const float4* src = reinterpret_cast<const float4*>(sk_slots + slot_idx(v, slot_of(v)) * 128 * kBN) + row;
-                float4 t[kFix / 4];
-#pragma unroll
-                for (int j = 0; j < kFix / 4; ++j) t[j] = __ldcg(src + (cb / 4 + j) * 128);
-#pragma unroll
-                for (int j = 0; j < kFix / 4; ++j) {
-                  q[j].x += t[j].x; q[j].y += t[j].y; q[j].z += t[j].z; q[j].w += t[j].w;
-                }
-              }
-            }
-#pragma unroll
-            for (int c0 = 0; c0 < kFix; c0 += 16) {
-              if (cb + c0 >= bn) break;  // a problem narrower than the kernel's tile
-              uint32_t r[16];
-              tmem_ld_x16(tbase + cb + c0, r);
-              tmem_ld_wait();
-              float v[16];
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const float4 t = q[c0 / 4 + j];
-                v[4 * j] = __uint_as_float(r[4 * j]) + t.x;
-                v[4 * j + 1] = __uint_as_float(r[4 * j + 1]) + t.y;
-                v[4 * j + 2] = __uint_as_float(r[4 * j + 2]) + t.z;
-                v[4 * j + 3] = __uint_as_float(r[4 * j + 3]) + t.w;
-              }
-              store16_any(v, cb + c0);
-            }
-          }
-          release_acc();
-          named_bar_sync(1, 128);  // every read of the partials precedes the reset
-          if (et == 0) {
-            // ready for the next call
-            for (int v = c_first; v <= c_last; ++v)
-              if (v != unit) sk_flags[slot_idx(v, slot_of(v))] = 0u;
-            P.ws_counters[cslot] = 0u;
-          }
-          if (!have) *abort_flag = 1;
         }
+        release_acc();
+        named_bar_sync(1, 128);  // every read of the partials precedes the reset
+        if (et == 0)  // ready for the next call
+          for (int v = c_first + 1; v <= c_last; ++v)
+            if (live(v)) sk_flags[slot_idx(v)] = 0u;
+        if (!have) *abort_flag = 1;
       }
       ++acc_i;
     }

@@ -159,29 +159,78 @@ int stage_k(int mode, bool bf16) {
   return bf16 ? 64 : 128;
 }
 
-// Stream-K workspace: two partial-tile slots per scheduling unit (and pair
-// half), a flag per slot, and an arrival counter per tile (and pair half).
-size_t sk_slot_count(const Plan& pl) { return (size_t)pl.grid * (pl.pair ? 2 : 1) * 2; }
+// Stream-K workspace: one partial-tile slot per scheduling unit (and pair
+// half) and a flag per slot.  A unit stores at most one partial tile (for its
+// first segment, when its range starts inside a tile); the unit holding a
+// split tile's first K-stage finishes it.
+size_t sk_slot_count(const Plan& pl) { return (size_t)pl.grid * (pl.pair ? 2 : 1); }
 size_t round256(size_t b) { return (b + 255) & ~(size_t)255; }
 size_t sk_slots_bytes(const Plan& pl) { return round256(sk_slot_count(pl) * pl.bn * 128 * sizeof(float)); }
 size_t sk_flags_bytes(const Plan& pl) { return round256(sk_slot_count(pl) * sizeof(unsigned int)); }
-
-size_t sk_counters_bytes(const Plan& pl) {
-  return round256((size_t)pl.total_tiles * (pl.pair ? 2 : 1) * sizeof(unsigned int));
-}
-// Layout: [counters][flags][partial-tile slots]; the first two are the state
-// that must be zero between calls.
-size_t sk_state_bytes(const Plan& pl) { return sk_counters_bytes(pl) + sk_flags_bytes(pl); }
+// Layout: [flags][partial-tile slots]; the flags are the state that must be
+// zero between calls.
+size_t sk_state_bytes(const Plan& pl) { return sk_flags_bytes(pl); }
 size_t sk_ws_bytes(const Plan& pl) { return sk_state_bytes(pl) + sk_slots_bytes(pl); }
+
+// Costs for cutting the stream-K ranges, in units of ~1/64 of a K-stage: a
+// stage streams the same weight bytes at every token-tile width, and a
+// 128-wide token tile adds its B tile (from L2) and longer MMAs (~4%,
+// measured per CTA on the decode workload); every tile a unit starts adds
+// its accumulator hand-over and epilogue (~0.2-0.5 us, measured as the
+// difference between problems with 20- and 100-stage tiles).
+constexpr int64_t kSkStageCost = 64, kSkTileCost = 32;
+int64_t sk_stage_cost(int bn) { return kSkStageCost + (bn >= 128 ? 3 : bn >= 64 ? 2 : 0); }
+
+// Cost of the first k stages of a problem (tiles of num_kt stages): k stages
+// plus one tile start per tile begun.
+int64_t sk_prefix_cost(int64_t k, int num_kt, int64_t c) {
+  return k * c + (k + num_kt - 1) / num_kt * kSkTileCost;
+}
+
+// Cuts the stream-K ranges: unit u gets the global K-stages from bound[u] to
+// bound[u + 1], so that every unit's summed cost is as equal as whole stages
+// allow.
+void set_sk_bounds(GemmParams& gp, const Plan& pl) {
+  if (pl.sched != kSchedStreamK) return;
+  int64_t total = 0;
+  for (int i = 0; i < pl.n; ++i) {
+    const int64_t stages = (int64_t)pl.tiles_a[i] * pl.tiles_b[i] * pl.num_kt[i];
+    total += sk_prefix_cost(stages, pl.num_kt[i], sk_stage_cost(pl.bn_i[i]));
+  }
+  int64_t stage0 = 0, cost0 = 0;  // first global stage and cost before problem i
+  int i = 0;
+  gp.sk_bound[0] = 0;
+  for (int u = 1; u < pl.grid; ++u) {
+    const int64_t target = total * u / pl.grid;
+    int64_t stages = (int64_t)pl.tiles_a[i] * pl.tiles_b[i] * pl.num_kt[i];
+    int64_t c = sk_stage_cost(pl.bn_i[i]);
+    while (i + 1 < pl.n && cost0 + sk_prefix_cost(stages, pl.num_kt[i], c) <= target) {
+      stage0 += stages;
+      cost0 += sk_prefix_cost(stages, pl.num_kt[i], c);
+      ++i;
+      stages = (int64_t)pl.tiles_a[i] * pl.tiles_b[i] * pl.num_kt[i];
+      c = sk_stage_cost(pl.bn_i[i]);
+    }
+    // the first stage k of problem i whose prefix cost reaches the target
+    int64_t lo = 0, hi = stages;
+    while (lo < hi) {
+      const int64_t mid = (lo + hi) / 2;
+      if (cost0 + sk_prefix_cost(mid, pl.num_kt[i], c) >= target) hi = mid;
+      else lo = mid + 1;
+    }
+    gp.sk_bound[u] = std::max(stage0 + lo, gp.sk_bound[u - 1]);
+  }
+  gp.sk_bound[pl.grid] = pl.total_iters;
+}
 
 // Work schedule, from a cost model in units of one K-stage of one scheduling
 // unit (an SM, or a CTA pair; streaming one stage of weights takes about the
 // same time on every unit when all units stream):
 //   whole tiles round-robin: ceil(tiles / SMs) * stages of the longest tile
 //   stream-K:                ceil(tiles * stages / SMs) + the cost of finishing
-//                            the split tiles (fp32 atomics into an accumulator,
-//                            then one pass over it), which grows with the tile
-//                            width BN: about 2 + BN^2 / 800 stage-equivalents.
+//                            the split tiles (partials stored, then added by
+//                            the finisher), which grows with the tile width
+//                            BN: at most 2 + BN^2 / 800 stage-equivalents.
 // Stream-K needs a workspace for the accumulators; without enough of it the
 // whole-tile schedule is used.
 void choose_schedule(Plan& pl, int sms, size_t ws_cap) {
@@ -214,7 +263,7 @@ void choose_schedule(Plan& pl, int sms, size_t ws_cap) {
   const double cost_sk = (double)((iters + sms - 1) / sms) + 2.0 + pl.bn * pl.bn / 800.0;
   Plan t = pl;
   t.sched = kSchedStreamK;
-  t.grid = (int)std::min<int64_t>(iters, sms);
+  t.grid = (int)std::min<int64_t>(std::min<int64_t>(iters, sms), kMaxSkUnits);
   t.ws_bytes = sk_ws_bytes(t);
   if (cost_sk < cost_dp && t.ws_bytes <= ws_cap) pl = t;
 }
@@ -450,7 +499,7 @@ Plan plan_gemm(const sp24_gemm_args* a, const DeviceInfo& di, size_t ws_cap) { r
 // Tensor maps and problem record of problem i of a launch.
 template <int kMaxProb>
 bool fill_problem(GemmLaunch<kMaxProb>& gl, int i, const sp24_gemm_args* a, const Plan& pl,
-                  int64_t iter_begin, int tile_begin, unsigned int* counters) {
+                  int64_t iter_begin, int tile_begin) {
   const int eb = dtype_bytes(a->in_dtype);
   const int box_elems = 128 / eb;  // 128 bytes
   bool ok = true;
@@ -499,7 +548,6 @@ bool fill_problem(GemmLaunch<kMaxProb>& gl, int i, const sp24_gemm_args* a, cons
   P.scale_b = a->in_dtype == SP24_E4M3 ? a->x_scales : nullptr;
   P.Y = a->Y;
   P.ldy = a->ldy;
-  P.ws_counters = counters;
   return ok;
 }
 
@@ -512,19 +560,18 @@ int build_launch(GemmLaunch<kMaxProb>& gl, const sp24_gemm_args* const* a, int n
   int tile = 0;
   const bool sk = pl.sched == kSchedStreamK;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  unsigned int* counters = sk ? reinterpret_cast<unsigned int*>(ws) : nullptr;
   for (int i = 0; i < n; ++i) {
     const int tiles = pl.tiles_a[i] * pl.tiles_b[i];
-    if (!fill_problem(gl, i, a[i], pl, iter, tile, sk ? counters : nullptr)) return SP24_ERR_CUDA;
-    if (sk) counters += (size_t)tiles * (pl.pair ? 2 : 1);
+    if (!fill_problem(gl, i, a[i], pl, iter, tile)) return SP24_ERR_CUDA;
     iter += (int64_t)tiles * pl.num_kt[i];
     tile += tiles;
   }
-  gl.p.sk_flags = sk ? reinterpret_cast<unsigned int*>(ws + sk_counters_bytes(pl)) : nullptr;
+  gl.p.sk_flags = sk ? reinterpret_cast<unsigned int*>(ws) : nullptr;
   gl.p.sk_slots = sk ? reinterpret_cast<float*>(ws + sk_state_bytes(pl)) : nullptr;
   gl.p.n_prob = n;
   gl.p.sched = pl.sched;
   gl.p.total_iters = pl.total_iters;
+  set_sk_bounds(gl.p, pl);
   gl.p.total_tiles = pl.total_tiles;
   gl.p.out_f32 = a[0]->out_dtype == SP24_F32;
   gl.p.use_pdl = 1;
@@ -1012,12 +1059,12 @@ int build_launch_nvfp4(GemmLaunch<1>& gl, const sp24_nvfp4_gemm_args* a, const P
   P.scale_b = a->x_tensor_scale;
   P.Y = a->Y;
   P.ldy = a->ldy;
-  P.ws_counters = sk ? reinterpret_cast<unsigned int*>(ws) : nullptr;
-  gl.p.sk_flags = sk ? reinterpret_cast<unsigned int*>(ws + sk_counters_bytes(pl)) : nullptr;
+  gl.p.sk_flags = sk ? reinterpret_cast<unsigned int*>(ws) : nullptr;
   gl.p.sk_slots = sk ? reinterpret_cast<float*>(ws + sk_state_bytes(pl)) : nullptr;
   gl.p.n_prob = 1;
   gl.p.sched = pl.sched;
   gl.p.total_iters = pl.total_iters;
+  set_sk_bounds(gl.p, pl);
   gl.p.total_tiles = pl.total_tiles;
   gl.p.out_f32 = a->out_dtype == SP24_F32;
   gl.p.use_pdl = 1;

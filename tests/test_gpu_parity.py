@@ -307,6 +307,27 @@ def test_grouped_gemm_mixed_token_classes(group, e4, tactic, use_ws):
         check_group(items, "mixed group %s e4=%s tactic=%d ws=%s f32=%s" % (group, e4, tactic, use_ws, out_f32))
 
 
+@pytest.mark.parametrize("group", ["decode", "to32"])
+def test_stream_k_split_is_fixed_and_repeats_bitwise(group):
+    """A split tile is finished by the unit that holds its first K-stage, so the
+    split and the fp32 addition order depend only on the plan: repeated calls
+    (and a call after other launches on the same workspace) give identical
+    bytes, and agree with the oracle."""
+    shapes = GROUPS[group] if group in GROUPS else MIXED_GROUPS[group]
+    grp, items = run_group(shapes, True, sp24.SPARSE, True, seed=11)
+    assert grp.workspace_bytes() > 0  # the stream-K schedule, with split tiles
+    first = [Y.clone() for (_, Y, _, _) in items]
+    for _ in range(3):
+        for (_, Y, _, _) in items:
+            Y.fill_(float("nan"))
+        grp()
+        torch.cuda.synchronize()
+        assert sp24.last_device_error() == sp24.SP24_OK
+        for y0, (_, Y, _, _) in zip(first, items):
+            assert torch.equal(y0.view(torch.int32), Y.view(torch.int32))
+    check_group(items, "stream-K repeat %s" % group)
+
+
 @pytest.mark.parametrize("e4", [False, True])
 def test_grouped_gemm_whole_tiles_without_workspace(e4):
     grp, items = run_group(GROUPS["decode"], e4, sp24.SPARSE, True, use_ws=False)
@@ -937,12 +958,14 @@ def test_tiny_configuration_seed0_matches_oracle():
     check_tolerance(y, y_ref, a_ref, "tiny e4m3")
 
 
-def test_decode_step_full_size_grouped_sampled():
+@pytest.mark.parametrize("grouping", ["one_launch", "by_class"])
+def test_decode_step_full_size_grouped_sampled(grouping):
     """The decode step as the benchmark times it: 16 GEMMs (M in 1, 8, 32, 128
     times the four weight shapes, e4m3 2:4 weights), one grouped per-token cast,
-    then one grouped launch per token-count class, weights marked static, the
-    second and third groups chained after the first as independent launches.
-    Sampled outputs of every GEMM against the oracle."""
+    then the 16 GEMMs as one grouped launch (each problem with its own
+    token-tile width), or as one launch per token-count class with the second
+    and third chained after the first as independent launches; weights marked
+    static.  Sampled outputs of every GEMM against the oracle."""
     g = np.random.default_rng(7)
     Wb = {}
     for (N, K) in inputs.DECODE_NK:
@@ -966,9 +989,9 @@ def test_decode_step_full_size_grouped_sampled():
     cast = sp24.QuantGroup([(it["Xd"], it["xq"], it["xs"]) for it in items])
     by = {}
     for it in items:
-        by.setdefault(sp24.m_class(it["M"]), []).append(it["a"])
+        by.setdefault(sp24.m_class(it["M"]) if grouping == "by_class" else 0, []).append(it["a"])
     groups = [sp24.GemmGroup(v, after_independent=i > 0) for i, (_, v) in enumerate(sorted(by.items()))]
-    assert len(groups) == 3
+    assert len(groups) == (3 if grouping == "by_class" else 1)
     torch.cuda.synchronize()
     for _ in range(2):  # the second pass runs on workspaces the first left at zero
         cast()
