@@ -174,12 +174,14 @@ size_t sk_ws_bytes(const Plan& pl) { return sk_state_bytes(pl) + sk_slots_bytes(
 
 // Costs for cutting the stream-K ranges, in units of ~1/64 of a K-stage: a
 // stage streams the same weight bytes at every token-tile width, and a
-// 128-wide token tile adds its B tile (from L2) and longer MMAs (~4%,
+// 128-wide token tile adds its B tile (from L2) and longer MMAs (~4-8%,
 // measured per CTA on the decode workload); every tile a unit starts adds
 // its accumulator hand-over and epilogue (~0.2-0.5 us, measured as the
-// difference between problems with 20- and 100-stage tiles).
-constexpr int64_t kSkStageCost = 64, kSkTileCost = 32;
-int64_t sk_stage_cost(int bn) { return kSkStageCost + (bn >= 128 ? 3 : bn >= 64 ? 2 : 0); }
+// difference between problems with 20- and 100-stage tiles).  Against equal
+// stage counts per unit these weights took the decode step's one launch from
+// 0.160 to 0.151 ms (a first set, 3 and 32, to 0.153).
+constexpr int64_t kSkStageCost = 64, kSkTileCost = 48;
+int64_t sk_stage_cost(int bn) { return kSkStageCost + (bn >= 128 ? 5 : bn >= 64 ? 3 : 0); }
 
 // Cost of the first k stages of a problem (tiles of num_kt stages): k stages
 // plus one tile start per tile begun.
