@@ -265,7 +265,11 @@ int sp24_gemm(const sp24_gemm_args *args, void *stream);
  * stream their weights next to wider ones (fewer pipeline stages than a
  * launch of small-M problems alone).  Hybrid problems run 128-row tiles on
  * single CTAs, each stage two tile columns, dense or sparse as their flags
- * say.  Each args'
+ * say.  On the stream-K schedule, the first call with a given argument block
+ * copies the problems' tile masks to the host (a small copy on `stream`,
+ * waited for; skipped while `stream` is being captured) to cut the K ranges
+ * by the bytes each step streams; the masks only steer that balance, the
+ * kernel reads them itself.  The same holds for sp24_gemm.  Each args'
  * own workspace fields are ignored: the group uses `workspace` (size from
  * sp24_gemm_grouped_workspace_bytes, same zero-fill rule as sp24_gemm).
  * SP24_GEMM_W_STATIC applies when every problem sets it. */

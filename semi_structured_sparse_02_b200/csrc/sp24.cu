@@ -189,11 +189,71 @@ int64_t sk_prefix_cost(int64_t k, int num_kt, int64_t c) {
   return k * c + (k + num_kt - 1) / num_kt * kSkTileCost;
 }
 
+// Hybrid weights: the cost of each scheduling step from the tile masks, in the
+// same units: two sparse tile columns 64, two dense 100, one of each 120 (a
+// mixed step costs more than its 26 KB: measured ~0.94 us against ~0.47 for
+// two sparse columns and ~0.71 for two dense ones; with costs proportional
+// to bytes the cut measured no better than equal step counts, with these it
+// took the four 25%-dense GEMMs at one token from 35.0 to 34.3 us), plus the
+// tile starts.  The masks are copied to the host once, when the launch is first
+// planned, and only when the stream is not being captured; they only steer
+// the balance (the kernel reads the masks itself).  Returns false when the
+// masks cannot be read.
+bool hybrid_step_costs(const Plan& pl, const sp24_gemm_args* const* a, cudaStream_t stream,
+                       std::vector<int64_t>& cost) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) {
+    cudaGetLastError();
+    return false;
+  }
+  cost.clear();
+  std::vector<uint8_t> mask;
+  for (int i = 0; i < pl.n; ++i) {
+    const int64_t kcols = a[i]->K / 128, blocks = (a[i]->N + 127) / 128;
+    mask.resize((size_t)(kcols * blocks));
+    if (cudaMemcpyAsync(mask.data(), a[i]->tile_dense_mask, mask.size(), cudaMemcpyDeviceToHost, stream) !=
+            cudaSuccess ||
+        cudaStreamSynchronize(stream) != cudaSuccess) {
+      cudaGetLastError();
+      return false;
+    }
+    for (int64_t t = 0; t < (int64_t)pl.tiles_a[i] * pl.tiles_b[i]; ++t) {
+      const int64_t ta = t % pl.tiles_a[i];
+      for (int kt = 0; kt < pl.num_kt[i]; ++kt) {
+        const int64_t c0 = 2 * (int64_t)kt, c1 = c0 + 1;
+        const bool d0 = mask[(size_t)(ta * kcols + c0)] != 0;
+        int64_t c;
+        if (c1 >= kcols) c = d0 ? 51 : 32;
+        else {
+          const bool d1 = mask[(size_t)(ta * kcols + c1)] != 0;
+          c = (d0 && d1) ? 100 : (d0 || d1) ? 120 : 64;
+        }
+        cost.push_back(c + (kt == 0 ? kSkTileCost : 0));
+      }
+    }
+  }
+  return (int64_t)cost.size() == pl.total_iters;
+}
+
 // Cuts the stream-K ranges: unit u gets the global K-stages from bound[u] to
 // bound[u + 1], so that every unit's summed cost is as equal as whole stages
 // allow.
-void set_sk_bounds(GemmParams& gp, const Plan& pl) {
+void set_sk_bounds(GemmParams& gp, const Plan& pl, const sp24_gemm_args* const* a, cudaStream_t stream) {
   if (pl.sched != kSchedStreamK) return;
+  std::vector<int64_t> cost;
+  if (pl.mode == kModeHybrid && a != nullptr && hybrid_step_costs(pl, a, stream, cost)) {
+    int64_t total = 0;
+    for (int64_t c : cost) total += c;
+    int64_t acc = 0, st = 0;  // cost of the stages before stage st
+    gp.sk_bound[0] = 0;
+    for (int u = 1; u < pl.grid; ++u) {
+      const int64_t target = total * u / pl.grid;
+      while (st < pl.total_iters && acc < target) acc += cost[(size_t)st++];
+      gp.sk_bound[u] = std::max(st, gp.sk_bound[u - 1]);
+    }
+    gp.sk_bound[pl.grid] = pl.total_iters;
+    return;
+  }
   int64_t total = 0;
   for (int i = 0; i < pl.n; ++i) {
     const int64_t stages = (int64_t)pl.tiles_a[i] * pl.tiles_b[i] * pl.num_kt[i];
@@ -556,7 +616,7 @@ bool fill_problem(GemmLaunch<kMaxProb>& gl, int i, const sp24_gemm_args* a, cons
 // Fills a launch for n problems with the plan's schedule and workspace.
 template <int kMaxProb>
 int build_launch(GemmLaunch<kMaxProb>& gl, const sp24_gemm_args* const* a, int n, const Plan& pl,
-                 void* workspace, bool w_static) {
+                 void* workspace, bool w_static, cudaStream_t stream) {
   memset(&gl, 0, sizeof gl);
   int64_t iter = 0;
   int tile = 0;
@@ -573,7 +633,7 @@ int build_launch(GemmLaunch<kMaxProb>& gl, const sp24_gemm_args* const* a, int n
   gl.p.n_prob = n;
   gl.p.sched = pl.sched;
   gl.p.total_iters = pl.total_iters;
-  set_sk_bounds(gl.p, pl);
+  set_sk_bounds(gl.p, pl, a, stream);
   gl.p.total_tiles = pl.total_tiles;
   gl.p.out_f32 = a[0]->out_dtype == SP24_F32;
   gl.p.use_pdl = 1;
@@ -898,7 +958,8 @@ int run_gemm(const sp24_gemm_args* a, cudaStream_t stream) {
   if (g_cache_single.find(key, [&](const SingleLaunch& v) { st = dispatch_gemm(v.pl, v.gl, stream); })) return st;
   static thread_local SingleLaunch v;
   v.pl = plan_gemm(a, di, ws_cap);
-  if ((st = build_launch(v.gl, &a, 1, v.pl, a->workspace, (a->flags & SP24_GEMM_W_STATIC) != 0)) != SP24_OK)
+  if ((st = build_launch(v.gl, &a, 1, v.pl, a->workspace, (a->flags & SP24_GEMM_W_STATIC) != 0, stream)) !=
+      SP24_OK)
     return st;
   g_cache_single.put(key, v);
   return dispatch_gemm(v.pl, v.gl, stream);
@@ -1066,7 +1127,7 @@ int build_launch_nvfp4(GemmLaunch<1>& gl, const sp24_nvfp4_gemm_args* a, const P
   gl.p.n_prob = 1;
   gl.p.sched = pl.sched;
   gl.p.total_iters = pl.total_iters;
-  set_sk_bounds(gl.p, pl);
+  set_sk_bounds(gl.p, pl, nullptr, nullptr);
   gl.p.total_tiles = pl.total_tiles;
   gl.p.out_f32 = a->out_dtype == SP24_F32;
   gl.p.use_pdl = 1;
@@ -1371,7 +1432,7 @@ int sp24_gemm_grouped(const sp24_gemm_args* args, int n, void* workspace, size_t
   if (g_cache_group.find(key, [&](const GroupLaunch& v) { st = dispatch_gemm_group(v.pl, v.gl, s); })) return st;
   static thread_local GroupLaunch v;  // large: keep it off the stack
   v.pl = plan_group(ptrs, n, di, workspace != nullptr ? workspace_bytes : 0);
-  if ((st = build_launch(v.gl, ptrs, n, v.pl, workspace, w_static)) != SP24_OK) return st;
+  if ((st = build_launch(v.gl, ptrs, n, v.pl, workspace, w_static, s)) != SP24_OK) return st;
   g_cache_group.put(key, v);
   return dispatch_gemm_group(v.pl, v.gl, s);
 }
@@ -1390,7 +1451,7 @@ int sp24_gemm_noalloc(const sp24_gemm_args* a, void* stream) {
   if (pl.ws_bytes > kStaticScratchBytes) return SP24_ERR_WORKSPACE;
   void* scratch = nullptr;
   if ((st = static_scratch(&scratch)) != SP24_OK) return st;
-  // the flags and counters must start at zero; the array keeps whatever
+  // the partial-tile flags must start at zero; the array keeps whatever
   // the previous call on this device left in it
   if (pl.sched == kSchedStreamK && cudaMemsetAsync(scratch, 0, sk_state_bytes(pl), s) != cudaSuccess) {
     cudaGetLastError();
