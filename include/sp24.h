@@ -201,9 +201,10 @@ typedef struct sp24_gemm_args {
 #define SP24_GEMM_W_STATIC 1u
 
 /* Shapes with M >= 256 tokens and N >= 256 output features run on CTA
- * pairs: one tcgen05 MMA over two SMs computes a 256 x 256 output tile, each
- * SM loading half of both operands (no workspace).  With a hybrid mask they
- * do so only when the 256 x 256 tiles are at least as many as the pairs that
+ * pairs: one tcgen05 MMA over two SMs computes a 256 x 256 output tile (256
+ * weight rows x 240 tokens when the weights are sparse or hybrid), each SM
+ * loading half of both operands (no workspace).  With a hybrid mask they
+ * do so only when those tiles are at least as many as the pairs that
  * fit on the device at once (a pair's K-step runs dense when either of its
  * two row blocks is dense there, which costs more than the one-CTA kernel's
  * per-tile choice unless the one-CTA kernel is short of tiles).  This flag
@@ -225,7 +226,7 @@ typedef struct sp24_gemm_args {
  * kernel).  The call then starts its work as soon as SMs free up, without
  * waiting for the preceding GEMM to finish, and waits for it only before
  * exiting, so that its own completion still implies the preceding call's.
- * Ignored by the CTA-pair (256 x 256 tile) kernel, which always waits.  In a
+ * Ignored by the CTA-pair kernel, which always waits.  In a
  * grouped call it applies when every problem sets it.  Meant for chains of
  * independent GEMMs after one producer, such as a layer's projections after
  * one activation cast. */
