@@ -9,20 +9,22 @@
 //                shared -> tensor memory) and tcgen05.mma into one of two fp32
 //                accumulators in tensor memory, then tcgen05.commit.
 //   warps 2..5   epilogue: tcgen05.ld of the accumulator, scales, output
-//                store; or a stream-K partial add + last-arriver finish.
+//                store; or a stream-K partial store / finish.
 //
 // Work schedule.  "Data-parallel": each CTA takes whole output tiles
 // round-robin over the tiles of all problems.  "Stream-K" (few tiles, e.g.
 // decode): the K-iterations of all tiles of all problems are laid end to end
-// and every CTA streams one equal contiguous range of them, so every SM moves
-// the same number of bytes and a group streams without gaps between problems.
-// A tile split between CTAs is finished by whichever contributor takes the
-// last ticket: every other contributor stores its fp32 partial tile with
-// plain stores into a slot of its own (a unit has at most two split tiles,
-// its first and its last segment) and raises a flag; the last one adds those
-// partials to its own accumulator as it drains tensor memory, stores Y and
-// clears the flags and the ticket for the next call.  Which contributor
-// finishes varies between runs, and with it the fp32 addition order.
+// and every CTA streams one contiguous range of them (the host cuts the
+// ranges by estimated cost and passes the boundaries), so a group streams
+// without gaps between problems.  A tile split between CTAs is finished by
+// the unit that holds its first K-iteration: that unit's range ends inside
+// the tile, so the tile is its last segment, while every other contributor's
+// segment lies at the start of (or spans) its own range.  The others store
+// their fp32 partial tile with plain stores into their one slot and raise a
+// flag; the finisher checks the flags before its own accumulator is ready,
+// adds the partials as it drains tensor memory, stores Y and clears the
+// flags for the next call.  The split, and with it the fp32 addition order,
+// is fixed by the plan.
 //
 // Kernel chaining.  Every CTA triggers the dependent grid at once
 // (programmatic dependent launch).  With w_static the producer starts
