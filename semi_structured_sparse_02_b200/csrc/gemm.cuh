@@ -148,7 +148,10 @@ struct GemmCfg {
   // bookkeeping after the stages: barriers, slots, the B-scale slice, and a
   // 2 KB output-staging tile per epilogue warp
   static constexpr int kBarOffset = kStages * kStageBytes;
-  static constexpr int kScaleOffset = kBarOffset + 256;
+  static constexpr int kScaleOffset = kBarOffset + 512;
+  // NVFP4: a seventh warp issues each stage's scale and metadata copies into
+  // tensor memory, so the MMA thread issues only the stage's four MMAs
+  static constexpr int kThreads = kNv ? 224 : kGemmThreads;
   static constexpr int kEpiOffset = kScaleOffset + ((kBN * 4 + 127) / 128) * 128;
   static constexpr int kSmemBytes = kEpiOffset + 4 * 2048 + 1024;  // + alignment slack
   static_assert(kSmemBytes <= 232448, "shared memory overflow");
@@ -251,7 +254,7 @@ __device__ __forceinline__ int sk_owner(const GemmParams& p, int units, int64_t 
 }
 
 template <int kMode, bool kBf16, int kBN, bool kAIsW, int kMaxProb, bool kPair = false>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(GemmCfg<kMode, kBf16, kBN, kPair>::kThreads, 1)
 k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
   using C = GemmCfg<kMode, kBf16, kBN, kPair>;
   constexpr int S = C::kStages;
@@ -274,8 +277,9 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
                                              ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOffset);
   // bars[0..S): full, [S..2S): empty, [2S..2S+2): acc_full, [2S+2..2S+4): acc_empty,
-  // [2S+4]: drain.  In a pair the full, acc_empty and drain barriers of rank 0 are used.
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
+  // [2S+4]: drain, [2S+5..3S+5): copies done (NVFP4), [3S+5]: copy drain (NVFP4).
+  // In a pair the full, acc_empty and drain barriers of rank 0 are used.
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * S + 6);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* last_flag = reinterpret_cast<int*>(tmem_slot + 2);
   // hybrid: the kind of each stage in flight (1 = dense), producer -> MMA
@@ -296,6 +300,8 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
   auto accf_bar = [&](int b) { return smem_u32(&bars[2 * S + b]); };
   auto acce_bar = [&](int b) { return smem_u32(&bars[2 * S + 2 + b]); };
   const uint32_t drain_bar = smem_u32(&bars[2 * S + 4]);
+  auto cpd_bar = [&](int s) { return smem_u32(&bars[2 * S + 5 + s]); };
+  const uint32_t cpdrain_bar = smem_u32(&bars[3 * S + 5]);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -307,6 +313,10 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
       mbar_init(acce_bar(b), kPair ? 8 : 4);  // one arrive per epilogue warp (of both CTAs)
     }
     mbar_init(drain_bar, 1);
+    if (C::kNv) {
+      for (int s = 0; s < S; ++s) mbar_init(cpd_bar(s), 1);
+      mbar_init(cpdrain_bar, 1);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -690,7 +700,9 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
         tc_fence_after_sync();
         const uint32_t d = tmem_base + buf * kBN;
         for (int kt = kb; kt < ke; ++kt) {
-          if (!mbar_wait(full_bar(stage), phase, p.timeout_ns, kDevErrWaitFull)) {
+          // NVFP4: the copy warp's commit for this stage completes after the
+          // stage's data arrived and its copies into tensor memory are done
+          if (!mbar_wait(C::kNv ? cpd_bar(stage) : full_bar(stage), phase, p.timeout_ns, kDevErrWaitFull)) {
             ok = false;
             *abort_flag = 1;
             break;
@@ -740,19 +752,10 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
             }
           } else if (C::kNv) {
             const uint64_t so = (uint64_t)((uint32_t)stage * (uint32_t)(C::kStageBytes >> 4));
-            const uint64_t da = da0 + so, db = db0 + so, dsf = dsf0 + so;
+            const uint64_t da = da0 + so, db = db0 + so;
             const uint32_t scol = mcol + C::kMetaChunks * 4;  // A scales; B scales 16 columns on
             auto issue = [&](auto mmas_c) {
               constexpr int kMmas = decltype(mmas_c)::value;
-              if (C::kNvSparse) {
-                if (kMmas == 4) tc_cp_128x256b(tmem_base + mcol, dm2 + so);
-                else tc_cp_128x128b(tmem_base + mcol, dm0 + so);
-              }
-#pragma unroll
-              for (int j = 0; j < kMmas; ++j) {
-                tc_cp_32x128b_x4(tmem_base + scol + 4 * j, dsf + (uint64_t)(32 * j));
-                tc_cp_32x128b_x4(tmem_base + scol + 16 + 4 * j, dsf + (uint64_t)(128 + 32 * j));
-              }
 #pragma unroll
               for (int j = 0; j < kMmas; ++j) {
                 const uint32_t acc = (first && j == 0) ? 0u : 1u;
@@ -841,6 +844,68 @@ k_gemm(const __grid_constant__ GemmLaunch<kMaxProb> g) {
       if (kPair) tc_commit_pair(drain_bar, 0x1);
       else tc_commit(drain_bar);
       mbar_wait(drain_bar, 0, p.timeout_ns, kDevErrWaitDrain);
+    }
+    __syncwarp();
+  } else if (C::kNv && warp == 6) {
+    // ------------------------------------------------------------------ tensor-memory copies (NVFP4)
+    // For every stage, once its data arrived: the metadata chunk(s) (sparse)
+    // and each MMA's A and B scale chunks into the stage's tensor-memory slot,
+    // then a commit to the stage's copies-done barrier, which the MMA thread
+    // waits on instead of the data barrier.  A slot is refilled only after the
+    // producer re-armed its stage, i.e. after the MMAs that read the slot's
+    // previous contents completed.
+    if (wait_first) {
+      pdl_wait();
+      pdl_launch_dependents();
+    }
+    if (lane == 0) {
+      const uint32_t s0 = smem_u32(smem);
+      const uint64_t dm0 = smem_desc(s0 + C::kABytes + C::kBBytes, 16, 128, kLayoutNone);
+      const uint64_t dm2 = smem_desc(s0 + C::kABytes + C::kBBytes, 2048, 128, kLayoutNone);
+      const uint64_t dsf0 = smem_desc(s0 + C::kABytes + C::kBBytes + C::kMetaBytes, 16, 128, kLayoutNone);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      SegIter<kMaxProb> it;
+      it.init(g, unit, units);
+      int pr, tile, kb, ke, seg;
+      while (ok && it.next(g, units, pr, tile, kb, ke, seg)) {
+        const GemmProblem& P = g.prob[pr];
+        for (int kt = kb; kt < ke; ++kt) {
+          if (!mbar_wait(full_bar(stage), phase, p.timeout_ns, kDevErrWaitFull)) {
+            ok = false;
+            *abort_flag = 1;
+            break;
+          }
+          tc_fence_after_sync();
+          const uint64_t so = (uint64_t)((uint32_t)stage * (uint32_t)(C::kStageBytes >> 4));
+          const uint32_t mcol = C::kAccCols + stage * C::kMetaCols;
+          const uint32_t scol = mcol + C::kMetaChunks * 4;  // A scales; B scales 16 columns on
+          const uint64_t dsf = dsf0 + so;
+          auto issue = [&](auto mmas_c) {
+            constexpr int kMmas = decltype(mmas_c)::value;
+            if (C::kNvSparse) {
+              if (kMmas == 4) tc_cp_128x256b(tmem_base + mcol, dm2 + so);
+              else tc_cp_128x128b(tmem_base + mcol, dm0 + so);
+            }
+#pragma unroll
+            for (int j = 0; j < kMmas; ++j) {
+              tc_cp_32x128b_x4(tmem_base + scol + 4 * j, dsf + (uint64_t)(32 * j));
+              tc_cp_32x128b_x4(tmem_base + scol + 16 + 4 * j, dsf + (uint64_t)(128 + 32 * j));
+            }
+          };
+          if (nv_half(P, kt)) issue(std::integral_constant<int, 2>{});
+          else issue(std::integral_constant<int, 4>{});
+          tc_commit(cpd_bar(stage));
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      // drain: every copy issued above has completed
+      tc_commit(cpdrain_bar);
+      mbar_wait(cpdrain_bar, 0, p.timeout_ns, kDevErrWaitDrain);
     }
     __syncwarp();
   } else {

@@ -350,7 +350,7 @@ int launch_gemm_inst(const GemmLaunch<kMaxProb>& gl, int grid, cudaStream_t stre
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(kPair ? 2 * grid : grid);
-  cfg.blockDim = dim3(kGemmThreads);
+  cfg.blockDim = dim3(C::kThreads);
   cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
