@@ -293,12 +293,15 @@ size_t sp24_gemm_grouped_workspace_bytes(const sp24_gemm_args *args, int n);
  * caller that owns every byte of device memory and has none to lend.  It
  * behaves like sp24_gemm but takes its stream-K scratch from a fixed 8 MiB
  * array inside this library (args->workspace and args->workspace_bytes are
- * ignored) and never allocates or frees anything.
+ * ignored) and never allocates or frees device memory.
  * Not from the pages: they have no counterpart; this is an operational
  * variant of sp24_gemm.
  *  - The first call on each device looks up the array's device address (with
  *    that device current) and caches it; make that first call before any
- *    stream capture.
+ *    stream capture.  With hybrid weights on the stream-K schedule, the first
+ *    call with a given argument block also reads the tile mask back to the
+ *    host to balance the schedule (as sp24_gemm does; skipped while `stream`
+ *    is being captured, which leaves the balance unweighted).
  *  - The schedule is the one sp24_gemm picks when given a workspace of
  *    sp24_gemm_noalloc_max_scratch_bytes(): a shape whose stream-K schedule
  *    would need more scratch than that runs whole tiles per CTA (no scratch),
