@@ -169,6 +169,50 @@ def test_nvfp4_device_cast_then_gemm_full_size_sampled():
     del ws
 
 
+@pytest.mark.parametrize("tactic", [sp24.SPARSE, sp24.DENSE])
+def test_nvfp4_prefill_full_size_sampled(tactic):
+    """The prefill shape 8192 x 4096 x 4096 end to end on the device (W pruned
+    and cast, or cast, by the device kernels; X cast per call; the block-scaled
+    GEMM on 128-row tiles); sampled outputs against the oracle's fp64 product of
+    the dequantized operands, with the tensor scales over all of W and X."""
+    M, N, K = 8192, 4096, 4096
+    X, W = inputs.linear_pair(M, N, K, seed=77)
+    blk = 32 if tactic == sp24.SPARSE else 16
+    if tactic == sp24.SPARSE:
+        vals, meta, wsc, wts = _device_48(W)
+    else:
+        vals = torch.empty(N, K // 2, dtype=torch.uint8, device="cuda")
+        wsc = torch.empty(sp24.nvfp4_scales_bytes(N, K, 16), dtype=torch.uint8, device="cuda")
+        wts = torch.empty(1, dtype=torch.float32, device="cuda")
+        sp24.quantize_nvfp4(dev_bf16(W), 16, vals, wsc, wts)
+        meta = None
+    xc = torch.empty(M, K // 2, dtype=torch.uint8, device="cuda")
+    xs = torch.empty(sp24.nvfp4_scales_bytes(M, K, blk), dtype=torch.uint8, device="cuda")
+    xts = torch.empty(1, dtype=torch.float32, device="cuda")
+    sp24.quantize_nvfp4(dev_bf16(X), blk, xc, xs, xts)
+    Y = torch.empty(M, N, dtype=torch.float32, device="cuda")
+    a = sp24.nvfp4_gemm_args(xc, xs, xts, vals, wsc, wts, Y, K, tactic, W_meta=meta)
+    ws = workspace_for_nv(a)
+    sp24.gemm_nvfp4(a)
+    torch.cuda.synchronize()
+    assert sp24.last_device_error() == sp24.SP24_OK
+    g = np.random.default_rng(9)
+    ns = g.choice(N, size=48, replace=False)
+    ms = g.choice(M, size=48, replace=False)
+    if tactic == sp24.SPARSE:
+        wv, wm, wsc_o, wst = orc.nvfp4_48_compress(W)  # tensor scale over all of W
+        W_hat = orc.nvfp4_48_dequant(wv[ns], wm[ns], wsc_o[ns], wst, ns.size, K)
+    else:
+        wv, wsc_o, wst = orc.nvfp4_quantize(W, block=16)
+        W_hat = orc.nvfp4_dequant(wv[ns], wsc_o[ns], wst, ns.size, K, block=16)
+    xc_o, xs_o, xst = orc.nvfp4_quantize(X, block=blk)
+    X_hat = orc.nvfp4_dequant(xc_o[ms], xs_o[ms], xst, ms.size, K, block=blk)
+    y_ref, a_ref = orc.gemm_f64_sampled(X_hat, W_hat, np.arange(ms.size), np.arange(ns.size))
+    y_gpu = Y.cpu().numpy().astype(np.float64)[ms, ns]
+    check_tolerance(y_gpu, y_ref, a_ref, "nvfp4 prefill sampled tactic %d" % tactic)
+    del ws
+
+
 def workspace_for_nv(a):
     n = sp24.gemm_nvfp4_workspace_bytes(a)
     if n == 0:
