@@ -1362,6 +1362,81 @@ def cfg_nvfp4(dev, T, shapes):
     return rows
 
 
+def cfg_nvfp4_step(dev, T):
+    """The decode step's 16 GEMMs (M in 1, 8, 32, 128 times the four weight
+    shapes) in NVFP4: pairwise 4:8 against dense, each as one grouped launch
+    (sp24_gemm_nvfp4_grouped), every GEMM with its own copy of its weights
+    (together larger than L2), X cast to NVFP4 beforehand; CUDA-graph replays
+    of the launch, weights marked static."""
+    import torch
+
+    from semi_structured_sparse_02_b200 import inputs, sp24
+    gemms = [(M, N, K) for M in inputs.DECODE_M for (N, K) in inputs.DECODE_NK]
+    stream = torch.cuda.Stream(device=dev)
+    times, wins, byts, keep = {}, {}, {}, []
+    F = sum(2.0 * M * N * K for M, N, K in gemms)
+    Wb = {(N, K): inputs.normal_bf16((N, K), 0.02, seed=N + K) for (N, K) in inputs.DECODE_NK}
+    for sparse in (True, False):
+        blk = 32 if sparse else 16
+        base = {}
+        for (N, K) in inputs.DECODE_NK:
+            W = _bf16_dev(Wb[(N, K)], dev)
+            wts = torch.empty(1, dtype=torch.float32, device=dev)
+            wsc = torch.empty(sp24.nvfp4_scales_bytes(N, K, blk), dtype=torch.uint8, device=dev)
+            if sparse:
+                wv = torch.empty(N, K // 4, dtype=torch.uint8, device=dev)
+                meta = torch.empty(sp24.nvfp4_48_meta_bytes(N, K), dtype=torch.uint8, device=dev)
+                sp24.prune_compress_nvfp4_48(W, wv, meta, wsc, wts)
+            else:
+                wv = torch.empty(N, K // 2, dtype=torch.uint8, device=dev)
+                meta = None
+                sp24.quantize_nvfp4(W, 16, wv, wsc, wts)
+            base[(N, K)] = (wv, meta, wsc, wts)
+            del W
+        al, b = [], 0
+        for i, (M, N, K) in enumerate(gemms):
+            wv, meta, wsc, wts = base[(N, K)]
+            wv, wsc = wv.clone(), wsc.clone()  # a distinct weight copy per GEMM
+            meta = meta.clone() if meta is not None else None
+            X = _bf16_dev(inputs.normal_bf16((M, K), 1.0, seed=2000 + i), dev)
+            xc = torch.empty(M, K // 2, dtype=torch.uint8, device=dev)
+            xs = torch.empty(sp24.nvfp4_scales_bytes(M, K, blk), dtype=torch.uint8, device=dev)
+            xts = torch.empty(1, dtype=torch.float32, device=dev)
+            sp24.quantize_nvfp4(X, blk, xc, xs, xts)
+            Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+            al.append(sp24.nvfp4_gemm_args(xc, xs, xts, wv, wsc, wts, Y, K, sp24.SPARSE if sparse else sp24.DENSE,
+                                           W_meta=meta, flags=sp24.GEMM_W_STATIC))
+            b += (N * K * (0.25 + 1 / 16 + 1 / 32) if sparse else N * K * (0.5 + 1 / 16)) + \
+                M * K * (0.5 + 1 / blk) + 2 * M * N
+        del base
+        grp = sp24.Nvfp4GemmGroup(al)
+        with torch.cuda.stream(stream):
+            grp(stream=stream)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            grp(stream=stream)
+        g._keep = (grp, al)
+        times[sparse], wins[sparse] = T.graph([g], stream)
+        byts[sparse] = b
+        keep.append(g)
+    del Wb
+    t_sp, t_dn = times[True], times[False]
+    row = dict(gemm="nvfp4_step", gemms=len(gemms), dtype="nvfp4", us_sparse=round(t_sp, 2), us_dense=round(t_dn, 2),
+               gbs_sparse=round(byts[True] / t_sp / 1e3, 1), gbs_dense=round(byts[False] / t_dn / 1e3, 1),
+               weight_mb_sparse=round(byts[True] / 1e6, 1), weight_mb_dense=round(byts[False] / 1e6, 1),
+               speedup_vs_dense=round(t_dn / t_sp, 3), selected="sparse" if t_sp < t_dn else "dense",
+               roofline_sparse=_roofline(F, byts[True], t_sp, 8 * T.bf16_tf, T.hbm),
+               roofline_dense=_roofline(F, byts[False], t_dn, 4 * T.bf16_tf, T.hbm),
+               _win=_win(wins[True], wins[False]),
+               note="one grouped launch of the 16 decode GEMMs per tactic, CUDA-graph replays, distinct weight "
+                    "copies per GEMM (larger than L2 together); X cast outside the timed launch")
+    print(json.dumps({k: v for k, v in row.items() if not k.startswith("_")}), file=sys.stderr, flush=True)
+    del keep
+    torch.cuda.empty_cache()
+    return [row]
+
+
 NVFP4_SHAPES = [(8, N, K) for N, K in [(5120, 5120), (25600, 5120), (5120, 25600), (10240, 5120)]] + \
     [(128, 5120, 25600), (8192, 4096, 4096), (8192, 12288, 4096)]
 
@@ -1439,7 +1514,7 @@ def run_config(args):
     elif args.config == "prune":
         rows = cfg_prune(dev, T)
     elif args.config == "nvfp4":
-        rows = cfg_nvfp4(dev, T, NVFP4_SHAPES)
+        rows = cfg_nvfp4_step(dev, T) + cfg_nvfp4(dev, T, NVFP4_SHAPES)
     time.sleep(0.2)
     sampler.stop()
     out["rows"] = _finish_rows(rows, sampler)
@@ -1475,10 +1550,10 @@ def run_configs_compact(dev):
     torch.cuda.empty_cache()
     out["tiny"] = cfg_tiny(dev, T)
     torch.cuda.empty_cache()
-    out["nvfp4"] = cfg_nvfp4(dev, T, [(8, 25600, 5120), (128, 5120, 25600), (8192, 4096, 4096)])
+    out["nvfp4"] = cfg_nvfp4_step(dev, T) + cfg_nvfp4(dev, T, [(8, 25600, 5120), (128, 5120, 25600), (8192, 4096, 4096)])
     time.sleep(0.2)
     sampler.stop()
-    keep = ("gemm", "block_step", "M", "N", "K", "dtype", "us_sparse", "us_dense", "us_fused", "us_hybrid",
+    keep = ("gemm", "gemms", "block_step", "M", "N", "K", "dtype", "us_sparse", "us_dense", "us_fused", "us_hybrid",
             "tflops_sparse", "tflops_fused", "speedup_vs_dense", "selected", "reason", "clocks")
     for name, rows in out.items():
         _finish_rows(rows, sampler)

@@ -475,6 +475,21 @@ size_t sp24_gemm_nvfp4_workspace_bytes(const sp24_nvfp4_gemm_args *args);
  * 16-byte aligned, ldy * out bytes % 16 == 0. */
 int sp24_gemm_nvfp4(const sp24_nvfp4_gemm_args *args, void *stream);
 
+/* Up to 16 independent NVFP4 GEMMs in one launch (the decode regime, where
+ * one launch per GEMM pays its ramp and tail every time): all problems share
+ * the tactic (all 4:8 SPARSE or all DENSE) and the output type; each may have
+ * its own M, N, K and buffers, and runs its own token-tile width inside the
+ * widest problem's tile, with stream-K across problem boundaries as
+ * sp24_gemm_grouped does.  Each args' own workspace fields are ignored: the
+ * group uses `workspace` (size from sp24_gemm_nvfp4_grouped_workspace_bytes,
+ * the zero-fill rule of sp24_gemm_workspace_bytes).  SP24_GEMM_W_STATIC and
+ * SP24_GEMM_AFTER_INDEPENDENT apply when every problem sets them.  Errors:
+ * SP24_ERR_INVALID_ARG for n outside 1..16 or mixed tactics,
+ * SP24_ERR_DTYPE for mixed output types, and each problem's own checks. */
+int sp24_gemm_nvfp4_grouped(const sp24_nvfp4_gemm_args *args, int n, void *workspace_dev, size_t workspace_bytes,
+                            void *stream);
+size_t sp24_gemm_nvfp4_grouped_workspace_bytes(const sp24_nvfp4_gemm_args *args, int n);
+
 /* ---------------------------------------------------------------------- */
 /* Tactic selection (kernel 5)                                             */
 /* ---------------------------------------------------------------------- */

@@ -473,6 +473,8 @@ int dispatch_gemm_group(const Plan& pl, const GemmLaunch<kMaxGroup>& gl, cudaStr
                    : launch_gemm_bn<kModeDense, false, true, kMaxGroup>(pl.bn, gl, pl.grid, s);
   if (pl.mode == kModeHybrid && !pl.bf16)
     return launch_gemm_bn<kModeHybrid, false, true, kMaxGroup>(pl.bn, gl, pl.grid, s);
+  if (pl.mode == kModeNvSparse) return launch_gemm_bn<kModeNvSparse, false, true, kMaxGroup>(pl.bn, gl, pl.grid, s);
+  if (pl.mode == kModeNvDense) return launch_gemm_bn<kModeNvDense, false, true, kMaxGroup>(pl.bn, gl, pl.grid, s);
   return SP24_ERR_DTYPE;
 }
 
@@ -1077,62 +1079,97 @@ int validate_nvfp4(const sp24_nvfp4_gemm_args* a) {
   return SP24_OK;
 }
 
-// Token tiles (pick_bn) of fewer than 128 rows only occur when the tokens fit
-// one tile, so every tile's B scales start a 128-row chunk of the scale image.
-Plan plan_nvfp4(const sp24_nvfp4_gemm_args* a, const DeviceInfo& di, size_t ws_cap) {
+// Checks that n NVFP4 GEMMs can share one launch: one tactic (4:8 sparse or
+// dense) and one output type.
+int validate_nvfp4_group(const sp24_nvfp4_gemm_args* a, int n) {
+  if (a == nullptr) return SP24_ERR_NULL;
+  if (n < 1 || n > kMaxGroup) return SP24_ERR_INVALID_ARG;
+  for (int i = 0; i < n; ++i) {
+    const int st = validate_nvfp4(&a[i]);
+    if (st != SP24_OK) return st;
+    if (a[i].tactic != a[0].tactic) return SP24_ERR_INVALID_ARG;
+    if (a[i].out_dtype != a[0].out_dtype) return SP24_ERR_DTYPE;
+  }
+  return SP24_OK;
+}
+
+// Token tiles (pick_bn) of fewer than 128 rows only occur when a problem's
+// tokens fit one tile, so every tile's B scales start a 128-row chunk of the
+// scale image.  In a group the kernel takes the widest problem's tile and
+// every problem runs its own width.
+Plan plan_nvfp4(const sp24_nvfp4_gemm_args* const* a, int n, const DeviceInfo& di, size_t ws_cap) {
   Plan pl;
   memset(&pl, 0, sizeof pl);
-  pl.mode = a->tactic == SP24_TACTIC_SPARSE ? kModeNvSparse : kModeNvDense;
+  pl.mode = a[0]->tactic == SP24_TACTIC_SPARSE ? kModeNvSparse : kModeNvDense;
   pl.bf16 = false;
   pl.a_is_w = true;
-  pl.bn = pick_bn(a->M);
   pl.kt = stage_k(pl.mode, false);
-  pl.n = 1;
-  pl.num_kt[0] = (int)((a->K + pl.kt - 1) / pl.kt);
-  pl.tiles_a[0] = (int)((a->N + kBlockA - 1) / kBlockA);
-  pl.tiles_b[0] = (int)((a->M + pl.bn - 1) / pl.bn);
+  pl.n = n;
+  pl.bn = 16;
+  for (int i = 0; i < n; ++i) pl.bn = std::max(pl.bn, pick_bn(a[i]->M));
+  for (int i = 0; i < n; ++i) {
+    pl.bn_i[i] = pick_bn(a[i]->M);
+    pl.num_kt[i] = (int)((a[i]->K + pl.kt - 1) / pl.kt);
+    pl.tiles_a[i] = (int)((a[i]->N + kBlockA - 1) / kBlockA);
+    pl.tiles_b[i] = (int)((a[i]->M + pl.bn_i[i] - 1) / pl.bn_i[i]);
+  }
   choose_schedule(pl, di.sms, ws_cap);
   return pl;
 }
 
-int build_launch_nvfp4(GemmLaunch<1>& gl, const sp24_nvfp4_gemm_args* a, const Plan& pl) {
+template <int kMaxProb>
+int build_launch_nvfp4(GemmLaunch<kMaxProb>& gl, const sp24_nvfp4_gemm_args* const* a, int n, const Plan& pl,
+                       void* workspace) {
   memset(&gl, 0, sizeof gl);
   const bool sparse = pl.mode == kModeNvSparse;
-  const uint64_t a_bytes = (uint64_t)(sparse ? a->K / 4 : a->K / 2);  // bytes of a W row
-  bool ok = make_map(&gl.tm_a[0], a->W, 1, a_bytes, a->N, a_bytes, 128, kBlockA, CU_TENSOR_MAP_SWIZZLE_128B);
-  ok &= make_map(&gl.tm_b[0], a->X, 1, a->K / 2, a->M, a->K / 2, 128, pl.bn, CU_TENSOR_MAP_SWIZZLE_128B);
-  if (!ok) return SP24_ERR_CUDA;
-  gl.tm_a2[0] = gl.tm_a[0];
-  gl.tm_a3[0] = gl.tm_a[0];
   const bool sk = pl.sched == kSchedStreamK;
-  uint8_t* ws = static_cast<uint8_t*>(a->workspace);
-  GemmProblem& P = gl.prob[0];
-  P.rows_a = (int32_t)a->N;
-  P.rows_b = (int32_t)a->M;
-  P.K = (int32_t)a->K;
-  P.num_kt = pl.num_kt[0];
-  P.tiles_a = pl.tiles_a[0];
-  P.tiles_b = pl.tiles_b[0];
-  P.meta_blocks = (int32_t)((a->N + 127) / 128);
-  P.bn = pl.bn;
-  P.meta = static_cast<const uint8_t*>(a->W_meta);
-  P.sfa = static_cast<const uint8_t*>(a->w_scales);
-  P.sfb = static_cast<const uint8_t*>(a->x_scales);
-  P.scale_a = a->w_tensor_scale;
-  P.scale_b = a->x_tensor_scale;
-  P.Y = a->Y;
-  P.ldy = a->ldy;
+  int64_t iter = 0;
+  int tile = 0;
+  bool w_static = true, indep = true;
+  for (int i = 0; i < n; ++i) {
+    const uint64_t a_bytes = (uint64_t)(sparse ? a[i]->K / 4 : a[i]->K / 2);  // bytes of a W row
+    bool ok = make_map(&gl.tm_a[i], a[i]->W, 1, a_bytes, a[i]->N, a_bytes, 128, kBlockA, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok &= make_map(&gl.tm_b[i], a[i]->X, 1, a[i]->K / 2, a[i]->M, a[i]->K / 2, 128, (uint32_t)pl.bn_i[i],
+                   CU_TENSOR_MAP_SWIZZLE_128B);
+    if (!ok) return SP24_ERR_CUDA;
+    gl.tm_a2[i] = gl.tm_a[i];
+    gl.tm_a3[i] = gl.tm_a[i];
+    GemmProblem& P = gl.prob[i];
+    P.rows_a = (int32_t)a[i]->N;
+    P.rows_b = (int32_t)a[i]->M;
+    P.K = (int32_t)a[i]->K;
+    P.num_kt = pl.num_kt[i];
+    P.tiles_a = pl.tiles_a[i];
+    P.tiles_b = pl.tiles_b[i];
+    P.tile_begin = tile;
+    P.iter_begin = iter;
+    P.meta_blocks = (int32_t)((a[i]->N + 127) / 128);
+    P.bn = pl.bn_i[i];
+    P.meta = static_cast<const uint8_t*>(a[i]->W_meta);
+    P.sfa = static_cast<const uint8_t*>(a[i]->w_scales);
+    P.sfb = static_cast<const uint8_t*>(a[i]->x_scales);
+    P.scale_a = a[i]->w_tensor_scale;
+    P.scale_b = a[i]->x_tensor_scale;
+    P.Y = a[i]->Y;
+    P.ldy = a[i]->ldy;
+    const int tiles = pl.tiles_a[i] * pl.tiles_b[i];
+    iter += (int64_t)tiles * pl.num_kt[i];
+    tile += tiles;
+    w_static = w_static && (a[i]->flags & SP24_GEMM_W_STATIC) != 0;
+    indep = indep && (a[i]->flags & SP24_GEMM_AFTER_INDEPENDENT) != 0;
+  }
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
   gl.p.sk_flags = sk ? reinterpret_cast<unsigned int*>(ws) : nullptr;
   gl.p.sk_slots = sk ? reinterpret_cast<float*>(ws + sk_state_bytes(pl)) : nullptr;
-  gl.p.n_prob = 1;
+  gl.p.n_prob = n;
   gl.p.sched = pl.sched;
   gl.p.total_iters = pl.total_iters;
   set_sk_bounds(gl.p, pl, nullptr, nullptr);
   gl.p.total_tiles = pl.total_tiles;
-  gl.p.out_f32 = a->out_dtype == SP24_F32;
+  gl.p.out_f32 = a[0]->out_dtype == SP24_F32;
   gl.p.use_pdl = 1;
-  gl.p.w_static = (a->flags & SP24_GEMM_W_STATIC) != 0;
-  gl.p.after_independent = (a->flags & SP24_GEMM_AFTER_INDEPENDENT) != 0;
+  gl.p.w_static = w_static ? 1 : 0;
+  gl.p.after_independent = indep ? 1 : 0;
   gl.p.timeout_ns = g_timeout_ns.load();
   return SP24_OK;
 }
@@ -1572,7 +1609,7 @@ size_t sp24_gemm_nvfp4_workspace_bytes(const sp24_nvfp4_gemm_args* a) {
   if (validate_nvfp4(a) != SP24_OK) return 0;
   DeviceInfo di;
   if (current_device_info(&di) != SP24_OK) return 0;
-  return plan_nvfp4(a, di, (size_t)-1).ws_bytes;
+  return plan_nvfp4(&a, 1, di, (size_t)-1).ws_bytes;
 }
 
 int sp24_gemm_nvfp4(const sp24_nvfp4_gemm_args* a, void* stream) {
@@ -1582,9 +1619,33 @@ int sp24_gemm_nvfp4(const sp24_nvfp4_gemm_args* a, void* stream) {
   DeviceInfo di;
   if ((st = current_device_info(&di)) != SP24_OK) return st;
   static thread_local SingleLaunch v;
-  v.pl = plan_nvfp4(a, di, a->workspace != nullptr ? a->workspace_bytes : 0);
-  if ((st = build_launch_nvfp4(v.gl, a, v.pl)) != SP24_OK) return st;
+  v.pl = plan_nvfp4(&a, 1, di, a->workspace != nullptr ? a->workspace_bytes : 0);
+  if ((st = build_launch_nvfp4(v.gl, &a, 1, v.pl, a->workspace)) != SP24_OK) return st;
   return dispatch_gemm(v.pl, v.gl, static_cast<cudaStream_t>(stream));
+}
+
+size_t sp24_gemm_nvfp4_grouped_workspace_bytes(const sp24_nvfp4_gemm_args* args, int n) {
+  if (validate_nvfp4_group(args, n) != SP24_OK) return 0;
+  DeviceInfo di;
+  if (current_device_info(&di) != SP24_OK) return 0;
+  const sp24_nvfp4_gemm_args* ptrs[kMaxGroup];
+  for (int i = 0; i < n; ++i) ptrs[i] = &args[i];
+  return plan_nvfp4(ptrs, n, di, (size_t)-1).ws_bytes;
+}
+
+int sp24_gemm_nvfp4_grouped(const sp24_nvfp4_gemm_args* args, int n, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+  int st = validate_nvfp4_group(args, n);
+  if (st != SP24_OK) return st;
+  if (workspace != nullptr && !aligned16(workspace)) return SP24_ERR_ALIGNMENT;
+  DeviceInfo di;
+  if ((st = current_device_info(&di)) != SP24_OK) return st;
+  const sp24_nvfp4_gemm_args* ptrs[kMaxGroup];
+  for (int i = 0; i < n; ++i) ptrs[i] = &args[i];
+  static thread_local GroupLaunch v;  // large: keep it off the stack
+  v.pl = plan_nvfp4(ptrs, n, di, workspace != nullptr ? workspace_bytes : 0);
+  if ((st = build_launch_nvfp4(v.gl, ptrs, n, v.pl, workspace)) != SP24_OK) return st;
+  return dispatch_gemm_group(v.pl, v.gl, static_cast<cudaStream_t>(stream));
 }
 
 size_t sp24_activations_workspace_bytes(int64_t M, int64_t K) {

@@ -135,6 +135,8 @@ def lib() -> ctypes.CDLL:
         "sp24_quantize_nvfp4": (I, [P, I64, I64, I64, I, P, P, P, P]),
         "sp24_gemm_nvfp4_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(Nvfp4GemmArgs)]),
         "sp24_gemm_nvfp4": (I, [ctypes.POINTER(Nvfp4GemmArgs), P]),
+        "sp24_gemm_nvfp4_grouped": (I, [ctypes.POINTER(Nvfp4GemmArgs), I, P, ctypes.c_size_t, P]),
+        "sp24_gemm_nvfp4_grouped_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(Nvfp4GemmArgs), I]),
         "sp24_prune_activations_in_gemm": (I, [P, I64, I64, I64, P, I64, I64, P, I64, I, P, P, P]),
         "sp24_status_string": (ctypes.c_char_p, [I]),
         "sp24_last_device_error": (I, []),
@@ -502,6 +504,30 @@ def gemm_nvfp4_workspace_bytes(args: Nvfp4GemmArgs) -> int:
 
 def gemm_nvfp4(args: Nvfp4GemmArgs, stream=None):
     _check(lib().sp24_gemm_nvfp4(ctypes.byref(args), _stream(stream)), "sp24_gemm_nvfp4")
+
+
+class Nvfp4GemmGroup:
+    """Up to 16 independent NVFP4 GEMMs (one tactic, one output type) run by
+    one sp24_gemm_nvfp4_grouped launch; `workspace` (zero-filled, reusable
+    across calls on one stream) is allocated here when the schedule needs
+    one.  The argument objects are held for the group's lifetime."""
+
+    def __init__(self, args_list, workspace: Optional[torch.Tensor] = None):
+        self.args_list = list(args_list)
+        self.n = len(self.args_list)
+        self.arr = (Nvfp4GemmArgs * self.n)(*self.args_list)
+        need = lib().sp24_gemm_nvfp4_grouped_workspace_bytes(self.arr, self.n)
+        if workspace is None and need > 0:
+            workspace = torch.zeros(need, dtype=torch.uint8, device=torch.cuda.current_device())
+        self.workspace = workspace
+        self.ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+
+    def workspace_bytes(self) -> int:
+        return lib().sp24_gemm_nvfp4_grouped_workspace_bytes(self.arr, self.n)
+
+    def __call__(self, stream=None):
+        _check(lib().sp24_gemm_nvfp4_grouped(self.arr, self.n, _ptr(self.workspace), self.ws_bytes,
+                                             _stream(stream)), "sp24_gemm_nvfp4_grouped")
 
 
 # ---------------------------------------------------------------------------

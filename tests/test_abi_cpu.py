@@ -226,7 +226,7 @@ def test_nvfp4_sizes():
     assert sparse * 8 == rows * K * 2.75 and dense * 8 == rows * K * 4.5
 
 
-def nvgemm(**kw):
+def nvargs(**kw):
     a = sp24.Nvfp4GemmArgs()
     a.M, a.N, a.K = kw.get("M", 16), kw.get("N", 256), kw.get("K", 512)
     a.tactic = kw.get("tactic", sp24.SPARSE)
@@ -234,7 +234,27 @@ def nvgemm(**kw):
     for f in ("X", "x_scales", "x_tensor_scale", "W", "W_meta", "w_scales", "w_tensor_scale", "Y"):
         setattr(a, f, kw.get(f, FAKE))
     a.ldy = kw.get("ldy", a.N)
-    return L.sp24_gemm_nvfp4(ctypes.byref(a), None)
+    return a
+
+
+def nvgemm(**kw):
+    return L.sp24_gemm_nvfp4(ctypes.byref(nvargs(**kw)), None)
+
+
+def test_nvfp4_grouped_validation():
+    G = L.sp24_gemm_nvfp4_grouped
+    arr = lambda *xs: (sp24.Nvfp4GemmArgs * len(xs))(*xs)
+    assert G(None, 1, None, 0, None) == sp24.SP24_ERR_NULL
+    one = arr(nvargs())
+    assert G(one, 0, None, 0, None) == sp24.SP24_ERR_INVALID_ARG
+    assert G(arr(*[nvargs() for _ in range(17)]), 17, None, 0, None) == sp24.SP24_ERR_INVALID_ARG
+    assert G(arr(nvargs(), nvargs(tactic=sp24.DENSE)), 2, None, 0, None) == sp24.SP24_ERR_INVALID_ARG
+    assert G(arr(nvargs(), nvargs(out_dtype=sp24.F32)), 2, None, 0, None) == sp24.SP24_ERR_DTYPE
+    assert G(arr(nvargs(), nvargs(K=384)), 2, None, 0, None) == sp24.SP24_ERR_NOT_2_4  # each problem's own checks
+    assert G(one, 1, FAKE + 4, 1024, None) == sp24.SP24_ERR_ALIGNMENT
+    assert L.sp24_gemm_nvfp4_grouped_workspace_bytes(arr(nvargs(), nvargs(tactic=sp24.DENSE)), 2) == 0
+    if NO_GPU:
+        assert G(arr(nvargs(M=1), nvargs(M=128, N=512, K=1024)), 2, None, 0, None) == sp24.SP24_ERR_UNSUPPORTED_DEVICE
 
 
 def test_nvfp4_validation():

@@ -127,6 +127,38 @@ def test_gemm_nvfp4_parity(M, N, K, tactic):
                         "nvfp4 M%d N%d K%d tactic %d f32=%s" % (M, N, K, tactic, out_f32))
 
 
+# NVFP4 groups: token-count classes, shapes and stage counts mixed in one launch
+NV_GROUPS = {
+    "decode": [(1, 256, 512), (8, 1024, 5120), (16, 512, 1024), (40, 384, 768)],
+    "to128": [(1, 512, 1024), (128, 256, 2048), (33, 384, 512), (200, 256, 1024), (8, 768, 2560)],
+}
+
+
+@pytest.mark.parametrize("group", sorted(NV_GROUPS))
+@pytest.mark.parametrize("tactic", [sp24.SPARSE, sp24.DENSE])
+def test_gemm_nvfp4_grouped_parity(group, tactic):
+    """One sp24_gemm_nvfp4_grouped launch over problems of different M, N and
+    K (each with its own token-tile width; one output type per group, as the
+    call requires), with the group's workspace and without one (whole tiles),
+    twice each; every output against the oracle."""
+    out_f32 = group == "decode"  # one output type per group: fp32 here, bf16 for the other
+    cases = [_gemm_case(M, N, K, tactic, out_f32=out_f32, seed=17 * i, use_ws=False)
+             for i, (M, N, K) in enumerate(NV_GROUPS[group])]
+    for use_ws in (True, False):
+        grp = sp24.Nvfp4GemmGroup([c[0] for c in cases])  # allocates the workspace the schedule needs
+        if not use_ws:
+            grp.workspace, grp.ws_bytes = None, 0  # whole tiles per CTA
+        for _ in range(2):
+            for (_, Y, _, _) in cases:
+                Y.fill_(float("nan"))
+            grp()
+            torch.cuda.synchronize()
+            assert sp24.last_device_error() == sp24.SP24_OK
+            for i, (_, Y, y_ref, a_ref) in enumerate(cases):
+                check_tolerance(Y.float().cpu().numpy().astype(np.float64), y_ref, a_ref,
+                                "nvfp4 group %s problem %d tactic %d ws=%s" % (group, i, tactic, use_ws))
+
+
 @pytest.mark.parametrize("tactic", [sp24.SPARSE, sp24.DENSE])
 def test_gemm_nvfp4_whole_tiles_and_static_weights(tactic):
     # without a workspace the stream-K shape runs whole tiles; with
