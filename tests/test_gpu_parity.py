@@ -511,6 +511,38 @@ def test_grouped_hybrid_gemm_parity(group, use_ws, kind):
         check_group(items, "hybrid group %s ws=%s %s call %d" % (group, use_ws, kind, call))
 
 
+def test_grouped_hybrid_first_call_inside_stream_capture():
+    """A hybrid group whose first call is made while its stream is being
+    captured into a CUDA graph: the planner skips reading the tile masks back
+    (the schedule is then cut by stage counts alone) and the replayed graph
+    still gives the oracle's results; later eager calls reuse that plan."""
+    shapes = [(1, 768, 1024), (16, 512, 2048), (8, 1536, 512)]
+    items = []
+    for i, (M, N, K) in enumerate(shapes):
+        X, W = inputs.linear_pair(M, N, K, seed=41 * i + M + K, outliers=True)
+        items.append(prepare_gemm(X, W, True, sp24.SPARSE, True, mask=inputs.hybrid_mask(N, K, seed=3 + i),
+                                  flags=sp24.GEMM_W_STATIC))
+    grp = sp24.GemmGroup([it[0] for it in items])  # workspace allocated before the capture
+    assert grp.ws_bytes > 0  # the stream-K schedule, whose cut reads the masks when it can
+    stream = torch.cuda.Stream()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        grp(stream=stream)
+    for _ in range(2):
+        for it in items:
+            it[1].fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        assert sp24.last_device_error() == sp24.SP24_OK
+        check_group(items, "hybrid group, first call captured")
+    for it in items:
+        it[1].fill_(float("nan"))
+    grp()
+    torch.cuda.synchronize()
+    check_group(items, "hybrid group, eager call after the capture")
+
+
 def test_grouped_hybrid_mixed_token_classes():
     shapes = [(1, 768, 512), (16, 512, 1024), (32, 256, 5120), (100, 384, 640)]
     items = []
