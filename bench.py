@@ -708,8 +708,9 @@ def run_other_case(args):
     act:M,N,K,bf16|e4m3|ingemm -- the online-activation path (prune of X every
     call, then the sparse GEMM; ingemm: the prune inside the GEMM kernel);
     nv:M,N,K,sparse|dense -- the NVFP4 GEMM (pairwise
-    4:8 or dense), X cast to NVFP4 once.  Eager calls, CUDA-event timing, L2
-    flushed before each call (for profiler captures)."""
+    4:8 or dense), X cast to NVFP4 once; nvstep:sparse|dense -- the NVFP4
+    decode step's 16 GEMMs as one grouped launch.  Eager calls, CUDA-event
+    timing, L2 flushed before each call (for profiler captures)."""
     import torch
 
     from semi_structured_sparse_02_b200 import inputs, sp24
@@ -745,6 +746,11 @@ def run_other_case(args):
         t, _, _ = T.calls(fn)
         print(json.dumps({"case": args.case, "us_median": round(t, 3),
                           "TFLOPS": round(2.0 * M * N * K / t / 1e6, 1)}), flush=True)
+    elif kind == "nvstep":
+        grp, byts = nvfp4_step_group(dev, (f[0] if f else "sparse") == "sparse")
+        t, _, _ = T.calls(lambda: grp())
+        print(json.dumps({"case": args.case, "us_median": round(t, 3), "GBps": round(byts / t / 1e3, 1),
+                          "bytes": int(byts), "workspace_bytes": grp.ws_bytes}), flush=True)
     elif kind == "nv":
         M, N, K = int(f[0]), int(f[1]), int(f[2])
         sparse = (f[3] if len(f) > 3 else "sparse") == "sparse"
@@ -789,7 +795,7 @@ def run_case(args):
     if args.case.startswith("group:"):
         run_group_case(args)
         return
-    if args.case.split(":", 1)[0] in ("prune", "act", "nv"):
+    if args.case.split(":", 1)[0] in ("prune", "act", "nv", "nvstep"):
         run_other_case(args)
         return
     f = args.case.split(",")
@@ -1362,64 +1368,75 @@ def cfg_nvfp4(dev, T, shapes):
     return rows
 
 
-def cfg_nvfp4_step(dev, T):
+def nvfp4_step_group(dev, sparse, Wb=None):
     """The decode step's 16 GEMMs (M in 1, 8, 32, 128 times the four weight
-    shapes) in NVFP4: pairwise 4:8 against dense, each as one grouped launch
-    (sp24_gemm_nvfp4_grouped), every GEMM with its own copy of its weights
-    (together larger than L2), X cast to NVFP4 beforehand; CUDA-graph replays
-    of the launch, weights marked static."""
+    shapes) in NVFP4 as one sp24_gemm_nvfp4_grouped launch: pairwise 4:8 or
+    dense, every GEMM with its own copy of its weights (together larger than
+    L2), X cast to NVFP4 beforehand, weights marked static.  Returns the group
+    and the step's algorithmic bytes."""
     import torch
 
     from semi_structured_sparse_02_b200 import inputs, sp24
     gemms = [(M, N, K) for M in inputs.DECODE_M for (N, K) in inputs.DECODE_NK]
+    if Wb is None:
+        Wb = {(N, K): inputs.normal_bf16((N, K), 0.02, seed=N + K) for (N, K) in inputs.DECODE_NK}
+    blk = 32 if sparse else 16
+    base = {}
+    for (N, K) in inputs.DECODE_NK:
+        W = _bf16_dev(Wb[(N, K)], dev)
+        wts = torch.empty(1, dtype=torch.float32, device=dev)
+        wsc = torch.empty(sp24.nvfp4_scales_bytes(N, K, blk), dtype=torch.uint8, device=dev)
+        if sparse:
+            wv = torch.empty(N, K // 4, dtype=torch.uint8, device=dev)
+            meta = torch.empty(sp24.nvfp4_48_meta_bytes(N, K), dtype=torch.uint8, device=dev)
+            sp24.prune_compress_nvfp4_48(W, wv, meta, wsc, wts)
+        else:
+            wv = torch.empty(N, K // 2, dtype=torch.uint8, device=dev)
+            meta = None
+            sp24.quantize_nvfp4(W, 16, wv, wsc, wts)
+        base[(N, K)] = (wv, meta, wsc, wts)
+        del W
+    al, b = [], 0
+    for i, (M, N, K) in enumerate(gemms):
+        wv, meta, wsc, wts = base[(N, K)]
+        wv, wsc = wv.clone(), wsc.clone()  # a distinct weight copy per GEMM
+        meta = meta.clone() if meta is not None else None
+        X = _bf16_dev(inputs.normal_bf16((M, K), 1.0, seed=2000 + i), dev)
+        xc = torch.empty(M, K // 2, dtype=torch.uint8, device=dev)
+        xs = torch.empty(sp24.nvfp4_scales_bytes(M, K, blk), dtype=torch.uint8, device=dev)
+        xts = torch.empty(1, dtype=torch.float32, device=dev)
+        sp24.quantize_nvfp4(X, blk, xc, xs, xts)
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        al.append(sp24.nvfp4_gemm_args(xc, xs, xts, wv, wsc, wts, Y, K, sp24.SPARSE if sparse else sp24.DENSE,
+                                       W_meta=meta, flags=sp24.GEMM_W_STATIC))
+        b += (N * K * (0.25 + 1 / 16 + 1 / 32) if sparse else N * K * (0.5 + 1 / 16)) + \
+            M * K * (0.5 + 1 / blk) + 2 * M * N
+    return sp24.Nvfp4GemmGroup(al), b
+
+
+def cfg_nvfp4_step(dev, T):
+    """The NVFP4 decode step (nvfp4_step_group), pairwise 4:8 against dense,
+    timed as CUDA-graph replays of the one launch."""
+    import torch
+
+    from semi_structured_sparse_02_b200 import inputs
+    gemms = [(M, N, K) for M in inputs.DECODE_M for (N, K) in inputs.DECODE_NK]
     stream = torch.cuda.Stream(device=dev)
-    times, wins, byts, keep = {}, {}, {}, []
+    times, wins, byts = {}, {}, {}
     F = sum(2.0 * M * N * K for M, N, K in gemms)
     Wb = {(N, K): inputs.normal_bf16((N, K), 0.02, seed=N + K) for (N, K) in inputs.DECODE_NK}
     for sparse in (True, False):
-        blk = 32 if sparse else 16
-        base = {}
-        for (N, K) in inputs.DECODE_NK:
-            W = _bf16_dev(Wb[(N, K)], dev)
-            wts = torch.empty(1, dtype=torch.float32, device=dev)
-            wsc = torch.empty(sp24.nvfp4_scales_bytes(N, K, blk), dtype=torch.uint8, device=dev)
-            if sparse:
-                wv = torch.empty(N, K // 4, dtype=torch.uint8, device=dev)
-                meta = torch.empty(sp24.nvfp4_48_meta_bytes(N, K), dtype=torch.uint8, device=dev)
-                sp24.prune_compress_nvfp4_48(W, wv, meta, wsc, wts)
-            else:
-                wv = torch.empty(N, K // 2, dtype=torch.uint8, device=dev)
-                meta = None
-                sp24.quantize_nvfp4(W, 16, wv, wsc, wts)
-            base[(N, K)] = (wv, meta, wsc, wts)
-            del W
-        al, b = [], 0
-        for i, (M, N, K) in enumerate(gemms):
-            wv, meta, wsc, wts = base[(N, K)]
-            wv, wsc = wv.clone(), wsc.clone()  # a distinct weight copy per GEMM
-            meta = meta.clone() if meta is not None else None
-            X = _bf16_dev(inputs.normal_bf16((M, K), 1.0, seed=2000 + i), dev)
-            xc = torch.empty(M, K // 2, dtype=torch.uint8, device=dev)
-            xs = torch.empty(sp24.nvfp4_scales_bytes(M, K, blk), dtype=torch.uint8, device=dev)
-            xts = torch.empty(1, dtype=torch.float32, device=dev)
-            sp24.quantize_nvfp4(X, blk, xc, xs, xts)
-            Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
-            al.append(sp24.nvfp4_gemm_args(xc, xs, xts, wv, wsc, wts, Y, K, sp24.SPARSE if sparse else sp24.DENSE,
-                                           W_meta=meta, flags=sp24.GEMM_W_STATIC))
-            b += (N * K * (0.25 + 1 / 16 + 1 / 32) if sparse else N * K * (0.5 + 1 / 16)) + \
-                M * K * (0.5 + 1 / blk) + 2 * M * N
-        del base
-        grp = sp24.Nvfp4GemmGroup(al)
+        grp, byts[sparse] = nvfp4_step_group(dev, sparse, Wb)
         with torch.cuda.stream(stream):
             grp(stream=stream)
         torch.cuda.synchronize()
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
             grp(stream=stream)
-        g._keep = (grp, al)
+        g._keep = grp
         times[sparse], wins[sparse] = T.graph([g], stream)
-        byts[sparse] = b
-        keep.append(g)
+        del g, grp
+        torch.cuda.empty_cache()
     del Wb
     t_sp, t_dn = times[True], times[False]
     row = dict(gemm="nvfp4_step", gemms=len(gemms), dtype="nvfp4", us_sparse=round(t_sp, 2), us_dense=round(t_dn, 2),
@@ -1432,8 +1449,6 @@ def cfg_nvfp4_step(dev, T):
                note="one grouped launch of the 16 decode GEMMs per tactic, CUDA-graph replays, distinct weight "
                     "copies per GEMM (larger than L2 together); X cast outside the timed launch")
     print(json.dumps({k: v for k, v in row.items() if not k.startswith("_")}), file=sys.stderr, flush=True)
-    del keep
-    torch.cuda.empty_cache()
     return [row]
 
 
