@@ -103,8 +103,10 @@ size_t sp24_meta_bytes(int64_t rows, int64_t K);
 /* ---------------------------------------------------------------------- */
 
 /* Magnitude 2:4 prune of src along K and compression, in one pass over src
- * for BF16 output (three stream-ordered launches for E4M3: row amax, prune,
- * scale finalize).
+ * for BF16 output, and for E4M3 output without a tile mask on rows up to
+ * 28672 wide (the row held in registers: amax, prune, cast and scale in one
+ * launch); E4M3 with a tile mask or longer rows takes three stream-ordered
+ * launches (row amax, prune, scale finalize).  Same results either way.
  *   src_dev     bf16 [rows x K], row pitch ld elements.
  *   out_dtype   SP24_BF16: values are the kept bf16 values.
  *               SP24_E4M3: kept values quantized per row: scale = amax/448,

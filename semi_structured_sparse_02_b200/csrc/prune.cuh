@@ -494,73 +494,176 @@ k_quantize_rows_e4m3_seg(const __grid_constant__ QuantSegGroup g) {
 }
 
 // ---------------------------------------------------------------------------
-// Online activations at the FP8 floor in one pass: per-token amax, 2:4 prune
-// on the bf16 magnitudes, E4M3 cast of the kept values with the row scale,
-// the metadata image and the scale, from one HBM read of X.  Rows are held in
-// registers as warp segments (the layout of k_quantize_rows_e4m3_seg: a row
-// takes w warps of kQWarpVecs 16-byte vectors per lane, a CTA floor(16 / w)
-// rows), the row amax is combined across its warps in shared memory.  Each
-// 16-byte vector is two groups: one metadata byte (image row = the row for
-// 8-bit values, byte idx % 16 of chunk idx / 16) and four E4M3 codes.  Same
-// results as k_row_amax + k_prune_compress<true> + k_finalize_scales.
+// Rows pruned and cast to E4M3 in one pass: per-row amax, 2:4 prune on the
+// bf16 magnitudes, E4M3 cast of the kept values with the row scale, the
+// metadata image and the scale, from one HBM read of the row.  Same results
+// as k_row_amax + k_prune_compress<true> + k_finalize_scales.
+//
+// A row is held in registers by w warps of V 16-byte vectors per lane (the
+// host picks V in 4..8 so that w * 32 * V is the row length where it can:
+// kExact then drops every bounds check).  A CTA takes rows_per_cta rows at a
+// time; the row amax is combined across its warps in shared memory.
+//
+// The selection runs before the amax: the largest key of each group is its
+// largest magnitude, so the row amax is the maximum of those keys (the pruned
+// row's amax equals the row's).  The two kept positions come from a 16-entry
+// table indexed by the tie-break codes of the top two keys, which holds the
+// byte-permute selector of the kept pair and the nibble; that takes the
+// ordering of the codes off the integer ALU pipe, this kernel's limit.
+//
+// Each 16-byte vector is two groups: one metadata byte (image row = the row
+// for 8-bit values, byte idx % 16 of chunk idx / 16) and four E4M3 codes.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kQWarps * 32, 2)
+constexpr int kPcMaxWarps = 16;  // warps per row at most (512-thread CTAs)
+
+// table entry for codes (ct, cs) of the top two keys (position i has code
+// 3 - i): byte-permute selector of x_i0 | x_i1 << 16 in bits 0..15, nibble
+// i0 | i1 << 2 in bits 16..19 (i0 < i1)
+__device__ __forceinline__ void pick_table_init(uint32_t* table) {
+  if (threadIdx.x < 16) {
+    const uint32_t ct = threadIdx.x >> 2, cs = threadIdx.x & 3u;
+    uint32_t e = 0;
+    if (ct != cs) {
+      const uint32_t i0 = 3u - max(ct, cs), i1 = 3u - min(ct, cs);
+      e = (0x1010u + 0x22u * i0 + 0x2200u * i1) | ((i0 | (i1 << 2)) << 16);
+    }
+    table[threadIdx.x] = e;
+  }
+}
+
+// prune_pick4w with the index arithmetic from the table: returns the entry,
+// the kept pair in kept and the top key (magnitude bits at 17..31) in top_key
+__device__ __forceinline__ uint32_t prune_pick4t(uint32_t lo, uint32_t hi, const uint32_t* table, uint32_t& kept,
+                                                 uint32_t& top_key) {
+  const uint32_t k0 = mad_u32(lo, 131072u, 3u);
+  const uint32_t k1 = (mad_u32(lo, 2u, 0u) & 0xFFFE0000u) | 2u;
+  const uint32_t k2 = mad_u32(hi, 131072u, 1u);
+  const uint32_t k3 = mad_u32(hi, 2u, 0u) & 0xFFFE0000u;
+  const uint32_t m01 = max(k0, k1), n01 = min(k0, k1), m23 = max(k2, k3), n23 = min(k2, k3);
+  const uint32_t top = max(m01, m23);
+  const uint32_t sec = max(min(m01, m23), max(n01, n23));
+  top_key = top;
+  // byte offset of entry (top & 3) * 4 + (sec & 3): bits 2..16 of a key are zero
+  const uint32_t off = mad_u32(top, 16u, mad_u32(sec, 4u, 0u)) & 60u;
+  const uint32_t e = *reinterpret_cast<const uint32_t*>(reinterpret_cast<const uint8_t*>(table) + off);
+  kept = __byte_perm(lo, hi, e);
+  return e;
+}
+
+// two products of one rounding each (mul.rn.f32x2): {lo * s, hi * s}
+__device__ __forceinline__ uint32_t e4m3x2_scaled(uint32_t lo_bits, uint32_t hi_bits, unsigned long long s2) {
+  unsigned long long a, d;
+  uint32_t plo, phi;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(a) : "r"(lo_bits), "r"(hi_bits));
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(s2));
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(plo), "=r"(phi) : "l"(d));
+  return e4m3x2_of(__uint_as_float(plo), __uint_as_float(phi));
+}
+
+// Persistent CTAs (two per SM for 256 threads, one for 512) step over batches
+// of rows_per_cta rows, gridDim.x batches apart; each thread holds two
+// register buffers and loads the next batch's vectors while it prunes, casts
+// and stores this one, so the row loads stay in flight across the CTA's
+// barriers.  The row amax of batch k goes to s_amax[k & 1] tagged k << 16 (at
+// most 65535 batches per CTA, which the host's grid size keeps): an atomic max
+// then replaces the value batch k - 2 left there, and the barrier of batch
+// k + 1 keeps batch k + 2 from writing before batch k has read it.
+template <int kThreads, int V, bool kExact>
+__global__ void __launch_bounds__(kThreads, kThreads == 256 ? 2 : 1)
 k_prune_cast_rows_e4m3(const uint16_t* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
                        int warps_per_row, int rows_per_cta, uint8_t* __restrict__ values,
                        uint8_t* __restrict__ meta, float* __restrict__ scales) {
-  __shared__ uint32_t s_amax[kQWarps];
+  __shared__ uint32_t s_amax[2][kPcMaxWarps];
+  __shared__ uint32_t s_table[16];
   pdl_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (threadIdx.x < kQWarps) s_amax[threadIdx.x] = 0u;
+  if (threadIdx.x < 2 * kPcMaxWarps) (&s_amax[0][0])[threadIdx.x] = 0u;
+  pick_table_init(s_table);
   const int w = warps_per_row, slot = warp / w, seg = warp - slot * w;
-  const int64_t row = (int64_t)blockIdx.x * rows_per_cta + slot;
   // rows from `rows` to the end of the last 128-row block only get their
   // metadata (the prune of zeros: positions 0 and 1)
   const int64_t rows_pad = (rows + kChunkRows - 1) / kChunkRows * kChunkRows;
-  const bool active = slot < rows_per_cta && row < rows_pad;
-  const bool live = active && row < rows;
   const int64_t nv = K / 8;
-  pdl_wait();  // the activations may be written by the upstream grid
-  uint4 reg[kQWarpVecs];
-  uint32_t m2 = 0;
-  const int64_t idx0 = (int64_t)seg * kQSegVecs + lane;  // vector j of this thread: idx0 + 32 j
-  const uint4* p = reinterpret_cast<const uint4*>(src + (live ? row : 0) * ld) + idx0;
+  const int64_t idx0 = (int64_t)seg * (32 * V) + lane;  // vector j of this thread: idx0 + 32 j
+  const int64_t stride = (int64_t)gridDim.x * rows_per_cta;
+  int64_t base = (int64_t)blockIdx.x * rows_per_cta;  // first row of this CTA's batch
+  __syncthreads();  // table and s_amax initialized
+  if (base >= rows_pad) return;
+  pdl_wait();  // the rows may be written by the upstream grid
+
+  auto load = [&](uint4 (&reg)[V], int64_t row) {
+    const uint4* p = reinterpret_cast<const uint4*>(src + (row < rows ? row : 0) * ld) + idx0;
+    if (kExact) {
+      if (row < rows) {
 #pragma unroll
-  for (int j = 0; j < kQWarpVecs; ++j) {
-    reg[j] = (live && idx0 + j * 32 < nv) ? __ldg(p + j * 32) : make_uint4(0, 0, 0, 0);
-    m2 = amax_lanes8(m2, reg[j]);
-  }
-  uint32_t m = amax_lanes_reduce(m2);
+        for (int j = 0; j < V; ++j) reg[j] = __ldg(p + j * 32);
+      } else {
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-  __syncthreads();  // s_amax initialized
-  if (active && lane == 0) atomicMax(&s_amax[slot], m);
-  __syncthreads();
-  if (!active) return;
-  const float amax = bf16_bits_to_float(s_amax[slot]);
-  const float inv = e4m3_inv_scale(amax);
-  if (live && seg == 0 && lane == 0) scales[row] = amax == 0.0f ? 1.0f : __fdiv_rn(amax, 448.0f);
-  const int64_t KC = K / kChunkK;
-  const int64_t rb = row / kChunkRows, L = row % kChunkRows;
-  // vector idx of the row: 4 value bytes at idx * 4, its metadata byte in
-  // chunk idx / 16 at L * 16 + idx % 16; idx0 % 16 == lane % 16 since the
-  // warp segment length is a multiple of 32, so vector j's byte is 2 chunks on
-  uint32_t* vrow = reinterpret_cast<uint32_t*>(values + row * (K / 2)) + idx0;
-  uint8_t* mrow = meta + (rb * KC + idx0 / 16) * kChunkBytes + L * 16 + (lane & 15);
+        for (int j = 0; j < V; ++j) reg[j] = make_uint4(0, 0, 0, 0);
+      }
+    } else {
 #pragma unroll
-  for (int j = 0; j < kQWarpVecs; ++j) {
-    if (idx0 + j * 32 < nv) {
-      const uint4 v = reg[j];
-      uint32_t w0, w1;
-      const uint32_t nib0 = prune_pick4w(v.x, v.y, w0);
-      const uint32_t nib1 = prune_pick4w(v.z, v.w, w1);
-      const uint32_t q0 = e4m3x2_of(__fmul_rn(__uint_as_float(mad_u32(w0, 65536u, 0u)), inv),
-                                    __fmul_rn(__uint_as_float(w0 & 0xFFFF0000u), inv));
-      const uint32_t q1 = e4m3x2_of(__fmul_rn(__uint_as_float(mad_u32(w1, 65536u, 0u)), inv),
-                                    __fmul_rn(__uint_as_float(w1 & 0xFFFF0000u), inv));
-      if (live) vrow[j * 32] = mad_u32(q1, 65536u, q0);
-      mrow[j * 2 * kChunkBytes] = (uint8_t)mad_u32(nib1, 16u, nib0);
+      for (int j = 0; j < V; ++j)
+        reg[j] = (row < rows && idx0 + j * 32 < nv) ? __ldg(p + j * 32) : make_uint4(0, 0, 0, 0);
     }
+  };
+
+  auto process = [&](const uint4 (&reg)[V], int par, uint32_t tag, int64_t row) {
+    uint32_t kept0[V], kept1[V], nib[V];
+    uint32_t m = 0;
+#pragma unroll
+    for (int j = 0; j < V; ++j) {
+      uint32_t t0, t1;
+      const uint32_t e0 = prune_pick4t(reg[j].x, reg[j].y, s_table, kept0[j], t0);
+      const uint32_t e1 = prune_pick4t(reg[j].z, reg[j].w, s_table, kept1[j], t1);
+      nib[j] = mad_u32(__umulhi(e1, 65536u), 16u, __umulhi(e0, 65536u));  // the metadata byte
+      m = max(m, max(t0, t1));
+    }
+    m = __umulhi(m, 32768u);  // magnitude bits: key >> 17
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    const bool active = row < rows_pad, live = row < rows;
+    if (active && lane == 0) atomicMax(&s_amax[par][slot], tag | m);
+    __syncthreads();
+    if (!active) return;
+    const float amax = bf16_bits_to_float(s_amax[par][slot] & 0xFFFFu);
+    const float inv = e4m3_inv_scale(amax);
+    if (live && seg == 0 && lane == 0) scales[row] = amax == 0.0f ? 1.0f : __fdiv_rn(amax, 448.0f);
+    unsigned long long inv2;
+    asm("mov.b64 %0, {%1, %1};" : "=l"(inv2) : "r"(__float_as_uint(inv)));
+    const int64_t KC = K / kChunkK;
+    const int64_t rb = row / kChunkRows, L = row % kChunkRows;
+    // vector idx of the row: 4 value bytes at idx * 4, its metadata byte in
+    // chunk idx / 16 at L * 16 + idx % 16; idx0 % 16 == lane % 16 since the
+    // warp segment length is a multiple of 32, so vector j's byte is 2 chunks on
+    uint32_t* vrow = reinterpret_cast<uint32_t*>(values + row * (K / 2)) + idx0;
+    uint8_t* mrow = meta + (rb * KC + idx0 / 16) * kChunkBytes + L * 16 + (lane & 15);
+#pragma unroll
+    for (int j = 0; j < V; ++j) {
+      if (kExact || idx0 + j * 32 < nv) {
+        const uint32_t w0 = kept0[j], w1 = kept1[j];
+        const uint32_t q0 = e4m3x2_scaled(mad_u32(w0, 65536u, 0u), w0 & 0xFFFF0000u, inv2);
+        const uint32_t q1 = e4m3x2_scaled(mad_u32(w1, 65536u, 0u), w1 & 0xFFFF0000u, inv2);
+        if (live) vrow[j * 32] = mad_u32(q1, 65536u, q0);
+        mrow[j * 2 * kChunkBytes] = (uint8_t)nib[j];
+      }
+    }
+  };
+
+  uint4 ra[V], rb[V];
+  load(ra, base + slot);
+  for (uint32_t k = 0;; k += 2) {  // batch k in ra, batch k + 1 in rb
+    const int64_t b1 = base + stride;
+    const bool has1 = b1 < rows_pad;  // uniform over the CTA
+    if (has1) load(rb, b1 + slot);
+    process(ra, 0, k << 16, base + slot);
+    if (!has1) break;
+    const int64_t b2 = b1 + stride;
+    const bool has2 = b2 < rows_pad;
+    if (has2) load(ra, b2 + slot);
+    process(rb, 1, (k + 1) << 16, b1 + slot);
+    if (!has2) break;
+    base = b2;
   }
 }
 

@@ -1293,6 +1293,45 @@ size_t sp24_meta_bytes(int64_t rows, int64_t K) {
   return (size_t)((rows + 127) / 128) * (size_t)(K / 128) * 2048;
 }
 
+// ---------------------------------------------------------------------------
+// One-pass prune + E4M3 cast of rows up to kQMaxVecs 16-byte vectors (the row
+// held in registers): V vectors per lane and w warps per row with
+// w * 32 * V == K / 8 where some V in 4..8 gives that (no bounds checks),
+// else V = 8 with checks.  Rows of up to 8 warps run in 256-thread CTAs
+// (floor(8 / w) rows at a time, two CTAs per SM), longer ones one row at a
+// time in CTAs of up to 512 threads (one per SM); the CTAs are persistent,
+// with at most 65535 batches each.
+// ---------------------------------------------------------------------------
+int launch_prune_cast_rows_e4m3(const uint16_t* src, int64_t rows, int64_t K, int64_t ld, uint8_t* values,
+                                uint8_t* meta, float* scales, int sms, cudaStream_t s) {
+  const int64_t nv = K / 8;
+  int V = 8, w = (int)((nv + 255) / 256);
+  bool exact = false;
+  for (int v = 8; v >= 4 && !exact; --v) {
+    if (nv % (32 * v) == 0 && nv / (32 * v) <= kPcMaxWarps) {
+      V = v;
+      w = (int)(nv / (32 * v));
+      exact = true;
+    }
+  }
+  const bool wide = w > 8;
+  const int rpc = wide ? 1 : 8 / w;
+  const int64_t rows_pad = (rows + kChunkRows - 1) / kChunkRows * kChunkRows;
+  const int64_t batches = (rows_pad + rpc - 1) / rpc;
+  const int64_t resident = (int64_t)sms * (wide ? 1 : 2);
+  const int64_t ctas = std::min(batches, std::max(resident, (batches + 65534) / 65535));
+  const dim3 grid((unsigned)ctas), block((unsigned)(rpc * w * 32));
+  auto go = [&](auto kernel) { return launch_pdl(kernel, grid, block, 0, s, src, rows, K, ld, w, rpc, values, meta, scales); };
+  if (!exact) return wide ? go(k_prune_cast_rows_e4m3<512, 8, false>) : go(k_prune_cast_rows_e4m3<256, 8, false>);
+  switch (V) {
+    case 8: return wide ? go(k_prune_cast_rows_e4m3<512, 8, true>) : go(k_prune_cast_rows_e4m3<256, 8, true>);
+    case 7: return wide ? go(k_prune_cast_rows_e4m3<512, 7, true>) : go(k_prune_cast_rows_e4m3<256, 7, true>);
+    case 6: return wide ? go(k_prune_cast_rows_e4m3<512, 6, true>) : go(k_prune_cast_rows_e4m3<256, 6, true>);
+    case 5: return wide ? go(k_prune_cast_rows_e4m3<512, 5, true>) : go(k_prune_cast_rows_e4m3<256, 5, true>);
+    default: return wide ? go(k_prune_cast_rows_e4m3<512, 4, true>) : go(k_prune_cast_rows_e4m3<256, 4, true>);
+  }
+}
+
 int sp24_prune_compress(const void* src, int64_t rows, int64_t K, int64_t ld, sp24_dtype out_dtype,
                         void* values, void* meta, float* row_scales, const uint8_t* tile_mask,
                         void* dense_tiles, void* stream) {
@@ -1316,6 +1355,11 @@ int sp24_prune_compress(const void* src, int64_t rows, int64_t K, int64_t ld, sp
     k_prune_compress<false><<<grid, kPruneThreads, 0, s>>>(src16, rows, K, ld, values, meta8, nullptr,
                                                            tile_mask, dense_tiles);
     return launch_result(cudaGetLastError());
+  }
+  if (tile_mask == nullptr && K / 8 <= kQMaxVecs) {
+    // rows that fit in registers: amax, prune, cast, metadata and scale in one pass
+    return launch_prune_cast_rows_e4m3(src16, rows, K, ld, static_cast<uint8_t*>(values), meta8, row_scales, di.sms,
+                                       s);
   }
   const int agrid = (int)std::min<int64_t>((rows + 7) / 8, (int64_t)di.sms * 8);
   k_row_amax<<<agrid, 256, 0, s>>>(src16, rows, K, ld, row_scales);
@@ -1693,11 +1737,8 @@ int sp24_prune_compress_activations_fused_e4m3(const void* X, int64_t M, int64_t
   if (K / 8 <= kQMaxVecs) {
     // rows that fit in registers: amax, prune, cast, metadata and scale in
     // one pass over X, chained to the GEMM
-    const int w = (int)((K / 8 + kQSegVecs - 1) / kQSegVecs);
-    const int rpc = kQWarps / w;
-    const int64_t rows_pad = (M + 127) / 128 * 128;
-    st = launch_pdl(k_prune_cast_rows_e4m3, dim3((unsigned)((rows_pad + rpc - 1) / rpc)), dim3(kQWarps * 32), 0, s,
-                    x16, M, K, ldx, w, rpc, static_cast<uint8_t*>(x_values), static_cast<uint8_t*>(x_meta), x_scales);
+    st = launch_prune_cast_rows_e4m3(x16, M, K, ldx, static_cast<uint8_t*>(x_values), static_cast<uint8_t*>(x_meta),
+                                     x_scales, di.sms, s);
     if (st != SP24_OK) return st;
     return run_activation_gemm(false, x_values, x_meta, x_scales, Wq, ldw, w_scales, M, N, K, Y, ldy,
                                out_dtype == SP24_F32, di, s);

@@ -59,6 +59,28 @@ def test_prune_compress_e4m3_bit_exact(rows, K):
     assert np.array_equal(u8(dst), orc.decompress(ref.values, ref.canon, rows, K))
 
 
+# the one-pass prune + cast kernel over each of its row mappings: 8, 7, 6, 5 or 4
+# vectors per lane with no bounds checks (K = 4096, 1792, 1536 and 3072, 5120,
+# 1024), 8 with checks (768, 25600), 256-thread CTAs of several rows and
+# 512-thread CTAs of one (20480, 25600, 28672); ragged row counts; 30720 takes
+# the amax / prune / scale passes
+@pytest.mark.parametrize("rows,K", [(300, 4096), (130, 1792), (9, 1536), (37, 3072), (37, 5120), (200, 1024),
+                                    (129, 768), (5, 20480), (3, 25600), (2, 28672), (3, 30720)])
+def test_prune_compress_e4m3_one_pass_row_mappings(rows, K):
+    W = inputs.weights_with_outliers(rows, K, seed=rows + 3 * K)
+    W[0, :] = 0  # an all-zero row: scale 1, the metadata of zeros
+    ref = OracleSparseW(W, e4m3=True)
+    vals = torch.empty(rows, K // 2, dtype=torch.uint8, device="cuda")
+    meta = torch.empty(sp24.meta_bytes(rows, K), dtype=torch.uint8, device="cuda")
+    sc = torch.empty(rows, dtype=torch.float32, device="cuda")
+    sp24.prune_compress(dev_bf16(W), sp24.E4M3, vals, meta, row_scales=sc)
+    torch.cuda.synchronize()
+    assert sp24.last_device_error() == sp24.SP24_OK
+    assert np.array_equal(u8(vals), ref.values)
+    assert np.array_equal(u8(meta), ref.image)
+    assert np.array_equal(sc.cpu().numpy().view(np.uint32), ref.scales.view(np.uint32))
+
+
 def test_prune_handles_zero_rows_and_ties():
     W = np.zeros((128, 256), np.uint16)
     W[1, :8] = inputs.to_bf16_bits(np.array([1, 1, 1, 1, -2, 2, -2, 2], np.float32))
@@ -810,7 +832,8 @@ def _prepare_large(X_bits, W_bits, e4, tactic):
 
 
 @pytest.mark.parametrize("M,N,K", [(128, 384, 512), (200, 256, 1280), (1, 128, 128), (512, 384, 512),
-                                   (300, 640, 768), (5, 256, 32768)])
+                                   (300, 640, 768), (37, 128, 4096), (20, 128, 5120), (3, 128, 20480),
+                                   (2, 128, 25600), (5, 256, 32768)])
 def test_activation_fused_e4m3_parity(M, N, K):
     # rows up to 28672 wide take the one-pass kernel (row in registers); the
     # 32768-wide case takes the amax / prune / scale passes
