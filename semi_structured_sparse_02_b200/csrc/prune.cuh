@@ -1,7 +1,8 @@
 // prune.cuh -- kernel 1 (magnitude 2:4 prune + compress, emitting values and
-// the metadata image the sparse MMA reads), the per-row E4M3 quantizer and
-// the decompress (scatter) kernel.  All are HBM-bound: 128-bit loads, each
-// input byte read once per pass, outputs written with coalesced stores.
+// the metadata image the sparse MMA reads), the one-pass prune + per-row E4M3
+// cast, the per-row E4M3 quantizer and the decompress (scatter) kernel.  All
+// are HBM-bound: 128-bit loads, each input byte read once per pass, outputs
+// written with coalesced stores.
 //
 // Method: "2:4 Structured Sparsity Explained" (tensorcore.si), sections
 // "How 2:4 sparsity works" and "How to make a model 2:4 sparse"; E4M3 with one
